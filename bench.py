@@ -1,0 +1,374 @@
+"""Benchmark of the GDN token mixer on B200.
+
+A step is one gdn_prefill call of the long-prefill workload (1 sequence x
+32768 tokens, 32 heads, dk = dv = 128, bf16 inputs and output, fp32 state,
+S0 ~ N(0, 0.02)): ShortConv, SiLU, L2Norm, gates, the chunked gated delta rule
+and the gated RMSNorm output.  The decode workload (256 sequences x 32 heads,
+fp32 state updated in place, 1000 consecutive steps) is timed in the same run
+and reported under "decode".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (one process per GPU under torchrun) every rank runs its own
+independent long-prefill problem (weak scaling, no collective on the data
+path); the step time is the max over ranks.  `--impl reference` times the fp64
+CPU oracle (the only reference this method has) on a bounded sample.
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+from dataclasses import replace
+from datetime import timedelta
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from linear_attention_token_shortconv_b200 import gdn  # noqa: E402
+from linear_attention_token_shortconv_b200.workloads import (DECODE, LONG, make_decode_inputs,  # noqa: E402
+                                                             make_prefill_inputs, to_oracle_bits)
+
+METRIC = "GDN prefill tokens/s at T=32K H=32 (% TC peak); decode state GB/s (% HBM)"
+# Algorithmic work per token-head of the fused chunked prefill (chunk C = 64, d = 128):
+# MMA flops C(6dk+4dv) + 6 dk dv, and one pass over bf16 q,k,v,z, the two gate
+# logits and a bf16 output.
+PREFILL_FLOP_PER_TOKEN_HEAD = 64 * (6 * 128 + 4 * 128) + 6 * 128 * 128   # 180,224
+PREFILL_BYTES_PER_TOKEN_HEAD = 4 * 128 * 2 + 2 * 2 + 128 * 2           # 1,284
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return FALLBACK_PEAKS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples every 200 ms during a region."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.fh,
+                stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), float(parts[2]), parts[4:8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3]) if v == "Active"})
+        loaded = [r[0] for r in rows if r[2] > 200.0] or [r[0] for r in rows]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": max(r[2] for r in rows), "samples": len(rows), "reasons": reasons}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def prefill_call(inp, out, S_final):
+    gdn.prefill(inp["q"], inp["k"], inp["v"], inp["conv_w"], inp["a_logit"], inp["b_logit"],
+                inp["A"], inp["b_alpha"], inp["z"], inp["norm_w"], S0=inp["S0"],
+                cu_seqlens=inp["cu_seqlens"], out=out, S_final=S_final)
+
+
+def bench_prefill(cfg, steps, warmup, world, rank, dev):
+    inp = make_prefill_inputs(cfg, dev, seed=cfg.seed + 1000 * rank)
+    n_tok, H = cfg.total_tokens, cfg.H
+    out = torch.empty((n_tok, H, cfg.dv), dtype=torch.bfloat16, device=dev)
+    S_final = torch.empty((cfg.num_seqs, H, cfg.dk, cfg.dv), dtype=torch.float32, device=dev)
+    for _ in range(warmup):
+        prefill_call(inp, out, S_final)
+    torch.cuda.synchronize()
+    evb = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    eve = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for e in evb + eve:      # materialise the events before handing them to the library
+        e.record()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        start.record()
+        for i in range(steps):
+            gdn.set_timing_events(evb[i], eve[i])
+            prefill_call(inp, out, S_final)
+        end.record()
+        gdn.set_timing_events(None, None)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(start.elapsed_time(end) / steps, world)
+    kern_ms = max_over_ranks(sum(b.elapsed_time(e) for b, e in zip(evb, eve)) / steps, world)
+    return ms, kern_ms, clk.summary(), inp
+
+
+def bench_e2e(cfg, steps, warmup, world, rank, dev):
+    """Same metric through the public API with the inputs in pinned host memory:
+    every step copies the step's inputs host->device and reads out + S_final back."""
+    src = make_prefill_inputs(cfg, dev, seed=cfg.seed + 1000 * rank)
+    host = {k: (None if v is None else v.cpu().pin_memory()) for k, v in src.items()}
+    dev_in = {k: (None if v is None else torch.empty_like(v)) for k, v in src.items()}
+    del src
+    n_tok, H = cfg.total_tokens, cfg.H
+    out = torch.empty((n_tok, H, cfg.dv), dtype=torch.bfloat16, device=dev)
+    S_final = torch.empty((cfg.num_seqs, H, cfg.dk, cfg.dv), dtype=torch.float32, device=dev)
+    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    S_h = torch.empty(S_final.shape, dtype=S_final.dtype, pin_memory=True)
+    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+    d2h = out.numel() * out.element_size() + S_final.numel() * S_final.element_size()
+
+    def step():
+        for k, v in host.items():
+            if v is not None:
+                dev_in[k].copy_(v, non_blocking=True)
+        prefill_call(dev_in, out, S_final)
+        out_h.copy_(out, non_blocking=True)
+        S_h.copy_(S_final, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps):
+        step()
+    end.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(start.elapsed_time(end) / steps, world)
+    return ms, h2d, d2h
+
+
+def bench_decode(cfg, steps, dev):
+    d = make_decode_inputs(cfg, dev)
+    S, hist = d["S"], d["ring"]
+    out = torch.empty((cfg.B, cfg.H, cfg.dv), dtype=torch.bfloat16, device=dev)
+    P = cfg.pool
+
+    def step(t):
+        p = t % P
+        gdn.decode_step(d["q"][p], d["k"][p], d["v"][p], d["conv_w"], hist, d["a_logit"][p],
+                        d["b_logit"][p], d["A"], d["b_alpha"], d["z"][p], d["norm_w"], S, out=out)
+
+    for t in range(5):
+        step(t)
+    torch.cuda.synchronize()
+    evb = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    eve = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for e in evb + eve:
+        e.record()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record()
+    for t in range(steps):
+        gdn.set_timing_events(evb[t], eve[t])
+        step(t)
+    end.record()
+    gdn.set_timing_events(None, None)
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end) / steps
+    kern_ms = sum(b.elapsed_time(e) for b, e in zip(evb, eve)) / steps
+    state_bytes = 2 * cfg.B * cfg.H * cfg.dk * cfg.dv * 4
+    return ms, kern_ms, state_bytes
+
+
+def oracle_sample_rate(inp, cfg, tokens, heads, n_threads):
+    """Oracle (fp64, token by token) on `heads` chains of the first `tokens`
+    tokens; returns (token-heads per second, seconds, threads used)."""
+    import oracle
+    idx = torch.arange(heads)
+    dk, dv, H = cfg.dk, cfg.dv, cfg.H
+    take = lambda k: to_oracle_bits(inp[k][:tokens].index_select(1, idx.to(inp[k].device)))
+    rows = torch.cat([torch.arange(h * dk, (h + 1) * dk) for h in range(heads)] +
+                     [H * dk + torch.arange(h * dk, (h + 1) * dk) for h in range(heads)] +
+                     [2 * H * dk + torch.arange(h * dv, (h + 1) * dv) for h in range(heads)])
+    cw = to_oracle_bits(inp["conv_w"].index_select(0, rows.to(inp["conv_w"].device)))
+    S0 = None if inp["S0"] is None else to_oracle_bits(inp["S0"][:1].index_select(1, idx.to(inp["S0"].device)))
+    args = (take("q"), take("k"), take("v"), cw, take("a_logit"), take("b_logit"),
+            to_oracle_bits(inp["A"][:heads]), to_oracle_bits(inp["b_alpha"][:heads]), take("z"),
+            to_oracle_bits(inp["norm_w"]))
+    t0 = time.perf_counter()
+    oracle.prefill(*args, S0=S0, n_threads=n_threads)
+    dt = time.perf_counter() - t0
+    return tokens * heads / dt, dt, oracle.threads(n_threads)
+
+
+def run_reference(args, world, rank):
+    """The fp64 CPU oracle on the host cores: each step a bounded sample (one
+    head chain per core over 4096 tokens) of the long-prefill workload."""
+    if rank != 0:
+        return
+    cfg = LONG
+    inp = make_prefill_inputs(replace(cfg, lengths=(4096,)), "cpu")
+    cores = os.cpu_count() or 1
+    heads = min(cfg.H, cores)
+    for _ in range(args.warmup):
+        oracle_sample_rate(inp, cfg, 4096, heads, heads)
+    total_th, total_s = 0.0, 0.0
+    for _ in range(args.steps):
+        rate, dt, thr = oracle_sample_rate(inp, cfg, 4096, heads, heads)
+        total_th += 4096 * heads
+        total_s += dt
+    value = total_th / total_s / cfg.H
+    sample = f"{heads} head chains x 4096 tokens per step of the T=32768 H=32 workload; tokens/s scaled to all 32 heads"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_s / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": cfg.name, "seq_len": 32768, "H": 32},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--decode-steps", type=int, default=1000)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("at least 3 warm-up steps")
+
+    world, rank, local = dist_setup() if args.impl == "ours" else (
+        int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    pk, pk_kind = peaks()
+
+    cfg = LONG
+    ms, kern_ms, clocks, inp = bench_prefill(cfg, args.steps, args.warmup, world, rank, dev)
+    token_heads = cfg.total_tokens * cfg.H
+    value = world * cfg.total_tokens / (ms * 1e-3)
+    hbm_achieved = PREFILL_BYTES_PER_TOKEN_HEAD * token_heads / (kern_ms * 1e-3) / 1e9
+    tc_achieved = PREFILL_FLOP_PER_TOKEN_HEAD * token_heads / (kern_ms * 1e-3) / 1e12
+
+    result = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "long prefill: 1 seq x T=32768, H=32, dk=dv=128, bf16 in/out, "
+                               "fp32 state, S0~N(0,0.02), per GPU",
+                   "global_batch": world, "seq_len": cfg.total_tokens, "parallelism": f"dp{world}",
+                   "l2": "inputs larger than L2 (1.07 GB of bf16 q,k,v,z read per step)"},
+        "roofline": {"bound": "hbm", "achieved": hbm_achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": hbm_achieved / pk["hbm_gbs"], "traffic": None,
+                     "kernel": "state recurrence (chain) kernel", "kernel_ms": kern_ms,
+                     "peak_kind": pk_kind},
+        "tc": {"achieved_tflops": tc_achieved, "peak_tflops": pk["bf16_tflops"],
+               "frac": tc_achieved / pk["bf16_tflops"], "peak_kind": pk_kind + " burst",
+               "flop_per_token_head": PREFILL_FLOP_PER_TOKEN_HEAD},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+    }
+    del inp
+    torch.cuda.empty_cache()
+
+    if rank == 0 and args.decode_steps > 0:
+        dms, dk_ms, sbytes = bench_decode(DECODE, args.decode_steps, dev)
+        gbs = sbytes / (dk_ms * 1e-3) / 1e9
+        result["decode"] = {"workload": DECODE.name, "steps": args.decode_steps,
+                            "ms_per_step": dms, "kernel_ms": dk_ms,
+                            "state_gbs": gbs, "peak_gbs": pk["hbm_gbs"],
+                            "frac": gbs / pk["hbm_gbs"], "state_bytes_per_step": sbytes,
+                            "gpu_launches": args.decode_steps}
+        torch.cuda.empty_cache()
+
+    if not args.no_e2e:
+        e_ms, h2d, d2h = bench_e2e(cfg, max(3, args.steps // 2), args.warmup, world, rank, dev)
+        result["e2e"] = {"value": world * cfg.total_tokens / (e_ms * 1e-3), "unit": "tokens/s",
+                         "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        torch.cuda.empty_cache()
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cores = os.cpu_count() or 1
+        heads = min(cfg.H, cores)
+        inp = make_prefill_inputs(replace(cfg, lengths=(8192,)), "cpu")
+        rate, dt, thr = oracle_sample_rate(inp, cfg, 8192, heads, heads)
+        result["cpu_baseline"] = {"value": rate / cfg.H, "unit": "tokens/s", "cores": thr,
+                                  "kind": "oracle", "seconds": dt,
+                                  "sample": f"{heads} head chains x 8192 tokens of the T=32768 "
+                                            "H=32 workload; tokens/s scaled to all 32 heads"}
+    if rank == 0:
+        print(json.dumps(result))
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,154 @@
+/*
+ * gdn.h -- C ABI of the B200 (sm_100a) Gated DeltaNet (GDN) token mixer.
+ *
+ * The operation (web write-ups of "On the Design of Qwen3.8-Next Architecture"):
+ *   paper.rainbus.top digest, 方法步骤详情 step (1), and the slinene.github.io
+ *   write-up, 模块 A — Gated DeltaNet 混合层 (递归状态, 参数化):
+ *
+ *   q_t = L2Norm(SiLU(ShortConv(q_raw)))    k_t = L2Norm(SiLU(ShortConv(k_raw)))
+ *   v_t = SiLU(ShortConv(v_raw))
+ *   beta_t  = sigmoid(b_logit_t)
+ *   alpha_t = exp(-exp(A_h) * softplus(a_logit_t + b_alpha_h))
+ *   S_t = alpha_t S_{t-1};  e_t = v_t - S_t^T k_t;  S_t += beta_t k_t e_t^T
+ *         (= alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T)
+ *   y_t = S_t^T q_t
+ *   out_t = sigmoid(z_t) * y_t / sqrt(mean(y_t^2) + eps) * (1 + norm_w)
+ *
+ * per head h, with the state S in R^{dk x dv} (the transposed convention of the
+ * write-up), stored row-major [dk][dv] in fp32.  Readings where the pages are
+ * silent: ShortConv is a causal depthwise cross-correlation of width conv_k
+ * (tap conv_k-1 multiplies the current token), no bias, zero history at each
+ * sequence start; eps = 1e-6 in both L2Norm (x / sqrt(sum x^2 + eps)) and
+ * RMSNorm; the zero-centred RMSNorm gain is (1 + norm_w); no scale on q.
+ *
+ * Conventions shared by every call:
+ *   - Every pointer is a DEVICE pointer unless stated otherwise; the caller
+ *     allocates and frees all buffers it passes.
+ *   - Token tensors are packed [N_tok, H, d] row-major (d fastest); gate
+ *     logits are [N_tok, H]; conv weights are [H*(2*dk+dv), conv_k] fp32 with
+ *     channels ordered [q heads | k heads | v heads]: channel h*dk+i of q,
+ *     H*dk + h*dk+i of k, 2*H*dk + h*dv+i of v.
+ *   - in_dtype applies to q, k, v, z, a_logit, b_logit (and the decode conv
+ *     history); out_dtype to out.  Parameters and states are fp32.
+ *   - Calls are asynchronous on `stream` (NULL = legacy default stream).
+ *     Arguments are validated on the host before anything is launched; an
+ *     invalid call returns an error and launches nothing.  Faults of a kernel
+ *     surface at the caller's next synchronisation, as with any CUDA launch.
+ *   - Every pointer must be 16-byte aligned (GDN_ERR_ALIGNMENT otherwise).
+ *   - Supported sizes: dk, dv in {64, 128}; conv_k = 4 (GDN_ERR_UNSUPPORTED
+ *     otherwise).
+ */
+#ifndef GDN_H
+#define GDN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define GDN_API __attribute__((visibility("default")))
+#else
+#define GDN_API
+#endif
+
+/* Same type as cudaStream_t; declared here so the header needs no CUDA headers. */
+typedef struct CUstream_st *gdn_stream_t;
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1,  /* NULL where a buffer is required, bad sizes */
+    GDN_ERR_UNSUPPORTED = 2,  /* valid but not implemented (head dim, conv width, dtype) */
+    GDN_ERR_ALIGNMENT = 3,    /* a pointer is not 16-byte aligned */
+    GDN_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+    GDN_ERR_TIMEOUT = 5       /* a bounded device-side wait expired */
+} gdn_status_t;
+
+typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype_t;
+
+typedef struct {
+    int32_t num_seqs;      /* sequences in the batch (decode: batch size B) */
+    int32_t total_tokens;  /* packed tokens N_tok (decode: must equal num_seqs) */
+    int32_t H;             /* heads */
+    int32_t dk, dv;        /* key / value head dims */
+    int32_t conv_k;        /* ShortConv width */
+    gdn_dtype_t in_dtype;  /* q, k, v, z, gate logits */
+    gdn_dtype_t out_dtype; /* out */
+} gdn_dims_t;
+
+/*
+ * gdn_prefill -- the whole mixer over a packed batch of sequences.
+ *
+ *   q, k       [N_tok, H, dk]   raw (pre-conv) projections, in_dtype
+ *   v, z       [N_tok, H, dv]   raw value projection and output-gate logits
+ *   conv_w     [H(2dk+dv), conv_k] fp32
+ *   a_logit    [N_tok, H]       decay-gate logits (W_alpha x), in_dtype
+ *   b_logit    [N_tok, H]       write-gate logits (W_beta x), in_dtype
+ *   A, b_alpha [H] fp32         per-head decay parameters
+ *   norm_w     [dv] fp32        zero-centred RMSNorm weight (gain 1 + w)
+ *   S0         [N_seq, H, dk, dv] fp32 initial states, or NULL for zeros
+ *   cu_seqlens [N_seq + 1] int32 DEVICE prefix offsets (cu[0] = 0, non-
+ *              decreasing, cu[N_seq] = N_tok; empty sequences allowed), or
+ *              NULL for N_seq equal lengths N_tok / N_seq.  Not checked on the
+ *              device: a malformed array is undefined behaviour.
+ *   out        [N_tok, H, dv]   out_dtype, written
+ *   S_final    [N_seq, H, dk, dv] fp32 final states, written (may alias S0;
+ *              may be NULL when not wanted)
+ *
+ * Each sequence starts with an empty conv history.  `out` must not alias any
+ * input.  When total_tokens is 0 the token tensors (q, k, v, z, a_logit,
+ * b_logit, out) may be NULL and the call only writes S_final = S0 (or zeros).  The call takes a stream-ordered workspace of
+ * gdn_prefill_workspace_size() bytes from a private CUDA memory pool of the
+ * current device and returns it to the pool on the same stream.
+ */
+GDN_API gdn_status_t gdn_prefill(const gdn_dims_t *dims, const void *q, const void *k, const void *v,
+                         const float *conv_w, const void *a_logit, const void *b_logit,
+                         const float *A, const float *b_alpha, const void *z,
+                         const float *norm_w, const float *S0, const int32_t *cu_seqlens,
+                         void *out, float *S_final, gdn_stream_t stream);
+
+/* Bytes of device workspace one gdn_prefill call with these dims uses (host call). */
+GDN_API gdn_status_t gdn_prefill_workspace_size(const gdn_dims_t *dims, size_t *bytes);
+
+/*
+ * gdn_decode_step -- one token for each of B = dims->num_seqs sequences,
+ * reading and updating the per-head state in place.
+ *
+ *   q, k       [B, H, dk]; v, z [B, H, dv]; a_logit, b_logit [B, H]  (in_dtype)
+ *   conv_w, A, b_alpha, norm_w   as for gdn_prefill
+ *   conv_hist  [B, conv_k-1, H(2dk+dv)] in_dtype, in/out: the raw (pre-conv)
+ *              q|k|v channels of the previous conv_k-1 tokens, oldest first.
+ *              The step convolves [hist, current], then shifts the history by
+ *              one so the current raw token becomes the newest entry.  Zeros
+ *              mean "no history" (a fresh sequence).
+ *   S          [B, H, dk, dv] fp32, in/out (updated in place)
+ *   out        [B, H, dv] out_dtype, written
+ *
+ * dims->total_tokens must equal dims->num_seqs.  No workspace is used.
+ */
+GDN_API gdn_status_t gdn_decode_step(const gdn_dims_t *dims, const void *q, const void *k,
+                             const void *v, const float *conv_w, void *conv_hist,
+                             const void *a_logit, const void *b_logit, const float *A,
+                             const float *b_alpha, const void *z, const float *norm_w, float *S,
+                             void *out, gdn_stream_t stream);
+
+/*
+ * gdn_set_timing_events -- optional profiling hook (host call, not thread-safe).
+ * When both handles are non-NULL (cudaEvent_t values), each following
+ * gdn_prefill / gdn_decode_step records `begin` on its stream immediately before
+ * its dominant kernel (the state recurrence) and `end` immediately after it,
+ * until the hook is cleared with (NULL, NULL).  Recording adds no work to the
+ * kernels; it lets a caller time the dominant kernel with CUDA events.
+ */
+GDN_API gdn_status_t gdn_set_timing_events(void *begin, void *end);
+
+/* Human-readable name of a status code (static string, never NULL). */
+GDN_API const char *gdn_status_string(gdn_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H */

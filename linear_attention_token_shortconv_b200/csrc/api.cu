@@ -1,0 +1,201 @@
+// Host side of the C ABI declared in include/gdn.h: argument validation,
+// workspace management and kernel dispatch.  No kernel launches before every
+// argument has been checked.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/gdn.h"
+#include "gdn_internal.h"
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+gdn_status_t check_dims(const gdn_dims_t *d, bool decode) {
+    if (!d) return GDN_ERR_INVALID_ARG;
+    if (d->num_seqs <= 0 || d->total_tokens < 0 || d->H <= 0 || d->dk <= 0 || d->dv <= 0 ||
+        d->conv_k <= 0)
+        return GDN_ERR_INVALID_ARG;
+    if ((d->in_dtype != GDN_F32 && d->in_dtype != GDN_BF16) ||
+        (d->out_dtype != GDN_F32 && d->out_dtype != GDN_BF16))
+        return GDN_ERR_INVALID_ARG;
+    if (decode && d->total_tokens != d->num_seqs) return GDN_ERR_INVALID_ARG;
+    if ((d->dk != 64 && d->dk != 128) || (d->dv != 64 && d->dv != 128) || d->conv_k != 4)
+        return GDN_ERR_UNSUPPORTED;
+    // packed index arithmetic stays in 64 bits inside the kernels; keep the
+    // per-tensor element counts within int64 and the token count within int32
+    if ((int64_t)d->H * (2 * d->dk + d->dv) > (int64_t)1 << 30) return GDN_ERR_UNSUPPORTED;
+    return GDN_OK;
+}
+
+size_t round_up(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// fp32 workspace of the SIMT chain: q_hat, k_hat [N_tok,H,dk], v_hat [N_tok,H,dv]
+size_t workspace_bytes(const gdn_dims_t *d) {
+    const size_t nt = (size_t)d->total_tokens * d->H;
+    return 2 * round_up(nt * d->dk * sizeof(float)) + round_up(nt * d->dv * sizeof(float));
+}
+
+// One private stream-ordered pool per device; memory stays reserved between calls.
+std::mutex g_pool_mu;
+cudaMemPool_t g_pools[64] = {};
+
+cudaError_t get_pool(cudaMemPool_t *pool) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_pool_mu);
+    if (!g_pools[dev]) {
+        cudaMemPoolProps props = {};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.handleTypes = cudaMemHandleTypeNone;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t p;
+        e = cudaMemPoolCreate(&p, &props);
+        if (e != cudaSuccess) return e;
+        uint64_t keep = UINT64_MAX;
+        e = cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &keep);
+        if (e != cudaSuccess) return e;
+        g_pools[dev] = p;
+    }
+    *pool = g_pools[dev];
+    return cudaSuccess;
+}
+
+// profiling hook: events recorded around the dominant kernel of each call
+cudaEvent_t g_ev_begin = nullptr, g_ev_end = nullptr;
+
+cudaError_t record(cudaEvent_t ev, cudaStream_t s) {
+    return ev ? cudaEventRecord(ev, s) : cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" {
+
+gdn_status_t gdn_set_timing_events(void *begin, void *end) {
+    if ((begin == nullptr) != (end == nullptr)) return GDN_ERR_INVALID_ARG;
+    g_ev_begin = static_cast<cudaEvent_t>(begin);
+    g_ev_end = static_cast<cudaEvent_t>(end);
+    return GDN_OK;
+}
+
+const char *gdn_status_string(gdn_status_t s) {
+    switch (s) {
+    case GDN_OK: return "GDN_OK";
+    case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG";
+    case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED";
+    case GDN_ERR_ALIGNMENT: return "GDN_ERR_ALIGNMENT";
+    case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
+    case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
+    }
+    return "GDN_ERR_UNKNOWN";
+}
+
+gdn_status_t gdn_prefill_workspace_size(const gdn_dims_t *dims, size_t *bytes) {
+    gdn_status_t st = check_dims(dims, false);
+    if (st != GDN_OK) return st;
+    if (!bytes) return GDN_ERR_INVALID_ARG;
+    *bytes = workspace_bytes(dims);
+    return GDN_OK;
+}
+
+gdn_status_t gdn_prefill(const gdn_dims_t *dims, const void *q, const void *k, const void *v,
+                         const float *conv_w, const void *a_logit, const void *b_logit,
+                         const float *A, const float *b_alpha, const void *z,
+                         const float *norm_w, const float *S0, const int32_t *cu_seqlens,
+                         void *out, float *S_final, gdn_stream_t stream) {
+    gdn_status_t st = check_dims(dims, false);
+    if (st != GDN_OK) return st;
+    if (!cu_seqlens && dims->total_tokens % dims->num_seqs != 0) return GDN_ERR_INVALID_ARG;
+    // token tensors may be NULL only when there are no tokens
+    const bool no_tokens = dims->total_tokens == 0;
+    const void *tok[] = {q, k, v, a_logit, b_logit, z, out};
+    for (const void *p : tok) {
+        if (!p && !no_tokens) return GDN_ERR_INVALID_ARG;
+        if (p && !aligned16(p)) return GDN_ERR_ALIGNMENT;
+    }
+    const void *req[] = {conv_w, A, b_alpha, norm_w};
+    for (const void *p : req) {
+        if (!p) return GDN_ERR_INVALID_ARG;
+        if (!aligned16(p)) return GDN_ERR_ALIGNMENT;
+    }
+    const void *opt[] = {S0, cu_seqlens, S_final};
+    for (const void *p : opt)
+        if (p && !aligned16(p)) return GDN_ERR_ALIGNMENT;
+
+    gdn::PrefillArgs a;
+    a.n_seq = dims->num_seqs;
+    a.n_tok = dims->total_tokens;
+    a.H = dims->H;
+    a.dk = dims->dk;
+    a.dv = dims->dv;
+    a.in_bf16 = dims->in_dtype == GDN_BF16;
+    a.out_bf16 = dims->out_dtype == GDN_BF16;
+    a.q = q; a.k = k; a.v = v; a.z = z; a.a_logit = a_logit; a.b_logit = b_logit;
+    a.conv_w = conv_w; a.A = A; a.b_alpha = b_alpha; a.norm_w = norm_w; a.S0 = S0;
+    a.cu_seqlens = cu_seqlens;
+    a.out = out;
+    a.S_final = S_final;
+    a.stream = reinterpret_cast<cudaStream_t>(stream);
+
+    const size_t nt = (size_t)a.n_tok * a.H;
+    const size_t ws_bytes = workspace_bytes(dims);
+    char *ws = nullptr;
+    if (ws_bytes) {
+        cudaMemPool_t pool;
+        if (get_pool(&pool) != cudaSuccess) return GDN_ERR_CUDA;
+        if (cudaMallocFromPoolAsync(reinterpret_cast<void **>(&ws), ws_bytes, pool, a.stream) !=
+            cudaSuccess)
+            return GDN_ERR_CUDA;
+    }
+    float *qn = reinterpret_cast<float *>(ws);
+    float *kn = reinterpret_cast<float *>(ws + round_up(nt * a.dk * sizeof(float)));
+    float *vn = reinterpret_cast<float *>(ws + 2 * round_up(nt * a.dk * sizeof(float)));
+    cudaError_t e = gdn::launch_prelude_f32(a, qn, kn, vn);
+    if (e == cudaSuccess) e = record(g_ev_begin, a.stream);
+    if (e == cudaSuccess) e = gdn::launch_recurrent(a, qn, kn, vn);
+    if (e == cudaSuccess) e = record(g_ev_end, a.stream);
+    if (ws) {
+        cudaError_t ef = cudaFreeAsync(ws, a.stream);
+        if (e == cudaSuccess) e = ef;
+    }
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status_t gdn_decode_step(const gdn_dims_t *dims, const void *q, const void *k,
+                             const void *v, const float *conv_w, void *conv_hist,
+                             const void *a_logit, const void *b_logit, const float *A,
+                             const float *b_alpha, const void *z, const float *norm_w, float *S,
+                             void *out, gdn_stream_t stream) {
+    gdn_status_t st = check_dims(dims, true);
+    if (st != GDN_OK) return st;
+    const void *req[] = {q, k, v, conv_w, conv_hist, a_logit, b_logit, A, b_alpha, z, norm_w, S, out};
+    for (const void *p : req) {
+        if (!p) return GDN_ERR_INVALID_ARG;
+        if (!aligned16(p)) return GDN_ERR_ALIGNMENT;
+    }
+    gdn::DecodeArgs a;
+    a.B = dims->num_seqs;
+    a.H = dims->H;
+    a.dk = dims->dk;
+    a.dv = dims->dv;
+    a.in_bf16 = dims->in_dtype == GDN_BF16;
+    a.out_bf16 = dims->out_dtype == GDN_BF16;
+    a.q = q; a.k = k; a.v = v; a.z = z; a.a_logit = a_logit; a.b_logit = b_logit;
+    a.conv_w = conv_w; a.A = A; a.b_alpha = b_alpha; a.norm_w = norm_w;
+    a.conv_hist = conv_hist;
+    a.S = S;
+    a.out = out;
+    a.stream = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = record(g_ev_begin, a.stream);
+    if (e == cudaSuccess) e = gdn::launch_decode(a);
+    if (e == cudaSuccess) e = record(g_ev_end, a.stream);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,44 @@
+// Internal launch interface between the host ABI layer and the kernels.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gdn {
+
+struct PrefillArgs {
+    int n_seq, n_tok, H, dk, dv;
+    bool in_bf16, out_bf16;
+    const void *q, *k, *v, *z, *a_logit, *b_logit;
+    const float *conv_w, *A, *b_alpha, *norm_w, *S0;
+    const int32_t *cu_seqlens;
+    void *out;
+    float *S_final;
+    cudaStream_t stream;
+};
+
+struct DecodeArgs {
+    int B, H, dk, dv;
+    bool in_bf16, out_bf16;
+    const void *q, *k, *v, *z, *a_logit, *b_logit;
+    const float *conv_w, *A, *b_alpha, *norm_w;
+    void *conv_hist;
+    float *S;
+    void *out;
+    cudaStream_t stream;
+};
+
+// K1: conv + SiLU + L2Norm into a workspace (fp32 for the SIMT chain, fp16 for
+// the tensor-core chain).
+cudaError_t launch_prelude_f32(const PrefillArgs &a, float *qn, float *kn, float *vn);
+cudaError_t launch_prelude_f16(const PrefillArgs &a, __half *qn, __half *kn, __half *vn);
+
+// K2f: token-by-token recurrence with the fused gates and output stage (SIMT fp32).
+cudaError_t launch_recurrent(const PrefillArgs &a, const float *qn, const float *kn,
+                             const float *vn);
+
+// K3: one decode step.
+cudaError_t launch_decode(const DecodeArgs &a);
+
+}  // namespace gdn

@@ -1,0 +1,156 @@
+"""Thin Python binding of the C ABI in include/gdn.h (argument marshalling only).
+
+Every step of the mixer runs in the CUDA library ``libgdn.so`` built in-tree by
+``build.py``; this module only checks tensor placement, allocates outputs with
+PyTorch and passes raw device pointers and the current CUDA stream.  There is
+no fallback: if the library is missing or a tensor is not on a CUDA device the
+call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgdn.so")
+
+GDN_F32, GDN_BF16 = 0, 1
+STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "GDN_ERR_ALIGNMENT",
+          4: "GDN_ERR_CUDA", 5: "GDN_ERR_TIMEOUT"}
+
+# Every function the header declares (checked by the tests).
+EXPORTS = ("gdn_prefill", "gdn_prefill_workspace_size", "gdn_decode_step", "gdn_status_string",
+           "gdn_set_timing_events")
+
+
+class GdnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+        self.status = status
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("num_seqs", ctypes.c_int32), ("total_tokens", ctypes.c_int32),
+                ("H", ctypes.c_int32), ("dk", ctypes.c_int32), ("dv", ctypes.c_int32),
+                ("conv_k", ctypes.c_int32), ("in_dtype", ctypes.c_int32),
+                ("out_dtype", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libgdn.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"CUDA library not built: {LIB_PATH} is missing "
+                               "(run linear_attention_token_shortconv_b200/build.py)")
+        lib = ctypes.CDLL(LIB_PATH)
+        P, D = ctypes.c_void_p, ctypes.POINTER(Dims)
+        lib.gdn_prefill.argtypes = [D] + [P] * 15
+        lib.gdn_prefill.restype = ctypes.c_int
+        lib.gdn_prefill_workspace_size.argtypes = [D, ctypes.POINTER(ctypes.c_size_t)]
+        lib.gdn_prefill_workspace_size.restype = ctypes.c_int
+        lib.gdn_decode_step.argtypes = [D] + [P] * 14
+        lib.gdn_decode_step.restype = ctypes.c_int
+        lib.gdn_set_timing_events.argtypes = [P, P]
+        lib.gdn_set_timing_events.restype = ctypes.c_int
+        lib.gdn_status_string.argtypes = [ctypes.c_int]
+        lib.gdn_status_string.restype = ctypes.c_char_p
+        _lib = lib
+    return _lib
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return GDN_BF16
+    if t.dtype == torch.float32:
+        return GDN_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("all tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("all tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(rc: int, where: str):
+    if rc != 0:
+        raise GdnError(rc, where)
+
+
+def prefill(q, k, v, conv_w, a_logit, b_logit, A, b_alpha, z, norm_w, S0=None, cu_seqlens=None,
+            *, num_seqs=None, out=None, S_final=None, out_dtype=torch.float32, want_state=True,
+            stream=None):
+    """gdn_prefill on torch tensors.  q,k [N_tok,H,dk]; v,z [N_tok,H,dv]; a,b [N_tok,H].
+
+    Returns (out [N_tok,H,dv], S_final [N_seq,H,dk,dv] or None)."""
+    n_tok, H, dk = q.shape
+    dv = v.shape[2]
+    if cu_seqlens is not None:
+        n_seq = cu_seqlens.shape[0] - 1
+    else:
+        n_seq = num_seqs if num_seqs is not None else (S0.shape[0] if S0 is not None else 1)
+    if out is None:
+        out = torch.empty((n_tok, H, dv), dtype=out_dtype, device=q.device)
+    if S_final is None and want_state:
+        S_final = torch.empty((n_seq, H, dk, dv), dtype=torch.float32, device=q.device)
+    dims = Dims(n_seq, n_tok, H, dk, dv, conv_w.shape[1], _dt(q), _dt(out))
+    rc = load().gdn_prefill(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w),
+                            _ptr(a_logit), _ptr(b_logit), _ptr(A), _ptr(b_alpha), _ptr(z),
+                            _ptr(norm_w), _ptr(S0), _ptr(cu_seqlens), _ptr(out), _ptr(S_final),
+                            _stream(stream))
+    _check(rc, "gdn_prefill")
+    return out, S_final
+
+
+def prefill_workspace_size(n_seq, n_tok, H, dk, dv, conv_k=4, in_dtype=torch.bfloat16,
+                           out_dtype=torch.float32) -> int:
+    dims = Dims(n_seq, n_tok, H, dk, dv, conv_k,
+                GDN_BF16 if in_dtype == torch.bfloat16 else GDN_F32,
+                GDN_BF16 if out_dtype == torch.bfloat16 else GDN_F32)
+    n = ctypes.c_size_t(0)
+    _check(load().gdn_prefill_workspace_size(ctypes.byref(dims), ctypes.byref(n)),
+           "gdn_prefill_workspace_size")
+    return int(n.value)
+
+
+def decode_step(q, k, v, conv_w, conv_hist, a_logit, b_logit, A, b_alpha, z, norm_w, S, *,
+                out=None, out_dtype=torch.float32, stream=None):
+    """gdn_decode_step on torch tensors; updates conv_hist and S in place, returns out."""
+    B, H, dk = q.shape
+    dv = v.shape[2]
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=out_dtype, device=q.device)
+    dims = Dims(B, B, H, dk, dv, conv_w.shape[1], _dt(q), _dt(out))
+    rc = load().gdn_decode_step(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w),
+                                _ptr(conv_hist), _ptr(a_logit), _ptr(b_logit), _ptr(A),
+                                _ptr(b_alpha), _ptr(z), _ptr(norm_w), _ptr(S), _ptr(out),
+                                _stream(stream))
+    _check(rc, "gdn_decode_step")
+    return out
+
+
+def set_timing_events(begin=None, end=None):
+    """Record torch.cuda.Event `begin`/`end` around the dominant kernel of each
+    following call (None, None clears the hook)."""
+    b = None if begin is None else ctypes.c_void_p(begin.cuda_event)
+    e = None if end is None else ctypes.c_void_p(end.cuda_event)
+    _check(load().gdn_set_timing_events(b, e), "gdn_set_timing_events")
+
+
+def status_string(status: int) -> str:
+    return load().gdn_status_string(int(status)).decode()

@@ -27,7 +27,7 @@ def lib():
         vp, ip, dp, fp = ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p
         _lib.gdn_oracle_prefill.argtypes = [ip] * 7 + [vp] * 14 + [ip]
         _lib.gdn_oracle_prefill.restype = ip
-        _lib.gdn_oracle_decode_step.argtypes = [ip] * 6 + [vp] * 14 + [ip]
+        _lib.gdn_oracle_decode_step.argtypes = [ip] * 6 + [vp] * 13 + [ip]
         _lib.gdn_oracle_decode_step.restype = ip
         _lib.gdn_oracle_delta_rule.argtypes = [ip] * 3 + [dp] * 7
         _lib.gdn_oracle_delta_rule.restype = ip
@@ -97,24 +97,24 @@ def prefill(q, k, v, conv_w, a_logit, b_logit, A, b_alpha, z, norm_w, S0=None,
     return out, S_final
 
 
-def decode_step(q, k, v, conv_w, ring, ring_pos, a_logit, b_logit, A, b_alpha, z, norm_w, S,
+def decode_step(q, k, v, conv_w, hist, a_logit, b_logit, A, b_alpha, z, norm_w, S,
                 n_threads=0):
-    """One fp64 decode step.  ``ring`` (raw history, input dtype), ``ring_pos`` (int32)
-    and ``S`` (float64 [B,H,dk,dv]) are updated IN PLACE; returns out [B,H,dv]."""
+    """One fp64 decode step.  ``hist`` (raw conv history [B,K-1,C], oldest first,
+    input dtype) and ``S`` (float64 [B,H,dk,dv]) are updated IN PLACE; returns
+    out [B,H,dv]."""
     q, k, v, z, a_logit, b_logit = (_c(x) for x in (q, k, v, z, a_logit, b_logit))
     dt = _dtype_code(q)
     B, H, dk = q.shape
     dv = v.shape[2]
     conv_w = _c(conv_w, np.float32)
     K = conv_w.shape[1]
-    for name, arr, want in (("ring", ring, q.dtype), ("ring_pos", ring_pos, np.int32),
-                            ("S", S, np.float64)):
+    for name, arr, want in (("hist", hist, q.dtype), ("S", S, np.float64)):
         if arr.dtype != want or not arr.flags["C_CONTIGUOUS"]:
             raise TypeError(f"{name} must be a C-contiguous {np.dtype(want)} array")
     A, b_alpha, norm_w = _c(A, np.float32), _c(b_alpha, np.float32), _c(norm_w, np.float32)
     out = np.zeros((B, H, dv), np.float64)
     rc = lib().gdn_oracle_decode_step(B, H, dk, dv, K, dt, _ptr(q), _ptr(k), _ptr(v),
-                                      _ptr(conv_w), _ptr(ring), _ptr(ring_pos), _ptr(a_logit),
+                                      _ptr(conv_w), _ptr(hist), _ptr(a_logit),
                                       _ptr(b_logit), _ptr(A), _ptr(b_alpha), _ptr(z),
                                       _ptr(norm_w), _ptr(S), _ptr(out), int(n_threads))
     if rc != 0:

@@ -30,9 +30,9 @@
  *   - zero-centred RMSNorm has gain (1 + w), w of shape [dv] shared by heads.
  *   - A and b_alpha are one scalar per head; no 1/sqrt(dk) scale on q.
  *   - The readout uses the post-update state.
- *   - Decode keeps the last K-1 raw (pre-conv) tokens in a ring; slot
- *     (pos + j) mod (K-1) holds tap j (oldest first); after the step the
- *     current token overwrites slot pos and pos advances by one.
+ *   - Decode keeps the last K-1 raw (pre-conv) tokens of each sequence in a
+ *     history buffer, oldest first (slot j holds tap j); after the step the
+ *     buffer shifts by one and the current raw token enters the last slot.
  *
  * Inputs are read from the exact stored bits (fp32, or bf16 widened exactly)
  * and every operation is done in double precision, token by token.
@@ -257,13 +257,13 @@ int gdn_oracle_prefill(int n_seq, int n_tok, int H, int dk, int dv, int K, int i
 
 /*
  * One decode step for B sequences of one token each.  q,k [B,H,dk], v,z [B,H,dv],
- * a,b [B,H] in in_dtype; ring [B,K-1,H(2dk+dv)] in in_dtype (raw pre-conv
- * history, updated in place); ring_pos [B] (updated); S [B,H,dk,dv] double
- * (updated in place); out [B,H,dv] double.
+ * a,b [B,H] in in_dtype; hist [B,K-1,H(2dk+dv)] in in_dtype (raw pre-conv
+ * history, oldest first, shifted in place); S [B,H,dk,dv] double (updated in
+ * place); out [B,H,dv] double.
  */
 int gdn_oracle_decode_step(int B, int H, int dk, int dv, int K, int in_dtype,
                            const void *q, const void *k, const void *v, const float *conv_w,
-                           void *ring, int32_t *ring_pos, const void *a_logit,
+                           void *hist, const void *a_logit,
                            const void *b_logit, const float *A, const float *b_alpha,
                            const void *z, const float *norm_w, double *S, double *out,
                            int n_threads)
@@ -272,15 +272,11 @@ int gdn_oracle_decode_step(int B, int H, int dk, int dv, int K, int in_dtype,
         return -1;
     const int R = K - 1;
     const size_t C = (size_t)H * (2 * dk + dv);
-    for (int bq = 0; bq < B; ++bq)
-        if (ring_pos[bq] < 0 || ring_pos[bq] >= R)
-            return -1;
     set_threads(n_threads);
     const long pairs = (long)B * H;
 #pragma omp parallel for schedule(dynamic, 1)
     for (long ph = 0; ph < pairs; ++ph) {
         const int bq = (int)(ph / H), h = (int)(ph % H);
-        const int pos = ring_pos[bq];
         double *buf = malloc(sizeof(double) * (size_t)(2 * dk + 4 * dv));
         double *qh = buf, *kh = qh + dk, *vh = kh + dk, *e = vh + dv, *y = e + dv, *zz = y + dv;
         /* the three tensors of this head: (source, width, column in its tensor row, conv channel) */
@@ -295,11 +291,9 @@ int gdn_oracle_decode_step(int B, int H, int dk, int dv, int K, int in_dtype,
             for (int i = 0; i < width[s]; ++i) {
                 const size_t c = chan[s] + i;
                 double acc = 0.0;
-                for (int j = 0; j < R; ++j) {
-                    const int slot = (pos + j) % R;
+                for (int j = 0; j < R; ++j)
                     acc += (double)conv_w[c * K + j] *
-                           load_elem(ring, in_dtype, ((size_t)bq * R + slot) * C + c);
-                }
+                           load_elem(hist, in_dtype, ((size_t)bq * R + j) * C + c);
                 acc += (double)conv_w[c * K + (K - 1)] *
                        load_elem(src[s], in_dtype, (size_t)bq * row_elems[s] + col[s] + i);
                 dst[s][i] = silu(acc);
@@ -315,15 +309,18 @@ int gdn_oracle_decode_step(int B, int H, int dk, int dv, int K, int in_dtype,
         for (int j = 0; j < dv; ++j)
             zz[j] = load_elem(z, in_dtype, gi * dv + j);
         gated_rmsnorm(dv, y, zz, norm_w, out + gi * dv);
-        /* the current raw token replaces the oldest ring slot (channels of this head only) */
+        /* shift the history of this head's channels by one; the raw token enters last */
         for (int s = 0; s < 3; ++s)
-            for (int i = 0; i < width[s]; ++i)
-                copy_elem(ring, ((size_t)bq * R + pos) * C + chan[s] + i, src[s],
+            for (int i = 0; i < width[s]; ++i) {
+                const size_t c = chan[s] + i;
+                for (int j = 0; j + 1 < R; ++j)
+                    copy_elem(hist, ((size_t)bq * R + j) * C + c, hist,
+                              ((size_t)bq * R + j + 1) * C + c, in_dtype);
+                copy_elem(hist, ((size_t)bq * R + R - 1) * C + c, src[s],
                           (size_t)bq * row_elems[s] + col[s] + i, in_dtype);
+            }
         free(buf);
     }
-    for (int bq = 0; bq < B; ++bq)
-        ring_pos[bq] = (ring_pos[bq] + 1) % R;
     return 0;
 }
 

@@ -1,0 +1,97 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every function include/gdn.h declares, and rejects bad arguments before it
+touches CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from linear_attention_token_shortconv_b200 import gdn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"GDN_API\s+[\w\s\*]*?\b(gdn_\w+)\s*\(", src))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from linear_attention_token_shortconv_b200 import build
+    build.build()
+    return gdn.load()
+
+
+def test_library_exports_every_declared_function(lib):
+    names = declared_functions()
+    assert {"gdn_prefill", "gdn_decode_step", "gdn_status_string"} <= names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(gdn.EXPORTS) == names
+
+
+def test_status_strings(lib):
+    for code, name in gdn.STATUS.items():
+        assert gdn.status_string(code) == name
+    assert gdn.status_string(99) == "GDN_ERR_UNKNOWN"
+
+
+def _dims(**kw):
+    base = dict(num_seqs=1, total_tokens=64, H=2, dk=128, dv=128, conv_k=4, in_dtype=1, out_dtype=0)
+    base.update(kw)
+    return gdn.Dims(**base)
+
+
+def _prefill(lib, dims, ptrs):
+    return lib.gdn_prefill(ctypes.byref(dims) if dims is not None else None, *ptrs)
+
+
+FAKE = [ctypes.c_void_p(4096 * (i + 1)) for i in range(11)]   # aligned, never dereferenced
+
+
+def _args(q=FAKE[0], S0=None, cu=None, S_final=None, out=FAKE[10]):
+    return [q, FAKE[1], FAKE[2], FAKE[3], FAKE[4], FAKE[5], FAKE[6], FAKE[7], FAKE[8], FAKE[9],
+            S0, cu, out, S_final, None]
+
+
+def test_prefill_argument_validation(lib):
+    assert _prefill(lib, None, _args()) == 1
+    assert _prefill(lib, _dims(num_seqs=0), _args()) == 1
+    assert _prefill(lib, _dims(total_tokens=-1), _args()) == 1
+    assert _prefill(lib, _dims(in_dtype=7), _args()) == 1
+    assert _prefill(lib, _dims(num_seqs=3, total_tokens=64), _args()) == 1   # not divisible, no cu
+    assert _prefill(lib, _dims(dk=96), _args()) == 2
+    assert _prefill(lib, _dims(dv=256), _args()) == 2
+    assert _prefill(lib, _dims(conv_k=3), _args()) == 2
+    assert _prefill(lib, _dims(), _args(q=None)) == 1
+    assert _prefill(lib, _dims(), _args(out=None)) == 1
+    assert _prefill(lib, _dims(), _args(q=ctypes.c_void_p(4104))) == 3
+    assert _prefill(lib, _dims(), _args(S0=ctypes.c_void_p(4100))) == 3
+    assert _prefill(lib, _dims(), _args(cu=ctypes.c_void_p(4098))) == 3
+
+
+def test_decode_argument_validation(lib):
+    args = [FAKE[i] for i in range(11)] + [ctypes.c_void_p(8192), ctypes.c_void_p(12288), None]
+    d = _dims(num_seqs=4, total_tokens=4)
+    assert lib.gdn_decode_step(ctypes.byref(_dims(num_seqs=4, total_tokens=5)), *args) == 1
+    assert lib.gdn_decode_step(ctypes.byref(_dims(num_seqs=4, total_tokens=4, dk=32)), *args) == 2
+    bad = list(args)
+    bad[4] = None   # conv history is required
+    assert lib.gdn_decode_step(ctypes.byref(d), *bad) == 1
+    bad = list(args)
+    bad[11] = ctypes.c_void_p(8200)  # S misaligned
+    assert lib.gdn_decode_step(ctypes.byref(d), *bad) == 3
+
+
+def test_workspace_size_query(lib):
+    n = gdn.prefill_workspace_size(2, 1000, 4, 128, 64)
+    assert n >= 1000 * 4 * (128 + 128 + 64) * 2
+    assert gdn.prefill_workspace_size(1, 0, 1, 64, 64) == 0
+    with pytest.raises(gdn.GdnError):
+        gdn.prefill_workspace_size(1, 10, 1, 48, 64)

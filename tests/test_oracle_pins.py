@@ -363,8 +363,8 @@ def test_bf16_inputs_are_widened_exactly():
 
 
 def test_decode_steps_equal_prefill():
-    """T decode steps from an empty ring (any start slot) equal a prefill of T
-    tokens, and the ring ends holding the last K-1 raw tokens, oldest at ring_pos."""
+    """T decode steps from an empty history equal a prefill of T tokens, and the
+    history ends holding the last K-1 raw tokens, oldest first."""
     rng = np.random.default_rng(27)
     T, B, H, dk, dv, K = 9, 3, 2, 8, 4, 4
     C = H * (2 * dk + dv)
@@ -373,13 +373,12 @@ def test_decode_steps_equal_prefill():
     for s in seqs:
         s.update(shared)
     S0 = rng.standard_normal((B, H, dk, dv)).astype(np.float32)
-    ring = np.zeros((B, K - 1, C), np.float32)
-    pos = np.array([0, 1, 2], np.int32)
+    hist = np.zeros((B, K - 1, C), np.float32)
     S = S0.astype(np.float64).copy()
     outs = []
     for t in range(T):
         g = lambda key: np.stack([s[key][t] for s in seqs])
-        outs.append(oracle.decode_step(g("q"), g("k"), g("v"), shared["conv_w"], ring, pos,
+        outs.append(oracle.decode_step(g("q"), g("k"), g("v"), shared["conv_w"], hist,
                                        g("a_logit"), g("b_logit"), shared["A"],
                                        shared["b_alpha"], g("z"), shared["norm_w"], S))
     for b in range(B):
@@ -391,4 +390,4 @@ def test_decode_steps_equal_prefill():
                               seqs[b]["v"].reshape(T, -1)], axis=1)
         # channel order [q heads | k heads | v heads] matches the (T, H, d) reshapes
         for j in range(K - 1):
-            assert np.array_equal(ring[b, (pos[b] + j) % (K - 1)], raw[T - (K - 1) + j])
+            assert np.array_equal(hist[b, j], raw[T - (K - 1) + j])
