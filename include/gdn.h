@@ -34,7 +34,10 @@
  *     Arguments are validated on the host before anything is launched; an
  *     invalid call returns an error and launches nothing.  Faults of a kernel
  *     surface at the caller's next synchronisation, as with any CUDA launch.
- *   - Every pointer must be 16-byte aligned (GDN_ERR_ALIGNMENT otherwise).
+ *   - Tensors read or written in vectors (q, k, v, z, conv_w, S0, S_final, S,
+ *     conv_hist, out) must be 16-byte aligned (GDN_ERR_ALIGNMENT otherwise);
+ *     the per-token gate logits, A, b_alpha, norm_w and cu_seqlens need only
+ *     the alignment of their element type.
  *   - Supported sizes: dk, dv in {64, 128}; conv_k = 4 (GDN_ERR_UNSUPPORTED
  *     otherwise).
  */

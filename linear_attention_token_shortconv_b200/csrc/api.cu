@@ -12,6 +12,7 @@
 namespace {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned_to(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 gdn_status_t check_dims(const gdn_dims_t *d, bool decode) {
     if (!d) return GDN_ERR_INVALID_ARG;
@@ -114,19 +115,28 @@ gdn_status_t gdn_prefill(const gdn_dims_t *dims, const void *q, const void *k, c
     if (!cu_seqlens && dims->total_tokens % dims->num_seqs != 0) return GDN_ERR_INVALID_ARG;
     // token tensors may be NULL only when there are no tokens
     const bool no_tokens = dims->total_tokens == 0;
-    const void *tok[] = {q, k, v, a_logit, b_logit, z, out};
+    const uintptr_t in_sz = dims->in_dtype == GDN_BF16 ? 2 : 4;
+    const void *tok[] = {q, k, v, z, out};
     for (const void *p : tok) {
         if (!p && !no_tokens) return GDN_ERR_INVALID_ARG;
         if (p && !aligned16(p)) return GDN_ERR_ALIGNMENT;
     }
-    const void *req[] = {conv_w, A, b_alpha, norm_w};
-    for (const void *p : req) {
-        if (!p) return GDN_ERR_INVALID_ARG;
-        if (!aligned16(p)) return GDN_ERR_ALIGNMENT;
+    const void *gates[] = {a_logit, b_logit};
+    for (const void *p : gates) {
+        if (!p && !no_tokens) return GDN_ERR_INVALID_ARG;
+        if (p && !aligned_to(p, in_sz)) return GDN_ERR_ALIGNMENT;
     }
-    const void *opt[] = {S0, cu_seqlens, S_final};
+    if (!conv_w) return GDN_ERR_INVALID_ARG;
+    if (!aligned16(conv_w)) return GDN_ERR_ALIGNMENT;
+    const void *params[] = {A, b_alpha, norm_w};
+    for (const void *p : params) {
+        if (!p) return GDN_ERR_INVALID_ARG;
+        if (!aligned_to(p, 4)) return GDN_ERR_ALIGNMENT;
+    }
+    const void *opt[] = {S0, S_final};
     for (const void *p : opt)
         if (p && !aligned16(p)) return GDN_ERR_ALIGNMENT;
+    if (cu_seqlens && !aligned_to(cu_seqlens, 4)) return GDN_ERR_ALIGNMENT;
 
     gdn::PrefillArgs a;
     a.n_seq = dims->num_seqs;
@@ -174,10 +184,21 @@ gdn_status_t gdn_decode_step(const gdn_dims_t *dims, const void *q, const void *
                              void *out, gdn_stream_t stream) {
     gdn_status_t st = check_dims(dims, true);
     if (st != GDN_OK) return st;
-    const void *req[] = {q, k, v, conv_w, conv_hist, a_logit, b_logit, A, b_alpha, z, norm_w, S, out};
-    for (const void *p : req) {
+    const void *vec[] = {q, k, v, conv_w, conv_hist, z, S, out};
+    for (const void *p : vec) {
         if (!p) return GDN_ERR_INVALID_ARG;
         if (!aligned16(p)) return GDN_ERR_ALIGNMENT;
+    }
+    const uintptr_t in_sz = dims->in_dtype == GDN_BF16 ? 2 : 4;
+    const void *gates[] = {a_logit, b_logit};
+    for (const void *p : gates) {
+        if (!p) return GDN_ERR_INVALID_ARG;
+        if (!aligned_to(p, in_sz)) return GDN_ERR_ALIGNMENT;
+    }
+    const void *params[] = {A, b_alpha, norm_w};
+    for (const void *p : params) {
+        if (!p) return GDN_ERR_INVALID_ARG;
+        if (!aligned_to(p, 4)) return GDN_ERR_ALIGNMENT;
     }
     gdn::DecodeArgs a;
     a.B = dims->num_seqs;

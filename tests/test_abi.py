@@ -74,6 +74,9 @@ def test_prefill_argument_validation(lib):
     assert _prefill(lib, _dims(), _args(q=ctypes.c_void_p(4104))) == 3
     assert _prefill(lib, _dims(), _args(S0=ctypes.c_void_p(4100))) == 3
     assert _prefill(lib, _dims(), _args(cu=ctypes.c_void_p(4098))) == 3
+    args = _args()
+    args[4] = ctypes.c_void_p(4099)   # a_logit: bf16 needs 2-byte alignment
+    assert _prefill(lib, _dims(), args) == 3
 
 
 def test_decode_argument_validation(lib):
