@@ -33,9 +33,17 @@ gdn_status_t check_dims(const gdn_dims_t *d, bool decode) {
 
 size_t round_up(size_t x) { return (x + 255) & ~(size_t)255; }
 
-// fp32 workspace of the SIMT chain: q_hat, k_hat [N_tok,H,dk], v_hat [N_tok,H,dv]
+// The chunked tensor-core path serves bf16 inputs with dk = 128; everything
+// else (the fp32 workload, dk = 64) runs the fp32 token-by-token recurrence.
+bool use_tensor_cores(const gdn_dims_t *d) { return d->in_dtype == GDN_BF16 && d->dk == 128; }
+
+// Workspace: tensor-core path: Qt, Kt, -W [dk], U' [dv], Aqk [64] in fp16 and
+// e^{G_C} in fp32 per token-head; fp32 path: q_hat, k_hat, v_hat in fp32.
 size_t workspace_bytes(const gdn_dims_t *d) {
     const size_t nt = (size_t)d->total_tokens * d->H;
+    if (use_tensor_cores(d))
+        return 3 * round_up(nt * d->dk * 2) + round_up(nt * d->dv * 2) + round_up(nt * 64 * 2) +
+               round_up(nt * 4);
     return 2 * round_up(nt * d->dk * sizeof(float)) + round_up(nt * d->dv * sizeof(float));
 }
 
@@ -163,13 +171,30 @@ gdn_status_t gdn_prefill(const gdn_dims_t *dims, const void *q, const void *k, c
             cudaSuccess)
             return GDN_ERR_CUDA;
     }
-    float *qn = reinterpret_cast<float *>(ws);
-    float *kn = reinterpret_cast<float *>(ws + round_up(nt * a.dk * sizeof(float)));
-    float *vn = reinterpret_cast<float *>(ws + 2 * round_up(nt * a.dk * sizeof(float)));
-    cudaError_t e = gdn::launch_prelude_f32(a, qn, kn, vn);
-    if (e == cudaSuccess) e = record(g_ev_begin, a.stream);
-    if (e == cudaSuccess) e = gdn::launch_recurrent(a, qn, kn, vn);
-    if (e == cudaSuccess) e = record(g_ev_end, a.stream);
+    cudaError_t e;
+    if (use_tensor_cores(dims)) {
+        gdn::TcWorkspace w;
+        char *p = ws;
+        auto take = [&](size_t bytes) { char *r = p; p += round_up(bytes); return r; };
+        w.Qt = reinterpret_cast<__half *>(take(nt * a.dk * 2));
+        w.Kt = reinterpret_cast<__half *>(take(nt * a.dk * 2));
+        w.Wn = reinterpret_cast<__half *>(take(nt * a.dk * 2));
+        w.Up = reinterpret_cast<__half *>(take(nt * a.dv * 2));
+        w.Aqk = reinterpret_cast<__half *>(take(nt * 64 * 2));
+        w.decay = reinterpret_cast<float *>(take(nt * 4));
+        e = gdn::launch_chunk_prep(a, w);
+        if (e == cudaSuccess) e = record(g_ev_begin, a.stream);
+        if (e == cudaSuccess) e = gdn::launch_chunk_chain(a, w);
+        if (e == cudaSuccess) e = record(g_ev_end, a.stream);
+    } else {
+        float *qn = reinterpret_cast<float *>(ws);
+        float *kn = reinterpret_cast<float *>(ws + round_up(nt * a.dk * sizeof(float)));
+        float *vn = reinterpret_cast<float *>(ws + 2 * round_up(nt * a.dk * sizeof(float)));
+        e = gdn::launch_prelude_f32(a, qn, kn, vn);
+        if (e == cudaSuccess) e = record(g_ev_begin, a.stream);
+        if (e == cudaSuccess) e = gdn::launch_recurrent(a, qn, kn, vn);
+        if (e == cudaSuccess) e = record(g_ev_end, a.stream);
+    }
     if (ws) {
         cudaError_t ef = cudaFreeAsync(ws, a.stream);
         if (e == cudaSuccess) e = ef;

@@ -1,0 +1,409 @@
+// K2a -- prelude plus the state-independent part of the chunked gated delta
+// rule, one 64-token chunk of one head per iteration, chunks of all sequences
+// and heads in parallel.
+//
+// Prelude (slinene.github.io write-up of "On the Design of Qwen3.8-Next
+// Architecture", 模块 A, 参数化): q = L2Norm(SiLU(ShortConv(q_raw))), k likewise,
+// v = SiLU(ShortConv(v_raw)), beta = sigmoid(b), log alpha = -e^A softplus(a + b_alpha).
+//
+// Chunk form (derived from the erase-then-write update of the same section,
+// 递归状态): with u_i = beta_i (v_i - alpha_i S_{i-1}^T k_i) the update is
+// S_i = alpha_i S_{i-1} + k_i u_i^T.  With G_i = sum_{j<=i} log alpha_j inside
+// the chunk and S the state before it,
+//     (I + L) U = diag(beta) (V - diag(e^G) K S),
+//     L_ij = beta_i (k_i . k_j) e^{G_i - G_j}  (j < i),
+// so U = U' - W S with T = (I + L)^-1, W = T diag(beta e^G) K, U' = T diag(beta) V.
+// The chain kernel needs, per chunk: -W, U', Qt = diag(e^G) Q,
+// Kt = diag(e^{G_C - G}) K, Aqk_ij = (q_i . k_j) e^{G_i - G_j} (j <= i), e^{G_C}.
+// Every decay is exp of a non-positive difference of log sums.
+//
+// The output RMSNorm is scale-invariant, so for short-memory heads the output
+// is sensitive to the *relative* error of q_i . k_i, which can be tiny.  The
+// q.k and k.k products therefore use a two-term fp16 split of the fp32 q and k
+// (x = hi + lo): [Qh;Kh]Kh^T + [Qh;Kh]Kl^T + [Ql;Kl]Kh^T, fp32 accumulation.
+//
+// Per chunk: prelude in registers -> fp16 hi/lo tiles in smem; the split
+// [Q;K]K^T on tcgen05 (M=128, N=64) -> TMEM; Aqk and L from TMEM; T by forward
+// substitution in fp32; [T diag(beta e^G); T diag(beta)] times K and V on
+// tcgen05 -> TMEM; results to global memory in fp16.
+#include <cuda_fp16.h>
+
+#include "gdn_device.cuh"
+#include "gdn_internal.h"
+#include "umma.cuh"
+
+namespace gdn {
+
+__device__ unsigned int g_prep_err;
+
+namespace prep {
+constexpr int C = 64;          // chunk length
+constexpr int DK = 128;
+constexpr int OFF_HI = 0;      // [Qh;Kh] K-major, 2 k-blocks x 16 KB
+constexpr int OFF_LO = 32768;  // [Ql;Kl] K-major, 2 k-blocks x 16 KB; later L fp32 [64][64]
+constexpr int OFF_V = 65536;   // V MN-major, DV/64 mn-blocks x 8 KB
+constexpr int OFF_T = 81920;   // [T'; T''] K-major, 1 k-block x 16 KB
+constexpr int OFF_MISC = 98304;
+constexpr int SMEM = OFF_MISC + 1024 + 1024;
+constexpr uint32_t TMEM_COLS = 256;
+}  // namespace prep
+
+__device__ __forceinline__ void split_store(uint8_t *hi_blk, uint8_t *lo_blk, int row, int chunk,
+                                            const float (&x)[8]) {
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const __half2 hh = __floats2half2_rn(x[2 * e], x[2 * e + 1]);
+        const float2 hf = __half22float2(hh);
+        const __half2 ll = __floats2half2_rn(x[2 * e] - hf.x, x[2 * e + 1] - hf.y);
+        h[e] = *reinterpret_cast<const uint32_t *>(&hh);
+        l[e] = *reinterpret_cast<const uint32_t *>(&ll);
+    }
+    umma::st_chunk(hi_blk, row, chunk, make_uint4(h[0], h[1], h[2], h[3]));
+    umma::st_chunk(lo_blk, row, chunk, make_uint4(l[0], l[1], l[2], l[3]));
+}
+
+// Conv + SiLU of 8 channels for tokens [i0, i0 + n) of a chunk (sliding window
+// over the raw rows, zero before the sequence start); emits each row to `emit`.
+template <typename Tin, typename Emit>
+__device__ __forceinline__ void conv_rows(const Tin *src, size_t row_stride, int col,
+                                          const float (&w)[8][4], int t0, int s_begin, int i0,
+                                          int n, int len, Emit emit) {
+    float h0[8], h1[8], h2[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) h0[e] = h1[e] = h2[e] = 0.f;
+    const int ta = t0 + i0;
+    if (ta - 3 >= s_begin) load8(src + (size_t)(ta - 3) * row_stride + col, h0);
+    if (ta - 2 >= s_begin) load8(src + (size_t)(ta - 2) * row_stride + col, h1);
+    if (ta - 1 >= s_begin) load8(src + (size_t)(ta - 1) * row_stride + col, h2);
+    for (int ii = 0; ii < n; ++ii) {
+        const int i = i0 + ii;
+        float x[8], y[8];
+        if (i < len) load8(src + (size_t)(t0 + i) * row_stride + col, x);
+        else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] = 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            float a = w[e][0] * h0[e];
+            a = fmaf(w[e][1], h1[e], a);
+            a = fmaf(w[e][2], h2[e], a);
+            a = fmaf(w[e][3], x[e], a);
+            y[e] = (i < len) ? siluf_(a) : 0.f;
+            h0[e] = h1[e]; h1[e] = h2[e]; h2[e] = x[e];
+        }
+        emit(i, y);
+    }
+}
+
+template <int DV, typename Tin>
+__global__ void __launch_bounds__(128)
+chunk_prep_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
+                  const float *__restrict__ conv_w, const Tin *__restrict__ a_logit,
+                  const Tin *__restrict__ b_logit, const float *__restrict__ A,
+                  const float *__restrict__ b_alpha, const int32_t *__restrict__ cu_seqlens,
+                  int n_seq, int n_tok, int H, __half *__restrict__ Qt, __half *__restrict__ Kt,
+                  __half *__restrict__ Wn, __half *__restrict__ Up, __half *__restrict__ Aqk,
+                  float *__restrict__ decay) {
+    using namespace prep;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sHI = sm + OFF_HI, *sLO = sm + OFF_LO, *sV = sm + OFF_V, *sT = sm + OFF_T;
+    float *sL = reinterpret_cast<float *>(sm + OFF_LO);          // aliases [Ql;Kl] after the q.k MMA
+    float *sG = reinterpret_cast<float *>(sm + OFF_MISC);        // 64
+    float *sBeta = sG + 64;                                      // 64
+    float *sTot = sBeta + 64;                                    // 1
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + OFF_MISC + 768);
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + OFF_MISC + 784);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int h = blockIdx.x, n = blockIdx.y;
+    int s_begin, s_end;
+    if (cu_seqlens) { s_begin = __ldg(cu_seqlens + n); s_end = __ldg(cu_seqlens + n + 1); }
+    else { const int L = n_tok / n_seq; s_begin = n * L; s_end = s_begin + L; }
+    const int n_chunks = (s_end - s_begin + C - 1) / C;
+    if ((int)blockIdx.z >= n_chunks) return;   // uniform per block
+
+    if (warp == 0) umma::tmem_alloc(tslot, TMEM_COLS);
+    if (tid == 0) { umma::mbar_init(bar, 1); umma::fence_mbar_init(); }
+    __syncthreads();
+    const uint32_t tbase = *tslot;
+    const uint32_t trow = tbase + ((uint32_t)(warp * 32) << 16);
+    const float eA = expf(__ldg(A + h)), ba = __ldg(b_alpha + h);
+
+    // this thread's prelude channels: q/k octet (tid % 32, tokens 16 * (tid / 32) ..)
+    // and v octet (tid % (DV / 8), tokens (DV / 8) * 8 / ... )
+    const int qk_oct = tid & 31;                  // 0..15 q, 16..31 k
+    const bool is_k = qk_oct >= 16;
+    const int qk_col = h * DK + (qk_oct & 15) * 8;
+    const int qk_chan = (is_k ? H * DK : 0) + qk_col;
+    constexpr int VO = DV / 8;                    // v octets
+    constexpr int VPARTS = 128 / VO;              // token parts for v
+    const int v_oct = tid % VO, v_part = tid / VO;
+    const int v_col = h * DV + v_oct * 8;
+    const int v_chan = 2 * H * DK + v_col;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int c = blockIdx.z; c < n_chunks && ok; c += gridDim.z) {
+        const int t0 = s_begin + c * C;
+        const int len = min(C, s_end - t0);
+        // ---- 1. prelude: q, k -> L2-normalised fp32 -> hi/lo fp16 tiles; v -> fp16 tile
+        // (conv weights re-read per chunk from L1/L2 to keep them out of the solve's registers)
+        float wqk[8][4], wv[8][4];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float4 a4 = __ldg(reinterpret_cast<const float4 *>(conv_w) + qk_chan + e);
+            wqk[e][0] = a4.x; wqk[e][1] = a4.y; wqk[e][2] = a4.z; wqk[e][3] = a4.w;
+        }
+        conv_rows(is_k ? k : q, (size_t)H * DK, qk_col, wqk, t0, s_begin, 16 * warp, 16, len,
+                  [&](int i, float (&y)[8]) {
+                      float ss = 0.f;
+#pragma unroll
+                      for (int e = 0; e < 8; ++e) ss = fmaf(y[e], y[e], ss);
+                      ss = group_sum<16>(ss);
+                      const float r = rsqrtf(ss + kNormEps);
+#pragma unroll
+                      for (int e = 0; e < 8; ++e) y[e] *= r;
+                      const int row = (is_k ? 64 : 0) + i, oc = qk_oct & 15;
+                      split_store(sHI + (oc / 8) * 16384, sLO + (oc / 8) * 16384, row, oc % 8, y);
+                  });
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float4 b4 = __ldg(reinterpret_cast<const float4 *>(conv_w) + v_chan + e);
+            wv[e][0] = b4.x; wv[e][1] = b4.y; wv[e][2] = b4.z; wv[e][3] = b4.w;
+        }
+        conv_rows(v, (size_t)H * DV, v_col, wv, t0, s_begin, (C / VPARTS) * v_part, C / VPARTS, len,
+                  [&](int i, float (&y)[8]) {
+                      umma::st_chunk(sV + (v_oct / 8) * 8192, i, v_oct % 8,
+                                     make_uint4(umma::pack_half2(y[0], y[1]), umma::pack_half2(y[2], y[3]),
+                                                umma::pack_half2(y[4], y[5]), umma::pack_half2(y[6], y[7])));
+                  });
+        if (tid < C) {
+            float g = 0.f, be = 0.f;
+            if (tid < len) {
+                const size_t gi = (size_t)(t0 + tid) * H + h;
+                g = -eA * softplus_acc(to_f32(a_logit[gi]) + ba);
+                be = sigmoid_acc(to_f32(b_logit[gi]));
+            }
+            // inclusive scan of the log decays within each warp, then across the two
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, g, o);
+                if (lane >= o) g += y;
+            }
+            if (tid == 31) *sTot = g;
+            sBeta[tid] = be;
+            sG[tid] = g;
+        }
+        __syncthreads();
+        if (tid >= 32 && tid < C) sG[tid] += *sTot;
+        umma::fence_proxy_async_smem();
+        __syncthreads();
+
+        // ---- 2. [Q;K] K^T = [Qh;Kh]Kh^T + [Qh;Kh]Kl^T + [Ql;Kl]Kh^T -> TMEM [0, 64)
+        if (tid == 0) {
+            umma::tc_fence_after();
+            const uint32_t hi = umma::smem_u32(sHI), lo = umma::smem_u32(sLO);
+            const uint32_t idesc = umma::idesc_f16(128, 64, false, false);
+#pragma unroll
+            for (int s = 0; s < DK / 16; ++s) {
+                const uint32_t off = (s / 4) * 16384 + (s % 4) * 32;
+                const uint64_t ah = umma::sw128_desc(hi + off, 16, 1024), al = umma::sw128_desc(lo + off, 16, 1024);
+                const uint64_t bh = umma::sw128_desc(hi + off + 8192, 16, 1024), bl = umma::sw128_desc(lo + off + 8192, 16, 1024);
+                umma::mma_f16(tbase, ah, bh, idesc, s > 0);
+                umma::mma_f16(tbase, ah, bl, idesc, 1u);
+                umma::mma_f16(tbase, al, bh, idesc, 1u);
+            }
+            umma::mma_commit(bar);
+        }
+        ok = __syncthreads_and(umma::mbar_wait_bounded(bar, phase, 1u << 22));
+        phase ^= 1;
+        umma::tc_fence_after();
+        if (!ok) break;
+
+        // ---- 3. rows 0..63: Aqk (masked, decayed q.k) -> global; rows 64..127: L -> smem
+        {
+            float v0[32], v1[32];
+            umma::tmem_ld32(trow + 0, v0);
+            umma::tmem_ld32(trow + 32, v1);
+            const int i = (warp * 32 + lane) & 63;
+            const float Gi = sG[i];
+            if (warp < 2) {
+                if (i < len) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(Aqk + ((size_t)(t0 + i) * H + h) * C);
+#pragma unroll
+                    for (int q8 = 0; q8 < 8; ++q8) {
+                        float x[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int j = q8 * 8 + e;
+                            const float raw = (j < 32) ? v0[j & 31] : v1[j & 31];
+                            x[e] = (j <= i) ? raw * __expf(Gi - sG[j]) : 0.f;
+                        }
+                        dst[q8] = make_uint4(umma::pack_half2(x[0], x[1]), umma::pack_half2(x[2], x[3]),
+                                             umma::pack_half2(x[4], x[5]), umma::pack_half2(x[6], x[7]));
+                    }
+                }
+            } else {
+                const float bi = sBeta[i];
+                float4 *dst = reinterpret_cast<float4 *>(sL + i * C);
+#pragma unroll
+                for (int q4 = 0; q4 < 16; ++q4) {
+                    float x[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int j = q4 * 4 + e;
+                        const float raw = (j < 32) ? v0[j & 31] : v1[j & 31];
+                        x[e] = (j < i) ? bi * raw * __expf(Gi - sG[j]) : 0.f;
+                    }
+                    dst[q4] = make_float4(x[0], x[1], x[2], x[3]);
+                }
+            }
+        }
+        umma::tc_fence_before();
+        __syncthreads();
+
+        // ---- 4. T = (I + L)^-1 by forward substitution, thread c owns column c
+        if (tid < C) {
+            const int cc = tid;
+            float Tc[C];
+#pragma unroll
+            for (int i = 0; i < C; ++i) {
+                float acc = (i == cc) ? 1.f : 0.f;
+                const float4 *Li = reinterpret_cast<const float4 *>(sL + i * C);
+#pragma unroll
+                for (int j4 = 0; j4 < i / 4; ++j4) {
+                    const float4 l = Li[j4];
+                    acc = fmaf(-l.x, Tc[4 * j4], acc);
+                    acc = fmaf(-l.y, Tc[4 * j4 + 1], acc);
+                    acc = fmaf(-l.z, Tc[4 * j4 + 2], acc);
+                    acc = fmaf(-l.w, Tc[4 * j4 + 3], acc);
+                }
+#pragma unroll
+                for (int j = (i / 4) * 4; j < i; ++j) acc = fmaf(-sL[i * C + j], Tc[j], acc);
+                Tc[i] = acc;
+            }
+            // T' = T diag(beta e^G) (rows 0..63), T'' = T diag(beta) (rows 64..127); K index = cc
+            const float bc = sBeta[cc], bgc = bc * __expf(sG[cc]);
+            const int chunk = cc / 8, within = (cc % 8) * 2;
+#pragma unroll
+            for (int i = 0; i < C; ++i) {
+                *reinterpret_cast<__half *>(sT + umma::sw128_offset(i, chunk) + within) = __float2half_rn(Tc[i] * bgc);
+                *reinterpret_cast<__half *>(sT + umma::sw128_offset(64 + i, chunk) + within) = __float2half_rn(Tc[i] * bc);
+            }
+        } else {
+            // Qt = e^{G_i} q_i and Kt = e^{G_C - G_i} k_i from the hi tiles (fp16 outputs)
+            const float GC = sG[C - 1];
+            for (int idx = tid - C; idx < len * (DK / 8); idx += 128 - C) {
+                const int i = idx / (DK / 8), ch = idx % (DK / 8);
+                const float sq = __expf(sG[i]), sk = __expf(GC - sG[i]);
+                const uint4 qv = *reinterpret_cast<const uint4 *>(sHI + (ch / 8) * 16384 + umma::sw128_offset(i, ch % 8));
+                const uint4 kv = *reinterpret_cast<const uint4 *>(sHI + (ch / 8) * 16384 + umma::sw128_offset(64 + i, ch % 8));
+                const __half2 *q2 = reinterpret_cast<const __half2 *>(&qv);
+                const __half2 *k2 = reinterpret_cast<const __half2 *>(&kv);
+                uint4 qo, ko;
+                uint32_t *qo32 = reinterpret_cast<uint32_t *>(&qo), *ko32 = reinterpret_cast<uint32_t *>(&ko);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 qf = __half22float2(q2[e]), kf = __half22float2(k2[e]);
+                    qo32[e] = umma::pack_half2(qf.x * sq, qf.y * sq);
+                    ko32[e] = umma::pack_half2(kf.x * sk, kf.y * sk);
+                }
+                const size_t g = ((size_t)(t0 + i) * H + h) * DK + ch * 8;
+                *reinterpret_cast<uint4 *>(Qt + g) = qo;
+                *reinterpret_cast<uint4 *>(Kt + g) = ko;
+            }
+            if (tid == C) decay[(size_t)t0 * H + h] = __expf(GC);
+        }
+        umma::fence_proxy_async_smem();
+        __syncthreads();
+
+        // ---- 5. W-part = T' K -> TMEM [0, DK);  U'-part = T'' V -> TMEM [DK, DK + DV)
+        if (tid == 0) {
+            umma::tc_fence_after();
+            const uint32_t aT = umma::smem_u32(sT), aK = umma::smem_u32(sHI) + 8192, aV = umma::smem_u32(sV);
+            const uint32_t idw = umma::idesc_f16(128, DK, false, true);
+            const uint32_t idu = umma::idesc_f16(128, DV, false, true);
+#pragma unroll
+            for (int s = 0; s < C / 16; ++s) {
+                const uint64_t ad = umma::sw128_desc(aT + s * 32, 16, 1024);
+                umma::mma_f16(tbase, ad, umma::sw128_desc(aK + s * 2048, 16384, 1024), idw, s > 0);
+                umma::mma_f16(tbase + DK, ad, umma::sw128_desc(aV + s * 2048, 8192, 1024), idu, s > 0);
+            }
+            umma::mma_commit(bar);
+        }
+        ok = __syncthreads_and(umma::mbar_wait_bounded(bar, phase, 1u << 22));
+        phase ^= 1;
+        umma::tc_fence_after();
+        if (!ok) break;
+
+        // ---- 6. rows 0..63 of the W-part -> -W; rows 64..127 of the U'-part -> U'
+        //         (TMEM loads are warp-collective: every lane loads, valid rows store)
+        {
+            const int i = (warp * 32 + lane) & 63;
+            if (warp < 2) {
+                __half *dst = Wn + ((size_t)(t0 + i) * H + h) * DK;
+#pragma unroll
+                for (int c0 = 0; c0 < DK; c0 += 32) {
+                    float vv[32];
+                    umma::tmem_ld32(trow + c0, vv);
+                    if (i < len) {
+#pragma unroll
+                        for (int q8 = 0; q8 < 4; ++q8)
+                            reinterpret_cast<uint4 *>(dst + c0)[q8] = make_uint4(
+                                umma::pack_half2(-vv[q8 * 8 + 0], -vv[q8 * 8 + 1]), umma::pack_half2(-vv[q8 * 8 + 2], -vv[q8 * 8 + 3]),
+                                umma::pack_half2(-vv[q8 * 8 + 4], -vv[q8 * 8 + 5]), umma::pack_half2(-vv[q8 * 8 + 6], -vv[q8 * 8 + 7]));
+                    }
+                }
+            } else {
+                __half *dst = Up + ((size_t)(t0 + i) * H + h) * DV;
+#pragma unroll
+                for (int c0 = 0; c0 < DV; c0 += 32) {
+                    float vv[32];
+                    umma::tmem_ld32(trow + DK + c0, vv);
+                    if (i < len) {
+#pragma unroll
+                        for (int q8 = 0; q8 < 4; ++q8)
+                            reinterpret_cast<uint4 *>(dst + c0)[q8] = make_uint4(
+                                umma::pack_half2(vv[q8 * 8 + 0], vv[q8 * 8 + 1]), umma::pack_half2(vv[q8 * 8 + 2], vv[q8 * 8 + 3]),
+                                umma::pack_half2(vv[q8 * 8 + 4], vv[q8 * 8 + 5]), umma::pack_half2(vv[q8 * 8 + 6], vv[q8 * 8 + 7]));
+                    }
+                }
+            }
+        }
+        umma::tc_fence_before();
+        __syncthreads();
+    }
+    if (!ok && tid == 0) atomicOr(&g_prep_err, 1u);
+    umma::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) umma::tmem_dealloc(tbase, TMEM_COLS);
+}
+
+cudaError_t launch_chunk_prep(const PrefillArgs &a, const TcWorkspace &w) {
+    if (a.n_tok == 0) return cudaSuccess;
+    // blocks per (head, sequence): the longest sequence may hold every chunk, so
+    // give each (head, sequence) ~8 x 148 / H blocks; blocks past the end exit
+    int split = max(1, (8 * 148) / a.H);
+    split = min(split, (a.n_tok + 63) / 64);
+    dim3 grid(a.H, a.n_seq, split);
+    cudaError_t e;
+#define GDN_PREP(DV_, TIN)                                                                        \
+    e = cudaFuncSetAttribute(chunk_prep_kernel<DV_, TIN>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             prep::SMEM);                                                       \
+    if (e != cudaSuccess) return e;                                                              \
+    chunk_prep_kernel<DV_, TIN><<<grid, 128, prep::SMEM, a.stream>>>(                            \
+        (const TIN *)a.q, (const TIN *)a.k, (const TIN *)a.v, a.conv_w, (const TIN *)a.a_logit,  \
+        (const TIN *)a.b_logit, a.A, a.b_alpha, a.cu_seqlens, a.n_seq, a.n_tok, a.H, w.Qt, w.Kt, \
+        w.Wn, w.Up, w.Aqk, w.decay)
+    if (a.dv == 128) {
+        if (a.in_bf16) { GDN_PREP(128, bf16); } else { GDN_PREP(128, float); }
+    } else {
+        if (a.in_bf16) { GDN_PREP(64, bf16); } else { GDN_PREP(64, float); }
+    }
+#undef GDN_PREP
+    return cudaGetLastError();
+}
+
+}  // namespace gdn

@@ -34,6 +34,17 @@ struct DecodeArgs {
 cudaError_t launch_prelude_f32(const PrefillArgs &a, float *qn, float *kn, float *vn);
 cudaError_t launch_prelude_f16(const PrefillArgs &a, __half *qn, __half *kn, __half *vn);
 
+// Workspace of the tensor-core prefill (all token-indexed, [N_tok, H, *]).
+struct TcWorkspace {
+    __half *Qt, *Kt, *Wn;   // e^G q, e^{G_C - G} k, -W  [dk]
+    __half *Up, *Aqk;       // U' [dv], decayed masked q.k [64]
+    float *decay;           // e^{G_C} at the first token row of each chunk
+};
+
+// K2a (prelude fused) / K2b: chunked prefill on tcgen05 (dk = 128, dv in {64, 128}).
+cudaError_t launch_chunk_prep(const PrefillArgs &a, const TcWorkspace &w);
+cudaError_t launch_chunk_chain(const PrefillArgs &a, const TcWorkspace &w);
+
 // K2f: token-by-token recurrence with the fused gates and output stage (SIMT fp32).
 cudaError_t launch_recurrent(const PrefillArgs &a, const float *qn, const float *kn,
                              const float *vn);

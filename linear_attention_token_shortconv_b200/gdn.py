@@ -22,7 +22,7 @@ STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "G
 
 # Every function the header declares (checked by the tests).
 EXPORTS = ("gdn_prefill", "gdn_prefill_workspace_size", "gdn_decode_step", "gdn_status_string",
-           "gdn_set_timing_events")
+           "gdn_set_timing_events", "gdn_selftest_umma")
 
 
 class GdnError(RuntimeError):
@@ -56,6 +56,8 @@ def load() -> ctypes.CDLL:
         lib.gdn_prefill_workspace_size.restype = ctypes.c_int
         lib.gdn_decode_step.argtypes = [D] + [P] * 14
         lib.gdn_decode_step.restype = ctypes.c_int
+        lib.gdn_selftest_umma.argtypes = [ctypes.c_int] * 5 + [P] * 5
+        lib.gdn_selftest_umma.restype = ctypes.c_int
         lib.gdn_set_timing_events.argtypes = [P, P]
         lib.gdn_set_timing_events.restype = ctypes.c_int
         lib.gdn_status_string.argtypes = [ctypes.c_int]
@@ -150,6 +152,20 @@ def set_timing_events(begin=None, end=None):
     b = None if begin is None else ctypes.c_void_p(begin.cuda_event)
     e = None if end is None else ctypes.c_void_p(end.cuda_event)
     _check(load().gdn_set_timing_events(b, e), "gdn_set_timing_events")
+
+
+def selftest_umma(A, B, init=None, *, a_mn=False, b_mn=False, negate_a=False, stream=None):
+    """D = init + (+/-A) B computed on the tensor cores with the given shared-memory
+    operand layouts (A [128,K], B [K,N] fp16 CUDA tensors)."""
+    M, K = A.shape
+    N = B.shape[1]
+    if M != 128 or B.shape[0] != K or A.dtype != torch.float16 or B.dtype != torch.float16:
+        raise ValueError("A must be [128, K] and B [K, N], both fp16")
+    D = torch.empty((128, N), dtype=torch.float32, device=A.device)
+    rc = load().gdn_selftest_umma(int(a_mn), int(b_mn), int(negate_a), N, K, _ptr(A), _ptr(B),
+                                  _ptr(init), _ptr(D), _stream(stream))
+    _check(rc, "gdn_selftest_umma")
+    return D
 
 
 def status_string(status: int) -> str:

@@ -33,7 +33,7 @@ def test_library_exports_every_declared_function(lib):
     assert {"gdn_prefill", "gdn_decode_step", "gdn_status_string"} <= names
     for n in names:
         assert hasattr(lib, n), n
-    assert set(gdn.EXPORTS) == names
+    assert set(gdn.EXPORTS) == names, (set(gdn.EXPORTS) ^ names)
 
 
 def test_status_strings(lib):
