@@ -138,6 +138,40 @@ GDN_API gdn_status_t gdn_decode_step(const gdn_dims_t *dims, const void *q, cons
                              void *out, gdn_stream_t stream);
 
 /*
+ * gdn_prefill_noalloc -- gdn_prefill for callers that cannot allocate device
+ * memory.  The pages have no counterpart: this is an interface choice of the
+ * library.  Callers that may not call cudaMalloc or any allocator while they
+ * run the layer (code inside host callbacks or allocation-free regions,
+ * embedders whose device memory is partitioned up-front by another runtime,
+ * real-time paths that must not take an allocator lock or fail with
+ * out-of-memory mid-request) cannot use gdn_prefill, which takes its workspace
+ * from a memory pool.  This call takes the same arguments and runs the same
+ * tensor-core kernels, with the workspace in a fixed array of
+ * GDN_NOALLOC_SCRATCH_BYTES inside the library's device memory; it allocates
+ * nothing.  The caller still allocates every input and output.
+ *
+ *   - Supported: in_dtype = GDN_BF16, dk = 128, dv in {64, 128}, conv_k = 4
+ *     (GDN_ERR_UNSUPPORTED otherwise).
+ *   - Size limit: the workspace of 3*dk*2 + dv*2 + 64*2 + 4 bytes per token
+ *     and head (each of its six arrays rounded up to 256 bytes) must fit in
+ *     GDN_NOALLOC_SCRATCH_BYTES, about 29,000 token-heads at dk = dv = 128;
+ *     larger calls return GDN_ERR_INVALID_ARG and launch nothing.
+ *   - The array exists once per GPU that loads the library, until exit.  The
+ *     first call on a device looks up its device address; make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the array, which keeps the last call's
+ *     contents (nothing in it must start at zero).  Calls whose GPU work
+ *     overlaps, e.g. on two streams at once, race on it: serialise them.
+ */
+#define GDN_NOALLOC_SCRATCH_BYTES (32u << 20)
+GDN_API gdn_status_t gdn_prefill_noalloc(const gdn_dims_t *dims, const void *q, const void *k,
+                                         const void *v, const float *conv_w, const void *a_logit,
+                                         const void *b_logit, const float *A, const float *b_alpha,
+                                         const void *z, const float *norm_w, const float *S0,
+                                         const int32_t *cu_seqlens, void *out, float *S_final,
+                                         gdn_stream_t stream);
+
+/*
  * gdn_set_timing_events -- optional profiling hook (host call, not thread-safe).
  * When both handles are non-NULL (cudaEvent_t values), each following
  * gdn_prefill / gdn_decode_step records `begin` on its stream immediately before

@@ -22,7 +22,7 @@ STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "G
 
 # Every function the header declares (checked by the tests).
 EXPORTS = ("gdn_prefill", "gdn_prefill_workspace_size", "gdn_decode_step", "gdn_status_string",
-           "gdn_set_timing_events", "gdn_selftest_umma")
+           "gdn_set_timing_events", "gdn_selftest_umma", "gdn_prefill_noalloc")
 
 
 class GdnError(RuntimeError):
@@ -56,6 +56,8 @@ def load() -> ctypes.CDLL:
         lib.gdn_prefill_workspace_size.restype = ctypes.c_int
         lib.gdn_decode_step.argtypes = [D] + [P] * 14
         lib.gdn_decode_step.restype = ctypes.c_int
+        lib.gdn_prefill_noalloc.argtypes = [D] + [P] * 15
+        lib.gdn_prefill_noalloc.restype = ctypes.c_int
         lib.gdn_selftest_umma.argtypes = [ctypes.c_int] * 5 + [P] * 5
         lib.gdn_selftest_umma.restype = ctypes.c_int
         lib.gdn_set_timing_events.argtypes = [P, P]
@@ -116,6 +118,32 @@ def prefill(q, k, v, conv_w, a_logit, b_logit, A, b_alpha, z, norm_w, S0=None, c
                             _ptr(norm_w), _ptr(S0), _ptr(cu_seqlens), _ptr(out), _ptr(S_final),
                             _stream(stream))
     _check(rc, "gdn_prefill")
+    return out, S_final
+
+
+def prefill_noalloc(q, k, v, conv_w, a_logit, b_logit, A, b_alpha, z, norm_w, S0=None,
+                    cu_seqlens=None, *, num_seqs=None, out=None, S_final=None,
+                    out_dtype=torch.float32, want_state=True, stream=None):
+    """gdn_prefill_noalloc on torch tensors: the tensor-core prefill with its
+    workspace in the library's fixed device array (for callers that cannot
+    allocate while running the layer; the outputs here are still allocated by
+    torch when not supplied).  Same arguments and results as `prefill`."""
+    n_tok, H, dk = q.shape
+    dv = v.shape[2]
+    if cu_seqlens is not None:
+        n_seq = cu_seqlens.shape[0] - 1
+    else:
+        n_seq = num_seqs if num_seqs is not None else (S0.shape[0] if S0 is not None else 1)
+    if out is None:
+        out = torch.empty((n_tok, H, dv), dtype=out_dtype, device=q.device)
+    if S_final is None and want_state:
+        S_final = torch.empty((n_seq, H, dk, dv), dtype=torch.float32, device=q.device)
+    dims = Dims(n_seq, n_tok, H, dk, dv, conv_w.shape[1], _dt(q), _dt(out))
+    rc = load().gdn_prefill_noalloc(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w),
+                                    _ptr(a_logit), _ptr(b_logit), _ptr(A), _ptr(b_alpha), _ptr(z),
+                                    _ptr(norm_w), _ptr(S0), _ptr(cu_seqlens), _ptr(out),
+                                    _ptr(S_final), _stream(stream))
+    _check(rc, "gdn_prefill_noalloc")
     return out, S_final
 
 
