@@ -3,18 +3,27 @@
 // zero-centred RMSNorm fused (slinene.github.io write-up of "On the Design of
 // Qwen3.8-Next Architecture", 模块 A: 递归状态 and 参数化).
 //
-// Per chunk, with the per-chunk tensors of the chunk-prep kernel
-// (-W, U', Qt, Kt, Aqk, e^{G_C}) and the state S before the chunk:
-//     P[0:64]   = U' + (-W) S        = U            (tcgen05, M=128 with rows 64..127)
-//     P[64:128] = Qt S                               (... = diag(e^G) Q S)
-//     P[64:128] += Aqk U             = Y            (tcgen05)
-//     dS        = Kt^T U                              (tcgen05)
-//     S         = e^{G_C} S + dS                      (fp32, registers)
+// Per chunk, with the chunk-prep tensors (-W, U', Qt, Kt, Aqk, e^{G_C}) and the
+// state S before the chunk:
+//     P[0:64]   = (-W) S      then U = U' + P[0:64]      (tcgen05 + registers)
+//     P[64:128] = Qt S        (= diag(e^G) Q S)
+//     P[64:128] += Aqk U      = Y                        (tcgen05)
+//     dS        = Kt^T U                                  (tcgen05)
+//     S         = e^{G_C} S + dS                          (fp32, registers)
 //     out       = sigmoid(z) * Y / sqrt(mean(Y^2) + eps) * (1 + w)
-// One CTA of 128 threads: thread r holds row r of the fp32 state S [dk=128][dv]
-// (TMEM lane r of dS), and an fp16 copy of S in shared memory is the B operand
-// of the next chunk.  All accumulators live in tensor memory.
+//
+// One CTA of 4 * dv threads per (sequence, head).  Warp w reads tensor-memory
+// lane quadrant w % 4 and owns the 32-column group w / 4: each thread holds 32
+// columns of one row of the fp32 state S [dk=128][dv], and an fp16 copy of S in
+// shared memory is the B operand of the next chunk.  Tiles of the next chunk
+// arrive by TMA (128-byte swizzled) into a second stage while the current chunk
+// runs; P is double-buffered in tensor memory so the output stage of chunk c
+// (quadrants 2, 3) overlaps the first MMA and the U conversion of chunk c + 1
+// (quadrants 0, 1).  Every wait is bounded.
+#include <cuda.h>
 #include <cuda_fp16.h>
+
+#include <cstring>
 
 #include "gdn_device.cuh"
 #include "gdn_internal.h"
@@ -27,21 +36,28 @@ __device__ unsigned int g_chain_err;
 namespace chain {
 constexpr int C = 64;
 constexpr int DK = 128;
-constexpr int OFF_AP = 0;                // [-W; Qt] K-major: 2 k-blocks x 16 KB
-constexpr int OFF_BP = 32768;            // S MN-major: rows = dk, DV/64 mn-blocks x 16 KB
-constexpr int OFF_AS = 65536;            // Kt MN-major: rows = tokens, 2 mn-blocks x 8 KB
-constexpr int OFF_AY = 81920;            // [0; Aqk] K-major: 1 k-block x 16 KB
-constexpr int OFF_BU = 98304;            // U MN-major: rows = tokens, DV/64 mn-blocks x 8 KB
-constexpr int OFF_MISC = 114688;
-constexpr int SMEM = OFF_MISC + 1024 + 1024;
+// one stage: [-W; Qt] 32 KB | Kt 16 KB | Aqk 8 KB | U' 16 KB | z 16 KB
+constexpr int ST_AP = 0, ST_AS = 32768, ST_AQK = 49152, ST_US = 57344, ST_ZS = 73728;
+constexpr int STAGE = 90112;
+constexpr int OFF_BP = 2 * STAGE;          // S fp16 MN-major (rows = dk), 32 KB
+constexpr int OFF_BU = OFF_BP + 32768;     // U fp16 MN-major (rows = tokens), 16 KB
+constexpr int OFF_MISC = OFF_BU + 16384;
+// misc: barriers [0, 128), 1 + w [128, 640), partial sums [640, 1664); + alignment slack
+constexpr int SMEM = OFF_MISC + 1664 + 1024;
+static_assert(SMEM <= 232448, "227 KB per block");
+constexpr uint32_t kMaxPolls = 1u << 24;
 }  // namespace chain
+
+struct ChainMaps {
+    CUtensorMap wn, qt, kt, aqk, up, z;
+};
 
 __device__ __forceinline__ uint4 pack8(const float *x) {
     return make_uint4(umma::pack_half2(x[0], x[1]), umma::pack_half2(x[2], x[3]),
                       umma::pack_half2(x[4], x[5]), umma::pack_half2(x[6], x[7]));
 }
 
-__device__ __forceinline__ void unpack8(uint4 u, float *x) {
+__device__ __forceinline__ void unpack8h(uint4 u, float *x) {
     const __half2 *h = reinterpret_cast<const __half2 *>(&u);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -50,8 +66,6 @@ __device__ __forceinline__ void unpack8(uint4 u, float *x) {
         x[2 * e + 1] = f.y;
     }
 }
-
-template <typename T> __device__ __forceinline__ void load8_any(const T *p, float (&x)[8]) { load8(p, x); }
 
 template <typename Tout> __device__ __forceinline__ void store8_out(Tout *p, const float (&x)[8]);
 template <> __device__ __forceinline__ void store8_out<float>(float *p, const float (&x)[8]) {
@@ -68,25 +82,47 @@ template <> __device__ __forceinline__ void store8_out<bf16>(bf16 *p, const floa
     *reinterpret_cast<uint4 *>(p) = u;
 }
 
-template <int DV, typename Tin, typename Tout>
-__global__ void __launch_bounds__(128, 1)
-chunk_chain_kernel(const __half *__restrict__ Qt, const __half *__restrict__ Kt,
-                   const __half *__restrict__ Wn, const __half *__restrict__ Up,
-                   const __half *__restrict__ Aqk, const float *__restrict__ decay,
-                   const Tin *__restrict__ z, const float *__restrict__ norm_w,
-                   const float *__restrict__ S0, const int32_t *__restrict__ cu_seqlens,
-                   int n_seq, int n_tok, int H, Tout *__restrict__ out,
-                   float *__restrict__ S_final) {
+// Bounded wait; on expiry raise the CTA's abort flag and the device error word.
+// Once the flag is up every other wait of the CTA gives up quickly, so the
+// kernel always finishes.
+__device__ __forceinline__ bool chain_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+    for (uint32_t i = 0; i < chain::kMaxPolls; ++i) {
+        if (umma::mbar_try_wait(bar, parity)) return true;
+        if ((i & 255u) == 255u && *abort_flag) return false;
+    }
+    *abort_flag = 1;
+    atomicOr(&g_chain_err, 1u);
+    return false;
+}
+
+template <int DV, typename Tout>
+__global__ void __launch_bounds__(4 * DV, 1)
+chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const float *__restrict__ decay,
+                   const float *__restrict__ norm_w, const float *__restrict__ S0,
+                   const int32_t *__restrict__ cu_seqlens, int n_seq, int n_tok, int H,
+                   Tout *__restrict__ out, float *__restrict__ S_final) {
     using namespace chain;
+    // 4 * DV threads: warp w reads TMEM lane quadrant q = w % 4 and owns the
+    // 32-column group cg = w / 4 of every row it touches.
+    constexpr int NT = 4 * DV;
+    constexpr int NCG = DV / 32;
+    constexpr int HALF = NT / 2;                             // threads of one role
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sAP = sm + OFF_AP, *sBP = sm + OFF_BP, *sAS = sm + OFF_AS, *sAY = sm + OFF_AY,
-            *sBU = sm + OFF_BU;
-    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + OFF_MISC);
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + OFF_MISC + 16);
-    constexpr uint32_t TMEM_COLS = 2 * DV;   // P [0, DV), dS [DV, 2 DV)
+    uint8_t *sBP = sm + OFF_BP, *sBU = sm + OFF_BU;
+    uint64_t *full_a = reinterpret_cast<uint64_t *>(sm + OFF_MISC);   // [2]
+    uint64_t *full_z = full_a + 2;                                     // [2]
+    uint64_t *bar_p = full_a + 4, *bar_ys = full_a + 5;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + OFF_MISC + 64);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OFF_MISC + 68);
+    float *w1 = reinterpret_cast<float *>(sm + OFF_MISC + 128);      // 1 + norm_w  [DV]
+    float *red = w1 + DV;                                             // [NCG][64] partial sums
+    constexpr uint32_t TMEM_COLS = DV == 128 ? 512 : 256;   // P0, P1, dS
+    constexpr uint32_t BYTES_A = 4 * 8192 + 2 * 8192 + 8192 + C * DV * 2;
+    constexpr uint32_t BYTES_Z = C * DV * 2;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q = warp & 3, cg = warp >> 2, col0 = 32 * cg;
     const int h = blockIdx.x, n = blockIdx.y;
     int s_begin, s_end;
     if (cu_seqlens) { s_begin = __ldg(cu_seqlens + n); s_end = __ldg(cu_seqlens + n + 1); }
@@ -94,221 +130,227 @@ chunk_chain_kernel(const __half *__restrict__ Qt, const __half *__restrict__ Kt,
     const int n_chunks = (s_end - s_begin + C - 1) / C;
 
     if (warp == 0) umma::tmem_alloc(tslot, TMEM_COLS);
-    if (tid == 0) { umma::mbar_init(bar, 1); umma::fence_mbar_init(); }
-    // rows 0..63 of the A operand of Aqk U stay zero
-    for (int idx = tid; idx < 64 * 8; idx += 128)
-        umma::st_chunk(sAY, idx / 8, idx % 8, make_uint4(0, 0, 0, 0));
-
-    // fp32 master state: thread r owns row r of S; fp16 copy into sBP (rows = dk)
-    const size_t sbase = ((size_t)n * H + h) * DK * DV;
-    float S[DV];
-    {
-        const int r = tid;
-#pragma unroll
-        for (int c8 = 0; c8 < DV / 8; ++c8) {
-            float x[8];
-            if (S0) load8(S0 + sbase + (size_t)r * DV + c8 * 8, x);
-            else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] = 0.f;
-            }
-#pragma unroll
-            for (int e = 0; e < 8; ++e) S[c8 * 8 + e] = x[e];
-            umma::st_chunk(sBP + (c8 / 8) * 16384, r, c8 % 8, pack8(x));
-        }
+    if (tid == 0) {
+        for (int i = 0; i < 6; ++i) umma::mbar_init(full_a + i, 1);
+        *abort_flag = 0;
+        umma::fence_mbar_init();
     }
+    for (int j = tid; j < DV; j += NT) w1[j] = 1.0f + __ldg(norm_w + j);
+    // fp32 master state: this thread owns S[32 q + lane][col0 .. col0 + 32); fp16 copy in sBP
+    const int srow = 32 * q + lane;
+    const size_t sbase = ((size_t)n * H + h) * DK * DV;
+    float S[32];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        float x[8];
+        if (S0) load8(S0 + sbase + (size_t)srow * DV + col0 + 8 * m, x);
+        else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] = 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) S[8 * m + e] = x[e];
+        const int col = col0 + 8 * m;
+        umma::st_chunk(sBP + (col / 64) * 16384, srow, (col % 64) / 8, pack8(x));
+    }
+    umma::fence_proxy_async_smem();
+    umma::tc_fence_before();
     __syncthreads();
+    umma::tc_fence_after();
     const uint32_t tbase = *tslot;
-    const uint32_t tP = tbase, tS = tbase + DV;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    uint32_t phase = 0;
-    bool ok = true;
+    const uint32_t tD = tbase + 2 * DV;
+    const uint32_t lane_off = (uint32_t)(32 * q) << 16;
 
-    for (int c = 0; c < n_chunks && ok; ++c) {
+    auto stage = [&](int b) { return sm + b * STAGE; };
+    auto issue_a = [&](int cc, int b) {
+        const int t0 = s_begin + cc * C;
+        uint8_t *st = stage(b);
+        umma::mbar_expect_tx(full_a + b, BYTES_A);
+        umma::tma_load_3d(st + ST_AP, &maps.wn, 0, h, t0, full_a + b);
+        umma::tma_load_3d(st + ST_AP + 8192, &maps.qt, 0, h, t0, full_a + b);
+        umma::tma_load_3d(st + ST_AP + 16384, &maps.wn, 64, h, t0, full_a + b);
+        umma::tma_load_3d(st + ST_AP + 24576, &maps.qt, 64, h, t0, full_a + b);
+        umma::tma_load_3d(st + ST_AS, &maps.kt, 0, h, t0, full_a + b);
+        umma::tma_load_3d(st + ST_AS + 8192, &maps.kt, 64, h, t0, full_a + b);
+        umma::tma_load_3d(st + ST_AQK, &maps.aqk, 0, h, t0, full_a + b);
+#pragma unroll
+        for (int x = 0; x < DV; x += 64) umma::tma_load_3d(st + ST_US + x * 128, &maps.up, x, h, t0, full_a + b);
+    };
+    auto issue_z = [&](int cc, int b) {
+        umma::mbar_expect_tx(full_z + b, BYTES_Z);
+#pragma unroll
+        for (int x = 0; x < DV; x += 64)
+            umma::tma_load_3d(stage(b) + ST_ZS + x * 128, &maps.z, x, h, s_begin + cc * C, full_z + b);
+    };
+    if (tid == 0 && n_chunks > 0) {
+        issue_a(0, 0);
+        issue_z(0, 0);
+    }
+    // byte offset of the 8-column chunk `col` of row i in a 64-column-block swizzled tile
+    auto tile_off = [](int i, int col) { return (col / 64) * 8192 + umma::sw128_offset(i, (col % 64) / 8); };
+
+    for (int c = 0; c < n_chunks; ++c) {
+        const int b = c & 1;
         const int t0 = s_begin + c * C;
         const int len = min(C, s_end - t0);
+        const uint32_t ph_stage = (uint32_t)(c >> 1) & 1u, ph = (uint32_t)c & 1u;
+        uint8_t *st = stage(b);
+        const uint32_t tP = tbase + b * DV;
         const float dec = __ldg(decay + (size_t)t0 * H + h);
-        // ---- 1. stage -W, Qt (A of P), Kt (A of dS), Aqk (A of Y); U' / 0 into TMEM P
-        for (int idx = tid; idx < C * (DK / 8); idx += 128) {
-            const int i = idx / (DK / 8), ch = idx % (DK / 8);
-            uint4 w = make_uint4(0, 0, 0, 0), q = w, k = w;
-            if (i < len) {
-                const size_t g = ((size_t)(t0 + i) * H + h) * DK + ch * 8;
-                w = *reinterpret_cast<const uint4 *>(Wn + g);
-                q = *reinterpret_cast<const uint4 *>(Qt + g);
-                k = *reinterpret_cast<const uint4 *>(Kt + g);
+        if (tid == 0 && c + 1 < n_chunks) {
+            umma::fence_proxy_async_smem();
+            issue_a(c + 1, b ^ 1);
+        }
+        if (q < 2) {
+            // ---- P = [-W; Qt] S  (M=128, N=DV, K=dk)
+            if (tid == 0) {
+                chain_wait(full_a + b, ph_stage, abort_flag);
+                umma::tc_fence_after();
+                const uint32_t a0 = umma::smem_u32(st + ST_AP), b0 = umma::smem_u32(sBP);
+                const uint32_t idesc = umma::idesc_f16(128, DV, false, true);
+#pragma unroll
+                for (int s = 0; s < DK / 16; ++s)
+                    umma::mma_f16(tP, umma::sw128_desc(a0 + (s / 4) * 16384 + (s % 4) * 32, 16, 1024),
+                                  umma::sw128_desc(b0 + s * 2048, 16384, 1024), idesc, s > 0);
+                umma::mma_commit(bar_p);
             }
-            umma::st_chunk(sAP + (ch / 8) * 16384, i, ch % 8, w);
-            umma::st_chunk(sAP + (ch / 8) * 16384, 64 + i, ch % 8, q);
-            umma::st_chunk(sAS + (ch / 8) * 8192, i, ch % 8, k);
-        }
-        for (int idx = tid; idx < C * 8; idx += 128) {
-            const int i = idx / 8, ch = idx % 8;
-            uint4 a = make_uint4(0, 0, 0, 0);
-            if (i < len) a = *reinterpret_cast<const uint4 *>(Aqk + ((size_t)(t0 + i) * H + h) * C + ch * 8);
-            umma::st_chunk(sAY, 64 + i, ch, a);
-        }
-        {
-            const int i = (warp * 32 + lane) & 63;
-            const bool has = warp < 2 && i < len;
-            const __half *src = Up + ((size_t)(t0 + i) * H + h) * DV;
-#pragma unroll
-            for (int c0 = 0; c0 < DV; c0 += 32) {
-                float v[32];
-#pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) {
-                    if (has) unpack8(*reinterpret_cast<const uint4 *>(src + c0 + q8 * 8), v + q8 * 8);
-                    else {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) v[q8 * 8 + e] = 0.f;
-                    }
-                }
-                umma::tmem_st32(tP + lane_off + c0, v);
-            }
-            umma::tmem_st_wait();
-        }
-        umma::fence_proxy_async_smem();
-        umma::tc_fence_before();
-        __syncthreads();
-
-        // ---- 2. P += [-W; Qt] S    (M=128, N=DV, K=dk)
-        if (tid == 0) {
+            chain_wait(full_a + b, ph_stage, abort_flag);
+            chain_wait(bar_p, ph, abort_flag);
             umma::tc_fence_after();
-            const uint32_t a0 = umma::smem_u32(sAP), b0 = umma::smem_u32(sBP);
-            const uint32_t idesc = umma::idesc_f16(128, DV, false, true);
+            // ---- U = U' + P[0:64] (zero past the sequence end) -> fp16 MN-major B operand
+            const int i = srow;
+            float v[32];
+            umma::tmem_ld32(tP + lane_off + col0, v);
 #pragma unroll
-            for (int s = 0; s < DK / 16; ++s)
-                umma::mma_f16(tP, umma::sw128_desc(a0 + (s / 4) * 16384 + (s % 4) * 32, 16, 1024),
-                              umma::sw128_desc(b0 + s * 2048, 16384, 1024), idesc, 1u);
-            umma::mma_commit(bar);
-        }
-        ok = __syncthreads_and(umma::mbar_wait_bounded(bar, phase, 1u << 22));
-        phase ^= 1;
-        umma::tc_fence_after();
-        if (!ok) break;
-
-        // ---- 3. U = P[0:64] -> fp16 MN-major (rows = tokens) as the B operand
-        if (warp < 2) {
-            const int i = warp * 32 + lane;
+            for (int m = 0; m < 4; ++m) {
+                const int col = col0 + 8 * m;
+                float up[8], u[8];
+                unpack8h(*reinterpret_cast<const uint4 *>(st + ST_US + tile_off(i, col)), up);
 #pragma unroll
-            for (int c0 = 0; c0 < DV; c0 += 32) {
-                float v[32];
-                umma::tmem_ld32(tP + lane_off + c0, v);
+                for (int e = 0; e < 8; ++e) u[e] = (i < len) ? v[8 * m + e] + up[e] : 0.f;
+                umma::st_chunk(sBU + (col / 64) * 8192, i, (col % 64) / 8, pack8(u));
+            }
+            umma::fence_proxy_async_smem();
+            umma::tc_fence_before();
+            umma::named_bar_sync(1, HALF);
+            // ---- P[64:128] += [*; Aqk] U  (rows 0..63 of A are don't-care);  dS = Kt^T U
+            if (tid == 0) {
+                umma::tc_fence_after();
+                const uint32_t aY = umma::smem_u32(st + ST_AS + 8192), aS = umma::smem_u32(st + ST_AS);
+                const uint32_t bU = umma::smem_u32(sBU);
+                const uint32_t idy = umma::idesc_f16(128, DV, false, true);
+                const uint32_t ids = umma::idesc_f16(128, DV, true, true);
 #pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) {
-                    const int col = c0 + q8 * 8;
-                    umma::st_chunk(sBU + (col / 64) * 8192, i, (col % 64) / 8, pack8(v + q8 * 8));
+                for (int s = 0; s < C / 16; ++s) {
+                    const uint64_t bd = umma::sw128_desc(bU + s * 2048, 8192, 1024);
+                    umma::mma_f16(tP, umma::sw128_desc(aY + s * 32, 16, 1024), bd, idy, 1u);
+                    umma::mma_f16(tD, umma::sw128_desc(aS + s * 2048, 8192, 1024), bd, ids, s > 0);
                 }
+                umma::mma_commit(bar_ys);
+            }
+        }
+        chain_wait(bar_ys, ph, abort_flag);
+        umma::tc_fence_after();
+        // ---- S = e^{G_C} S + dS; fp16 copy for the next chunk
+        {
+            float v[32];
+            umma::tmem_ld32(tD + lane_off + col0, v);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) S[j] = fmaf(dec, S[j], v[j]);
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int col = col0 + 8 * m;
+                umma::st_chunk(sBP + (col / 64) * 16384, srow, (col % 64) / 8, pack8(S + 8 * m));
             }
         }
         umma::fence_proxy_async_smem();
         umma::tc_fence_before();
         __syncthreads();
-
-        // ---- 4. P += [0; Aqk] U  (Y in rows 64..127);  dS = Kt^T U
-        if (tid == 0) {
-            umma::tc_fence_after();
-            const uint32_t aY = umma::smem_u32(sAY), aS = umma::smem_u32(sAS), bU = umma::smem_u32(sBU);
-            const uint32_t idy = umma::idesc_f16(128, DV, false, true);
-            const uint32_t ids = umma::idesc_f16(128, DV, true, true);
-#pragma unroll
-            for (int s = 0; s < C / 16; ++s) {
-                const uint64_t bd = umma::sw128_desc(bU + s * 2048, 8192, 1024);
-                umma::mma_f16(tP, umma::sw128_desc(aY + s * 32, 16, 1024), bd, idy, 1u);
-                umma::mma_f16(tS, umma::sw128_desc(aS + s * 2048, 8192, 1024), bd, ids, s > 0);
-            }
-            umma::mma_commit(bar);
-        }
-        ok = __syncthreads_and(umma::mbar_wait_bounded(bar, phase, 1u << 22));
-        phase ^= 1;
         umma::tc_fence_after();
-        if (!ok) break;
-
-        // ---- 5a. S = e^{G_C} S + dS; fp16 copy for the next chunk
-        {
-            const int r = tid;
-#pragma unroll
-            for (int c0 = 0; c0 < DV; c0 += 32) {
-                float v[32];
-                umma::tmem_ld32(tS + lane_off + c0, v);
-#pragma unroll
-                for (int j = 0; j < 32; ++j) S[c0 + j] = fmaf(dec, S[c0 + j], v[j]);
-#pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) {
-                    const int col = c0 + q8 * 8;
-                    umma::st_chunk(sBP + (col / 64) * 16384, r, (col % 64) / 8, pack8(S + col));
-                }
-            }
+        if (tid == 0 && c + 1 < n_chunks) {
+            umma::fence_proxy_async_smem();
+            issue_z(c + 1, b ^ 1);
         }
-        // ---- 5b. output stage on Y = P[64:128] (warps 2, 3): two passes over TMEM
-        if (warp >= 2) {
-            const int i = (warp - 2) * 32 + lane;
+        // ---- output stage of this chunk on P[64:128] (quadrants 2, 3): overlaps chunk c + 1
+        if (q >= 2) {
+            const int i = srow - 64;
+            float v[32];
+            umma::tmem_ld32(tP + lane_off + col0, v);
             float ss = 0.f;
 #pragma unroll
-            for (int c0 = 0; c0 < DV; c0 += 32) {
-                float v[32];
-                umma::tmem_ld32(tP + lane_off + c0, v);
+            for (int j = 0; j < 32; ++j) ss = fmaf(v[j], v[j], ss);
+            red[cg * 64 + i] = ss;
+            chain_wait(full_z + b, ph_stage, abort_flag);
+            umma::named_bar_sync(2, HALF);
+            float tot = 0.f;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) ss = fmaf(v[j], v[j], ss);
-            }
-            const float rr = 1.0f / sqrtf(ss / DV + kNormEps);
-            const size_t g = ((size_t)(t0 + i) * H + h) * DV;
+            for (int g2 = 0; g2 < NCG; ++g2) tot += red[g2 * 64 + i];
+            const float rr = rsqrtf(tot / DV + kNormEps);
+            if (i < len) {
+                const size_t g = ((size_t)(t0 + i) * H + h) * DV;
 #pragma unroll
-            for (int c0 = 0; c0 < DV; c0 += 32) {
-                float v[32];
-                umma::tmem_ld32(tP + lane_off + c0, v);
-                if (i < len) {
+                for (int m = 0; m < 4; ++m) {
+                    const int col = col0 + 8 * m;
+                    const uint4 zz = *reinterpret_cast<const uint4 *>(st + ST_ZS + tile_off(i, col));
+                    const uint32_t zw[4] = {zz.x, zz.y, zz.z, zz.w};
+                    float o[8];
 #pragma unroll
-                    for (int q8 = 0; q8 < 4; ++q8) {
-                        const int col = c0 + q8 * 8;
-                        float zz[8], o[8];
-                        load8(z + g + col, zz);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const float w1 = 1.0f + __ldg(norm_w + col + e);
-                            o[e] = sigmoid_acc(zz[e]) * v[q8 * 8 + e] * rr * w1;
-                        }
-                        store8_out<Tout>(out + g + col, o);
+                    for (int e = 0; e < 4; ++e) {
+                        const float z0 = bf16lo(zw[e]), z1 = bf16hi(zw[e]);
+                        o[2 * e] = __fdividef(v[8 * m + 2 * e] * rr * w1[col + 2 * e], 1.0f + __expf(-z0));
+                        o[2 * e + 1] = __fdividef(v[8 * m + 2 * e + 1] * rr * w1[col + 2 * e + 1], 1.0f + __expf(-z1));
                     }
+                    store8_out<Tout>(out + g + col, o);
                 }
             }
         }
-        umma::fence_proxy_async_smem();
-        umma::tc_fence_before();
-        __syncthreads();
     }
-    if (!ok && tid == 0) atomicOr(&g_chain_err, 1u);
-    if (ok && S_final) {
-        const int r = tid;
+    if (S_final && !*abort_flag) {
 #pragma unroll
-        for (int c8 = 0; c8 < DV / 8; ++c8) {
+        for (int m = 0; m < 4; ++m) {
             float x[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] = S[c8 * 8 + e];
-            store8(S_final + sbase + (size_t)r * DV + c8 * 8, x);
+            for (int e = 0; e < 8; ++e) x[e] = S[8 * m + e];
+            store8(S_final + sbase + (size_t)srow * DV + col0 + 8 * m, x);
         }
     }
     umma::tc_fence_before();
     __syncthreads();
+    if (*abort_flag && tid == 0 && n_chunks > 0) {
+        // let any tile copy still in flight land before the CTA exits (bounded)
+        for (int b = 0; b < 2 && b < n_chunks; ++b) {
+            const int last = ((n_chunks - 1 - b) / 2) * 2 + b;   // last chunk that used stage b
+            umma::mbar_wait_bounded(full_a + b, (uint32_t)(last >> 1) & 1u, 1u << 16);
+            umma::mbar_wait_bounded(full_z + b, (uint32_t)(last >> 1) & 1u, 1u << 16);
+        }
+    }
     if (warp == 0) umma::tmem_dealloc(tbase, TMEM_COLS);
 }
 
 cudaError_t launch_chunk_chain(const PrefillArgs &a, const TcWorkspace &w) {
+    ChainMaps m;
+    std::memset(&m, 0, sizeof m);
+    if (a.n_tok > 0) {
+        cudaError_t e;
+        if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.wn), w.Wn, false, 128, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
+        if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.qt), w.Qt, false, 128, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
+        if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.kt), w.Kt, false, 128, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
+        if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.aqk), w.Aqk, false, 64, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
+        if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.up), w.Up, false, a.dv, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
+        if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.z), a.z, true, a.dv, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
+    }
     dim3 grid(a.H, a.n_seq);
     cudaError_t e;
-#define GDN_CHAIN(DV_, TIN, TOUT)                                                                 \
-    e = cudaFuncSetAttribute(chunk_chain_kernel<DV_, TIN, TOUT>,                                  \
+#define GDN_CHAIN(DV_, TOUT)                                                                      \
+    e = cudaFuncSetAttribute(chunk_chain_kernel<DV_, TOUT>,                                       \
                              cudaFuncAttributeMaxDynamicSharedMemorySize, chain::SMEM);            \
     if (e != cudaSuccess) return e;                                                               \
-    chunk_chain_kernel<DV_, TIN, TOUT><<<grid, 128, chain::SMEM, a.stream>>>(                     \
-        w.Qt, w.Kt, w.Wn, w.Up, w.Aqk, w.decay, (const TIN *)a.z, a.norm_w, a.S0, a.cu_seqlens, \
-        a.n_seq, a.n_tok, a.H, (TOUT *)a.out, a.S_final)
+    chunk_chain_kernel<DV_, TOUT><<<grid, 4 * DV_, chain::SMEM, a.stream>>>(                          \
+        m, w.decay, a.norm_w, a.S0, a.cu_seqlens, a.n_seq, a.n_tok, a.H, (TOUT *)a.out, a.S_final)
     if (a.dv == 128) {
-        if (a.in_bf16) { if (a.out_bf16) { GDN_CHAIN(128, bf16, bf16); } else { GDN_CHAIN(128, bf16, float); } }
-        else { if (a.out_bf16) { GDN_CHAIN(128, float, bf16); } else { GDN_CHAIN(128, float, float); } }
+        if (a.out_bf16) { GDN_CHAIN(128, bf16); } else { GDN_CHAIN(128, float); }
     } else {
-        if (a.in_bf16) { if (a.out_bf16) { GDN_CHAIN(64, bf16, bf16); } else { GDN_CHAIN(64, bf16, float); } }
-        else { if (a.out_bf16) { GDN_CHAIN(64, float, bf16); } else { GDN_CHAIN(64, float, float); } }
+        if (a.out_bf16) { GDN_CHAIN(64, bf16); } else { GDN_CHAIN(64, float); }
     }
 #undef GDN_CHAIN
     return cudaGetLastError();

@@ -45,6 +45,12 @@ struct TcWorkspace {
 cudaError_t launch_chunk_prep(const PrefillArgs &a, const TcWorkspace &w);
 cudaError_t launch_chunk_chain(const PrefillArgs &a, const TcWorkspace &w);
 
+// Host side of TMA: a 3-D tiled tensor map over a token-indexed [N_tok][H][inner]
+// tensor (16-bit elements), box {box_inner, 1, box_rows}.
+struct TmaMap { alignas(64) unsigned char bytes[128]; };
+cudaError_t make_tma_3d(TmaMap *out, const void *base, bool bf16, int inner, int H, int n_tok,
+                        int box_inner, int box_rows, bool swizzle128);
+
 // K2f: token-by-token recurrence with the fused gates and output stage (SIMT fp32).
 cudaError_t launch_recurrent(const PrefillArgs &a, const float *qn, const float *kn,
                              const float *vn);

@@ -192,3 +192,33 @@ __device__ __forceinline__ void st_chunk(uint8_t *block, int r, int chunk, uint4
 
 }  // namespace umma
 }  // namespace gdn
+
+// ------------------------------------------------------------------ TMA loads
+// Tiled bulk-tensor loads (no multicast) into this CTA's shared memory,
+// completing on an mbarrier with a transaction count.
+#include <cuda.h>
+
+namespace gdn {
+namespace umma {
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int x, int y, int z,
+                                            uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+}  // namespace umma
+}  // namespace gdn
