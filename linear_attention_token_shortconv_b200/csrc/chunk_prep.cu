@@ -23,9 +23,10 @@
 // (x = hi + lo): [Qh;Kh]Kh^T + [Qh;Kh]Kl^T + [Ql;Kl]Kh^T, fp32 accumulation.
 //
 // Per chunk: prelude in registers -> fp16 hi/lo tiles in smem; the split
-// [Q;K]K^T on tcgen05 (M=128, N=64) -> TMEM; Aqk and L from TMEM; T by forward
-// substitution in fp32; [T diag(beta e^G); T diag(beta)] times K and V on
-// tcgen05 -> TMEM; results to global memory in fp16.
+// [Q;K]K^T on tcgen05 (M=128, N=64) -> TMEM, with Qt and Kt written out while
+// it runs; Aqk and L from TMEM; T by blocked forward substitution in fp32 over
+// all 128 threads; [T diag(beta e^G); T diag(beta)] times K and V on tcgen05 ->
+// TMEM; results to global memory in fp16.
 #include <cuda_fp16.h>
 
 #include "gdn_device.cuh"
@@ -40,11 +41,11 @@ namespace prep {
 constexpr int C = 64;          // chunk length
 constexpr int DK = 128;
 constexpr int OFF_HI = 0;      // [Qh;Kh] K-major, 2 k-blocks x 16 KB
-constexpr int OFF_LO = 32768;  // [Ql;Kl] K-major, 2 k-blocks x 16 KB; later L fp32 [64][64]
+constexpr int OFF_LO = 32768;  // [Ql;Kl] K-major, 2 k-blocks x 16 KB; later L and T fp32 [64][64]
 constexpr int OFF_V = 65536;   // V MN-major, DV/64 mn-blocks x 8 KB
 constexpr int OFF_T = 81920;   // [T'; T''] K-major, 1 k-block x 16 KB
-constexpr int OFF_MISC = 98304;
-constexpr int SMEM = OFF_MISC + 1024 + 1024;
+constexpr int OFF_MISC = 98304;  // G, beta, barriers [0, 1024); block products [1024, 4096)
+constexpr int SMEM = OFF_MISC + 4096 + 1024;
 constexpr uint32_t TMEM_COLS = 256;
 }  // namespace prep
 
@@ -63,45 +64,132 @@ __device__ __forceinline__ void split_store(uint8_t *hi_blk, uint8_t *lo_blk, in
     umma::st_chunk(lo_blk, row, chunk, make_uint4(l[0], l[1], l[2], l[3]));
 }
 
-// Conv + SiLU of 8 channels for tokens [i0, i0 + n) of a chunk (sliding window
-// over the raw rows, zero before the sequence start); emits each row to `emit`.
-template <typename Tin, typename Emit>
-__device__ __forceinline__ void conv_rows(const Tin *src, size_t row_stride, int col,
+// Conv + SiLU of 8 channels for tokens [i0, i0 + N) of a chunk: all N + 3 raw
+// rows (zero before the sequence start and past its end) are loaded first, then
+// the window slides over them; each output row goes to `emit`.
+template <int N, typename Emit>
+__device__ __forceinline__ void conv_rows(const bf16 *src, size_t row_stride, int col,
                                           const float (&w)[8][4], int t0, int s_begin, int i0,
-                                          int n, int len, Emit emit) {
-    float h0[8], h1[8], h2[8];
+                                          int len, Emit emit) {
+    uint4 raw[N + 3];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) h0[e] = h1[e] = h2[e] = 0.f;
-    const int ta = t0 + i0;
-    if (ta - 3 >= s_begin) load8(src + (size_t)(ta - 3) * row_stride + col, h0);
-    if (ta - 2 >= s_begin) load8(src + (size_t)(ta - 2) * row_stride + col, h1);
-    if (ta - 1 >= s_begin) load8(src + (size_t)(ta - 1) * row_stride + col, h2);
-    for (int ii = 0; ii < n; ++ii) {
+    for (int r = 0; r < N + 3; ++r) {
+        const int i = i0 + r - 3;            // chunk-relative row
+        const int t = t0 + i;
+        const bool ok = (i < len) && (t >= s_begin);
+        raw[r] = ok ? __ldg(reinterpret_cast<const uint4 *>(src + (size_t)t * row_stride + col))
+                    : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int ii = 0; ii < N; ++ii) {
         const int i = i0 + ii;
-        float x[8], y[8];
-        if (i < len) load8(src + (size_t)(t0 + i) * row_stride + col, x);
-        else {
+        float x[4][8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] = 0.f;
+        for (int r = 0; r < 4; ++r) {
+            const uint4 u = raw[ii + r];
+            x[r][0] = bf16lo(u.x); x[r][1] = bf16hi(u.x); x[r][2] = bf16lo(u.y); x[r][3] = bf16hi(u.y);
+            x[r][4] = bf16lo(u.z); x[r][5] = bf16hi(u.z); x[r][6] = bf16lo(u.w); x[r][7] = bf16hi(u.w);
         }
+        float y[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-            float a = w[e][0] * h0[e];
-            a = fmaf(w[e][1], h1[e], a);
-            a = fmaf(w[e][2], h2[e], a);
-            a = fmaf(w[e][3], x[e], a);
-            y[e] = (i < len) ? siluf_(a) : 0.f;
-            h0[e] = h1[e]; h1[e] = h2[e]; h2[e] = x[e];
+            float a = w[e][0] * x[0][e];
+            a = fmaf(w[e][1], x[1][e], a);
+            a = fmaf(w[e][2], x[2][e], a);
+            a = fmaf(w[e][3], x[3][e], a);
+            y[e] = (i < len) ? __fdividef(a, 1.0f + __expf(-a)) : 0.f;
         }
         emit(i, y);
     }
 }
 
-template <int DV, typename Tin>
+// acc(r, c) += sum_k A[ar + r][ac + k] * B[br + k][bc + c] over a 16 x 16 block
+// product, A and B row-major fp32 [64][64] in shared memory.
+__device__ __forceinline__ float blk16(const float *A, int ar, int ac, const float *B, int br, int bc,
+                                       int r, int c, float acc) {
+    const float4 *a = reinterpret_cast<const float4 *>(A + (ar + r) * 64 + ac);
+#pragma unroll
+    for (int k4 = 0; k4 < 4; ++k4) {
+        const float4 av = a[k4];
+        acc = fmaf(av.x, B[(br + 4 * k4 + 0) * 64 + bc + c], acc);
+        acc = fmaf(av.y, B[(br + 4 * k4 + 1) * 64 + bc + c], acc);
+        acc = fmaf(av.z, B[(br + 4 * k4 + 2) * 64 + bc + c], acc);
+        acc = fmaf(av.w, B[(br + 4 * k4 + 3) * 64 + bc + c], acc);
+    }
+    return acc;
+}
+
+// T = (I + L)^-1 for a strictly lower triangular 64 x 64 L, by 16 x 16 blocks:
+// diagonal blocks by forward substitution, then block row-diagonals
+//   T_{b+d,b} = -D_{b+d} sum_{j=b}^{b+d-1} L_{b+d,j} T_{j,b},  D_b = (I + L_bb)^-1.
+// 128 threads; X is a [3][16][16] scratch.  Only the block-lower part of T is written.
+__device__ __forceinline__ void solve_unit_lower(const float *L, float *T, float *X, int tid) {
+    if (tid < 64) {   // diagonal blocks: thread (b, c) owns column c of D_b
+        const int b = tid >> 4, cc = tid & 15, o = 16 * b;
+        float x[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            float acc = (r == cc) ? 1.f : 0.f;
+#pragma unroll
+            for (int j = 0; j < r; ++j) acc = fmaf(-L[(o + r) * 64 + o + j], x[j], acc);
+            x[r] = acc;
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) T[(o + r) * 64 + o + cc] = x[r];
+    }
+    __syncthreads();
+    // d = 1: X_b = L_{b+1,b} D_b, then T_{b+1,b} = -D_{b+1} X_b   (b = 0, 1, 2)
+    for (int e = tid; e < 3 * 256; e += 128) {
+        const int b = e >> 8, r = (e >> 4) & 15, cc = e & 15;
+        X[e] = blk16(L, 16 * (b + 1), 16 * b, T, 16 * b, 16 * b, r, cc, 0.f);
+    }
+    __syncthreads();
+    for (int e = tid; e < 3 * 256; e += 128) {
+        const int b = e >> 8, r = (e >> 4) & 15, cc = e & 15;
+        float acc = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) acc = fmaf(T[(16 * (b + 1) + r) * 64 + 16 * (b + 1) + k], X[(b << 8) + k * 16 + cc], acc);
+        T[(16 * (b + 1) + r) * 64 + 16 * b + cc] = -acc;
+    }
+    __syncthreads();
+    // d = 2: X_b = L_{b+2,b} D_b + L_{b+2,b+1} T_{b+1,b}, then T_{b+2,b} = -D_{b+2} X_b   (b = 0, 1)
+    for (int e = tid; e < 2 * 256; e += 128) {
+        const int b = e >> 8, r = (e >> 4) & 15, cc = e & 15;
+        float acc = blk16(L, 16 * (b + 2), 16 * b, T, 16 * b, 16 * b, r, cc, 0.f);
+        X[e] = blk16(L, 16 * (b + 2), 16 * (b + 1), T, 16 * (b + 1), 16 * b, r, cc, acc);
+    }
+    __syncthreads();
+    for (int e = tid; e < 2 * 256; e += 128) {
+        const int b = e >> 8, r = (e >> 4) & 15, cc = e & 15;
+        float acc = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) acc = fmaf(T[(16 * (b + 2) + r) * 64 + 16 * (b + 2) + k], X[(b << 8) + k * 16 + cc], acc);
+        T[(16 * (b + 2) + r) * 64 + 16 * b + cc] = -acc;
+    }
+    __syncthreads();
+    // d = 3: X = L_30 D_0 + L_31 T_10 + L_32 T_20, then T_30 = -D_3 X
+    for (int e = tid; e < 256; e += 128) {
+        const int r = e >> 4, cc = e & 15;
+        float acc = blk16(L, 48, 0, T, 0, 0, r, cc, 0.f);
+        acc = blk16(L, 48, 16, T, 16, 0, r, cc, acc);
+        X[e] = blk16(L, 48, 32, T, 32, 0, r, cc, acc);
+    }
+    __syncthreads();
+    for (int e = tid; e < 256; e += 128) {
+        const int r = e >> 4, cc = e & 15;
+        float acc = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) acc = fmaf(T[(48 + r) * 64 + 48 + k], X[k * 16 + cc], acc);
+        T[(48 + r) * 64 + cc] = -acc;
+    }
+    __syncthreads();
+}
+
+template <int DV>
 __global__ void __launch_bounds__(128)
-chunk_prep_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
-                  const float *__restrict__ conv_w, const Tin *__restrict__ a_logit,
-                  const Tin *__restrict__ b_logit, const float *__restrict__ A,
+chunk_prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const bf16 *__restrict__ v,
+                  const float *__restrict__ conv_w, const bf16 *__restrict__ a_logit,
+                  const bf16 *__restrict__ b_logit, const float *__restrict__ A,
                   const float *__restrict__ b_alpha, const int32_t *__restrict__ cu_seqlens,
                   int n_seq, int n_tok, int H, __half *__restrict__ Qt, __half *__restrict__ Kt,
                   __half *__restrict__ Wn, __half *__restrict__ Up, __half *__restrict__ Aqk,
@@ -111,6 +199,8 @@ chunk_prep_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Ti
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sHI = sm + OFF_HI, *sLO = sm + OFF_LO, *sV = sm + OFF_V, *sT = sm + OFF_T;
     float *sL = reinterpret_cast<float *>(sm + OFF_LO);          // aliases [Ql;Kl] after the q.k MMA
+    float *sTf = sL + 64 * 64;                                   // fp32 T, same region
+    float *sX = reinterpret_cast<float *>(sm + OFF_MISC + 1024); // [3][16][16]
     float *sG = reinterpret_cast<float *>(sm + OFF_MISC);        // 64
     float *sBeta = sG + 64;                                      // 64
     float *sTot = sBeta + 64;                                    // 1
@@ -150,35 +240,40 @@ chunk_prep_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Ti
         const int len = min(C, s_end - t0);
         // ---- 1. prelude: q, k -> L2-normalised fp32 -> hi/lo fp16 tiles; v -> fp16 tile
         // (conv weights re-read per chunk from L1/L2 to keep them out of the solve's registers)
-        float wqk[8][4], wv[8][4];
+        {
+            float wqk[8][4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const float4 a4 = __ldg(reinterpret_cast<const float4 *>(conv_w) + qk_chan + e);
-            wqk[e][0] = a4.x; wqk[e][1] = a4.y; wqk[e][2] = a4.z; wqk[e][3] = a4.w;
+            for (int e = 0; e < 8; ++e) {
+                const float4 a4 = __ldg(reinterpret_cast<const float4 *>(conv_w) + qk_chan + e);
+                wqk[e][0] = a4.x; wqk[e][1] = a4.y; wqk[e][2] = a4.z; wqk[e][3] = a4.w;
+            }
+            conv_rows<16>(is_k ? k : q, (size_t)H * DK, qk_col, wqk, t0, s_begin, 16 * warp, len,
+                          [&](int i, float (&y)[8]) {
+                              float ss = 0.f;
+#pragma unroll
+                              for (int e = 0; e < 8; ++e) ss = fmaf(y[e], y[e], ss);
+                              ss = group_sum<16>(ss);
+                              const float r = rsqrtf(ss + kNormEps);
+#pragma unroll
+                              for (int e = 0; e < 8; ++e) y[e] *= r;
+                              const int row = (is_k ? 64 : 0) + i, oc = qk_oct & 15;
+                              split_store(sHI + (oc / 8) * 16384, sLO + (oc / 8) * 16384, row, oc % 8, y);
+                          });
         }
-        conv_rows(is_k ? k : q, (size_t)H * DK, qk_col, wqk, t0, s_begin, 16 * warp, 16, len,
-                  [&](int i, float (&y)[8]) {
-                      float ss = 0.f;
+        {
+            float wv[8][4];
 #pragma unroll
-                      for (int e = 0; e < 8; ++e) ss = fmaf(y[e], y[e], ss);
-                      ss = group_sum<16>(ss);
-                      const float r = rsqrtf(ss + kNormEps);
-#pragma unroll
-                      for (int e = 0; e < 8; ++e) y[e] *= r;
-                      const int row = (is_k ? 64 : 0) + i, oc = qk_oct & 15;
-                      split_store(sHI + (oc / 8) * 16384, sLO + (oc / 8) * 16384, row, oc % 8, y);
-                  });
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const float4 b4 = __ldg(reinterpret_cast<const float4 *>(conv_w) + v_chan + e);
-            wv[e][0] = b4.x; wv[e][1] = b4.y; wv[e][2] = b4.z; wv[e][3] = b4.w;
+            for (int e = 0; e < 8; ++e) {
+                const float4 b4 = __ldg(reinterpret_cast<const float4 *>(conv_w) + v_chan + e);
+                wv[e][0] = b4.x; wv[e][1] = b4.y; wv[e][2] = b4.z; wv[e][3] = b4.w;
+            }
+            conv_rows<C / VPARTS>(v, (size_t)H * DV, v_col, wv, t0, s_begin, (C / VPARTS) * v_part, len,
+                                  [&](int i, float (&y)[8]) {
+                                      umma::st_chunk(sV + (v_oct / 8) * 8192, i, v_oct % 8,
+                                                     make_uint4(umma::pack_half2(y[0], y[1]), umma::pack_half2(y[2], y[3]),
+                                                                umma::pack_half2(y[4], y[5]), umma::pack_half2(y[6], y[7])));
+                                  });
         }
-        conv_rows(v, (size_t)H * DV, v_col, wv, t0, s_begin, (C / VPARTS) * v_part, C / VPARTS, len,
-                  [&](int i, float (&y)[8]) {
-                      umma::st_chunk(sV + (v_oct / 8) * 8192, i, v_oct % 8,
-                                     make_uint4(umma::pack_half2(y[0], y[1]), umma::pack_half2(y[2], y[3]),
-                                                umma::pack_half2(y[4], y[5]), umma::pack_half2(y[6], y[7])));
-                  });
         if (tid < C) {
             float g = 0.f, be = 0.f;
             if (tid < len) {
@@ -216,6 +311,30 @@ chunk_prep_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Ti
                 umma::mma_f16(tbase, al, bh, idesc, 1u);
             }
             umma::mma_commit(bar);
+        }
+        // while the MMA runs: Qt = e^{G_i} q_i, Kt = e^{G_C - G_i} k_i (fp16) and e^{G_C}
+        {
+            const float GC = sG[C - 1];
+            for (int idx = tid; idx < len * (DK / 8); idx += 128) {
+                const int i = idx / (DK / 8), ch = idx % (DK / 8);
+                const float sq = __expf(sG[i]), sk = __expf(GC - sG[i]);
+                const uint4 qv = *reinterpret_cast<const uint4 *>(sHI + (ch / 8) * 16384 + umma::sw128_offset(i, ch % 8));
+                const uint4 kv = *reinterpret_cast<const uint4 *>(sHI + (ch / 8) * 16384 + umma::sw128_offset(64 + i, ch % 8));
+                const __half2 *q2 = reinterpret_cast<const __half2 *>(&qv);
+                const __half2 *k2 = reinterpret_cast<const __half2 *>(&kv);
+                uint4 qo, ko;
+                uint32_t *qo32 = reinterpret_cast<uint32_t *>(&qo), *ko32 = reinterpret_cast<uint32_t *>(&ko);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 qf = __half22float2(q2[e]), kf = __half22float2(k2[e]);
+                    qo32[e] = umma::pack_half2(qf.x * sq, qf.y * sq);
+                    ko32[e] = umma::pack_half2(kf.x * sk, kf.y * sk);
+                }
+                const size_t g = ((size_t)(t0 + i) * H + h) * DK + ch * 8;
+                *reinterpret_cast<uint4 *>(Qt + g) = qo;
+                *reinterpret_cast<uint4 *>(Kt + g) = ko;
+            }
+            if (tid == 0) decay[(size_t)t0 * H + h] = __expf(GC);
         }
         ok = __syncthreads_and(umma::mbar_wait_bounded(bar, phase, 1u << 22));
         phase ^= 1;
@@ -264,57 +383,28 @@ chunk_prep_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Ti
         umma::tc_fence_before();
         __syncthreads();
 
-        // ---- 4. T = (I + L)^-1 by forward substitution, thread c owns column c
-        if (tid < C) {
-            const int cc = tid;
-            float Tc[C];
+        // ---- 4. T = (I + L)^-1 (fp32, blocked); then T' = T diag(beta e^G) in rows
+        //         0..63 and T'' = T diag(beta) in rows 64..127 of an fp16 K-major tile
+        solve_unit_lower(sL, sTf, sX, tid);
+        for (int idx = tid; idx < C * 8; idx += 128) {
+            const int i = idx >> 3, ch = idx & 7;
+            const float4 *tr = reinterpret_cast<const float4 *>(sTf + i * C + ch * 8);
+            const float4 t0v = tr[0], t1v = tr[1];
+            const float tv[8] = {t0v.x, t0v.y, t0v.z, t0v.w, t1v.x, t1v.y, t1v.z, t1v.w};
+            float a1[8], a2[8];
 #pragma unroll
-            for (int i = 0; i < C; ++i) {
-                float acc = (i == cc) ? 1.f : 0.f;
-                const float4 *Li = reinterpret_cast<const float4 *>(sL + i * C);
-#pragma unroll
-                for (int j4 = 0; j4 < i / 4; ++j4) {
-                    const float4 l = Li[j4];
-                    acc = fmaf(-l.x, Tc[4 * j4], acc);
-                    acc = fmaf(-l.y, Tc[4 * j4 + 1], acc);
-                    acc = fmaf(-l.z, Tc[4 * j4 + 2], acc);
-                    acc = fmaf(-l.w, Tc[4 * j4 + 3], acc);
-                }
-#pragma unroll
-                for (int j = (i / 4) * 4; j < i; ++j) acc = fmaf(-sL[i * C + j], Tc[j], acc);
-                Tc[i] = acc;
+            for (int e = 0; e < 8; ++e) {
+                const int j = ch * 8 + e;
+                // only the block-lower part of T was written: zero the rest
+                const float t = ((j >> 4) <= (i >> 4)) ? tv[e] : 0.f;
+                const float bj = sBeta[j];
+                a1[e] = t * bj * __expf(sG[j]);
+                a2[e] = t * bj;
             }
-            // T' = T diag(beta e^G) (rows 0..63), T'' = T diag(beta) (rows 64..127); K index = cc
-            const float bc = sBeta[cc], bgc = bc * __expf(sG[cc]);
-            const int chunk = cc / 8, within = (cc % 8) * 2;
-#pragma unroll
-            for (int i = 0; i < C; ++i) {
-                *reinterpret_cast<__half *>(sT + umma::sw128_offset(i, chunk) + within) = __float2half_rn(Tc[i] * bgc);
-                *reinterpret_cast<__half *>(sT + umma::sw128_offset(64 + i, chunk) + within) = __float2half_rn(Tc[i] * bc);
-            }
-        } else {
-            // Qt = e^{G_i} q_i and Kt = e^{G_C - G_i} k_i from the hi tiles (fp16 outputs)
-            const float GC = sG[C - 1];
-            for (int idx = tid - C; idx < len * (DK / 8); idx += 128 - C) {
-                const int i = idx / (DK / 8), ch = idx % (DK / 8);
-                const float sq = __expf(sG[i]), sk = __expf(GC - sG[i]);
-                const uint4 qv = *reinterpret_cast<const uint4 *>(sHI + (ch / 8) * 16384 + umma::sw128_offset(i, ch % 8));
-                const uint4 kv = *reinterpret_cast<const uint4 *>(sHI + (ch / 8) * 16384 + umma::sw128_offset(64 + i, ch % 8));
-                const __half2 *q2 = reinterpret_cast<const __half2 *>(&qv);
-                const __half2 *k2 = reinterpret_cast<const __half2 *>(&kv);
-                uint4 qo, ko;
-                uint32_t *qo32 = reinterpret_cast<uint32_t *>(&qo), *ko32 = reinterpret_cast<uint32_t *>(&ko);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 qf = __half22float2(q2[e]), kf = __half22float2(k2[e]);
-                    qo32[e] = umma::pack_half2(qf.x * sq, qf.y * sq);
-                    ko32[e] = umma::pack_half2(kf.x * sk, kf.y * sk);
-                }
-                const size_t g = ((size_t)(t0 + i) * H + h) * DK + ch * 8;
-                *reinterpret_cast<uint4 *>(Qt + g) = qo;
-                *reinterpret_cast<uint4 *>(Kt + g) = ko;
-            }
-            if (tid == C) decay[(size_t)t0 * H + h] = __expf(GC);
+            umma::st_chunk(sT, i, ch, make_uint4(umma::pack_half2(a1[0], a1[1]), umma::pack_half2(a1[2], a1[3]),
+                                                 umma::pack_half2(a1[4], a1[5]), umma::pack_half2(a1[6], a1[7])));
+            umma::st_chunk(sT, 64 + i, ch, make_uint4(umma::pack_half2(a2[0], a2[1]), umma::pack_half2(a2[2], a2[3]),
+                                                      umma::pack_half2(a2[4], a2[5]), umma::pack_half2(a2[6], a2[7])));
         }
         umma::fence_proxy_async_smem();
         __syncthreads();
@@ -389,19 +479,16 @@ cudaError_t launch_chunk_prep(const PrefillArgs &a, const TcWorkspace &w) {
     split = min(split, (a.n_tok + 63) / 64);
     dim3 grid(a.H, a.n_seq, split);
     cudaError_t e;
-#define GDN_PREP(DV_, TIN)                                                                        \
-    e = cudaFuncSetAttribute(chunk_prep_kernel<DV_, TIN>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                             prep::SMEM);                                                       \
-    if (e != cudaSuccess) return e;                                                              \
-    chunk_prep_kernel<DV_, TIN><<<grid, 128, prep::SMEM, a.stream>>>(                            \
-        (const TIN *)a.q, (const TIN *)a.k, (const TIN *)a.v, a.conv_w, (const TIN *)a.a_logit,  \
-        (const TIN *)a.b_logit, a.A, a.b_alpha, a.cu_seqlens, a.n_seq, a.n_tok, a.H, w.Qt, w.Kt, \
+#define GDN_PREP(DV_)                                                                             \
+    e = cudaFuncSetAttribute(chunk_prep_kernel<DV_>, cudaFuncAttributeMaxDynamicSharedMemorySize,  \
+                             prep::SMEM);                                                          \
+    if (e != cudaSuccess) return e;                                                                 \
+    chunk_prep_kernel<DV_><<<grid, 128, prep::SMEM, a.stream>>>(                                    \
+        (const bf16 *)a.q, (const bf16 *)a.k, (const bf16 *)a.v, a.conv_w, (const bf16 *)a.a_logit, \
+        (const bf16 *)a.b_logit, a.A, a.b_alpha, a.cu_seqlens, a.n_seq, a.n_tok, a.H, w.Qt, w.Kt,   \
         w.Wn, w.Up, w.Aqk, w.decay)
-    if (a.dv == 128) {
-        if (a.in_bf16) { GDN_PREP(128, bf16); } else { GDN_PREP(128, float); }
-    } else {
-        if (a.in_bf16) { GDN_PREP(64, bf16); } else { GDN_PREP(64, float); }
-    }
+    if (!a.in_bf16) return cudaErrorInvalidValue;   // the tensor-core path takes bf16 inputs
+    if (a.dv == 128) { GDN_PREP(128); } else { GDN_PREP(64); }
 #undef GDN_PREP
     return cudaGetLastError();
 }
