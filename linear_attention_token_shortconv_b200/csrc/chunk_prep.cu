@@ -25,7 +25,7 @@
 // Per chunk: prelude in registers -> fp16 hi/lo tiles in smem; the split
 // [Q;K]K^T on tcgen05 (M=128, N=64) -> TMEM, with Qt and Kt written out while
 // it runs; Aqk and L from TMEM; T by blocked forward substitution in fp32 over
-// all 128 threads; [T diag(beta e^G); T diag(beta)] times K and V on tcgen05 ->
+// all 256 threads; [T diag(beta e^G); T diag(beta)] times K and V on tcgen05 ->
 // TMEM; results to global memory in fp16.
 #include <cuda_fp16.h>
 
@@ -122,7 +122,8 @@ __device__ __forceinline__ float blk16(const float *A, int ar, int ac, const flo
 // T = (I + L)^-1 for a strictly lower triangular 64 x 64 L, by 16 x 16 blocks:
 // diagonal blocks by forward substitution, then block row-diagonals
 //   T_{b+d,b} = -D_{b+d} sum_{j=b}^{b+d-1} L_{b+d,j} T_{j,b},  D_b = (I + L_bb)^-1.
-// 128 threads; X is a [3][16][16] scratch.  Only the block-lower part of T is written.
+// NT threads; X is a [3][16][16] scratch.  Only the block-lower part of T is written.
+template <int NT>
 __device__ __forceinline__ void solve_unit_lower(const float *L, float *T, float *X, int tid) {
     if (tid < 64) {   // diagonal blocks: thread (b, c) owns column c of D_b
         const int b = tid >> 4, cc = tid & 15, o = 16 * b;
@@ -139,12 +140,12 @@ __device__ __forceinline__ void solve_unit_lower(const float *L, float *T, float
     }
     __syncthreads();
     // d = 1: X_b = L_{b+1,b} D_b, then T_{b+1,b} = -D_{b+1} X_b   (b = 0, 1, 2)
-    for (int e = tid; e < 3 * 256; e += 128) {
+    for (int e = tid; e < 3 * 256; e += NT) {
         const int b = e >> 8, r = (e >> 4) & 15, cc = e & 15;
         X[e] = blk16(L, 16 * (b + 1), 16 * b, T, 16 * b, 16 * b, r, cc, 0.f);
     }
     __syncthreads();
-    for (int e = tid; e < 3 * 256; e += 128) {
+    for (int e = tid; e < 3 * 256; e += NT) {
         const int b = e >> 8, r = (e >> 4) & 15, cc = e & 15;
         float acc = 0.f;
 #pragma unroll
@@ -153,13 +154,13 @@ __device__ __forceinline__ void solve_unit_lower(const float *L, float *T, float
     }
     __syncthreads();
     // d = 2: X_b = L_{b+2,b} D_b + L_{b+2,b+1} T_{b+1,b}, then T_{b+2,b} = -D_{b+2} X_b   (b = 0, 1)
-    for (int e = tid; e < 2 * 256; e += 128) {
+    for (int e = tid; e < 2 * 256; e += NT) {
         const int b = e >> 8, r = (e >> 4) & 15, cc = e & 15;
         float acc = blk16(L, 16 * (b + 2), 16 * b, T, 16 * b, 16 * b, r, cc, 0.f);
         X[e] = blk16(L, 16 * (b + 2), 16 * (b + 1), T, 16 * (b + 1), 16 * b, r, cc, acc);
     }
     __syncthreads();
-    for (int e = tid; e < 2 * 256; e += 128) {
+    for (int e = tid; e < 2 * 256; e += NT) {
         const int b = e >> 8, r = (e >> 4) & 15, cc = e & 15;
         float acc = 0.f;
 #pragma unroll
@@ -168,14 +169,14 @@ __device__ __forceinline__ void solve_unit_lower(const float *L, float *T, float
     }
     __syncthreads();
     // d = 3: X = L_30 D_0 + L_31 T_10 + L_32 T_20, then T_30 = -D_3 X
-    for (int e = tid; e < 256; e += 128) {
+    for (int e = tid; e < 256; e += NT) {
         const int r = e >> 4, cc = e & 15;
         float acc = blk16(L, 48, 0, T, 0, 0, r, cc, 0.f);
         acc = blk16(L, 48, 16, T, 16, 0, r, cc, acc);
         X[e] = blk16(L, 48, 32, T, 32, 0, r, cc, acc);
     }
     __syncthreads();
-    for (int e = tid; e < 256; e += 128) {
+    for (int e = tid; e < 256; e += NT) {
         const int r = e >> 4, cc = e & 15;
         float acc = 0.f;
 #pragma unroll
@@ -186,7 +187,7 @@ __device__ __forceinline__ void solve_unit_lower(const float *L, float *T, float
 }
 
 template <int DV>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(256, 2)
 chunk_prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const bf16 *__restrict__ v,
                   const float *__restrict__ conv_w, const bf16 *__restrict__ a_logit,
                   const bf16 *__restrict__ b_logit, const float *__restrict__ A,
@@ -219,17 +220,18 @@ chunk_prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const 
     if (tid == 0) { umma::mbar_init(bar, 1); umma::fence_mbar_init(); }
     __syncthreads();
     const uint32_t tbase = *tslot;
-    const uint32_t trow = tbase + ((uint32_t)(warp * 32) << 16);
+    const uint32_t trow = tbase + ((uint32_t)(32 * (warp & 3)) << 16);
     const float eA = expf(__ldg(A + h)), ba = __ldg(b_alpha + h);
 
-    // this thread's prelude channels: q/k octet (tid % 32, tokens 16 * (tid / 32) ..)
-    // and v octet (tid % (DV / 8), tokens (DV / 8) * 8 / ... )
+    // this thread's prelude channels: q/k octet tid % 32 for tokens 8 * warp .. + 8,
+    // and v octet tid % (DV / 8) for a 64 / VPARTS-token part of the chunk
+    constexpr int NT = 256;
     const int qk_oct = tid & 31;                  // 0..15 q, 16..31 k
     const bool is_k = qk_oct >= 16;
     const int qk_col = h * DK + (qk_oct & 15) * 8;
     const int qk_chan = (is_k ? H * DK : 0) + qk_col;
     constexpr int VO = DV / 8;                    // v octets
-    constexpr int VPARTS = 128 / VO;              // token parts for v
+    constexpr int VPARTS = NT / VO;               // token parts for v
     const int v_oct = tid % VO, v_part = tid / VO;
     const int v_col = h * DV + v_oct * 8;
     const int v_chan = 2 * H * DK + v_col;
@@ -247,7 +249,7 @@ chunk_prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const 
                 const float4 a4 = __ldg(reinterpret_cast<const float4 *>(conv_w) + qk_chan + e);
                 wqk[e][0] = a4.x; wqk[e][1] = a4.y; wqk[e][2] = a4.z; wqk[e][3] = a4.w;
             }
-            conv_rows<16>(is_k ? k : q, (size_t)H * DK, qk_col, wqk, t0, s_begin, 16 * warp, len,
+            conv_rows<8>(is_k ? k : q, (size_t)H * DK, qk_col, wqk, t0, s_begin, 8 * warp, len,
                           [&](int i, float (&y)[8]) {
                               float ss = 0.f;
 #pragma unroll
@@ -315,7 +317,7 @@ chunk_prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const 
         // while the MMA runs: Qt = e^{G_i} q_i, Kt = e^{G_C - G_i} k_i (fp16) and e^{G_C}
         {
             const float GC = sG[C - 1];
-            for (int idx = tid; idx < len * (DK / 8); idx += 128) {
+            for (int idx = tid; idx < len * (DK / 8); idx += NT) {
                 const int i = idx / (DK / 8), ch = idx % (DK / 8);
                 const float sq = __expf(sG[i]), sk = __expf(GC - sG[i]);
                 const uint4 qv = *reinterpret_cast<const uint4 *>(sHI + (ch / 8) * 16384 + umma::sw128_offset(i, ch % 8));
@@ -342,23 +344,23 @@ chunk_prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const 
         if (!ok) break;
 
         // ---- 3. rows 0..63: Aqk (masked, decayed q.k) -> global; rows 64..127: L -> smem
+        //         warp w reads lane quadrant w % 4, columns [32 (w / 4), + 32)
         {
-            float v0[32], v1[32];
-            umma::tmem_ld32(trow + 0, v0);
-            umma::tmem_ld32(trow + 32, v1);
-            const int i = (warp * 32 + lane) & 63;
+            float v[32];
+            const int j0 = 32 * (warp >> 2);
+            umma::tmem_ld32(trow + j0, v);
+            const int i = (32 * (warp & 3) + lane) & 63;
             const float Gi = sG[i];
-            if (warp < 2) {
+            if ((warp & 3) < 2) {
                 if (i < len) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(Aqk + ((size_t)(t0 + i) * H + h) * C);
+                    uint4 *dst = reinterpret_cast<uint4 *>(Aqk + ((size_t)(t0 + i) * H + h) * C + j0);
 #pragma unroll
-                    for (int q8 = 0; q8 < 8; ++q8) {
+                    for (int q8 = 0; q8 < 4; ++q8) {
                         float x[8];
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
-                            const int j = q8 * 8 + e;
-                            const float raw = (j < 32) ? v0[j & 31] : v1[j & 31];
-                            x[e] = (j <= i) ? raw * __expf(Gi - sG[j]) : 0.f;
+                            const int j = j0 + q8 * 8 + e;
+                            x[e] = (j <= i) ? v[q8 * 8 + e] * __expf(Gi - sG[j]) : 0.f;
                         }
                         dst[q8] = make_uint4(umma::pack_half2(x[0], x[1]), umma::pack_half2(x[2], x[3]),
                                              umma::pack_half2(x[4], x[5]), umma::pack_half2(x[6], x[7]));
@@ -366,15 +368,14 @@ chunk_prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const 
                 }
             } else {
                 const float bi = sBeta[i];
-                float4 *dst = reinterpret_cast<float4 *>(sL + i * C);
+                float4 *dst = reinterpret_cast<float4 *>(sL + i * C + j0);
 #pragma unroll
-                for (int q4 = 0; q4 < 16; ++q4) {
+                for (int q4 = 0; q4 < 8; ++q4) {
                     float x[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int j = q4 * 4 + e;
-                        const float raw = (j < 32) ? v0[j & 31] : v1[j & 31];
-                        x[e] = (j < i) ? bi * raw * __expf(Gi - sG[j]) : 0.f;
+                        const int j = j0 + q4 * 4 + e;
+                        x[e] = (j < i) ? bi * v[q4 * 4 + e] * __expf(Gi - sG[j]) : 0.f;
                     }
                     dst[q4] = make_float4(x[0], x[1], x[2], x[3]);
                 }
@@ -385,8 +386,8 @@ chunk_prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const 
 
         // ---- 4. T = (I + L)^-1 (fp32, blocked); then T' = T diag(beta e^G) in rows
         //         0..63 and T'' = T diag(beta) in rows 64..127 of an fp16 K-major tile
-        solve_unit_lower(sL, sTf, sX, tid);
-        for (int idx = tid; idx < C * 8; idx += 128) {
+        solve_unit_lower<NT>(sL, sTf, sX, tid);
+        for (int idx = tid; idx < C * 8; idx += NT) {
             const int i = idx >> 3, ch = idx & 7;
             const float4 *tr = reinterpret_cast<const float4 *>(sTf + i * C + ch * 8);
             const float4 t0v = tr[0], t1v = tr[1];
@@ -429,13 +430,15 @@ chunk_prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const 
         if (!ok) break;
 
         // ---- 6. rows 0..63 of the W-part -> -W; rows 64..127 of the U'-part -> U'
-        //         (TMEM loads are warp-collective: every lane loads, valid rows store)
+        //         (warp w: lane quadrant w % 4, column half w / 4; TMEM loads are
+        //         warp-collective: every lane loads, valid rows store)
         {
-            const int i = (warp * 32 + lane) & 63;
-            if (warp < 2) {
+            const int i = (32 * (warp & 3) + lane) & 63;
+            const int half = warp >> 2;
+            if ((warp & 3) < 2) {
                 __half *dst = Wn + ((size_t)(t0 + i) * H + h) * DK;
 #pragma unroll
-                for (int c0 = 0; c0 < DK; c0 += 32) {
+                for (int c0 = half * (DK / 2); c0 < (half + 1) * (DK / 2); c0 += 32) {
                     float vv[32];
                     umma::tmem_ld32(trow + c0, vv);
                     if (i < len) {
@@ -449,7 +452,7 @@ chunk_prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const 
             } else {
                 __half *dst = Up + ((size_t)(t0 + i) * H + h) * DV;
 #pragma unroll
-                for (int c0 = 0; c0 < DV; c0 += 32) {
+                for (int c0 = half * (DV / 2); c0 < (half + 1) * (DV / 2); c0 += 32) {
                     float vv[32];
                     umma::tmem_ld32(trow + DK + c0, vv);
                     if (i < len) {
@@ -483,7 +486,7 @@ cudaError_t launch_chunk_prep(const PrefillArgs &a, const TcWorkspace &w) {
     e = cudaFuncSetAttribute(chunk_prep_kernel<DV_>, cudaFuncAttributeMaxDynamicSharedMemorySize,  \
                              prep::SMEM);                                                          \
     if (e != cudaSuccess) return e;                                                                 \
-    chunk_prep_kernel<DV_><<<grid, 128, prep::SMEM, a.stream>>>(                                    \
+    chunk_prep_kernel<DV_><<<grid, 256, prep::SMEM, a.stream>>>(                                    \
         (const bf16 *)a.q, (const bf16 *)a.k, (const bf16 *)a.v, a.conv_w, (const bf16 *)a.a_logit, \
         (const bf16 *)a.b_logit, a.A, a.b_alpha, a.cu_seqlens, a.n_seq, a.n_tok, a.H, w.Qt, w.Kt,   \
         w.Wn, w.Up, w.Aqk, w.decay)
