@@ -11,6 +11,8 @@
 //     dS        = Kt^T U                                  (tcgen05)
 //     S         = e^{G_C} S + dS                          (fp32, registers)
 //     out       = sigmoid(z) * Y / sqrt(mean(Y^2) + eps) * (1 + w)
+// (sigmoid(z) = (1 + tanh(z/2)) / 2 with the hardware tanh: absolute error
+// about 2^-12 on the gate, applied linearly to the normalised output)
 //
 // One CTA of 4 * dv threads per (sequence, head).  Warp w reads tensor-memory
 // lane quadrant w % 4 and owns the 32-column group w / 4: each thread holds 32
@@ -49,8 +51,15 @@ constexpr uint32_t kMaxPolls = 1u << 24;
 }  // namespace chain
 
 struct ChainMaps {
-    CUtensorMap wn, qt, kt, aqk, up, z;
+    CUtensorMap wn, qt, kt, aqk, up, z, out;   // `out` only for bf16 output
 };
+
+// tanh on the special-function unit (absolute error about 2^-11)
+__device__ __forceinline__ float tanh_approx(float x) {
+    float r;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
 
 __device__ __forceinline__ uint4 pack8(const float *x) {
     return make_uint4(umma::pack_half2(x[0], x[1]), umma::pack_half2(x[2], x[3]),
@@ -112,7 +121,7 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const float *__restri
     uint8_t *sBP = sm + OFF_BP, *sBU = sm + OFF_BU;
     uint64_t *full_a = reinterpret_cast<uint64_t *>(sm + OFF_MISC);   // [2]
     uint64_t *full_z = full_a + 2;                                     // [2]
-    uint64_t *bar_p = full_a + 4, *bar_ys = full_a + 5;
+    uint64_t *bar_p = full_a + 4, *bar_s = full_a + 5, *bar_y = full_a + 6;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + OFF_MISC + 64);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OFF_MISC + 68);
     float *w1 = reinterpret_cast<float *>(sm + OFF_MISC + 128);      // 1 + norm_w  [DV]
@@ -131,7 +140,7 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const float *__restri
 
     if (warp == 0) umma::tmem_alloc(tslot, TMEM_COLS);
     if (tid == 0) {
-        for (int i = 0; i < 6; ++i) umma::mbar_init(full_a + i, 1);
+        for (int i = 0; i < 7; ++i) umma::mbar_init(full_a + i, 1);
         *abort_flag = 0;
         umma::fence_mbar_init();
     }
@@ -160,6 +169,11 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const float *__restri
     const uint32_t tbase = *tslot;
     const uint32_t tD = tbase + 2 * DV;
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
+    // output gain of this thread's 32 columns, halved: sigmoid(z) (1 + w) y =
+    // (1 + tanh(z / 2)) * ((1 + w) / 2) * y
+    float w1h[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) w1h[j] = 0.5f * w1[col0 + j];
 
     auto stage = [&](int b) { return sm + b * STAGE; };
     auto issue_a = [&](int cc, int b) {
@@ -182,12 +196,32 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const float *__restri
         for (int x = 0; x < DV; x += 64)
             umma::tma_load_3d(stage(b) + ST_ZS + x * 128, &maps.z, x, h, s_begin + cc * C, full_z + b);
     };
-    if (tid == 0 && n_chunks > 0) {
-        issue_a(0, 0);
-        issue_z(0, 0);
+    // Tile producers: tid kTmaA (a U-warp lane, idle while the first MMA runs)
+    // refills, at the start of chunk c, the stage of chunk c - 1 (drained before
+    // the last block barrier) with the operand tiles of chunk c + 1; tid kTma (an
+    // output-stage lane) issues the z tiles one chunk ahead and the TMA stores of
+    // finished bf16 output tiles.
+    constexpr int kTmaA = 32, kTma = 64;
+    constexpr bool kTmaOut = sizeof(Tout) == 2;
+    if (tid == kTma) {
+        umma::prefetch_tensormap(&maps.wn);
+        umma::prefetch_tensormap(&maps.qt);
+        umma::prefetch_tensormap(&maps.kt);
+        umma::prefetch_tensormap(&maps.aqk);
+        umma::prefetch_tensormap(&maps.up);
+        umma::prefetch_tensormap(&maps.z);
+        if (kTmaOut) umma::prefetch_tensormap(&maps.out);
+        for (int cc = 0; cc < 2 && cc < n_chunks; ++cc) issue_a(cc, cc);
+        if (n_chunks > 0) issue_z(0, 0);
     }
     // byte offset of the 8-column chunk `col` of row i in a 64-column-block swizzled tile
     auto tile_off = [](int i, int col) { return (col / 64) * 8192 + umma::sw128_offset(i, (col % 64) / 8); };
+    // descriptor bases (start-address field advanced by offset >> 4 per K step)
+    const uint64_t dBP = umma::sw128_desc(umma::smem_u32(sBP), 16384, 1024);
+    const uint64_t dBU = umma::sw128_desc(umma::smem_u32(sBU), 8192, 1024);
+    const uint32_t id_p = umma::idesc_f16(128, DV, false, true);
+    const uint32_t id_y = umma::idesc_f16(128, DV, false, true);
+    const uint32_t id_s = umma::idesc_f16(128, DV, true, true);
 
     for (int c = 0; c < n_chunks; ++c) {
         const int b = c & 1;
@@ -197,35 +231,36 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const float *__restri
         uint8_t *st = stage(b);
         const uint32_t tP = tbase + b * DV;
         const float dec = __ldg(decay + (size_t)t0 * H + h);
-        if (tid == 0 && c + 1 < n_chunks) {
-            umma::fence_proxy_async_smem();
-            issue_a(c + 1, b ^ 1);
-        }
+        if (tid == kTmaA && c >= 1 && c + 1 < n_chunks) issue_a(c + 1, b ^ 1);
         if (q < 2) {
             // ---- P = [-W; Qt] S  (M=128, N=DV, K=dk)
             if (tid == 0) {
                 chain_wait(full_a + b, ph_stage, abort_flag);
                 umma::tc_fence_after();
-                const uint32_t a0 = umma::smem_u32(st + ST_AP), b0 = umma::smem_u32(sBP);
-                const uint32_t idesc = umma::idesc_f16(128, DV, false, true);
+                const uint64_t dA = umma::sw128_desc(umma::smem_u32(st + ST_AP), 16, 1024);
 #pragma unroll
                 for (int s = 0; s < DK / 16; ++s)
-                    umma::mma_f16(tP, umma::sw128_desc(a0 + (s / 4) * 16384 + (s % 4) * 32, 16, 1024),
-                                  umma::sw128_desc(b0 + s * 2048, 16384, 1024), idesc, s > 0);
+                    umma::mma_f16(tP, dA + (uint64_t)(((s / 4) * 16384 + (s % 4) * 32) >> 4),
+                                  dBP + (uint64_t)((s * 2048) >> 4), id_p, s > 0);
                 umma::mma_commit(bar_p);
             }
+            // U' of this thread's row and columns, read while the MMA runs
+            const int i = srow;
             chain_wait(full_a + b, ph_stage, abort_flag);
+            uint4 upk[4];
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+                upk[m] = *reinterpret_cast<const uint4 *>(st + ST_US + tile_off(i, col0 + 8 * m));
             chain_wait(bar_p, ph, abort_flag);
             umma::tc_fence_after();
             // ---- U = U' + P[0:64] (zero past the sequence end) -> fp16 MN-major B operand
-            const int i = srow;
             float v[32];
             umma::tmem_ld32(tP + lane_off + col0, v);
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
                 const int col = col0 + 8 * m;
                 float up[8], u[8];
-                unpack8h(*reinterpret_cast<const uint4 *>(st + ST_US + tile_off(i, col)), up);
+                unpack8h(upk[m], up);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) u[e] = (i < len) ? v[8 * m + e] + up[e] : 0.f;
                 umma::st_chunk(sBU + (col / 64) * 8192, i, (col % 64) / 8, pack8(u));
@@ -233,23 +268,22 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const float *__restri
             umma::fence_proxy_async_smem();
             umma::tc_fence_before();
             umma::named_bar_sync(1, HALF);
-            // ---- P[64:128] += [*; Aqk] U  (rows 0..63 of A are don't-care);  dS = Kt^T U
+            // ---- dS = Kt^T U (on the state path, committed first);  P[64:128] += [*; Aqk] U
             if (tid == 0) {
                 umma::tc_fence_after();
-                const uint32_t aY = umma::smem_u32(st + ST_AS + 8192), aS = umma::smem_u32(st + ST_AS);
-                const uint32_t bU = umma::smem_u32(sBU);
-                const uint32_t idy = umma::idesc_f16(128, DV, false, true);
-                const uint32_t ids = umma::idesc_f16(128, DV, true, true);
+                const uint64_t dS = umma::sw128_desc(umma::smem_u32(st + ST_AS), 8192, 1024);
+                const uint64_t dY = umma::sw128_desc(umma::smem_u32(st + ST_AS + 8192), 16, 1024);
 #pragma unroll
-                for (int s = 0; s < C / 16; ++s) {
-                    const uint64_t bd = umma::sw128_desc(bU + s * 2048, 8192, 1024);
-                    umma::mma_f16(tP, umma::sw128_desc(aY + s * 32, 16, 1024), bd, idy, 1u);
-                    umma::mma_f16(tD, umma::sw128_desc(aS + s * 2048, 8192, 1024), bd, ids, s > 0);
-                }
-                umma::mma_commit(bar_ys);
+                for (int s = 0; s < C / 16; ++s)
+                    umma::mma_f16(tD, dS + (uint64_t)((s * 2048) >> 4), dBU + (uint64_t)((s * 2048) >> 4), id_s, s > 0);
+                umma::mma_commit(bar_s);
+#pragma unroll
+                for (int s = 0; s < C / 16; ++s)
+                    umma::mma_f16(tP, dY + (uint64_t)((s * 32) >> 4), dBU + (uint64_t)((s * 2048) >> 4), id_y, 1u);
+                umma::mma_commit(bar_y);
             }
         }
-        chain_wait(bar_ys, ph, abort_flag);
+        chain_wait(bar_s, ph, abort_flag);
         umma::tc_fence_after();
         // ---- S = e^{G_C} S + dS; fp16 copy for the next chunk
         {
@@ -264,47 +298,70 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const float *__restri
             }
         }
         umma::fence_proxy_async_smem();
+        if (q >= 2) {
+            // Y of this chunk is complete (waited before the block barrier, so this
+            // barrier's phases never run ahead of the waits); stage b is drained.
+            chain_wait(bar_y, ph, abort_flag);
+        }
         umma::tc_fence_before();
         __syncthreads();
         umma::tc_fence_after();
-        if (tid == 0 && c + 1 < n_chunks) {
-            umma::fence_proxy_async_smem();
-            issue_z(c + 1, b ^ 1);
-        }
         // ---- output stage of this chunk on P[64:128] (quadrants 2, 3): overlaps chunk c + 1
         if (q >= 2) {
             const int i = srow - 64;
             float v[32];
             umma::tmem_ld32(tP + lane_off + col0, v);
-            float ss = 0.f;
+            float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int j = 0; j < 32; ++j) ss = fmaf(v[j], v[j], ss);
-            red[cg * 64 + i] = ss;
+            for (int j = 0; j < 32; ++j) s4[j & 3] = fmaf(v[j], v[j], s4[j & 3]);
+            red[cg * 64 + i] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
             chain_wait(full_z + b, ph_stage, abort_flag);
             umma::named_bar_sync(2, HALF);
             float tot = 0.f;
 #pragma unroll
             for (int g2 = 0; g2 < NCG; ++g2) tot += red[g2 * 64 + i];
             const float rr = rsqrtf(tot / DV + kNormEps);
-            if (i < len) {
-                const size_t g = ((size_t)(t0 + i) * H + h) * DV;
+            float rw[32];
 #pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    const int col = col0 + 8 * m;
-                    const uint4 zz = *reinterpret_cast<const uint4 *>(st + ST_ZS + tile_off(i, col));
-                    const uint32_t zw[4] = {zz.x, zz.y, zz.z, zz.w};
-                    float o[8];
+            for (int j = 0; j < 32; ++j) rw[j] = rr * w1h[j];
+            // full chunks of a bf16 output leave through one TMA store of the z tile,
+            // overwritten in place; ragged chunks store their valid rows directly
+            const bool tile_store = kTmaOut && len == C;
+            const size_t g = ((size_t)(t0 + i) * H + h) * DV;
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float z0 = bf16lo(zw[e]), z1 = bf16hi(zw[e]);
-                        o[2 * e] = __fdividef(v[8 * m + 2 * e] * rr * w1[col + 2 * e], 1.0f + __expf(-z0));
-                        o[2 * e + 1] = __fdividef(v[8 * m + 2 * e + 1] * rr * w1[col + 2 * e + 1], 1.0f + __expf(-z1));
-                    }
-                    store8_out<Tout>(out + g + col, o);
+            for (int m = 0; m < 4; ++m) {
+                const int col = col0 + 8 * m;
+                uint4 *zp = reinterpret_cast<uint4 *>(st + ST_ZS + tile_off(i, col));
+                const uint4 zz = *zp;
+                const uint32_t zw[4] = {zz.x, zz.y, zz.z, zz.w};
+                float o[8];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float t0z = tanh_approx(0.5f * bf16lo(zw[e])), t1z = tanh_approx(0.5f * bf16hi(zw[e]));
+                    const float a0 = v[8 * m + 2 * e] * rw[8 * m + 2 * e];
+                    const float a1 = v[8 * m + 2 * e + 1] * rw[8 * m + 2 * e + 1];
+                    o[2 * e] = fmaf(a0, t0z, a0);
+                    o[2 * e + 1] = fmaf(a1, t1z, a1);
                 }
+                if (tile_store) store8_out<bf16>(reinterpret_cast<bf16 *>(zp), o);
+                else if (i < len) store8_out<Tout>(out + g + col, o);
+            }
+            if (tile_store) umma::fence_proxy_async_smem();
+            umma::named_bar_sync(2, HALF);
+            if (tid == kTma) {
+                if (tile_store) {
+#pragma unroll
+                    for (int x = 0; x < DV; x += 64)
+                        umma::tma_store_3d(&maps.out, x, h, t0, st + ST_ZS + x * 128);
+                    umma::bulk_commit();
+                }
+                // the z tile of stage b ^ 1 is free once the store of chunk c - 1 has read it
+                umma::bulk_wait_read<1>();
+                if (c + 1 < n_chunks) issue_z(c + 1, b ^ 1);
             }
         }
     }
+    if (tid == kTma) umma::bulk_wait_all();
     if (S_final && !*abort_flag) {
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
@@ -338,6 +395,8 @@ cudaError_t launch_chunk_chain(const PrefillArgs &a, const TcWorkspace &w) {
         if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.aqk), w.Aqk, false, 64, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
         if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.up), w.Up, false, a.dv, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
         if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.z), a.z, true, a.dv, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
+        if (a.out_bf16 &&
+            (e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.out), a.out, true, a.dv, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
     }
     dim3 grid(a.H, a.n_seq);
     cudaError_t e;
