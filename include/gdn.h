@@ -101,7 +101,10 @@ typedef struct {
  *              may be NULL when not wanted)
  *
  * Each sequence starts with an empty conv history.  `out` must not alias any
- * input.  When total_tokens is 0 the token tensors (q, k, v, z, a_logit,
+ * input.  On the tensor-core path (bf16 inputs, dk = 128) long inputs run in
+ * chunk segments whose kernels overlap on `stream` and on a library-owned
+ * second stream of the same device, forked from and joined back into `stream`
+ * with events, so work queued on `stream` afterwards sees the results.  When total_tokens is 0 the token tensors (q, k, v, z, a_logit,
  * b_logit, out) may be NULL and the call only writes S_final = S0 (or zeros).  The call takes a stream-ordered workspace of
  * gdn_prefill_workspace_size() bytes from a private CUDA memory pool of the
  * current device and returns it to the pool on the same stream.
@@ -173,11 +176,12 @@ GDN_API gdn_status_t gdn_prefill_noalloc(const gdn_dims_t *dims, const void *q, 
 
 /*
  * gdn_set_timing_events -- optional profiling hook (host call, not thread-safe).
- * When both handles are non-NULL (cudaEvent_t values), each following
- * gdn_prefill / gdn_decode_step records `begin` on its stream immediately before
- * its dominant kernel (the state recurrence) and `end` immediately after it,
- * until the hook is cleared with (NULL, NULL).  Recording adds no work to the
- * kernels; it lets a caller time the dominant kernel with CUDA events.
+ * When both handles are non-NULL (cudaEvent_t values), each following call
+ * records `begin` and `end` on its stream: gdn_prefill around all of its GPU
+ * work on the tensor-core path (whose kernels overlap on two streams) and around
+ * the state recurrence on the fp32 path; gdn_decode_step around its kernel.
+ * The hook stays until cleared with (NULL, NULL).  Recording adds no work to
+ * the kernels; it lets a caller time the library's GPU work with CUDA events.
  */
 GDN_API gdn_status_t gdn_set_timing_events(void *begin, void *end);
 

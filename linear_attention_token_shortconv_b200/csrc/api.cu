@@ -3,8 +3,12 @@
 // argument has been checked.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <mutex>
+#include <vector>
+
+using std::max;
 
 #include "../../include/gdn.h"
 #include "gdn_internal.h"
@@ -37,13 +41,30 @@ size_t round_up(size_t x) { return (x + 255) & ~(size_t)255; }
 // else (the fp32 workload, dk = 64) runs the fp32 token-by-token recurrence.
 bool use_tensor_cores(const gdn_dims_t *d) { return d->in_dtype == GDN_BF16 && d->dk == 128; }
 
+// Chunk segments of the tensor-core path: the prep kernel of segment s + 1 runs
+// on the caller's stream while the chain kernel of segment s runs on a second,
+// higher-priority stream; segments are ordered by events, and the state passes
+// from one chain launch to the next through a state buffer.
+struct Segments {
+    int seg, n;
+};
+Segments segments(const gdn_dims_t *d) {
+    const int max_chunks = (d->total_tokens + 63) / 64;
+    Segments g;
+    g.seg = max(8, (max_chunks + 23) / 24);
+    g.n = max(1, (max_chunks + g.seg - 1) / g.seg);
+    return g;
+}
+
 // Workspace: tensor-core path: Qt, Kt, -W [dk], U' [dv], Aqk [64] in fp16 and
-// e^{G_C} in fp32 per token-head; fp32 path: q_hat, k_hat, v_hat in fp32.
+// e^{G_C} in fp32 per token-head, plus an fp32 state buffer [N_seq, H, dk, dv]
+// when the call runs in several segments; fp32 path: q_hat, k_hat, v_hat in fp32.
 size_t workspace_bytes(const gdn_dims_t *d) {
     const size_t nt = (size_t)d->total_tokens * d->H;
     if (use_tensor_cores(d))
         return 3 * round_up(nt * d->dk * 2) + round_up(nt * d->dv * 2) + round_up(nt * 64 * 2) +
-               round_up(nt * 4);
+               round_up(nt * 4) +
+               (segments(d).n > 1 ? round_up((size_t)d->num_seqs * d->H * d->dk * d->dv * 4) : 0);
     return 2 * round_up(nt * d->dk * sizeof(float)) + round_up(nt * d->dv * sizeof(float));
 }
 
@@ -72,6 +93,34 @@ cudaError_t get_pool(cudaMemPool_t *pool) {
         g_pools[dev] = p;
     }
     *pool = g_pools[dev];
+    return cudaSuccess;
+}
+
+// Per-device side stream (highest priority) and event pool for the segments.
+struct SideStream {
+    cudaStream_t stream = nullptr;
+    std::vector<cudaEvent_t> events;
+};
+std::mutex g_side_mu[64];
+SideStream g_side[64];
+
+// Returns the side stream of the current device with at least n events; the
+// caller holds g_side_mu[dev] while it records and waits on them.
+cudaError_t side_stream(int dev, int n, SideStream **out) {
+    SideStream &ss = g_side[dev];
+    cudaError_t e;
+    if (!ss.stream) {
+        int lo = 0, hi = 0;
+        if ((e = cudaDeviceGetStreamPriorityRange(&lo, &hi)) != cudaSuccess) return e;
+        if ((e = cudaStreamCreateWithPriority(&ss.stream, cudaStreamNonBlocking, hi)) != cudaSuccess)
+            return e;
+    }
+    while ((int)ss.events.size() < n) {
+        cudaEvent_t ev;
+        if ((e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming)) != cudaSuccess) return e;
+        ss.events.push_back(ev);
+    }
+    *out = &ss;
     return cudaSuccess;
 }
 
@@ -182,9 +231,38 @@ gdn_status_t gdn_prefill(const gdn_dims_t *dims, const void *q, const void *k, c
         w.Up = reinterpret_cast<__half *>(take(nt * a.dv * 2));
         w.Aqk = reinterpret_cast<__half *>(take(nt * 64 * 2));
         w.decay = reinterpret_cast<float *>(take(nt * 4));
-        e = gdn::launch_chunk_prep(a, w);
-        if (e == cudaSuccess) e = record(g_ev_begin, a.stream);
-        if (e == cudaSuccess) e = gdn::launch_chunk_chain(a, w);
+        const Segments g = segments(dims);
+        e = record(g_ev_begin, a.stream);
+        if (g.n == 1) {
+            if (e == cudaSuccess) e = gdn::launch_chunk_prep(a, w);
+            if (e == cudaSuccess) e = gdn::launch_chunk_chain(a, w);
+        } else {
+            float *state = reinterpret_cast<float *>(take((size_t)a.n_seq * a.H * a.dk * a.dv * 4));
+            int dev = 0;
+            if (e == cudaSuccess) e = cudaGetDevice(&dev);
+            if (e == cudaSuccess && (dev < 0 || dev >= 64)) e = cudaErrorInvalidDevice;
+            if (e == cudaSuccess) {
+                std::lock_guard<std::mutex> lock(g_side_mu[dev]);
+                SideStream *ss = nullptr;
+                e = side_stream(dev, g.n + 2, &ss);
+                // fork: the side stream starts after the caller's prior work
+                if (e == cudaSuccess) e = cudaEventRecord(ss->events[g.n], a.stream);
+                if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->stream, ss->events[g.n], 0);
+                for (int sgi = 0; sgi < g.n && e == cudaSuccess; ++sgi) {
+                    const int c_lo = sgi * g.seg, c_hi = c_lo + g.seg;
+                    e = gdn::launch_chunk_prep(a, w, c_lo, c_hi, a.stream);
+                    if (e == cudaSuccess) e = cudaEventRecord(ss->events[sgi], a.stream);
+                    if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->stream, ss->events[sgi], 0);
+                    const float *sin = sgi == 0 ? a.S0 : state;
+                    float *sout = sgi == g.n - 1 ? a.S_final : state;
+                    if (e == cudaSuccess)
+                        e = gdn::launch_chunk_chain(a, w, c_lo, c_hi, sin, sout, ss->stream);
+                }
+                // join: the caller's stream continues after the last chain launch
+                if (e == cudaSuccess) e = cudaEventRecord(ss->events[g.n + 1], ss->stream);
+                if (e == cudaSuccess) e = cudaStreamWaitEvent(a.stream, ss->events[g.n + 1], 0);
+            }
+        }
         if (e == cudaSuccess) e = record(g_ev_end, a.stream);
     } else {
         float *qn = reinterpret_cast<float *>(ws);

@@ -107,9 +107,9 @@ __device__ __forceinline__ bool chain_wait(uint64_t *bar, uint32_t parity, volat
 template <int DV, typename Tout>
 __global__ void __launch_bounds__(4 * DV, 1)
 chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const float *__restrict__ decay,
-                   const float *__restrict__ norm_w, const float *__restrict__ S0,
-                   const int32_t *__restrict__ cu_seqlens, int n_seq, int n_tok, int H,
-                   Tout *__restrict__ out, float *__restrict__ S_final) {
+                   const float *__restrict__ norm_w, const float *state_in,
+                   const int32_t *__restrict__ cu_seqlens, int n_seq, int n_tok, int H, int c_lo,
+                   int c_hi, Tout *__restrict__ out, float *state_out) {
     using namespace chain;
     // 4 * DV threads: warp w reads TMEM lane quadrant q = w % 4 and owns the
     // 32-column group cg = w / 4 of every row it touches.
@@ -136,7 +136,10 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const float *__restri
     int s_begin, s_end;
     if (cu_seqlens) { s_begin = __ldg(cu_seqlens + n); s_end = __ldg(cu_seqlens + n + 1); }
     else { const int L = n_tok / n_seq; s_begin = n * L; s_end = s_begin + L; }
-    const int n_chunks = (s_end - s_begin + C - 1) / C;
+    // chunks [c_lo, c_end) of this sequence; the state enters from state_in (NULL:
+    // zeros) and leaves to state_out (NULL: dropped); they may be the same buffer
+    const int c_end = min((s_end - s_begin + C - 1) / C, c_hi);
+    const int n_chunks = max(0, c_end - c_lo);   // chunks handled by this launch
 
     if (warp == 0) umma::tmem_alloc(tslot, TMEM_COLS);
     if (tid == 0) {
@@ -152,7 +155,7 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const float *__restri
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
         float x[8];
-        if (S0) load8(S0 + sbase + (size_t)srow * DV + col0 + 8 * m, x);
+        if (state_in) load8(state_in + sbase + (size_t)srow * DV + col0 + 8 * m, x);
         else {
 #pragma unroll
             for (int e = 0; e < 8; ++e) x[e] = 0.f;
@@ -176,8 +179,8 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const float *__restri
     for (int j = 0; j < 32; ++j) w1h[j] = 0.5f * w1[col0 + j];
 
     auto stage = [&](int b) { return sm + b * STAGE; };
-    auto issue_a = [&](int cc, int b) {
-        const int t0 = s_begin + cc * C;
+    auto issue_a = [&](int cc, int b) {   // cc: chunk index within this launch
+        const int t0 = s_begin + (c_lo + cc) * C;
         uint8_t *st = stage(b);
         umma::mbar_expect_tx(full_a + b, BYTES_A);
         umma::tma_load_3d(st + ST_AP, &maps.wn, 0, h, t0, full_a + b);
@@ -194,7 +197,7 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const float *__restri
         umma::mbar_expect_tx(full_z + b, BYTES_Z);
 #pragma unroll
         for (int x = 0; x < DV; x += 64)
-            umma::tma_load_3d(stage(b) + ST_ZS + x * 128, &maps.z, x, h, s_begin + cc * C, full_z + b);
+            umma::tma_load_3d(stage(b) + ST_ZS + x * 128, &maps.z, x, h, s_begin + (c_lo + cc) * C, full_z + b);
     };
     // Tile producers: tid kTmaA (a U-warp lane, idle while the first MMA runs)
     // refills, at the start of chunk c, the stage of chunk c - 1 (drained before
@@ -223,9 +226,9 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const float *__restri
     const uint32_t id_y = umma::idesc_f16(128, DV, false, true);
     const uint32_t id_s = umma::idesc_f16(128, DV, true, true);
 
-    for (int c = 0; c < n_chunks; ++c) {
+    for (int c = 0; c < n_chunks; ++c) {   // c: chunk index within this launch
         const int b = c & 1;
-        const int t0 = s_begin + c * C;
+        const int t0 = s_begin + (c_lo + c) * C;
         const int len = min(C, s_end - t0);
         const uint32_t ph_stage = (uint32_t)(c >> 1) & 1u, ph = (uint32_t)c & 1u;
         uint8_t *st = stage(b);
@@ -362,13 +365,13 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const float *__restri
         }
     }
     if (tid == kTma) umma::bulk_wait_all();
-    if (S_final && !*abort_flag) {
+    if (state_out && !*abort_flag) {
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
             float x[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) x[e] = S[8 * m + e];
-            store8(S_final + sbase + (size_t)srow * DV + col0 + 8 * m, x);
+            store8(state_out + sbase + (size_t)srow * DV + col0 + 8 * m, x);
         }
     }
     umma::tc_fence_before();
@@ -384,7 +387,8 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const float *__restri
     if (warp == 0) umma::tmem_dealloc(tbase, TMEM_COLS);
 }
 
-cudaError_t launch_chunk_chain(const PrefillArgs &a, const TcWorkspace &w) {
+cudaError_t launch_chunk_chain(const PrefillArgs &a, const TcWorkspace &w, int c_lo, int c_hi,
+                               const float *state_in, float *state_out, cudaStream_t stream) {
     ChainMaps m;
     std::memset(&m, 0, sizeof m);
     if (a.n_tok > 0) {
@@ -404,8 +408,9 @@ cudaError_t launch_chunk_chain(const PrefillArgs &a, const TcWorkspace &w) {
     e = cudaFuncSetAttribute(chunk_chain_kernel<DV_, TOUT>,                                       \
                              cudaFuncAttributeMaxDynamicSharedMemorySize, chain::SMEM);            \
     if (e != cudaSuccess) return e;                                                               \
-    chunk_chain_kernel<DV_, TOUT><<<grid, 4 * DV_, chain::SMEM, a.stream>>>(                          \
-        m, w.decay, a.norm_w, a.S0, a.cu_seqlens, a.n_seq, a.n_tok, a.H, (TOUT *)a.out, a.S_final)
+    chunk_chain_kernel<DV_, TOUT><<<grid, 4 * DV_, chain::SMEM, stream>>>(                        \
+        m, w.decay, a.norm_w, state_in, a.cu_seqlens, a.n_seq, a.n_tok, a.H, c_lo, c_hi,        \
+        (TOUT *)a.out, state_out)
     if (a.dv == 128) {
         if (a.out_bf16) { GDN_CHAIN(128, bf16); } else { GDN_CHAIN(128, float); }
     } else {
@@ -413,6 +418,10 @@ cudaError_t launch_chunk_chain(const PrefillArgs &a, const TcWorkspace &w) {
     }
 #undef GDN_CHAIN
     return cudaGetLastError();
+}
+
+cudaError_t launch_chunk_chain(const PrefillArgs &a, const TcWorkspace &w) {
+    return launch_chunk_chain(a, w, 0, (a.n_tok + 63) / 64 + 1, a.S0, a.S_final, a.stream);
 }
 
 }  // namespace gdn

@@ -49,28 +49,13 @@ constexpr int SMEM = OFF_MISC + 4096 + 1024;
 constexpr uint32_t TMEM_COLS = 256;
 }  // namespace prep
 
-__device__ __forceinline__ void split_store(uint8_t *hi_blk, uint8_t *lo_blk, int row, int chunk,
-                                            const float (&x)[8]) {
-    uint32_t h[4], l[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const __half2 hh = __floats2half2_rn(x[2 * e], x[2 * e + 1]);
-        const float2 hf = __half22float2(hh);
-        const __half2 ll = __floats2half2_rn(x[2 * e] - hf.x, x[2 * e + 1] - hf.y);
-        h[e] = *reinterpret_cast<const uint32_t *>(&hh);
-        l[e] = *reinterpret_cast<const uint32_t *>(&ll);
-    }
-    umma::st_chunk(hi_blk, row, chunk, make_uint4(h[0], h[1], h[2], h[3]));
-    umma::st_chunk(lo_blk, row, chunk, make_uint4(l[0], l[1], l[2], l[3]));
-}
-
-// Conv + SiLU of 8 channels for tokens [i0, i0 + N) of a chunk: all N + 3 raw
-// rows (zero before the sequence start and past its end) are loaded first, then
-// the window slides over them; each output row goes to `emit`.
-template <int N, typename Emit>
-__device__ __forceinline__ void conv_rows(const bf16 *src, size_t row_stride, int col,
-                                          const float (&w)[8][4], int t0, int s_begin, int i0,
-                                          int len, Emit emit) {
+// Conv + SiLU of 8 channels (4 pairs) for tokens [i0, i0 + N) of a chunk: all
+// N + 3 raw rows (zero before the sequence start and past its end) are loaded
+// first, then a sliding window of converted rows produces y[N][4] (pairs).
+template <int N>
+__device__ __forceinline__ void conv_silu(const bf16 *src, size_t row_stride, int col,
+                                          const float2 (&w)[4][4], int t0, int s_begin, int i0,
+                                          int len, float2 (&y)[N][4]) {
     uint4 raw[N + 3];
 #pragma unroll
     for (int r = 0; r < N + 3; ++r) {
@@ -80,26 +65,63 @@ __device__ __forceinline__ void conv_rows(const bf16 *src, size_t row_stride, in
         raw[r] = ok ? __ldg(reinterpret_cast<const uint4 *>(src + (size_t)t * row_stride + col))
                     : make_uint4(0, 0, 0, 0);
     }
+    auto cvt = [](uint4 u, float2 (&x)[4]) {
+        x[0] = make_float2(bf16lo(u.x), bf16hi(u.x));
+        x[1] = make_float2(bf16lo(u.y), bf16hi(u.y));
+        x[2] = make_float2(bf16lo(u.z), bf16hi(u.z));
+        x[3] = make_float2(bf16lo(u.w), bf16hi(u.w));
+    };
+    float2 h0[4], h1[4], h2[4];
+    cvt(raw[0], h0);
+    cvt(raw[1], h1);
+    cvt(raw[2], h2);
+    const float2 nl2e = make_float2(-1.4426950408889634f, -1.4426950408889634f);
+    const float2 one = make_float2(1.f, 1.f);
 #pragma unroll
     for (int ii = 0; ii < N; ++ii) {
-        const int i = i0 + ii;
-        float x[4][8];
+        float2 x[4];
+        cvt(raw[ii + 3], x);
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const uint4 u = raw[ii + r];
-            x[r][0] = bf16lo(u.x); x[r][1] = bf16hi(u.x); x[r][2] = bf16lo(u.y); x[r][3] = bf16hi(u.y);
-            x[r][4] = bf16lo(u.z); x[r][5] = bf16hi(u.z); x[r][6] = bf16lo(u.w); x[r][7] = bf16hi(u.w);
+        for (int p = 0; p < 4; ++p) {
+            float2 a = fmul2(w[p][0], h0[p]);
+            a = ffma2(w[p][1], h1[p], a);
+            a = ffma2(w[p][2], h2[p], a);
+            a = ffma2(w[p][3], x[p], a);
+            // silu(a) = a / (1 + 2^(-a log2 e))
+            const float2 e = fmul2(a, nl2e);
+            const float2 d = fadd2(one, make_float2(exp2f(e.x), exp2f(e.y)));
+            y[ii][p] = make_float2(__fdividef(a.x, d.x), __fdividef(a.y, d.y));
+            h0[p] = h1[p]; h1[p] = h2[p]; h2[p] = x[p];
         }
-        float y[8];
+        if (i0 + ii >= len) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            float a = w[e][0] * x[0][e];
-            a = fmaf(w[e][1], x[1][e], a);
-            a = fmaf(w[e][2], x[2][e], a);
-            a = fmaf(w[e][3], x[3][e], a);
-            y[e] = (i < len) ? __fdividef(a, 1.0f + __expf(-a)) : 0.f;
+            for (int p = 0; p < 4; ++p) y[ii][p] = make_float2(0.f, 0.f);
         }
-        emit(i, y);
+    }
+}
+
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+// L2 prefetch of the raw rows conv_silu<N> will read for the chunk at t0.
+template <int N>
+__device__ __forceinline__ void prefetch_rows(const bf16 *src, size_t row_stride, int col, int t0,
+                                             int s_begin, int s_end, int i0) {
+#pragma unroll
+    for (int r = 0; r < N + 3; ++r) {
+        const int t = t0 + i0 + r - 3;
+        if (t >= s_begin && t < s_end) prefetch_l2(src + (size_t)t * row_stride + col);
+    }
+}
+
+__device__ __forceinline__ void load_conv_w(const float *conv_w, int chan, float2 (&w)[4][4]) {
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const float4 a = __ldg(reinterpret_cast<const float4 *>(conv_w) + chan + 2 * p);
+        const float4 b = __ldg(reinterpret_cast<const float4 *>(conv_w) + chan + 2 * p + 1);
+        w[p][0] = make_float2(a.x, b.x); w[p][1] = make_float2(a.y, b.y);
+        w[p][2] = make_float2(a.z, b.z); w[p][3] = make_float2(a.w, b.w);
     }
 }
 
@@ -192,9 +214,9 @@ chunk_prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const 
                   const float *__restrict__ conv_w, const bf16 *__restrict__ a_logit,
                   const bf16 *__restrict__ b_logit, const float *__restrict__ A,
                   const float *__restrict__ b_alpha, const int32_t *__restrict__ cu_seqlens,
-                  int n_seq, int n_tok, int H, __half *__restrict__ Qt, __half *__restrict__ Kt,
-                  __half *__restrict__ Wn, __half *__restrict__ Up, __half *__restrict__ Aqk,
-                  float *__restrict__ decay) {
+                  int n_seq, int n_tok, int H, int c_lo, int c_hi, __half *__restrict__ Qt,
+                  __half *__restrict__ Kt, __half *__restrict__ Wn, __half *__restrict__ Up,
+                  __half *__restrict__ Aqk, float *__restrict__ decay) {
     using namespace prep;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -213,8 +235,9 @@ chunk_prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const 
     int s_begin, s_end;
     if (cu_seqlens) { s_begin = __ldg(cu_seqlens + n); s_end = __ldg(cu_seqlens + n + 1); }
     else { const int L = n_tok / n_seq; s_begin = n * L; s_end = s_begin + L; }
-    const int n_chunks = (s_end - s_begin + C - 1) / C;
-    if ((int)blockIdx.z >= n_chunks) return;   // uniform per block
+    // chunks [c_lo, c_end) of this sequence, strided over blockIdx.z
+    const int c_end = min((s_end - s_begin + C - 1) / C, c_hi);
+    if (c_lo + (int)blockIdx.z >= c_end) return;   // uniform per block
 
     if (warp == 0) umma::tmem_alloc(tslot, TMEM_COLS);
     if (tid == 0) { umma::mbar_init(bar, 1); umma::fence_mbar_init(); }
@@ -237,51 +260,69 @@ chunk_prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const 
     const int v_chan = 2 * H * DK + v_col;
     uint32_t phase = 0;
     bool ok = true;
-    for (int c = blockIdx.z; c < n_chunks && ok; c += gridDim.z) {
+    for (int c = c_lo + blockIdx.z; c < c_end && ok; c += gridDim.z) {
         const int t0 = s_begin + c * C;
         const int len = min(C, s_end - t0);
         // ---- 1. prelude: q, k -> L2-normalised fp32 -> hi/lo fp16 tiles; v -> fp16 tile
         // (conv weights re-read per chunk from L1/L2 to keep them out of the solve's registers)
         {
-            float wqk[8][4];
+            float2 w[4][4];
+            load_conv_w(conv_w, qk_chan, w);
+            float2 y[8][4];
+            conv_silu<8>(is_k ? k : q, (size_t)H * DK, qk_col, w, t0, s_begin, 8 * warp, len, y);
+            // L2 norm over the 16 lanes that hold this head's q (or k): all 8 tokens at once
+            float ss[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float4 a4 = __ldg(reinterpret_cast<const float4 *>(conv_w) + qk_chan + e);
-                wqk[e][0] = a4.x; wqk[e][1] = a4.y; wqk[e][2] = a4.z; wqk[e][3] = a4.w;
+            for (int ii = 0; ii < 8; ++ii) {
+                float2 acc = fmul2(y[ii][0], y[ii][0]);
+#pragma unroll
+                for (int p = 1; p < 4; ++p) acc = ffma2(y[ii][p], y[ii][p], acc);
+                ss[ii] = acc.x + acc.y;
             }
-            conv_rows<8>(is_k ? k : q, (size_t)H * DK, qk_col, wqk, t0, s_begin, 8 * warp, len,
-                          [&](int i, float (&y)[8]) {
-                              float ss = 0.f;
 #pragma unroll
-                              for (int e = 0; e < 8; ++e) ss = fmaf(y[e], y[e], ss);
-                              ss = group_sum<16>(ss);
-                              const float r = rsqrtf(ss + kNormEps);
+            for (int o = 8; o > 0; o >>= 1) {
 #pragma unroll
-                              for (int e = 0; e < 8; ++e) y[e] *= r;
-                              const int row = (is_k ? 64 : 0) + i, oc = qk_oct & 15;
-                              split_store(sHI + (oc / 8) * 16384, sLO + (oc / 8) * 16384, row, oc % 8, y);
-                          });
+                for (int ii = 0; ii < 8; ++ii) ss[ii] += __shfl_xor_sync(0xffffffffu, ss[ii], o);
+            }
+            const int oc = qk_oct & 15;
+            uint8_t *hb = sHI + (oc / 8) * 16384, *lb = sLO + (oc / 8) * 16384;
+#pragma unroll
+            for (int ii = 0; ii < 8; ++ii) {
+                const float r = rsqrtf(ss[ii] + kNormEps);
+                const float2 rr = make_float2(r, r);
+                uint32_t hw[4], lw[4];
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    const float2 x = fmul2(y[ii][p], rr);
+                    const __half2 hh = __floats2half2_rn(x.x, x.y);
+                    const float2 hf = __half22float2(hh);
+                    const __half2 ll = __floats2half2_rn(x.x - hf.x, x.y - hf.y);
+                    hw[p] = *reinterpret_cast<const uint32_t *>(&hh);
+                    lw[p] = *reinterpret_cast<const uint32_t *>(&ll);
+                }
+                const int row = (is_k ? 64 : 0) + 8 * warp + ii;
+                umma::st_chunk(hb, row, oc % 8, make_uint4(hw[0], hw[1], hw[2], hw[3]));
+                umma::st_chunk(lb, row, oc % 8, make_uint4(lw[0], lw[1], lw[2], lw[3]));
+            }
         }
         {
-            float wv[8][4];
+            float2 w[4][4];
+            load_conv_w(conv_w, v_chan, w);
+            constexpr int NV = C / VPARTS;
+            float2 y[NV][4];
+            conv_silu<NV>(v, (size_t)H * DV, v_col, w, t0, s_begin, NV * v_part, len, y);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float4 b4 = __ldg(reinterpret_cast<const float4 *>(conv_w) + v_chan + e);
-                wv[e][0] = b4.x; wv[e][1] = b4.y; wv[e][2] = b4.z; wv[e][3] = b4.w;
-            }
-            conv_rows<C / VPARTS>(v, (size_t)H * DV, v_col, wv, t0, s_begin, (C / VPARTS) * v_part, len,
-                                  [&](int i, float (&y)[8]) {
-                                      umma::st_chunk(sV + (v_oct / 8) * 8192, i, v_oct % 8,
-                                                     make_uint4(umma::pack_half2(y[0], y[1]), umma::pack_half2(y[2], y[3]),
-                                                                umma::pack_half2(y[4], y[5]), umma::pack_half2(y[6], y[7])));
-                                  });
+            for (int ii = 0; ii < NV; ++ii)
+                umma::st_chunk(sV + (v_oct / 8) * 8192, NV * v_part + ii, v_oct % 8,
+                               make_uint4(umma::pack_half2(y[ii][0].x, y[ii][0].y), umma::pack_half2(y[ii][1].x, y[ii][1].y),
+                                          umma::pack_half2(y[ii][2].x, y[ii][2].y), umma::pack_half2(y[ii][3].x, y[ii][3].y)));
         }
         if (tid < C) {
             float g = 0.f, be = 0.f;
             if (tid < len) {
                 const size_t gi = (size_t)(t0 + tid) * H + h;
-                g = -eA * softplus_acc(to_f32(a_logit[gi]) + ba);
-                be = sigmoid_acc(to_f32(b_logit[gi]));
+                g = -eA * softplus_fast(to_f32(a_logit[gi]) + ba);
+                be = sigmoid_fast(to_f32(b_logit[gi]));
             }
             // inclusive scan of the log decays within each warp, then across the two
 #pragma unroll
@@ -386,6 +427,19 @@ chunk_prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const 
 
         // ---- 4. T = (I + L)^-1 (fp32, blocked); then T' = T diag(beta e^G) in rows
         //         0..63 and T'' = T diag(beta) in rows 64..127 of an fp16 K-major tile
+        // while the solve runs: pull the next chunk's raw rows and gate logits into L2
+        {
+            const int cn = c + gridDim.z;
+            if (cn < c_end) {
+                const int tn = s_begin + cn * C;
+                prefetch_rows<8>(is_k ? k : q, (size_t)H * DK, qk_col, tn, s_begin, s_end, 8 * warp);
+                prefetch_rows<C / VPARTS>(v, (size_t)H * DV, v_col, tn, s_begin, s_end, (C / VPARTS) * v_part);
+                if (tid < C && tn + tid < s_end) {
+                    prefetch_l2(a_logit + (size_t)(tn + tid) * H + h);
+                    prefetch_l2(b_logit + (size_t)(tn + tid) * H + h);
+                }
+            }
+        }
         solve_unit_lower<NT>(sL, sTf, sX, tid);
         for (int idx = tid; idx < C * 8; idx += NT) {
             const int i = idx >> 3, ch = idx & 7;
@@ -474,26 +528,33 @@ chunk_prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const 
     if (warp == 0) umma::tmem_dealloc(tbase, TMEM_COLS);
 }
 
-cudaError_t launch_chunk_prep(const PrefillArgs &a, const TcWorkspace &w) {
-    if (a.n_tok == 0) return cudaSuccess;
-    // blocks per (head, sequence): the longest sequence may hold every chunk, so
-    // give each (head, sequence) ~8 x 148 / H blocks; blocks past the end exit
+cudaError_t launch_chunk_prep(const PrefillArgs &a, const TcWorkspace &w, int c_lo, int c_hi,
+                              cudaStream_t stream) {
+    if (a.n_tok == 0 || c_hi <= c_lo) return cudaSuccess;
+    // blocks per (head, sequence): ~8 x 148 / H in total, at most one per chunk
+    // of the range (the longest sequence may fill it); blocks past the end exit
+    const int max_chunks = (a.n_tok + 63) / 64;
     int split = max(1, (8 * 148) / a.H);
-    split = min(split, (a.n_tok + 63) / 64);
+    split = min(split, min(c_hi, max_chunks) - c_lo);
+    if (split <= 0) return cudaSuccess;
     dim3 grid(a.H, a.n_seq, split);
     cudaError_t e;
 #define GDN_PREP(DV_)                                                                             \
     e = cudaFuncSetAttribute(chunk_prep_kernel<DV_>, cudaFuncAttributeMaxDynamicSharedMemorySize,  \
                              prep::SMEM);                                                          \
     if (e != cudaSuccess) return e;                                                                 \
-    chunk_prep_kernel<DV_><<<grid, 256, prep::SMEM, a.stream>>>(                                    \
+    chunk_prep_kernel<DV_><<<grid, 256, prep::SMEM, stream>>>(                                      \
         (const bf16 *)a.q, (const bf16 *)a.k, (const bf16 *)a.v, a.conv_w, (const bf16 *)a.a_logit, \
-        (const bf16 *)a.b_logit, a.A, a.b_alpha, a.cu_seqlens, a.n_seq, a.n_tok, a.H, w.Qt, w.Kt,   \
-        w.Wn, w.Up, w.Aqk, w.decay)
+        (const bf16 *)a.b_logit, a.A, a.b_alpha, a.cu_seqlens, a.n_seq, a.n_tok, a.H, c_lo, c_hi,   \
+        w.Qt, w.Kt, w.Wn, w.Up, w.Aqk, w.decay)
     if (!a.in_bf16) return cudaErrorInvalidValue;   // the tensor-core path takes bf16 inputs
     if (a.dv == 128) { GDN_PREP(128); } else { GDN_PREP(64); }
 #undef GDN_PREP
     return cudaGetLastError();
+}
+
+cudaError_t launch_chunk_prep(const PrefillArgs &a, const TcWorkspace &w) {
+    return launch_chunk_prep(a, w, 0, (a.n_tok + 63) / 64, a.stream);
 }
 
 }  // namespace gdn

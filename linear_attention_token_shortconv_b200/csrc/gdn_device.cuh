@@ -60,6 +60,37 @@ __device__ __forceinline__ float log_decay(float a_logit, float A, float b_alpha
     return -expf(A) * softplus_acc(a_logit + b_alpha);
 }
 
+// ---- packed fp32x2 arithmetic (sm_100): two lanes of work per instruction
+union F2 {
+    unsigned long long u;
+    float2 f;
+};
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    F2 x, y, z, r;
+    x.f = a; y.f = b; z.f = c;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r.u) : "l"(x.u), "l"(y.u), "l"(z.u));
+    return r.f;
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+    F2 x, y, r;
+    x.f = a; y.f = b;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r.u) : "l"(x.u), "l"(y.u));
+    return r.f;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+    F2 x, y, r;
+    x.f = a; y.f = b;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r.u) : "l"(x.u), "l"(y.u));
+    return r.f;
+}
+
+// Fast-math gates for the tensor-core path: softplus with the exp / log
+// intrinsics (absolute error ~1e-7), sigmoid with the intrinsic exp.
+__device__ __forceinline__ float softplus_fast(float x) {
+    return fmaxf(x, 0.f) + __logf(1.0f + __expf(-fabsf(x)));
+}
+__device__ __forceinline__ float sigmoid_fast(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
+
 template <int W>
 __device__ __forceinline__ float group_sum(float v) {
 #pragma unroll

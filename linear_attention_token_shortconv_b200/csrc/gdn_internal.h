@@ -42,8 +42,15 @@ struct TcWorkspace {
 };
 
 // K2a (prelude fused) / K2b: chunked prefill on tcgen05 (dk = 128, dv in {64, 128}).
+// The two-argument forms cover every chunk on a.stream, from a.S0 to a.S_final.
+// The ranged forms cover chunks [c_lo, c_hi) of every sequence on `stream`; the
+// chain carries the state from state_in (NULL: zeros) to state_out (NULL: dropped).
 cudaError_t launch_chunk_prep(const PrefillArgs &a, const TcWorkspace &w);
 cudaError_t launch_chunk_chain(const PrefillArgs &a, const TcWorkspace &w);
+cudaError_t launch_chunk_prep(const PrefillArgs &a, const TcWorkspace &w, int c_lo, int c_hi,
+                              cudaStream_t stream);
+cudaError_t launch_chunk_chain(const PrefillArgs &a, const TcWorkspace &w, int c_lo, int c_hi,
+                               const float *state_in, float *state_out, cudaStream_t stream);
 
 // Host side of TMA: a 3-D tiled tensor map over a token-indexed [N_tok][H][inner]
 // tensor (16-bit elements), box {box_inner, 1, box_rows}.
