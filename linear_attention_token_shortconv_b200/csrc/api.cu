@@ -317,7 +317,7 @@ gdn_status_t gdn_decode_step(const gdn_dims_t *dims, const void *q, const void *
     a.out = out;
     a.stream = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = record(g_ev_begin, a.stream);
-    if (e == cudaSuccess) e = gdn::launch_decode(a);
+    if (e == cudaSuccess) e = gdn::decode_stream_supported(a) ? gdn::launch_decode_stream(a) : gdn::launch_decode(a);
     if (e == cudaSuccess) e = record(g_ev_end, a.stream);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }

@@ -1,0 +1,266 @@
+// K3s -- the decode step as a streaming kernel (bf16 inputs, dk = dv = 128).
+//
+// Same arithmetic as K3 (slinene.github.io write-up of "On the Design of
+// Qwen3.8-Next Architecture", 模块 A; decode time is set by the bytes moved, as
+// the digest's 前置知识 notes): conv over [history, token], SiLU, L2Norm, gates,
+//     S' = alpha S + beta k e^T,  e = v - alpha S^T k,
+//     y  = alpha S^T q + beta (k.q) e,   out = sigmoid(z) RMSNorm(y) (1 + w).
+//
+// One persistent CTA per SM walks the (sequence, head) items.  Each item's
+// inputs -- the 64 KB fp32 state, the token's q, k, v, z rows and the three
+// history rows -- arrive by bulk copies (TMA, cp.async.bulk) into one of three
+// shared-memory stages, completing on the stage's mbarrier.  The CTA moves the
+// stage into registers at once and refills it with the item three ahead, so
+// three state loads are in flight while it computes; S' leaves from registers
+// with coalesced streaming stores.  Every wait is bounded.
+#include <cuda_bf16.h>
+
+#include "gdn_device.cuh"
+#include "gdn_internal.h"
+#include "umma.cuh"
+
+namespace gdn {
+
+__device__ unsigned int g_decode_err;
+
+namespace dstream {
+constexpr int D = 128;                      // dk = dv
+constexpr int NT = 256;
+constexpr int STATE = D * D * 4;            // 64 KB
+constexpr int OFF_TOK = STATE;              // q, k, v, z rows: 4 x 256 B
+constexpr int OFF_HIST = OFF_TOK + 1024;    // 3 slots x (q, k, v) x 256 B
+constexpr int STAGE = OFF_HIST + 2304;      // 68,864 B (multiple of 128)
+constexpr int NSTAGE = 3;
+constexpr int OFF_MISC = NSTAGE * STAGE;    // barriers, reductions, prelude values
+constexpr int SMEM = OFF_MISC + 128 + (2 * 384 + 2 * 8 * 128 + 256) * 4 + 128;
+static_assert(STAGE % 128 == 0, "stage alignment");
+static_assert(SMEM <= 232448, "227 KB per block");
+constexpr uint32_t kMaxPolls = 1u << 24;
+}  // namespace dstream
+
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            umma::smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(umma::smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+                 "r"(umma::smem_u32(src)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool dwait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+    for (uint32_t i = 0; i < dstream::kMaxPolls; ++i) {
+        if (umma::mbar_try_wait(bar, parity)) return true;
+        if ((i & 255u) == 255u && *abort_flag) return false;
+    }
+    *abort_flag = 1;
+    atomicOr(&g_decode_err, 1u);
+    return false;
+}
+
+template <typename Tout>
+__global__ void __launch_bounds__(dstream::NT, 1)
+decode_stream_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
+                     const bf16 *__restrict__ v, const float *__restrict__ conv_w,
+                     bf16 *__restrict__ hist, const bf16 *__restrict__ a_logit,
+                     const bf16 *__restrict__ b_logit, const float *__restrict__ A,
+                     const float *__restrict__ b_alpha, const bf16 *__restrict__ z,
+                     const float *__restrict__ norm_w, float *__restrict__ S,
+                     Tout *__restrict__ out, int B, int H) {
+    using namespace dstream;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + OFF_MISC);            // [3]
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OFF_MISC + 32);
+    float *scal = reinterpret_cast<float *>(sm + OFF_MISC + 64);             // |q|^2, |k|^2, q.k, alpha, beta
+    float *xs2 = reinterpret_cast<float *>(sm + OFF_MISC + 128);             // [2][384] conv+SiLU values
+    float *red = xs2 + 2 * 384;                                              // [2][8][128]
+    float *ey = red + 2 * 8 * 128;                                           // e[128], y[128]
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n_items = B * H;
+    const size_t C = (size_t)H * 3 * D;   // conv channels per token
+
+    if (tid == 0) {
+        for (int i = 0; i < NSTAGE; ++i) umma::mbar_init(full + i, 1);
+        *abort_flag = 0;
+        umma::fence_mbar_init();
+    }
+    __syncthreads();
+
+    auto issue = [&](int item, int s) {   // tid 0 only
+        const int b = item / H, h = item % H;
+        uint8_t *st = sm + s * STAGE;
+        uint64_t *bar = full + s;
+        umma::mbar_expect_tx(bar, STAGE);
+        const float *Sh = S + ((size_t)b * H + h) * D * D;
+#pragma unroll
+        for (int p = 0; p < 4; ++p) bulk_load(st + p * (STATE / 4), Sh + p * (D * D / 4), STATE / 4, bar);
+        const size_t tok = ((size_t)b * H + h) * D;
+        bulk_load(st + OFF_TOK, q + tok, 256, bar);
+        bulk_load(st + OFF_TOK + 256, k + tok, 256, bar);
+        bulk_load(st + OFF_TOK + 512, v + tok, 256, bar);
+        bulk_load(st + OFF_TOK + 768, z + tok, 256, bar);
+#pragma unroll
+        for (int j = 0; j < 3; ++j) {
+            const bf16 *hr = hist + ((size_t)b * 3 + j) * C;
+            bulk_load(st + OFF_HIST + j * 768, hr + (size_t)h * D, 256, bar);
+            bulk_load(st + OFF_HIST + j * 768 + 256, hr + (size_t)H * D + (size_t)h * D, 256, bar);
+            bulk_load(st + OFF_HIST + j * 768 + 512, hr + (size_t)2 * H * D + (size_t)h * D, 256, bar);
+        }
+    };
+    const int first = blockIdx.x, stride = gridDim.x;
+    if (tid == 0) {
+#pragma unroll
+        for (int i = 0; i < NSTAGE; ++i)
+            if (first + i * stride < n_items) issue(first + i * stride, i);
+    }
+
+    int j = 0;
+    for (int item = first; item < n_items; item += stride, ++j) {
+        const int s = j % NSTAGE;
+        const uint32_t parity = (uint32_t)(j / NSTAGE) & 1u;
+        const uint8_t *st = sm + s * STAGE;
+        float *xs = xs2 + (j & 1) * 384;
+        const int b = item / H, h = item % H;
+        const size_t gi = (size_t)b * H + h;
+        const float a_l = __bfloat162float(a_logit[gi]), b_l = __bfloat162float(b_logit[gi]);
+        // this thread's conv weights: channel tid (q or k) and, for tid < 128, v channel tid
+        const float4 w0 = __ldg(reinterpret_cast<const float4 *>(conv_w) +
+                                (tid < D ? (size_t)h * D + tid : (size_t)H * D + (size_t)h * D + (tid - D)));
+        const float4 w1 = tid < D ? __ldg(reinterpret_cast<const float4 *>(conv_w) + (size_t)2 * H * D + (size_t)h * D + tid)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+        dwait(full + s, parity, abort_flag);
+
+        // ---- take everything out of the stage: the state into registers (thread t
+        // holds float4 t + 256 r, i.e. row t/32 + 8 r, columns 4 (t%32) ..), the
+        // conv inputs through the prelude into xs, z into warp 7's registers; the
+        // shifted history goes straight back to global memory.
+        const float4 *Sv = reinterpret_cast<const float4 *>(st);
+        float4 sreg[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) sreg[r] = Sv[tid + r * NT];
+        const bf16 *tok = reinterpret_cast<const bf16 *>(st + OFF_TOK);
+        const bf16 *hs = reinterpret_cast<const bf16 *>(st + OFF_HIST);
+        bf16 *hb = hist + (size_t)b * 3 * C;
+        for (int ch = tid; ch < 3 * D; ch += NT) {
+            const int part = ch / D, i = ch % D;   // part 0 q, 1 k, 2 v
+            const float4 w = ch < NT ? w0 : w1;
+            const bf16 h1 = hs[1 * 384 + part * 128 + i], h2 = hs[2 * 384 + part * 128 + i];
+            const bf16 xc = tok[part * 128 + i];
+            float acc = w.x * __bfloat162float(hs[0 * 384 + part * 128 + i]);
+            acc = fmaf(w.y, __bfloat162float(h1), acc);
+            acc = fmaf(w.z, __bfloat162float(h2), acc);
+            acc = fmaf(w.w, __bfloat162float(xc), acc);
+            xs[ch] = __fdividef(acc, 1.0f + __expf(-acc));
+            const size_t c = (size_t)part * H * D + (size_t)h * D + i;
+            hb[c] = h1;
+            hb[C + c] = h2;
+            hb[2 * C + c] = xc;
+        }
+        float zr[4];
+        if (warp == NT / 32 - 1) {
+#pragma unroll
+            for (int m = 0; m < 4; ++m) zr[m] = __bfloat162float(tok[3 * 128 + lane + 32 * m]);
+        }
+        __syncthreads();   // stage s is consumed and xs is complete
+        if (tid == 0 && item + NSTAGE * stride < n_items) issue(item + NSTAGE * stride, s);
+
+        if (warp < 3) {   // warp 0: |q|^2, warp 1: |k|^2, warp 2: q.k
+            const float *xa = xs + (warp == 1 ? D : 0), *xb = xs + (warp == 0 ? 0 : D);
+            float acc = 0.f;
+#pragma unroll
+            for (int i = lane; i < D; i += 32) acc = fmaf(xa[i], xb[i], acc);
+            acc = group_sum<32>(acc);
+            if (lane == 0) scal[warp] = acc;
+        } else if (tid == 96) {
+            scal[3] = expf(log_decay(a_l, __ldg(A + h), __ldg(b_alpha + h)));
+            scal[4] = sigmoid_acc(b_l);
+        }
+        // ---- partial S^T k and S^T q over this thread's 16 rows
+        float pk[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            const int i = warp + 8 * r;
+            const float kk = xs[D + i], qq = xs[i];
+            pk[0] = fmaf(sreg[r].x, kk, pk[0]); pk[1] = fmaf(sreg[r].y, kk, pk[1]);
+            pk[2] = fmaf(sreg[r].z, kk, pk[2]); pk[3] = fmaf(sreg[r].w, kk, pk[3]);
+            pq[0] = fmaf(sreg[r].x, qq, pq[0]); pq[1] = fmaf(sreg[r].y, qq, pq[1]);
+            pq[2] = fmaf(sreg[r].z, qq, pq[2]); pq[3] = fmaf(sreg[r].w, qq, pq[3]);
+        }
+        reinterpret_cast<float4 *>(red + warp * D)[lane] = make_float4(pk[0], pk[1], pk[2], pk[3]);
+        reinterpret_cast<float4 *>(red + 8 * D + warp * D)[lane] = make_float4(pq[0], pq[1], pq[2], pq[3]);
+        __syncthreads();
+        const float rq = rsqrtf(scal[0] + kNormEps), rk = rsqrtf(scal[1] + kNormEps);
+        const float kq = scal[2] * rq * rk, alpha = scal[3], beta = scal[4];
+        if (tid < D) {
+            float sk = 0.f, sq = 0.f;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) { sk += red[w * D + tid]; sq += red[8 * D + w * D + tid]; }
+            const float e = xs[2 * D + tid] - alpha * rk * sk;
+            ey[tid] = e;
+            ey[D + tid] = fmaf(beta * kq, e, alpha * rq * sq);
+        }
+        __syncthreads();
+        // ---- S' = alpha S + beta k e^T, from registers straight to HBM
+        {
+            const float4 e4 = reinterpret_cast<const float4 *>(ey)[lane];
+            float4 *Sg = reinterpret_cast<float4 *>(S + gi * D * D);
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                const float bk = beta * rk * xs[D + warp + 8 * r];
+                float4 o;
+                o.x = fmaf(bk, e4.x, alpha * sreg[r].x);
+                o.y = fmaf(bk, e4.y, alpha * sreg[r].y);
+                o.z = fmaf(bk, e4.z, alpha * sreg[r].z);
+                o.w = fmaf(bk, e4.w, alpha * sreg[r].w);
+                __stcs(Sg + tid + r * NT, o);
+            }
+        }
+        // ---- output (warp 7)
+        if (warp == NT / 32 - 1) {
+            float yv[4], ss = 0.f;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) { yv[m] = ey[D + lane + 32 * m]; ss = fmaf(yv[m], yv[m], ss); }
+            ss = group_sum<32>(ss);
+            const float rr = rsqrtf(ss / D + kNormEps);
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int col = lane + 32 * m;
+                out[gi * D + col] = from_f32<Tout>(sigmoid_fast(zr[m]) * yv[m] * rr * (1.0f + __ldg(norm_w + col)));
+            }
+        }
+        // No barrier here: the next item writes the other xs buffer before its
+        // first barrier, and red / ey / scal only after it.
+    }
+}
+
+bool decode_stream_supported(const DecodeArgs &a) {
+    return a.in_bf16 && a.dk == 128 && a.dv == 128;
+}
+
+cudaError_t launch_decode_stream(const DecodeArgs &a) {
+    int dev = 0, sms = 148;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    const int items = a.B * a.H;
+    const int grid = items < sms ? items : sms;
+#define GDN_DSTREAM(TOUT)                                                                          \
+    e = cudaFuncSetAttribute(decode_stream_kernel<TOUT>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             dstream::SMEM);                                                      \
+    if (e != cudaSuccess) return e;                                                                \
+    decode_stream_kernel<TOUT><<<grid, dstream::NT, dstream::SMEM, a.stream>>>(                    \
+        (const bf16 *)a.q, (const bf16 *)a.k, (const bf16 *)a.v, a.conv_w, (bf16 *)a.conv_hist,   \
+        (const bf16 *)a.a_logit, (const bf16 *)a.b_logit, a.A, a.b_alpha, (const bf16 *)a.z,      \
+        a.norm_w, a.S, (TOUT *)a.out, a.B, a.H)
+    if (a.out_bf16) { GDN_DSTREAM(bf16); } else { GDN_DSTREAM(float); }
+#undef GDN_DSTREAM
+    return cudaGetLastError();
+}
+
+}  // namespace gdn

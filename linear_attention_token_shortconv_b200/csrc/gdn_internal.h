@@ -62,7 +62,10 @@ cudaError_t make_tma_3d(TmaMap *out, const void *base, bool bf16, int inner, int
 cudaError_t launch_recurrent(const PrefillArgs &a, const float *qn, const float *kn,
                              const float *vn);
 
-// K3: one decode step.
+// K3: one decode step (any supported dims / dtypes).
 cudaError_t launch_decode(const DecodeArgs &a);
+// K3s: the streaming decode step for bf16 inputs with dk = dv = 128.
+bool decode_stream_supported(const DecodeArgs &a);
+cudaError_t launch_decode_stream(const DecodeArgs &a);
 
 }  // namespace gdn
