@@ -41,7 +41,31 @@ METRIC = "GDN prefill tokens/s at T=32K H=32 (% TC peak); decode state GB/s (% H
 # logits and a bf16 output.
 PREFILL_FLOP_PER_TOKEN_HEAD = 64 * (6 * 128 + 4 * 128) + 6 * 128 * 128   # 180,224
 PREFILL_BYTES_PER_TOKEN_HEAD = 4 * 128 * 2 + 2 * 2 + 128 * 2           # 1,284
+# ... of which each kernel of the two-kernel split touches: chunk_prep reads
+# q, k, v and the two logits; chunk_chain reads z and writes the output.
+KERNEL_BYTES_PER_TOKEN_HEAD = {"chunk_prep": 3 * 128 * 2 + 2 * 2,          # 772
+                               "chunk_chain": 128 * 2 + 128 * 2}           # 512
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per token-head from
+# an ncu capture of each kernel, valid only while the kernel's source is the one
+# captured (sha1 of the .cu file); otherwise the JSON reports traffic null.
+NCU_TRAFFIC = {}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def kernel_traffic(name, units):
+    """ncu DRAM bytes for one launch of `name` processing `units` token-heads,
+    or None when no capture of the kernel's current source exists."""
+    rec = NCU_TRAFFIC.get(name)
+    if rec is None:
+        return None
+    import hashlib
+    path = os.path.join(ROOT, "linear_attention_token_shortconv_b200", "csrc", rec["source"])
+    try:
+        with open(path, "rb") as f:
+            sha = hashlib.sha1(f.read()).hexdigest()
+    except OSError:
+        return None
+    return rec["bytes_per_token_head"] * units if sha == rec["sha1"] else None
 
 
 def peaks():
@@ -140,33 +164,52 @@ def prefill_call(inp, out, S_final):
 
 
 def bench_prefill(cfg, steps, warmup, world, rank, dev):
+    """Times `steps` gdn_prefill calls.  Besides the whole-call events (on the
+    caller's stream, which the library forks from and joins), every kernel
+    launch is bracketed by its own pair of events on the stream it runs on."""
     inp = make_prefill_inputs(cfg, dev, seed=cfg.seed + 1000 * rank)
     n_tok, H = cfg.total_tokens, cfg.H
     out = torch.empty((n_tok, H, cfg.dv), dtype=torch.bfloat16, device=dev)
     S_final = torch.empty((cfg.num_seqs, H, cfg.dk, cfg.dv), dtype=torch.float32, device=dev)
     for _ in range(warmup):
         prefill_call(inp, out, S_final)
+    n_launch = gdn.last_call_launches()
     torch.cuda.synchronize()
-    evb = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
-    eve = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
-    for e in evb + eve:      # materialise the events before handing them to the library
+    mk = lambda n: [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    evb, eve = mk(steps), mk(steps)
+    kb, ke = [mk(n_launch) for _ in range(steps)], [mk(n_launch) for _ in range(steps)]
+    for e in evb + eve + sum(kb, []) + sum(ke, []):   # materialise the CUDA handles
         e.record()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
+    launches = 0
     with ClockSampler(dev.index) as clk:
         start.record()
         for i in range(steps):
             gdn.set_timing_events(evb[i], eve[i])
+            gdn.set_kernel_events(kb[i], ke[i])
             prefill_call(inp, out, S_final)
+            launches += gdn.last_call_launches()
         end.record()
         gdn.set_timing_events(None, None)
+        gdn.set_kernel_events()
         torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(start.elapsed_time(end) / steps, world)
     kern_ms = max_over_ranks(sum(b.elapsed_time(e) for b, e in zip(evb, eve)) / steps, world)
-    return ms, kern_ms, clk.summary(), inp
+    # slots alternate chunk_prep (even) and chunk_chain (odd)
+    per = {"chunk_prep": [], "chunk_chain": []}
+    for i in range(steps):
+        for j in range(n_launch):
+            per["chunk_prep" if j % 2 == 0 else "chunk_chain"].append(kb[i][j].elapsed_time(ke[i][j]))
+    kernels = {}
+    for name, xs in per.items():
+        kernels[name] = {"launches_per_step": len(xs) // steps,
+                         "avg_launch_ms": max_over_ranks(statistics.fmean(xs), world),
+                         "ms_per_step": max_over_ranks(sum(xs) / steps, world)}
+    return ms, kern_ms, clk.summary(), kernels, launches, inp
 
 
 def bench_e2e(cfg, steps, warmup, world, rank, dev):
@@ -227,17 +270,19 @@ def bench_decode(cfg, steps, dev):
         e.record()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
+    launches = 0
     start.record()
     for t in range(steps):
         gdn.set_timing_events(evb[t], eve[t])
         step(t)
+        launches += gdn.last_call_launches()
     end.record()
     gdn.set_timing_events(None, None)
     torch.cuda.synchronize()
     ms = start.elapsed_time(end) / steps
     kern_ms = sum(b.elapsed_time(e) for b, e in zip(evb, eve)) / steps
     state_bytes = 2 * cfg.B * cfg.H * cfg.dk * cfg.dv * 4
-    return ms, kern_ms, state_bytes
+    return ms, kern_ms, state_bytes, launches
 
 
 def oracle_sample_rate(inp, cfg, tokens, heads, n_threads):
@@ -312,11 +357,17 @@ def main():
     pk, pk_kind = peaks()
 
     cfg = LONG
-    ms, kern_ms, clocks, inp = bench_prefill(cfg, args.steps, args.warmup, world, rank, dev)
+    ms, kern_ms, clocks, kernels, launches, inp = bench_prefill(cfg, args.steps, args.warmup, world,
+                                                                rank, dev)
     token_heads = cfg.total_tokens * cfg.H
     value = world * cfg.total_tokens / (ms * 1e-3)
-    hbm_achieved = PREFILL_BYTES_PER_TOKEN_HEAD * token_heads / (kern_ms * 1e-3) / 1e9
+    path_gbs = PREFILL_BYTES_PER_TOKEN_HEAD * token_heads / (kern_ms * 1e-3) / 1e9
     tc_achieved = PREFILL_FLOP_PER_TOKEN_HEAD * token_heads / (kern_ms * 1e-3) / 1e12
+    dom = max(kernels, key=lambda n: kernels[n]["ms_per_step"])
+    kd = kernels[dom]
+    units_per_launch = token_heads / kd["launches_per_step"]
+    dom_gbs = KERNEL_BYTES_PER_TOKEN_HEAD[dom] * units_per_launch / (kd["avg_launch_ms"] * 1e-3) / 1e9
+    traffic = kernel_traffic(dom, units_per_launch)
 
     result = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -326,27 +377,32 @@ def main():
                                "fp32 state, S0~N(0,0.02), per GPU",
                    "global_batch": world, "seq_len": cfg.total_tokens, "parallelism": f"dp{world}",
                    "l2": "inputs larger than L2 (1.07 GB of bf16 q,k,v,z read per step)"},
-        "roofline": {"bound": "hbm", "achieved": hbm_achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                     "frac": hbm_achieved / pk["hbm_gbs"], "traffic": None,
-                     "kernel": "state recurrence (chain) kernel", "kernel_ms": kern_ms,
-                     "peak_kind": pk_kind},
+        "roofline": {"bound": "hbm", "achieved": dom_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": dom_gbs / pk["hbm_gbs"], "traffic": traffic, "kernel": dom,
+                     "bytes_per_token_head": KERNEL_BYTES_PER_TOKEN_HEAD[dom],
+                     "token_heads_per_launch": units_per_launch,
+                     "avg_launch_ms": kd["avg_launch_ms"], "peak_kind": pk_kind,
+                     "kernels": kernels,
+                     "path": {"what": "whole gdn_prefill call (both kernels, two streams)",
+                              "call_ms": kern_ms, "bytes_per_token_head": PREFILL_BYTES_PER_TOKEN_HEAD,
+                              "achieved_gbs": path_gbs, "frac": path_gbs / pk["hbm_gbs"]}},
         "tc": {"achieved_tflops": tc_achieved, "peak_tflops": pk["bf16_tflops"],
                "frac": tc_achieved / pk["bf16_tflops"], "peak_kind": pk_kind + " burst",
-               "flop_per_token_head": PREFILL_FLOP_PER_TOKEN_HEAD},
-        "gpu_launches": 2 * args.steps,
+               "flop_per_token_head": PREFILL_FLOP_PER_TOKEN_HEAD, "over": "whole gdn_prefill call"},
+        "gpu_launches": launches,
         "clocks": clocks,
     }
     del inp
     torch.cuda.empty_cache()
 
     if rank == 0 and args.decode_steps > 0:
-        dms, dk_ms, sbytes = bench_decode(DECODE, args.decode_steps, dev)
+        dms, dk_ms, sbytes, dlaunch = bench_decode(DECODE, args.decode_steps, dev)
         gbs = sbytes / (dk_ms * 1e-3) / 1e9
         result["decode"] = {"workload": DECODE.name, "steps": args.decode_steps,
                             "ms_per_step": dms, "kernel_ms": dk_ms,
                             "state_gbs": gbs, "peak_gbs": pk["hbm_gbs"],
                             "frac": gbs / pk["hbm_gbs"], "state_bytes_per_step": sbytes,
-                            "gpu_launches": args.decode_steps}
+                            "kernel": "decode_stream", "gpu_launches": dlaunch}
         torch.cuda.empty_cache()
 
     if not args.no_e2e:

@@ -185,6 +185,48 @@ GDN_API gdn_status_t gdn_prefill_noalloc(const gdn_dims_t *dims, const void *q, 
  */
 GDN_API gdn_status_t gdn_set_timing_events(void *begin, void *end);
 
+/*
+ * gdn_set_kernel_events -- optional per-launch profiling hook (host call, not
+ * thread-safe).  begin[i] / end[i] (cudaEvent_t values, created and owned by
+ * the caller; the library copies the n handles) are recorded around launch
+ * slot i of every following gdn_prefill / gdn_decode_step call, on the stream
+ * that slot's kernel runs on.  Slots in launch order:
+ *   gdn_prefill, tensor-core path, n segments: chunk_prep(0), chunk_chain(0),
+ *     chunk_prep(1), chunk_chain(1), ... -- chunk_prep on the caller's stream,
+ *     chunk_chain on the library's side stream of the device;
+ *   gdn_prefill, fp32 path: prelude, recurrent;
+ *   gdn_decode_step: the decode kernel.
+ * Slots beyond n are not recorded.  n = 0 clears the hook.  Returns
+ * GDN_ERR_INVALID_ARG for n < 0 or a NULL handle among the first n.
+ */
+GDN_API gdn_status_t gdn_set_kernel_events(void *const *begin, void *const *end, int n);
+
+/*
+ * Number of kernels the calling thread's most recent gdn_prefill,
+ * gdn_prefill_noalloc or gdn_decode_step call launched (0 after a call that
+ * returned before its first launch).  Host-side count, no synchronisation.
+ */
+GDN_API int gdn_last_call_launches(void);
+
+/*
+ * Device error flags.  Every wait inside the kernels (on an mbarrier fed by TMA
+ * or by the tensor cores) is bounded; when one expires the kernel raises its
+ * family's device error word, gives up its remaining waits promptly and
+ * returns, so a stuck transfer shows up as an error status instead of a hang.
+ */
+#define GDN_ERRF_PREP 1u    /* chunk_prep (gdn_prefill, tensor-core path) */
+#define GDN_ERRF_CHAIN 2u   /* chunk_chain (gdn_prefill, tensor-core path) */
+#define GDN_ERRF_DECODE 4u  /* streaming decode kernel (gdn_decode_step) */
+
+/*
+ * gdn_device_error_status -- reads the current device's error words into
+ * *flags (a GDN_ERRF_* mask; may be NULL) and, when `clear` is non-zero, resets
+ * them.  Synchronises `stream` (the reads are ordered after the work queued on
+ * it).  Returns GDN_ERR_TIMEOUT when any flag is set, GDN_OK when none is,
+ * GDN_ERR_CUDA if the reads fail.
+ */
+GDN_API gdn_status_t gdn_device_error_status(unsigned *flags, int clear, gdn_stream_t stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 GDN_API const char *gdn_status_string(gdn_status_t status);
 

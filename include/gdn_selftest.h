@@ -30,6 +30,23 @@ GDN_API gdn_status_t gdn_selftest_umma(int a_mn, int b_mn, int negate_a, int N, 
                                        const void *A, const void *B, const float *init,
                                        float *D, gdn_stream_t stream);
 
+/*
+ * gdn_selftest_wait_timeout -- failure-detection check of one kernel family's
+ * bounded wait.  Launches one CTA that waits, through the family's own wait
+ * routine, for an mbarrier phase that nothing completes; after `max_polls`
+ * polls the wait gives up and raises the family's device error word, which
+ * gdn_device_error_status then reports.  Nothing faults and the context stays
+ * usable.
+ *
+ *   family     GDN_ERRF_PREP, GDN_ERRF_CHAIN or GDN_ERRF_DECODE (one bit)
+ *   max_polls  1 .. 65536
+ *
+ * Asynchronous on `stream`.  GDN_ERR_INVALID_ARG for another family value or
+ * max_polls out of range, GDN_ERR_CUDA if the launch fails.
+ */
+GDN_API gdn_status_t gdn_selftest_wait_timeout(unsigned family, unsigned max_polls,
+                                               gdn_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -131,9 +131,55 @@ cudaError_t record(cudaEvent_t ev, cudaStream_t s) {
     return ev ? cudaEventRecord(ev, s) : cudaSuccess;
 }
 
+// Per-launch timing hook (gdn_set_kernel_events): slot i of a call is recorded
+// around that call's i-th kernel launch, on the stream the kernel runs on.
+std::vector<cudaEvent_t> g_kev_begin, g_kev_end;
+thread_local int tl_launches = 0;
+
+template <class F>
+cudaError_t slot_launch(int *slot, cudaStream_t s, F &&launch) {
+    const int i = (*slot)++;
+    const bool rec = i < (int)g_kev_begin.size();
+    cudaError_t e = rec ? cudaEventRecord(g_kev_begin[i], s) : cudaSuccess;
+    if (e == cudaSuccess) e = launch();
+    if (e == cudaSuccess && rec) e = cudaEventRecord(g_kev_end[i], s);
+    return e;
+}
+
 }  // namespace
 
+namespace gdn {
+void note_launch() { ++tl_launches; }
+void reset_launch_count() { tl_launches = 0; }
+}  // namespace gdn
+
 extern "C" {
+
+gdn_status_t gdn_set_kernel_events(void *const *begin, void *const *end, int n) {
+    if (n < 0 || (n > 0 && (!begin || !end))) return GDN_ERR_INVALID_ARG;
+    for (int i = 0; i < n; ++i)
+        if (!begin[i] || !end[i]) return GDN_ERR_INVALID_ARG;
+    g_kev_begin.assign(reinterpret_cast<cudaEvent_t const *>(begin),
+                       reinterpret_cast<cudaEvent_t const *>(begin) + n);
+    g_kev_end.assign(reinterpret_cast<cudaEvent_t const *>(end),
+                     reinterpret_cast<cudaEvent_t const *>(end) + n);
+    return GDN_OK;
+}
+
+int gdn_last_call_launches(void) { return tl_launches; }
+
+gdn_status_t gdn_device_error_status(unsigned *flags, int clear, gdn_stream_t stream) {
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    unsigned w[3] = {0, 0, 0};
+    cudaError_t e = gdn::prep_error_word(&w[0], clear != 0, s);
+    if (e == cudaSuccess) e = gdn::chain_error_word(&w[1], clear != 0, s);
+    if (e == cudaSuccess) e = gdn::decode_error_word(&w[2], clear != 0, s);
+    if (e != cudaSuccess) return GDN_ERR_CUDA;
+    const unsigned f = (w[0] ? GDN_ERRF_PREP : 0u) | (w[1] ? GDN_ERRF_CHAIN : 0u) |
+                       (w[2] ? GDN_ERRF_DECODE : 0u);
+    if (flags) *flags = f;
+    return f ? GDN_ERR_TIMEOUT : GDN_OK;
+}
 
 gdn_status_t gdn_set_timing_events(void *begin, void *end) {
     if ((begin == nullptr) != (end == nullptr)) return GDN_ERR_INVALID_ARG;
@@ -167,6 +213,7 @@ gdn_status_t gdn_prefill(const gdn_dims_t *dims, const void *q, const void *k, c
                          const float *A, const float *b_alpha, const void *z,
                          const float *norm_w, const float *S0, const int32_t *cu_seqlens,
                          void *out, float *S_final, gdn_stream_t stream) {
+    tl_launches = 0;
     gdn_status_t st = check_dims(dims, false);
     if (st != GDN_OK) return st;
     if (!cu_seqlens && dims->total_tokens % dims->num_seqs != 0) return GDN_ERR_INVALID_ARG;
@@ -232,10 +279,13 @@ gdn_status_t gdn_prefill(const gdn_dims_t *dims, const void *q, const void *k, c
         w.Aqk = reinterpret_cast<__half *>(take(nt * 64 * 2));
         w.decay = reinterpret_cast<float *>(take(nt * 4));
         const Segments g = segments(dims);
+        int slot = 0;
         e = record(g_ev_begin, a.stream);
         if (g.n == 1) {
-            if (e == cudaSuccess) e = gdn::launch_chunk_prep(a, w);
-            if (e == cudaSuccess) e = gdn::launch_chunk_chain(a, w);
+            if (e == cudaSuccess)
+                e = slot_launch(&slot, a.stream, [&] { return gdn::launch_chunk_prep(a, w); });
+            if (e == cudaSuccess)
+                e = slot_launch(&slot, a.stream, [&] { return gdn::launch_chunk_chain(a, w); });
         } else {
             float *state = reinterpret_cast<float *>(take((size_t)a.n_seq * a.H * a.dk * a.dv * 4));
             int dev = 0;
@@ -250,13 +300,16 @@ gdn_status_t gdn_prefill(const gdn_dims_t *dims, const void *q, const void *k, c
                 if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->stream, ss->events[g.n], 0);
                 for (int sgi = 0; sgi < g.n && e == cudaSuccess; ++sgi) {
                     const int c_lo = sgi * g.seg, c_hi = c_lo + g.seg;
-                    e = gdn::launch_chunk_prep(a, w, c_lo, c_hi, a.stream);
+                    e = slot_launch(&slot, a.stream,
+                                    [&] { return gdn::launch_chunk_prep(a, w, c_lo, c_hi, a.stream); });
                     if (e == cudaSuccess) e = cudaEventRecord(ss->events[sgi], a.stream);
                     if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->stream, ss->events[sgi], 0);
                     const float *sin = sgi == 0 ? a.S0 : state;
                     float *sout = sgi == g.n - 1 ? a.S_final : state;
                     if (e == cudaSuccess)
-                        e = gdn::launch_chunk_chain(a, w, c_lo, c_hi, sin, sout, ss->stream);
+                        e = slot_launch(&slot, ss->stream, [&] {
+                            return gdn::launch_chunk_chain(a, w, c_lo, c_hi, sin, sout, ss->stream);
+                        });
                 }
                 // join: the caller's stream continues after the last chain launch
                 if (e == cudaSuccess) e = cudaEventRecord(ss->events[g.n + 1], ss->stream);
@@ -268,9 +321,11 @@ gdn_status_t gdn_prefill(const gdn_dims_t *dims, const void *q, const void *k, c
         float *qn = reinterpret_cast<float *>(ws);
         float *kn = reinterpret_cast<float *>(ws + round_up(nt * a.dk * sizeof(float)));
         float *vn = reinterpret_cast<float *>(ws + 2 * round_up(nt * a.dk * sizeof(float)));
-        e = gdn::launch_prelude_f32(a, qn, kn, vn);
+        int slot = 0;
+        e = slot_launch(&slot, a.stream, [&] { return gdn::launch_prelude_f32(a, qn, kn, vn); });
         if (e == cudaSuccess) e = record(g_ev_begin, a.stream);
-        if (e == cudaSuccess) e = gdn::launch_recurrent(a, qn, kn, vn);
+        if (e == cudaSuccess)
+            e = slot_launch(&slot, a.stream, [&] { return gdn::launch_recurrent(a, qn, kn, vn); });
         if (e == cudaSuccess) e = record(g_ev_end, a.stream);
     }
     if (ws) {
@@ -285,6 +340,7 @@ gdn_status_t gdn_decode_step(const gdn_dims_t *dims, const void *q, const void *
                              const void *a_logit, const void *b_logit, const float *A,
                              const float *b_alpha, const void *z, const float *norm_w, float *S,
                              void *out, gdn_stream_t stream) {
+    tl_launches = 0;
     gdn_status_t st = check_dims(dims, true);
     if (st != GDN_OK) return st;
     const void *vec[] = {q, k, v, conv_w, conv_hist, z, S, out};
@@ -317,7 +373,11 @@ gdn_status_t gdn_decode_step(const gdn_dims_t *dims, const void *q, const void *
     a.out = out;
     a.stream = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = record(g_ev_begin, a.stream);
-    if (e == cudaSuccess) e = gdn::decode_stream_supported(a) ? gdn::launch_decode_stream(a) : gdn::launch_decode(a);
+    int slot = 0;
+    if (e == cudaSuccess)
+        e = slot_launch(&slot, a.stream, [&] {
+            return gdn::decode_stream_supported(a) ? gdn::launch_decode_stream(a) : gdn::launch_decode(a);
+        });
     if (e == cudaSuccess) e = record(g_ev_end, a.stream);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }

@@ -94,8 +94,9 @@ template <> __device__ __forceinline__ void store8_out<bf16>(bf16 *p, const floa
 // Bounded wait; on expiry raise the CTA's abort flag and the device error word.
 // Once the flag is up every other wait of the CTA gives up quickly, so the
 // kernel always finishes.
-__device__ __forceinline__ bool chain_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
-    for (uint32_t i = 0; i < chain::kMaxPolls; ++i) {
+__device__ __forceinline__ bool chain_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                           uint32_t max_polls = chain::kMaxPolls) {
+    for (uint32_t i = 0; i < max_polls; ++i) {
         if (umma::mbar_try_wait(bar, parity)) return true;
         if ((i & 255u) == 255u && *abort_flag) return false;
     }
@@ -417,11 +418,33 @@ cudaError_t launch_chunk_chain(const PrefillArgs &a, const TcWorkspace &w, int c
         if (a.out_bf16) { GDN_CHAIN(64, bf16); } else { GDN_CHAIN(64, float); }
     }
 #undef GDN_CHAIN
-    return cudaGetLastError();
+    return launched();
 }
 
 cudaError_t launch_chunk_chain(const PrefillArgs &a, const TcWorkspace &w) {
     return launch_chunk_chain(a, w, 0, (a.n_tok + 63) / 64 + 1, a.S0, a.S_final, a.stream);
+}
+
+// One CTA waits, through chain_wait, for a barrier phase that nothing completes.
+__global__ void chain_wait_selftest_kernel(uint32_t max_polls) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        umma::mbar_init(&bar, 1);
+        abort_flag = 0;
+        umma::fence_mbar_init();
+    }
+    __syncthreads();
+    chain_wait(&bar, 0, &abort_flag, max_polls);
+}
+
+cudaError_t chain_wait_selftest(uint32_t max_polls, cudaStream_t s) {
+    chain_wait_selftest_kernel<<<1, 32, 0, s>>>(max_polls);
+    return cudaGetLastError();
+}
+
+cudaError_t chain_error_word(unsigned *v, bool clear, cudaStream_t s) {
+    return read_error_word(g_chain_err, v, clear, s);
 }
 
 }  // namespace gdn

@@ -36,6 +36,15 @@
 namespace gdn {
 
 __device__ unsigned int g_prep_err;
+constexpr uint32_t kPrepMaxPolls = 1u << 22;
+
+// Block-wide bounded wait for phase `phase` of `bar`: true only if every thread
+// saw it complete; on expiry thread 0 raises the device error word.
+__device__ __forceinline__ bool prep_wait(uint64_t *bar, uint32_t phase, uint32_t max_polls) {
+    const bool ok = __syncthreads_and(umma::mbar_wait_bounded(bar, phase, max_polls));
+    if (!ok && threadIdx.x == 0) atomicOr(&g_prep_err, 1u);
+    return ok;
+}
 
 namespace prep {
 constexpr int C = 64;          // chunk length
@@ -379,7 +388,7 @@ chunk_prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const 
             }
             if (tid == 0) decay[(size_t)t0 * H + h] = __expf(GC);
         }
-        ok = __syncthreads_and(umma::mbar_wait_bounded(bar, phase, 1u << 22));
+        ok = prep_wait(bar, phase, kPrepMaxPolls);
         phase ^= 1;
         umma::tc_fence_after();
         if (!ok) break;
@@ -478,7 +487,7 @@ chunk_prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const 
             }
             umma::mma_commit(bar);
         }
-        ok = __syncthreads_and(umma::mbar_wait_bounded(bar, phase, 1u << 22));
+        ok = prep_wait(bar, phase, kPrepMaxPolls);
         phase ^= 1;
         umma::tc_fence_after();
         if (!ok) break;
@@ -522,7 +531,6 @@ chunk_prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const 
         umma::tc_fence_before();
         __syncthreads();
     }
-    if (!ok && tid == 0) atomicOr(&g_prep_err, 1u);
     umma::tc_fence_before();
     __syncthreads();
     if (warp == 0) umma::tmem_dealloc(tbase, TMEM_COLS);
@@ -550,11 +558,31 @@ cudaError_t launch_chunk_prep(const PrefillArgs &a, const TcWorkspace &w, int c_
     if (!a.in_bf16) return cudaErrorInvalidValue;   // the tensor-core path takes bf16 inputs
     if (a.dv == 128) { GDN_PREP(128); } else { GDN_PREP(64); }
 #undef GDN_PREP
-    return cudaGetLastError();
+    return launched();
 }
 
 cudaError_t launch_chunk_prep(const PrefillArgs &a, const TcWorkspace &w) {
     return launch_chunk_prep(a, w, 0, (a.n_tok + 63) / 64, a.stream);
+}
+
+// One CTA waits, through prep_wait, for a barrier phase that nothing completes.
+__global__ void prep_wait_selftest_kernel(uint32_t max_polls) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        umma::mbar_init(&bar, 1);
+        umma::fence_mbar_init();
+    }
+    __syncthreads();
+    prep_wait(&bar, 0, max_polls);
+}
+
+cudaError_t prep_wait_selftest(uint32_t max_polls, cudaStream_t s) {
+    prep_wait_selftest_kernel<<<1, 64, 0, s>>>(max_polls);
+    return cudaGetLastError();
+}
+
+cudaError_t prep_error_word(unsigned *v, bool clear, cudaStream_t s) {
+    return read_error_word(g_prep_err, v, clear, s);
 }
 
 }  // namespace gdn

@@ -157,7 +157,7 @@ static cudaError_t launch_dec_dims(const DecodeArgs &a) {
         if (a.out_bf16) GDN_DEC(float, bf16); else GDN_DEC(float, float);
     }
 #undef GDN_DEC
-    return cudaGetLastError();
+    return launched();
 }
 
 cudaError_t launch_decode(const DecodeArgs &a) {

@@ -52,8 +52,9 @@ __device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t 
                  : "memory");
 }
 
-__device__ __forceinline__ bool dwait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
-    for (uint32_t i = 0; i < dstream::kMaxPolls; ++i) {
+__device__ __forceinline__ bool dwait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                      uint32_t max_polls = dstream::kMaxPolls) {
+    for (uint32_t i = 0; i < max_polls; ++i) {
         if (umma::mbar_try_wait(bar, parity)) return true;
         if ((i & 255u) == 255u && *abort_flag) return false;
     }
@@ -260,7 +261,29 @@ cudaError_t launch_decode_stream(const DecodeArgs &a) {
         a.norm_w, a.S, (TOUT *)a.out, a.B, a.H)
     if (a.out_bf16) { GDN_DSTREAM(bf16); } else { GDN_DSTREAM(float); }
 #undef GDN_DSTREAM
+    return launched();
+}
+
+// One CTA waits, through dwait, for a barrier phase that nothing completes.
+__global__ void decode_wait_selftest_kernel(uint32_t max_polls) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        umma::mbar_init(&bar, 1);
+        abort_flag = 0;
+        umma::fence_mbar_init();
+    }
+    __syncthreads();
+    dwait(&bar, 0, &abort_flag, max_polls);
+}
+
+cudaError_t decode_wait_selftest(uint32_t max_polls, cudaStream_t s) {
+    decode_wait_selftest_kernel<<<1, 32, 0, s>>>(max_polls);
     return cudaGetLastError();
+}
+
+cudaError_t decode_error_word(unsigned *v, bool clear, cudaStream_t s) {
+    return read_error_word(g_decode_err, v, clear, s);
 }
 
 }  // namespace gdn

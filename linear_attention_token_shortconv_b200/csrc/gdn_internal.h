@@ -68,4 +68,36 @@ cudaError_t launch_decode(const DecodeArgs &a);
 bool decode_stream_supported(const DecodeArgs &a);
 cudaError_t launch_decode_stream(const DecodeArgs &a);
 
+// Kernel-launch accounting for gdn_last_call_launches(): every launcher returns
+// launched() right after its <<<...>>>, which counts the launch on this thread.
+void note_launch();
+void reset_launch_count();   // at the entry of every public call that launches
+inline cudaError_t launched() {
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) note_launch();
+    return e;
+}
+
+// Device error words: a kernel family raises its word when one of its bounded
+// waits expires.  *_error_word copies the word to *v (zeroing it when `clear`)
+// and synchronises `s`; *_wait_selftest runs one CTA whose wait -- the family's
+// own wait routine -- targets a barrier phase that nothing completes.
+template <class Sym>
+cudaError_t read_error_word(Sym &sym, unsigned *v, bool clear, cudaStream_t s) {
+    cudaError_t e = cudaMemcpyFromSymbolAsync(v, sym, sizeof(unsigned), 0, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess && clear) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, sym);
+        if (e == cudaSuccess) e = cudaMemsetAsync(p, 0, sizeof(unsigned), s);
+    }
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    return e;
+}
+cudaError_t prep_error_word(unsigned *v, bool clear, cudaStream_t s);
+cudaError_t chain_error_word(unsigned *v, bool clear, cudaStream_t s);
+cudaError_t decode_error_word(unsigned *v, bool clear, cudaStream_t s);
+cudaError_t prep_wait_selftest(uint32_t max_polls, cudaStream_t s);
+cudaError_t chain_wait_selftest(uint32_t max_polls, cudaStream_t s);
+cudaError_t decode_wait_selftest(uint32_t max_polls, cudaStream_t s);
+
 }  // namespace gdn

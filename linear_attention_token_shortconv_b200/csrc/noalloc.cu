@@ -67,6 +67,7 @@ extern "C" gdn_status_t gdn_prefill_noalloc(const gdn_dims_t *dims, const void *
                                             const float *norm_w, const float *S0,
                                             const int32_t *cu_seqlens, void *out, float *S_final,
                                             gdn_stream_t stream) {
+    gdn::reset_launch_count();
     if (!dims) return GDN_ERR_INVALID_ARG;
     const gdn_dims_t &d = *dims;
     if (d.num_seqs <= 0 || d.total_tokens < 0 || d.H <= 0 || d.dk <= 0 || d.dv <= 0 || d.conv_k <= 0)

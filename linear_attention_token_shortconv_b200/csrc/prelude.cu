@@ -111,7 +111,7 @@ cudaError_t launch_prelude_t(const PrefillArgs &a, Tws *qn, Tws *kn, Tws *vn) {
     else if (a.dk == 128 && a.dv == 64) GDN_PRELUDE(128, 64);
     else GDN_PRELUDE(64, 128);
 #undef GDN_PRELUDE
-    return cudaGetLastError();
+    return launched();
 }
 
 cudaError_t launch_prelude_f32(const PrefillArgs &a, float *qn, float *kn, float *vn) {

@@ -136,7 +136,7 @@ static cudaError_t launch_rec_dims(const PrefillArgs &a, const float *qn, const 
         if (a.out_bf16) GDN_REC(float, bf16); else GDN_REC(float, float);
     }
 #undef GDN_REC
-    return cudaGetLastError();
+    return launched();
 }
 
 cudaError_t launch_recurrent(const PrefillArgs &a, const float *qn, const float *kn,

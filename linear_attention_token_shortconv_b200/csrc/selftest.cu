@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/gdn_selftest.h"
+#include "gdn_internal.h"
 #include "umma.cuh"
 
 namespace gdn {
@@ -129,4 +130,18 @@ extern "C" gdn_status_t gdn_selftest_umma(int a_mn, int b_mn, int negate_a, int 
         return GDN_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return GDN_ERR_CUDA;
     return err ? GDN_ERR_TIMEOUT : GDN_OK;
+}
+
+extern "C" gdn_status_t gdn_selftest_wait_timeout(unsigned family, unsigned max_polls,
+                                                  gdn_stream_t stream) {
+    if (max_polls < 1 || max_polls > 65536) return GDN_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    switch (family) {
+    case GDN_ERRF_PREP: e = gdn::prep_wait_selftest(max_polls, s); break;
+    case GDN_ERRF_CHAIN: e = gdn::chain_wait_selftest(max_polls, s); break;
+    case GDN_ERRF_DECODE: e = gdn::decode_wait_selftest(max_polls, s); break;
+    default: return GDN_ERR_INVALID_ARG;
+    }
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }

@@ -22,7 +22,10 @@ STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "G
 
 # Every function the header declares (checked by the tests).
 EXPORTS = ("gdn_prefill", "gdn_prefill_workspace_size", "gdn_decode_step", "gdn_status_string",
-           "gdn_set_timing_events", "gdn_selftest_umma", "gdn_prefill_noalloc")
+           "gdn_set_timing_events", "gdn_selftest_umma", "gdn_prefill_noalloc",
+           "gdn_set_kernel_events", "gdn_last_call_launches", "gdn_device_error_status",
+           "gdn_selftest_wait_timeout")
+ERRF_PREP, ERRF_CHAIN, ERRF_DECODE = 1, 2, 4
 
 
 class GdnError(RuntimeError):
@@ -62,6 +65,14 @@ def load() -> ctypes.CDLL:
         lib.gdn_selftest_umma.restype = ctypes.c_int
         lib.gdn_set_timing_events.argtypes = [P, P]
         lib.gdn_set_timing_events.restype = ctypes.c_int
+        lib.gdn_set_kernel_events.argtypes = [ctypes.POINTER(P), ctypes.POINTER(P), ctypes.c_int]
+        lib.gdn_set_kernel_events.restype = ctypes.c_int
+        lib.gdn_last_call_launches.argtypes = []
+        lib.gdn_last_call_launches.restype = ctypes.c_int
+        lib.gdn_device_error_status.argtypes = [ctypes.POINTER(ctypes.c_uint), ctypes.c_int, P]
+        lib.gdn_device_error_status.restype = ctypes.c_int
+        lib.gdn_selftest_wait_timeout.argtypes = [ctypes.c_uint, ctypes.c_uint, P]
+        lib.gdn_selftest_wait_timeout.restype = ctypes.c_int
         lib.gdn_status_string.argtypes = [ctypes.c_int]
         lib.gdn_status_string.restype = ctypes.c_char_p
         _lib = lib
@@ -180,6 +191,42 @@ def set_timing_events(begin=None, end=None):
     b = None if begin is None else ctypes.c_void_p(begin.cuda_event)
     e = None if end is None else ctypes.c_void_p(end.cuda_event)
     _check(load().gdn_set_timing_events(b, e), "gdn_set_timing_events")
+
+
+def set_kernel_events(begins=(), ends=()):
+    """Record torch.cuda.Event begins[i] / ends[i] around launch slot i of each
+    following call (slot order: prep/chain per segment for a prefill, the
+    kernel for a decode step); empty sequences clear the hook.  The events must
+    have been recorded once so that their CUDA handles exist."""
+    if len(begins) != len(ends):
+        raise ValueError("begins and ends differ in length")
+    n = len(begins)
+    arr = ctypes.c_void_p * max(n, 1)
+    b = arr(*[e.cuda_event for e in begins])
+    e = arr(*[x.cuda_event for x in ends])
+    _check(load().gdn_set_kernel_events(b, e, n), "gdn_set_kernel_events")
+
+
+def last_call_launches() -> int:
+    """Kernels launched by this thread's most recent prefill / decode call."""
+    return int(load().gdn_last_call_launches())
+
+
+def device_error_status(clear=False, stream=None):
+    """(status, flags): the current device's error words as a GDN_ERRF_* mask
+    after the work queued on `stream`; status is GDN_ERR_TIMEOUT (5) when any
+    flag is set.  Clears the words when `clear`."""
+    flags = ctypes.c_uint(0)
+    st = load().gdn_device_error_status(ctypes.byref(flags), int(bool(clear)), _stream(stream))
+    if st not in (0, 5):
+        raise GdnError(st, "gdn_device_error_status")
+    return st, flags.value
+
+
+def selftest_wait_timeout(family, max_polls=1024, stream=None):
+    """Launch one CTA whose bounded wait (kernel family `family`) runs out."""
+    _check(load().gdn_selftest_wait_timeout(family, max_polls, _stream(stream)),
+           "gdn_selftest_wait_timeout")
 
 
 def selftest_umma(A, B, init=None, *, a_mn=False, b_mn=False, negate_a=False, stream=None):

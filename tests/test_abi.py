@@ -98,3 +98,28 @@ def test_workspace_size_query(lib):
     assert gdn.prefill_workspace_size(1, 0, 1, 64, 64) == 0
     with pytest.raises(gdn.GdnError):
         gdn.prefill_workspace_size(1, 10, 1, 48, 64)
+
+
+def test_kernel_events_hook_validation(lib):
+    P = ctypes.c_void_p
+    two = (P * 2)(P(16), P(32))
+    assert lib.gdn_set_kernel_events(two, two, -1) == 1
+    assert lib.gdn_set_kernel_events(None, two, 1) == 1
+    holes = (P * 2)(P(16), None)
+    assert lib.gdn_set_kernel_events(two, holes, 2) == 1
+    assert lib.gdn_set_kernel_events(None, None, 0) == 0     # clears the hook
+
+
+def test_rejected_calls_launch_nothing(lib):
+    assert _prefill(lib, _dims(dk=96), _args()) == 2
+    assert lib.gdn_last_call_launches() == 0
+    args = [FAKE[i] for i in range(11)] + [ctypes.c_void_p(8192), ctypes.c_void_p(12288), None]
+    assert lib.gdn_decode_step(ctypes.byref(_dims(num_seqs=4, total_tokens=5)), *args) == 1
+    assert lib.gdn_last_call_launches() == 0
+
+
+def test_wait_selftest_validation(lib):
+    assert lib.gdn_selftest_wait_timeout(8, 16, None) == 1       # not a family bit
+    assert lib.gdn_selftest_wait_timeout(3, 16, None) == 1       # two bits
+    assert lib.gdn_selftest_wait_timeout(1, 0, None) == 1
+    assert lib.gdn_selftest_wait_timeout(1, 65537, None) == 1

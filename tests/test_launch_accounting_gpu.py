@@ -1,0 +1,56 @@
+"""Launch accounting through the C ABI: gdn_last_call_launches() counts the
+kernels a call launched, and gdn_set_kernel_events() brackets each launch slot
+with the caller's events (the hooks bench.py uses for its per-kernel timing)."""
+import pytest
+import torch
+
+from harness import gpu_prefill, to_device
+from linear_attention_token_shortconv_b200 import gdn
+from linear_attention_token_shortconv_b200.workloads import (DECODE, PRETRAIN, make_decode_inputs,
+                                                             make_prefill_inputs, scaled)
+
+pytestmark = pytest.mark.gpu
+
+
+def _events(n):
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    for e in ev:
+        e.record()
+    torch.cuda.synchronize()
+    return ev
+
+
+@pytest.mark.parametrize("tokens,segments", [(320, 1), (1280, 3)])
+def test_prefill_launch_slots(cuda_device, tokens, segments):
+    # segments hold at least 8 chunks of 64 tokens: 5 chunks run as one
+    # prep + chain pair, 20 chunks as three segments (8, 8, 4 chunks)
+    cfg = scaled(PRETRAIN, lengths=(tokens,), H=2)
+    inp = to_device(make_prefill_inputs(cfg, "cpu"), cuda_device)
+    n_slots = 2 * segments + 2
+    b, e = _events(n_slots), _events(n_slots)
+    gdn.set_kernel_events(b, e)
+    try:
+        gpu_prefill(inp, 1)
+    finally:
+        gdn.set_kernel_events()
+    launched = gdn.last_call_launches()
+    assert launched == 2 * segments
+    torch.cuda.synchronize()
+    for i in range(launched):
+        assert b[i].elapsed_time(e[i]) > 0.0, i
+
+
+def test_decode_launch_slot(cuda_device):
+    from dataclasses import replace
+    cfg = replace(DECODE, B=4, H=2)
+    g = to_device(make_decode_inputs(cfg, "cpu"), cuda_device)
+    b, e = _events(1), _events(1)
+    gdn.set_kernel_events(b, e)
+    try:
+        gdn.decode_step(g["q"][0], g["k"][0], g["v"][0], g["conv_w"], g["ring"], g["a_logit"][0],
+                        g["b_logit"][0], g["A"], g["b_alpha"], g["z"][0], g["norm_w"], g["S"])
+    finally:
+        gdn.set_kernel_events()
+    assert gdn.last_call_launches() == 1
+    torch.cuda.synchronize()
+    assert b[0].elapsed_time(e[0]) > 0.0
