@@ -78,59 +78,105 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples every 200 ms during a region."""
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock, power and clock-event (throttle) reasons sampled during a
+    region: NVML polled every 5 ms from a thread (the counters nvidia-smi
+    prints), else nvidia-smi every 200 ms.  Read-only: no setting is changed."""
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
+    SMI_FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, index):
         self.index = index
-        self.proc = None
-        self.path = None
+        self.rows = []          # (sm_mhz, max_mhz, watts, set of reason names)
+        self.source = None
+        self._stop = None
+        self._thread = None
+        self._proc = None
+        self._path = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            p = torch.cuda.get_device_properties(self.index)
+            bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.index)
+
+    def _poll(self, nv, h):
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                w = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                r = get_reasons(h)
+                self.rows.append((float(sm), float(mx), w,
+                                  {n for bit, n in self.REASONS.items() if r & bit}))
+            except Exception:
+                break
+            self._stop.wait(0.005)
 
     def __enter__(self):
+        import threading
         try:
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            nv, h = self._nvml_handle()
+            self._stop = threading.Event()
+            self._thread = threading.Thread(target=self._poll, args=(nv, h), daemon=True)
+            self._thread.start()
+            self.source = "nvml 5 ms"
+            return self
+        except Exception:
+            pass
+        try:
+            fd, self._path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
-            self.fh = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.fh,
+            self._fh = open(self._path, "w")
+            self._proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.SMI_FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self._fh,
                 stderr=subprocess.DEVNULL)
             time.sleep(0.3)
+            self.source = "nvidia-smi 200 ms"
         except (OSError, ValueError):
-            self.proc = None
+            self._proc = None
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
+        if self._proc is not None:
+            self._proc.terminate()
             try:
-                self.proc.wait(timeout=5)
+                self._proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
-                self.proc.kill()
-            self.fh.close()
+                self._proc.kill()
+            self._fh.close()
+            names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+            for line in open(self._path):
+                parts = [p.strip() for p in line.split(",")]
+                try:
+                    self.rows.append((float(parts[0]), float(parts[1]), float(parts[2]),
+                                      {names[i] for i, v in enumerate(parts[4:8]) if v == "Active"}))
+                except (ValueError, IndexError):
+                    continue
+            os.unlink(self._path)
 
     def summary(self):
-        if self.proc is None or not self.path:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        rows = []
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 8:
-                continue
-            try:
-                rows.append((float(parts[0]), float(parts[1]), float(parts[2]), parts[4:8]))
-            except ValueError:
-                continue
-        os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3]) if v == "Active"})
-        loaded = [r[0] for r in rows if r[2] > 200.0] or [r[0] for r in rows]
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(r[1] for r in rows),
-                "power_w_max": max(r[2] for r in rows), "samples": len(rows), "reasons": reasons}
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None,
+                    "reasons": ["no samples" if self.source else "no clock source"]}
+        reasons = sorted(set().union(*(r[3] for r in self.rows)))
+        return {"sm_mhz": statistics.median(r[0] for r in self.rows),
+                "sm_max_mhz": max(r[1] for r in self.rows),
+                "sm_mhz_min": min(r[0] for r in self.rows),
+                "power_w_max": max(r[2] for r in self.rows), "samples": len(self.rows),
+                "source": self.source, "reasons": reasons}
 
 
 def dist_setup():
@@ -271,18 +317,19 @@ def bench_decode(cfg, steps, dev):
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     launches = 0
-    start.record()
-    for t in range(steps):
-        gdn.set_timing_events(evb[t], eve[t])
-        step(t)
-        launches += gdn.last_call_launches()
-    end.record()
-    gdn.set_timing_events(None, None)
-    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        start.record()
+        for t in range(steps):
+            gdn.set_timing_events(evb[t], eve[t])
+            step(t)
+            launches += gdn.last_call_launches()
+        end.record()
+        gdn.set_timing_events(None, None)
+        torch.cuda.synchronize()
     ms = start.elapsed_time(end) / steps
     kern_ms = sum(b.elapsed_time(e) for b, e in zip(evb, eve)) / steps
     state_bytes = 2 * cfg.B * cfg.H * cfg.dk * cfg.dv * 4
-    return ms, kern_ms, state_bytes, launches
+    return ms, kern_ms, state_bytes, launches, clk.summary()
 
 
 def oracle_sample_rate(inp, cfg, tokens, heads, n_threads):
@@ -396,13 +443,13 @@ def main():
     torch.cuda.empty_cache()
 
     if rank == 0 and args.decode_steps > 0:
-        dms, dk_ms, sbytes, dlaunch = bench_decode(DECODE, args.decode_steps, dev)
+        dms, dk_ms, sbytes, dlaunch, dclk = bench_decode(DECODE, args.decode_steps, dev)
         gbs = sbytes / (dk_ms * 1e-3) / 1e9
         result["decode"] = {"workload": DECODE.name, "steps": args.decode_steps,
                             "ms_per_step": dms, "kernel_ms": dk_ms,
                             "state_gbs": gbs, "peak_gbs": pk["hbm_gbs"],
                             "frac": gbs / pk["hbm_gbs"], "state_bytes_per_step": sbytes,
-                            "kernel": "decode_stream", "gpu_launches": dlaunch}
+                            "kernel": "decode_stream", "gpu_launches": dlaunch, "clocks": dclk}
         torch.cuda.empty_cache()
 
     if not args.no_e2e:

@@ -102,10 +102,12 @@ typedef struct {
  *
  * Each sequence starts with an empty conv history.  `out` must not alias any
  * input.  On the tensor-core path (bf16 inputs, dk = 128) long inputs run in
- * chunk segments whose kernels overlap on `stream` and on a library-owned
- * second stream of the same device, forked from and joined back into `stream`
- * with events, so work queued on `stream` afterwards sees the results.  When total_tokens is 0 the token tensors (q, k, v, z, a_logit,
- * b_logit, out) may be NULL and the call only writes S_final = S0 (or zeros).  The call takes a stream-ordered workspace of
+ * chunk segments whose kernels overlap on `stream` and on two library-owned
+ * streams of the same device, forked from and joined back into `stream` with
+ * events, so work queued on `stream` afterwards sees the results.  When
+ * total_tokens is 0 the token tensors (q, k, v, z, a_logit, b_logit, out) may
+ * be NULL and the call only writes S_final = S0 (or zeros).  The call takes a
+ * stream-ordered workspace of
  * gdn_prefill_workspace_size() bytes from a private CUDA memory pool of the
  * current device and returns it to the pool on the same stream.
  */
@@ -192,8 +194,9 @@ GDN_API gdn_status_t gdn_set_timing_events(void *begin, void *end);
  * slot i of every following gdn_prefill / gdn_decode_step call, on the stream
  * that slot's kernel runs on.  Slots in launch order:
  *   gdn_prefill, tensor-core path, n segments: chunk_prep(0), chunk_chain(0),
- *     chunk_prep(1), chunk_chain(1), ... -- chunk_prep on the caller's stream,
- *     chunk_chain on the library's side stream of the device;
+ *     chunk_prep(1), chunk_chain(1), ... -- chunk_prep of even segments on the
+ *     caller's stream, of odd segments on a second library stream, chunk_chain
+ *     on the library's highest-priority stream of the device;
  *   gdn_prefill, fp32 path: prelude, recurrent;
  *   gdn_decode_step: the decode kernel.
  * Slots beyond n are not recorded.  n = 0 clears the hook.  Returns

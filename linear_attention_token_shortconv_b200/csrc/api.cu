@@ -41,10 +41,12 @@ size_t round_up(size_t x) { return (x + 255) & ~(size_t)255; }
 // else (the fp32 workload, dk = 64) runs the fp32 token-by-token recurrence.
 bool use_tensor_cores(const gdn_dims_t *d) { return d->in_dtype == GDN_BF16 && d->dk == 128; }
 
-// Chunk segments of the tensor-core path: the prep kernel of segment s + 1 runs
-// on the caller's stream while the chain kernel of segment s runs on a second,
-// higher-priority stream; segments are ordered by events, and the state passes
-// from one chain launch to the next through a state buffer.
+// Chunk segments of the tensor-core path.  Prep segments are independent of one
+// another (each writes its own token rows of the workspace): they alternate
+// between the caller's stream and a second stream, so segment s + 1 fills the
+// SMs that segment s's last CTAs leave idle.  The chain kernel of segment s runs
+// on a third, highest-priority stream after prep s and chain s - 1 (events);
+// the state passes from one chain launch to the next through a state buffer.
 struct Segments {
     int seg, n;
 };
@@ -96,9 +98,11 @@ cudaError_t get_pool(cudaMemPool_t *pool) {
     return cudaSuccess;
 }
 
-// Per-device side stream (highest priority) and event pool for the segments.
+// Per-device side streams (chain: highest priority; prep2: default priority)
+// and event pool for the segments.
 struct SideStream {
     cudaStream_t stream = nullptr;
+    cudaStream_t prep2 = nullptr;
     std::vector<cudaEvent_t> events;
 };
 std::mutex g_side_mu[64];
@@ -114,6 +118,9 @@ cudaError_t side_stream(int dev, int n, SideStream **out) {
         if ((e = cudaDeviceGetStreamPriorityRange(&lo, &hi)) != cudaSuccess) return e;
         if ((e = cudaStreamCreateWithPriority(&ss.stream, cudaStreamNonBlocking, hi)) != cudaSuccess)
             return e;
+    }
+    if (!ss.prep2) {
+        if ((e = cudaStreamCreateWithFlags(&ss.prep2, cudaStreamNonBlocking)) != cudaSuccess) return e;
     }
     while ((int)ss.events.size() < n) {
         cudaEvent_t ev;
@@ -295,14 +302,15 @@ gdn_status_t gdn_prefill(const gdn_dims_t *dims, const void *q, const void *k, c
                 std::lock_guard<std::mutex> lock(g_side_mu[dev]);
                 SideStream *ss = nullptr;
                 e = side_stream(dev, g.n + 2, &ss);
-                // fork: the side stream starts after the caller's prior work
+                // fork: the side streams start after the caller's prior work
                 if (e == cudaSuccess) e = cudaEventRecord(ss->events[g.n], a.stream);
                 if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->stream, ss->events[g.n], 0);
+                if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->prep2, ss->events[g.n], 0);
                 for (int sgi = 0; sgi < g.n && e == cudaSuccess; ++sgi) {
                     const int c_lo = sgi * g.seg, c_hi = c_lo + g.seg;
-                    e = slot_launch(&slot, a.stream,
-                                    [&] { return gdn::launch_chunk_prep(a, w, c_lo, c_hi, a.stream); });
-                    if (e == cudaSuccess) e = cudaEventRecord(ss->events[sgi], a.stream);
+                    cudaStream_t ps = (sgi & 1) ? ss->prep2 : a.stream;
+                    e = slot_launch(&slot, ps, [&] { return gdn::launch_chunk_prep(a, w, c_lo, c_hi, ps); });
+                    if (e == cudaSuccess) e = cudaEventRecord(ss->events[sgi], ps);
                     if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->stream, ss->events[sgi], 0);
                     const float *sin = sgi == 0 ? a.S0 : state;
                     float *sout = sgi == g.n - 1 ? a.S_final : state;
@@ -311,6 +319,8 @@ gdn_status_t gdn_prefill(const gdn_dims_t *dims, const void *q, const void *k, c
                             return gdn::launch_chunk_chain(a, w, c_lo, c_hi, sin, sout, ss->stream);
                         });
                 }
+                // every prep launch precedes a chain launch on the chain stream, so
+                // joining the chain stream joins all of the call's work
                 // join: the caller's stream continues after the last chain launch
                 if (e == cudaSuccess) e = cudaEventRecord(ss->events[g.n + 1], ss->stream);
                 if (e == cudaSuccess) e = cudaStreamWaitEvent(a.stream, ss->events[g.n + 1], 0);
