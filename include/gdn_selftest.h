@@ -20,8 +20,10 @@ extern "C" {
  *   B     [K, N]   fp16 row-major, device      (N in {64, 128})
  *   init  [128, N] fp32 device or NULL (then D = +/-A*B)
  *   D     [128, N] fp32 device, written
- *   a_mn, b_mn  stage A / B MN-major (1) or K-major (0) in shared memory
- *   negate_a    use -A
+ *   a_mn        A in shared memory MN-major (1) or K-major (0), or in tensor
+ *               memory (2: row m in lane m, elements 2c, 2c+1 in column c)
+ *   b_mn        B in shared memory MN-major (1) or K-major (0)
+ *   negate_a    use -A (A in shared memory only)
  *
  * Synchronises `stream`.  Returns GDN_ERR_TIMEOUT if the MMA completion wait
  * expired, GDN_ERR_INVALID_ARG for unsupported sizes or NULL buffers.

@@ -1,6 +1,7 @@
 // Self-test of the tcgen05 operand layouts the GDN kernels rely on: one CTA
 // stages A [128 x K] and B [K x N] (fp16, row-major in global memory) into
-// shared memory in the requested K-major or MN-major 128-byte-swizzled layout,
+// shared memory in the requested K-major or MN-major 128-byte-swizzled layout
+// (A alternatively into tensor memory, row m in lane m, K pairs per column),
 // runs K/16 tcgen05.mma (kind::f16, fp32 accumulation in TMEM, optionally onto
 // an initial value written with tcgen05.st, optionally with A negated) and
 // writes D [128 x N] back.  The host compares D with a plain matmul.
@@ -31,7 +32,7 @@ umma_selftest_kernel(int a_mn, int b_mn, int neg_a, int N, int K, const __half *
     uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + kStMisc + 16);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-    if (warp == 0) umma::tmem_alloc(tslot, 128);
+    if (warp == 0) umma::tmem_alloc(tslot, 256);
     if (tid == 0) {
         umma::mbar_init(bar, 1);
         umma::fence_mbar_init();
@@ -40,7 +41,8 @@ umma_selftest_kernel(int a_mn, int b_mn, int neg_a, int N, int K, const __half *
     for (int idx = tid; idx < 128 * K / 8; idx += 128) {
         const int m = idx / (K / 8), k8 = idx % (K / 8);
         const uint4 v = reinterpret_cast<const uint4 *>(A + (size_t)m * K)[k8];
-        if (!a_mn) {          // K-major: k-block k/64, row m
+        if (a_mn == 2) {      // tensor memory: staged after the allocation below
+        } else if (!a_mn) {   // K-major: k-block k/64, row m
             umma::st_chunk(As + (k8 / 8) * 16384, m, k8 % 8, v);
         } else {              // MN-major: rows = k, mn-block m/64 -- scatter the 8 k values
             const __half *hv = reinterpret_cast<const __half *>(&v);
@@ -68,6 +70,18 @@ umma_selftest_kernel(int a_mn, int b_mn, int neg_a, int N, int K, const __half *
     __syncthreads();
     const uint32_t tbase = *tslot;
     const uint32_t trow = tbase + ((uint32_t)(warp * 32) << 16);
+    if (a_mn == 2) {          // A rows into lanes, K pairs into columns [128, 128 + K/2)
+        const int m = warp * 32 + lane;
+        for (int c0 = 0; c0 < K / 2; c0 += 32) {
+            float v[32];
+            for (int j = 0; j < 32; ++j) {
+                const __half2 h2 = *reinterpret_cast<const __half2 *>(A + (size_t)m * K + 2 * (c0 + j));
+                v[j] = __uint_as_float(*reinterpret_cast<const uint32_t *>(&h2));
+            }
+            umma::tmem_st32(trow + 128 + c0, v);
+        }
+        umma::tmem_st_wait();
+    }
     if (init) {
         for (int c = 0; c < N; c += 32) {
             float v[32];
@@ -81,15 +95,16 @@ umma_selftest_kernel(int a_mn, int b_mn, int neg_a, int N, int K, const __half *
     __syncthreads();
     if (tid == 0) {
         umma::tc_fence_after();
-        const uint32_t idesc = umma::idesc_f16(128, N, a_mn != 0, b_mn != 0, neg_a != 0);
+        const uint32_t idesc = umma::idesc_f16(128, N, a_mn == 1, b_mn != 0, neg_a != 0);   // A from TMEM: K-major only
         const uint32_t a0 = umma::smem_u32(As), b0 = umma::smem_u32(Bs);
         for (int s = 0; s < K / 16; ++s) {
-            uint64_t ad, bd;
-            if (!a_mn) ad = umma::sw128_desc(a0 + (s / 4) * 16384 + (s % 4) * 32, 16, 1024);
-            else       ad = umma::sw128_desc(a0 + s * 2048, K * 128, 1024);
+            uint64_t ad = 0, bd;
+            if (a_mn == 0)      ad = umma::sw128_desc(a0 + (s / 4) * 16384 + (s % 4) * 32, 16, 1024);
+            else if (a_mn == 1) ad = umma::sw128_desc(a0 + s * 2048, K * 128, 1024);
             if (b_mn)  bd = umma::sw128_desc(b0 + s * 2048, K * 128, 1024);
             else       bd = umma::sw128_desc(b0 + (s / 4) * (N * 128) + (s % 4) * 32, 16, 1024);
-            umma::mma_f16(tbase, ad, bd, idesc, (s > 0 || init) ? 1u : 0u);
+            if (a_mn == 2) umma::mma_f16_ts(tbase, tbase + 128 + s * 8, bd, idesc, (s > 0 || init) ? 1u : 0u);
+            else           umma::mma_f16(tbase, ad, bd, idesc, (s > 0 || init) ? 1u : 0u);
         }
         umma::mma_commit(bar);
     }
@@ -106,7 +121,7 @@ umma_selftest_kernel(int a_mn, int b_mn, int neg_a, int N, int K, const __half *
     }
     umma::tc_fence_before();
     __syncthreads();
-    if (warp == 0) umma::tmem_dealloc(tbase, 128);
+    if (warp == 0) umma::tmem_dealloc(tbase, 256);
 }
 
 }  // namespace gdn
@@ -115,6 +130,7 @@ extern "C" gdn_status_t gdn_selftest_umma(int a_mn, int b_mn, int negate_a, int 
                                           const void *A, const void *B, const float *init,
                                           float *D, gdn_stream_t stream) {
     if ((N != 64 && N != 128) || (K != 64 && K != 128) || !A || !B || !D) return GDN_ERR_INVALID_ARG;
+    if (a_mn < 0 || a_mn > 2 || (a_mn == 2 && negate_a)) return GDN_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     unsigned int zero = 0, err = 0;
     if (cudaMemcpyToSymbolAsync(gdn::g_selftest_err, &zero, sizeof zero, 0, cudaMemcpyHostToDevice, s) != cudaSuccess)

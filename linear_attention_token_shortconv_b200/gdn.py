@@ -230,8 +230,9 @@ def selftest_wait_timeout(family, max_polls=1024, stream=None):
 
 
 def selftest_umma(A, B, init=None, *, a_mn=False, b_mn=False, negate_a=False, stream=None):
-    """D = init + (+/-A) B computed on the tensor cores with the given shared-memory
-    operand layouts (A [128,K], B [K,N] fp16 CUDA tensors)."""
+    """D = init + (+/-A) B computed on the tensor cores with the given operand
+    layouts (A [128,K], B [K,N] fp16 CUDA tensors): a_mn 0 / 1 = A K-major /
+    MN-major in shared memory, 2 = A in tensor memory; b_mn likewise for B."""
     M, K = A.shape
     N = B.shape[1]
     if M != 128 or B.shape[0] != K or A.dtype != torch.float16 or B.dtype != torch.float16:
