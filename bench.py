@@ -41,10 +41,14 @@ METRIC = "GDN prefill tokens/s at T=32K H=32 (% TC peak); decode state GB/s (% H
 # logits and a bf16 output.
 PREFILL_FLOP_PER_TOKEN_HEAD = 64 * (6 * 128 + 4 * 128) + 6 * 128 * 128   # 180,224
 PREFILL_BYTES_PER_TOKEN_HEAD = 4 * 128 * 2 + 2 * 2 + 128 * 2           # 1,284
-# ... of which each kernel of the two-kernel split touches: chunk_prep reads
-# q, k, v and the two logits; chunk_chain reads z and writes the output.
-KERNEL_BYTES_PER_TOKEN_HEAD = {"chunk_prep": 3 * 128 * 2 + 2 * 2,          # 772
-                               "chunk_chain": 128 * 2 + 128 * 2}           # 512
+# Per-kernel roofline units.  chunk_prep reads q, k, v and the two logits: 772 of
+# the 1,284 B above; the rest (z in, the output out) belongs to chunk_chain, whose
+# algorithmic work is, though, the state-dependent MMAs of the chunk form:
+# 2 C dk dv (U) + 2 C dk dv (Q S) + 2 C^2 dv (Aqk U) + 2 C dk dv (S update) per
+# chunk = 114,688 flop per token-head (chunk_prep's state-independent MMAs are the
+# other 65,536 of the 180,224 above).  Each kernel is reported against its bound.
+KERNEL_ROOFLINE = {"chunk_prep": ("hbm", 3 * 128 * 2 + 2 * 2),                      # 772 B
+                   "chunk_chain": ("tensor", 3 * 2 * 128 * 128 + 2 * 64 * 128)}        # 114,688 flop
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per token-head from
 # an ncu capture of each kernel, valid only while the kernel's source is the one
 # captured (sha1 of the .cu file); otherwise the JSON reports traffic null.
@@ -245,11 +249,12 @@ def bench_prefill(cfg, steps, warmup, world, rank, dev):
     barrier(world)
     ms = max_over_ranks(start.elapsed_time(end) / steps, world)
     kern_ms = max_over_ranks(sum(b.elapsed_time(e) for b, e in zip(evb, eve)) / steps, world)
-    # slots alternate chunk_prep (even) and chunk_chain (odd)
-    per = {"chunk_prep": [], "chunk_chain": []}
+    # launch slots per segment: chunk_prep, chunk_chain
+    names = ("chunk_prep", "chunk_chain")
+    per = {n: [] for n in names}
     for i in range(steps):
         for j in range(n_launch):
-            per["chunk_prep" if j % 2 == 0 else "chunk_chain"].append(kb[i][j].elapsed_time(ke[i][j]))
+            per[names[j % 2]].append(kb[i][j].elapsed_time(ke[i][j]))
     kernels = {}
     for name, xs in per.items():
         kernels[name] = {"launches_per_step": len(xs) // steps,
@@ -413,8 +418,18 @@ def main():
     dom = max(kernels, key=lambda n: kernels[n]["ms_per_step"])
     kd = kernels[dom]
     units_per_launch = token_heads / kd["launches_per_step"]
-    dom_gbs = KERNEL_BYTES_PER_TOKEN_HEAD[dom] * units_per_launch / (kd["avg_launch_ms"] * 1e-3) / 1e9
+    bound, per_unit = KERNEL_ROOFLINE[dom]
+    rate = per_unit * units_per_launch / (kd["avg_launch_ms"] * 1e-3)
+    if bound == "hbm":
+        dom_ach, dom_peak, dom_unit = rate / 1e9, pk["hbm_gbs"], "GB/s"
+    else:
+        dom_ach, dom_peak, dom_unit = rate / 1e12, pk["bf16_tflops"], "TFLOP/s"
     traffic = kernel_traffic(dom, units_per_launch)
+    for name, rec in kernels.items():   # every kernel against its own bound, for context
+        b_, u_ = KERNEL_ROOFLINE[name]
+        r_ = u_ * (token_heads / rec["launches_per_step"]) / (rec["avg_launch_ms"] * 1e-3)
+        rec["bound"] = b_
+        rec["frac"] = r_ / 1e9 / pk["hbm_gbs"] if b_ == "hbm" else r_ / 1e12 / pk["bf16_tflops"]
 
     result = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -424,9 +439,9 @@ def main():
                                "fp32 state, S0~N(0,0.02), per GPU",
                    "global_batch": world, "seq_len": cfg.total_tokens, "parallelism": f"dp{world}",
                    "l2": "inputs larger than L2 (1.07 GB of bf16 q,k,v,z read per step)"},
-        "roofline": {"bound": "hbm", "achieved": dom_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                     "frac": dom_gbs / pk["hbm_gbs"], "traffic": traffic, "kernel": dom,
-                     "bytes_per_token_head": KERNEL_BYTES_PER_TOKEN_HEAD[dom],
+        "roofline": {"bound": bound, "achieved": dom_ach, "peak": dom_peak, "unit": dom_unit,
+                     "frac": dom_ach / dom_peak, "traffic": traffic, "kernel": dom,
+                     ("bytes_per_token_head" if bound == "hbm" else "flop_per_token_head"): per_unit,
                      "token_heads_per_launch": units_per_launch,
                      "avg_launch_ms": kd["avg_launch_ms"], "peak_kind": pk_kind,
                      "kernels": kernels,
