@@ -53,7 +53,7 @@ struct Segments {
 Segments segments(const gdn_dims_t *d) {
     const int max_chunks = (d->total_tokens + 63) / 64;
     Segments g;
-    g.seg = max(8, (max_chunks + 23) / 24);
+    g.seg = max(8, (max_chunks + 15) / 16);
     g.n = max(1, (max_chunks + g.seg - 1) / g.seg);
     return g;
 }
