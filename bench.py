@@ -41,14 +41,18 @@ METRIC = "GDN prefill tokens/s at T=32K H=32 (% TC peak); decode state GB/s (% H
 # logits and a bf16 output.
 PREFILL_FLOP_PER_TOKEN_HEAD = 64 * (6 * 128 + 4 * 128) + 6 * 128 * 128   # 180,224
 PREFILL_BYTES_PER_TOKEN_HEAD = 4 * 128 * 2 + 2 * 2 + 128 * 2           # 1,284
-# Per-kernel roofline units.  chunk_prep reads q, k, v and the two logits: 772 of
+# Per-kernel roofline units (a few (sequence, head) chains run as one fused
+# persistent kernel; many chains as chunk_prep / chunk_chain launches per
+# segment).  chunk_prep reads q, k, v and the two logits: 772 of
 # the 1,284 B above; the rest (z in, the output out) belongs to chunk_chain, whose
 # algorithmic work is, though, the state-dependent MMAs of the chunk form:
 # 2 C dk dv (U) + 2 C dk dv (Q S) + 2 C^2 dv (Aqk U) + 2 C dk dv (S update) per
 # chunk = 114,688 flop per token-head (chunk_prep's state-independent MMAs are the
 # other 65,536 of the 180,224 above).  Each kernel is reported against its bound.
 KERNEL_ROOFLINE = {"chunk_prep": ("hbm", 3 * 128 * 2 + 2 * 2),                      # 772 B
-                   "chunk_chain": ("tensor", 3 * 2 * 128 * 128 + 2 * 64 * 128)}        # 114,688 flop
+                   "chunk_chain": ("tensor", 3 * 2 * 128 * 128 + 2 * 64 * 128),        # 114,688 flop
+                   # both in one persistent launch: the whole pass's 1,284 B
+                   "prefill_fused": ("hbm", PREFILL_BYTES_PER_TOKEN_HEAD)}
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per token-head from
 # an ncu capture of each kernel, valid only while the kernel's source is the one
 # captured (sha1 of the .cu file); otherwise the JSON reports traffic null.
@@ -249,12 +253,12 @@ def bench_prefill(cfg, steps, warmup, world, rank, dev):
     barrier(world)
     ms = max_over_ranks(start.elapsed_time(end) / steps, world)
     kern_ms = max_over_ranks(sum(b.elapsed_time(e) for b, e in zip(evb, eve)) / steps, world)
-    # launch slots per segment: chunk_prep, chunk_chain
-    names = ("chunk_prep", "chunk_chain")
+    # launch slots: one fused persistent kernel, or chunk_prep / chunk_chain per segment
+    names = ("prefill_fused",) if n_launch == 1 else ("chunk_prep", "chunk_chain")
     per = {n: [] for n in names}
     for i in range(steps):
         for j in range(n_launch):
-            per[names[j % 2]].append(kb[i][j].elapsed_time(ke[i][j]))
+            per[names[j % len(names)]].append(kb[i][j].elapsed_time(ke[i][j]))
     kernels = {}
     for name, xs in per.items():
         kernels[name] = {"launches_per_step": len(xs) // steps,

@@ -101,10 +101,12 @@ typedef struct {
  *              may be NULL when not wanted)
  *
  * Each sequence starts with an empty conv history.  `out` must not alias any
- * input.  On the tensor-core path (bf16 inputs, dk = 128) long inputs run in
- * chunk segments whose kernels overlap on `stream` and on two library-owned
- * streams of the same device, forked from and joined back into `stream` with
- * events, so work queued on `stream` afterwards sees the results.  When
+ * input.  On the tensor-core path (bf16 inputs, dk = 128) a call with
+ * dk = dv = 128 and at most SMs / 4 (sequence, head) pairs runs as one
+ * cooperative persistent kernel on `stream` (one CTA per SM); other long inputs
+ * run in chunk segments whose kernels overlap on `stream` and on two
+ * library-owned streams of the same device, forked from and joined back into
+ * `stream` with events, so work queued on `stream` afterwards sees the results.  When
  * total_tokens is 0 the token tensors (q, k, v, z, a_logit, b_logit, out) may
  * be NULL and the call only writes S_final = S0 (or zeros).  The call takes a
  * stream-ordered workspace of
@@ -193,10 +195,13 @@ GDN_API gdn_status_t gdn_set_timing_events(void *begin, void *end);
  * the caller; the library copies the n handles) are recorded around launch
  * slot i of every following gdn_prefill / gdn_decode_step call, on the stream
  * that slot's kernel runs on.  Slots in launch order:
- *   gdn_prefill, tensor-core path, n segments: chunk_prep(0), chunk_chain(0),
- *     chunk_prep(1), chunk_chain(1), ... -- chunk_prep of even segments on the
- *     caller's stream, of odd segments on a second library stream, chunk_chain
- *     on the library's highest-priority stream of the device;
+ *   gdn_prefill, tensor-core path with dk = dv = 128 and at most a quarter as
+ *     many (sequence, head) pairs as the device has SMs: one slot, the fused
+ *     persistent kernel, on the caller's stream;
+ *   gdn_prefill, other tensor-core shapes, n segments: chunk_prep(0),
+ *     chunk_chain(0), chunk_prep(1), chunk_chain(1), ... -- chunk_prep of even
+ *     segments on the caller's stream, of odd segments on a second library
+ *     stream, chunk_chain on the library's highest-priority stream;
  *   gdn_prefill, fp32 path: prelude, recurrent;
  *   gdn_decode_step: the decode kernel.
  * Slots beyond n are not recorded.  n = 0 clears the hook.  Returns

@@ -59,14 +59,17 @@ Segments segments(const gdn_dims_t *d) {
 }
 
 // Workspace: tensor-core path: Qt, Kt, -W [dk], U' [dv], Aqk [64] in fp16 and
-// e^{G_C} in fp32 per token-head, plus an fp32 state buffer [N_seq, H, dk, dv]
+// e^{G_C} in fp32 per token-head, the fused kernel's ready flags and task
+// counter, plus an fp32 state buffer [N_seq, H, dk, dv]
 // when the call runs in several segments; fp32 path: q_hat, k_hat, v_hat in fp32.
 size_t workspace_bytes(const gdn_dims_t *d) {
     const size_t nt = (size_t)d->total_tokens * d->H;
-    if (use_tensor_cores(d))
+    if (use_tensor_cores(d)) {
+        const size_t flags = ((size_t)d->num_seqs * d->H * ((d->total_tokens + 63) / 64) + 1) * 4;
         return 3 * round_up(nt * d->dk * 2) + round_up(nt * d->dv * 2) + round_up(nt * 64 * 2) +
-               round_up(nt * 4) +
+               round_up(nt * 4) + round_up(flags) +
                (segments(d).n > 1 ? round_up((size_t)d->num_seqs * d->H * d->dk * d->dv * 4) : 0);
+    }
     return 2 * round_up(nt * d->dk * sizeof(float)) + round_up(nt * d->dv * sizeof(float));
 }
 
@@ -95,6 +98,22 @@ cudaError_t get_pool(cudaMemPool_t *pool) {
         g_pools[dev] = p;
     }
     *pool = g_pools[dev];
+    return cudaSuccess;
+}
+
+// SM count of the current device (cached per device).
+cudaError_t sm_count(int *out) {
+    static int cache[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!cache[dev]) {
+        int n = 0;
+        if ((e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+        cache[dev] = n;
+    }
+    *out = cache[dev];
     return cudaSuccess;
 }
 
@@ -285,10 +304,16 @@ gdn_status_t gdn_prefill(const gdn_dims_t *dims, const void *q, const void *k, c
         w.Up = reinterpret_cast<__half *>(take(nt * a.dv * 2));
         w.Aqk = reinterpret_cast<__half *>(take(nt * 64 * 2));
         w.decay = reinterpret_cast<float *>(take(nt * 4));
+        int *ready = reinterpret_cast<int *>(take(((size_t)a.n_seq * a.H * ((a.n_tok + 63) / 64) + 1) * 4));
         const Segments g = segments(dims);
-        int slot = 0;
+        int slot = 0, sms = 0;
         e = record(g_ev_begin, a.stream);
-        if (g.n == 1) {
+        if (e == cudaSuccess) e = sm_count(&sms);
+        if (e == cudaSuccess && gdn::fused_chain_ctas(a, sms) > 0) {
+            // few (sequence, head) chains: one persistent launch, prep and chain
+            // ordered by per-chunk flags
+            e = slot_launch(&slot, a.stream, [&] { return gdn::launch_prefill_fused(a, w, ready, sms, a.stream); });
+        } else if (g.n == 1) {
             if (e == cudaSuccess)
                 e = slot_launch(&slot, a.stream, [&] { return gdn::launch_chunk_prep(a, w); });
             if (e == cudaSuccess)

@@ -22,10 +22,13 @@
 // runs; P is double-buffered in tensor memory so the output stage of chunk c
 // (quadrants 2, 3) overlaps the first MMA and the U conversion of chunk c + 1
 // (quadrants 0, 1).  Every wait is bounded.
+//
+// Device code only: the kernels that run it and the device error word it raises
+// (g_chain_err, defined before this header is included) live in prefill_tc.cu.
+#pragma once
+
 #include <cuda.h>
 #include <cuda_fp16.h>
-
-#include <cstring>
 
 #include "gdn_device.cuh"
 #include "gdn_internal.h"
@@ -33,7 +36,6 @@
 
 namespace gdn {
 
-__device__ unsigned int g_chain_err;
 
 namespace chain {
 constexpr int C = 64;
@@ -105,12 +107,35 @@ __device__ __forceinline__ bool chain_wait(uint64_t *bar, uint32_t parity, volat
     return false;
 }
 
+// Spin (bounded, with back-off) until a chunk's ready flag, published with release
+// semantics by the prep worker that wrote its workspace rows, is set; then make the
+// async proxy (the TMA loads that follow) observe those rows.
+__device__ __forceinline__ bool wait_ready(const int *flag, volatile int *abort_flag) {
+    for (uint32_t i = 0; i < (1u << 22); ++i) {
+        int v;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+        if (v) {
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            return true;
+        }
+        if (*abort_flag) return false;
+        __nanosleep(i < 64 ? 32 : 256);
+    }
+    *abort_flag = 1;
+    atomicOr(&g_chain_err, 1u);
+    return false;
+}
+
+// The chain of head h of sequence n over chunks [c_lo, c_hi), by a CTA of 4 * DV
+// threads.  With `ready` non-NULL (the fused prefill kernel) the workspace rows of
+// chunk c are read only after ready[c] is set.
 template <int DV, typename Tout>
-__global__ void __launch_bounds__(4 * DV, 1)
-chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const float *__restrict__ decay,
-                   const float *__restrict__ norm_w, const float *state_in,
-                   const int32_t *__restrict__ cu_seqlens, int n_seq, int n_tok, int H, int c_lo,
-                   int c_hi, Tout *__restrict__ out, float *state_out) {
+__device__ __forceinline__ void chain_body(const ChainMaps &maps, const float *__restrict__ decay,
+                                           const float *__restrict__ norm_w, const float *state_in,
+                                           const int32_t *__restrict__ cu_seqlens, int n_seq, int n_tok,
+                                           int H, int h, int n, int c_lo, int c_hi,
+                                           Tout *__restrict__ out, float *state_out,
+                                           const int *ready) {
     using namespace chain;
     // 4 * DV threads: warp w reads TMEM lane quadrant q = w % 4 and owns the
     // 32-column group cg = w / 4 of every row it touches.
@@ -133,7 +158,6 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const float *__restri
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q = warp & 3, cg = warp >> 2, col0 = 32 * cg;
-    const int h = blockIdx.x, n = blockIdx.y;
     int s_begin, s_end;
     if (cu_seqlens) { s_begin = __ldg(cu_seqlens + n); s_end = __ldg(cu_seqlens + n + 1); }
     else { const int L = n_tok / n_seq; s_begin = n * L; s_end = s_begin + L; }
@@ -183,6 +207,7 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const float *__restri
     auto issue_a = [&](int cc, int b) {   // cc: chunk index within this launch
         const int t0 = s_begin + (c_lo + cc) * C;
         uint8_t *st = stage(b);
+        if (ready) wait_ready(ready + c_lo + cc, abort_flag);
         umma::mbar_expect_tx(full_a + b, BYTES_A);
         umma::tma_load_3d(st + ST_AP, &maps.wn, 0, h, t0, full_a + b);
         umma::tma_load_3d(st + ST_AP + 8192, &maps.qt, 0, h, t0, full_a + b);
@@ -218,6 +243,7 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const float *__restri
         for (int cc = 0; cc < 2 && cc < n_chunks; ++cc) issue_a(cc, cc);
         if (n_chunks > 0) issue_z(0, 0);
     }
+    __syncthreads();   // the ready flags of chunks 0, 1 were acquired before any decay read
     // byte offset of the 8-column chunk `col` of row i in a 64-column-block swizzled tile
     auto tile_off = [](int i, int col) { return (col / 64) * 8192 + umma::sw128_offset(i, (col % 64) / 8); };
     // descriptor bases (start-address field advanced by offset >> 4 per K step)
@@ -234,7 +260,7 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const float *__restri
         const uint32_t ph_stage = (uint32_t)(c >> 1) & 1u, ph = (uint32_t)c & 1u;
         uint8_t *st = stage(b);
         const uint32_t tP = tbase + b * DV;
-        const float dec = __ldg(decay + (size_t)t0 * H + h);
+        const float dec = __ldcg(decay + (size_t)t0 * H + h);
         if (tid == kTmaA && c >= 1 && c + 1 < n_chunks) issue_a(c + 1, b ^ 1);
         if (q < 2) {
             // ---- P = [-W; Qt] S  (M=128, N=DV, K=dk)
@@ -255,6 +281,15 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const float *__restri
 #pragma unroll
             for (int m = 0; m < 4; ++m)
                 upk[m] = *reinterpret_cast<const uint4 *>(st + ST_US + tile_off(i, col0 + 8 * m));
+            if (i >= len) {
+                // rows past the end of a ragged chunk belong to another sequence (or lie
+                // past the tensor) and may not be written yet: dS = Kt^T U multiplies
+                // them by U = 0, so make them zero rather than trust them to be finite
+#pragma unroll
+                for (int m = 0; m < 4; ++m)
+                    *reinterpret_cast<uint4 *>(st + ST_AS + (cg >> 1) * 8192 + i * 128 + (cg & 1) * 64 + 16 * m) =
+                        make_uint4(0, 0, 0, 0);
+            }
             chain_wait(bar_p, ph, abort_flag);
             umma::tc_fence_after();
             // ---- U = U' + P[0:64] (zero past the sequence end) -> fp16 MN-major B operand
@@ -386,65 +421,6 @@ chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const float *__restri
         }
     }
     if (warp == 0) umma::tmem_dealloc(tbase, TMEM_COLS);
-}
-
-cudaError_t launch_chunk_chain(const PrefillArgs &a, const TcWorkspace &w, int c_lo, int c_hi,
-                               const float *state_in, float *state_out, cudaStream_t stream) {
-    ChainMaps m;
-    std::memset(&m, 0, sizeof m);
-    if (a.n_tok > 0) {
-        cudaError_t e;
-        if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.wn), w.Wn, false, 128, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
-        if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.qt), w.Qt, false, 128, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
-        if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.kt), w.Kt, false, 128, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
-        if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.aqk), w.Aqk, false, 64, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
-        if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.up), w.Up, false, a.dv, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
-        if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.z), a.z, true, a.dv, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
-        if (a.out_bf16 &&
-            (e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.out), a.out, true, a.dv, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
-    }
-    dim3 grid(a.H, a.n_seq);
-    cudaError_t e;
-#define GDN_CHAIN(DV_, TOUT)                                                                      \
-    e = cudaFuncSetAttribute(chunk_chain_kernel<DV_, TOUT>,                                       \
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, chain::SMEM);            \
-    if (e != cudaSuccess) return e;                                                               \
-    chunk_chain_kernel<DV_, TOUT><<<grid, 4 * DV_, chain::SMEM, stream>>>(                        \
-        m, w.decay, a.norm_w, state_in, a.cu_seqlens, a.n_seq, a.n_tok, a.H, c_lo, c_hi,        \
-        (TOUT *)a.out, state_out)
-    if (a.dv == 128) {
-        if (a.out_bf16) { GDN_CHAIN(128, bf16); } else { GDN_CHAIN(128, float); }
-    } else {
-        if (a.out_bf16) { GDN_CHAIN(64, bf16); } else { GDN_CHAIN(64, float); }
-    }
-#undef GDN_CHAIN
-    return launched();
-}
-
-cudaError_t launch_chunk_chain(const PrefillArgs &a, const TcWorkspace &w) {
-    return launch_chunk_chain(a, w, 0, (a.n_tok + 63) / 64 + 1, a.S0, a.S_final, a.stream);
-}
-
-// One CTA waits, through chain_wait, for a barrier phase that nothing completes.
-__global__ void chain_wait_selftest_kernel(uint32_t max_polls) {
-    __shared__ uint64_t bar;
-    __shared__ int abort_flag;
-    if (threadIdx.x == 0) {
-        umma::mbar_init(&bar, 1);
-        abort_flag = 0;
-        umma::fence_mbar_init();
-    }
-    __syncthreads();
-    chain_wait(&bar, 0, &abort_flag, max_polls);
-}
-
-cudaError_t chain_wait_selftest(uint32_t max_polls, cudaStream_t s) {
-    chain_wait_selftest_kernel<<<1, 32, 0, s>>>(max_polls);
-    return cudaGetLastError();
-}
-
-cudaError_t chain_error_word(unsigned *v, bool clear, cudaStream_t s) {
-    return read_error_word(g_chain_err, v, clear, s);
 }
 
 }  // namespace gdn

@@ -46,6 +46,14 @@ struct TcWorkspace {
 // The ranged forms cover chunks [c_lo, c_hi) of every sequence on `stream`; the
 // chain carries the state from state_in (NULL: zeros) to state_out (NULL: dropped).
 cudaError_t launch_chunk_prep(const PrefillArgs &a, const TcWorkspace &w);
+// The fused persistent prefill (dk = dv = 128, few (sequence, head) pairs): chain
+// CTAs and prep workers in one cooperative launch of one CTA per SM, ordered by
+// per-chunk ready flags.  fused_chain_ctas returns its chain CTA count, or 0 when
+// the shape does not suit it.  `ready` holds n_seq * H * ceil(n_tok / 64) + 1
+// ints (flags and the task counter), zeroed by the launcher on `stream`.
+int fused_chain_ctas(const PrefillArgs &a, int sms);
+cudaError_t launch_prefill_fused(const PrefillArgs &a, const TcWorkspace &w, int *ready, int sms,
+                                 cudaStream_t stream);
 cudaError_t launch_chunk_chain(const PrefillArgs &a, const TcWorkspace &w);
 cudaError_t launch_chunk_prep(const PrefillArgs &a, const TcWorkspace &w, int c_lo, int c_hi,
                               cudaStream_t stream);

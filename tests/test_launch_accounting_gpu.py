@@ -20,23 +20,23 @@ def _events(n):
     return ev
 
 
-@pytest.mark.parametrize("tokens,segments", [(320, 1), (1280, 3)])
-def test_prefill_launch_slots(cuda_device, tokens, segments):
-    # segments hold at least 8 chunks of 64 tokens: 5 chunks run as one
-    # prep + chain pair, 20 chunks as three segments (8, 8, 4 chunks)
-    cfg = scaled(PRETRAIN, lengths=(tokens,), H=2)
+@pytest.mark.parametrize("tokens,H,launches", [
+    (1280, 2, 1),     # few (sequence, head) chains: the fused persistent kernel
+    (320, 40, 2),     # 40 chains: segmented pipeline, one segment (prep, chain)
+    (1280, 40, 6),    # three segments of 8, 8 and 4 chunks
+])
+def test_prefill_launch_slots(cuda_device, tokens, H, launches):
+    cfg = scaled(PRETRAIN, lengths=(tokens,), H=H)
     inp = to_device(make_prefill_inputs(cfg, "cpu"), cuda_device)
-    n_slots = 2 * segments + 2
-    b, e = _events(n_slots), _events(n_slots)
+    b, e = _events(launches + 2), _events(launches + 2)
     gdn.set_kernel_events(b, e)
     try:
         gpu_prefill(inp, 1)
     finally:
         gdn.set_kernel_events()
-    launched = gdn.last_call_launches()
-    assert launched == 2 * segments
+    assert gdn.last_call_launches() == launches
     torch.cuda.synchronize()
-    for i in range(launched):
+    for i in range(launches):
         assert b[i].elapsed_time(e[i]) > 0.0, i
 
 

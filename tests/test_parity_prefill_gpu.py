@@ -26,6 +26,8 @@ SMALL = [
     ("long-small-S0", scaled(LONG, lengths=(1000,), H=2), TOL_BF16),
     ("varlen-edges", scaled(VARLEN, lengths=(1, 63, 64, 65, 0, 200, 130, 2), H=2), TOL_BF16),
     ("long-memory", scaled(PRETRAIN, lengths=(700, 64), H=2, long_memory=True, s0_var=0.02), TOL_BF16),
+    # 40 (sequence, head) chains: the segmented pipeline (two segments) instead of the fused kernel
+    ("many-chains-segmented", scaled(PRETRAIN, lengths=(700, 129), H=20, s0_var=0.02), TOL_BF16),
     ("dk64-dv128", replace(scaled(PRETRAIN, lengths=(190,), H=2), dk=64, dv=128, s0_var=0.02), TOL_BF16),
     ("dk128-dv64", replace(scaled(PRETRAIN, lengths=(190, 3), H=2), dk=128, dv=64, s0_var=0.02), TOL_BF16),
 ]
