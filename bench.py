@@ -53,27 +53,33 @@ KERNEL_ROOFLINE = {"chunk_prep": ("hbm", 3 * 128 * 2 + 2 * 2),                  
                    "chunk_chain": ("tensor", 3 * 2 * 128 * 128 + 2 * 64 * 128),        # 114,688 flop
                    # both in one persistent launch: the whole pass's 1,284 B
                    "prefill_fused": ("hbm", PREFILL_BYTES_PER_TOKEN_HEAD)}
-# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per token-head from
-# an ncu capture of each kernel, valid only while the kernel's source is the one
-# captured (sha1 of the .cu file); otherwise the JSON reports traffic null.
-NCU_TRAFFIC = {}
-FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per unit from one
+# ncu capture of each kernel (profiles/), valid only while the kernel's sources
+# are the ones captured (sha1 over them); otherwise the JSON reports traffic null.
+#   prefill_fused: `profile_case prefill 8192` (T = 8192, H = 32): 276.6 MB read +
+#     344.2 MB written for 262,144 token-heads; per token-head, scaled to the launch.
+NCU_TRAFFIC = {
+    "prefill_fused": {"sources": ["prefill_tc.cu", "prep_body.cuh", "chain_body.cuh"],
+                      "sha1": "7caf39c1df4352a7253886555f70271f46a7b57d",
+                      "bytes_per_unit": (276.562688e6 + 344.203776e6) / (8192 * 32)},
+}
 
 
 def kernel_traffic(name, units):
-    """ncu DRAM bytes for one launch of `name` processing `units` token-heads,
-    or None when no capture of the kernel's current source exists."""
+    """ncu DRAM bytes for one launch of `name` processing `units` (token-heads),
+    or None when no capture of the kernel's current sources exists."""
     rec = NCU_TRAFFIC.get(name)
     if rec is None:
         return None
     import hashlib
-    path = os.path.join(ROOT, "linear_attention_token_shortconv_b200", "csrc", rec["source"])
+    h = hashlib.sha1()
     try:
-        with open(path, "rb") as f:
-            sha = hashlib.sha1(f.read()).hexdigest()
+        for f in rec["sources"]:
+            with open(os.path.join(ROOT, "linear_attention_token_shortconv_b200", "csrc", f), "rb") as fh:
+                h.update(fh.read())
     except OSError:
         return None
-    return rec["bytes_per_token_head"] * units if sha == rec["sha1"] else None
+    return rec["bytes_per_unit"] * units if h.hexdigest() == rec["sha1"] else None
 
 
 def peaks():

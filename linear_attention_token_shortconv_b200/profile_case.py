@@ -1,0 +1,45 @@
+"""Small workloads for ncu captures (a few hundred MB on the device, inputs
+larger than L2), run through the public binding:
+
+    python -m linear_attention_token_shortconv_b200.profile_case prefill 8192
+        long-prefill shape with T tokens, H = 32, d = 128, S0 ~ N(0, 0.02):
+        two warm-up calls, then one call
+    python -m linear_attention_token_shortconv_b200.profile_case decode 64
+        decode step for B sequences x 32 heads, d = 128: three steps
+"""
+import sys
+from dataclasses import replace
+
+import torch
+
+from linear_attention_token_shortconv_b200 import gdn
+from linear_attention_token_shortconv_b200.workloads import (DECODE, LONG, make_decode_inputs,
+                                                             make_prefill_inputs, scaled)
+
+
+def prefill(T: int):
+    cfg = scaled(LONG, lengths=(T,))
+    inp = make_prefill_inputs(cfg, "cuda")
+    out = torch.empty((T, cfg.H, cfg.dv), dtype=torch.bfloat16, device="cuda")
+    S = torch.empty((1, cfg.H, cfg.dk, cfg.dv), device="cuda")
+    for _ in range(3):
+        gdn.prefill(inp["q"], inp["k"], inp["v"], inp["conv_w"], inp["a_logit"], inp["b_logit"], inp["A"],
+                    inp["b_alpha"], inp["z"], inp["norm_w"], S0=inp["S0"], out=out, S_final=S)
+    torch.cuda.synchronize()
+    print("ok", float(out.float().abs().mean()))
+
+
+def decode(B: int):
+    cfg = replace(DECODE, B=B)
+    d = make_decode_inputs(cfg, "cuda")
+    out = torch.empty((cfg.B, cfg.H, cfg.dv), dtype=torch.bfloat16, device="cuda")
+    for t in range(3):
+        gdn.decode_step(d["q"][t], d["k"][t], d["v"][t], d["conv_w"], d["ring"], d["a_logit"][t],
+                        d["b_logit"][t], d["A"], d["b_alpha"], d["z"][t], d["norm_w"], d["S"], out=out)
+    torch.cuda.synchronize()
+    print("ok", float(out.float().abs().mean()))
+
+
+if __name__ == "__main__":
+    kind, size = sys.argv[1], int(sys.argv[2])
+    {"prefill": prefill, "decode": decode}[kind](size)
