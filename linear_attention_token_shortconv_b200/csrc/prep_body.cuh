@@ -288,41 +288,46 @@ __device__ __forceinline__ bool prep_one_chunk(const Sync &sy, const PrepArgs pa
     {
         float2 w[4][4];
         load_conv_w(conv_w, qk_chan, w);
-        float2 y[8][4];
-        conv_silu<8>(is_k ? k : q, (size_t)H * DK, qk_col, w, t0, s_begin, 8 * warp, len, y);
-        // L2 norm over the 16 lanes that hold this head's q (or k): all 8 tokens at once
-        float ss[8];
-#pragma unroll
-        for (int ii = 0; ii < 8; ++ii) {
-            float2 acc = fmul2(y[ii][0], y[ii][0]);
-#pragma unroll
-            for (int p = 1; p < 4; ++p) acc = ffma2(y[ii][p], y[ii][p], acc);
-            ss[ii] = acc.x + acc.y;
-        }
-#pragma unroll
-        for (int o = 8; o > 0; o >>= 1) {
-#pragma unroll
-            for (int ii = 0; ii < 8; ++ii) ss[ii] += __shfl_xor_sync(0xffffffffu, ss[ii], o);
-        }
         const int oc = qk_oct & 15;
         uint8_t *hb = sHI + (oc / 8) * 16384, *lb = sLO + (oc / 8) * 16384;
+        // the warp's 8 tokens in two halves of 4 (a 7-row window each; the halo rows
+        // are re-read from L1), which keeps the prelude's registers in bounds
+#pragma unroll 1
+        for (int hf = 0; hf < 2; ++hf) {
+            float2 y[4][4];
+            conv_silu<4>(is_k ? k : q, (size_t)H * DK, qk_col, w, t0, s_begin, 8 * warp + 4 * hf, len, y);
+            // L2 norm over the 16 lanes that hold this head's q (or k): 4 tokens at once
+            float ss[4];
 #pragma unroll
-        for (int ii = 0; ii < 8; ++ii) {
-            const float r = rsqrtf(ss[ii] + kNormEps);
-            const float2 rr = make_float2(r, r);
-            uint32_t hw[4], lw[4];
+            for (int ii = 0; ii < 4; ++ii) {
+                float2 acc = fmul2(y[ii][0], y[ii][0]);
 #pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                const float2 x = fmul2(y[ii][p], rr);
-                const __half2 hh = __floats2half2_rn(x.x, x.y);
-                const float2 hf = __half22float2(hh);
-                const __half2 ll = __floats2half2_rn(x.x - hf.x, x.y - hf.y);
-                hw[p] = *reinterpret_cast<const uint32_t *>(&hh);
-                lw[p] = *reinterpret_cast<const uint32_t *>(&ll);
+                for (int p = 1; p < 4; ++p) acc = ffma2(y[ii][p], y[ii][p], acc);
+                ss[ii] = acc.x + acc.y;
             }
-            const int row = (is_k ? 64 : 0) + 8 * warp + ii;
-            umma::st_chunk(hb, row, oc % 8, make_uint4(hw[0], hw[1], hw[2], hw[3]));
-            umma::st_chunk(lb, row, oc % 8, make_uint4(lw[0], lw[1], lw[2], lw[3]));
+#pragma unroll
+            for (int o = 8; o > 0; o >>= 1) {
+#pragma unroll
+                for (int ii = 0; ii < 4; ++ii) ss[ii] += __shfl_xor_sync(0xffffffffu, ss[ii], o);
+            }
+#pragma unroll
+            for (int ii = 0; ii < 4; ++ii) {
+                const float r = rsqrtf(ss[ii] + kNormEps);
+                const float2 rr = make_float2(r, r);
+                uint32_t hw[4], lw[4];
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    const float2 x = fmul2(y[ii][p], rr);
+                    const __half2 hh = __floats2half2_rn(x.x, x.y);
+                    const float2 hf2 = __half22float2(hh);
+                    const __half2 ll = __floats2half2_rn(x.x - hf2.x, x.y - hf2.y);
+                    hw[p] = *reinterpret_cast<const uint32_t *>(&hh);
+                    lw[p] = *reinterpret_cast<const uint32_t *>(&ll);
+                }
+                const int row = (is_k ? 64 : 0) + 8 * warp + 4 * hf + ii;
+                umma::st_chunk(hb, row, oc % 8, make_uint4(hw[0], hw[1], hw[2], hw[3]));
+                umma::st_chunk(lb, row, oc % 8, make_uint4(lw[0], lw[1], lw[2], lw[3]));
+            }
         }
     }
     {
