@@ -347,6 +347,39 @@ def bench_decode(cfg, steps, dev):
     return ms, kern_ms, state_bytes, launches, clk.summary()
 
 
+def bench_decode_multi(cfg, T, steps, dev):
+    """T consecutive tokens per sequence per step (gdn_decode_multi, all committed):
+    the pool's entries [0, T) and [T, 2T) as two alternating multi-token inputs."""
+    d = make_decode_inputs(cfg, dev)
+    S, hist = d["S"], d["ring"]
+    sets = [{key: d[key][o:o + T].transpose(0, 1).contiguous()
+             for key in ("q", "k", "v", "z", "a_logit", "b_logit")} for o in (0, T)]
+    out = torch.empty((cfg.B, T, cfg.H, cfg.dv), dtype=torch.bfloat16, device=dev)
+
+    def step(t):
+        m = sets[t % 2]
+        gdn.decode_multi(m["q"], m["k"], m["v"], d["conv_w"], hist, m["a_logit"], m["b_logit"], d["A"],
+                         d["b_alpha"], m["z"], d["norm_w"], S, out=out)
+
+    for t in range(5):
+        step(t)
+    torch.cuda.synchronize()
+    evb = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    eve = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for e in evb + eve:
+        e.record()
+    torch.cuda.synchronize()
+    launches = 0
+    for t in range(steps):
+        gdn.set_timing_events(evb[t], eve[t])
+        step(t)
+        launches += gdn.last_call_launches()
+    gdn.set_timing_events(None, None)
+    torch.cuda.synchronize()
+    kern_ms = sum(b.elapsed_time(e) for b, e in zip(evb, eve)) / steps
+    return kern_ms, launches
+
+
 def oracle_sample_rate(inp, cfg, tokens, heads, n_threads):
     """Oracle (fp64, token by token) on `heads` chains of the first `tokens`
     tokens; returns (token-heads per second, seconds, threads used)."""
@@ -475,6 +508,16 @@ def main():
                             "state_gbs": gbs, "peak_gbs": pk["hbm_gbs"],
                             "frac": gbs / pk["hbm_gbs"], "state_bytes_per_step": sbytes,
                             "kernel": "decode_stream", "gpu_launches": dlaunch, "clocks": dclk}
+        torch.cuda.empty_cache()
+        T = 4
+        mk_ms, mlaunch = bench_decode_multi(DECODE, T, max(50, args.decode_steps // 4), dev)
+        mgbs = sbytes / (mk_ms * 1e-3) / 1e9
+        result["decode_multi"] = {"workload": f"multi-token decode B={DECODE.B} H={DECODE.H} d=128, "
+                                              f"T={T} tokens per sequence per step, all committed",
+                                  "kernel_ms": mk_ms, "tokens_per_s": DECODE.B * T / (mk_ms * 1e-3),
+                                  "single_token_steps_ms": T * dk_ms,
+                                  "state_gbs": mgbs, "peak_gbs": pk["hbm_gbs"], "frac": mgbs / pk["hbm_gbs"],
+                                  "kernel": "decode_stream (T <= 4)", "gpu_launches": mlaunch}
         torch.cuda.empty_cache()
 
     if not args.no_e2e:

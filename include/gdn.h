@@ -145,6 +145,36 @@ GDN_API gdn_status_t gdn_decode_step(const gdn_dims_t *dims, const void *q, cons
                              void *out, gdn_stream_t stream);
 
 /*
+ * gdn_decode_multi -- T consecutive tokens (1 <= T <= 4) for each of
+ * B = dims->num_seqs sequences in one step: the verification step of
+ * speculative decoding, where a draft of several tokens is checked by the
+ * backbone in parallel (the digest's 前置知识, on multi-token prediction).  The
+ * state is read once and written at most once for all T tokens.
+ *
+ *   q, k       [B, T, H, dk]; v, z [B, T, H, dv]; a_logit, b_logit [B, T, H] (bf16)
+ *   conv_w, A, b_alpha, norm_w   as for gdn_prefill
+ *   conv_hist  [B, 3, H(2dk+dv)] bf16, in/out, as for gdn_decode_step
+ *   S          [B, H, dk, dv] fp32, in/out
+ *   out        [B, T, H, dv] out_dtype, written for all T tokens
+ *   n_keep     [B] int32 device array or NULL (NULL = T for every sequence):
+ *              the number of leading tokens of sequence b committed to S and
+ *              conv_hist (values outside [0, T] are clamped).  n_keep[b] = 0
+ *              leaves both untouched (the state is not written at all).
+ *
+ * out is exactly what T successive gdn_decode_step calls would produce; S and
+ * conv_hist end as after the first n_keep[b] of those calls.  A verifier can
+ * run the draft with n_keep = 0 and commit the accepted prefix with a second
+ * call of those tokens.  dims->total_tokens must equal B * T.  Supported:
+ * in_dtype = GDN_BF16, dk = dv = 128 (GDN_ERR_UNSUPPORTED otherwise); T outside
+ * [1, 4] is GDN_ERR_INVALID_ARG.  No workspace is used.
+ */
+GDN_API gdn_status_t gdn_decode_multi(const gdn_dims_t *dims, int T, const void *q, const void *k,
+                                      const void *v, const float *conv_w, void *conv_hist,
+                                      const void *a_logit, const void *b_logit, const float *A,
+                                      const float *b_alpha, const void *z, const float *norm_w,
+                                      float *S, void *out, const int32_t *n_keep, gdn_stream_t stream);
+
+/*
  * gdn_prefill_noalloc -- gdn_prefill for callers that cannot allocate device
  * memory.  The pages have no counterpart: this is an interface choice of the
  * library.  Callers that may not call cudaMalloc or any allocator while they

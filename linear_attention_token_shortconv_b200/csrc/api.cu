@@ -417,4 +417,55 @@ gdn_status_t gdn_decode_step(const gdn_dims_t *dims, const void *q, const void *
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
+gdn_status_t gdn_decode_multi(const gdn_dims_t *dims, int T, const void *q, const void *k,
+                              const void *v, const float *conv_w, void *conv_hist, const void *a_logit,
+                              const void *b_logit, const float *A, const float *b_alpha, const void *z,
+                              const float *norm_w, float *S, void *out, const int32_t *n_keep,
+                              gdn_stream_t stream) {
+    tl_launches = 0;
+    if (!dims) return GDN_ERR_INVALID_ARG;
+    if (T < 1 || T > 4) return GDN_ERR_INVALID_ARG;
+    gdn_dims_t one = *dims;   // validate as a single-token step of the same shape
+    if ((int64_t)dims->total_tokens != (int64_t)dims->num_seqs * T) return GDN_ERR_INVALID_ARG;
+    one.total_tokens = dims->num_seqs;
+    gdn_status_t st = check_dims(&one, true);
+    if (st != GDN_OK) return st;
+    if (dims->in_dtype != GDN_BF16 || dims->dk != 128 || dims->dv != 128) return GDN_ERR_UNSUPPORTED;
+    const void *vec[] = {q, k, v, conv_w, conv_hist, z, S, out};
+    for (const void *p : vec) {
+        if (!p) return GDN_ERR_INVALID_ARG;
+        if (!aligned16(p)) return GDN_ERR_ALIGNMENT;
+    }
+    const void *gates[] = {a_logit, b_logit};
+    for (const void *p : gates) {
+        if (!p) return GDN_ERR_INVALID_ARG;
+        if (!aligned_to(p, 2)) return GDN_ERR_ALIGNMENT;
+    }
+    const void *params[] = {A, b_alpha, norm_w};
+    for (const void *p : params) {
+        if (!p) return GDN_ERR_INVALID_ARG;
+        if (!aligned_to(p, 4)) return GDN_ERR_ALIGNMENT;
+    }
+    if (n_keep && !aligned_to(n_keep, 4)) return GDN_ERR_ALIGNMENT;
+    gdn::DecodeArgs a;
+    a.B = dims->num_seqs;
+    a.H = dims->H;
+    a.dk = dims->dk;
+    a.dv = dims->dv;
+    a.in_bf16 = true;
+    a.out_bf16 = dims->out_dtype == GDN_BF16;
+    a.q = q; a.k = k; a.v = v; a.z = z; a.a_logit = a_logit; a.b_logit = b_logit;
+    a.conv_w = conv_w; a.A = A; a.b_alpha = b_alpha; a.norm_w = norm_w;
+    a.conv_hist = conv_hist;
+    a.S = S;
+    a.out = out;
+    a.stream = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = record(g_ev_begin, a.stream);
+    int slot = 0;
+    if (e == cudaSuccess)
+        e = slot_launch(&slot, a.stream, [&] { return gdn::launch_decode_stream(a, T, n_keep); });
+    if (e == cudaSuccess) e = record(g_ev_end, a.stream);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
 }  // extern "C"

@@ -1,18 +1,26 @@
-// K3s -- the decode step as a streaming kernel (bf16 inputs, dk = dv = 128).
+// K3s -- the decode step as a streaming kernel (bf16 inputs, dk = dv = 128),
+// for one token per sequence (gdn_decode_step) or up to four consecutive tokens
+// per sequence, as when a speculative (multi-token-prediction) draft is verified
+// (gdn_decode_multi).
 //
-// Same arithmetic as K3 (slinene.github.io write-up of "On the Design of
-// Qwen3.8-Next Architecture", 模块 A; decode time is set by the bytes moved, as
-// the digest's 前置知识 notes): conv over [history, token], SiLU, L2Norm, gates,
+// Same arithmetic as K3, token after token (slinene.github.io write-up of "On
+// the Design of Qwen3.8-Next Architecture", 模块 A; decode time is set by the
+// bytes moved, as the digest's 前置知识 notes): conv over [history, tokens],
+// SiLU, L2Norm, gates, and per token
 //     S' = alpha S + beta k e^T,  e = v - alpha S^T k,
 //     y  = alpha S^T q + beta (k.q) e,   out = sigmoid(z) RMSNorm(y) (1 + w).
+// With T tokens the state is read and written once for all of them.  The state
+// and history advance by n_keep[b] of the T tokens (all T when n_keep is NULL):
+// a verifier can compute the outputs of a draft without committing it
+// (n_keep = 0: the state is not written at all) and commit the accepted prefix.
 //
 // One persistent CTA per SM walks the (sequence, head) items.  Each item's
-// inputs -- the 64 KB fp32 state, the token's q, k, v, z rows and the three
-// history rows -- arrive by bulk copies (TMA, cp.async.bulk) into one of three
+// inputs -- the 64 KB fp32 state, the tokens' q, k, v, z rows and the three
+// history rows -- arrive by bulk copies (TMA, cp.async.bulk) into one of the
 // shared-memory stages, completing on the stage's mbarrier.  The CTA moves the
-// stage into registers at once and refills it with the item three ahead, so
-// three state loads are in flight while it computes; S' leaves from registers
-// with coalesced streaming stores.  Every wait is bounded.
+// stage into registers at once and refills it with a later item, so
+// NSTAGE - 1 state loads are in flight while it computes; S' leaves from
+// registers with coalesced streaming stores.  Every wait is bounded.
 #include <cuda_bf16.h>
 
 #include "gdn_device.cuh"
@@ -27,15 +35,23 @@ namespace dstream {
 constexpr int D = 128;                      // dk = dv
 constexpr int NT = 256;
 constexpr int STATE = D * D * 4;            // 64 KB
-constexpr int OFF_TOK = STATE;              // q, k, v, z rows: 4 x 256 B
-constexpr int OFF_HIST = OFF_TOK + 1024;    // 3 slots x (q, k, v) x 256 B
-constexpr int STAGE = OFF_HIST + 2304;      // 68,864 B (multiple of 128)
-constexpr int NSTAGE = 3;
-constexpr int OFF_MISC = NSTAGE * STAGE;    // barriers, reductions, prelude values
-constexpr int SMEM = OFF_MISC + 128 + (2 * 384 + 2 * 8 * 128 + 256) * 4 + 128;
-static_assert(STAGE % 128 == 0, "stage alignment");
-static_assert(SMEM <= 232448, "227 KB per block");
 constexpr uint32_t kMaxPolls = 1u << 24;
+// Layout for up to TMAX tokens per item: one token (three stages in flight) or
+// four (two stages: the state is reused over four token steps).
+template <int TMAX> struct Layout {
+    static constexpr int NSTAGE = TMAX == 1 ? 3 : 2;
+    static constexpr int OFF_TOK = STATE;                      // q, k, v, z rows: [4][TMAX] x 256 B
+    static constexpr int OFF_HIST = OFF_TOK + 4 * TMAX * 256;  // 3 slots x (q, k, v) x 256 B
+    static constexpr int STAGE = OFF_HIST + 2304;
+    static constexpr int OFF_MISC = NSTAGE * STAGE;            // barriers, reductions, prelude values
+    // misc: barriers / flag [0, 64), per-token scalars [64, 64 + 32 TMAX), then
+    // xs [2][TMAX][384], red [2][8][128], e [128], y [TMAX][128]
+    static constexpr int OFF_SCAL = 64;
+    static constexpr int OFF_XS = 64 + 32 * TMAX;
+    static constexpr int SMEM = OFF_MISC + OFF_XS + (2 * TMAX * 384 + 2 * 8 * 128 + 128 + TMAX * 128) * 4 + 128;
+    static_assert(STAGE % 128 == 0, "stage alignment");
+    static_assert(SMEM <= 232448, "227 KB per block");
+};
 }  // namespace dstream
 
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
@@ -63,7 +79,7 @@ __device__ __forceinline__ bool dwait(uint64_t *bar, uint32_t parity, volatile i
     return false;
 }
 
-template <typename Tout>
+template <typename Tout, int TMAX>
 __global__ void __launch_bounds__(dstream::NT, 1)
 decode_stream_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
                      const bf16 *__restrict__ v, const float *__restrict__ conv_w,
@@ -71,16 +87,21 @@ decode_stream_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
                      const bf16 *__restrict__ b_logit, const float *__restrict__ A,
                      const float *__restrict__ b_alpha, const bf16 *__restrict__ z,
                      const float *__restrict__ norm_w, float *__restrict__ S,
-                     Tout *__restrict__ out, int B, int H) {
+                     Tout *__restrict__ out, const int32_t *__restrict__ n_keep, int B, int H, int T_rt) {
     using namespace dstream;
+    using Lo = Layout<TMAX>;
+    constexpr int NSTAGE = Lo::NSTAGE, STAGE = Lo::STAGE, OFF_TOK = Lo::OFF_TOK, OFF_HIST = Lo::OFF_HIST;
+    const int T = TMAX == 1 ? 1 : T_rt;     // tokens per sequence in this call (<= TMAX)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-    uint64_t *full = reinterpret_cast<uint64_t *>(sm + OFF_MISC);            // [3]
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OFF_MISC + 32);
-    float *scal = reinterpret_cast<float *>(sm + OFF_MISC + 64);             // |q|^2, |k|^2, q.k, alpha, beta
-    float *xs2 = reinterpret_cast<float *>(sm + OFF_MISC + 128);             // [2][384] conv+SiLU values
-    float *red = xs2 + 2 * 384;                                              // [2][8][128]
-    float *ey = red + 2 * 8 * 128;                                           // e[128], y[128]
+    uint8_t *misc = sm + Lo::OFF_MISC;
+    uint64_t *full = reinterpret_cast<uint64_t *>(misc);                          // [NSTAGE]
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 32);
+    float *scal = reinterpret_cast<float *>(misc + Lo::OFF_SCAL);                 // [TMAX][8]: |q|^2, |k|^2, q.k, alpha, beta
+    float *xs2 = reinterpret_cast<float *>(misc + Lo::OFF_XS);                    // [2][TMAX][384] conv+SiLU values
+    float *red = xs2 + 2 * TMAX * 384;                                             // [2][8][128]
+    float *e_s = red + 2 * 8 * 128;                                                // e [128]
+    float *y_s = e_s + 128;                                                        // y [TMAX][128]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n_items = B * H;
@@ -97,15 +118,17 @@ decode_stream_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
         const int b = item / H, h = item % H;
         uint8_t *st = sm + s * STAGE;
         uint64_t *bar = full + s;
-        umma::mbar_expect_tx(bar, STAGE);
+        umma::mbar_expect_tx(bar, STATE + T * 1024 + 2304);
         const float *Sh = S + ((size_t)b * H + h) * D * D;
 #pragma unroll
         for (int p = 0; p < 4; ++p) bulk_load(st + p * (STATE / 4), Sh + p * (D * D / 4), STATE / 4, bar);
-        const size_t tok = ((size_t)b * H + h) * D;
-        bulk_load(st + OFF_TOK, q + tok, 256, bar);
-        bulk_load(st + OFF_TOK + 256, k + tok, 256, bar);
-        bulk_load(st + OFF_TOK + 512, v + tok, 256, bar);
-        bulk_load(st + OFF_TOK + 768, z + tok, 256, bar);
+        for (int t = 0; t < T; ++t) {
+            const size_t tok = (((size_t)b * T + t) * H + h) * D;
+            bulk_load(st + OFF_TOK + (0 * TMAX + t) * 256, q + tok, 256, bar);
+            bulk_load(st + OFF_TOK + (1 * TMAX + t) * 256, k + tok, 256, bar);
+            bulk_load(st + OFF_TOK + (2 * TMAX + t) * 256, v + tok, 256, bar);
+            bulk_load(st + OFF_TOK + (3 * TMAX + t) * 256, z + tok, 256, bar);
+        }
 #pragma unroll
         for (int j = 0; j < 3; ++j) {
             const bf16 *hr = hist + ((size_t)b * 3 + j) * C;
@@ -126,10 +149,11 @@ decode_stream_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
         const int s = j % NSTAGE;
         const uint32_t parity = (uint32_t)(j / NSTAGE) & 1u;
         const uint8_t *st = sm + s * STAGE;
-        float *xs = xs2 + (j & 1) * 384;
+        float *xs = xs2 + (j & 1) * TMAX * 384;
         const int b = item / H, h = item % H;
         const size_t gi = (size_t)b * H + h;
-        const float a_l = __bfloat162float(a_logit[gi]), b_l = __bfloat162float(b_logit[gi]);
+        // tokens of sequence b committed to the state and history
+        const int nk = TMAX == 1 ? 1 : (n_keep ? min(max(__ldg(n_keep + b), 0), T) : T);
         // this thread's conv weights: channel tid (q or k) and, for tid < 128, v channel tid
         const float4 w0 = __ldg(reinterpret_cast<const float4 *>(conv_w) +
                                 (tid < D ? (size_t)h * D + tid : (size_t)H * D + (size_t)h * D + (tid - D)));
@@ -140,7 +164,7 @@ decode_stream_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
         // ---- take everything out of the stage: the state into registers (thread t
         // holds float4 t + 256 r, i.e. row t/32 + 8 r, columns 4 (t%32) ..), the
         // conv inputs through the prelude into xs, z into warp 7's registers; the
-        // shifted history goes straight back to global memory.
+        // advanced history goes straight back to global memory.
         const float4 *Sv = reinterpret_cast<const float4 *>(st);
         float4 sreg[16];
 #pragma unroll
@@ -151,92 +175,128 @@ decode_stream_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
         for (int ch = tid; ch < 3 * D; ch += NT) {
             const int part = ch / D, i = ch % D;   // part 0 q, 1 k, 2 v
             const float4 w = ch < NT ? w0 : w1;
-            const bf16 h1 = hs[1 * 384 + part * 128 + i], h2 = hs[2 * 384 + part * 128 + i];
-            const bf16 xc = tok[part * 128 + i];
-            float acc = w.x * __bfloat162float(hs[0 * 384 + part * 128 + i]);
-            acc = fmaf(w.y, __bfloat162float(h1), acc);
-            acc = fmaf(w.z, __bfloat162float(h2), acc);
-            acc = fmaf(w.w, __bfloat162float(xc), acc);
-            xs[ch] = __fdividef(acc, 1.0f + __expf(-acc));
-            const size_t c = (size_t)part * H * D + (size_t)h * D + i;
-            hb[c] = h1;
-            hb[C + c] = h2;
-            hb[2 * C + c] = xc;
+            // the window [history slots 0..2, tokens 0..T-1] of this channel
+            bf16 win[3 + TMAX];
+#pragma unroll
+            for (int r = 0; r < 3; ++r) win[r] = hs[r * 384 + part * 128 + i];
+#pragma unroll
+            for (int t = 0; t < TMAX; ++t)
+                if (t < T) win[3 + t] = tok[(part * TMAX + t) * 128 + i];
+#pragma unroll
+            for (int t = 0; t < TMAX; ++t) {
+                if (t < T) {
+                    float acc = w.x * __bfloat162float(win[t]);
+                    acc = fmaf(w.y, __bfloat162float(win[t + 1]), acc);
+                    acc = fmaf(w.z, __bfloat162float(win[t + 2]), acc);
+                    acc = fmaf(w.w, __bfloat162float(win[t + 3]), acc);
+                    xs[t * 384 + ch] = __fdividef(acc, 1.0f + __expf(-acc));
+                }
+            }
+            if (nk > 0) {   // the history advances by the committed tokens
+                const size_t c = (size_t)part * H * D + (size_t)h * D + i;
+#pragma unroll
+                for (int r = 0; r < 3; ++r) {
+                    bf16 val = win[0];
+#pragma unroll
+                    for (int u = 1; u < 3 + TMAX; ++u)
+                        if (u == nk + r) val = win[u];
+                    hb[r * C + c] = val;
+                }
+            }
         }
-        float zr[4];
+        float zr[TMAX][4];
         if (warp == NT / 32 - 1) {
 #pragma unroll
-            for (int m = 0; m < 4; ++m) zr[m] = __bfloat162float(tok[3 * 128 + lane + 32 * m]);
+            for (int t = 0; t < TMAX; ++t)
+#pragma unroll
+                for (int m = 0; m < 4; ++m)
+                    zr[t][m] = t < T ? __bfloat162float(tok[(3 * TMAX + t) * 128 + lane + 32 * m]) : 0.f;
         }
         __syncthreads();   // stage s is consumed and xs is complete
         if (tid == 0 && item + NSTAGE * stride < n_items) issue(item + NSTAGE * stride, s);
 
-        if (warp < 3) {   // warp 0: |q|^2, warp 1: |k|^2, warp 2: q.k
-            const float *xa = xs + (warp == 1 ? D : 0), *xb = xs + (warp == 0 ? 0 : D);
-            float acc = 0.f;
+        // per-token norms and gates: warp w < 3 handles |q|^2 (0), |k|^2 (1), q.k (2)
+        if (warp < 3) {
+            for (int t = 0; t < T; ++t) {
+                const float *xa = xs + t * 384 + (warp == 1 ? D : 0), *xb = xs + t * 384 + (warp == 0 ? 0 : D);
+                float acc = 0.f;
 #pragma unroll
-            for (int i = lane; i < D; i += 32) acc = fmaf(xa[i], xb[i], acc);
-            acc = group_sum<32>(acc);
-            if (lane == 0) scal[warp] = acc;
-        } else if (tid == 96) {
-            scal[3] = expf(log_decay(a_l, __ldg(A + h), __ldg(b_alpha + h)));
-            scal[4] = sigmoid_acc(b_l);
-        }
-        // ---- partial S^T k and S^T q over this thread's 16 rows
-        float pk[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            const int i = warp + 8 * r;
-            const float kk = xs[D + i], qq = xs[i];
-            pk[0] = fmaf(sreg[r].x, kk, pk[0]); pk[1] = fmaf(sreg[r].y, kk, pk[1]);
-            pk[2] = fmaf(sreg[r].z, kk, pk[2]); pk[3] = fmaf(sreg[r].w, kk, pk[3]);
-            pq[0] = fmaf(sreg[r].x, qq, pq[0]); pq[1] = fmaf(sreg[r].y, qq, pq[1]);
-            pq[2] = fmaf(sreg[r].z, qq, pq[2]); pq[3] = fmaf(sreg[r].w, qq, pq[3]);
-        }
-        reinterpret_cast<float4 *>(red + warp * D)[lane] = make_float4(pk[0], pk[1], pk[2], pk[3]);
-        reinterpret_cast<float4 *>(red + 8 * D + warp * D)[lane] = make_float4(pq[0], pq[1], pq[2], pq[3]);
-        __syncthreads();
-        const float rq = rsqrtf(scal[0] + kNormEps), rk = rsqrtf(scal[1] + kNormEps);
-        const float kq = scal[2] * rq * rk, alpha = scal[3], beta = scal[4];
-        if (tid < D) {
-            float sk = 0.f, sq = 0.f;
-#pragma unroll
-            for (int w = 0; w < 8; ++w) { sk += red[w * D + tid]; sq += red[8 * D + w * D + tid]; }
-            const float e = xs[2 * D + tid] - alpha * rk * sk;
-            ey[tid] = e;
-            ey[D + tid] = fmaf(beta * kq, e, alpha * rq * sq);
+                for (int i = lane; i < D; i += 32) acc = fmaf(xa[i], xb[i], acc);
+                acc = group_sum<32>(acc);
+                if (lane == 0) scal[t * 8 + warp] = acc;
+            }
+        } else if (warp == 3 && lane < T) {
+            const size_t gt = ((size_t)b * T + lane) * H + h;
+            scal[lane * 8 + 3] = expf(log_decay(__bfloat162float(a_logit[gt]), __ldg(A + h), __ldg(b_alpha + h)));
+            scal[lane * 8 + 4] = sigmoid_acc(__bfloat162float(b_logit[gt]));
         }
         __syncthreads();
-        // ---- S' = alpha S + beta k e^T, from registers straight to HBM
-        {
-            const float4 e4 = reinterpret_cast<const float4 *>(ey)[lane];
-            float4 *Sg = reinterpret_cast<float4 *>(S + gi * D * D);
+        float4 *Sg = reinterpret_cast<float4 *>(S + gi * D * D);
+        for (int t = 0; t < T; ++t) {
+            const float *xt = xs + t * 384;
+            const float rq = rsqrtf(scal[t * 8 + 0] + kNormEps), rk = rsqrtf(scal[t * 8 + 1] + kNormEps);
+            const float kq = scal[t * 8 + 2] * rq * rk, alpha = scal[t * 8 + 3], beta = scal[t * 8 + 4];
+            // ---- partial S^T k and S^T q over this thread's 16 rows
+            float pk[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
-                const float bk = beta * rk * xs[D + warp + 8 * r];
-                float4 o;
-                o.x = fmaf(bk, e4.x, alpha * sreg[r].x);
-                o.y = fmaf(bk, e4.y, alpha * sreg[r].y);
-                o.z = fmaf(bk, e4.z, alpha * sreg[r].z);
-                o.w = fmaf(bk, e4.w, alpha * sreg[r].w);
-                __stcs(Sg + tid + r * NT, o);
+                const int i = warp + 8 * r;
+                const float kk = xt[D + i], qq = xt[i];
+                pk[0] = fmaf(sreg[r].x, kk, pk[0]); pk[1] = fmaf(sreg[r].y, kk, pk[1]);
+                pk[2] = fmaf(sreg[r].z, kk, pk[2]); pk[3] = fmaf(sreg[r].w, kk, pk[3]);
+                pq[0] = fmaf(sreg[r].x, qq, pq[0]); pq[1] = fmaf(sreg[r].y, qq, pq[1]);
+                pq[2] = fmaf(sreg[r].z, qq, pq[2]); pq[3] = fmaf(sreg[r].w, qq, pq[3]);
+            }
+            reinterpret_cast<float4 *>(red + warp * D)[lane] = make_float4(pk[0], pk[1], pk[2], pk[3]);
+            reinterpret_cast<float4 *>(red + 8 * D + warp * D)[lane] = make_float4(pq[0], pq[1], pq[2], pq[3]);
+            __syncthreads();
+            if (tid < D) {
+                float sk = 0.f, sq = 0.f;
+#pragma unroll
+                for (int w = 0; w < 8; ++w) { sk += red[w * D + tid]; sq += red[8 * D + w * D + tid]; }
+                const float e = xt[2 * D + tid] - alpha * rk * sk;
+                e_s[tid] = e;
+                y_s[t * D + tid] = fmaf(beta * kq, e, alpha * rq * sq);
+            }
+            __syncthreads();
+            // ---- S' = alpha S + beta k e^T in registers; the committed state leaves
+            //      after token nk - 1 (nothing is written when nk = 0)
+            const float4 e4 = reinterpret_cast<const float4 *>(e_s)[lane];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                const float bk = beta * rk * xt[D + warp + 8 * r];
+                sreg[r].x = fmaf(bk, e4.x, alpha * sreg[r].x);
+                sreg[r].y = fmaf(bk, e4.y, alpha * sreg[r].y);
+                sreg[r].z = fmaf(bk, e4.z, alpha * sreg[r].z);
+                sreg[r].w = fmaf(bk, e4.w, alpha * sreg[r].w);
+            }
+            if (t + 1 == nk) {
+#pragma unroll
+                for (int r = 0; r < 16; ++r) __stcs(Sg + tid + r * NT, sreg[r]);
             }
         }
-        // ---- output (warp 7)
+        // ---- outputs (warp 7)
         if (warp == NT / 32 - 1) {
-            float yv[4], ss = 0.f;
+            for (int t = 0; t < T; ++t) {
+                float yv[4], ss = 0.f;
 #pragma unroll
-            for (int m = 0; m < 4; ++m) { yv[m] = ey[D + lane + 32 * m]; ss = fmaf(yv[m], yv[m], ss); }
-            ss = group_sum<32>(ss);
-            const float rr = rsqrtf(ss / D + kNormEps);
+                for (int m = 0; m < 4; ++m) { yv[m] = y_s[t * D + lane + 32 * m]; ss = fmaf(yv[m], yv[m], ss); }
+                ss = group_sum<32>(ss);
+                const float rr = rsqrtf(ss / D + kNormEps);
+                const size_t go = (((size_t)b * T + t) * H + h) * D;
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const int col = lane + 32 * m;
-                out[gi * D + col] = from_f32<Tout>(sigmoid_fast(zr[m]) * yv[m] * rr * (1.0f + __ldg(norm_w + col)));
+                for (int m = 0; m < 4; ++m) {
+                    const int col = lane + 32 * m;
+                    float zt = zr[0][m];
+#pragma unroll
+                    for (int u = 1; u < TMAX; ++u)
+                        if (u == t) zt = zr[u][m];
+                    out[go + col] = from_f32<Tout>(sigmoid_fast(zt) * yv[m] * rr * (1.0f + __ldg(norm_w + col)));
+                }
             }
         }
         // No barrier here: the next item writes the other xs buffer before its
-        // first barrier, and red / ey / scal only after it.
+        // first barrier, and red / e / y / scal only after it.
     }
 }
 
@@ -244,25 +304,33 @@ bool decode_stream_supported(const DecodeArgs &a) {
     return a.in_bf16 && a.dk == 128 && a.dv == 128;
 }
 
-cudaError_t launch_decode_stream(const DecodeArgs &a) {
+cudaError_t launch_decode_stream(const DecodeArgs &a, int T, const int32_t *n_keep) {
     int dev = 0, sms = 148;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    if (T < 1 || T > 4) return cudaErrorInvalidValue;
     const int items = a.B * a.H;
+    if (items == 0) return cudaSuccess;
     const int grid = items < sms ? items : sms;
-#define GDN_DSTREAM(TOUT)                                                                          \
-    e = cudaFuncSetAttribute(decode_stream_kernel<TOUT>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                             dstream::SMEM);                                                      \
+#define GDN_DSTREAM(TOUT, TM)                                                                      \
+    e = cudaFuncSetAttribute(decode_stream_kernel<TOUT, TM>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             dstream::Layout<TM>::SMEM);                                          \
     if (e != cudaSuccess) return e;                                                                \
-    decode_stream_kernel<TOUT><<<grid, dstream::NT, dstream::SMEM, a.stream>>>(                    \
+    decode_stream_kernel<TOUT, TM><<<grid, dstream::NT, dstream::Layout<TM>::SMEM, a.stream>>>(    \
         (const bf16 *)a.q, (const bf16 *)a.k, (const bf16 *)a.v, a.conv_w, (bf16 *)a.conv_hist,   \
         (const bf16 *)a.a_logit, (const bf16 *)a.b_logit, a.A, a.b_alpha, (const bf16 *)a.z,      \
-        a.norm_w, a.S, (TOUT *)a.out, a.B, a.H)
-    if (a.out_bf16) { GDN_DSTREAM(bf16); } else { GDN_DSTREAM(float); }
+        a.norm_w, a.S, (TOUT *)a.out, n_keep, a.B, a.H, T)
+    if (T == 1 && !n_keep) {
+        if (a.out_bf16) { GDN_DSTREAM(bf16, 1); } else { GDN_DSTREAM(float, 1); }
+    } else {
+        if (a.out_bf16) { GDN_DSTREAM(bf16, 4); } else { GDN_DSTREAM(float, 4); }
+    }
 #undef GDN_DSTREAM
     return launched();
 }
+
+cudaError_t launch_decode_stream(const DecodeArgs &a) { return launch_decode_stream(a, 1, nullptr); }
 
 // One CTA waits, through dwait, for a barrier phase that nothing completes.
 __global__ void decode_wait_selftest_kernel(uint32_t max_polls) {

@@ -75,6 +75,9 @@ cudaError_t launch_decode(const DecodeArgs &a);
 // K3s: the streaming decode step for bf16 inputs with dk = dv = 128.
 bool decode_stream_supported(const DecodeArgs &a);
 cudaError_t launch_decode_stream(const DecodeArgs &a);
+// T (1..4) consecutive tokens per sequence: q, k, v, z, out [B, T, H, d], gate
+// logits [B, T, H]; the state and history advance by n_keep[b] tokens (NULL: T).
+cudaError_t launch_decode_stream(const DecodeArgs &a, int T, const int32_t *n_keep);
 
 // Kernel-launch accounting for gdn_last_call_launches(): every launcher returns
 // launched() right after its <<<...>>>, which counts the launch on this thread.

@@ -24,7 +24,7 @@ STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "G
 EXPORTS = ("gdn_prefill", "gdn_prefill_workspace_size", "gdn_decode_step", "gdn_status_string",
            "gdn_set_timing_events", "gdn_selftest_umma", "gdn_prefill_noalloc",
            "gdn_set_kernel_events", "gdn_last_call_launches", "gdn_device_error_status",
-           "gdn_selftest_wait_timeout")
+           "gdn_selftest_wait_timeout", "gdn_decode_multi")
 ERRF_PREP, ERRF_CHAIN, ERRF_DECODE = 1, 2, 4
 
 
@@ -59,6 +59,8 @@ def load() -> ctypes.CDLL:
         lib.gdn_prefill_workspace_size.restype = ctypes.c_int
         lib.gdn_decode_step.argtypes = [D] + [P] * 14
         lib.gdn_decode_step.restype = ctypes.c_int
+        lib.gdn_decode_multi.argtypes = [D, ctypes.c_int] + [P] * 15
+        lib.gdn_decode_multi.restype = ctypes.c_int
         lib.gdn_prefill_noalloc.argtypes = [D] + [P] * 15
         lib.gdn_prefill_noalloc.restype = ctypes.c_int
         lib.gdn_selftest_umma.argtypes = [ctypes.c_int] * 5 + [P] * 5
@@ -185,6 +187,24 @@ def decode_step(q, k, v, conv_w, conv_hist, a_logit, b_logit, A, b_alpha, z, nor
     return out
 
 
+def decode_multi(q, k, v, conv_w, conv_hist, a_logit, b_logit, A, b_alpha, z, norm_w, S, *,
+                 n_keep=None, out=None, out_dtype=torch.float32, stream=None):
+    """gdn_decode_multi on torch tensors: q, k [B, T, H, dk]; v, z [B, T, H, dv];
+    a_logit, b_logit [B, T, H].  Returns out [B, T, H, dv]; conv_hist and S
+    advance in place by n_keep[b] tokens (int32 [B] CUDA tensor; None = all T)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=out_dtype, device=q.device)
+    dims = Dims(B, B * T, H, dk, dv, conv_w.shape[1], _dt(q), _dt(out))
+    rc = load().gdn_decode_multi(ctypes.byref(dims), T, _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w),
+                                 _ptr(conv_hist), _ptr(a_logit), _ptr(b_logit), _ptr(A), _ptr(b_alpha),
+                                 _ptr(z), _ptr(norm_w), _ptr(S), _ptr(out), _ptr(n_keep),
+                                 _stream(stream))
+    _check(rc, "gdn_decode_multi")
+    return out
+
+
 def set_timing_events(begin=None, end=None):
     """Record torch.cuda.Event `begin`/`end` around the dominant kernel of each
     following call (None, None clears the hook)."""
@@ -226,7 +246,7 @@ def device_error_status(clear=False, stream=None):
 def selftest_wait_timeout(family, max_polls=1024, stream=None):
     """Launch one CTA whose bounded wait (kernel family `family`) runs out."""
     _check(load().gdn_selftest_wait_timeout(family, max_polls, _stream(stream)),
-           "gdn_selftest_wait_timeout")
+           "gdn_selftest_wait_timeout", "gdn_decode_multi")
 
 
 def selftest_umma(A, B, init=None, *, a_mn=False, b_mn=False, negate_a=False, stream=None):

@@ -123,3 +123,20 @@ def test_wait_selftest_validation(lib):
     assert lib.gdn_selftest_wait_timeout(3, 16, None) == 1       # two bits
     assert lib.gdn_selftest_wait_timeout(1, 0, None) == 1
     assert lib.gdn_selftest_wait_timeout(1, 65537, None) == 1
+
+
+def test_decode_multi_argument_validation(lib):
+    args = [FAKE[i] for i in range(11)] + [ctypes.c_void_p(8192), ctypes.c_void_p(12288), None, None]
+    ok = _dims(num_seqs=4, total_tokens=8, in_dtype=1)               # B = 4, T = 2
+    assert lib.gdn_decode_multi(ctypes.byref(ok), 0, *args) == 1      # T outside [1, 4]
+    assert lib.gdn_decode_multi(ctypes.byref(ok), 5, *args) == 1
+    assert lib.gdn_decode_multi(ctypes.byref(ok), 3, *args) == 1      # total_tokens != B * T
+    assert lib.gdn_decode_multi(ctypes.byref(_dims(num_seqs=4, total_tokens=8, dv=64)), 2, *args) == 2
+    assert lib.gdn_decode_multi(ctypes.byref(_dims(num_seqs=4, total_tokens=8, in_dtype=0)), 2, *args) == 2
+    bad = list(args)
+    bad[11] = ctypes.c_void_p(8200)                                   # S misaligned
+    assert lib.gdn_decode_multi(ctypes.byref(ok), 2, *bad) == 3
+    bad = list(args)
+    bad[13] = ctypes.c_void_p(4098)                                   # n_keep misaligned
+    assert lib.gdn_decode_multi(ctypes.byref(ok), 2, *bad) == 3
+    assert lib.gdn_last_call_launches() == 0
