@@ -283,6 +283,14 @@ __device__ __forceinline__ bool prep_one_chunk(const Sync &sy, const PrepArgs pa
     bool ok = true;
     const int t0 = s_begin + c * C;
     const int len = min(C, s_end - t0);
+    // the token's gate logits (thread tid < len), loaded first so that their latency
+    // passes while the convolutions run
+    bf16 a_raw = __float2bfloat16(0.f), b_raw = __float2bfloat16(0.f);
+    if (tid < len) {
+        const size_t gi = (size_t)(t0 + tid) * H + h;
+        a_raw = a_logit[gi];
+        b_raw = b_logit[gi];
+    }
     // ---- 1. prelude: q, k -> L2-normalised fp32 -> hi/lo fp16 tiles; v -> fp16 tile
     // (conv weights re-read per chunk from L1/L2 to keep them out of the solve's registers)
     {
@@ -345,9 +353,8 @@ __device__ __forceinline__ bool prep_one_chunk(const Sync &sy, const PrepArgs pa
     if (tid < C) {
         float g = 0.f, be = 0.f;
         if (tid < len) {
-            const size_t gi = (size_t)(t0 + tid) * H + h;
-            g = -eA * softplus_fast(to_f32(a_logit[gi]) + ba);
-            be = sigmoid_fast(to_f32(b_logit[gi]));
+            g = -eA * softplus_fast(to_f32(a_raw) + ba);
+            be = sigmoid_fast(to_f32(b_raw));
         }
         // inclusive scan of the log decays within each warp, then across the two
 #pragma unroll

@@ -246,7 +246,7 @@ def device_error_status(clear=False, stream=None):
 def selftest_wait_timeout(family, max_polls=1024, stream=None):
     """Launch one CTA whose bounded wait (kernel family `family`) runs out."""
     _check(load().gdn_selftest_wait_timeout(family, max_polls, _stream(stream)),
-           "gdn_selftest_wait_timeout", "gdn_decode_multi")
+           "gdn_selftest_wait_timeout")
 
 
 def selftest_umma(A, B, init=None, *, a_mn=False, b_mn=False, negate_a=False, stream=None):
