@@ -37,18 +37,19 @@ constexpr int NT = 256;
 constexpr int STATE = D * D * 4;            // 64 KB
 constexpr uint32_t kMaxPolls = 1u << 24;
 // Layout for up to TMAX tokens per item: one token (three stages in flight) or
-// four (two stages: the state is reused over four token steps).
+// four (two stages: the state is read once for four tokens).
 template <int TMAX> struct Layout {
     static constexpr int NSTAGE = TMAX == 1 ? 3 : 2;
     static constexpr int OFF_TOK = STATE;                      // q, k, v, z rows: [4][TMAX] x 256 B
     static constexpr int OFF_HIST = OFF_TOK + 4 * TMAX * 256;  // 3 slots x (q, k, v) x 256 B
     static constexpr int STAGE = OFF_HIST + 2304;
     static constexpr int OFF_MISC = NSTAGE * STAGE;            // barriers, reductions, prelude values
-    // misc: barriers / flag [0, 64), per-token scalars [64, 64 + 32 TMAX), then
-    // xs [2][TMAX][384], red [2][8][128], e [128], y [TMAX][128]
-    static constexpr int OFF_SCAL = 64;
-    static constexpr int OFF_XS = 64 + 32 * TMAX;
-    static constexpr int SMEM = OFF_MISC + OFF_XS + (2 * TMAX * 384 + 2 * 8 * 128 + 128 + TMAX * 128) * 4 + 128;
+    // misc: barriers / flag [0, 64), gates [TMAX][2], Gram products [4][TMAX][TMAX],
+    // then xs [2][TMAX][384], red [2][TMAX][8][128], e [TMAX][128], y [TMAX][128]
+    static constexpr int OFF_GATE = 64;
+    static constexpr int OFF_GRAM = OFF_GATE + 8 * TMAX;
+    static constexpr int OFF_XS = (OFF_GRAM + 16 * TMAX * TMAX + 15) / 16 * 16;
+    static constexpr int SMEM = OFF_MISC + OFF_XS + (2 * TMAX * 384 + 2 * TMAX * 8 * 128 + 2 * TMAX * 128) * 4 + 128;
     static_assert(STAGE % 128 == 0, "stage alignment");
     static_assert(SMEM <= 232448, "227 KB per block");
 };
@@ -97,11 +98,12 @@ decode_stream_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
     uint8_t *misc = sm + Lo::OFF_MISC;
     uint64_t *full = reinterpret_cast<uint64_t *>(misc);                          // [NSTAGE]
     volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 32);
-    float *scal = reinterpret_cast<float *>(misc + Lo::OFF_SCAL);                 // [TMAX][8]: |q|^2, |k|^2, q.k, alpha, beta
+    float *gate = reinterpret_cast<float *>(misc + Lo::OFF_GATE);                 // [TMAX][2]: alpha, beta
+    float *gram = reinterpret_cast<float *>(misc + Lo::OFF_GRAM);                 // [4][TMAX][TMAX]
     float *xs2 = reinterpret_cast<float *>(misc + Lo::OFF_XS);                    // [2][TMAX][384] conv+SiLU values
-    float *red = xs2 + 2 * TMAX * 384;                                             // [2][8][128]
-    float *e_s = red + 2 * 8 * 128;                                                // e [128]
-    float *y_s = e_s + 128;                                                        // y [TMAX][128]
+    float *red = xs2 + 2 * TMAX * 384;                                             // [2][TMAX][8][128]
+    float *e_s = red + 2 * TMAX * 8 * 128;                                         // e [TMAX][128]
+    float *y_s = e_s + TMAX * 128;                                                 // y [TMAX][128]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n_items = B * H;
@@ -154,6 +156,13 @@ decode_stream_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
         const size_t gi = (size_t)b * H + h;
         // tokens of sequence b committed to the state and history
         const int nk = TMAX == 1 ? 1 : (n_keep ? min(max(__ldg(n_keep + b), 0), T) : T);
+        // gate logits of this item's tokens (warp 3, lane t)
+        float a_l = 0.f, b_l = 0.f;
+        if (warp == 3 && lane < T) {
+            const size_t gt = ((size_t)b * T + lane) * H + h;
+            a_l = __bfloat162float(a_logit[gt]);
+            b_l = __bfloat162float(b_logit[gt]);
+        }
         // this thread's conv weights: channel tid (q or k) and, for tid < 128, v channel tid
         const float4 w0 = __ldg(reinterpret_cast<const float4 *>(conv_w) +
                                 (tid < D ? (size_t)h * D + tid : (size_t)H * D + (size_t)h * D + (tid - D)));
@@ -215,88 +224,176 @@ decode_stream_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
         __syncthreads();   // stage s is consumed and xs is complete
         if (tid == 0 && item + NSTAGE * stride < n_items) issue(item + NSTAGE * stride, s);
 
-        // per-token norms and gates: warp w < 3 handles |q|^2 (0), |k|^2 (1), q.k (2)
-        if (warp < 3) {
-            for (int t = 0; t < T; ++t) {
-                const float *xa = xs + t * 384 + (warp == 1 ? D : 0), *xb = xs + t * 384 + (warp == 0 ? 0 : D);
+        // ---- the Gram products of the raw conv outputs, alongside pass 1.  Token t
+        // owns entries t (t + 2) .. (t + 1)(t + 3) - 1: q_t.q_t (type 0), k_t.k_t
+        // (type 1), k_s.k_t for s < t (type 2), k_s.q_t for s <= t (type 3); warp w
+        // takes entries w, w + 8, ..  Warp 3, lane t, also computes token t's gates.
+        for (int d = warp; d < 2 * TMAX + TMAX * TMAX; d += NT / 32) {
+            int t = 0;
+            while ((t + 1) * (t + 3) <= d) ++t;
+            const int r = d - t * (t + 2);
+            const int type = r < 2 ? r : (r < 2 + t ? 2 : 3);
+            const int sx = r < 2 ? t : (type == 2 ? r - 2 : r - 2 - t);
+            if (t < T) {
+                const float *xa = xs + (type == 0 ? t * 384 : sx * 384 + D);
+                const float *xb = xs + t * 384 + (type == 1 || type == 2 ? D : 0);
                 float acc = 0.f;
 #pragma unroll
                 for (int i = lane; i < D; i += 32) acc = fmaf(xa[i], xb[i], acc);
                 acc = group_sum<32>(acc);
-                if (lane == 0) scal[t * 8 + warp] = acc;
+                if (lane == 0) gram[(type * TMAX + t) * TMAX + sx] = acc;
             }
-        } else if (warp == 3 && lane < T) {
-            const size_t gt = ((size_t)b * T + lane) * H + h;
-            scal[lane * 8 + 3] = expf(log_decay(__bfloat162float(a_logit[gt]), __ldg(A + h), __ldg(b_alpha + h)));
-            scal[lane * 8 + 4] = sigmoid_acc(__bfloat162float(b_logit[gt]));
         }
-        __syncthreads();
-        float4 *Sg = reinterpret_cast<float4 *>(S + gi * D * D);
-        for (int t = 0; t < T; ++t) {
-            const float *xt = xs + t * 384;
-            const float rq = rsqrtf(scal[t * 8 + 0] + kNormEps), rk = rsqrtf(scal[t * 8 + 1] + kNormEps);
-            const float kq = scal[t * 8 + 2] * rq * rk, alpha = scal[t * 8 + 3], beta = scal[t * 8 + 4];
-            // ---- partial S^T k and S^T q over this thread's 16 rows
-            float pk[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f};
+        if (warp == 3 && lane < T) {
+            gate[lane * 2 + 0] = expf(log_decay(a_l, __ldg(A + h), __ldg(b_alpha + h)));
+            gate[lane * 2 + 1] = sigmoid_acc(b_l);
+        }
+        // ---- pass 1: partial S0^T k_t and S0^T q_t over this thread's 16 rows
+        {
+            float4 pk[TMAX], pq[TMAX];
+#pragma unroll
+            for (int t = 0; t < TMAX; ++t) { pk[t] = make_float4(0.f, 0.f, 0.f, 0.f); pq[t] = pk[t]; }
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
                 const int i = warp + 8 * r;
-                const float kk = xt[D + i], qq = xt[i];
-                pk[0] = fmaf(sreg[r].x, kk, pk[0]); pk[1] = fmaf(sreg[r].y, kk, pk[1]);
-                pk[2] = fmaf(sreg[r].z, kk, pk[2]); pk[3] = fmaf(sreg[r].w, kk, pk[3]);
-                pq[0] = fmaf(sreg[r].x, qq, pq[0]); pq[1] = fmaf(sreg[r].y, qq, pq[1]);
-                pq[2] = fmaf(sreg[r].z, qq, pq[2]); pq[3] = fmaf(sreg[r].w, qq, pq[3]);
-            }
-            reinterpret_cast<float4 *>(red + warp * D)[lane] = make_float4(pk[0], pk[1], pk[2], pk[3]);
-            reinterpret_cast<float4 *>(red + 8 * D + warp * D)[lane] = make_float4(pq[0], pq[1], pq[2], pq[3]);
-            __syncthreads();
-            if (tid < D) {
-                float sk = 0.f, sq = 0.f;
 #pragma unroll
-                for (int w = 0; w < 8; ++w) { sk += red[w * D + tid]; sq += red[8 * D + w * D + tid]; }
-                const float e = xt[2 * D + tid] - alpha * rk * sk;
-                e_s[tid] = e;
-                y_s[t * D + tid] = fmaf(beta * kq, e, alpha * rq * sq);
+                for (int t = 0; t < TMAX; ++t) {
+                    if (t < T) {
+                        const float kk = xs[t * 384 + D + i], qq = xs[t * 384 + i];
+                        pk[t].x = fmaf(sreg[r].x, kk, pk[t].x); pk[t].y = fmaf(sreg[r].y, kk, pk[t].y);
+                        pk[t].z = fmaf(sreg[r].z, kk, pk[t].z); pk[t].w = fmaf(sreg[r].w, kk, pk[t].w);
+                        pq[t].x = fmaf(sreg[r].x, qq, pq[t].x); pq[t].y = fmaf(sreg[r].y, qq, pq[t].y);
+                        pq[t].z = fmaf(sreg[r].z, qq, pq[t].z); pq[t].w = fmaf(sreg[r].w, qq, pq[t].w);
+                    }
+                }
             }
-            __syncthreads();
-            // ---- S' = alpha S + beta k e^T in registers; the committed state leaves
-            //      after token nk - 1 (nothing is written when nk = 0)
-            const float4 e4 = reinterpret_cast<const float4 *>(e_s)[lane];
+#pragma unroll
+            for (int t = 0; t < TMAX; ++t) {
+                if (t < T) {
+                    reinterpret_cast<float4 *>(red + (t * 8 + warp) * D)[lane] = pk[t];
+                    reinterpret_cast<float4 *>(red + ((TMAX + t) * 8 + warp) * D)[lane] = pq[t];
+                }
+            }
+        }
+        __syncthreads();   // gram, gate and red are complete
+
+        // Per-token scalars, the same in every thread: rq, rk normalise q_t, k_t;
+        // cum[t] = alpha_0 .. alpha_{t-1} (the decay from the item's start to token t).
+        float rq[TMAX], rk[TMAX], al[TMAX], be[TMAX], cum[TMAX + 1];
+        cum[0] = 1.f;
+#pragma unroll
+        for (int t = 0; t < TMAX; ++t) {
+            if (t < T) {
+                rq[t] = rsqrtf(gram[(0 * TMAX + t) * TMAX + t] + kNormEps);
+                rk[t] = rsqrtf(gram[(1 * TMAX + t) * TMAX + t] + kNormEps);
+                al[t] = gate[t * 2 + 0];
+                be[t] = gate[t * 2 + 1];
+            } else {
+                rq[t] = rk[t] = be[t] = 0.f;
+                al[t] = 1.f;
+            }
+            cum[t + 1] = cum[t] * al[t];
+        }
+        // ---- column solve (thread j < 128 owns column j), from S0 alone:
+        //   e_t = v_t - cum_{t+1} S0^T k_t - sum_{s<t} (cum_{t+1}/cum_{s+1}) beta_s (k_s.k_t) e_s
+        //   y_t = cum_{t+1} S0^T q_t + sum_{s<=t} (cum_{t+1}/cum_{s+1}) beta_s (k_s.q_t) e_s
+        // with unit-norm k, q; the ratio is the product alpha_{s+1} .. alpha_t.
+        if (tid < D) {
+            float e[TMAX];
+#pragma unroll
+            for (int t = 0; t < TMAX; ++t) {
+                if (t < T) {
+                    float sk = 0.f, sq = 0.f;
+#pragma unroll
+                    for (int w = 0; w < 8; ++w) {
+                        sk += red[(t * 8 + w) * D + tid];
+                        sq += red[((TMAX + t) * 8 + w) * D + tid];
+                    }
+                    float ev = xs[t * 384 + 2 * D + tid] - cum[t + 1] * rk[t] * sk;
+                    float yv = cum[t + 1] * rq[t] * sq;
+                    float ratio = 1.f;   // alpha_{s+1} .. alpha_t, built downwards from s = t
+#pragma unroll
+                    for (int s2 = TMAX - 1; s2 >= 0; --s2) {
+                        if (s2 <= t) {
+                            if (s2 < t) {
+                                ratio *= al[s2 + 1];
+                                ev -= ratio * be[s2] * rk[s2] * rk[t] * gram[(2 * TMAX + t) * TMAX + s2] * e[s2];
+                            }
+                        }
+                    }
+                    e[t] = ev;
+                    ratio = 1.f;
+#pragma unroll
+                    for (int s2 = TMAX - 1; s2 >= 0; --s2) {
+                        if (s2 <= t) {
+                            if (s2 < t) ratio *= al[s2 + 1];
+                            yv = fmaf(ratio * be[s2] * rk[s2] * rq[t] * gram[(3 * TMAX + t) * TMAX + s2], e[s2], yv);
+                        }
+                    }
+                    e_s[t * D + tid] = ev;
+                    y_s[t * D + tid] = yv;
+                }
+            }
+        }
+        __syncthreads();   // e and y are complete
+        // ---- pass 2: the committed state
+        //   S_nk = cum_nk S0 + sum_{s<nk} (cum_nk/cum_{s+1}) beta_s k_s e_s^T
+        // from registers straight to HBM (nothing is written when nk = 0)
+        if (nk > 0) {
+            float cs[TMAX];
+            float4 e4[TMAX];
+            float ratio = 1.f;
+#pragma unroll
+            for (int s2 = TMAX - 1; s2 >= 0; --s2) {
+                cs[s2] = 0.f;
+                if (s2 < nk) {
+                    cs[s2] = ratio * be[s2] * rk[s2];
+                    ratio *= al[s2];
+                }
+            }
+            const float decay = cum[0] * ratio;   // = cum_nk
+#pragma unroll
+            for (int s2 = 0; s2 < TMAX; ++s2)
+                e4[s2] = s2 < nk ? reinterpret_cast<const float4 *>(e_s + s2 * D)[lane] : make_float4(0.f, 0.f, 0.f, 0.f);
+            float4 *Sg = reinterpret_cast<float4 *>(S + gi * D * D);
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
-                const float bk = beta * rk * xt[D + warp + 8 * r];
-                sreg[r].x = fmaf(bk, e4.x, alpha * sreg[r].x);
-                sreg[r].y = fmaf(bk, e4.y, alpha * sreg[r].y);
-                sreg[r].z = fmaf(bk, e4.z, alpha * sreg[r].z);
-                sreg[r].w = fmaf(bk, e4.w, alpha * sreg[r].w);
-            }
-            if (t + 1 == nk) {
+                const int i = warp + 8 * r;
+                float4 o = make_float4(decay * sreg[r].x, decay * sreg[r].y, decay * sreg[r].z, decay * sreg[r].w);
 #pragma unroll
-                for (int r = 0; r < 16; ++r) __stcs(Sg + tid + r * NT, sreg[r]);
+                for (int s2 = 0; s2 < TMAX; ++s2) {
+                    if (s2 < nk) {
+                        const float bk = cs[s2] * xs[s2 * 384 + D + i];
+                        o.x = fmaf(bk, e4[s2].x, o.x);
+                        o.y = fmaf(bk, e4[s2].y, o.y);
+                        o.z = fmaf(bk, e4[s2].z, o.z);
+                        o.w = fmaf(bk, e4[s2].w, o.w);
+                    }
+                }
+                __stcs(Sg + tid + r * NT, o);
             }
         }
         // ---- outputs (warp 7)
         if (warp == NT / 32 - 1) {
-            for (int t = 0; t < T; ++t) {
-                float yv[4], ss = 0.f;
 #pragma unroll
-                for (int m = 0; m < 4; ++m) { yv[m] = y_s[t * D + lane + 32 * m]; ss = fmaf(yv[m], yv[m], ss); }
-                ss = group_sum<32>(ss);
-                const float rr = rsqrtf(ss / D + kNormEps);
-                const size_t go = (((size_t)b * T + t) * H + h) * D;
+            for (int t = 0; t < TMAX; ++t) {
+                if (t < T) {
+                    float yv[4], ss = 0.f;
 #pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    const int col = lane + 32 * m;
-                    float zt = zr[0][m];
+                    for (int m = 0; m < 4; ++m) { yv[m] = y_s[t * D + lane + 32 * m]; ss = fmaf(yv[m], yv[m], ss); }
+                    ss = group_sum<32>(ss);
+                    const float rr = rsqrtf(ss / D + kNormEps);
+                    const size_t go = (((size_t)b * T + t) * H + h) * D;
 #pragma unroll
-                    for (int u = 1; u < TMAX; ++u)
-                        if (u == t) zt = zr[u][m];
-                    out[go + col] = from_f32<Tout>(sigmoid_fast(zt) * yv[m] * rr * (1.0f + __ldg(norm_w + col)));
+                    for (int m = 0; m < 4; ++m) {
+                        const int col = lane + 32 * m;
+                        out[go + col] = from_f32<Tout>(sigmoid_fast(zr[t][m]) * yv[m] * rr * (1.0f + __ldg(norm_w + col)));
+                    }
                 }
             }
         }
         // No barrier here: the next item writes the other xs buffer before its
-        // first barrier, and red / e / y / scal only after it.
+        // first barrier, and red / gram / gate / e / y only after it.
     }
 }
 
