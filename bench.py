@@ -24,13 +24,13 @@ import sys
 import tempfile
 import time
 from dataclasses import replace
-from datetime import timedelta
 
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+from linear_attention_token_shortconv_b200 import dist as rankio  # noqa: E402
 from linear_attention_token_shortconv_b200 import gdn  # noqa: E402
 from linear_attention_token_shortconv_b200.workloads import (DECODE, LONG, make_decode_inputs,  # noqa: E402
                                                              make_prefill_inputs, to_oracle_bits)
@@ -193,28 +193,12 @@ class ClockSampler:
                 "source": self.source, "reasons": reasons}
 
 
-def dist_setup():
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=timedelta(seconds=300),
-                                             device_id=torch.device("cuda", local))
-    return world, rank, local
-
-
 def barrier(world):
-    if world > 1:
-        torch.distributed.barrier()
+    rankio.barrier(world)
 
 
 def max_over_ranks(x, world):
-    if world == 1:
-        return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    return float(t.item())
+    return rankio.max_over_ranks(x, world, "cuda")
 
 
 def prefill_call(inp, out, S_final):
@@ -227,7 +211,7 @@ def bench_prefill(cfg, steps, warmup, world, rank, dev):
     """Times `steps` gdn_prefill calls.  Besides the whole-call events (on the
     caller's stream, which the library forks from and joins), every kernel
     launch is bracketed by its own pair of events on the stream it runs on."""
-    inp = make_prefill_inputs(cfg, dev, seed=cfg.seed + 1000 * rank)
+    inp = make_prefill_inputs(cfg, dev, seed=rankio.shard_seed(cfg.seed, rank))
     n_tok, H = cfg.total_tokens, cfg.H
     out = torch.empty((n_tok, H, cfg.dv), dtype=torch.bfloat16, device=dev)
     S_final = torch.empty((cfg.num_seqs, H, cfg.dk, cfg.dv), dtype=torch.float32, device=dev)
@@ -276,7 +260,7 @@ def bench_prefill(cfg, steps, warmup, world, rank, dev):
 def bench_e2e(cfg, steps, warmup, world, rank, dev):
     """Same metric through the public API with the inputs in pinned host memory:
     every step copies the step's inputs host->device and reads out + S_final back."""
-    src = make_prefill_inputs(cfg, dev, seed=cfg.seed + 1000 * rank)
+    src = make_prefill_inputs(cfg, dev, seed=rankio.shard_seed(cfg.seed, rank))
     host = {k: (None if v is None else v.cpu().pin_memory()) for k, v in src.items()}
     dev_in = {k: (None if v is None else torch.empty_like(v)) for k, v in src.items()}
     del src
@@ -442,8 +426,7 @@ def main():
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")
 
-    world, rank, local = dist_setup() if args.impl == "ours" else (
-        int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
+    world, rank, local = rankio.setup("nccl") if args.impl == "ours" else rankio.env_ranks()
     if args.impl == "reference":
         run_reference(args, world, rank)
         return
@@ -455,7 +438,7 @@ def main():
     ms, kern_ms, clocks, kernels, launches, inp = bench_prefill(cfg, args.steps, args.warmup, world,
                                                                 rank, dev)
     token_heads = cfg.total_tokens * cfg.H
-    value = world * cfg.total_tokens / (ms * 1e-3)
+    value = rankio.job_throughput(world, cfg.total_tokens, ms)
     path_gbs = PREFILL_BYTES_PER_TOKEN_HEAD * token_heads / (kern_ms * 1e-3) / 1e9
     tc_achieved = PREFILL_FLOP_PER_TOKEN_HEAD * token_heads / (kern_ms * 1e-3) / 1e12
     dom = max(kernels, key=lambda n: kernels[n]["ms_per_step"])
@@ -522,7 +505,7 @@ def main():
 
     if not args.no_e2e:
         e_ms, h2d, d2h = bench_e2e(cfg, max(3, args.steps // 2), args.warmup, world, rank, dev)
-        result["e2e"] = {"value": world * cfg.total_tokens / (e_ms * 1e-3), "unit": "tokens/s",
+        result["e2e"] = {"value": rankio.job_throughput(world, cfg.total_tokens, e_ms), "unit": "tokens/s",
                          "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
         torch.cuda.empty_cache()
 
