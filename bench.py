@@ -60,8 +60,8 @@ KERNEL_ROOFLINE = {"chunk_prep": ("hbm", 3 * 128 * 2 + 2 * 2),                  
 #     344.2 MB written for 262,144 token-heads; per token-head, scaled to the launch.
 NCU_TRAFFIC = {
     "prefill_fused": {"sources": ["prefill_tc.cu", "prep_body.cuh", "chain_body.cuh"],
-                      "sha1": "7caf39c1df4352a7253886555f70271f46a7b57d",
-                      "bytes_per_unit": (276.562688e6 + 344.203776e6) / (8192 * 32)},
+                      "sha1": "7f9f4aba8627ebcc0087792eddc6533e5c331e11",
+                      "bytes_per_unit": (277.407232e6 + 324.293888e6) / (8192 * 32)},
 }
 
 
