@@ -35,6 +35,8 @@ def lib():
         _lib.gdn_oracle_prelude.restype = ip
         _lib.gdn_oracle_gated_rmsnorm.argtypes = [ip, ip, dp, dp, fp, dp]
         _lib.gdn_oracle_gated_rmsnorm.restype = ip
+        _lib.gdn_oracle_backward.argtypes = [ip] * 7 + [vp] * 25 + [ip]
+        _lib.gdn_oracle_backward.restype = ip
         _lib.gdn_oracle_threads.argtypes = [ip]
         _lib.gdn_oracle_threads.restype = ip
     return _lib
@@ -167,3 +169,43 @@ def gated_rmsnorm(y, z, w):
     if rc != 0:
         raise ValueError("bad sizes")
     return o
+
+
+def backward(q, k, v, conv_w, a_logit, b_logit, A, b_alpha, z, norm_w, d_out, S0=None,
+             d_S_final=None, cu_seqlens=None, num_seqs=None, n_threads=0):
+    """Token-by-token fp64 gradients of <d_out, out> + <d_S_final, S_final> with
+    respect to every prefill input (same layouts as :func:`prefill`).
+
+    Returns a dict of float64 arrays: dq, dk, dv, d_conv_w, d_a_logit, d_b_logit,
+    d_A, d_b_alpha, d_z, d_norm_w, d_S0."""
+    q, k, v, z, a_logit, b_logit = (_c(x) for x in (q, k, v, z, a_logit, b_logit))
+    dt = _dtype_code(q)
+    for x in (k, v, z, a_logit, b_logit):
+        if _dtype_code(x) != dt:
+            raise TypeError("all token inputs must share one dtype")
+    n_tok, H, dk = q.shape
+    dv = v.shape[2]
+    conv_w = _c(conv_w, np.float32)
+    K = conv_w.shape[1]
+    A, b_alpha, norm_w = _c(A, np.float32), _c(b_alpha, np.float32), _c(norm_w, np.float32)
+    if cu_seqlens is not None:
+        cu_seqlens = _c(cu_seqlens, np.int32)
+        n_seq = cu_seqlens.shape[0] - 1
+    else:
+        n_seq = 1 if num_seqs is None else int(num_seqs)
+    S0 = _c(S0, np.float32)
+    d_out = _c(d_out, np.float64)
+    d_S_final = _c(d_S_final, np.float64)
+    g = {"dq": np.zeros((n_tok, H, dk)), "dk": np.zeros((n_tok, H, dk)), "dv": np.zeros((n_tok, H, dv)),
+         "d_conv_w": np.zeros(conv_w.shape), "d_a_logit": np.zeros((n_tok, H)),
+         "d_b_logit": np.zeros((n_tok, H)), "d_A": np.zeros(H), "d_b_alpha": np.zeros(H),
+         "d_z": np.zeros((n_tok, H, dv)), "d_norm_w": np.zeros(dv), "d_S0": np.zeros((n_seq, H, dk, dv))}
+    rc = lib().gdn_oracle_backward(
+        n_seq, n_tok, H, dk, dv, K, dt, _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w), _ptr(a_logit),
+        _ptr(b_logit), _ptr(A), _ptr(b_alpha), _ptr(z), _ptr(norm_w), _ptr(S0), _ptr(cu_seqlens),
+        _ptr(d_out), _ptr(d_S_final), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["d_conv_w"]),
+        _ptr(g["d_a_logit"]), _ptr(g["d_b_logit"]), _ptr(g["d_A"]), _ptr(g["d_b_alpha"]), _ptr(g["d_z"]),
+        _ptr(g["d_norm_w"]), _ptr(g["d_S0"]), int(n_threads))
+    if rc != 0:
+        raise ValueError("oracle backward rejected its arguments")
+    return g

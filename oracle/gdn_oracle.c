@@ -366,3 +366,268 @@ int gdn_oracle_gated_rmsnorm(int n, int dv, const double *y, const double *z, co
         gated_rmsnorm(dv, y + (size_t)r * dv, z + (size_t)r * dv, w, o + (size_t)r * dv);
     return 0;
 }
+
+/* ------------------------------------------------------------------ backward */
+
+static double dsilu(double x)   /* d/dx [x sigmoid(x)] */
+{
+    const double s = sigmoid(x);
+    return s * (1.0 + x * (1.0 - s));
+}
+
+/*
+ * Gradients of L = <d_out, out> + <d_S_final, S_final> for the prefill above, with
+ * respect to every input: the reverse-mode derivative of each forward step, taken
+ * in the reverse order of the tokens.  Per token t of a sequence (one head), with
+ * P = S_{t-1} (the state before the token), e = v - alpha P^T k, S_t = alpha P +
+ * beta k e^T, y = S_t^T q, n = y r, r = (mean y^2 + eps)^{-1/2},
+ * o = sigmoid(z) n (1 + w), and D the gradient of S_t:
+ *   dz = do n (1 + w) s'(z);  dw += do sigmoid(z) n;  dn = do sigmoid(z) (1 + w);
+ *   dy = r dn - r^3 y mean(dn y);           D += q dy^T;  dq = S_t dy;
+ *   de = beta D^T k;  dv = de;  dbeta = k^T D e;
+ *   dk = beta D e - alpha P de;  dalpha = <D, P> - k^T P de;
+ *   gradient of P = alpha D - alpha k de^T.
+ * Gates: alpha = exp(g), g = -e^A softplus(a + b_alpha): dg = alpha dalpha,
+ * da = dg (-e^A) sigmoid(a + b_alpha), dA += dg g, db_alpha += da; beta =
+ * sigmoid(b): db = dbeta beta (1 - beta).  L2Norm x -> x rho, rho = (|x|^2 +
+ * eps)^{-1/2}: dx = rho dxh - rho^3 x (x . dxh).  SiLU: du/dx = sigmoid(x)(1 + x
+ * (1 - sigmoid(x))).  ShortConv (tap j of K on token t - (K-1) + j): d_raw[t - (K-1)
+ * + j] += w_j dx_t and dw_j += dx_t raw[t - (K-1) + j], inside the sequence.
+ *
+ * Shapes as gdn_oracle_prefill; d_out [N_tok,H,dv] and d_S_final [N_seq,H,dk,dv]
+ * (or NULL = 0) in double.  Outputs in double: dq, dk [N_tok,H,dk], dv, dz
+ * [N_tok,H,dv], d_a, d_b [N_tok,H], d_conv_w [H(2dk+dv),K], d_A, d_b_alpha [H],
+ * d_norm_w [dv], d_S0 [N_seq,H,dk,dv].  Every state of a sequence is kept, so this
+ * is for small inputs.  Returns 0, or -1 on bad sizes.
+ */
+int gdn_oracle_backward(int n_seq, int n_tok, int H, int dk, int dv, int K, int in_dtype,
+                        const void *q, const void *k, const void *v, const float *conv_w,
+                        const void *a_logit, const void *b_logit, const float *A,
+                        const float *b_alpha, const void *z, const float *norm_w,
+                        const float *S0, const int32_t *cu_seqlens, const double *d_out,
+                        const double *d_S_final, double *dq, double *dk_out, double *dv_out,
+                        double *d_conv_w, double *d_a, double *d_b, double *d_A,
+                        double *d_b_alpha, double *d_z, double *d_norm_w, double *d_S0,
+                        int n_threads)
+{
+    if (n_seq <= 0 || n_tok < 0 || H <= 0 || dk <= 0 || dv <= 0 || K <= 0)
+        return -1;
+    if (!cu_seqlens && n_tok % n_seq != 0)
+        return -1;
+    set_threads(n_threads);
+    const size_t C = (size_t)H * (2 * dk + dv);
+    const long pairs = (long)n_seq * H;
+    /* per (sequence, head) partial sums of the parameter gradients */
+    double *part_w = calloc((size_t)pairs * (2 * dk + dv) * K, sizeof(double));
+    double *part_norm = calloc((size_t)pairs * dv, sizeof(double));
+    double *part_A = calloc((size_t)pairs, sizeof(double));
+    double *part_ba = calloc((size_t)pairs, sizeof(double));
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (long ph = 0; ph < pairs; ++ph) {
+        const int n = (int)(ph / H), h = (int)(ph % H);
+        const long t0 = cu_seqlens ? cu_seqlens[n] : (long)n * (n_tok / n_seq);
+        const long t1 = cu_seqlens ? cu_seqlens[n + 1] : (long)(n + 1) * (n_tok / n_seq);
+        if (t0 < 0 || t1 < t0 || t1 > n_tok) {
+            bad = 1;
+            continue;
+        }
+        const long T = t1 - t0;
+        const int wd[3] = {dk, dk, dv};
+        const void *src[3] = {q, k, v};
+        const size_t row_elems[3] = {(size_t)H * dk, (size_t)H * dk, (size_t)H * dv};
+        const size_t col[3] = {(size_t)h * dk, (size_t)h * dk, (size_t)h * dv};
+        const size_t chan[3] = {(size_t)h * dk, (size_t)H * dk + (size_t)h * dk,
+                                (size_t)2 * H * dk + (size_t)h * dv};
+        /* forward, keeping what the reverse sweep needs */
+        double *x[3], *u[3], *dx[3];
+        for (int s = 0; s < 3; ++s) {
+            x[s] = malloc(sizeof(double) * (size_t)(T ? T : 1) * wd[s]);    /* conv outputs */
+            u[s] = malloc(sizeof(double) * (size_t)(T ? T : 1) * wd[s]);    /* SiLU(x), normalised for q, k */
+            dx[s] = calloc((size_t)(T ? T : 1) * wd[s], sizeof(double));     /* gradient of x */
+        }
+        double *rho = malloc(sizeof(double) * (size_t)(T ? T : 1) * 2);     /* L2Norm factors of q, k */
+        double *al = malloc(sizeof(double) * (size_t)(T ? T : 1)), *be = malloc(sizeof(double) * (size_t)(T ? T : 1));
+        double *gl = malloc(sizeof(double) * (size_t)(T ? T : 1)), *ain = malloc(sizeof(double) * (size_t)(T ? T : 1));
+        double *P = malloc(sizeof(double) * (size_t)(T ? T : 1) * dk * dv);  /* state before each token */
+        double *E = malloc(sizeof(double) * (size_t)(T ? T : 1) * dv);       /* e of each token */
+        double *Y = malloc(sizeof(double) * (size_t)(T ? T : 1) * dv);       /* y of each token */
+        double *S = calloc((size_t)dk * dv, sizeof(double));
+        if (S0)
+            for (size_t i = 0; i < (size_t)dk * dv; ++i)
+                S[i] = (double)S0[((size_t)n * H + h) * dk * dv + i];
+        const double eA = exp((double)A[h]);
+        for (long t = 0; t < T; ++t) {
+            const long tt = t0 + t;
+            for (int s = 0; s < 3; ++s) {
+                shortconv_prefill(src[s], in_dtype, row_elems[s], col[s], conv_w, chan[s], K, tt,
+                                  t0, wd[s], x[s] + (size_t)t * wd[s]);
+                for (int i = 0; i < wd[s]; ++i)
+                    u[s][(size_t)t * wd[s] + i] = silu(x[s][(size_t)t * wd[s] + i]);
+            }
+            for (int s = 0; s < 2; ++s) {
+                double ss = 0.0;
+                for (int i = 0; i < dk; ++i)
+                    ss += u[s][(size_t)t * dk + i] * u[s][(size_t)t * dk + i];
+                rho[t * 2 + s] = 1.0 / sqrt(ss + ORACLE_EPS);
+            }
+            const size_t gi = (size_t)tt * H + h;
+            ain[t] = load_elem(a_logit, in_dtype, gi) + (double)b_alpha[h];
+            gl[t] = -eA * softplus(ain[t]);
+            al[t] = exp(gl[t]);
+            be[t] = write_gate(load_elem(b_logit, in_dtype, gi));
+            double qh[dk], kh[dk];
+            for (int i = 0; i < dk; ++i) {
+                qh[i] = u[0][(size_t)t * dk + i] * rho[t * 2];
+                kh[i] = u[1][(size_t)t * dk + i] * rho[t * 2 + 1];
+            }
+            memcpy(P + (size_t)t * dk * dv, S, sizeof(double) * dk * dv);
+            delta_rule_step(S, dk, dv, qh, kh, u[2] + (size_t)t * dv, al[t], be[t],
+                            E + (size_t)t * dv, Y + (size_t)t * dv);
+        }
+        /* reverse sweep */
+        double *D = calloc((size_t)dk * dv, sizeof(double));
+        double *St = malloc(sizeof(double) * (size_t)dk * dv);
+        if (d_S_final)
+            memcpy(D, d_S_final + ((size_t)n * H + h) * dk * dv, sizeof(double) * dk * dv);
+        for (long t = T - 1; t >= 0; --t) {
+            const long tt = t0 + t;
+            const size_t gi = (size_t)tt * H + h;
+            const double *Pt = P + (size_t)t * dk * dv, *e = E + (size_t)t * dv, *y = Y + (size_t)t * dv;
+            const double alpha = al[t], beta = be[t];
+            double qh[dk], kh[dk], dy[dv], dqh[dk], dkh[dk], de[dv], De[dk];
+            for (int i = 0; i < dk; ++i) {
+                qh[i] = u[0][(size_t)t * dk + i] * rho[t * 2];
+                kh[i] = u[1][(size_t)t * dk + i] * rho[t * 2 + 1];
+            }
+            /* output stage */
+            double ms = 0.0, dny = 0.0;
+            for (int j = 0; j < dv; ++j)
+                ms += y[j] * y[j];
+            const double r = 1.0 / sqrt(ms / dv + ORACLE_EPS);
+            double dn[dv];
+            for (int j = 0; j < dv; ++j) {
+                const double zj = load_elem(z, in_dtype, gi * dv + j), sz = sigmoid(zj);
+                const double doj = d_out[gi * dv + j], nj = y[j] * r, gain = 1.0 + (double)norm_w[j];
+                d_z[gi * dv + j] = doj * nj * gain * sz * (1.0 - sz);
+                part_norm[(size_t)ph * dv + j] += doj * sz * nj;
+                dn[j] = doj * sz * gain;
+                dny += dn[j] * y[j];
+            }
+            for (int j = 0; j < dv; ++j)
+                dy[j] = r * dn[j] - r * r * r * y[j] * dny / dv;
+            /* the update */
+            for (int i = 0; i < dk; ++i)
+                for (int j = 0; j < dv; ++j)
+                    St[(size_t)i * dv + j] = alpha * Pt[(size_t)i * dv + j] + beta * kh[i] * e[j];
+            for (int i = 0; i < dk; ++i)
+                for (int j = 0; j < dv; ++j)
+                    D[(size_t)i * dv + j] += qh[i] * dy[j];
+            for (int i = 0; i < dk; ++i) {
+                double s = 0.0;
+                for (int j = 0; j < dv; ++j)
+                    s += St[(size_t)i * dv + j] * dy[j];
+                dqh[i] = s;
+            }
+            for (int j = 0; j < dv; ++j) {
+                double s = 0.0;
+                for (int i = 0; i < dk; ++i)
+                    s += D[(size_t)i * dv + j] * kh[i];
+                de[j] = beta * s;
+            }
+            double dbeta = 0.0, dalpha = 0.0;
+            for (int i = 0; i < dk; ++i) {
+                double s = 0.0, pde = 0.0;
+                for (int j = 0; j < dv; ++j) {
+                    s += D[(size_t)i * dv + j] * e[j];
+                    pde += Pt[(size_t)i * dv + j] * de[j];
+                }
+                De[i] = s;
+                dbeta += kh[i] * s;
+                dkh[i] = beta * s - alpha * pde;
+                dalpha -= kh[i] * pde;
+            }
+            for (size_t i = 0; i < (size_t)dk * dv; ++i)
+                dalpha += D[i] * Pt[i];
+            for (int i = 0; i < dk; ++i)
+                for (int j = 0; j < dv; ++j)
+                    D[(size_t)i * dv + j] = alpha * D[(size_t)i * dv + j] - alpha * kh[i] * de[j];
+            /* gates */
+            const double dg = alpha * dalpha;
+            const double da = dg * (-eA) * sigmoid(ain[t]);
+            d_a[gi] = da;
+            part_A[ph] += dg * gl[t];
+            part_ba[ph] += da;
+            d_b[gi] = dbeta * beta * (1.0 - beta);
+            /* L2Norm and SiLU of q, k; SiLU of v */
+            const double *dxh[2] = {dqh, dkh};
+            for (int s = 0; s < 2; ++s) {
+                const double *uu = u[s] + (size_t)t * dk, rh = rho[t * 2 + s];
+                double dot = 0.0;
+                for (int i = 0; i < dk; ++i)
+                    dot += uu[i] * dxh[s][i];
+                for (int i = 0; i < dk; ++i) {
+                    const double du = rh * dxh[s][i] - rh * rh * rh * uu[i] * dot;
+                    dx[s][(size_t)t * dk + i] = du * dsilu(x[s][(size_t)t * dk + i]);
+                }
+            }
+            for (int j = 0; j < dv; ++j)
+                dx[2][(size_t)t * dv + j] = de[j] * dsilu(x[2][(size_t)t * dv + j]);
+        }
+        if (d_S0)
+            memcpy(d_S0 + ((size_t)n * H + h) * dk * dv, D, sizeof(double) * dk * dv);
+        /* ShortConv */
+        double *outs[3] = {dq, dk_out, dv_out};
+        for (int s = 0; s < 3; ++s) {
+            for (long t = 0; t < T; ++t)
+                for (int i = 0; i < wd[s]; ++i)
+                    outs[s][((size_t)(t0 + t)) * row_elems[s] + col[s] + i] = 0.0;
+            for (long t = 0; t < T; ++t)
+                for (int i = 0; i < wd[s]; ++i) {
+                    const double g = dx[s][(size_t)t * wd[s] + i];
+                    const size_t c = chan[s] + i;
+                    for (int j = 0; j < K; ++j) {
+                        const long srct = t - (K - 1) + j;
+                        if (srct < 0)
+                            continue;
+                        const size_t si = (size_t)(t0 + srct) * row_elems[s] + col[s] + i;
+                        outs[s][si] += (double)conv_w[c * K + j] * g;
+                        const size_t li = (s == 0 ? 0 : s == 1 ? (size_t)dk : (size_t)2 * dk) + i;
+                        part_w[((size_t)ph * (2 * dk + dv) + li) * K + j] += g * load_elem(src[s], in_dtype, si);
+                    }
+                }
+        }
+        for (int s = 0; s < 3; ++s) {
+            free(x[s]);
+            free(u[s]);
+            free(dx[s]);
+        }
+        free(rho); free(al); free(be); free(gl); free(ain);
+        free(P); free(E); free(Y); free(S); free(D); free(St);
+    }
+    if (!bad) {
+        memset(d_conv_w, 0, sizeof(double) * C * K);
+        memset(d_norm_w, 0, sizeof(double) * dv);
+        memset(d_A, 0, sizeof(double) * H);
+        memset(d_b_alpha, 0, sizeof(double) * H);
+        for (long ph = 0; ph < pairs; ++ph) {
+            const int h = (int)(ph % H);
+            const size_t chan[3] = {(size_t)h * dk, (size_t)H * dk + (size_t)h * dk,
+                                    (size_t)2 * H * dk + (size_t)h * dv};
+            for (int li = 0; li < 2 * dk + dv; ++li) {
+                const size_t c = li < dk ? chan[0] + li : li < 2 * dk ? chan[1] + (li - dk) : chan[2] + (li - 2 * dk);
+                for (int j = 0; j < K; ++j)
+                    d_conv_w[c * K + j] += part_w[((size_t)ph * (2 * dk + dv) + li) * K + j];
+            }
+            for (int j = 0; j < dv; ++j)
+                d_norm_w[j] += part_norm[(size_t)ph * dv + j];
+            d_A[h] += part_A[ph];
+            d_b_alpha[h] += part_ba[ph];
+        }
+    }
+    free(part_w);
+    free(part_norm);
+    free(part_A);
+    free(part_ba);
+    return bad ? -1 : 0;
+}
