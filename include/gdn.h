@@ -123,6 +123,45 @@ GDN_API gdn_status_t gdn_prefill(const gdn_dims_t *dims, const void *q, const vo
 GDN_API gdn_status_t gdn_prefill_workspace_size(const gdn_dims_t *dims, size_t *bytes);
 
 /*
+ * gdn_prefill_backward -- gradients of L = <d_out, out> + <d_S_final, S_final>
+ * for the gdn_prefill call with the same arguments, with respect to every
+ * input: the reverse-mode derivative of the forward the two web write-ups
+ * define (slinene.github.io write-up of "On the Design of Qwen3.8-Next
+ * Architecture", 模块 A: 递归状态, 参数化; paper.rainbus.top digest, 方法步骤详情
+ * step (1)).  Per token, with P the state before it, e = v - alpha P^T k and D
+ * the gradient of the state after it: D += q dy^T, dv = beta D^T k,
+ * dk = beta D e - alpha P dv, dq = S dy, dbeta = k^T D e,
+ * dalpha = <D, P> - k^T P dv, and the state before receives alpha (D - k dv^T);
+ * then the gates, L2Norm, SiLU and the short convolution in reverse.
+ *
+ * Forward inputs as gdn_prefill (q, k, v, z, a_logit, b_logit in fp32 here:
+ * dims->in_dtype and dims->out_dtype must be GDN_F32; dk = dv in {64, 128}).
+ *   d_out      [N_tok, H, dv] fp32 gradient of out
+ *   d_S_final  [N_seq, H, dk, dv] fp32 gradient of S_final, or NULL for zeros
+ * Written, fp32, same shapes as the inputs they belong to:
+ *   dq, dk [N_tok, H, dk]; dv, d_z [N_tok, H, dv]; d_a_logit, d_b_logit
+ *   [N_tok, H]; d_conv_w [H(2dk+dv), 4]; d_A, d_b_alpha [H]; d_norm_w [dv];
+ *   d_S0 [N_seq, H, dk, dv], or NULL when not wanted.
+ * Token tensors may be NULL only when total_tokens is 0; every pointer 16-byte
+ * aligned except the [H] and [N_tok, H] arrays (4-byte).  No output may alias an
+ * input.  The results do not depend on scheduling (every sum has a fixed order).
+ * The call recomputes the forward (states checkpointed every 16 tokens) and takes
+ * a stream-ordered workspace of gdn_prefill_backward_workspace_size() bytes from
+ * the library's private pool of the current device, returned on `stream`.
+ * GDN_ERR_UNSUPPORTED for bf16 tensors or dk != dv.
+ */
+GDN_API gdn_status_t gdn_prefill_backward(
+    const gdn_dims_t *dims, const void *q, const void *k, const void *v, const float *conv_w,
+    const void *a_logit, const void *b_logit, const float *A, const float *b_alpha, const void *z,
+    const float *norm_w, const float *S0, const int32_t *cu_seqlens, const void *d_out,
+    const float *d_S_final, void *dq, void *dk, void *dv, float *d_conv_w, void *d_a_logit,
+    void *d_b_logit, float *d_A, float *d_b_alpha, void *d_z, float *d_norm_w, float *d_S0,
+    gdn_stream_t stream);
+
+/* Bytes of device workspace one gdn_prefill_backward call with these dims uses (host call). */
+GDN_API gdn_status_t gdn_prefill_backward_workspace_size(const gdn_dims_t *dims, size_t *bytes);
+
+/*
  * gdn_decode_step -- one token for each of B = dims->num_seqs sequences,
  * reading and updating the per-head state in place.
  *

@@ -370,6 +370,89 @@ gdn_status_t gdn_prefill(const gdn_dims_t *dims, const void *q, const void *k, c
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
+gdn_status_t gdn_prefill_backward_workspace_size(const gdn_dims_t *dims, size_t *bytes) {
+    gdn_status_t st = check_dims(dims, false);
+    if (st != GDN_OK) return st;
+    if (!bytes) return GDN_ERR_INVALID_ARG;
+    if (dims->in_dtype != GDN_F32 || dims->out_dtype != GDN_F32 || dims->dk != dims->dv)
+        return GDN_ERR_UNSUPPORTED;
+    *bytes = gdn::backward_workspace_bytes(dims->num_seqs, dims->total_tokens, dims->H, dims->dk);
+    return GDN_OK;
+}
+
+gdn_status_t gdn_prefill_backward(const gdn_dims_t *dims, const void *q, const void *k, const void *v,
+                                  const float *conv_w, const void *a_logit, const void *b_logit,
+                                  const float *A, const float *b_alpha, const void *z, const float *norm_w,
+                                  const float *S0, const int32_t *cu_seqlens, const void *d_out,
+                                  const float *d_S_final, void *dq, void *dk, void *dv, float *d_conv_w,
+                                  void *d_a_logit, void *d_b_logit, float *d_A, float *d_b_alpha, void *d_z,
+                                  float *d_norm_w, float *d_S0, gdn_stream_t stream) {
+    tl_launches = 0;
+    gdn_status_t st = check_dims(dims, false);
+    if (st != GDN_OK) return st;
+    if (dims->in_dtype != GDN_F32 || dims->out_dtype != GDN_F32 || dims->dk != dims->dv)
+        return GDN_ERR_UNSUPPORTED;
+    if (!cu_seqlens && dims->total_tokens % dims->num_seqs != 0) return GDN_ERR_INVALID_ARG;
+    const bool no_tokens = dims->total_tokens == 0;
+    const void *tok[] = {q, k, v, z, d_out, dq, dk, dv, d_z};
+    for (const void *p : tok) {
+        if (!p && !no_tokens) return GDN_ERR_INVALID_ARG;
+        if (p && !aligned16(p)) return GDN_ERR_ALIGNMENT;
+    }
+    const void *per_tok[] = {a_logit, b_logit, d_a_logit, d_b_logit};
+    for (const void *p : per_tok) {
+        if (!p && !no_tokens) return GDN_ERR_INVALID_ARG;
+        if (p && !aligned_to(p, 4)) return GDN_ERR_ALIGNMENT;
+    }
+    const void *need16[] = {conv_w, d_conv_w, norm_w, d_norm_w};
+    for (const void *p : need16) {
+        if (!p) return GDN_ERR_INVALID_ARG;
+        if (!aligned16(p)) return GDN_ERR_ALIGNMENT;
+    }
+    const void *need4[] = {A, b_alpha, d_A, d_b_alpha};
+    for (const void *p : need4) {
+        if (!p) return GDN_ERR_INVALID_ARG;
+        if (!aligned_to(p, 4)) return GDN_ERR_ALIGNMENT;
+    }
+    const void *opt[] = {S0, d_S_final, d_S0};
+    for (const void *p : opt)
+        if (p && !aligned16(p)) return GDN_ERR_ALIGNMENT;
+    if (cu_seqlens && !aligned_to(cu_seqlens, 4)) return GDN_ERR_ALIGNMENT;
+
+    gdn::BackwardArgs b;
+    gdn::PrefillArgs &a = b.f;
+    a.n_seq = dims->num_seqs;
+    a.n_tok = dims->total_tokens;
+    a.H = dims->H;
+    a.dk = dims->dk;
+    a.dv = dims->dv;
+    a.in_bf16 = false;
+    a.out_bf16 = false;
+    a.q = q; a.k = k; a.v = v; a.z = z; a.a_logit = a_logit; a.b_logit = b_logit;
+    a.conv_w = conv_w; a.A = A; a.b_alpha = b_alpha; a.norm_w = norm_w; a.S0 = S0;
+    a.cu_seqlens = cu_seqlens;
+    a.out = nullptr;
+    a.S_final = nullptr;
+    a.stream = reinterpret_cast<cudaStream_t>(stream);
+    b.d_out = d_out;
+    b.d_S_final = d_S_final;
+    b.dq = dq; b.dk = dk; b.dv = dv; b.d_a_logit = d_a_logit; b.d_b_logit = d_b_logit; b.d_z = d_z;
+    b.d_conv_w = d_conv_w; b.d_A = d_A; b.d_b_alpha = d_b_alpha; b.d_norm_w = d_norm_w; b.d_S0 = d_S0;
+
+    const size_t ws_bytes = gdn::backward_workspace_bytes(a.n_seq, a.n_tok, a.H, a.dk);
+    char *ws = nullptr;
+    cudaMemPool_t pool;
+    if (get_pool(&pool) != cudaSuccess) return GDN_ERR_CUDA;
+    if (cudaMallocFromPoolAsync(reinterpret_cast<void **>(&ws), ws_bytes, pool, a.stream) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    cudaError_t e = record(g_ev_begin, a.stream);
+    if (e == cudaSuccess) e = gdn::launch_backward(b, ws);
+    if (e == cudaSuccess) e = record(g_ev_end, a.stream);
+    cudaError_t ef = cudaFreeAsync(ws, a.stream);
+    if (e == cudaSuccess) e = ef;
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
 gdn_status_t gdn_decode_step(const gdn_dims_t *dims, const void *q, const void *k,
                              const void *v, const float *conv_w, void *conv_hist,
                              const void *a_logit, const void *b_logit, const float *A,

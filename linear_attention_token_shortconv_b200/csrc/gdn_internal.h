@@ -66,6 +66,19 @@ struct TmaMap { alignas(64) unsigned char bytes[128]; };
 cudaError_t make_tma_3d(TmaMap *out, const void *base, bool bf16, int inner, int H, int n_tok,
                         int box_inner, int box_rows, bool swizzle128);
 
+// K4: prefill backward (fp32 inputs, dk = dv in {64, 128}); `f` holds the forward's
+// inputs (f.out and f.S_final are unused), the rest the incoming and outgoing
+// gradients, all fp32.
+struct BackwardArgs {
+    PrefillArgs f;
+    const void *d_out;
+    const float *d_S_final;
+    void *dq, *dk, *dv, *d_a_logit, *d_b_logit, *d_z;
+    float *d_conv_w, *d_A, *d_b_alpha, *d_norm_w, *d_S0;
+};
+size_t backward_workspace_bytes(int n_seq, int n_tok, int H, int D);
+cudaError_t launch_backward(const BackwardArgs &b, void *ws);
+
 // K2f: token-by-token recurrence with the fused gates and output stage (SIMT fp32).
 cudaError_t launch_recurrent(const PrefillArgs &a, const float *qn, const float *kn,
                              const float *vn);

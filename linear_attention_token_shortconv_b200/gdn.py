@@ -24,7 +24,8 @@ STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "G
 EXPORTS = ("gdn_prefill", "gdn_prefill_workspace_size", "gdn_decode_step", "gdn_status_string",
            "gdn_set_timing_events", "gdn_selftest_umma", "gdn_prefill_noalloc",
            "gdn_set_kernel_events", "gdn_last_call_launches", "gdn_device_error_status",
-           "gdn_selftest_wait_timeout", "gdn_decode_multi")
+           "gdn_selftest_wait_timeout", "gdn_decode_multi", "gdn_prefill_backward",
+           "gdn_prefill_backward_workspace_size")
 ERRF_PREP, ERRF_CHAIN, ERRF_DECODE = 1, 2, 4
 
 
@@ -61,6 +62,10 @@ def load() -> ctypes.CDLL:
         lib.gdn_decode_step.restype = ctypes.c_int
         lib.gdn_decode_multi.argtypes = [D, ctypes.c_int] + [P] * 15
         lib.gdn_decode_multi.restype = ctypes.c_int
+        lib.gdn_prefill_backward.argtypes = [D] + [P] * 26
+        lib.gdn_prefill_backward.restype = ctypes.c_int
+        lib.gdn_prefill_backward_workspace_size.argtypes = [D, ctypes.POINTER(ctypes.c_size_t)]
+        lib.gdn_prefill_backward_workspace_size.restype = ctypes.c_int
         lib.gdn_prefill_noalloc.argtypes = [D] + [P] * 15
         lib.gdn_prefill_noalloc.restype = ctypes.c_int
         lib.gdn_selftest_umma.argtypes = [ctypes.c_int] * 5 + [P] * 5
@@ -132,6 +137,44 @@ def prefill(q, k, v, conv_w, a_logit, b_logit, A, b_alpha, z, norm_w, S0=None, c
                             _stream(stream))
     _check(rc, "gdn_prefill")
     return out, S_final
+
+
+def prefill_backward(q, k, v, conv_w, a_logit, b_logit, A, b_alpha, z, norm_w, d_out, S0=None,
+                     d_S_final=None, cu_seqlens=None, *, num_seqs=None, want_d_S0=True, stream=None):
+    """gdn_prefill_backward on fp32 torch tensors (same layouts as `prefill`).
+
+    Returns a dict of fp32 tensors: dq, dk, dv, d_conv_w, d_a_logit, d_b_logit,
+    d_A, d_b_alpha, d_z, d_norm_w and d_S0 (None unless wanted)."""
+    n_tok, H, dk = q.shape
+    dv = v.shape[2]
+    if cu_seqlens is not None:
+        n_seq = cu_seqlens.shape[0] - 1
+    else:
+        n_seq = num_seqs if num_seqs is not None else (S0.shape[0] if S0 is not None else 1)
+    dev, f32 = q.device, torch.float32
+    g = {"dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),
+         "d_conv_w": torch.empty_like(conv_w), "d_a_logit": torch.empty_like(a_logit),
+         "d_b_logit": torch.empty_like(b_logit), "d_A": torch.empty_like(A),
+         "d_b_alpha": torch.empty_like(b_alpha), "d_z": torch.empty_like(z),
+         "d_norm_w": torch.empty_like(norm_w),
+         "d_S0": torch.empty((n_seq, H, dk, dv), dtype=f32, device=dev) if want_d_S0 else None}
+    dims = Dims(n_seq, n_tok, H, dk, dv, conv_w.shape[1], _dt(q), _dt(d_out))
+    rc = load().gdn_prefill_backward(
+        ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w), _ptr(a_logit), _ptr(b_logit),
+        _ptr(A), _ptr(b_alpha), _ptr(z), _ptr(norm_w), _ptr(S0), _ptr(cu_seqlens), _ptr(d_out),
+        _ptr(d_S_final), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["d_conv_w"]),
+        _ptr(g["d_a_logit"]), _ptr(g["d_b_logit"]), _ptr(g["d_A"]), _ptr(g["d_b_alpha"]), _ptr(g["d_z"]),
+        _ptr(g["d_norm_w"]), _ptr(g["d_S0"]), _stream(stream))
+    _check(rc, "gdn_prefill_backward")
+    return g
+
+
+def prefill_backward_workspace_size(n_seq, n_tok, H, dk, dv, conv_k=4) -> int:
+    dims = Dims(n_seq, n_tok, H, dk, dv, conv_k, GDN_F32, GDN_F32)
+    n = ctypes.c_size_t(0)
+    _check(load().gdn_prefill_backward_workspace_size(ctypes.byref(dims), ctypes.byref(n)),
+           "gdn_prefill_backward_workspace_size")
+    return n.value
 
 
 def prefill_noalloc(q, k, v, conv_w, a_logit, b_logit, A, b_alpha, z, norm_w, S0=None,

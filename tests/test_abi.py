@@ -140,3 +140,37 @@ def test_decode_multi_argument_validation(lib):
     bad[13] = ctypes.c_void_p(4098)                                   # n_keep misaligned
     assert lib.gdn_decode_multi(ctypes.byref(ok), 2, *bad) == 3
     assert lib.gdn_last_call_launches() == 0
+
+
+def _bwd_args(**over):
+    names = ["q", "k", "v", "conv_w", "a", "b", "A", "b_alpha", "z", "norm_w", "S0", "cu", "d_out", "d_S_final",
+             "dq", "dk", "dv", "d_conv_w", "d_a", "d_b", "d_A", "d_b_alpha", "d_z", "d_norm_w", "d_S0", "stream"]
+    vals = {n: ctypes.c_void_p(4096 * (i + 1)) for i, n in enumerate(names)}
+    for n in ("S0", "cu", "d_S_final", "d_S0", "stream"):
+        vals[n] = None
+    vals.update(over)
+    return [vals[n] for n in names]
+
+
+def test_backward_argument_validation(lib):
+    f32 = dict(in_dtype=0, out_dtype=0)
+    bwd = lambda dims, **kw: lib.gdn_prefill_backward(ctypes.byref(dims), *_bwd_args(**kw))
+    assert lib.gdn_prefill_backward(None, *_bwd_args()) == 1
+    assert bwd(_dims(in_dtype=1, out_dtype=0)) == 2                 # bf16 inputs
+    assert bwd(_dims(dk=128, dv=64, **f32)) == 2                     # dk != dv
+    assert bwd(_dims(num_seqs=3, total_tokens=64, **f32)) == 1       # not divisible, no cu
+    assert bwd(_dims(**f32), q=None) == 1
+    assert bwd(_dims(**f32), dq=None) == 1
+    assert bwd(_dims(**f32), d_conv_w=None) == 1
+    assert bwd(_dims(**f32), d_out=ctypes.c_void_p(4104)) == 3
+    assert bwd(_dims(**f32), d_a=ctypes.c_void_p(4098)) == 3
+    assert bwd(_dims(**f32), d_S0=ctypes.c_void_p(4100)) == 3
+    assert lib.gdn_last_call_launches() == 0
+
+
+def test_backward_workspace_size_query(lib):
+    n = gdn.prefill_backward_workspace_size(2, 1000, 4, 128, 128)
+    # q, k, v and their gradients in fp32, plus one 64 KB checkpoint per 16 tokens
+    assert n >= 6 * 1000 * 4 * 128 * 4 + (1000 // 16) * 4 * 128 * 128 * 4
+    with pytest.raises(gdn.GdnError):
+        gdn.prefill_backward_workspace_size(1, 10, 1, 128, 64)
