@@ -32,7 +32,7 @@ sys.path.insert(0, ROOT)
 
 from linear_attention_token_shortconv_b200 import dist as rankio  # noqa: E402
 from linear_attention_token_shortconv_b200 import gdn  # noqa: E402
-from linear_attention_token_shortconv_b200.workloads import (DECODE, LONG, make_decode_inputs,  # noqa: E402
+from linear_attention_token_shortconv_b200.workloads import (DECODE, LONG, PRETRAIN, make_decode_inputs,  # noqa: E402
                                                              make_prefill_inputs, to_oracle_bits)
 
 METRIC = "GDN prefill tokens/s at T=32K H=32 (% TC peak); decode state GB/s (% HBM)"
@@ -41,6 +41,16 @@ METRIC = "GDN prefill tokens/s at T=32K H=32 (% TC peak); decode state GB/s (% H
 # logits and a bf16 output.
 PREFILL_FLOP_PER_TOKEN_HEAD = 64 * (6 * 128 + 4 * 128) + 6 * 128 * 128   # 180,224
 PREFILL_BYTES_PER_TOKEN_HEAD = 4 * 128 * 2 + 2 * 2 + 128 * 2           # 1,284
+# Backward (fp32, d = 128), per token-head.  Bytes that must move: q, k, v, z and
+# d_out read, dq, dk, dv and d_z written (fp32 rows of 128), two gate logits read
+# and their two gradients written: 4,624 B.  SIMT arithmetic of the token-level
+# recurrence: the forward step re-run (S^T k, S^T q, the update: 6 d^2 flop) and
+# the backward step (D += q dy^T, D^T k, P dy, P de, D e, <D, P>, the decay of D:
+# 14 d^2 flop) = 20 d^2 = 327,680 flop.
+BACKWARD_BYTES_PER_TOKEN_HEAD = 9 * 128 * 4 + 4 * 4
+BACKWARD_FLOP_PER_TOKEN_HEAD = 20 * 128 * 128
+# fp32 SIMT peak: 148 SMs x 128 fp32 lanes x 2 flop (FMA) x 1.965 GHz (max SM clock)
+FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # Per-kernel roofline units (a few (sequence, head) chains run as one fused
 # persistent kernel; many chains as chunk_prep / chunk_chain launches per
 # segment).  chunk_prep reads q, k, v and the two logits: 772 of
@@ -331,6 +341,38 @@ def bench_decode(cfg, steps, dev):
     return ms, kern_ms, state_bytes, launches, clk.summary()
 
 
+def bench_backward(steps, dev):
+    """gdn_prefill_backward on the pretraining shape (4 sequences x 4096 tokens,
+    H = 16, d = 128) in fp32, gradients of every input; inputs (0.54 GB of fp32
+    token rows plus d_out) are larger than L2."""
+    cfg = replace(PRETRAIN, in_dtype=torch.float32)
+    inp = make_prefill_inputs(cfg, dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(cfg.seed + 100)
+    d_out = torch.randn((cfg.total_tokens, cfg.H, cfg.dv), generator=g, device=dev)
+
+    def call():
+        return gdn.prefill_backward(inp["q"], inp["k"], inp["v"], inp["conv_w"], inp["a_logit"], inp["b_logit"],
+                                    inp["A"], inp["b_alpha"], inp["z"], inp["norm_w"], d_out, S0=inp.get("S0"),
+                                    num_seqs=cfg.num_seqs)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches = 0
+    s.record()
+    for _ in range(steps):
+        call()
+        launches += gdn.last_call_launches()
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / steps
+    del inp, d_out
+    torch.cuda.empty_cache()
+    return cfg, ms, launches
+
+
 def bench_decode_multi(cfg, T, steps, dev):
     """T consecutive tokens per sequence per step (gdn_decode_multi, all committed):
     the pool's entries [0, T) and [T, 2T) as two alternating multi-token inputs."""
@@ -492,6 +534,19 @@ def main():
                             "frac": gbs / pk["hbm_gbs"], "state_bytes_per_step": sbytes,
                             "kernel": "decode_stream", "gpu_launches": dlaunch, "clocks": dclk}
         torch.cuda.empty_cache()
+        bcfg, b_ms, blaunch = bench_backward(5, dev)
+        th = bcfg.total_tokens * bcfg.H
+        b_tf = BACKWARD_FLOP_PER_TOKEN_HEAD * th / (b_ms * 1e-3) / 1e12
+        b_gbs = BACKWARD_BYTES_PER_TOKEN_HEAD * th / (b_ms * 1e-3) / 1e9
+        result["backward"] = {"workload": "prefill backward, pretraining shape B=4 x T=4096, H=16, d=128, fp32, "
+                                          "gradients of every input",
+                              "steps": 5, "ms_per_step": b_ms, "tokens_per_s": bcfg.total_tokens / (b_ms * 1e-3),
+                              "bound": "alu", "achieved_tflops": b_tf, "peak_tflops": FP32_SIMT_TFLOPS,
+                              "peak_kind": "derived: 148 SMs x 128 fp32 lanes x 2 x 1.965 GHz",
+                              "frac": b_tf / FP32_SIMT_TFLOPS, "flop_per_token_head": BACKWARD_FLOP_PER_TOKEN_HEAD,
+                              "hbm": {"bytes_per_token_head": BACKWARD_BYTES_PER_TOKEN_HEAD, "achieved_gbs": b_gbs,
+                                      "frac": b_gbs / pk["hbm_gbs"]},
+                              "kernel": "bwd_rec_kernel (dominant)", "gpu_launches": blaunch}
         T = 4
         mk_ms, mlaunch = bench_decode_multi(DECODE, T, max(50, args.decode_steps // 4), dev)
         mgbs = sbytes / (mk_ms * 1e-3) / 1e9

@@ -17,21 +17,24 @@
 //
 // Kernels (one launch each):
 //  (prelude)  q_hat, k_hat, v_hat in fp32: the forward's fp32 prelude kernel.
-//  K4a bwd_ckpt_kernel: the forward recurrence of one (sequence, head) per CTA,
-//      storing the state before every 16-token interval (checkpoints).
-//  K4b bwd_recurrence_kernel: one (sequence, head) per CTA, intervals in reverse.
-//      Per interval: the checkpoint is loaded and the interval run forward once,
-//      each state before a token going to a per-CTA scratch (16 x 64 KB, which
-//      stays in L2) with the token's e and y; the output-stage backward of the 16
-//      tokens (one warp per two tokens); then the token steps in reverse, the
-//      state gradient held in registers.  The state is laid out as in the decode
-//      kernel: thread (warp w, lane l) holds rows w + 8 r and columns
-//      (D / 32) l + m.  Column sums go through shared memory across the 8 warps;
-//      row sums are a reduce-scatter across the 32 lanes of a warp.
-//  K4c bwd_prelude_kernel: L2Norm, SiLU and conv backward per channel octet and
+//  K4a bwd_fwd_kernel: the forward recurrence, D / 32 CTAs of 32 state columns per
+//      (sequence, head) (the columns of the recurrence are independent): the
+//      state before every 16-token interval (checkpoints) and each token's e, y.
+//  K4b bwd_epi_kernel: the output-stage backward per token-head: dy, d_z, e . dy
+//      and per-block partial sums of d_norm_w.
+//  K4c bwd_rec_kernel: the reverse sweep, split by columns like K4a.  Per interval
+//      (in reverse) the checkpoint is re-run into an L2-resident scratch, then the
+//      token steps run backwards with the state gradient in registers, laid out
+//      as in the decode kernel (thread (warp w, lane l): rows w + 8 r, column
+//      c0 + l).  Column sums of D^T k cross the 8 warps through shared memory (one
+//      block barrier per token); the row sums P dy, P de, D e over the CTA's
+//      columns are a warp reduce-scatter, written as partials with <D, P>.
+//  K4d bwd_combine_kernel: per token-head, the partials of the column splits give
+//      dq_hat, dk_hat, dbeta and dg.
+//  K4e bwd_prelude_kernel: L2Norm, SiLU and conv backward per channel octet and
 //      64-token tile: d_q, d_k, d_v and per-tile partial sums of d_conv_w.
-//  K4d bwd_gates_kernel: d_a_logit, d_b_logit, and d_A, d_b_alpha per head.
-//  K4e bwd_reduce_kernel: the partial sums of d_conv_w and d_norm_w.
+//  K4f bwd_gates_kernel: d_a_logit, d_b_logit, and d_A, d_b_alpha per head.
+//  K4g bwd_reduce_kernel: the partial sums of d_conv_w and d_norm_w.
 // Every partial sum has a fixed order: the results do not depend on scheduling.
 #include "gdn_device.cuh"
 #include "gdn_internal.h"
@@ -87,17 +90,30 @@ __device__ __forceinline__ void warp_reduce_scatter(float (&v)[N], int lane) {
     }
 }
 
-// ---------------------------------------------------------------- K4a: checkpoints
-template <int D>
-__global__ void __launch_bounds__(bwd::NT, 1)
-bwd_ckpt_kernel(const float *__restrict__ kn, const float *__restrict__ vn, const float *__restrict__ a_logit,
-                const float *__restrict__ b_logit, const float *__restrict__ A, const float *__restrict__ b_alpha,
-                const float *__restrict__ S0, const int32_t *__restrict__ cu, int n_seq, int n_tok, int H,
-                float *__restrict__ ckpt) {
-    constexpr int RPT = D / 8, CPT = D / 32, IV = bwd::IV;
-    __shared__ float kk[IV][D], vv[IV][D], al[IV], be[IV];
-    __shared__ float red[2][8][D];
-    const int h = blockIdx.x, n = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+// Column split: the recurrence of column j of the state (S e_j and its gradient)
+// depends on the other columns only through the output stage (dy), which is
+// computed beforehand from the stored y, and through row sums over the columns,
+// which only produce outputs.  So one (sequence, head) runs as D / DC CTAs of DC
+// columns each; the row sums are written per CTA and combined per token.
+namespace bwd {
+constexpr int DC = 32;   // state columns per CTA
+}  // namespace bwd
+
+// ------------------------------------------------------- K4a: forward + checkpoints
+// The forward recurrence of DC columns of one (sequence, head): the state before
+// every 16-token interval (checkpoints), and each token's e and y (those columns).
+template <int D, int DC>
+__global__ void __launch_bounds__(bwd::NT, 2)
+bwd_fwd_kernel(const float *__restrict__ qn, const float *__restrict__ kn, const float *__restrict__ vn,
+               const float *__restrict__ a_logit, const float *__restrict__ b_logit, const float *__restrict__ A,
+               const float *__restrict__ b_alpha, const float *__restrict__ S0, const int32_t *__restrict__ cu,
+               int n_seq, int n_tok, int H, float *__restrict__ ckpt, float *__restrict__ y_out,
+               float *__restrict__ e_out) {
+    constexpr int RPT = D / 8, CPT = DC / 32, IV = bwd::IV;
+    __shared__ float qq[IV][D], kk[IV][D], vv[IV][DC], al[IV], be[IV], kq[IV];
+    __shared__ float red[2][2][8][DC];
+    const int h = blockIdx.x, n = blockIdx.y, c0 = blockIdx.z * DC;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     int s0, s1;
     bwd_seq_bounds(cu, n_seq, n_tok, n, s0, s1);
     float S[RPT][CPT];
@@ -105,7 +121,7 @@ bwd_ckpt_kernel(const float *__restrict__ kn, const float *__restrict__ vn, cons
 #pragma unroll
     for (int r = 0; r < RPT; ++r)
 #pragma unroll
-        for (int m = 0; m < CPT; ++m) S[r][m] = S0h ? S0h[(warp + 8 * r) * D + CPT * lane + m] : 0.f;
+        for (int m = 0; m < CPT; ++m) S[r][m] = S0h ? S0h[(warp + 8 * r) * D + c0 + CPT * lane + m] : 0.f;
     const size_t base = ckpt_base(s0, n);
     const float Ah = __ldg(A + h), bah = __ldg(b_alpha + h);
     for (int t0 = s0, I = 0; t0 < s1; t0 += IV, ++I) {
@@ -114,153 +130,22 @@ bwd_ckpt_kernel(const float *__restrict__ kn, const float *__restrict__ vn, cons
 #pragma unroll
         for (int r = 0; r < RPT; ++r)
 #pragma unroll
-            for (int m = 0; m < CPT; ++m) ck[(warp + 8 * r) * D + CPT * lane + m] = S[r][m];
+            for (int m = 0; m < CPT; ++m) ck[(warp + 8 * r) * D + c0 + CPT * lane + m] = S[r][m];
         __syncthreads();   // the previous interval's reads of the tile are done
-        for (int idx = tid; idx < cnt * D; idx += bwd::NT) {
-            const int t = idx / D, i = idx % D;
-            const size_t g = ((size_t)(t0 + t) * H + h) * D + i;
-            kk[t][i] = kn[g];
-            vv[t][i] = vn[g];
-        }
-        if (tid < cnt) {
-            const size_t gi = (size_t)(t0 + tid) * H + h;
-            bwd_gates(a_logit[gi], b_logit[gi], Ah, bah, al[tid], be[tid]);
-        }
-        __syncthreads();
-        for (int t = 0; t < cnt; ++t) {
-            float p[CPT];
-#pragma unroll
-            for (int m = 0; m < CPT; ++m) p[m] = 0.f;
-#pragma unroll
-            for (int r = 0; r < RPT; ++r) {
-                const float kr = kk[t][warp + 8 * r];
-#pragma unroll
-                for (int m = 0; m < CPT; ++m) p[m] = fmaf(S[r][m], kr, p[m]);
-            }
-#pragma unroll
-            for (int m = 0; m < CPT; ++m) red[t & 1][warp][CPT * lane + m] = p[m];
-            __syncthreads();
-            float e[CPT];
-#pragma unroll
-            for (int m = 0; m < CPT; ++m) {
-                float s = 0.f;
-#pragma unroll
-                for (int w = 0; w < 8; ++w) s += red[t & 1][w][CPT * lane + m];
-                e[m] = vv[t][CPT * lane + m] - al[t] * s;
-            }
-#pragma unroll
-            for (int r = 0; r < RPT; ++r) {
-                const float bk = be[t] * kk[t][warp + 8 * r];
-#pragma unroll
-                for (int m = 0; m < CPT; ++m) S[r][m] = fmaf(bk, e[m], al[t] * S[r][m]);
-            }
-        }
-    }
-}
-
-// ------------------------------------------------------------- K4b: recurrence
-namespace bwd {
-template <int D> struct RecLayout {
-    // floats: q, k, v, e, y, dy [IV][D]; red [2][2][8][D]; rowsum [2][3][D];
-    // alpha, beta, k.q, e.dy [IV]; per-token scalar partials [IV][8][3]
-    static constexpr int TILE = IV * D;
-    static constexpr int OFF_RED = 6 * TILE;
-    static constexpr int OFF_ROW = OFF_RED + 2 * 2 * 8 * D;
-    static constexpr int OFF_SMALL = OFF_ROW + 2 * 3 * D;
-    static constexpr int OFF_SC = OFF_SMALL + 4 * IV;
-    static constexpr int FLOATS = OFF_SC + IV * 8 * 3;
-    static constexpr int BYTES = FLOATS * 4;
-};
-}  // namespace bwd
-
-template <int D>
-__global__ void __launch_bounds__(bwd::NT, 1)
-bwd_recurrence_kernel(const float *__restrict__ qn, const float *__restrict__ kn, const float *__restrict__ vn,
-                      const float *__restrict__ a_logit, const float *__restrict__ b_logit,
-                      const float *__restrict__ A, const float *__restrict__ b_alpha, const float *__restrict__ z,
-                      const float *__restrict__ norm_w, const float *__restrict__ d_out,
-                      const float *__restrict__ d_S_final, const int32_t *__restrict__ cu, int n_seq, int n_tok,
-                      int H, const float *__restrict__ ckpt, float *__restrict__ scratch, float *__restrict__ dqn,
-                      float *__restrict__ dkn, float *__restrict__ dvn, float *__restrict__ dg,
-                      float *__restrict__ dbeta, float *__restrict__ d_z, float *__restrict__ dnorm_part,
-                      float *__restrict__ d_S0) {
-    using L = bwd::RecLayout<D>;
-    constexpr int RPT = D / 8, CPT = D / 32, IV = bwd::IV;
-    constexpr int NV = (3 * RPT + 31) / 32 * 32;   // row sums per thread, padded for the reduce-scatter
-    extern __shared__ float smf[];
-    float(*qq)[D] = reinterpret_cast<float(*)[D]>(smf);
-    float(*kk)[D] = qq + IV;
-    float(*vv)[D] = kk + IV;
-    float(*ee)[D] = vv + IV;
-    float(*yy)[D] = ee + IV;
-    float(*dyy)[D] = yy + IV;
-    float *red = smf + L::OFF_RED;      // [parity][quantity][warp][D]
-    float *rowsum = smf + L::OFF_ROW;   // [parity][A, B, C][D]
-    float *al = smf + L::OFF_SMALL, *be = al + IV, *kq = be + IV, *edy = kq + IV;
-    float *sc = smf + L::OFF_SC;        // [token][warp][<D,P>, k.(D e), k.(P de)]
-
-    const int h = blockIdx.x, n = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    int s0, s1;
-    bwd_seq_bounds(cu, n_seq, n_tok, n, s0, s1);
-    const int nI = (s1 - s0 + IV - 1) / IV;
-    const size_t base = ckpt_base(s0, n);
-    const float Ah = __ldg(A + h), bah = __ldg(b_alpha + h);
-    float *scr = scratch + ((size_t)n * H + h) * IV * D * D;
-    float gain[CPT], dwacc[CPT];
-#pragma unroll
-    for (int m = 0; m < CPT; ++m) {
-        gain[m] = 1.0f + __ldg(norm_w + CPT * lane + m);
-        dwacc[m] = 0.f;
-    }
-    // the gradient of the state after the current token
-    float Dg[RPT][CPT];
-    const float *dSf = d_S_final ? d_S_final + ((size_t)n * H + h) * D * D : nullptr;
-#pragma unroll
-    for (int r = 0; r < RPT; ++r)
-#pragma unroll
-        for (int m = 0; m < CPT; ++m) Dg[r][m] = dSf ? dSf[(warp + 8 * r) * D + CPT * lane + m] : 0.f;
-
-    for (int I = nI - 1; I >= 0; --I) {
-        const int t0 = s0 + I * IV, cnt = min(IV, s1 - t0);
-        auto finish_rows = [&](int t, int par) {   // threads tid < D: row tid of token t
-            const int i = tid;
-            const float Ai = rowsum[(par * 3 + 0) * D + i], Bi = rowsum[(par * 3 + 1) * D + i];
-            const float Ci = rowsum[(par * 3 + 2) * D + i], ki = kk[t][i];
-            const size_t g = ((size_t)(t0 + t) * H + h) * D + i;
-            dqn[g] = fmaf(al[t], Ai, be[t] * edy[t] * ki);
-            dkn[g] = fmaf(be[t], Ci, -al[t] * Bi);
-            const float kc = group_sum<32>(ki * Ci), kb = group_sum<32>(ki * Bi);
-            if (lane == 0) {
-                sc[(t * 8 + warp) * 3 + 1] = kc;
-                sc[(t * 8 + warp) * 3 + 2] = kb;
-            }
-        };
-        // (a) the state before the interval
-        float S[RPT][CPT];
-        {
-            const float *ck = ckpt + ((base + I) * H + h) * (size_t)D * D;
-#pragma unroll
-            for (int r = 0; r < RPT; ++r)
-#pragma unroll
-                for (int m = 0; m < CPT; ++m) S[r][m] = ck[(warp + 8 * r) * D + CPT * lane + m];
-        }
-        __syncthreads();   // the previous interval's shared-memory reads are done
-        // (b) the interval's q, k, v, gates and k.q: warp w stages tokens 2w, 2w + 1
+        // warp w stages tokens 2w, 2w + 1: q and k rows, k.q, the gates
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
             const int t = 2 * warp + u;
             if (t < cnt) {
                 const size_t row = ((size_t)(t0 + t) * H + h) * D;
                 float dot = 0.f;
-#pragma unroll
-                for (int m = 0; m < CPT; ++m) {
-                    const int j = CPT * lane + m;
+                for (int j = lane; j < D; j += 32) {
                     const float qv = qn[row + j], kv = kn[row + j];
                     qq[t][j] = qv;
                     kk[t][j] = kv;
-                    vv[t][j] = vn[row + j];
                     dot = fmaf(qv, kv, dot);
                 }
+                if (lane < DC) vv[t][lane] = vn[row + c0 + lane];
                 dot = group_sum<32>(dot);
                 if (lane == 0) {
                     kq[t] = dot;
@@ -269,16 +154,8 @@ bwd_recurrence_kernel(const float *__restrict__ qn, const float *__restrict__ kn
                 }
             }
         }
-        for (int idx = tid; idx < IV * 8 * 3; idx += bwd::NT) sc[idx] = 0.f;
         __syncthreads();
-        // (c) forward over the interval: the state before each token to the scratch;
-        //     e and y of each token
         for (int t = 0; t < cnt; ++t) {
-            float *st = scr + (size_t)t * D * D;
-#pragma unroll
-            for (int r = 0; r < RPT; ++r)
-#pragma unroll
-                for (int m = 0; m < CPT; ++m) st[(warp + 8 * r) * D + CPT * lane + m] = S[r][m];
             float p[CPT], pq[CPT];
 #pragma unroll
             for (int m = 0; m < CPT; ++m) p[m] = pq[m] = 0.f;
@@ -291,27 +168,27 @@ bwd_recurrence_kernel(const float *__restrict__ qn, const float *__restrict__ kn
                     pq[m] = fmaf(S[r][m], qr, pq[m]);
                 }
             }
-            float *rd = red + (t & 1) * 2 * 8 * D;
 #pragma unroll
             for (int m = 0; m < CPT; ++m) {
-                rd[warp * D + CPT * lane + m] = p[m];
-                rd[8 * D + warp * D + CPT * lane + m] = pq[m];
+                red[t & 1][0][warp][CPT * lane + m] = p[m];
+                red[t & 1][1][warp][CPT * lane + m] = pq[m];
             }
             __syncthreads();
             float e[CPT];
+            const size_t row = ((size_t)(t0 + t) * H + h) * D + c0;
 #pragma unroll
             for (int m = 0; m < CPT; ++m) {
                 const int j = CPT * lane + m;
-                float s = 0.f, sq = 0.f;
+                float sp = 0.f, sq = 0.f;
 #pragma unroll
                 for (int w = 0; w < 8; ++w) {
-                    s += rd[w * D + j];
-                    sq += rd[8 * D + w * D + j];
+                    sp += red[t & 1][0][w][j];
+                    sq += red[t & 1][1][w][j];
                 }
-                e[m] = vv[t][j] - al[t] * s;
-                if (warp == 0) {
-                    ee[t][j] = e[m];
-                    yy[t][j] = fmaf(al[t], sq, be[t] * kq[t] * e[m]);
+                e[m] = vv[t][j] - al[t] * sp;
+                if (warp == (t & 7)) {
+                    e_out[row + j] = e[m];
+                    y_out[row + j] = fmaf(al[t], sq, be[t] * kq[t] * e[m]);
                 }
             }
 #pragma unroll
@@ -321,62 +198,164 @@ bwd_recurrence_kernel(const float *__restrict__ qn, const float *__restrict__ kn
                 for (int m = 0; m < CPT; ++m) S[r][m] = fmaf(bk, e[m], al[t] * S[r][m]);
             }
         }
-        __syncthreads();   // e and y of the interval are complete
-        // (c') output-stage backward: warp w takes tokens 2w, 2w + 1
+    }
+}
+
+// ---------------------------------------------------- K4b: output-stage backward
+// One warp per token-head: dy, d_z and e . dy from y, e, z and d_out; the norm
+// weight's gradient summed per block (grid-stride, fixed order).
+template <int D>
+__global__ void __launch_bounds__(bwd::NT)
+bwd_epi_kernel(const float *__restrict__ y, const float *__restrict__ e, const float *__restrict__ z,
+               const float *__restrict__ norm_w, const float *__restrict__ d_out, int n_th,
+               float *__restrict__ dy_out, float *__restrict__ dz_out, float *__restrict__ edy_out,
+               float *__restrict__ dw_part) {
+    constexpr int CPL = D / 32;
+    __shared__ float part[8][D];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float gain[CPL], acc[CPL];
+#pragma unroll
+    for (int m = 0; m < CPL; ++m) {
+        gain[m] = 1.0f + __ldg(norm_w + CPL * lane + m);
+        acc[m] = 0.f;
+    }
+    for (int th = blockIdx.x * 8 + warp; th < n_th; th += gridDim.x * 8) {
+        const size_t row = (size_t)th * D + CPL * lane;
+        float yv[CPL], sz[CPL], dov[CPL], dn[CPL], ssq = 0.f, dny = 0.f;
+#pragma unroll
+        for (int m = 0; m < CPL; ++m) {
+            yv[m] = y[row + m];
+            sz[m] = sigmoid_acc(z[row + m]);
+            dov[m] = d_out[row + m];
+            ssq = fmaf(yv[m], yv[m], ssq);
+            dn[m] = dov[m] * sz[m] * gain[m];
+            dny = fmaf(dn[m], yv[m], dny);
+        }
+        ssq = group_sum<32>(ssq);
+        dny = group_sum<32>(dny);
+        const float r = 1.0f / sqrtf(ssq / D + kNormEps);
+        float edot = 0.f;
+#pragma unroll
+        for (int m = 0; m < CPL; ++m) {
+            const float nj = yv[m] * r;
+            dz_out[row + m] = dov[m] * nj * gain[m] * sz[m] * (1.0f - sz[m]);
+            acc[m] = fmaf(dov[m] * sz[m], nj, acc[m]);
+            const float dyv = r * dn[m] - r * r * r * yv[m] * (dny / D);
+            dy_out[row + m] = dyv;
+            edot = fmaf(e[row + m], dyv, edot);
+        }
+        edot = group_sum<32>(edot);
+        if (lane == 0) edy_out[th] = edot;
+    }
+#pragma unroll
+    for (int m = 0; m < CPL; ++m) part[warp][CPL * lane + m] = acc[m];
+    __syncthreads();
+    if (threadIdx.x < D) {
+        float s = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) s += part[w][threadIdx.x];
+        dw_part[(size_t)blockIdx.x * D + threadIdx.x] = s;
+    }
+}
+
+// ------------------------------------------------------------ K4c: reverse sweep
+// DC columns of one (sequence, head), intervals in reverse.  Per interval: the
+// checkpoint is loaded and the interval re-run (with the stored e: no sums),
+// each state before a token going to this CTA's scratch (16 x D x DC floats,
+// which stays in L2); then the token steps in reverse with the state gradient
+// in registers.  Per step one block barrier (the column sums of D^T k); the row
+// sums P dy, P de, D e over this CTA's columns are a warp reduce-scatter and go
+// to the partial buffer with <D, P> (one value per warp).
+template <int D, int DC>
+__global__ void __launch_bounds__(bwd::NT, 2)
+bwd_rec_kernel(const float *__restrict__ qn, const float *__restrict__ kn, const float *__restrict__ e_in,
+               const float *__restrict__ dy_in, const float *__restrict__ a_logit, const float *__restrict__ b_logit,
+               const float *__restrict__ A, const float *__restrict__ b_alpha, const float *__restrict__ d_S_final,
+               const int32_t *__restrict__ cu, int n_seq, int n_tok, int H, const float *__restrict__ ckpt,
+               float *__restrict__ scratch, float *__restrict__ dvn, float *__restrict__ part,
+               float *__restrict__ d_S0) {
+    constexpr int RPT = D / 8, CPT = DC / 32, IV = bwd::IV, NS = D / DC;
+    constexpr int NV = (3 * RPT + 31) / 32 * 32;
+    constexpr int PW = 3 * D + 8;   // partial row: P dy, P de, D e [D] each, <D, P> per warp [8]
+    __shared__ float qq[IV][D], kk[IV][D], ee[IV][DC], dyy[IV][DC], al[IV], be[IV];
+    __shared__ float red[2][8][DC];
+    const int h = blockIdx.x, n = blockIdx.y, zc = blockIdx.z, c0 = zc * DC;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    int s0, s1;
+    bwd_seq_bounds(cu, n_seq, n_tok, n, s0, s1);
+    const int nI = (s1 - s0 + IV - 1) / IV;
+    const size_t base = ckpt_base(s0, n);
+    const size_t n_th = (size_t)n_tok * H;
+    const float Ah = __ldg(A + h), bah = __ldg(b_alpha + h);
+    float *scr = scratch + (((size_t)n * H + h) * NS + zc) * IV * D * DC;
+    float Dg[RPT][CPT];   // the gradient of the state after the current token
+    const float *dSf = d_S_final ? d_S_final + ((size_t)n * H + h) * D * D : nullptr;
+#pragma unroll
+    for (int r = 0; r < RPT; ++r)
+#pragma unroll
+        for (int m = 0; m < CPT; ++m) Dg[r][m] = dSf ? dSf[(warp + 8 * r) * D + c0 + CPT * lane + m] : 0.f;
+
+    for (int I = nI - 1; I >= 0; --I) {
+        const int t0 = s0 + I * IV, cnt = min(IV, s1 - t0);
+        float S[RPT][CPT];
+        {
+            const float *ck = ckpt + ((base + I) * H + h) * (size_t)D * D;
+#pragma unroll
+            for (int r = 0; r < RPT; ++r)
+#pragma unroll
+                for (int m = 0; m < CPT; ++m) S[r][m] = ck[(warp + 8 * r) * D + c0 + CPT * lane + m];
+        }
+        __syncthreads();   // the previous interval's shared-memory reads are done
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
             const int t = 2 * warp + u;
             if (t < cnt) {
                 const size_t row = ((size_t)(t0 + t) * H + h) * D;
-                float yv[CPT], sz[CPT], dov[CPT], dn[CPT], ssq = 0.f, dny = 0.f;
-#pragma unroll
-                for (int m = 0; m < CPT; ++m) {
-                    const int j = CPT * lane + m;
-                    yv[m] = yy[t][j];
-                    sz[m] = sigmoid_acc(z[row + j]);
-                    dov[m] = d_out[row + j];
-                    ssq = fmaf(yv[m], yv[m], ssq);
-                    dn[m] = dov[m] * sz[m] * gain[m];
-                    dny = fmaf(dn[m], yv[m], dny);
+                for (int j = lane; j < D; j += 32) {
+                    qq[t][j] = qn[row + j];
+                    kk[t][j] = kn[row + j];
                 }
-                ssq = group_sum<32>(ssq);
-                dny = group_sum<32>(dny);
-                const float r = 1.0f / sqrtf(ssq / D + kNormEps);
-                float edot = 0.f;
-#pragma unroll
-                for (int m = 0; m < CPT; ++m) {
-                    const int j = CPT * lane + m;
-                    const float nj = yv[m] * r;
-                    d_z[row + j] = dov[m] * nj * gain[m] * sz[m] * (1.0f - sz[m]);
-                    dwacc[m] = fmaf(dov[m] * sz[m], nj, dwacc[m]);
-                    const float dyv = r * dn[m] - r * r * r * yv[m] * (dny / D);
-                    dyy[t][j] = dyv;
-                    edot = fmaf(ee[t][j], dyv, edot);
+                if (lane < DC) {
+                    ee[t][lane] = e_in[row + c0 + lane];
+                    dyy[t][lane] = dy_in[row + c0 + lane];
                 }
-                edot = group_sum<32>(edot);
-                if (lane == 0) edy[t] = edot;
+                if (lane == 0) {
+                    const size_t gi = (size_t)(t0 + t) * H + h;
+                    bwd_gates(a_logit[gi], b_logit[gi], Ah, bah, al[t], be[t]);
+                }
             }
         }
         __syncthreads();
-        // (d) token steps in reverse
+        // re-run the interval: the state before each token to the scratch
+        for (int t = 0; t < cnt; ++t) {
+            float *st = scr + (size_t)t * D * DC;
+#pragma unroll
+            for (int r = 0; r < RPT; ++r)
+#pragma unroll
+                for (int m = 0; m < CPT; ++m) st[(warp + 8 * r) * DC + CPT * lane + m] = S[r][m];
+#pragma unroll
+            for (int r = 0; r < RPT; ++r) {
+                const float bk = be[t] * kk[t][warp + 8 * r];
+#pragma unroll
+                for (int m = 0; m < CPT; ++m) S[r][m] = fmaf(bk, ee[t][CPT * lane + m], al[t] * S[r][m]);
+            }
+        }
+        // token steps in reverse
         for (int t = cnt - 1; t >= 0; --t) {
-            const int par = t & 1;
-            const float *st = scr + (size_t)t * D * D;
+            const float *st = scr + (size_t)t * D * DC;
             float P[RPT][CPT];
 #pragma unroll
             for (int r = 0; r < RPT; ++r)
 #pragma unroll
-                for (int m = 0; m < CPT; ++m) P[r][m] = st[(warp + 8 * r) * D + CPT * lane + m];
-            float dyl[CPT], el[CPT];
+                for (int m = 0; m < CPT; ++m) P[r][m] = st[(warp + 8 * r) * DC + CPT * lane + m];
+            float dyl[CPT], el[CPT], dp[CPT];
 #pragma unroll
             for (int m = 0; m < CPT; ++m) {
                 dyl[m] = dyy[t][CPT * lane + m];
                 el[m] = ee[t][CPT * lane + m];
+                dp[m] = 0.f;
             }
             // D += q dy^T, then the column partials of D^T k
-            float dp[CPT];
-#pragma unroll
-            for (int m = 0; m < CPT; ++m) dp[m] = 0.f;
 #pragma unroll
             for (int r = 0; r < RPT; ++r) {
                 const float qr = qq[t][warp + 8 * r], kr = kk[t][warp + 8 * r];
@@ -386,25 +365,23 @@ bwd_recurrence_kernel(const float *__restrict__ qn, const float *__restrict__ kn
                     dp[m] = fmaf(Dg[r][m], kr, dp[m]);
                 }
             }
-            float *rd = red + par * 2 * 8 * D;
 #pragma unroll
-            for (int m = 0; m < CPT; ++m) rd[warp * D + CPT * lane + m] = dp[m];
+            for (int m = 0; m < CPT; ++m) red[t & 1][warp][CPT * lane + m] = dp[m];
             __syncthreads();
-            // the rows of token t + 1 (their sums were completed before this barrier)
-            if (t + 1 < cnt && tid < D) finish_rows(t + 1, par ^ 1);
             float de[CPT];
 #pragma unroll
             for (int m = 0; m < CPT; ++m) {
                 float s = 0.f;
 #pragma unroll
-                for (int w = 0; w < 8; ++w) s += rd[w * D + CPT * lane + m];
+                for (int w = 0; w < 8; ++w) s += red[t & 1][w][CPT * lane + m];
                 de[m] = be[t] * s;
             }
-            if (warp == 0) {
+            const size_t th = (size_t)(t0 + t) * H + h;
+            if (warp == (t & 7)) {
 #pragma unroll
-                for (int m = 0; m < CPT; ++m) dvn[((size_t)(t0 + t) * H + h) * D + CPT * lane + m] = de[m];
+                for (int m = 0; m < CPT; ++m) dvn[th * D + c0 + CPT * lane + m] = de[m];
             }
-            // row sums: A = P dy, B = P de, C = D e; and <D, P>
+            // row sums over this CTA's columns: P dy, P de, D e; and <D, P>
             float v[NV];
             float dDP = 0.f;
 #pragma unroll
@@ -424,13 +401,14 @@ bwd_recurrence_kernel(const float *__restrict__ qn, const float *__restrict__ kn
 #pragma unroll
             for (int x = 3 * RPT; x < NV; ++x) v[x] = 0.f;
             warp_reduce_scatter<NV>(v, lane);
+            float *pr = part + ((size_t)zc * n_th + th) * PW;
 #pragma unroll
             for (int i = 0; i < NV / 32; ++i) {
                 const int idx = (NV / 32) * lane + i;
-                if (idx < 3 * RPT) rowsum[(par * 3 + idx / RPT) * D + warp + 8 * (idx % RPT)] = v[i];
+                if (idx < 3 * RPT) pr[(idx / RPT) * D + warp + 8 * (idx % RPT)] = v[i];
             }
             dDP = group_sum<32>(dDP);
-            if (lane == 0) sc[(t * 8 + warp) * 3 + 0] = dDP;
+            if (lane == 0) pr[3 * D + warp] = dDP;
             // the gradient of the state before token t
 #pragma unroll
             for (int r = 0; r < RPT; ++r) {
@@ -439,43 +417,64 @@ bwd_recurrence_kernel(const float *__restrict__ qn, const float *__restrict__ kn
                 for (int m = 0; m < CPT; ++m) Dg[r][m] = al[t] * fmaf(-kr, de[m], Dg[r][m]);
             }
         }
-        __syncthreads();
-        if (cnt > 0 && tid < D) finish_rows(0, 0);
-        __syncthreads();
-        if (tid < cnt) {
-            float dp_ = 0.f, kc = 0.f, kb = 0.f;
-#pragma unroll
-            for (int w = 0; w < 8; ++w) {
-                dp_ += sc[(tid * 8 + w) * 3 + 0];
-                kc += sc[(tid * 8 + w) * 3 + 1];
-                kb += sc[(tid * 8 + w) * 3 + 2];
-            }
-            const size_t gi = (size_t)(t0 + tid) * H + h;
-            dbeta[gi] = kc;
-            dg[gi] = al[tid] * (dp_ - kb);
-        }
     }
     if (d_S0) {
         float *o = d_S0 + ((size_t)n * H + h) * D * D;
 #pragma unroll
         for (int r = 0; r < RPT; ++r)
 #pragma unroll
-            for (int m = 0; m < CPT; ++m) o[(warp + 8 * r) * D + CPT * lane + m] = Dg[r][m];
-    }
-    // the norm-weight partial of this (sequence, head): sum of the 8 warps
-    __syncthreads();
-#pragma unroll
-    for (int m = 0; m < CPT; ++m) red[warp * D + CPT * lane + m] = dwacc[m];
-    __syncthreads();
-    if (tid < D) {
-        float s = 0.f;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) s += red[w * D + tid];
-        dnorm_part[((size_t)n * H + h) * D + tid] = s;
+            for (int m = 0; m < CPT; ++m) o[(warp + 8 * r) * D + c0 + CPT * lane + m] = Dg[r][m];
     }
 }
 
-// ------------------------------------------------------------ K4c: prelude backward
+// ------------------------------------------------------- K4d: per-token combine
+// One warp per token-head: the row sums of the column splits give dq = alpha P dy
+// + beta (e . dy) k and dk = beta D e - alpha P de; dbeta = k . (D e) and
+// dg = alpha (<D, P> - k . (P de)).
+template <int D, int NS>
+__global__ void __launch_bounds__(bwd::NT)
+bwd_combine_kernel(const float *__restrict__ part, const float *__restrict__ kn, const float *__restrict__ edy,
+                   const float *__restrict__ a_logit, const float *__restrict__ b_logit,
+                   const float *__restrict__ A, const float *__restrict__ b_alpha, int n_th, int H,
+                   float *__restrict__ dqn, float *__restrict__ dkn, float *__restrict__ dg,
+                   float *__restrict__ dbeta) {
+    constexpr int PW = 3 * D + 8;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int th = blockIdx.x * 8 + warp;
+    if (th >= n_th) return;   // warp-uniform
+    const int h = th % H;
+    float al, be;
+    bwd_gates(a_logit[th], b_logit[th], __ldg(A + h), __ldg(b_alpha + h), al, be);
+    const float ed = edy[th];
+    float kc = 0.f, kb = 0.f, dDP = 0.f;
+#pragma unroll
+    for (int u = 0; u < D / 32; ++u) {
+        const int i = lane + 32 * u;
+        float a_ = 0.f, b_ = 0.f, c_ = 0.f;
+#pragma unroll
+        for (int zc = 0; zc < NS; ++zc) {
+            const float *pr = part + ((size_t)zc * n_th + th) * PW;
+            a_ += pr[i];
+            b_ += pr[D + i];
+            c_ += pr[2 * D + i];
+        }
+        const float ki = kn[(size_t)th * D + i];
+        dqn[(size_t)th * D + i] = fmaf(al, a_, be * ed * ki);
+        dkn[(size_t)th * D + i] = fmaf(be, c_, -al * b_);
+        kc = fmaf(ki, c_, kc);
+        kb = fmaf(ki, b_, kb);
+    }
+    if (lane < 8 * NS) dDP = part[((size_t)(lane / 8) * n_th + th) * PW + 3 * D + (lane % 8)];
+    kc = group_sum<32>(kc);
+    kb = group_sum<32>(kb);
+    dDP = group_sum<32>(dDP);
+    if (lane == 0) {
+        dbeta[th] = kc;
+        dg[th] = al * (dDP - kb);
+    }
+}
+
+// ------------------------------------------------------------ K4e: prelude backward
 // One thread owns 8 consecutive conv channels (of q, k or v of one head) and a
 // 64-token tile.  It walks tokens t0 .. t1 + 2 (the conv looks 3 tokens back, so
 // its transpose looks 3 ahead), recomputing x = conv(raw), u = SiLU(x) and, for q
@@ -630,7 +629,7 @@ bwd_prelude_kernel(const float *__restrict__ q, const float *__restrict__ k, con
     }
 }
 
-// --------------------------------------------------------------- K4d: gates
+// --------------------------------------------------------------- K4f: gates
 __global__ void __launch_bounds__(bwd::NT)
 bwd_gates_kernel(const float *__restrict__ a_logit, const float *__restrict__ b_logit,
                  const float *__restrict__ A, const float *__restrict__ b_alpha, const float *__restrict__ dg,
@@ -670,7 +669,7 @@ bwd_gates_kernel(const float *__restrict__ a_logit, const float *__restrict__ b_
     }
 }
 
-// --------------------------------------------------------------- K4e: reductions
+// --------------------------------------------------------------- K4g: reductions
 __global__ void __launch_bounds__(bwd::NT)
 bwd_reduce_kernel(const float *__restrict__ dw_part, int n_tiles, int C4, const float *__restrict__ dnorm_part,
                   int n_pairs, int D, float *__restrict__ d_conv_w, float *__restrict__ d_norm_w) {
@@ -688,14 +687,19 @@ bwd_reduce_kernel(const float *__restrict__ dw_part, int n_tiles, int C4, const 
 }
 
 // ---------------------------------------------------------------------- host
+namespace bwd {
+constexpr int EPI_BLOCKS = 4 * 148;   // grid of the output-stage kernel (fixed: its partial sums have a fixed order)
+}  // namespace bwd
+
 size_t backward_workspace_bytes(int n_seq, int n_tok, int H, int D) {
     auto ru = [](size_t x) { return (x + 255) & ~(size_t)255; };
     const size_t nt = (size_t)n_tok * H;
     const size_t n_ckpt = (size_t)n_tok / bwd::IV + n_seq;
     const size_t n_tiles = ((size_t)n_tok + bwd::PT - 1) / bwd::PT;
-    return 6 * ru(nt * D * 4) + 2 * ru(nt * 4) + ru(n_ckpt * H * D * D * 4) +
-           ru((size_t)n_seq * H * bwd::IV * D * D * 4) + ru(n_tiles * 3 * H * D * 4 * 4) +
-           ru((size_t)n_seq * H * D * 4);
+    const size_t ns = (size_t)D / bwd::DC;
+    return 9 * ru(nt * D * 4) + 3 * ru(nt * 4) + ru(n_ckpt * H * D * D * 4) +
+           ru((size_t)n_seq * H * bwd::IV * D * D * 4) + ru(ns * nt * (3 * D + 8) * 4) +
+           ru(n_tiles * 3 * H * D * 4 * 4) + ru((size_t)bwd::EPI_BLOCKS * D * 4);
 }
 
 cudaError_t launch_backward(const BackwardArgs &b, void *ws) {
@@ -706,13 +710,15 @@ cudaError_t launch_backward(const BackwardArgs &b, void *ws) {
     auto take = [&](size_t bytes) { char *r = p; p += ru(bytes); return reinterpret_cast<float *>(r); };
     float *qn = take(nt * D * 4), *kn = take(nt * D * 4), *vn = take(nt * D * 4);
     float *dqn = take(nt * D * 4), *dkn = take(nt * D * 4), *dvn = take(nt * D * 4);
-    float *dgw = take(nt * 4), *dbw = take(nt * 4);
+    float *yw = take(nt * D * 4), *ew = take(nt * D * 4), *dyw = take(nt * D * 4);
+    float *dgw = take(nt * 4), *dbw = take(nt * 4), *edy = take(nt * 4);
     const size_t n_ckpt = (size_t)n_tok / bwd::IV + n_seq;
     float *ckpt = take(n_ckpt * H * D * D * 4);
     float *scratch = take((size_t)n_seq * H * bwd::IV * D * D * 4);
+    float *part = take((size_t)(D / bwd::DC) * nt * (3 * D + 8) * 4);
     const int n_tiles = (n_tok + bwd::PT - 1) / bwd::PT;
     float *dw_part = take((size_t)n_tiles * 3 * H * D * 4 * 4);
-    float *dnorm_part = take((size_t)n_seq * H * D * 4);
+    float *dnorm_part = take((size_t)bwd::EPI_BLOCKS * D * 4);
     cudaStream_t s = b.f.stream;
     const float *fq = static_cast<const float *>(b.f.q), *fk = static_cast<const float *>(b.f.k);
     const float *fv = static_cast<const float *>(b.f.v), *fz = static_cast<const float *>(b.f.z);
@@ -721,24 +727,29 @@ cudaError_t launch_backward(const BackwardArgs &b, void *ws) {
     if (n_tok > 0) {
         if ((e = launch_prelude_f32(b.f, qn, kn, vn)) != cudaSuccess) return e;
     }
-    const dim3 pairs(H, n_seq);
 #define GDN_BWD(D_)                                                                                          \
     do {                                                                                                     \
+        constexpr int NS_ = D_ / bwd::DC;                                                                    \
+        const dim3 split(H, n_seq, NS_);                                                                     \
         if (n_tok > 0) {                                                                                     \
-            bwd_ckpt_kernel<D_><<<pairs, bwd::NT, 0, s>>>(kn, vn, fa, fb, b.f.A, b.f.b_alpha, b.f.S0,        \
-                                                          b.f.cu_seqlens, n_seq, n_tok, H, ckpt);           \
+            bwd_fwd_kernel<D_, bwd::DC><<<split, bwd::NT, 0, s>>>(qn, kn, vn, fa, fb, b.f.A, b.f.b_alpha,    \
+                                                                 b.f.S0, b.f.cu_seqlens, n_seq, n_tok, H,  \
+                                                                 ckpt, yw, ew);                             \
             if ((e = launched()) != cudaSuccess) return e;                                                   \
         }                                                                                                    \
-        constexpr int SM_ = bwd::RecLayout<D_>::BYTES;                                                       \
-        if ((e = cudaFuncSetAttribute(bwd_recurrence_kernel<D_>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                                      SM_)) != cudaSuccess)                                                  \
-            return e;                                                                                        \
-        bwd_recurrence_kernel<D_><<<pairs, bwd::NT, SM_, s>>>(                                               \
-            qn, kn, vn, fa, fb, b.f.A, b.f.b_alpha, fz, b.f.norm_w, static_cast<const float *>(b.d_out),     \
-            b.d_S_final, b.f.cu_seqlens, n_seq, n_tok, H, ckpt, scratch, dqn, dkn, dvn, dgw, dbw,            \
-            static_cast<float *>(b.d_z), dnorm_part, b.d_S0);                                                \
+        bwd_epi_kernel<D_><<<bwd::EPI_BLOCKS, bwd::NT, 0, s>>>(yw, ew, fz, b.f.norm_w,                       \
+                                                               static_cast<const float *>(b.d_out), (int)nt, \
+                                                               dyw, static_cast<float *>(b.d_z), edy,        \
+                                                               dnorm_part);                                  \
+        if ((e = launched()) != cudaSuccess) return e;                                                       \
+        bwd_rec_kernel<D_, bwd::DC><<<split, bwd::NT, 0, s>>>(qn, kn, ew, dyw, fa, fb, b.f.A, b.f.b_alpha,   \
+                                                             b.d_S_final, b.f.cu_seqlens, n_seq, n_tok, H,  \
+                                                             ckpt, scratch, dvn, part, b.d_S0);             \
         if ((e = launched()) != cudaSuccess) return e;                                                       \
         if (n_tok > 0) {                                                                                     \
+            bwd_combine_kernel<D_, NS_><<<(unsigned)((nt + 7) / 8), bwd::NT, 0, s>>>(                        \
+                part, kn, edy, fa, fb, b.f.A, b.f.b_alpha, (int)nt, H, dqn, dkn, dgw, dbw);                 \
+            if ((e = launched()) != cudaSuccess) return e;                                                   \
             const dim3 g((3 * H * D_ / 8 + bwd::NT - 1) / bwd::NT, n_tiles);                                 \
             bwd_prelude_kernel<D_><<<g, bwd::NT, 0, s>>>(fq, fk, fv, b.f.conv_w, dqn, dkn, dvn,              \
                                                          b.f.cu_seqlens, n_seq, n_tok, H,                    \
@@ -755,7 +766,7 @@ cudaError_t launch_backward(const BackwardArgs &b, void *ws) {
     if ((e = launched()) != cudaSuccess) return e;
     const int C4 = 3 * H * D * 4;
     bwd_reduce_kernel<<<(C4 + D + bwd::NT - 1) / bwd::NT, bwd::NT, 0, s>>>(dw_part, n_tiles, C4, dnorm_part,
-                                                                           n_seq * H, D, b.d_conv_w,
+                                                                           bwd::EPI_BLOCKS, D, b.d_conv_w,
                                                                            b.d_norm_w);
     return launched();
 }
