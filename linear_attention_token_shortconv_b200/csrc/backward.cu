@@ -100,8 +100,13 @@ constexpr int DC = 32;   // state columns per CTA
 }  // namespace bwd
 
 // ------------------------------------------------------- K4a: forward + checkpoints
-// The forward recurrence of DC columns of one (sequence, head): the state before
-// every 16-token interval (checkpoints), and each token's e and y (those columns).
+// The forward recurrence of DC = 32 columns of one (sequence, head): the state
+// before every 16-token interval (checkpoints), and each token's e and y (those
+// columns).  Warp w owns columns 4w .. 4w + 3 whole: lane l holds column
+// 4w + l / 8 and, with g = l % 8, rows 4g + 32 j + i (i < 4): every column sum is
+// three shuffles, the token loop needs no block barrier, and a thread reads its
+// rows of q and k as 128-bit shared loads that the 8 lanes of a quarter-warp
+// take from one contiguous 128-byte line.
 template <int D, int DC>
 __global__ void __launch_bounds__(bwd::NT, 2)
 bwd_fwd_kernel(const float *__restrict__ qn, const float *__restrict__ kn, const float *__restrict__ vn,
@@ -109,28 +114,28 @@ bwd_fwd_kernel(const float *__restrict__ qn, const float *__restrict__ kn, const
                const float *__restrict__ b_alpha, const float *__restrict__ S0, const int32_t *__restrict__ cu,
                int n_seq, int n_tok, int H, float *__restrict__ ckpt, float *__restrict__ y_out,
                float *__restrict__ e_out) {
-    constexpr int RPT = D / 8, CPT = DC / 32, IV = bwd::IV;
-    __shared__ float qq[IV][D], kk[IV][D], vv[IV][DC], al[IV], be[IV], kq[IV];
-    __shared__ float red[2][2][8][DC];
+    static_assert(DC == 32, "8 warps x 4 columns");
+    constexpr int RPT = D / 8, IV = bwd::IV;
+    __shared__ __align__(16) float qq[IV][D];
+    __shared__ __align__(16) float kk[IV][D];
+    __shared__ float vv[IV][DC], al[IV], be[IV], kq[IV];
     const int h = blockIdx.x, n = blockIdx.y, c0 = blockIdx.z * DC;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c = 4 * warp + (lane >> 3), g = lane & 7;   // column c0 + c, rows row_of(r)
+    auto row_of = [&](int r) { return 4 * g + 32 * (r >> 2) + (r & 3); };
     int s0, s1;
     bwd_seq_bounds(cu, n_seq, n_tok, n, s0, s1);
-    float S[RPT][CPT];
+    float S[RPT];
     const float *S0h = S0 ? S0 + ((size_t)n * H + h) * D * D : nullptr;
 #pragma unroll
-    for (int r = 0; r < RPT; ++r)
-#pragma unroll
-        for (int m = 0; m < CPT; ++m) S[r][m] = S0h ? S0h[(warp + 8 * r) * D + c0 + CPT * lane + m] : 0.f;
+    for (int r = 0; r < RPT; ++r) S[r] = S0h ? S0h[row_of(r) * D + c0 + c] : 0.f;
     const size_t base = ckpt_base(s0, n);
     const float Ah = __ldg(A + h), bah = __ldg(b_alpha + h);
     for (int t0 = s0, I = 0; t0 < s1; t0 += IV, ++I) {
         const int cnt = min(IV, s1 - t0);
         float *ck = ckpt + ((base + I) * H + h) * (size_t)D * D;
 #pragma unroll
-        for (int r = 0; r < RPT; ++r)
-#pragma unroll
-            for (int m = 0; m < CPT; ++m) ck[(warp + 8 * r) * D + c0 + CPT * lane + m] = S[r][m];
+        for (int r = 0; r < RPT; ++r) ck[row_of(r) * D + c0 + c] = S[r];
         __syncthreads();   // the previous interval's reads of the tile are done
         // warp w stages tokens 2w, 2w + 1: q and k rows, k.q, the gates
 #pragma unroll
@@ -145,7 +150,7 @@ bwd_fwd_kernel(const float *__restrict__ qn, const float *__restrict__ kn, const
                     kk[t][j] = kv;
                     dot = fmaf(qv, kv, dot);
                 }
-                if (lane < DC) vv[t][lane] = vn[row + c0 + lane];
+                vv[t][lane] = vn[row + c0 + lane];
                 dot = group_sum<32>(dot);
                 if (lane == 0) {
                     kq[t] = dot;
@@ -156,47 +161,36 @@ bwd_fwd_kernel(const float *__restrict__ qn, const float *__restrict__ kn, const
         }
         __syncthreads();
         for (int t = 0; t < cnt; ++t) {
-            float p[CPT], pq[CPT];
+            float kr[RPT], qr[RPT];
 #pragma unroll
-            for (int m = 0; m < CPT; ++m) p[m] = pq[m] = 0.f;
+            for (int r = 0; r < RPT; r += 4) {
+                const float4 k4 = *reinterpret_cast<const float4 *>(&kk[t][row_of(r)]);
+                const float4 q4 = *reinterpret_cast<const float4 *>(&qq[t][row_of(r)]);
+                kr[r] = k4.x; kr[r + 1] = k4.y; kr[r + 2] = k4.z; kr[r + 3] = k4.w;
+                qr[r] = q4.x; qr[r + 1] = q4.y; qr[r + 2] = q4.z; qr[r + 3] = q4.w;
+            }
+            float p0 = 0.f, p1 = 0.f, q0 = 0.f, q1 = 0.f;
 #pragma unroll
-            for (int r = 0; r < RPT; ++r) {
-                const float kr = kk[t][warp + 8 * r], qr = qq[t][warp + 8 * r];
+            for (int r = 0; r < RPT; r += 2) {
+                p0 = fmaf(S[r], kr[r], p0);
+                p1 = fmaf(S[r + 1], kr[r + 1], p1);
+                q0 = fmaf(S[r], qr[r], q0);
+                q1 = fmaf(S[r + 1], qr[r + 1], q1);
+            }
+            float p = p0 + p1, pq = q0 + q1;
 #pragma unroll
-                for (int m = 0; m < CPT; ++m) {
-                    p[m] = fmaf(S[r][m], kr, p[m]);
-                    pq[m] = fmaf(S[r][m], qr, pq[m]);
-                }
+            for (int o = 1; o < 8; o <<= 1) {
+                p += __shfl_xor_sync(0xffffffffu, p, o);
+                pq += __shfl_xor_sync(0xffffffffu, pq, o);
+            }
+            const float e = vv[t][c] - al[t] * p;
+            if (g == 0) {
+                const size_t row = ((size_t)(t0 + t) * H + h) * D + c0 + c;
+                e_out[row] = e;
+                y_out[row] = fmaf(al[t], pq, be[t] * kq[t] * e);
             }
 #pragma unroll
-            for (int m = 0; m < CPT; ++m) {
-                red[t & 1][0][warp][CPT * lane + m] = p[m];
-                red[t & 1][1][warp][CPT * lane + m] = pq[m];
-            }
-            __syncthreads();
-            float e[CPT];
-            const size_t row = ((size_t)(t0 + t) * H + h) * D + c0;
-#pragma unroll
-            for (int m = 0; m < CPT; ++m) {
-                const int j = CPT * lane + m;
-                float sp = 0.f, sq = 0.f;
-#pragma unroll
-                for (int w = 0; w < 8; ++w) {
-                    sp += red[t & 1][0][w][j];
-                    sq += red[t & 1][1][w][j];
-                }
-                e[m] = vv[t][j] - al[t] * sp;
-                if (warp == (t & 7)) {
-                    e_out[row + j] = e[m];
-                    y_out[row + j] = fmaf(al[t], sq, be[t] * kq[t] * e[m]);
-                }
-            }
-#pragma unroll
-            for (int r = 0; r < RPT; ++r) {
-                const float bk = be[t] * kk[t][warp + 8 * r];
-#pragma unroll
-                for (int m = 0; m < CPT; ++m) S[r][m] = fmaf(bk, e[m], al[t] * S[r][m]);
-            }
+            for (int r = 0; r < RPT; ++r) S[r] = fmaf(be[t] * kr[r], e, al[t] * S[r]);
         }
     }
 }
@@ -259,13 +253,16 @@ bwd_epi_kernel(const float *__restrict__ y, const float *__restrict__ e, const f
 }
 
 // ------------------------------------------------------------ K4c: reverse sweep
+
 // DC columns of one (sequence, head), intervals in reverse.  Per interval: the
 // checkpoint is loaded and the interval re-run (with the stored e: no sums),
 // each state before a token going to this CTA's scratch (16 x D x DC floats,
 // which stays in L2); then the token steps in reverse with the state gradient
-// in registers.  Per step one block barrier (the column sums of D^T k); the row
-// sums P dy, P de, D e over this CTA's columns are a warp reduce-scatter and go
-// to the partial buffer with <D, P> (one value per warp).
+// in registers: thread (warp w, lane l) holds column c0 + l of rows w D / 8 ..
+// + D / 8 (contiguous, so a warp reads its rows of q and k with 128-bit shared
+// loads).  Per step one block barrier (the column sums of D^T k); the row sums
+// P dy, P de, D e over this CTA's columns are a warp reduce-scatter and go to the
+// partial buffer with <D, P> (one value per warp).
 template <int D, int DC>
 __global__ void __launch_bounds__(bwd::NT, 2)
 bwd_rec_kernel(const float *__restrict__ qn, const float *__restrict__ kn, const float *__restrict__ e_in,
@@ -277,7 +274,10 @@ bwd_rec_kernel(const float *__restrict__ qn, const float *__restrict__ kn, const
     constexpr int RPT = D / 8, CPT = DC / 32, IV = bwd::IV, NS = D / DC;
     constexpr int NV = (3 * RPT + 31) / 32 * 32;
     constexpr int PW = 3 * D + 8;   // partial row: P dy, P de, D e [D] each, <D, P> per warp [8]
-    __shared__ float qq[IV][D], kk[IV][D], ee[IV][DC], dyy[IV][DC], al[IV], be[IV];
+    static_assert(CPT == 1, "one column per lane");
+    __shared__ __align__(16) float qq[IV][D];
+    __shared__ __align__(16) float kk[IV][D];
+    __shared__ float ee[IV][DC], dyy[IV][DC], al[IV], be[IV];
     __shared__ float red[2][8][DC];
     const int h = blockIdx.x, n = blockIdx.y, zc = blockIdx.z, c0 = zc * DC;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -293,7 +293,7 @@ bwd_rec_kernel(const float *__restrict__ qn, const float *__restrict__ kn, const
 #pragma unroll
     for (int r = 0; r < RPT; ++r)
 #pragma unroll
-        for (int m = 0; m < CPT; ++m) Dg[r][m] = dSf ? dSf[(warp + 8 * r) * D + c0 + CPT * lane + m] : 0.f;
+        for (int m = 0; m < CPT; ++m) Dg[r][m] = dSf ? dSf[(warp * RPT + r) * D + c0 + CPT * lane + m] : 0.f;
 
     for (int I = nI - 1; I >= 0; --I) {
         const int t0 = s0 + I * IV, cnt = min(IV, s1 - t0);
@@ -303,7 +303,7 @@ bwd_rec_kernel(const float *__restrict__ qn, const float *__restrict__ kn, const
 #pragma unroll
             for (int r = 0; r < RPT; ++r)
 #pragma unroll
-                for (int m = 0; m < CPT; ++m) S[r][m] = ck[(warp + 8 * r) * D + c0 + CPT * lane + m];
+                for (int m = 0; m < CPT; ++m) S[r][m] = ck[(warp * RPT + r) * D + c0 + CPT * lane + m];
         }
         __syncthreads();   // the previous interval's shared-memory reads are done
 #pragma unroll
@@ -330,24 +330,30 @@ bwd_rec_kernel(const float *__restrict__ qn, const float *__restrict__ kn, const
         for (int t = 0; t < cnt; ++t) {
             float *st = scr + (size_t)t * D * DC;
 #pragma unroll
-            for (int r = 0; r < RPT; ++r)
+            for (int r = 0; r < RPT; ++r) st[(warp * RPT + r) * DC + lane] = S[r][0];
+            const float et = ee[t][lane];
 #pragma unroll
-                for (int m = 0; m < CPT; ++m) st[(warp + 8 * r) * DC + CPT * lane + m] = S[r][m];
-#pragma unroll
-            for (int r = 0; r < RPT; ++r) {
-                const float bk = be[t] * kk[t][warp + 8 * r];
-#pragma unroll
-                for (int m = 0; m < CPT; ++m) S[r][m] = fmaf(bk, ee[t][CPT * lane + m], al[t] * S[r][m]);
+            for (int r = 0; r < RPT; r += 4) {
+                const float4 k4 = *reinterpret_cast<const float4 *>(&kk[t][warp * RPT + r]);
+                S[r][0] = fmaf(be[t] * k4.x, et, al[t] * S[r][0]);
+                S[r + 1][0] = fmaf(be[t] * k4.y, et, al[t] * S[r + 1][0]);
+                S[r + 2][0] = fmaf(be[t] * k4.z, et, al[t] * S[r + 2][0]);
+                S[r + 3][0] = fmaf(be[t] * k4.w, et, al[t] * S[r + 3][0]);
             }
         }
         // token steps in reverse
         for (int t = cnt - 1; t >= 0; --t) {
             const float *st = scr + (size_t)t * D * DC;
-            float P[RPT][CPT];
+            float P[RPT][CPT], qr[RPT], kr[RPT];
 #pragma unroll
-            for (int r = 0; r < RPT; ++r)
+            for (int r = 0; r < RPT; ++r) P[r][0] = st[(warp * RPT + r) * DC + lane];
 #pragma unroll
-                for (int m = 0; m < CPT; ++m) P[r][m] = st[(warp + 8 * r) * DC + CPT * lane + m];
+            for (int r = 0; r < RPT; r += 4) {
+                const float4 q4 = *reinterpret_cast<const float4 *>(&qq[t][warp * RPT + r]);
+                const float4 k4 = *reinterpret_cast<const float4 *>(&kk[t][warp * RPT + r]);
+                qr[r] = q4.x; qr[r + 1] = q4.y; qr[r + 2] = q4.z; qr[r + 3] = q4.w;
+                kr[r] = k4.x; kr[r + 1] = k4.y; kr[r + 2] = k4.z; kr[r + 3] = k4.w;
+            }
             float dyl[CPT], el[CPT], dp[CPT];
 #pragma unroll
             for (int m = 0; m < CPT; ++m) {
@@ -358,11 +364,10 @@ bwd_rec_kernel(const float *__restrict__ qn, const float *__restrict__ kn, const
             // D += q dy^T, then the column partials of D^T k
 #pragma unroll
             for (int r = 0; r < RPT; ++r) {
-                const float qr = qq[t][warp + 8 * r], kr = kk[t][warp + 8 * r];
 #pragma unroll
                 for (int m = 0; m < CPT; ++m) {
-                    Dg[r][m] = fmaf(qr, dyl[m], Dg[r][m]);
-                    dp[m] = fmaf(Dg[r][m], kr, dp[m]);
+                    Dg[r][m] = fmaf(qr[r], dyl[m], Dg[r][m]);
+                    dp[m] = fmaf(Dg[r][m], kr[r], dp[m]);
                 }
             }
 #pragma unroll
@@ -405,16 +410,15 @@ bwd_rec_kernel(const float *__restrict__ qn, const float *__restrict__ kn, const
 #pragma unroll
             for (int i = 0; i < NV / 32; ++i) {
                 const int idx = (NV / 32) * lane + i;
-                if (idx < 3 * RPT) pr[(idx / RPT) * D + warp + 8 * (idx % RPT)] = v[i];
+                if (idx < 3 * RPT) pr[(idx / RPT) * D + warp * RPT + idx % RPT] = v[i];
             }
             dDP = group_sum<32>(dDP);
             if (lane == 0) pr[3 * D + warp] = dDP;
             // the gradient of the state before token t
 #pragma unroll
             for (int r = 0; r < RPT; ++r) {
-                const float kr = kk[t][warp + 8 * r];
 #pragma unroll
-                for (int m = 0; m < CPT; ++m) Dg[r][m] = al[t] * fmaf(-kr, de[m], Dg[r][m]);
+                for (int m = 0; m < CPT; ++m) Dg[r][m] = al[t] * fmaf(-kr[r], de[m], Dg[r][m]);
             }
         }
     }
@@ -423,7 +427,7 @@ bwd_rec_kernel(const float *__restrict__ qn, const float *__restrict__ kn, const
 #pragma unroll
         for (int r = 0; r < RPT; ++r)
 #pragma unroll
-            for (int m = 0; m < CPT; ++m) o[(warp + 8 * r) * D + c0 + CPT * lane + m] = Dg[r][m];
+            for (int m = 0; m < CPT; ++m) o[(warp * RPT + r) * D + c0 + CPT * lane + m] = Dg[r][m];
     }
 }
 
@@ -742,7 +746,7 @@ cudaError_t launch_backward(const BackwardArgs &b, void *ws) {
                                                                dyw, static_cast<float *>(b.d_z), edy,        \
                                                                dnorm_part);                                  \
         if ((e = launched()) != cudaSuccess) return e;                                                       \
-        bwd_rec_kernel<D_, bwd::DC><<<split, bwd::NT, 0, s>>>(qn, kn, ew, dyw, fa, fb, b.f.A, b.f.b_alpha,   \
+        bwd_rec_kernel<D_, bwd::DC><<<split, bwd::NT, 0, s>>>(qn, kn, ew, dyw, fa, fb, b.f.A, b.f.b_alpha, \
                                                              b.d_S_final, b.f.cu_seqlens, n_seq, n_tok, H,  \
                                                              ckpt, scratch, dvn, part, b.d_S0);             \
         if ((e = launched()) != cudaSuccess) return e;                                                       \

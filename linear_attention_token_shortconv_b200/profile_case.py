@@ -6,6 +6,8 @@ larger than L2), run through the public binding:
         two warm-up calls, then one call
     python -m linear_attention_token_shortconv_b200.profile_case decode 64
         decode step for B sequences x 32 heads, d = 128: three steps
+    python -m linear_attention_token_shortconv_b200.profile_case backward 1024
+        prefill backward, 4 sequences x T tokens, H = 16, d = 128, fp32: three calls
 """
 import sys
 from dataclasses import replace
@@ -13,7 +15,7 @@ from dataclasses import replace
 import torch
 
 from linear_attention_token_shortconv_b200 import gdn
-from linear_attention_token_shortconv_b200.workloads import (DECODE, LONG, make_decode_inputs,
+from linear_attention_token_shortconv_b200.workloads import (DECODE, LONG, PRETRAIN, make_decode_inputs,
                                                              make_prefill_inputs, scaled)
 
 
@@ -40,6 +42,20 @@ def decode(B: int):
     print("ok", float(out.float().abs().mean()))
 
 
+def backward(T: int):
+    cfg = replace(PRETRAIN, lengths=(T,) * 4, in_dtype=torch.float32)
+    inp = make_prefill_inputs(cfg, "cuda")
+    g = torch.Generator(device="cuda")
+    g.manual_seed(cfg.seed + 100)
+    d_out = torch.randn((cfg.total_tokens, cfg.H, cfg.dv), generator=g, device="cuda")
+    for _ in range(3):
+        grads = gdn.prefill_backward(inp["q"], inp["k"], inp["v"], inp["conv_w"], inp["a_logit"], inp["b_logit"],
+                                     inp["A"], inp["b_alpha"], inp["z"], inp["norm_w"], d_out, S0=inp.get("S0"),
+                                     num_seqs=cfg.num_seqs)
+    torch.cuda.synchronize()
+    print("ok", float(grads["dq"].abs().mean()))
+
+
 if __name__ == "__main__":
     kind, size = sys.argv[1], int(sys.argv[2])
-    {"prefill": prefill, "decode": decode}[kind](size)
+    {"prefill": prefill, "decode": decode, "backward": backward}[kind](size)
