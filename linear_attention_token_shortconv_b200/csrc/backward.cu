@@ -116,9 +116,11 @@ bwd_fwd_kernel(const float *__restrict__ qn, const float *__restrict__ kn, const
                float *__restrict__ e_out) {
     static_assert(DC == 32, "8 warps x 4 columns");
     constexpr int RPT = D / 8, IV = bwd::IV;
-    __shared__ __align__(16) float qq[IV][D];
-    __shared__ __align__(16) float kk[IV][D];
-    __shared__ float vv[IV][DC], al[IV], be[IV], kq[IV];
+    constexpr int JL = D / 32;   // elements of a q or k row per lane when staging
+    // two tile buffers: the next interval's rows are loaded during this one
+    __shared__ __align__(16) float qq[2][IV][D];
+    __shared__ __align__(16) float kk[2][IV][D];
+    __shared__ float vv[2][IV][DC], al[2][IV], be[2][IV], kq[2][IV];
     const int h = blockIdx.x, n = blockIdx.y, c0 = blockIdx.z * DC;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c = 4 * warp + (lane >> 3), g = lane & 7;   // column c0 + c, rows row_of(r)
@@ -131,41 +133,70 @@ bwd_fwd_kernel(const float *__restrict__ qn, const float *__restrict__ kn, const
     for (int r = 0; r < RPT; ++r) S[r] = S0h ? S0h[row_of(r) * D + c0 + c] : 0.f;
     const size_t base = ckpt_base(s0, n);
     const float Ah = __ldg(A + h), bah = __ldg(b_alpha + h);
-    for (int t0 = s0, I = 0; t0 < s1; t0 += IV, ++I) {
-        const int cnt = min(IV, s1 - t0);
-        float *ck = ckpt + ((base + I) * H + h) * (size_t)D * D;
-#pragma unroll
-        for (int r = 0; r < RPT; ++r) ck[row_of(r) * D + c0 + c] = S[r];
-        __syncthreads();   // the previous interval's reads of the tile are done
-        // warp w stages tokens 2w, 2w + 1: q and k rows, k.q, the gates
+    // warp w's share of a tile: tokens 2w, 2w + 1 (q and k rows, v of this CTA's
+    // columns, the two gate logits), held in registers between load and store
+    float rq[2][JL], rk[2][JL], rv[2], ra[2], rb[2];
+    auto load_tile = [&](int tt0, int tcnt) {
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
             const int t = 2 * warp + u;
-            if (t < cnt) {
-                const size_t row = ((size_t)(t0 + t) * H + h) * D;
-                float dot = 0.f;
-                for (int j = lane; j < D; j += 32) {
-                    const float qv = qn[row + j], kv = kn[row + j];
-                    qq[t][j] = qv;
-                    kk[t][j] = kv;
-                    dot = fmaf(qv, kv, dot);
+            if (t < tcnt) {
+                const size_t row = ((size_t)(tt0 + t) * H + h) * D;
+#pragma unroll
+                for (int x = 0; x < JL; ++x) {
+                    rq[u][x] = qn[row + lane + 32 * x];
+                    rk[u][x] = kn[row + lane + 32 * x];
                 }
-                vv[t][lane] = vn[row + c0 + lane];
-                dot = group_sum<32>(dot);
+                rv[u] = vn[row + c0 + lane];
                 if (lane == 0) {
-                    kq[t] = dot;
-                    const size_t gi = (size_t)(t0 + t) * H + h;
-                    bwd_gates(a_logit[gi], b_logit[gi], Ah, bah, al[t], be[t]);
+                    const size_t gi = (size_t)(tt0 + t) * H + h;
+                    ra[u] = a_logit[gi];
+                    rb[u] = b_logit[gi];
                 }
             }
         }
-        __syncthreads();
+    };
+    auto store_tile = [&](int buf, int tcnt) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int t = 2 * warp + u;
+            if (t < tcnt) {
+                float dot = 0.f;
+#pragma unroll
+                for (int x = 0; x < JL; ++x) {
+                    qq[buf][t][lane + 32 * x] = rq[u][x];
+                    kk[buf][t][lane + 32 * x] = rk[u][x];
+                    dot = fmaf(rq[u][x], rk[u][x], dot);
+                }
+                vv[buf][t][lane] = rv[u];
+                dot = group_sum<32>(dot);
+                if (lane == 0) {
+                    kq[buf][t] = dot;
+                    bwd_gates(ra[u], rb[u], Ah, bah, al[buf][t], be[buf][t]);
+                }
+            }
+        }
+    };
+    const int nI = (s1 - s0 + IV - 1) / IV;
+    if (nI > 0) {
+        load_tile(s0, min(IV, s1 - s0));
+        store_tile(0, min(IV, s1 - s0));
+    }
+    __syncthreads();
+    for (int I = 0; I < nI; ++I) {
+        const int t0 = s0 + I * IV, cnt = min(IV, s1 - t0), buf = I & 1;
+        float *ck = ckpt + ((base + I) * H + h) * (size_t)D * D;
+#pragma unroll
+        for (int r = 0; r < RPT; ++r) ck[row_of(r) * D + c0 + c] = S[r];
+        const bool more = I + 1 < nI;
+        const int cnt_next = more ? min(IV, s1 - t0 - IV) : 0;
+        if (more) load_tile(t0 + IV, cnt_next);   // in flight during the token loop
         for (int t = 0; t < cnt; ++t) {
             float kr[RPT], qr[RPT];
 #pragma unroll
             for (int r = 0; r < RPT; r += 4) {
-                const float4 k4 = *reinterpret_cast<const float4 *>(&kk[t][row_of(r)]);
-                const float4 q4 = *reinterpret_cast<const float4 *>(&qq[t][row_of(r)]);
+                const float4 k4 = *reinterpret_cast<const float4 *>(&kk[buf][t][row_of(r)]);
+                const float4 q4 = *reinterpret_cast<const float4 *>(&qq[buf][t][row_of(r)]);
                 kr[r] = k4.x; kr[r + 1] = k4.y; kr[r + 2] = k4.z; kr[r + 3] = k4.w;
                 qr[r] = q4.x; qr[r + 1] = q4.y; qr[r + 2] = q4.z; qr[r + 3] = q4.w;
             }
@@ -183,15 +214,19 @@ bwd_fwd_kernel(const float *__restrict__ qn, const float *__restrict__ kn, const
                 p += __shfl_xor_sync(0xffffffffu, p, o);
                 pq += __shfl_xor_sync(0xffffffffu, pq, o);
             }
-            const float e = vv[t][c] - al[t] * p;
+            const float alt = al[buf][t], bet = be[buf][t];
+            const float e = vv[buf][t][c] - alt * p;
             if (g == 0) {
                 const size_t row = ((size_t)(t0 + t) * H + h) * D + c0 + c;
                 e_out[row] = e;
-                y_out[row] = fmaf(al[t], pq, be[t] * kq[t] * e);
+                y_out[row] = fmaf(alt, pq, bet * kq[buf][t] * e);
             }
+            const float be_e = bet * e;
 #pragma unroll
-            for (int r = 0; r < RPT; ++r) S[r] = fmaf(be[t] * kr[r], e, al[t] * S[r]);
+            for (int r = 0; r < RPT; ++r) S[r] = fmaf(kr[r], be_e, alt * S[r]);
         }
+        if (more) store_tile(buf ^ 1, cnt_next);
+        __syncthreads();   // the next tile is complete; this one's reads are done
     }
 }
 
@@ -328,9 +363,11 @@ bwd_rec_kernel(const float *__restrict__ qn, const float *__restrict__ kn, const
         __syncthreads();
         // re-run the interval: the state before each token to the scratch
         for (int t = 0; t < cnt; ++t) {
-            float *st = scr + (size_t)t * D * DC;
+            // scratch of a token: float4 x of thread tid at x * NT + tid (coalesced)
+            float4 *st4 = reinterpret_cast<float4 *>(scr + (size_t)t * D * DC);
 #pragma unroll
-            for (int r = 0; r < RPT; ++r) st[(warp * RPT + r) * DC + lane] = S[r][0];
+            for (int r = 0; r < RPT; r += 4)
+                st4[(r >> 2) * bwd::NT + tid] = make_float4(S[r][0], S[r + 1][0], S[r + 2][0], S[r + 3][0]);
             const float et = ee[t][lane];
 #pragma unroll
             for (int r = 0; r < RPT; r += 4) {
@@ -343,10 +380,13 @@ bwd_rec_kernel(const float *__restrict__ qn, const float *__restrict__ kn, const
         }
         // token steps in reverse
         for (int t = cnt - 1; t >= 0; --t) {
-            const float *st = scr + (size_t)t * D * DC;
+            const float4 *st4 = reinterpret_cast<const float4 *>(scr + (size_t)t * D * DC);
             float P[RPT][CPT], qr[RPT], kr[RPT];
 #pragma unroll
-            for (int r = 0; r < RPT; ++r) P[r][0] = st[(warp * RPT + r) * DC + lane];
+            for (int r = 0; r < RPT; r += 4) {
+                const float4 x = st4[(r >> 2) * bwd::NT + tid];
+                P[r][0] = x.x; P[r + 1][0] = x.y; P[r + 2][0] = x.z; P[r + 3][0] = x.w;
+            }
 #pragma unroll
             for (int r = 0; r < RPT; r += 4) {
                 const float4 q4 = *reinterpret_cast<const float4 *>(&qq[t][warp * RPT + r]);
