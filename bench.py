@@ -32,8 +32,9 @@ sys.path.insert(0, ROOT)
 
 from linear_attention_token_shortconv_b200 import dist as rankio  # noqa: E402
 from linear_attention_token_shortconv_b200 import gdn  # noqa: E402
-from linear_attention_token_shortconv_b200.workloads import (DECODE, LONG, PRETRAIN, make_decode_inputs,  # noqa: E402
-                                                             make_prefill_inputs, to_oracle_bits)
+from linear_attention_token_shortconv_b200.workloads import (DECODE, LONG, PRETRAIN, QSA,  # noqa: E402
+                                                             make_decode_inputs, make_prefill_inputs,
+                                                             make_qsa_inputs, to_oracle_bits)
 
 METRIC = "GDN prefill tokens/s at T=32K H=32 (% TC peak); decode state GB/s (% HBM)"
 # Algorithmic work per token-head of the fused chunked prefill (chunk C = 64, d = 128):
@@ -373,6 +374,40 @@ def bench_backward(steps, dev):
     return cfg, ms, launches
 
 
+def bench_qsa(steps, dev):
+    """gdn_qsa_indexer on one 32,768-token sequence (K = 2048, r = 4, 4 heads of
+    128): the whole call, with the inputs resident; the score matrix (0.54 GB)
+    is larger than L2."""
+    cfg = QSA
+    inp = make_qsa_inputs(cfg, dev)
+    sel = torch.empty((cfg.B, cfg.n, cfg.budget // 4), dtype=torch.int32, device=dev)
+
+    def call():
+        gdn.qsa_indexer(inp["q"], inp["k"], inp["w_q"], inp["w_k"], budget=cfg.budget, sel=sel)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches = 0
+    s.record()
+    for _ in range(steps):
+        call()
+        launches += gdn.last_call_launches()
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / steps
+    n, nb = cfg.n, cfg.n // 4
+    pairs = sum((i + 1) // 4 for i in range(n))           # (query, complete block) pairs
+    flop = pairs * 4 * 128 * 2
+    hbm = (n * 4 * 128 * 2 + n * 128 * 2                     # q, k read (bf16)
+           + 2 * pairs * 4                                   # scores written, read back
+           + n * (cfg.budget // 4) * 4)                      # selection written
+    del inp, sel
+    torch.cuda.empty_cache()
+    return cfg, ms, launches, flop, hbm
+
+
 def bench_decode_multi(cfg, T, steps, dev):
     """T consecutive tokens per sequence per step (gdn_decode_multi, all committed):
     the pool's entries [0, T) and [T, 2T) as two alternating multi-token inputs."""
@@ -534,6 +569,15 @@ def main():
                             "frac": gbs / pk["hbm_gbs"], "state_bytes_per_step": sbytes,
                             "kernel": "decode_stream", "gpu_launches": dlaunch, "clocks": dclk}
         torch.cuda.empty_cache()
+        qcfg, q_ms, qlaunch, q_flop, q_hbm = bench_qsa(5, dev)
+        result["qsa_indexer"] = {
+            "workload": qcfg.name, "steps": 5, "ms_per_step": q_ms,
+            "queries_per_s": qcfg.n / (q_ms * 1e-3),
+            "bound": "hbm", "bytes_per_call": q_hbm, "achieved_gbs": q_hbm / (q_ms * 1e-3) / 1e9,
+            "peak_gbs": pk["hbm_gbs"], "frac": q_hbm / (q_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+            "tc": {"flop_per_call": q_flop, "achieved_tflops": q_flop / (q_ms * 1e-3) / 1e12,
+                   "peak_tflops": pk["bf16_tflops"], "frac": q_flop / (q_ms * 1e-3) / 1e12 / pk["bf16_tflops"]},
+            "kernels": "qsa_prep, qsa_score (tcgen05), qsa_topk", "gpu_launches": qlaunch}
         bcfg, b_ms, blaunch = bench_backward(5, dev)
         th = bcfg.total_tokens * bcfg.H
         b_tf = BACKWARD_FLOP_PER_TOKEN_HEAD * th / (b_ms * 1e-3) / 1e12

@@ -162,6 +162,41 @@ GDN_API gdn_status_t gdn_prefill_backward(
 GDN_API gdn_status_t gdn_prefill_backward_workspace_size(const gdn_dims_t *dims, size_t *bytes);
 
 /*
+ * gdn_qsa_indexer -- the compressed lightweight indexer of Qwen Sparse Attention
+ * (slinene.github.io write-up of "On the Design of Qwen3.8-Next Architecture",
+ * 模块 B: "压缩轻量 indexer" and the block selection paragraph), for `batch`
+ * independent sequences of n tokens:
+ *   q_i^h   = PRoPE(RMSNorm(q[i, h]) * w_q, i)          (h < heads = 4)
+ *   k_bar_b = PRoPE(RMSNorm(mean(k[4b .. 4b+3])) * w_k, 4b)   (b < n / 4)
+ *   I_ib    = sum_h ReLU(<q_i^h, k_bar_b>) for complete blocks (4b + 3 <= i)
+ *   sel[i]  = the budget / 4 highest-scoring complete blocks, ties to the smaller
+ *             block index, in ascending order, padded with -1.
+ * RMSNorm: x / sqrt(mean x^2 + 1e-6) times the weight; PRoPE rotates dims [0, 64)
+ * in pairs (j, j + 32) by p * 10000^(-j / 32), dims [64, 128) unchanged.  The
+ * token set of query i is the selected blocks expanded to tokens plus the tail
+ * 4 floor((i + 1) / 4) .. i.
+ *
+ *   q       [batch, n, 4, 128] bf16 (the per-head projections W_Q^h x_i)
+ *   k       [batch, n, 128] bf16    (the shared key projection W_K x_i)
+ *   w_q, w_k [128] fp32             RMSNorm weights
+ *   sel     [batch, n, budget / 4] int32, written
+ *   scores  [batch, n, n / 4] fp32: if non-NULL the block scores are written
+ *           there (entries of incomplete blocks are left untouched); NULL keeps
+ *           them in the workspace.
+ * Supported: heads = 4, d = 128, block = 4, budget a multiple of 4.  The scores
+ * are tcgen05 products of fp16-rounded rotated rows with fp32 accumulation.  The
+ * call takes a stream-ordered workspace of gdn_qsa_indexer_workspace_size()
+ * bytes (the fp16 rows and, unless `scores` is given, the score matrix) from the
+ * library's pool.  n = 0 writes nothing.
+ */
+GDN_API gdn_status_t gdn_qsa_indexer(int batch, int n, int heads, int d, int block, int budget, const void *q,
+                                     const void *k, const float *w_q, const float *w_k, int32_t *sel,
+                                     float *scores, gdn_stream_t stream);
+
+/* Bytes of device workspace one gdn_qsa_indexer call uses (host call). */
+GDN_API gdn_status_t gdn_qsa_indexer_workspace_size(int batch, int n, size_t *bytes);
+
+/*
  * gdn_decode_step -- one token for each of B = dims->num_seqs sequences,
  * reading and updating the per-head state in place.
  *
@@ -294,6 +329,7 @@ GDN_API int gdn_last_call_launches(void);
 #define GDN_ERRF_PREP 1u    /* chunk_prep (gdn_prefill, tensor-core path) */
 #define GDN_ERRF_CHAIN 2u   /* chunk_chain (gdn_prefill, tensor-core path) */
 #define GDN_ERRF_DECODE 4u  /* streaming decode kernel (gdn_decode_step) */
+#define GDN_ERRF_QSA 8u     /* QSA indexer score kernel (gdn_qsa_indexer) */
 
 /*
  * gdn_device_error_status -- reads the current device's error words into

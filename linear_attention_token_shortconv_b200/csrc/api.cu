@@ -196,13 +196,14 @@ int gdn_last_call_launches(void) { return tl_launches; }
 
 gdn_status_t gdn_device_error_status(unsigned *flags, int clear, gdn_stream_t stream) {
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    unsigned w[3] = {0, 0, 0};
+    unsigned w[4] = {0, 0, 0, 0};
     cudaError_t e = gdn::prep_error_word(&w[0], clear != 0, s);
     if (e == cudaSuccess) e = gdn::chain_error_word(&w[1], clear != 0, s);
     if (e == cudaSuccess) e = gdn::decode_error_word(&w[2], clear != 0, s);
+    if (e == cudaSuccess) e = gdn::qsa_error_word(&w[3], clear != 0, s);
     if (e != cudaSuccess) return GDN_ERR_CUDA;
     const unsigned f = (w[0] ? GDN_ERRF_PREP : 0u) | (w[1] ? GDN_ERRF_CHAIN : 0u) |
-                       (w[2] ? GDN_ERRF_DECODE : 0u);
+                       (w[2] ? GDN_ERRF_DECODE : 0u) | (w[3] ? GDN_ERRF_QSA : 0u);
     if (flags) *flags = f;
     return f ? GDN_ERR_TIMEOUT : GDN_OK;
 }
@@ -447,6 +448,60 @@ gdn_status_t gdn_prefill_backward(const gdn_dims_t *dims, const void *q, const v
         return GDN_ERR_CUDA;
     cudaError_t e = record(g_ev_begin, a.stream);
     if (e == cudaSuccess) e = gdn::launch_backward(b, ws);
+    if (e == cudaSuccess) e = record(g_ev_end, a.stream);
+    cudaError_t ef = cudaFreeAsync(ws, a.stream);
+    if (e == cudaSuccess) e = ef;
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status_t gdn_qsa_indexer_workspace_size(int batch, int n, size_t *bytes) {
+    if (batch <= 0 || n < 0 || !bytes) return GDN_ERR_INVALID_ARG;
+    *bytes = gdn::qsa_workspace_bytes(batch, n);
+    return GDN_OK;
+}
+
+gdn_status_t gdn_qsa_indexer(int batch, int n, int heads, int d, int block, int budget, const void *q,
+                             const void *k, const float *w_q, const float *w_k, int32_t *sel, float *scores,
+                             gdn_stream_t stream) {
+    tl_launches = 0;
+    if (batch <= 0 || n < 0 || heads <= 0 || d <= 0 || block <= 0 || budget <= 0) return GDN_ERR_INVALID_ARG;
+    if (heads != 4 || d != 128 || block != 4 || budget % block != 0) return GDN_ERR_UNSUPPORTED;
+    // row coordinates of the score kernel's tensor maps stay within int32
+    if ((int64_t)batch * n * heads >= ((int64_t)1 << 31)) return GDN_ERR_UNSUPPORTED;
+    const bool empty = n == 0;
+    const void *need16[] = {q, k};
+    for (const void *p : need16) {
+        if (!p && !empty) return GDN_ERR_INVALID_ARG;
+        if (p && !aligned16(p)) return GDN_ERR_ALIGNMENT;
+    }
+    if (!sel && !empty) return GDN_ERR_INVALID_ARG;
+    if (sel && !aligned_to(sel, 4)) return GDN_ERR_ALIGNMENT;
+    if (scores && !aligned16(scores)) return GDN_ERR_ALIGNMENT;
+    const void *need4[] = {w_q, w_k};
+    for (const void *p : need4) {
+        if (!p) return GDN_ERR_INVALID_ARG;
+        if (!aligned_to(p, 4)) return GDN_ERR_ALIGNMENT;
+    }
+    if (empty) return GDN_OK;
+    gdn::QsaArgs a;
+    a.B = batch;
+    a.n = n;
+    a.KB = budget / block;
+    a.q = q;
+    a.k = k;
+    a.w_q = w_q;
+    a.w_k = w_k;
+    a.sel = sel;
+    a.scores = scores;
+    a.stream = reinterpret_cast<cudaStream_t>(stream);
+    const size_t ws_bytes = gdn::qsa_workspace_bytes(batch, n);
+    char *ws = nullptr;
+    cudaMemPool_t pool;
+    if (get_pool(&pool) != cudaSuccess) return GDN_ERR_CUDA;
+    if (cudaMallocFromPoolAsync(reinterpret_cast<void **>(&ws), ws_bytes, pool, a.stream) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    cudaError_t e = record(g_ev_begin, a.stream);
+    if (e == cudaSuccess) e = gdn::launch_qsa_indexer(a, ws);
     if (e == cudaSuccess) e = record(g_ev_end, a.stream);
     cudaError_t ef = cudaFreeAsync(ws, a.stream);
     if (e == cudaSuccess) e = ef;

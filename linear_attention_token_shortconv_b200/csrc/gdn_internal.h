@@ -79,6 +79,22 @@ struct BackwardArgs {
 size_t backward_workspace_bytes(int n_seq, int n_tok, int H, int D);
 cudaError_t launch_backward(const BackwardArgs &b, void *ws);
 
+// K5: QSA compressed indexer (H = 4 heads of d = 128, blocks of 4 tokens): q
+// [B, n, 4, 128] and k [B, n, 128] bf16, weights [128] fp32; sel [B, n, KB] int32;
+// scores [B, n, n / 4] fp32 (NULL: kept in the workspace).
+struct QsaArgs {
+    int B, n, KB;
+    const void *q, *k;
+    const float *w_q, *w_k;
+    int32_t *sel;
+    float *scores;
+    cudaStream_t stream;
+};
+size_t qsa_workspace_bytes(int B, int n);
+size_t qsa_scores_bytes(int B, int n);
+cudaError_t launch_qsa_indexer(const QsaArgs &a, void *ws);
+cudaError_t qsa_error_word(unsigned *v, bool clear, cudaStream_t s);
+
 // K2f: token-by-token recurrence with the fused gates and output stage (SIMT fp32).
 cudaError_t launch_recurrent(const PrefillArgs &a, const float *qn, const float *kn,
                              const float *vn);

@@ -1,0 +1,345 @@
+// K5 -- the QSA compressed indexer (slinene.github.io write-up of "On the Design
+// of Qwen3.8-Next Architecture", 模块 B — Qwen Sparse Attention: "压缩轻量 indexer"
+// and the block selection paragraph), for H = 4 indexer heads of d = 128 and
+// blocks of r = 4 tokens:
+//   q_i^h = PRoPE(RMSNorm(q_raw_i^h) w_q, i),
+//   k_bar_b = PRoPE(RMSNorm(mean(k_raw_{4b .. 4b+3})) w_k, 4b),
+//   I_ib = sum_h ReLU(<q_i^h, k_bar_b>) for complete blocks (4b + 3 <= i),
+//   B_i = the ceil(K / 4) highest-scoring complete blocks (ties to the smaller
+//   block), ascending, padded with -1.  The tokens the sparse attention reads are
+//   the blocks expanded plus the tail 4 floor((i + 1) / 4) .. i (implied).
+// RMSNorm is x / sqrt(mean x^2 + 1e-6) times its weight; PRoPE rotates dims
+// [0, 64) as pairs (j, j + 32) by p 10000^(-j / 32) and keeps dims [64, 128).
+//
+// Kernels:
+//  K5a qsa_prep_kernel: one warp per query row (all 4 heads) or key block:
+//      RMSNorm, rotation (the angle reduced in double precision: positions reach
+//      1e5 and more), fp16 rows [(i, h)][128] and [b][128].
+//  K5b qsa_score_kernel: tcgen05, one CTA per (32 queries = 128 rows of (i, h),
+//      256 blocks): both operands by TMA in the 128-byte swizzled K-major layout,
+//      eight K = 16 MMAs into 256 TMEM columns; the epilogue applies ReLU and sums
+//      the 4 heads (lanes 4q .. 4q + 3) with two shuffles and stores the scores
+//      of complete blocks.  Tiles entirely past the causal limit do nothing.
+//  K5c qsa_topk_kernel: one CTA per query row: a radix select on the score bits
+//      (scores are >= 0, so their bit patterns order like the values) finds the
+//      threshold, then a block scan writes the selected blocks in ascending
+//      order, equal scores at the threshold taken from the smallest index.
+#include <cuda.h>
+#include <cuda_fp16.h>
+
+#include <cstring>
+
+#include "gdn_device.cuh"
+#include "gdn_internal.h"
+#include "umma.cuh"
+
+namespace gdn {
+
+__device__ unsigned int g_qsa_err;
+
+namespace qsa {
+constexpr int D = 128, HI = 4, R = 4;
+constexpr int QT = 32;          // queries per score tile (128 MMA rows)
+constexpr int BT = 256;         // blocks per score tile (MMA N)
+constexpr int OFF_A = 0;        // 2 k-blocks x 128 rows x 128 B
+constexpr int OFF_B = 32768;    // 2 k-blocks x 256 rows x 128 B
+constexpr int OFF_BAR = 98304;
+constexpr int SMEM = OFF_BAR + 64 + 1024;
+constexpr double ROPE_BASE = 10000.0;
+}  // namespace qsa
+
+// ------------------------------------------------------------------ K5a: prep
+__device__ __forceinline__ void qsa_norm_rope(float (&x)[4], const float *__restrict__ w, long long pos,
+                                              int lane) {
+    // lane holds dims lane, lane + 32, lane + 64, lane + 96
+    float ss = 0.f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) ss = fmaf(x[u], x[u], ss);
+    ss = group_sum<32>(ss);
+    const float rn = 1.0f / sqrtf(ss / qsa::D + kNormEps);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) x[u] *= rn * __ldg(w + lane + 32 * u);
+    // rotate the pair (lane, lane + 32) by pos * base^(-lane / 32)
+    const double ang = (double)pos * pow(qsa::ROPE_BASE, -(double)lane / 32.0);
+    double sd, cd;
+    sincos(ang, &sd, &cd);
+    const float c = (float)cd, s = (float)sd;
+    const float a = x[0], b = x[1];
+    x[0] = a * c - b * s;
+    x[1] = a * s + b * c;
+}
+
+__global__ void __launch_bounds__(256)
+qsa_prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const float *__restrict__ w_q,
+                const float *__restrict__ w_k, int B, int n, __half *__restrict__ qr, __half *__restrict__ kb) {
+    using namespace qsa;
+    const int nb = n / R;
+    const long long n_q = (long long)B * n, n_items = n_q + (long long)B * nb;
+    const int lane = threadIdx.x & 31;
+    for (long long it = (long long)blockIdx.x * 8 + (threadIdx.x >> 5); it < n_items; it += (long long)gridDim.x * 8) {
+        if (it < n_q) {   // query row (sequence it / n, token it % n), all heads
+            const long long i = it % n;
+#pragma unroll
+            for (int h = 0; h < HI; ++h) {
+                const bf16 *src = q + (it * HI + h) * D;
+                float x[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) x[u] = __bfloat162float(src[lane + 32 * u]);
+                qsa_norm_rope(x, w_q, i, lane);
+                __half *dst = qr + (it * HI + h) * D;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) dst[lane + 32 * u] = __float2half_rn(x[u]);
+            }
+        } else {          // key block: mean of 4 raw keys
+            const long long jb = it - n_q, s = jb / nb, b = jb % nb;
+            const bf16 *src = k + (s * n + b * R) * D;
+            float x[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                float acc = 0.f;
+#pragma unroll
+                for (int t = 0; t < R; ++t) acc += __bfloat162float(src[t * D + lane + 32 * u]);
+                x[u] = acc * (1.0f / R);
+            }
+            qsa_norm_rope(x, w_k, b * R, lane);
+            __half *dst = kb + jb * D;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) dst[lane + 32 * u] = __float2half_rn(x[u]);
+        }
+    }
+}
+
+// ------------------------------------------------------------------ K5b: scores
+struct QsaMaps {
+    CUtensorMap q, k;   // [rows][128] fp16, box {64, 128} and {64, 256}, 128-byte swizzle
+};
+
+__global__ void __launch_bounds__(128, 1)
+qsa_score_kernel(const __grid_constant__ QsaMaps maps, int n, float *__restrict__ scores) {
+    using namespace qsa;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bar_ld = reinterpret_cast<uint64_t *>(sm + OFF_BAR);        // operand loads
+    uint64_t *bar_mma = reinterpret_cast<uint64_t *>(sm + OFF_BAR + 8);   // MMA completion
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 16);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nb = n / R;
+    const int bt = blockIdx.x, qt = blockIdx.y, s = blockIdx.z;
+    const int i_last = min(QT * qt + QT - 1, n - 1);
+    // complete blocks of the tile's last query; nothing to do past them
+    if (BT * bt >= (i_last + 1) / R) return;   // uniform per CTA
+
+    if (warp == 0) umma::tmem_alloc(tslot, BT);
+    if (tid == 0) {
+        umma::mbar_init(bar_ld, 1);
+        umma::mbar_init(bar_mma, 1);
+        umma::fence_mbar_init();
+    }
+    umma::tc_fence_before();
+    __syncthreads();
+    umma::tc_fence_after();
+    const uint32_t tbase = *tslot;
+    bool ok = true;
+    if (tid == 0) {
+        umma::mbar_expect_tx(bar_ld, 2 * 128 * 128 + 2 * 256 * 128);
+        const int qrow = (s * n + QT * qt) * HI, krow = s * nb + BT * bt;
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb) {
+            umma::tma_load_3d(sm + OFF_A + kb * 16384, &maps.q, 64 * kb, 0, qrow, bar_ld);
+            umma::tma_load_3d(sm + OFF_B + kb * 32768, &maps.k, 64 * kb, 0, krow, bar_ld);
+        }
+        ok = umma::mbar_wait_bounded(bar_ld, 0, 1u << 24);
+        if (ok) {
+            umma::tc_fence_after();
+            const uint32_t a = umma::smem_u32(sm + OFF_A), b = umma::smem_u32(sm + OFF_B);
+            const uint32_t idesc = umma::idesc_f16(128, BT, false, false);
+#pragma unroll
+            for (int st = 0; st < D / 16; ++st) {
+                const uint64_t ad = umma::sw128_desc(a + (st / 4) * 16384 + (st % 4) * 32, 16, 1024);
+                const uint64_t bd = umma::sw128_desc(b + (st / 4) * 32768 + (st % 4) * 32, 16, 1024);
+                umma::mma_f16(tbase, ad, bd, idesc, st > 0);
+            }
+            umma::mma_commit(bar_mma);
+        } else {
+            atomicOr(&g_qsa_err, 1u);
+        }
+    }
+    ok = __syncthreads_and(ok);   // the MMA was issued
+    if (ok) ok = __syncthreads_and(umma::mbar_wait_bounded(bar_mma, 0, 1u << 24));
+    if (ok) {
+        umma::tc_fence_after();
+        // warp w: TMEM lanes 32w .. 32w + 31 = rows (query 8w + l / 4, head l % 4)
+        const int i = QT * qt + 8 * warp + (lane >> 2);
+        const int n_valid = (i + 1) / R;   // complete blocks of query i
+        const uint32_t trow = tbase + ((uint32_t)(32 * warp) << 16);
+        float *dst = scores + ((size_t)s * n + i) * nb;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BT; c0 += 32) {
+            if (BT * bt + c0 >= (i_last + 1) / R) break;   // uniform: nothing valid past here
+            float v[32];
+            umma::tmem_ld32(trow + c0, v);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                float x = fmaxf(v[j], 0.f);
+                x += __shfl_xor_sync(0xffffffffu, x, 1);
+                x += __shfl_xor_sync(0xffffffffu, x, 2);
+                v[j] = x;
+            }
+            if ((lane & 3) == 0 && i < n) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int b = BT * bt + c0 + j;
+                    if (b < n_valid) dst[b] = v[j];
+                }
+            }
+        }
+    } else if (tid == 0) {
+        atomicOr(&g_qsa_err, 1u);
+    }
+    umma::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) umma::tmem_dealloc(tbase, BT);
+}
+
+// ------------------------------------------------------------------ K5c: top-k
+// Block-wide exclusive scan of one int per thread (256 threads); returns the
+// thread's exclusive prefix and writes the total to *total.
+__device__ __forceinline__ int qsa_block_scan(int x, int *wsum, int *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    int base = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+        const int v = wsum[w];
+        if (w < warp) base += v;
+        tot += v;
+    }
+    __syncthreads();   // wsum is reused by the next scan
+    *total = tot;
+    return base + incl - x;
+}
+
+__global__ void __launch_bounds__(256)
+qsa_topk_kernel(const float *__restrict__ scores, int n, int KB, int32_t *__restrict__ sel) {
+    __shared__ int hist[256];
+    __shared__ int wsum[8];
+    __shared__ unsigned sh_prefix;
+    __shared__ int sh_remaining;
+    const int tid = threadIdx.x;
+    const long long row = blockIdx.x;   // s * n + i
+    const int i = (int)(row % n);
+    const int nb = n / qsa::R;
+    const int n_valid = (i + 1) / qsa::R;
+    const float *sc = scores + row * nb;
+    int32_t *out = sel + row * KB;
+    if (n_valid <= KB) {   // every complete block
+        for (int j = tid; j < KB; j += 256) out[j] = j < n_valid ? j : -1;
+        return;
+    }
+    auto key_of = [&](int b) -> unsigned {
+        const float v = sc[b];
+        return v > 0.f ? __float_as_uint(v) : 0u;   // scores >= 0: bits order like values (-0 -> 0)
+    };
+    // radix select of the KB-th largest key, 8 bits per pass from the top
+    unsigned prefix = 0, mask = 0;
+    int remaining = KB;
+#pragma unroll 1
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        hist[tid] = 0;
+        __syncthreads();
+        for (int b = tid; b < n_valid; b += 256) {
+            const unsigned key = key_of(b);
+            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+        }
+        __syncthreads();
+        if (tid == 0) {
+            int above = 0, d = 255;
+            for (; d > 0; --d) {
+                if (above + hist[d] >= remaining) break;
+                above += hist[d];
+            }
+            sh_remaining = remaining - above;
+            sh_prefix = prefix | ((unsigned)d << shift);
+        }
+        __syncthreads();
+        remaining = sh_remaining;
+        prefix = sh_prefix;
+        mask |= 255u << shift;
+        __syncthreads();   // hist is cleared by the next pass
+    }
+    // keys above the threshold, and the first `remaining` equal to it in index order
+    const unsigned T = prefix;
+    int eq_base = 0, out_base = 0;
+#pragma unroll 1
+    for (int c0 = 0; c0 < n_valid; c0 += 256) {
+        const int b = c0 + tid;
+        const unsigned key = b < n_valid ? key_of(b) : 0u;
+        const int gt = (b < n_valid && key > T) ? 1 : 0, eq = (b < n_valid && key == T) ? 1 : 0;
+        int eq_tot, sel_tot;
+        const int eq_rank = eq_base + qsa_block_scan(eq, wsum, &eq_tot);
+        const int take = gt || (eq && eq_rank < remaining);
+        const int pos = out_base + qsa_block_scan(take, wsum, &sel_tot);
+        if (take) out[pos] = b;
+        eq_base += eq_tot;
+        out_base += sel_tot;
+    }
+}
+
+// ------------------------------------------------------------------ host
+size_t qsa_scores_bytes(int B, int n) { return (size_t)B * n * (n / qsa::R) * 4; }
+
+size_t qsa_workspace_bytes(int B, int n) {
+    auto ru = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    return ru((size_t)B * n * qsa::HI * qsa::D * 2) + ru((size_t)B * (n / qsa::R) * qsa::D * 2) + ru(qsa_scores_bytes(B, n));
+}
+
+cudaError_t launch_qsa_indexer(const QsaArgs &a, void *ws) {
+    using namespace qsa;
+    auto ru = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    const int nb = a.n / R;
+    char *p = static_cast<char *>(ws);
+    __half *qr = reinterpret_cast<__half *>(p);
+    p += ru((size_t)a.B * a.n * HI * D * 2);
+    __half *kb = reinterpret_cast<__half *>(p);
+    p += ru((size_t)a.B * nb * D * 2);
+    float *scores = a.scores ? a.scores : reinterpret_cast<float *>(p);
+    cudaError_t e;
+    const long long items = (long long)a.B * a.n + (long long)a.B * nb;
+    if (items == 0) return cudaSuccess;
+    const long long want_blocks = (items + 7) / 8;
+    const int grid = (int)(want_blocks < 148LL * 16 ? want_blocks : 148LL * 16);
+    qsa_prep_kernel<<<grid, 256, 0, a.stream>>>((const bf16 *)a.q, (const bf16 *)a.k, a.w_q, a.w_k, a.B, a.n, qr, kb);
+    if ((e = launched()) != cudaSuccess) return e;
+    if (nb > 0) {
+        QsaMaps m;
+        std::memset(&m, 0, sizeof m);
+        if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.q), qr, false, D, 1, a.B * a.n * HI, 64, 128, true)) != cudaSuccess)
+            return e;
+        if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.k), kb, false, D, 1, a.B * nb, 64, BT, true)) != cudaSuccess)
+            return e;
+        if ((e = cudaFuncSetAttribute(qsa_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM)) != cudaSuccess)
+            return e;
+        const dim3 g((nb + BT - 1) / BT, (a.n + QT - 1) / QT, a.B);
+        qsa_score_kernel<<<g, 128, SMEM, a.stream>>>(m, a.n, scores);
+        if ((e = launched()) != cudaSuccess) return e;
+    }
+    if (a.n > 0) {
+        qsa_topk_kernel<<<(unsigned)((long long)a.B * a.n), 256, 0, a.stream>>>(scores, a.n, a.KB, a.sel);
+        if ((e = launched()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+cudaError_t qsa_error_word(unsigned *v, bool clear, cudaStream_t s) {
+    return read_error_word(g_qsa_err, v, clear, s);
+}
+
+}  // namespace gdn

@@ -25,8 +25,8 @@ EXPORTS = ("gdn_prefill", "gdn_prefill_workspace_size", "gdn_decode_step", "gdn_
            "gdn_set_timing_events", "gdn_selftest_umma", "gdn_prefill_noalloc",
            "gdn_set_kernel_events", "gdn_last_call_launches", "gdn_device_error_status",
            "gdn_selftest_wait_timeout", "gdn_decode_multi", "gdn_prefill_backward",
-           "gdn_prefill_backward_workspace_size")
-ERRF_PREP, ERRF_CHAIN, ERRF_DECODE = 1, 2, 4
+           "gdn_prefill_backward_workspace_size", "gdn_qsa_indexer", "gdn_qsa_indexer_workspace_size")
+ERRF_PREP, ERRF_CHAIN, ERRF_DECODE, ERRF_QSA = 1, 2, 4, 8
 
 
 class GdnError(RuntimeError):
@@ -66,6 +66,10 @@ def load() -> ctypes.CDLL:
         lib.gdn_prefill_backward.restype = ctypes.c_int
         lib.gdn_prefill_backward_workspace_size.argtypes = [D, ctypes.POINTER(ctypes.c_size_t)]
         lib.gdn_prefill_backward_workspace_size.restype = ctypes.c_int
+        lib.gdn_qsa_indexer.argtypes = [ctypes.c_int] * 6 + [P] * 7
+        lib.gdn_qsa_indexer.restype = ctypes.c_int
+        lib.gdn_qsa_indexer_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)]
+        lib.gdn_qsa_indexer_workspace_size.restype = ctypes.c_int
         lib.gdn_prefill_noalloc.argtypes = [D] + [P] * 15
         lib.gdn_prefill_noalloc.restype = ctypes.c_int
         lib.gdn_selftest_umma.argtypes = [ctypes.c_int] * 5 + [P] * 5
@@ -175,6 +179,28 @@ def prefill_backward_workspace_size(n_seq, n_tok, H, dk, dv, conv_k=4) -> int:
     _check(load().gdn_prefill_backward_workspace_size(ctypes.byref(dims), ctypes.byref(n)),
            "gdn_prefill_backward_workspace_size")
     return n.value
+
+
+def qsa_indexer(q, k, w_q, w_k, budget=2048, *, sel=None, scores=None, want_scores=False, stream=None):
+    """gdn_qsa_indexer on torch tensors: q [B, n, 4, 128] and k [B, n, 128] bf16
+    (a leading batch dimension may be omitted), w_q, w_k [128] fp32.
+
+    Returns (sel [B, n, budget / 4] int32, scores [B, n, n / 4] fp32 or None)."""
+    squeeze = q.dim() == 3
+    if squeeze:
+        q, k = q.unsqueeze(0), k.unsqueeze(0)
+    B, n, H, d = q.shape
+    if sel is None:
+        sel = torch.empty((B, n, budget // 4), dtype=torch.int32, device=q.device)
+    if scores is None and want_scores:
+        scores = torch.empty((B, n, n // 4), dtype=torch.float32, device=q.device)
+    rc = load().gdn_qsa_indexer(B, n, H, d, 4, budget, _ptr(q), _ptr(k), _ptr(w_q), _ptr(w_k), _ptr(sel),
+                                _ptr(scores), _stream(stream))
+    _check(rc, "gdn_qsa_indexer")
+    if squeeze:
+        sel = sel[0]
+        scores = None if scores is None else scores[0]
+    return sel, scores
 
 
 def prefill_noalloc(q, k, v, conv_w, a_logit, b_logit, A, b_alpha, z, norm_w, S0=None,

@@ -198,3 +198,30 @@ def to_oracle_bits(t: torch.Tensor) -> np.ndarray:
     if t.dtype == torch.int32:
         return t.numpy()
     raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+@dataclass(frozen=True)
+class QsaConfig:
+    """QSA compressed indexer workload: `B` sequences of `n` tokens, 4 indexer
+    heads of 128 dims, blocks of 4 tokens, a token budget of `budget`."""
+    name: str
+    B: int
+    n: int
+    budget: int = 2048
+    seed: int = 5
+
+
+QSA = QsaConfig("qsa indexer n=32768 B=1 K=2048 r=4 H=4 d=128", 1, 32768)
+
+
+def make_qsa_inputs(cfg: QsaConfig, device="cpu", seed=None) -> dict:
+    """Projected indexer queries [B, n, 4, 128] and shared keys [B, n, 128] ~ N(0, 1)
+    in bf16; RMSNorm weights 1 + N(0, 0.01) (std 0.1) in fp32."""
+    device = torch.device(device)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(cfg.seed if seed is None else seed)
+    d = {"q": _normal((cfg.B, cfg.n, 4, 128), gen, device).to(torch.bfloat16),
+         "k": _normal((cfg.B, cfg.n, 128), gen, device).to(torch.bfloat16),
+         "w_q": _normal((128,), gen, device, std=0.1, mean=1.0),
+         "w_k": _normal((128,), gen, device, std=0.1, mean=1.0)}
+    return d

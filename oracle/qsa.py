@@ -73,7 +73,7 @@ def scores(q_raw, k_raw, w_q, w_k, r=4):
     block b is not complete at token i."""
     q = queries(q_raw, w_q)
     kb = keys(k_raw, w_k, r)
-    s = np.maximum(np.einsum("ihd,bd->ihb", q, kb), 0.0).sum(axis=1)
+    s = np.maximum(q @ kb.T, 0.0).sum(axis=1)            # [n, H, nb] -> [n, nb]
     n, nb = s.shape
     complete = (np.arange(nb)[None, :] * r + r - 1) <= np.arange(n)[:, None]
     return np.where(complete, s, -np.inf)
