@@ -173,6 +173,7 @@ qsa_score_kernel(const __grid_constant__ QsaMaps maps, int n, float *__restrict_
         const int n_valid = (i + 1) / R;   // complete blocks of query i
         const uint32_t trow = tbase + ((uint32_t)(32 * warp) << 16);
         float *dst = scores + ((size_t)s * n + i) * nb;
+        const bool vec = (nb & 3) == 0;   // rows start on 16-byte boundaries
 #pragma unroll 1
         for (int c0 = 0; c0 < BT; c0 += 32) {
             if (BT * bt + c0 >= (i_last + 1) / R) break;   // uniform: nothing valid past here
@@ -185,11 +186,25 @@ qsa_score_kernel(const __grid_constant__ QsaMaps maps, int n, float *__restrict_
                 x += __shfl_xor_sync(0xffffffffu, x, 2);
                 v[j] = x;
             }
-            if ((lane & 3) == 0 && i < n) {
+            // the 4 lanes of a query hold the same sums: lane 4q + j stores scores
+            // 8j .. 8j + 7 of the chunk (two 16-byte stores when rows are aligned)
+            const int j8 = 8 * (lane & 3);
+            float o[8];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int b = BT * bt + c0 + j;
-                    if (b < n_valid) dst[b] = v[j];
+            for (int x = 0; x < 8; ++x) {
+                const float a0 = v[x], a1 = v[8 + x], a2 = v[16 + x], a3 = v[24 + x];
+                o[x] = j8 == 0 ? a0 : (j8 == 8 ? a1 : (j8 == 16 ? a2 : a3));
+            }
+            const int b0 = BT * bt + c0 + j8;
+            if (i < n) {
+                if (vec && b0 + 8 <= n_valid) {
+                    float4 *d4 = reinterpret_cast<float4 *>(dst + b0);
+                    d4[0] = make_float4(o[0], o[1], o[2], o[3]);
+                    d4[1] = make_float4(o[4], o[5], o[6], o[7]);
+                } else {
+#pragma unroll
+                    for (int x = 0; x < 8; ++x)
+                        if (b0 + x < n_valid) dst[b0 + x] = o[x];
                 }
             }
         }
@@ -202,37 +217,18 @@ qsa_score_kernel(const __grid_constant__ QsaMaps maps, int n, float *__restrict_
 }
 
 // ------------------------------------------------------------------ K5c: top-k
-// Block-wide exclusive scan of one int per thread (256 threads); returns the
-// thread's exclusive prefix and writes the total to *total.
-__device__ __forceinline__ int qsa_block_scan(int x, int *wsum, int *total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int incl = x;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-    }
-    if (lane == 31) wsum[warp] = incl;
-    __syncthreads();
-    int base = 0, tot = 0;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) {
-        const int v = wsum[w];
-        if (w < warp) base += v;
-        tot += v;
-    }
-    __syncthreads();   // wsum is reused by the next scan
-    *total = tot;
-    return base + incl - x;
-}
+namespace qsa {
+constexpr int TOPK_CAP = 12288;   // row keys kept in shared memory up to this many blocks (48 KB)
+}  // namespace qsa
 
 __global__ void __launch_bounds__(256)
 qsa_topk_kernel(const float *__restrict__ scores, int n, int KB, int32_t *__restrict__ sel) {
+    extern __shared__ unsigned keys_s[];   // [min(n_valid, TOPK_CAP)]
     __shared__ int hist[256];
-    __shared__ int wsum[8];
+    __shared__ int wcnt[8][2];
     __shared__ unsigned sh_prefix;
     __shared__ int sh_remaining;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const long long row = blockIdx.x;   // s * n + i
     const int i = (int)(row % n);
     const int nb = n / qsa::R;
@@ -247,6 +243,12 @@ qsa_topk_kernel(const float *__restrict__ scores, int n, int KB, int32_t *__rest
         const float v = sc[b];
         return v > 0.f ? __float_as_uint(v) : 0u;   // scores >= 0: bits order like values (-0 -> 0)
     };
+    const bool in_smem = n_valid <= qsa::TOPK_CAP;   // uniform
+    if (in_smem) {
+        for (int b = tid; b < n_valid; b += 256) keys_s[b] = key_of(b);
+        __syncthreads();
+    }
+    auto key_at = [&](int b) -> unsigned { return in_smem ? keys_s[b] : key_of(b); };
     // radix select of the KB-th largest key, 8 bits per pass from the top
     unsigned prefix = 0, mask = 0;
     int remaining = KB;
@@ -256,18 +258,28 @@ qsa_topk_kernel(const float *__restrict__ scores, int n, int KB, int32_t *__rest
         hist[tid] = 0;
         __syncthreads();
         for (int b = tid; b < n_valid; b += 256) {
-            const unsigned key = key_of(b);
+            const unsigned key = key_at(b);
             if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
         }
         __syncthreads();
-        if (tid == 0) {
-            int above = 0, d = 255;
-            for (; d > 0; --d) {
-                if (above + hist[d] >= remaining) break;
-                above += hist[d];
+        // the digit holding the remaining-th largest key: thread t takes digit
+        // 255 - t; a block scan of the counts in that order crosses `remaining`
+        // at exactly one thread
+        {
+            const int c = hist[255 - tid];
+            int incl = c;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
             }
-            sh_remaining = remaining - above;
-            sh_prefix = prefix | ((unsigned)d << shift);
+            if (lane == 31) wcnt[warp][0] = incl;
+            __syncthreads();
+            for (int w = 0; w < warp; ++w) incl += wcnt[w][0];
+            if (incl >= remaining && incl - c < remaining) {
+                sh_remaining = remaining - (incl - c);
+                sh_prefix = prefix | ((unsigned)(255 - tid) << shift);
+            }
         }
         __syncthreads();
         remaining = sh_remaining;
@@ -275,21 +287,42 @@ qsa_topk_kernel(const float *__restrict__ scores, int n, int KB, int32_t *__rest
         mask |= 255u << shift;
         __syncthreads();   // hist is cleared by the next pass
     }
-    // keys above the threshold, and the first `remaining` equal to it in index order
+    // Selection: the keys above the threshold T and the first `remaining` equal to
+    // it in index order.  Warp w owns a contiguous segment of the row; it counts
+    // its keys above and equal to T, the warps exchange counts once, and each
+    // warp then writes its selected blocks at their ascending positions.
     const unsigned T = prefix;
-    int eq_base = 0, out_base = 0;
-#pragma unroll 1
-    for (int c0 = 0; c0 < n_valid; c0 += 256) {
-        const int b = c0 + tid;
-        const unsigned key = b < n_valid ? key_of(b) : 0u;
-        const int gt = (b < n_valid && key > T) ? 1 : 0, eq = (b < n_valid && key == T) ? 1 : 0;
-        int eq_tot, sel_tot;
-        const int eq_rank = eq_base + qsa_block_scan(eq, wsum, &eq_tot);
-        const int take = gt || (eq && eq_rank < remaining);
-        const int pos = out_base + qsa_block_scan(take, wsum, &sel_tot);
-        if (take) out[pos] = b;
-        eq_base += eq_tot;
-        out_base += sel_tot;
+    const int seg = (((n_valid + 7) / 8) + 31) / 32 * 32;
+    const int b_lo = min(warp * seg, n_valid), b_hi = min(b_lo + seg, n_valid);
+    const unsigned lt = (1u << lane) - 1u;
+    int n_gt = 0, n_eq = 0;
+    for (int b0 = b_lo; b0 < b_hi; b0 += 32) {
+        const int b = b0 + lane;
+        const unsigned key = b < b_hi ? key_at(b) : 0u;
+        n_gt += __popc(__ballot_sync(0xffffffffu, b < b_hi && key > T));
+        n_eq += __popc(__ballot_sync(0xffffffffu, b < b_hi && key == T));
+    }
+    if (lane == 0) {
+        wcnt[warp][0] = n_gt;
+        wcnt[warp][1] = n_eq;
+    }
+    __syncthreads();
+    int gt_before = 0, eq_before = 0;
+    for (int w = 0; w < warp; ++w) {
+        gt_before += wcnt[w][0];
+        eq_before += wcnt[w][1];
+    }
+    int eq_run = eq_before, out_run = gt_before + min(eq_before, remaining);
+    for (int b0 = b_lo; b0 < b_hi; b0 += 32) {
+        const int b = b0 + lane;
+        const unsigned key = b < b_hi ? key_at(b) : 0u;
+        const bool gt = b < b_hi && key > T, eq = b < b_hi && key == T;
+        const unsigned eq_mask = __ballot_sync(0xffffffffu, eq);
+        const bool take = gt || (eq && eq_run + __popc(eq_mask & lt) < remaining);
+        const unsigned take_mask = __ballot_sync(0xffffffffu, take);
+        if (take) out[out_run + __popc(take_mask & lt)] = b;
+        eq_run += __popc(eq_mask);
+        out_run += __popc(take_mask);
     }
 }
 
@@ -332,7 +365,12 @@ cudaError_t launch_qsa_indexer(const QsaArgs &a, void *ws) {
         if ((e = launched()) != cudaSuccess) return e;
     }
     if (a.n > 0) {
-        qsa_topk_kernel<<<(unsigned)((long long)a.B * a.n), 256, 0, a.stream>>>(scores, a.n, a.KB, a.sel);
+        const int cap = nb < qsa::TOPK_CAP ? nb : qsa::TOPK_CAP;
+        if ((e = cudaFuncSetAttribute(qsa_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, cap * 4)) !=
+            cudaSuccess)
+            return e;
+        qsa_topk_kernel<<<(unsigned)((long long)a.B * a.n), 256, (size_t)cap * 4, a.stream>>>(scores, a.n, a.KB,
+                                                                                             a.sel);
         if ((e = launched()) != cudaSuccess) return e;
     }
     return cudaSuccess;
