@@ -15,11 +15,12 @@
 //  K5a qsa_prep_kernel: one warp per query row (all 4 heads) or key block:
 //      RMSNorm, rotation (the angle reduced in double precision: positions reach
 //      1e5 and more), fp16 rows [(i, h)][128] and [b][128].
-//  K5b qsa_score_kernel: tcgen05, one CTA per (32 queries = 128 rows of (i, h),
-//      256 blocks): both operands by TMA in the 128-byte swizzled K-major layout,
-//      eight K = 16 MMAs into 256 TMEM columns; the epilogue applies ReLU and sums
-//      the 4 heads (lanes 4q .. 4q + 3) with two shuffles and stores the scores
-//      of complete blocks.  Tiles entirely past the causal limit do nothing.
+//  K5b qsa_score_kernel: tcgen05, one CTA of 8 warps per (32 queries = 128 rows
+//      of (i, h), 256 blocks): both operands by TMA in the 128-byte swizzled
+//      K-major layout, eight K = 16 MMAs into 256 TMEM columns; the epilogue
+//      (two warps per TMEM lane quadrant, half the columns each) applies ReLU,
+//      sums the 4 heads (lanes 4q .. 4q + 3) with two shuffles and stores the
+//      scores of complete blocks.  Tiles entirely past the causal limit do nothing.
 //  K5c qsa_topk_kernel: one CTA per query row: a radix select on the score bits
 //      (scores are >= 0, so their bit patterns order like the values) finds the
 //      threshold, then a block scan writes the selected blocks in ascending
@@ -114,7 +115,7 @@ struct QsaMaps {
     CUtensorMap q, k;   // [rows][128] fp16, box {64, 128} and {64, 256}, 128-byte swizzle
 };
 
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(256, 1)
 qsa_score_kernel(const __grid_constant__ QsaMaps maps, int n, float *__restrict__ scores) {
     using namespace qsa;
     extern __shared__ uint8_t smem_raw[];
@@ -168,14 +169,16 @@ qsa_score_kernel(const __grid_constant__ QsaMaps maps, int n, float *__restrict_
     if (ok) ok = __syncthreads_and(umma::mbar_wait_bounded(bar_mma, 0, 1u << 24));
     if (ok) {
         umma::tc_fence_after();
-        // warp w: TMEM lanes 32w .. 32w + 31 = rows (query 8w + l / 4, head l % 4)
-        const int i = QT * qt + 8 * warp + (lane >> 2);
+        // warps w and w + 4: TMEM lanes 32 (w % 4) .. + 31 = rows (query 8 (w % 4) + l / 4,
+        // head l % 4); warp w takes block columns 128 (w / 4) .. + 127
+        const int quad = warp & 3, half = warp >> 2;
+        const int i = QT * qt + 8 * quad + (lane >> 2);
         const int n_valid = (i + 1) / R;   // complete blocks of query i
-        const uint32_t trow = tbase + ((uint32_t)(32 * warp) << 16);
+        const uint32_t trow = tbase + ((uint32_t)(32 * quad) << 16);
         float *dst = scores + ((size_t)s * n + i) * nb;
         const bool vec = (nb & 3) == 0;   // rows start on 16-byte boundaries
 #pragma unroll 1
-        for (int c0 = 0; c0 < BT; c0 += 32) {
+        for (int c0 = (BT / 2) * half; c0 < (BT / 2) * (half + 1); c0 += 32) {
             if (BT * bt + c0 >= (i_last + 1) / R) break;   // uniform: nothing valid past here
             float v[32];
             umma::tmem_ld32(trow + c0, v);
@@ -361,7 +364,7 @@ cudaError_t launch_qsa_indexer(const QsaArgs &a, void *ws) {
         if ((e = cudaFuncSetAttribute(qsa_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM)) != cudaSuccess)
             return e;
         const dim3 g((nb + BT - 1) / BT, (a.n + QT - 1) / QT, a.B);
-        qsa_score_kernel<<<g, 128, SMEM, a.stream>>>(m, a.n, scores);
+        qsa_score_kernel<<<g, 256, SMEM, a.stream>>>(m, a.n, scores);
         if ((e = launched()) != cudaSuccess) return e;
     }
     if (a.n > 0) {
