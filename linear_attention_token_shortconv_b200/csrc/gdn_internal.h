@@ -94,6 +94,7 @@ size_t qsa_workspace_bytes(int B, int n);
 size_t qsa_scores_bytes(int B, int n);
 cudaError_t launch_qsa_indexer(const QsaArgs &a, void *ws);
 cudaError_t qsa_error_word(unsigned *v, bool clear, cudaStream_t s);
+cudaError_t qsa_wait_selftest(uint32_t max_polls, cudaStream_t s);
 
 // K2f: token-by-token recurrence with the fused gates and output stage (SIMT fp32).
 cudaError_t launch_recurrent(const PrefillArgs &a, const float *qn, const float *kn,

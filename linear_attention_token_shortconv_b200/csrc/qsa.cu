@@ -111,6 +111,14 @@ qsa_prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const fl
 }
 
 // ------------------------------------------------------------------ K5b: scores
+// Bounded wait of the score kernel: false (and the device error word raised)
+// when the phase does not complete within max_polls polls.
+__device__ __forceinline__ bool qsa_wait(uint64_t *bar, uint32_t parity, uint32_t max_polls) {
+    const bool ok = umma::mbar_wait_bounded(bar, parity, max_polls);
+    if (!ok) atomicOr(&g_qsa_err, 1u);
+    return ok;
+}
+
 struct QsaMaps {
     CUtensorMap q, k;   // [rows][128] fp16, box {64, 128} and {64, 256}, 128-byte swizzle
 };
@@ -149,7 +157,7 @@ qsa_score_kernel(const __grid_constant__ QsaMaps maps, int n, float *__restrict_
             umma::tma_load_3d(sm + OFF_A + kb * 16384, &maps.q, 64 * kb, 0, qrow, bar_ld);
             umma::tma_load_3d(sm + OFF_B + kb * 32768, &maps.k, 64 * kb, 0, krow, bar_ld);
         }
-        ok = umma::mbar_wait_bounded(bar_ld, 0, 1u << 24);
+        ok = qsa_wait(bar_ld, 0, 1u << 24);
         if (ok) {
             umma::tc_fence_after();
             const uint32_t a = umma::smem_u32(sm + OFF_A), b = umma::smem_u32(sm + OFF_B);
@@ -161,12 +169,10 @@ qsa_score_kernel(const __grid_constant__ QsaMaps maps, int n, float *__restrict_
                 umma::mma_f16(tbase, ad, bd, idesc, st > 0);
             }
             umma::mma_commit(bar_mma);
-        } else {
-            atomicOr(&g_qsa_err, 1u);
         }
     }
     ok = __syncthreads_and(ok);   // the MMA was issued
-    if (ok) ok = __syncthreads_and(umma::mbar_wait_bounded(bar_mma, 0, 1u << 24));
+    if (ok) ok = __syncthreads_and(qsa_wait(bar_mma, 0, 1u << 24));
     if (ok) {
         umma::tc_fence_after();
         // warps w and w + 4: TMEM lanes 32 (w % 4) .. + 31 = rows (query 8 (w % 4) + l / 4,
@@ -211,8 +217,6 @@ qsa_score_kernel(const __grid_constant__ QsaMaps maps, int n, float *__restrict_
                 }
             }
         }
-    } else if (tid == 0) {
-        atomicOr(&g_qsa_err, 1u);
     }
     umma::tc_fence_before();
     __syncthreads();
@@ -377,6 +381,22 @@ cudaError_t launch_qsa_indexer(const QsaArgs &a, void *ws) {
         if ((e = launched()) != cudaSuccess) return e;
     }
     return cudaSuccess;
+}
+
+// One CTA waits, through qsa_wait, for a barrier phase that nothing completes.
+__global__ void qsa_wait_selftest_kernel(uint32_t max_polls) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        umma::mbar_init(&bar, 1);
+        umma::fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) qsa_wait(&bar, 0, max_polls);
+}
+
+cudaError_t qsa_wait_selftest(uint32_t max_polls, cudaStream_t s) {
+    qsa_wait_selftest_kernel<<<1, 32, 0, s>>>(max_polls);
+    return cudaGetLastError();
 }
 
 cudaError_t qsa_error_word(unsigned *v, bool clear, cudaStream_t s) {

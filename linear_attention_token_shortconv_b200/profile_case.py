@@ -8,6 +8,8 @@ larger than L2), run through the public binding:
         decode step for B sequences x 32 heads, d = 128: three steps
     python -m linear_attention_token_shortconv_b200.profile_case backward 1024
         prefill backward, 4 sequences x T tokens, H = 16, d = 128, fp32: three calls
+    python -m linear_attention_token_shortconv_b200.profile_case qsa 16384
+        QSA indexer on one sequence of n tokens, K = 2048: three calls
 """
 import sys
 from dataclasses import replace
@@ -15,8 +17,8 @@ from dataclasses import replace
 import torch
 
 from linear_attention_token_shortconv_b200 import gdn
-from linear_attention_token_shortconv_b200.workloads import (DECODE, LONG, PRETRAIN, make_decode_inputs,
-                                                             make_prefill_inputs, scaled)
+from linear_attention_token_shortconv_b200.workloads import (DECODE, LONG, PRETRAIN, QSA, make_decode_inputs,
+                                                             make_prefill_inputs, make_qsa_inputs, scaled)
 
 
 def prefill(T: int):
@@ -56,6 +58,15 @@ def backward(T: int):
     print("ok", float(grads["dq"].abs().mean()))
 
 
+def qsa(n: int):
+    cfg = replace(QSA, n=n)
+    inp = make_qsa_inputs(cfg, "cuda")
+    for _ in range(3):
+        sel, _ = gdn.qsa_indexer(inp["q"], inp["k"], inp["w_q"], inp["w_k"], budget=cfg.budget)
+    torch.cuda.synchronize()
+    print("ok", int(sel[-1, -1, 0]))
+
+
 if __name__ == "__main__":
     kind, size = sys.argv[1], int(sys.argv[2])
-    {"prefill": prefill, "decode": decode, "backward": backward}[kind](size)
+    {"prefill": prefill, "decode": decode, "backward": backward, "qsa": qsa}[kind](size)
