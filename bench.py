@@ -33,8 +33,8 @@ sys.path.insert(0, ROOT)
 from linear_attention_token_shortconv_b200 import dist as rankio  # noqa: E402
 from linear_attention_token_shortconv_b200 import gdn  # noqa: E402
 from linear_attention_token_shortconv_b200.workloads import (DECODE, LONG, PRETRAIN, QSA,  # noqa: E402
-                                                             make_decode_inputs, make_prefill_inputs,
-                                                             make_qsa_inputs, to_oracle_bits)
+                                                             make_decode_inputs, make_layer_inputs,
+                                                             make_prefill_inputs, make_qsa_inputs, to_oracle_bits)
 
 METRIC = "GDN prefill tokens/s at T=32K H=32 (% TC peak); decode state GB/s (% HBM)"
 # Algorithmic work per token-head of the fused chunked prefill (chunk C = 64, d = 128):
@@ -408,6 +408,37 @@ def bench_qsa(steps, dev):
     return cfg, ms, launches, flop, hbm
 
 
+def bench_layer(steps, dev, d_model=2048):
+    """gdn_layer_forward on the pretraining shape (4 x 4096 tokens, H = 16, d = 128)
+    with d_model = 2048: in-projection GEMMs, the mixer, W_o; bf16."""
+    cfg = PRETRAIN
+    inp = make_layer_inputs(cfg, d_model, dev)
+    y = torch.empty((cfg.total_tokens, d_model), dtype=torch.bfloat16, device=dev)
+
+    def call():
+        gdn.layer_forward(inp["x"], inp["w_in"], inp["conv_w"], inp["A"], inp["b_alpha"], inp["norm_w"],
+                          inp["w_o"], cfg.H, cfg.dk, cfg.dv, S0=inp["S0"], num_seqs=cfg.num_seqs, y=y)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches = 0
+    s.record()
+    for _ in range(steps):
+        call()
+        launches += gdn.last_call_launches()
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / steps
+    c_in = cfg.H * (2 * cfg.dk + 2 * cfg.dv) + 2 * cfg.H
+    gemm_flop = 2 * cfg.total_tokens * d_model * (c_in + cfg.H * cfg.dv)
+    mixer_flop = PREFILL_FLOP_PER_TOKEN_HEAD * cfg.total_tokens * cfg.H
+    del inp, y
+    torch.cuda.empty_cache()
+    return cfg, d_model, ms, launches, gemm_flop, mixer_flop
+
+
 def bench_decode_multi(cfg, T, steps, dev):
     """T consecutive tokens per sequence per step (gdn_decode_multi, all committed):
     the pool's entries [0, T) and [T, 2T) as two alternating multi-token inputs."""
@@ -578,6 +609,15 @@ def main():
             "tc": {"flop_per_call": q_flop, "achieved_tflops": q_flop / (q_ms * 1e-3) / 1e12,
                    "peak_tflops": pk["bf16_tflops"], "frac": q_flop / (q_ms * 1e-3) / 1e12 / pk["bf16_tflops"]},
             "kernels": "qsa_prep, qsa_score (tcgen05), qsa_topk", "gpu_launches": qlaunch}
+        lcfg, l_dm, l_ms, llaunch, l_gemm, l_mix = bench_layer(5, dev)
+        l_tf = (l_gemm + l_mix) / (l_ms * 1e-3) / 1e12
+        result["layer"] = {
+            "workload": f"layer forward, B=4 x T=4096, H=16, d=128, d_model={l_dm}, bf16 "
+                        "(in-projection GEMMs on cuBLAS, the mixer, W_o)",
+            "steps": 5, "ms_per_step": l_ms, "tokens_per_s": lcfg.total_tokens / (l_ms * 1e-3),
+            "bound": "tensor", "flop_per_call": l_gemm + l_mix, "achieved_tflops": l_tf,
+            "peak_tflops": pk["bf16_tflops"], "frac": l_tf / pk["bf16_tflops"],
+            "gemm_flop_share": l_gemm / (l_gemm + l_mix), "gpu_launches": llaunch}
         bcfg, b_ms, blaunch = bench_backward(5, dev)
         th = bcfg.total_tokens * bcfg.H
         b_tf = BACKWARD_FLOP_PER_TOKEN_HEAD * th / (b_ms * 1e-3) / 1e12

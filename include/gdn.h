@@ -197,6 +197,32 @@ GDN_API gdn_status_t gdn_qsa_indexer(int batch, int n, int heads, int d, int blo
 GDN_API gdn_status_t gdn_qsa_indexer_workspace_size(int batch, int n, size_t *bytes);
 
 /*
+ * gdn_layer_forward -- the GDN layer from the hidden states to the output
+ * projection (slinene.github.io write-up of "On the Design of Qwen3.8-Next
+ * Architecture", 模块 A, 参数化: q, k, v, z and the two gate logits are linear
+ * projections of x, and o = W_o[sigmoid(z) RMSNorm(y)]):
+ *   [q | k | v | z | a | b] = x W_in,  out = gdn_prefill(...),  y = out W_o.
+ *   x      [N_tok, d_model] bf16
+ *   w_in   [d_model, H(2dk + 2dv) + 2H] bf16, row-major; column blocks q [H dk],
+ *          k [H dk], v [H dv], z [H dv], a [H], b [H]
+ *   w_o    [H dv, d_model] bf16, row-major
+ *   y      [N_tok, d_model] bf16, written
+ * and the mixer's parameters as gdn_prefill (dims->in_dtype and out_dtype must be
+ * GDN_BF16; d_model a multiple of 8).  The projections are stored in bf16 between
+ * the steps.  The three GEMM steps are plain bf16 GEMMs with fp32 accumulation on
+ * cuBLAS, loaded at the first call (GDN_ERR_UNSUPPORTED when it cannot be
+ * loaded); they are not fused with the mixer's prelude.  Stream-ordered workspace
+ * from the library's pool: gdn_layer_workspace_size() bytes.
+ */
+GDN_API gdn_status_t gdn_layer_forward(const gdn_dims_t *dims, int d_model, const void *x, const void *w_in,
+                                       const float *conv_w, const float *A, const float *b_alpha,
+                                       const float *norm_w, const void *w_o, const float *S0,
+                                       const int32_t *cu_seqlens, void *y, float *S_final, gdn_stream_t stream);
+
+/* Bytes of device workspace one gdn_layer_forward call uses, the mixer's included (host call). */
+GDN_API gdn_status_t gdn_layer_workspace_size(const gdn_dims_t *dims, int d_model, size_t *bytes);
+
+/*
  * gdn_decode_step -- one token for each of B = dims->num_seqs sequences,
  * reading and updating the per-head state in place.
  *

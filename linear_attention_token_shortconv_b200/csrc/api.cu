@@ -172,6 +172,106 @@ cudaError_t slot_launch(int *slot, cudaStream_t s, F &&launch) {
     return e;
 }
 
+// The prefill after validation: workspace from the pool, then the kernels.
+cudaError_t prefill_dispatch(const gdn::PrefillArgs &a) {
+    gdn_dims_t dd;
+    dd.num_seqs = a.n_seq;
+    dd.total_tokens = a.n_tok;
+    dd.H = a.H;
+    dd.dk = a.dk;
+    dd.dv = a.dv;
+    dd.conv_k = 4;
+    dd.in_dtype = a.in_bf16 ? GDN_BF16 : GDN_F32;
+    dd.out_dtype = a.out_bf16 ? GDN_BF16 : GDN_F32;
+    const gdn_dims_t *dims = &dd;
+    const size_t nt = (size_t)a.n_tok * a.H;
+    const size_t ws_bytes = workspace_bytes(dims);
+    char *ws = nullptr;
+    if (ws_bytes) {
+        cudaMemPool_t pool;
+        cudaError_t ep = get_pool(&pool);
+        if (ep != cudaSuccess) return ep;
+        if (cudaMallocFromPoolAsync(reinterpret_cast<void **>(&ws), ws_bytes, pool, a.stream) !=
+            cudaSuccess)
+            return cudaErrorMemoryAllocation;
+    }
+    cudaError_t e;
+    if (use_tensor_cores(dims)) {
+        gdn::TcWorkspace w;
+        char *p = ws;
+        auto take = [&](size_t bytes) { char *r = p; p += round_up(bytes); return r; };
+        w.Qt = reinterpret_cast<__half *>(take(nt * a.dk * 2));
+        w.Kt = reinterpret_cast<__half *>(take(nt * a.dk * 2));
+        w.Wn = reinterpret_cast<__half *>(take(nt * a.dk * 2));
+        w.Up = reinterpret_cast<__half *>(take(nt * a.dv * 2));
+        w.Aqk = reinterpret_cast<__half *>(take(nt * 64 * 2));
+        w.decay = reinterpret_cast<float *>(take(nt * 4));
+        int *ready = reinterpret_cast<int *>(take(((size_t)a.n_seq * a.H * ((a.n_tok + 63) / 64) + 1) * 4));
+        const Segments g = segments(dims);
+        int slot = 0, sms = 0;
+        e = record(g_ev_begin, a.stream);
+        if (e == cudaSuccess) e = sm_count(&sms);
+        if (e == cudaSuccess && gdn::fused_chain_ctas(a, sms) > 0) {
+            // few (sequence, head) chains: one persistent launch, prep and chain
+            // ordered by per-chunk flags
+            e = slot_launch(&slot, a.stream, [&] { return gdn::launch_prefill_fused(a, w, ready, sms, a.stream); });
+        } else if (g.n == 1) {
+            if (e == cudaSuccess)
+                e = slot_launch(&slot, a.stream, [&] { return gdn::launch_chunk_prep(a, w); });
+            if (e == cudaSuccess)
+                e = slot_launch(&slot, a.stream, [&] { return gdn::launch_chunk_chain(a, w); });
+        } else {
+            float *state = reinterpret_cast<float *>(take((size_t)a.n_seq * a.H * a.dk * a.dv * 4));
+            int dev = 0;
+            if (e == cudaSuccess) e = cudaGetDevice(&dev);
+            if (e == cudaSuccess && (dev < 0 || dev >= 64)) e = cudaErrorInvalidDevice;
+            if (e == cudaSuccess) {
+                std::lock_guard<std::mutex> lock(g_side_mu[dev]);
+                SideStream *ss = nullptr;
+                e = side_stream(dev, g.n + 2, &ss);
+                // fork: the side streams start after the caller's prior work
+                if (e == cudaSuccess) e = cudaEventRecord(ss->events[g.n], a.stream);
+                if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->stream, ss->events[g.n], 0);
+                if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->prep2, ss->events[g.n], 0);
+                for (int sgi = 0; sgi < g.n && e == cudaSuccess; ++sgi) {
+                    const int c_lo = sgi * g.seg, c_hi = c_lo + g.seg;
+                    cudaStream_t ps = (sgi & 1) ? ss->prep2 : a.stream;
+                    e = slot_launch(&slot, ps, [&] { return gdn::launch_chunk_prep(a, w, c_lo, c_hi, ps); });
+                    if (e == cudaSuccess) e = cudaEventRecord(ss->events[sgi], ps);
+                    if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->stream, ss->events[sgi], 0);
+                    const float *sin = sgi == 0 ? a.S0 : state;
+                    float *sout = sgi == g.n - 1 ? a.S_final : state;
+                    if (e == cudaSuccess)
+                        e = slot_launch(&slot, ss->stream, [&] {
+                            return gdn::launch_chunk_chain(a, w, c_lo, c_hi, sin, sout, ss->stream);
+                        });
+                }
+                // every prep launch precedes a chain launch on the chain stream, so
+                // joining the chain stream joins all of the call's work
+                // join: the caller's stream continues after the last chain launch
+                if (e == cudaSuccess) e = cudaEventRecord(ss->events[g.n + 1], ss->stream);
+                if (e == cudaSuccess) e = cudaStreamWaitEvent(a.stream, ss->events[g.n + 1], 0);
+            }
+        }
+        if (e == cudaSuccess) e = record(g_ev_end, a.stream);
+    } else {
+        float *qn = reinterpret_cast<float *>(ws);
+        float *kn = reinterpret_cast<float *>(ws + round_up(nt * a.dk * sizeof(float)));
+        float *vn = reinterpret_cast<float *>(ws + 2 * round_up(nt * a.dk * sizeof(float)));
+        int slot = 0;
+        e = slot_launch(&slot, a.stream, [&] { return gdn::launch_prelude_f32(a, qn, kn, vn); });
+        if (e == cudaSuccess) e = record(g_ev_begin, a.stream);
+        if (e == cudaSuccess)
+            e = slot_launch(&slot, a.stream, [&] { return gdn::launch_recurrent(a, qn, kn, vn); });
+        if (e == cudaSuccess) e = record(g_ev_end, a.stream);
+    }
+    if (ws) {
+        cudaError_t ef = cudaFreeAsync(ws, a.stream);
+        if (e == cudaSuccess) e = ef;
+    }
+    return e;
+}
+
 }  // namespace
 
 namespace gdn {
@@ -284,91 +384,7 @@ gdn_status_t gdn_prefill(const gdn_dims_t *dims, const void *q, const void *k, c
     a.S_final = S_final;
     a.stream = reinterpret_cast<cudaStream_t>(stream);
 
-    const size_t nt = (size_t)a.n_tok * a.H;
-    const size_t ws_bytes = workspace_bytes(dims);
-    char *ws = nullptr;
-    if (ws_bytes) {
-        cudaMemPool_t pool;
-        if (get_pool(&pool) != cudaSuccess) return GDN_ERR_CUDA;
-        if (cudaMallocFromPoolAsync(reinterpret_cast<void **>(&ws), ws_bytes, pool, a.stream) !=
-            cudaSuccess)
-            return GDN_ERR_CUDA;
-    }
-    cudaError_t e;
-    if (use_tensor_cores(dims)) {
-        gdn::TcWorkspace w;
-        char *p = ws;
-        auto take = [&](size_t bytes) { char *r = p; p += round_up(bytes); return r; };
-        w.Qt = reinterpret_cast<__half *>(take(nt * a.dk * 2));
-        w.Kt = reinterpret_cast<__half *>(take(nt * a.dk * 2));
-        w.Wn = reinterpret_cast<__half *>(take(nt * a.dk * 2));
-        w.Up = reinterpret_cast<__half *>(take(nt * a.dv * 2));
-        w.Aqk = reinterpret_cast<__half *>(take(nt * 64 * 2));
-        w.decay = reinterpret_cast<float *>(take(nt * 4));
-        int *ready = reinterpret_cast<int *>(take(((size_t)a.n_seq * a.H * ((a.n_tok + 63) / 64) + 1) * 4));
-        const Segments g = segments(dims);
-        int slot = 0, sms = 0;
-        e = record(g_ev_begin, a.stream);
-        if (e == cudaSuccess) e = sm_count(&sms);
-        if (e == cudaSuccess && gdn::fused_chain_ctas(a, sms) > 0) {
-            // few (sequence, head) chains: one persistent launch, prep and chain
-            // ordered by per-chunk flags
-            e = slot_launch(&slot, a.stream, [&] { return gdn::launch_prefill_fused(a, w, ready, sms, a.stream); });
-        } else if (g.n == 1) {
-            if (e == cudaSuccess)
-                e = slot_launch(&slot, a.stream, [&] { return gdn::launch_chunk_prep(a, w); });
-            if (e == cudaSuccess)
-                e = slot_launch(&slot, a.stream, [&] { return gdn::launch_chunk_chain(a, w); });
-        } else {
-            float *state = reinterpret_cast<float *>(take((size_t)a.n_seq * a.H * a.dk * a.dv * 4));
-            int dev = 0;
-            if (e == cudaSuccess) e = cudaGetDevice(&dev);
-            if (e == cudaSuccess && (dev < 0 || dev >= 64)) e = cudaErrorInvalidDevice;
-            if (e == cudaSuccess) {
-                std::lock_guard<std::mutex> lock(g_side_mu[dev]);
-                SideStream *ss = nullptr;
-                e = side_stream(dev, g.n + 2, &ss);
-                // fork: the side streams start after the caller's prior work
-                if (e == cudaSuccess) e = cudaEventRecord(ss->events[g.n], a.stream);
-                if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->stream, ss->events[g.n], 0);
-                if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->prep2, ss->events[g.n], 0);
-                for (int sgi = 0; sgi < g.n && e == cudaSuccess; ++sgi) {
-                    const int c_lo = sgi * g.seg, c_hi = c_lo + g.seg;
-                    cudaStream_t ps = (sgi & 1) ? ss->prep2 : a.stream;
-                    e = slot_launch(&slot, ps, [&] { return gdn::launch_chunk_prep(a, w, c_lo, c_hi, ps); });
-                    if (e == cudaSuccess) e = cudaEventRecord(ss->events[sgi], ps);
-                    if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->stream, ss->events[sgi], 0);
-                    const float *sin = sgi == 0 ? a.S0 : state;
-                    float *sout = sgi == g.n - 1 ? a.S_final : state;
-                    if (e == cudaSuccess)
-                        e = slot_launch(&slot, ss->stream, [&] {
-                            return gdn::launch_chunk_chain(a, w, c_lo, c_hi, sin, sout, ss->stream);
-                        });
-                }
-                // every prep launch precedes a chain launch on the chain stream, so
-                // joining the chain stream joins all of the call's work
-                // join: the caller's stream continues after the last chain launch
-                if (e == cudaSuccess) e = cudaEventRecord(ss->events[g.n + 1], ss->stream);
-                if (e == cudaSuccess) e = cudaStreamWaitEvent(a.stream, ss->events[g.n + 1], 0);
-            }
-        }
-        if (e == cudaSuccess) e = record(g_ev_end, a.stream);
-    } else {
-        float *qn = reinterpret_cast<float *>(ws);
-        float *kn = reinterpret_cast<float *>(ws + round_up(nt * a.dk * sizeof(float)));
-        float *vn = reinterpret_cast<float *>(ws + 2 * round_up(nt * a.dk * sizeof(float)));
-        int slot = 0;
-        e = slot_launch(&slot, a.stream, [&] { return gdn::launch_prelude_f32(a, qn, kn, vn); });
-        if (e == cudaSuccess) e = record(g_ev_begin, a.stream);
-        if (e == cudaSuccess)
-            e = slot_launch(&slot, a.stream, [&] { return gdn::launch_recurrent(a, qn, kn, vn); });
-        if (e == cudaSuccess) e = record(g_ev_end, a.stream);
-    }
-    if (ws) {
-        cudaError_t ef = cudaFreeAsync(ws, a.stream);
-        if (e == cudaSuccess) e = ef;
-    }
-    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+    return prefill_dispatch(a) == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
 gdn_status_t gdn_prefill_backward_workspace_size(const gdn_dims_t *dims, size_t *bytes) {
@@ -503,6 +519,80 @@ gdn_status_t gdn_qsa_indexer(int batch, int n, int heads, int d, int block, int 
     cudaError_t e = record(g_ev_begin, a.stream);
     if (e == cudaSuccess) e = gdn::launch_qsa_indexer(a, ws);
     if (e == cudaSuccess) e = record(g_ev_end, a.stream);
+    cudaError_t ef = cudaFreeAsync(ws, a.stream);
+    if (e == cudaSuccess) e = ef;
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status_t gdn_layer_workspace_size(const gdn_dims_t *dims, int d_model, size_t *bytes) {
+    gdn_status_t st = check_dims(dims, false);
+    if (st != GDN_OK) return st;
+    if (!bytes || d_model <= 0) return GDN_ERR_INVALID_ARG;
+    *bytes = gdn::layer_workspace_bytes(dims->total_tokens, dims->H, dims->dk, dims->dv) + workspace_bytes(dims);
+    return GDN_OK;
+}
+
+gdn_status_t gdn_layer_forward(const gdn_dims_t *dims, int d_model, const void *x, const void *w_in,
+                               const float *conv_w, const float *A, const float *b_alpha, const float *norm_w,
+                               const void *w_o, const float *S0, const int32_t *cu_seqlens, void *y, float *S_final,
+                               gdn_stream_t stream) {
+    tl_launches = 0;
+    gdn_status_t st = check_dims(dims, false);
+    if (st != GDN_OK) return st;
+    if (dims->in_dtype != GDN_BF16 || dims->out_dtype != GDN_BF16) return GDN_ERR_UNSUPPORTED;
+    if (d_model <= 0) return GDN_ERR_INVALID_ARG;
+    if (d_model % 8 != 0) return GDN_ERR_UNSUPPORTED;   // 16-byte rows for the GEMMs
+    if (!cu_seqlens && dims->total_tokens % dims->num_seqs != 0) return GDN_ERR_INVALID_ARG;
+    const bool no_tokens = dims->total_tokens == 0;
+    const void *tok[] = {x, y};
+    for (const void *p : tok) {
+        if (!p && !no_tokens) return GDN_ERR_INVALID_ARG;
+        if (p && !aligned16(p)) return GDN_ERR_ALIGNMENT;
+    }
+    const void *weights[] = {w_in, w_o, conv_w};
+    for (const void *p : weights) {
+        if (!p) return GDN_ERR_INVALID_ARG;
+        if (!aligned16(p)) return GDN_ERR_ALIGNMENT;
+    }
+    const void *params[] = {A, b_alpha, norm_w};
+    for (const void *p : params) {
+        if (!p) return GDN_ERR_INVALID_ARG;
+        if (!aligned_to(p, 4)) return GDN_ERR_ALIGNMENT;
+    }
+    const void *opt[] = {S0, S_final};
+    for (const void *p : opt)
+        if (p && !aligned16(p)) return GDN_ERR_ALIGNMENT;
+    if (cu_seqlens && !aligned_to(cu_seqlens, 4)) return GDN_ERR_ALIGNMENT;
+    if (!no_tokens && !gdn::layer_blas_available()) return GDN_ERR_UNSUPPORTED;
+
+    gdn::LayerArgs L;
+    gdn::PrefillArgs &a = L.f;
+    a.n_seq = dims->num_seqs;
+    a.n_tok = dims->total_tokens;
+    a.H = dims->H;
+    a.dk = dims->dk;
+    a.dv = dims->dv;
+    a.in_bf16 = true;
+    a.out_bf16 = true;
+    a.q = a.k = a.v = a.z = a.a_logit = a.b_logit = nullptr;
+    a.conv_w = conv_w; a.A = A; a.b_alpha = b_alpha; a.norm_w = norm_w; a.S0 = S0;
+    a.cu_seqlens = cu_seqlens;
+    a.out = nullptr;
+    a.S_final = S_final;
+    a.stream = reinterpret_cast<cudaStream_t>(stream);
+    L.d_model = d_model;
+    L.x = x;
+    L.w_in = w_in;
+    L.w_o = w_o;
+    L.y = y;
+    if (no_tokens) return prefill_dispatch(a) == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+    const size_t ws_bytes = gdn::layer_workspace_bytes(a.n_tok, a.H, a.dk, a.dv);
+    char *ws = nullptr;
+    cudaMemPool_t pool;
+    if (get_pool(&pool) != cudaSuccess) return GDN_ERR_CUDA;
+    if (cudaMallocFromPoolAsync(reinterpret_cast<void **>(&ws), ws_bytes, pool, a.stream) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    cudaError_t e = gdn::launch_layer(L, ws, &prefill_dispatch);
     cudaError_t ef = cudaFreeAsync(ws, a.stream);
     if (e == cudaSuccess) e = ef;
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;

@@ -96,6 +96,20 @@ cudaError_t launch_qsa_indexer(const QsaArgs &a, void *ws);
 cudaError_t qsa_error_word(unsigned *v, bool clear, cudaStream_t s);
 cudaError_t qsa_wait_selftest(uint32_t max_polls, cudaStream_t s);
 
+// K6: the layer from the hidden states (in-projection GEMMs, the mixer, W_o).
+// x [N, d_model], w_in [d_model, H(2dk + 2dv) + 2H], w_o [H dv, d_model], y
+// [N, d_model], all bf16; f carries the mixer's parameters (its token pointers
+// are set by launch_layer).
+struct LayerArgs {
+    PrefillArgs f;
+    int d_model;
+    const void *x, *w_in, *w_o;
+    void *y;
+};
+size_t layer_workspace_bytes(int n_tok, int H, int dk, int dv);
+bool layer_blas_available();
+cudaError_t launch_layer(const LayerArgs &L, void *ws, cudaError_t (*run_prefill)(const PrefillArgs &));
+
 // K2f: token-by-token recurrence with the fused gates and output stage (SIMT fp32).
 cudaError_t launch_recurrent(const PrefillArgs &a, const float *qn, const float *kn,
                              const float *vn);

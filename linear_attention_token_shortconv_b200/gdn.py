@@ -25,7 +25,8 @@ EXPORTS = ("gdn_prefill", "gdn_prefill_workspace_size", "gdn_decode_step", "gdn_
            "gdn_set_timing_events", "gdn_selftest_umma", "gdn_prefill_noalloc",
            "gdn_set_kernel_events", "gdn_last_call_launches", "gdn_device_error_status",
            "gdn_selftest_wait_timeout", "gdn_decode_multi", "gdn_prefill_backward",
-           "gdn_prefill_backward_workspace_size", "gdn_qsa_indexer", "gdn_qsa_indexer_workspace_size")
+           "gdn_prefill_backward_workspace_size", "gdn_qsa_indexer", "gdn_qsa_indexer_workspace_size",
+           "gdn_layer_forward", "gdn_layer_workspace_size")
 ERRF_PREP, ERRF_CHAIN, ERRF_DECODE, ERRF_QSA = 1, 2, 4, 8
 
 
@@ -70,6 +71,10 @@ def load() -> ctypes.CDLL:
         lib.gdn_qsa_indexer.restype = ctypes.c_int
         lib.gdn_qsa_indexer_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)]
         lib.gdn_qsa_indexer_workspace_size.restype = ctypes.c_int
+        lib.gdn_layer_forward.argtypes = [D, ctypes.c_int] + [P] * 12
+        lib.gdn_layer_forward.restype = ctypes.c_int
+        lib.gdn_layer_workspace_size.argtypes = [D, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)]
+        lib.gdn_layer_workspace_size.restype = ctypes.c_int
         lib.gdn_prefill_noalloc.argtypes = [D] + [P] * 15
         lib.gdn_prefill_noalloc.restype = ctypes.c_int
         lib.gdn_selftest_umma.argtypes = [ctypes.c_int] * 5 + [P] * 5
@@ -201,6 +206,29 @@ def qsa_indexer(q, k, w_q, w_k, budget=2048, *, sel=None, scores=None, want_scor
         sel = sel[0]
         scores = None if scores is None else scores[0]
     return sel, scores
+
+
+def layer_forward(x, w_in, conv_w, A, b_alpha, norm_w, w_o, H, dk, dv, S0=None, cu_seqlens=None, *,
+                  num_seqs=None, y=None, S_final=None, want_state=True, stream=None):
+    """gdn_layer_forward on torch tensors: x [N_tok, d_model], w_in [d_model,
+    H(2dk + 2dv) + 2H], w_o [H dv, d_model], all bf16.
+
+    Returns (y [N_tok, d_model] bf16, S_final [N_seq, H, dk, dv] fp32 or None)."""
+    n_tok, d_model = x.shape
+    if cu_seqlens is not None:
+        n_seq = cu_seqlens.shape[0] - 1
+    else:
+        n_seq = num_seqs if num_seqs is not None else (S0.shape[0] if S0 is not None else 1)
+    if y is None:
+        y = torch.empty((n_tok, d_model), dtype=torch.bfloat16, device=x.device)
+    if S_final is None and want_state:
+        S_final = torch.empty((n_seq, H, dk, dv), dtype=torch.float32, device=x.device)
+    dims = Dims(n_seq, n_tok, H, dk, dv, conv_w.shape[1], GDN_BF16, GDN_BF16)
+    rc = load().gdn_layer_forward(ctypes.byref(dims), d_model, _ptr(x), _ptr(w_in), _ptr(conv_w), _ptr(A),
+                                  _ptr(b_alpha), _ptr(norm_w), _ptr(w_o), _ptr(S0), _ptr(cu_seqlens), _ptr(y),
+                                  _ptr(S_final), _stream(stream))
+    _check(rc, "gdn_layer_forward")
+    return y, S_final
 
 
 def prefill_noalloc(q, k, v, conv_w, a_logit, b_logit, A, b_alpha, z, norm_w, S0=None,

@@ -225,3 +225,22 @@ def make_qsa_inputs(cfg: QsaConfig, device="cpu", seed=None) -> dict:
          "w_q": _normal((128,), gen, device, std=0.1, mean=1.0),
          "w_k": _normal((128,), gen, device, std=0.1, mean=1.0)}
     return d
+
+
+def make_layer_inputs(cfg: PrefillConfig, d_model: int, device="cpu", seed=None) -> dict:
+    """Inputs of the layer from the hidden states: x [N_tok, d_model] ~ N(0, 1),
+    W_in [d_model, H(2dk + 2dv) + 2H] ~ N(0, 1 / d_model) (so the projections are
+    about N(0, 1), like the mixer's inputs), W_o [H dv, d_model] ~ N(0, 1 / (H dv)),
+    all bf16; the mixer's parameters (conv_w, A, b_alpha, norm_w, S0, cu_seqlens)
+    drawn as for the prefill of `cfg`."""
+    device = torch.device(device)
+    base = make_prefill_inputs(cfg, device, seed)
+    gen = torch.Generator(device=device)
+    gen.manual_seed((cfg.seed if seed is None else seed) + 7919)
+    H, dk, dv, N = cfg.H, cfg.dk, cfg.dv, cfg.total_tokens
+    c_in = H * (2 * dk + 2 * dv) + 2 * H
+    d = {key: base[key] for key in ("conv_w", "A", "b_alpha", "norm_w", "S0", "cu_seqlens")}
+    d["x"] = _normal((N, d_model), gen, device).to(torch.bfloat16)
+    d["w_in"] = _normal((d_model, c_in), gen, device, std=d_model ** -0.5).to(torch.bfloat16)
+    d["w_o"] = _normal((H * dv, d_model), gen, device, std=(H * dv) ** -0.5).to(torch.bfloat16)
+    return d

@@ -174,3 +174,34 @@ def test_backward_workspace_size_query(lib):
     assert n >= 6 * 1000 * 4 * 128 * 4 + (1000 // 16) * 4 * 128 * 128 * 4
     with pytest.raises(gdn.GdnError):
         gdn.prefill_backward_workspace_size(1, 10, 1, 128, 64)
+
+
+def test_layer_argument_validation(lib):
+    P = ctypes.c_void_p
+    ptrs = [P(4096 * (i + 1)) for i in range(7)]                  # x, w_in, conv_w, A, b_alpha, norm_w, w_o
+    ok = _dims(num_seqs=1, total_tokens=64, in_dtype=1, out_dtype=1)
+    call = lambda dims, d_model, y=P(65536), x=ptrs[0]: lib.gdn_layer_forward(
+        ctypes.byref(dims) if dims is not None else None, d_model, x, *ptrs[1:], None, None, y, None, None)
+    assert call(None, 256) == 1
+    assert call(_dims(in_dtype=0, out_dtype=1), 256) == 2            # fp32 activations
+    assert call(_dims(in_dtype=1, out_dtype=0), 256) == 2            # fp32 output
+    assert call(ok, 0) == 1
+    assert call(ok, 260) == 2                                        # d_model not a multiple of 8
+    assert call(ok, 256, y=None) == 1
+    assert call(ok, 256, x=P(4100)) == 3
+    assert lib.gdn_last_call_launches() == 0
+    n = ctypes.c_size_t(0)
+    assert lib.gdn_layer_workspace_size(ctypes.byref(ok), 256, ctypes.byref(n)) == 0 and n.value > 0
+
+
+def test_qsa_argument_validation(lib):
+    P = ctypes.c_void_p
+    q, k, wq, wk, sel = (P(4096 * (i + 1)) for i in range(5))
+    call = lambda *dims, q=q, sel=sel: lib.gdn_qsa_indexer(*dims, q, k, wq, wk, sel, None, None)
+    assert call(0, 64, 4, 128, 4, 2048) == 1
+    assert call(1, 64, 8, 128, 4, 2048) == 2                         # heads
+    assert call(1, 64, 4, 64, 4, 2048) == 2                          # d
+    assert call(1, 64, 4, 128, 4, 2046) == 2                         # budget not a multiple of the block
+    assert call(1, 64, 4, 128, 4, 2048, q=P(4100)) == 3
+    assert call(1, 64, 4, 128, 4, 2048, sel=None) == 1
+    assert call(1, 0, 4, 128, 4, 2048, q=None, sel=None) == 0        # nothing to do
