@@ -68,24 +68,59 @@ __device__ __forceinline__ void bwd_gates(float a_l, float b_l, float A, float b
     be = sigmoid_acc(b_l);
 }
 
-// Reduce-scatter of N values across the 32 lanes of a warp (N a multiple of 32):
-// afterwards v[i], i < N / 32, of lane l holds the warp-wide sum of entry
-// (N / 32) l + i.  Each round halves the array: a lane keeps the half selected by
-// its lane bit and adds the partner lane's copy of that half.
+// Reduce-scatter of N values across the 32 lanes of a warp, in five rounds with
+// lane offsets 16, 8, .., 1.  A round halves the array while its length is even
+// (a lane keeps the half its lane bit selects and adds the partner lane's copy of
+// it); once the length is odd a round adds the partner's whole array.  Afterwards
+// a lane with no bit of rs_plain<N>() set holds in v[0 .. rs_len<N>(5)) the warp
+// sums of entries rs_offset<N>(lane) + i (the other lanes hold copies).
+__host__ __device__ constexpr int rs_len(int N, int rounds) {
+    int L = N;
+    for (int r = 0; r < rounds; ++r)
+        if (L % 2 == 0) L /= 2;
+    return L;
+}
+__host__ __device__ constexpr int rs_plain(int N) {
+    int L = N, m = 0;
+    for (int r = 0; r < 5; ++r) {
+        if (L % 2 == 0) L /= 2;
+        else m |= 16 >> r;
+    }
+    return m;
+}
+__device__ __forceinline__ int rs_offset(int N, int lane) {
+    int L = N, off = 0;
+#pragma unroll
+    for (int r = 0; r < 5; ++r) {
+        if (L % 2 == 0) {
+            L /= 2;
+            if (lane & (16 >> r)) off += L;
+        }
+    }
+    return off;
+}
+
 template <int N>
 __device__ __forceinline__ void warp_reduce_scatter(float (&v)[N], int lane) {
 #pragma unroll
     for (int rd = 0; rd < 5; ++rd) {
         const int o = 16 >> rd;
-        const bool up = (lane & o) != 0;
-        const int half = N >> (rd + 1);
+        const int len = rs_len(N, rd);
+        if (len % 2 == 0) {
+            const bool up = (lane & o) != 0;
+            const int half = len / 2;
 #pragma unroll
-        for (int i = 0; i < (N >> 1); ++i) {
-            if (i < half) {
-                const float send = up ? v[i] : v[i + half];
-                const float keep = up ? v[i + half] : v[i];
-                v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+            for (int i = 0; i < N / 2; ++i) {
+                if (i < half) {
+                    const float send = up ? v[i] : v[i + half];
+                    const float keep = up ? v[i + half] : v[i];
+                    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+                }
             }
+        } else {
+#pragma unroll
+            for (int i = 0; i < N; ++i)
+                if (i < len) v[i] += __shfl_xor_sync(0xffffffffu, v[i], o);
         }
     }
 }
@@ -307,7 +342,7 @@ bwd_rec_kernel(const float *__restrict__ qn, const float *__restrict__ kn, const
                float *__restrict__ scratch, float *__restrict__ dvn, float *__restrict__ part,
                float *__restrict__ d_S0) {
     constexpr int RPT = D / 8, CPT = DC / 32, IV = bwd::IV, NS = D / DC;
-    constexpr int NV = (3 * RPT + 31) / 32 * 32;
+    constexpr int NV = 3 * RPT;   // row sums per thread: P dy, P de, D e
     constexpr int PW = 3 * D + 8;   // partial row: P dy, P de, D e [D] each, <D, P> per warp [8]
     static_assert(CPT == 1, "one column per lane");
     __shared__ __align__(16) float qq[IV][D];
@@ -443,14 +478,15 @@ bwd_rec_kernel(const float *__restrict__ qn, const float *__restrict__ kn, const
                 v[RPT + r] = b_;
                 v[2 * RPT + r] = c_;
             }
-#pragma unroll
-            for (int x = 3 * RPT; x < NV; ++x) v[x] = 0.f;
             warp_reduce_scatter<NV>(v, lane);
             float *pr = part + ((size_t)zc * n_th + th) * PW;
+            if ((lane & rs_plain(NV)) == 0) {
+                const int off = rs_offset(NV, lane);
 #pragma unroll
-            for (int i = 0; i < NV / 32; ++i) {
-                const int idx = (NV / 32) * lane + i;
-                if (idx < 3 * RPT) pr[(idx / RPT) * D + warp * RPT + idx % RPT] = v[i];
+                for (int i = 0; i < rs_len(NV, 5); ++i) {
+                    const int idx = off + i;
+                    pr[(idx / RPT) * D + warp * RPT + idx % RPT] = v[i];
+                }
             }
             dDP = group_sum<32>(dDP);
             if (lane == 0) pr[3 * D + warp] = dDP;
