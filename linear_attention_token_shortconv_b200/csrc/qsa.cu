@@ -22,8 +22,10 @@
 //      sums the 4 heads (lanes 4q .. 4q + 3) with two shuffles and stores the
 //      scores of complete blocks.  Tiles entirely past the causal limit do nothing.
 //  K5c qsa_topk_kernel: one CTA per query row: a radix select on the score bits
-//      (scores are >= 0, so their bit patterns order like the values) finds the
-//      threshold, then a block scan writes the selected blocks in ascending
+//      (scores are >= 0, so their bit patterns order like the values; digits of
+//      11, 11 and 9 bits, the first counted while the row is read into shared
+//      memory, stopping at the first digit whose bucket is taken whole) finds the
+//      threshold, then warp segments write the selected blocks in ascending
 //      order, equal scores at the threshold taken from the smallest index.
 #include <cuda.h>
 #include <cuda_fp16.h>
@@ -226,15 +228,63 @@ qsa_score_kernel(const __grid_constant__ QsaMaps maps, int n, float *__restrict_
 // ------------------------------------------------------------------ K5c: top-k
 namespace qsa {
 constexpr int TOPK_CAP = 12288;   // row keys kept in shared memory up to this many blocks (48 KB)
+constexpr int HB = 2048;          // histogram buckets of the 11-bit digits
 }  // namespace qsa
+
+// One digit of the radix select: among the keys matching `prefix`, the bucket of
+// the digit at `shift` (NB buckets) that holds the remaining-th largest key.
+// Thread t sums buckets NB-1-PER*t down to NB-PER*(t+1); a block scan of those
+// sums crosses `remaining` at exactly one thread, which walks its buckets and
+// publishes the extended prefix, the rank left inside the bucket and the
+// bucket's count.  Ends with a block barrier.
+template <int NB>
+__device__ __forceinline__ void topk_pick(const int *hist, int *wsum, int remaining, unsigned prefix, int shift,
+                                          int tid, unsigned *sh_prefix, int *sh_rem, int *sh_cnt) {
+    constexpr int PER = NB / 256;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int top = NB - 1 - PER * tid;
+    int c = 0;
+#pragma unroll
+    for (int j = 0; j < PER; ++j) c += hist[top - j];
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    for (int w = 0; w < warp; ++w) incl += wsum[w];
+    int run = incl - c;
+    if (incl >= remaining && run < remaining) {
+#pragma unroll
+        for (int j = 0; j < PER; ++j) {
+            const int h = hist[top - j];
+            if (run + h >= remaining) {
+                *sh_prefix = prefix | ((unsigned)(top - j) << shift);
+                *sh_rem = remaining - run;
+                *sh_cnt = h;
+                break;
+            }
+            run += h;
+        }
+    }
+    __syncthreads();
+}
+
+__device__ __forceinline__ unsigned topk_key(float v) {
+    return v > 0.f ? __float_as_uint(v) : 0u;   // scores >= 0: bits order like values (-0 -> 0)
+}
 
 __global__ void __launch_bounds__(256)
 qsa_topk_kernel(const float *__restrict__ scores, int n, int KB, int32_t *__restrict__ sel) {
-    extern __shared__ unsigned keys_s[];   // [min(n_valid, TOPK_CAP)]
-    __shared__ int hist[256];
+    extern __shared__ uint4 keys4[];   // the row's keys when n_valid <= TOPK_CAP
+    unsigned *keys_s = reinterpret_cast<unsigned *>(keys4);
+    __shared__ int hist[qsa::HB];
+    __shared__ int wsum[8];
     __shared__ int wcnt[8][2];
     __shared__ unsigned sh_prefix;
-    __shared__ int sh_remaining;
+    __shared__ int sh_rem, sh_cnt;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const long long row = blockIdx.x;   // s * n + i
     const int i = (int)(row % n);
@@ -246,68 +296,83 @@ qsa_topk_kernel(const float *__restrict__ scores, int n, int KB, int32_t *__rest
         for (int j = tid; j < KB; j += 256) out[j] = j < n_valid ? j : -1;
         return;
     }
-    auto key_of = [&](int b) -> unsigned {
-        const float v = sc[b];
-        return v > 0.f ? __float_as_uint(v) : 0u;   // scores >= 0: bits order like values (-0 -> 0)
-    };
+    for (int j = tid; j < qsa::HB; j += 256) hist[j] = 0;
+    __syncthreads();
+    // The keys (into shared memory when they fit) and the histogram of their first
+    // digit, bits 30..20 (bit 31 of a key is 0).  Rows start on 16-byte boundaries
+    // when nb % 4 == 0; the last quad may reach past n_valid, never past the row.
     const bool in_smem = n_valid <= qsa::TOPK_CAP;   // uniform
-    if (in_smem) {
-        for (int b = tid; b < n_valid; b += 256) keys_s[b] = key_of(b);
-        __syncthreads();
+    if (in_smem && (nb & 3) == 0) {
+        const float4 *sc4 = reinterpret_cast<const float4 *>(sc);
+        const int n4 = (n_valid + 3) >> 2;
+        for (int b4 = tid; b4 < n4; b4 += 256) {
+            const float4 v = sc4[b4];
+            const uint4 kk = make_uint4(topk_key(v.x), topk_key(v.y), topk_key(v.z), topk_key(v.w));
+            keys4[b4] = kk;
+            const int b = 4 * b4;
+            atomicAdd(&hist[kk.x >> 20], 1);
+            if (b + 1 < n_valid) atomicAdd(&hist[kk.y >> 20], 1);
+            if (b + 2 < n_valid) atomicAdd(&hist[kk.z >> 20], 1);
+            if (b + 3 < n_valid) atomicAdd(&hist[kk.w >> 20], 1);
+        }
+    } else {
+        for (int b = tid; b < n_valid; b += 256) {
+            const unsigned key = topk_key(sc[b]);
+            if (in_smem) keys_s[b] = key;
+            atomicAdd(&hist[key >> 20], 1);
+        }
     }
-    auto key_at = [&](int b) -> unsigned { return in_smem ? keys_s[b] : key_of(b); };
-    // radix select of the KB-th largest key, 8 bits per pass from the top
-    unsigned prefix = 0, mask = 0;
-    int remaining = KB;
-#pragma unroll 1
-    for (int pass = 0; pass < 4; ++pass) {
-        const int shift = 24 - 8 * pass;
-        hist[tid] = 0;
+    __syncthreads();
+    auto key_at = [&](int b) -> unsigned { return in_smem ? keys_s[b] : topk_key(sc[b]); };
+    // Radix select of the KB-th largest key with digits of 11, 11 and 9 bits.  A
+    // digit whose bucket holds exactly the keys still wanted ends it early: every
+    // key of that bucket is taken, so the lower bits need not be resolved.
+    topk_pick<qsa::HB>(hist, wsum, KB, 0u, 20, tid, &sh_prefix, &sh_rem, &sh_cnt);
+    unsigned prefix = sh_prefix, mask = 0xFFF00000u;
+    int remaining = sh_rem;
+    if (sh_cnt != remaining) {   // uniform
+        for (int j = tid; j < qsa::HB; j += 256) hist[j] = 0;
         __syncthreads();
         for (int b = tid; b < n_valid; b += 256) {
             const unsigned key = key_at(b);
-            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+            if ((key & mask) == prefix) atomicAdd(&hist[(key >> 9) & 2047u], 1);
         }
         __syncthreads();
-        // the digit holding the remaining-th largest key: thread t takes digit
-        // 255 - t; a block scan of the counts in that order crosses `remaining`
-        // at exactly one thread
-        {
-            const int c = hist[255 - tid];
-            int incl = c;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += y;
-            }
-            if (lane == 31) wcnt[warp][0] = incl;
-            __syncthreads();
-            for (int w = 0; w < warp; ++w) incl += wcnt[w][0];
-            if (incl >= remaining && incl - c < remaining) {
-                sh_remaining = remaining - (incl - c);
-                sh_prefix = prefix | ((unsigned)(255 - tid) << shift);
-            }
-        }
-        __syncthreads();
-        remaining = sh_remaining;
+        topk_pick<qsa::HB>(hist, wsum, remaining, prefix, 9, tid, &sh_prefix, &sh_rem, &sh_cnt);
         prefix = sh_prefix;
-        mask |= 255u << shift;
-        __syncthreads();   // hist is cleared by the next pass
+        remaining = sh_rem;
+        mask = 0xFFFFFE00u;
+        if (sh_cnt != remaining) {
+            for (int j = tid; j < 512; j += 256) hist[j] = 0;
+            __syncthreads();
+            for (int b = tid; b < n_valid; b += 256) {
+                const unsigned key = key_at(b);
+                if ((key & mask) == prefix) atomicAdd(&hist[key & 511u], 1);
+            }
+            __syncthreads();
+            topk_pick<512>(hist, wsum, remaining, prefix, 0, tid, &sh_prefix, &sh_rem, &sh_cnt);
+            prefix = sh_prefix;
+            remaining = sh_rem;
+            mask = 0xFFFFFFFFu;
+        }
     }
-    // Selection: the keys above the threshold T and the first `remaining` equal to
-    // it in index order.  Warp w owns a contiguous segment of the row; it counts
-    // its keys above and equal to T, the warps exchange counts once, and each
-    // warp then writes its selected blocks at their ascending positions.
-    const unsigned T = prefix;
+    // Selection: the keys whose masked bits are above the prefix, and the first
+    // `remaining` equal to it in index order.  Warp w owns a contiguous segment of
+    // the row; it counts its keys above and equal, the warps exchange counts
+    // once, and each warp then writes its selected blocks at their ascending
+    // positions.
     const int seg = (((n_valid + 7) / 8) + 31) / 32 * 32;
     const int b_lo = min(warp * seg, n_valid), b_hi = min(b_lo + seg, n_valid);
-    const unsigned lt = (1u << lane) - 1u;
     int n_gt = 0, n_eq = 0;
-    for (int b0 = b_lo; b0 < b_hi; b0 += 32) {
-        const int b = b0 + lane;
-        const unsigned key = b < b_hi ? key_at(b) : 0u;
-        n_gt += __popc(__ballot_sync(0xffffffffu, b < b_hi && key > T));
-        n_eq += __popc(__ballot_sync(0xffffffffu, b < b_hi && key == T));
+    for (int b = b_lo + lane; b < b_hi; b += 32) {
+        const unsigned km = key_at(b) & mask;
+        n_gt += km > prefix;
+        n_eq += km == prefix;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        n_gt += __shfl_xor_sync(0xffffffffu, n_gt, o);
+        n_eq += __shfl_xor_sync(0xffffffffu, n_eq, o);
     }
     if (lane == 0) {
         wcnt[warp][0] = n_gt;
@@ -319,16 +384,21 @@ qsa_topk_kernel(const float *__restrict__ scores, int n, int KB, int32_t *__rest
         gt_before += wcnt[w][0];
         eq_before += wcnt[w][1];
     }
+    const unsigned lt = (1u << lane) - 1u;
     int eq_run = eq_before, out_run = gt_before + min(eq_before, remaining);
     for (int b0 = b_lo; b0 < b_hi; b0 += 32) {
         const int b = b0 + lane;
-        const unsigned key = b < b_hi ? key_at(b) : 0u;
-        const bool gt = b < b_hi && key > T, eq = b < b_hi && key == T;
+        const bool in = b < b_hi;
+        const unsigned km = in ? (key_at(b) & mask) : 0u;
+        const bool eq = in && km == prefix;
+        bool take = in && km > prefix;
         const unsigned eq_mask = __ballot_sync(0xffffffffu, eq);
-        const bool take = gt || (eq && eq_run + __popc(eq_mask & lt) < remaining);
+        if (eq_mask) {   // uniform
+            take = take || (eq && eq_run + __popc(eq_mask & lt) < remaining);
+            eq_run += __popc(eq_mask);
+        }
         const unsigned take_mask = __ballot_sync(0xffffffffu, take);
         if (take) out[out_run + __popc(take_mask & lt)] = b;
-        eq_run += __popc(eq_mask);
         out_run += __popc(take_mask);
     }
 }
