@@ -227,25 +227,30 @@ qsa_score_kernel(const __grid_constant__ QsaMaps maps, int n, float *__restrict_
 
 // ------------------------------------------------------------------ K5c: top-k
 namespace qsa {
-constexpr int TOPK_CAP = 12288;   // row keys kept in shared memory up to this many blocks (48 KB)
-constexpr int HB = 2048;          // histogram buckets of the 11-bit digits
+constexpr int TOPK_CAP = 12288;      // row keys kept in shared memory up to this many blocks (48 KB)
+constexpr int HB = 2048;             // buckets of the 11-bit digits
+constexpr int HB_SLOTS = HB + HB / 32;   // with one pad counter per 32
 }  // namespace qsa
+
+// Counter of the bucket at descending rank u (u = NB - 1 - digit): one pad word
+// per 32 counters, so the PER consecutive ranks that each thread of a warp scans
+// fall in distinct banks (thread t reads ranks PER t .. PER t + PER - 1).
+__device__ __forceinline__ int topk_slot(int u) { return u + (u >> 5); }
 
 // One digit of the radix select: among the keys matching `prefix`, the bucket of
 // the digit at `shift` (NB buckets) that holds the remaining-th largest key.
-// Thread t sums buckets NB-1-PER*t down to NB-PER*(t+1); a block scan of those
-// sums crosses `remaining` at exactly one thread, which walks its buckets and
-// publishes the extended prefix, the rank left inside the bucket and the
-// bucket's count.  Ends with a block barrier.
+// Thread t sums the buckets of ranks PER t .. PER t + PER - 1 (descending
+// digits); a block scan of those sums crosses `remaining` at exactly one thread,
+// which walks its buckets and publishes the extended prefix, the rank left
+// inside the bucket and the bucket's count.  Ends with a block barrier.
 template <int NB>
 __device__ __forceinline__ void topk_pick(const int *hist, int *wsum, int remaining, unsigned prefix, int shift,
                                           int tid, unsigned *sh_prefix, int *sh_rem, int *sh_cnt) {
     constexpr int PER = NB / 256;
     const int warp = tid >> 5, lane = tid & 31;
-    const int top = NB - 1 - PER * tid;
     int c = 0;
 #pragma unroll
-    for (int j = 0; j < PER; ++j) c += hist[top - j];
+    for (int j = 0; j < PER; ++j) c += hist[topk_slot(PER * tid + j)];
     int incl = c;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -259,9 +264,9 @@ __device__ __forceinline__ void topk_pick(const int *hist, int *wsum, int remain
     if (incl >= remaining && run < remaining) {
 #pragma unroll
         for (int j = 0; j < PER; ++j) {
-            const int h = hist[top - j];
+            const int h = hist[topk_slot(PER * tid + j)];
             if (run + h >= remaining) {
-                *sh_prefix = prefix | ((unsigned)(top - j) << shift);
+                *sh_prefix = prefix | ((unsigned)(NB - 1 - (PER * tid + j)) << shift);
                 *sh_rem = remaining - run;
                 *sh_cnt = h;
                 break;
@@ -276,98 +281,121 @@ __device__ __forceinline__ unsigned topk_key(float v) {
     return v > 0.f ? __float_as_uint(v) : 0u;   // scores >= 0: bits order like values (-0 -> 0)
 }
 
-__global__ void __launch_bounds__(256)
-qsa_topk_kernel(const float *__restrict__ scores, int n, int KB, int32_t *__restrict__ sel) {
-    extern __shared__ uint4 keys4[];   // the row's keys when n_valid <= TOPK_CAP
-    unsigned *keys_s = reinterpret_cast<unsigned *>(keys4);
-    __shared__ int hist[qsa::HB];
-    __shared__ int wsum[8];
-    __shared__ int wcnt[8][2];
-    __shared__ unsigned sh_prefix;
-    __shared__ int sh_rem, sh_cnt;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const long long row = blockIdx.x;   // s * n + i
-    const int i = (int)(row % n);
-    const int nb = n / qsa::R;
-    const int n_valid = (i + 1) / qsa::R;
-    const float *sc = scores + row * nb;
-    int32_t *out = sel + row * KB;
-    if (n_valid <= KB) {   // every complete block
-        for (int j = tid; j < KB; j += 256) out[j] = j < n_valid ? j : -1;
-        return;
-    }
-    for (int j = tid; j < qsa::HB; j += 256) hist[j] = 0;
-    __syncthreads();
-    // The keys (into shared memory when they fit) and the histogram of their first
-    // digit, bits 30..20 (bit 31 of a key is 0).  Rows start on 16-byte boundaries
-    // when nb % 4 == 0; the last quad may reach past n_valid, never past the row.
-    const bool in_smem = n_valid <= qsa::TOPK_CAP;   // uniform
-    if (in_smem && (nb & 3) == 0) {
-        const float4 *sc4 = reinterpret_cast<const float4 *>(sc);
+// Shared state of one row's select.
+struct TopkSmem {
+    int hist[qsa::HB_SLOTS];
+    int wsum[8];
+    int wcnt[8][2];
+    unsigned prefix;
+    int rem, cnt;
+};
+
+// Histogram of the digit (key >> shift) & (NB - 1) over the keys with
+// (key & mask) == prefix; SMEM: the keys are in shared memory (read 16 bytes at
+// a time), else they are read from the score row.
+template <bool SMEM, int NB>
+__device__ __forceinline__ void topk_count(TopkSmem &S, const uint4 *keys4, const float *sc, int n_valid,
+                                           unsigned mask, unsigned prefix, int shift, int tid) {
+    if (SMEM) {
         const int n4 = (n_valid + 3) >> 2;
-        for (int b4 = tid; b4 < n4; b4 += 256) {
-            const float4 v = sc4[b4];
-            const uint4 kk = make_uint4(topk_key(v.x), topk_key(v.y), topk_key(v.z), topk_key(v.w));
-            keys4[b4] = kk;
-            const int b = 4 * b4;
-            atomicAdd(&hist[kk.x >> 20], 1);
-            if (b + 1 < n_valid) atomicAdd(&hist[kk.y >> 20], 1);
-            if (b + 2 < n_valid) atomicAdd(&hist[kk.z >> 20], 1);
-            if (b + 3 < n_valid) atomicAdd(&hist[kk.w >> 20], 1);
+        for (int q = tid; q < n4; q += 256) {
+            const uint4 kk = keys4[q];
+            const unsigned k[4] = {kk.x, kk.y, kk.z, kk.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (4 * q + j < n_valid && (k[j] & mask) == prefix)
+                    atomicAdd(&S.hist[topk_slot(NB - 1 - (int)((k[j] >> shift) & (NB - 1)))], 1);
         }
     } else {
         for (int b = tid; b < n_valid; b += 256) {
             const unsigned key = topk_key(sc[b]);
-            if (in_smem) keys_s[b] = key;
-            atomicAdd(&hist[key >> 20], 1);
+            if ((key & mask) == prefix) atomicAdd(&S.hist[topk_slot(NB - 1 - (int)((key >> shift) & (NB - 1)))], 1);
+        }
+    }
+}
+
+template <bool SMEM>
+__device__ __forceinline__ void topk_row(TopkSmem &S, uint4 *keys4, const float *__restrict__ sc, int nb,
+                                         int n_valid, int KB, int32_t *__restrict__ out, int tid) {
+    unsigned *keys_s = reinterpret_cast<unsigned *>(keys4);
+    const int warp = tid >> 5, lane = tid & 31;
+    for (int j = tid; j < qsa::HB_SLOTS; j += 256) S.hist[j] = 0;
+    __syncthreads();
+    // The keys (into shared memory when they fit) and the histogram of their first
+    // digit, bits 30..20 (bit 31 of a key is 0).  Rows start on 16-byte boundaries
+    // when nb % 4 == 0; the last quad may reach past n_valid, never past the row.
+    if (SMEM && (nb & 3) == 0) {
+        const float4 *sc4 = reinterpret_cast<const float4 *>(sc);
+        const int n4 = (n_valid + 3) >> 2;
+        for (int q = tid; q < n4; q += 256) {
+            const float4 v = sc4[q];
+            const unsigned k[4] = {topk_key(v.x), topk_key(v.y), topk_key(v.z), topk_key(v.w)};
+            keys4[q] = make_uint4(k[0], k[1], k[2], k[3]);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (4 * q + j < n_valid) atomicAdd(&S.hist[topk_slot(qsa::HB - 1 - (int)(k[j] >> 20))], 1);
+        }
+    } else {
+        for (int b = tid; b < n_valid; b += 256) {
+            const unsigned key = topk_key(sc[b]);
+            if (SMEM) keys_s[b] = key;
+            atomicAdd(&S.hist[topk_slot(qsa::HB - 1 - (int)(key >> 20))], 1);
         }
     }
     __syncthreads();
-    auto key_at = [&](int b) -> unsigned { return in_smem ? keys_s[b] : topk_key(sc[b]); };
     // Radix select of the KB-th largest key with digits of 11, 11 and 9 bits.  A
     // digit whose bucket holds exactly the keys still wanted ends it early: every
     // key of that bucket is taken, so the lower bits need not be resolved.
-    topk_pick<qsa::HB>(hist, wsum, KB, 0u, 20, tid, &sh_prefix, &sh_rem, &sh_cnt);
-    unsigned prefix = sh_prefix, mask = 0xFFF00000u;
-    int remaining = sh_rem;
-    if (sh_cnt != remaining) {   // uniform
-        for (int j = tid; j < qsa::HB; j += 256) hist[j] = 0;
+    topk_pick<qsa::HB>(S.hist, S.wsum, KB, 0u, 20, tid, &S.prefix, &S.rem, &S.cnt);
+    unsigned prefix = S.prefix, mask = 0xFFF00000u;
+    int remaining = S.rem;
+    if (S.cnt != remaining) {   // uniform
+        for (int j = tid; j < qsa::HB_SLOTS; j += 256) S.hist[j] = 0;
         __syncthreads();
-        for (int b = tid; b < n_valid; b += 256) {
-            const unsigned key = key_at(b);
-            if ((key & mask) == prefix) atomicAdd(&hist[(key >> 9) & 2047u], 1);
-        }
+        topk_count<SMEM, qsa::HB>(S, keys4, sc, n_valid, mask, prefix, 9, tid);
         __syncthreads();
-        topk_pick<qsa::HB>(hist, wsum, remaining, prefix, 9, tid, &sh_prefix, &sh_rem, &sh_cnt);
-        prefix = sh_prefix;
-        remaining = sh_rem;
+        topk_pick<qsa::HB>(S.hist, S.wsum, remaining, prefix, 9, tid, &S.prefix, &S.rem, &S.cnt);
+        prefix = S.prefix;
+        remaining = S.rem;
         mask = 0xFFFFFE00u;
-        if (sh_cnt != remaining) {
-            for (int j = tid; j < 512; j += 256) hist[j] = 0;
+        if (S.cnt != remaining) {
+            for (int j = tid; j < topk_slot(512); j += 256) S.hist[j] = 0;
             __syncthreads();
-            for (int b = tid; b < n_valid; b += 256) {
-                const unsigned key = key_at(b);
-                if ((key & mask) == prefix) atomicAdd(&hist[key & 511u], 1);
-            }
+            topk_count<SMEM, 512>(S, keys4, sc, n_valid, mask, prefix, 0, tid);
             __syncthreads();
-            topk_pick<512>(hist, wsum, remaining, prefix, 0, tid, &sh_prefix, &sh_rem, &sh_cnt);
-            prefix = sh_prefix;
-            remaining = sh_rem;
+            topk_pick<512>(S.hist, S.wsum, remaining, prefix, 0, tid, &S.prefix, &S.rem, &S.cnt);
+            prefix = S.prefix;
+            remaining = S.rem;
             mask = 0xFFFFFFFFu;
         }
     }
     // Selection: the keys whose masked bits are above the prefix, and the first
     // `remaining` equal to it in index order.  Warp w owns a contiguous segment of
-    // the row; it counts its keys above and equal, the warps exchange counts
-    // once, and each warp then writes its selected blocks at their ascending
-    // positions.
+    // the row (starting on a multiple of 32 when not empty); it counts its keys
+    // above and equal, the warps exchange counts once, and each warp then writes
+    // its selected blocks at their ascending positions.
+    auto key_at = [&](int b) -> unsigned { return SMEM ? keys_s[b] : topk_key(sc[b]); };
     const int seg = (((n_valid + 7) / 8) + 31) / 32 * 32;
     const int b_lo = min(warp * seg, n_valid), b_hi = min(b_lo + seg, n_valid);
     int n_gt = 0, n_eq = 0;
-    for (int b = b_lo + lane; b < b_hi; b += 32) {
-        const unsigned km = key_at(b) & mask;
-        n_gt += km > prefix;
-        n_eq += km == prefix;
+    if (SMEM) {
+        for (int q = (b_lo >> 2) + lane; 4 * q < b_hi; q += 32) {
+            const uint4 kk = keys4[q];
+            const unsigned k[4] = {kk.x, kk.y, kk.z, kk.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const unsigned km = k[j] & mask;
+                const bool in = 4 * q + j >= b_lo && 4 * q + j < b_hi;   // an empty segment starts mid-quad
+                n_gt += in && km > prefix;
+                n_eq += in && km == prefix;
+            }
+        }
+    } else {
+        for (int b = b_lo + lane; b < b_hi; b += 32) {
+            const unsigned km = key_at(b) & mask;
+            n_gt += km > prefix;
+            n_eq += km == prefix;
+        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -375,14 +403,14 @@ qsa_topk_kernel(const float *__restrict__ scores, int n, int KB, int32_t *__rest
         n_eq += __shfl_xor_sync(0xffffffffu, n_eq, o);
     }
     if (lane == 0) {
-        wcnt[warp][0] = n_gt;
-        wcnt[warp][1] = n_eq;
+        S.wcnt[warp][0] = n_gt;
+        S.wcnt[warp][1] = n_eq;
     }
     __syncthreads();
     int gt_before = 0, eq_before = 0;
     for (int w = 0; w < warp; ++w) {
-        gt_before += wcnt[w][0];
-        eq_before += wcnt[w][1];
+        gt_before += S.wcnt[w][0];
+        eq_before += S.wcnt[w][1];
     }
     const unsigned lt = (1u << lane) - 1u;
     int eq_run = eq_before, out_run = gt_before + min(eq_before, remaining);
@@ -401,6 +429,27 @@ qsa_topk_kernel(const float *__restrict__ scores, int n, int KB, int32_t *__rest
         if (take) out[out_run + __popc(take_mask & lt)] = b;
         out_run += __popc(take_mask);
     }
+}
+
+__global__ void __launch_bounds__(256)
+qsa_topk_kernel(const float *__restrict__ scores, int n, int KB, int32_t *__restrict__ sel) {
+    extern __shared__ uint4 keys4[];   // the row's keys when n_valid <= TOPK_CAP
+    __shared__ TopkSmem S;
+    const int tid = threadIdx.x;
+    const unsigned row = blockIdx.x;   // s * n + i (batch * n < 2^29)
+    const int i = (int)(row % (unsigned)n);
+    const int nb = n / qsa::R;
+    const int n_valid = (i + 1) / qsa::R;
+    const float *sc = scores + (size_t)row * nb;
+    int32_t *out = sel + (size_t)row * KB;
+    if (n_valid <= KB) {   // every complete block
+        for (int j = tid; j < KB; j += 256) out[j] = j < n_valid ? j : -1;
+        return;
+    }
+    if (n_valid <= qsa::TOPK_CAP)   // uniform
+        topk_row<true>(S, keys4, sc, nb, n_valid, KB, out, tid);
+    else
+        topk_row<false>(S, keys4, sc, nb, n_valid, KB, out, tid);
 }
 
 // ------------------------------------------------------------------ host
@@ -442,7 +491,8 @@ cudaError_t launch_qsa_indexer(const QsaArgs &a, void *ws) {
         if ((e = launched()) != cudaSuccess) return e;
     }
     if (a.n > 0) {
-        const int cap = nb < qsa::TOPK_CAP ? nb : qsa::TOPK_CAP;
+        // the row's keys, rounded up to whole 16-byte quads
+        const int cap = ((nb < qsa::TOPK_CAP ? nb : qsa::TOPK_CAP) + 3) & ~3;
         if ((e = cudaFuncSetAttribute(qsa_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, cap * 4)) !=
             cudaSuccess)
             return e;
