@@ -18,6 +18,14 @@ def test_rmsnorm_closed_form():
     np.testing.assert_allclose(qsa.rmsnorm(x, w), y * w, rtol=1e-12)
 
 
+def test_rmsnorm_epsilon():
+    # mean(x^2) = eps exactly: the normalised vector has RMS sqrt(eps / (2 eps)) = 1 / sqrt(2)
+    x = np.full(128, np.sqrt(qsa.EPS))
+    y = qsa.rmsnorm(x, np.ones(128))
+    np.testing.assert_allclose(np.sqrt(np.mean(y * y)), np.sqrt(0.5), rtol=1e-12)
+    assert qsa.EPS == 1e-6
+
+
 def test_prope_basis_vectors():
     # e_j (j < 32) at position p turns in the plane (j, j + 32) by p * 10000^(-j/32)
     for j, p in ((0, 5), (1, 3), (31, 1000)):
@@ -130,6 +138,14 @@ def test_constructed_winner():
     B, I = qsa.indexer(q, k, np.ones(128), np.ones(128), K=4, r=r)
     assert B[i, 0] == target
     assert np.argmax(np.where(np.isfinite(I[i]), I[i], -1)) == target
+    # rotated at position i, the normalised query is k_bar_6 / sqrt(mean(k_bar_6^2) + eps),
+    # so the score is |k_bar_6|^2 over that root (the other heads are zero: ReLU(0) = 0);
+    # rotating the query at position i + 1 instead gives a value about 1% smaller (only
+    # the fast pairs turn far), which the 1e-12 closed form tells apart
+    kk = kb[target]
+    assert I[i, target] == pytest.approx(kk @ kk / np.sqrt(np.mean(kk * kk) + qsa.EPS), rel=1e-12)
+    off = qsa.prope(qsa.rmsnorm(q_hat, np.ones(128)), i + 1) @ kk
+    assert off < (1 - 1e-3) * I[i, target]
 
 
 def test_expand_with_tail():
@@ -138,3 +154,6 @@ def test_expand_with_tail():
     assert toks == [8, 9, 10, 11, 16, 17, 18, 19, 20, 21, 22]   # two blocks and the tail 20 .. 22
     assert all(t <= 22 for t in toks)
     assert qsa.expand(np.array([0]), 3, K=8, r=4) == [0, 1, 2, 3]   # (i + 1) % r == 0: empty tail
+    # at i = 7 block 1 (tokens 4 .. 7) is complete: unless selected it is not in the set
+    assert qsa.expand(np.array([0, -1]), 7, K=8, r=4) == [0, 1, 2, 3]
+    assert qsa.expand(np.array([0, -1]), 8, K=8, r=4) == [0, 1, 2, 3, 8]
