@@ -211,8 +211,10 @@ GDN_API gdn_status_t gdn_qsa_indexer_workspace_size(int batch, int n, size_t *by
  * GDN_BF16; d_model a multiple of 8).  The projections are stored in bf16 between
  * the steps.  The three GEMM steps are plain bf16 GEMMs with fp32 accumulation on
  * cuBLAS, loaded at the first call (GDN_ERR_UNSUPPORTED when it cannot be
- * loaded); they are not fused with the mixer's prelude.  Stream-ordered workspace
- * from the library's pool: gdn_layer_workspace_size() bytes.
+ * loaded); they are not fused with the mixer's prelude.  Each host thread gets its
+ * own cuBLAS handle per device (created at its first call), so threads may run
+ * layers at the same time.  Stream-ordered workspace from the library's pool:
+ * gdn_layer_workspace_size() bytes.
  */
 GDN_API gdn_status_t gdn_layer_forward(const gdn_dims_t *dims, int d_model, const void *x, const void *w_in,
                                        const float *conv_w, const float *A, const float *b_alpha,

@@ -33,27 +33,32 @@ struct Blas {
     CreateFn create = nullptr;
     SetStreamFn set_stream = nullptr;
     GemmExFn gemm = nullptr;
-    cublasHandle_t handle[64] = {};
 };
 std::mutex g_blas_mu;
 Blas g_blas;
 
-// The cuBLAS entry points and this device's handle (created once per device).
+// The cuBLAS entry points (resolved once) and the calling thread's handle for this
+// device.  A handle carries the stream of the call in progress, so threads that
+// run layers at the same time must not share one: each (host thread, device)
+// gets its own, created at its first use and kept for the thread's lifetime.
 bool blas_handle(int dev, cublasHandle_t *h) {
-    std::lock_guard<std::mutex> lock(g_blas_mu);
-    if (!g_blas.tried) {
-        g_blas.tried = true;
-        void *lib = dlopen("libcublas.so.12", RTLD_NOW | RTLD_GLOBAL);
-        if (lib) {
-            g_blas.create = reinterpret_cast<CreateFn>(dlsym(lib, "cublasCreate_v2"));
-            g_blas.set_stream = reinterpret_cast<SetStreamFn>(dlsym(lib, "cublasSetStream_v2"));
-            g_blas.gemm = reinterpret_cast<GemmExFn>(dlsym(lib, "cublasGemmEx"));
-            g_blas.ok = g_blas.create && g_blas.set_stream && g_blas.gemm;
+    {
+        std::lock_guard<std::mutex> lock(g_blas_mu);
+        if (!g_blas.tried) {
+            g_blas.tried = true;
+            void *lib = dlopen("libcublas.so.12", RTLD_NOW | RTLD_GLOBAL);
+            if (lib) {
+                g_blas.create = reinterpret_cast<CreateFn>(dlsym(lib, "cublasCreate_v2"));
+                g_blas.set_stream = reinterpret_cast<SetStreamFn>(dlsym(lib, "cublasSetStream_v2"));
+                g_blas.gemm = reinterpret_cast<GemmExFn>(dlsym(lib, "cublasGemmEx"));
+                g_blas.ok = g_blas.create && g_blas.set_stream && g_blas.gemm;
+            }
         }
     }
     if (!g_blas.ok || dev < 0 || dev >= 64) return false;
-    if (!g_blas.handle[dev] && g_blas.create(&g_blas.handle[dev]) != CUBLAS_STATUS_SUCCESS) return false;
-    *h = g_blas.handle[dev];
+    thread_local cublasHandle_t tl_handle[64] = {};
+    if (!tl_handle[dev] && g_blas.create(&tl_handle[dev]) != CUBLAS_STATUS_SUCCESS) return false;
+    *h = tl_handle[dev];
     return true;
 }
 
