@@ -116,3 +116,29 @@ def test_qsa_deterministic(cuda_device):
     b, _ = gdn.qsa_indexer(inp["q"], inp["k"], inp["w_q"], inp["w_k"], budget=cfg.budget)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
+
+
+def test_qsa_rows_past_the_shared_memory_cap(cuda_device):
+    """n = 49,203: rows with more than 12,288 complete blocks keep their keys in the
+    score row instead of shared memory (and 12,287 blocks: the last row in shared
+    memory); sampled rows against the oracle."""
+    cfg = replace(QSA, n=49203, budget=2048, seed=11)
+    inp = make_qsa_inputs(cfg, "cpu")
+    dev = {key: val.to(cuda_device) for key, val in inp.items()}
+    sel, sc = gdn.qsa_indexer(dev["q"], dev["k"], dev["w_q"], dev["w_k"], budget=cfg.budget, want_scores=True)
+    torch.cuda.synchronize()
+    rows = [49150, 49155, 49170, 49202]
+    assert (49150 + 1) // 4 <= 12288 < (49155 + 1) // 4
+    sel_rows = sel[0, rows].cpu().numpy()
+    sc_rows = sc[0, rows].cpu().numpy()
+    del sel, sc
+    q = inp["q"][0].float().numpy()
+    kb = oq.keys(inp["k"][0].float().numpy(), inp["w_k"].numpy())
+    KB = cfg.budget // 4
+    for r, i in enumerate(rows):
+        qi = oq.prope(oq.rmsnorm(q[i], inp["w_q"].numpy()), np.full(4, i))
+        n_valid = (i + 1) // 4
+        I_row = np.maximum(qi @ kb[:n_valid].T, 0.0).sum(axis=0)
+        got = sc_rows[r, :n_valid]
+        assert normwise(got, I_row) <= TOL_SCORE, i
+        _oracle_row_check(I_row, sel_rows[r], n_valid, KB, 2 * np.abs(got - I_row).max())
