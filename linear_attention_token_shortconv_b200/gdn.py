@@ -118,6 +118,61 @@ def _stream(stream):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+F32, BF16, I32 = torch.float32, torch.bfloat16, torch.int32
+
+
+def _expect(name, t, shape, dtypes):
+    """Raises unless tensor `t` (None: absent, accepted) has this shape (None entries:
+    any size) and one of these dtypes.  The library sees only raw pointers, so a
+    mismatch here would otherwise be read as other bytes, or past the tensor."""
+    if t is None:
+        return
+    dtypes = dtypes if isinstance(dtypes, tuple) else (dtypes,)
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {' or '.join(str(d) for d in dtypes)}")
+    if t.dim() != len(shape) or any(w is not None and n != w for n, w in zip(t.shape, shape)):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _device(*ts):
+    """The one CUDA device that every given tensor (None entries skipped) is on;
+    the call runs there."""
+    dev = None
+    for t in ts:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("all tensors must live on a CUDA device")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"tensors on {dev} and {t.device}: all must be on one device")
+    return dev
+
+
+def _check_mixer(q, k, v, conv_w, a_logit, b_logit, A, b_alpha, z, norm_w, S0, cu_seqlens, out, S_final,
+                 n_seq, io=None, names=("out", "S_final")):
+    """Shapes and dtypes of the mixer's arguments in the packed token layout
+    (`names`: what the caller calls its out and S_final slots)."""
+    if q.dim() != 3 or v.dim() != 3 or conv_w.dim() != 2:
+        raise ValueError("q, k [N_tok, H, dk], v, z [N_tok, H, dv] and conv_w [C, K] expected")
+    n_tok, H, dk = q.shape
+    dv, K = v.shape[2], conv_w.shape[1]
+    io = (BF16, F32) if io is None else io
+    _expect("q", q, (n_tok, H, dk), io)
+    for name, t, shape in (("k", k, (n_tok, H, dk)), ("v", v, (n_tok, H, dv)), ("z", z, (n_tok, H, dv)),
+                           ("a_logit", a_logit, (n_tok, H)), ("b_logit", b_logit, (n_tok, H))):
+        _expect(name, t, shape, q.dtype)
+    _expect("conv_w", conv_w, (H * (2 * dk + dv), K), F32)
+    _expect("A", A, (H,), F32)
+    _expect("b_alpha", b_alpha, (H,), F32)
+    _expect("norm_w", norm_w, (dv,), F32)
+    _expect("S0", S0, (n_seq, H, dk, dv), F32)
+    _expect("cu_seqlens", cu_seqlens, (n_seq + 1,), I32)
+    _expect(names[0], out, (n_tok, H, dv), (F32, BF16))
+    _expect(names[1], S_final, (n_seq, H, dk, dv), F32)
+
+
 def _check(rc: int, where: str):
     if rc != 0:
         raise GdnError(rc, where)
@@ -139,11 +194,14 @@ def prefill(q, k, v, conv_w, a_logit, b_logit, A, b_alpha, z, norm_w, S0=None, c
         out = torch.empty((n_tok, H, dv), dtype=out_dtype, device=q.device)
     if S_final is None and want_state:
         S_final = torch.empty((n_seq, H, dk, dv), dtype=torch.float32, device=q.device)
+    _check_mixer(q, k, v, conv_w, a_logit, b_logit, A, b_alpha, z, norm_w, S0, cu_seqlens, out, S_final, n_seq)
     dims = Dims(n_seq, n_tok, H, dk, dv, conv_w.shape[1], _dt(q), _dt(out))
-    rc = load().gdn_prefill(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w),
-                            _ptr(a_logit), _ptr(b_logit), _ptr(A), _ptr(b_alpha), _ptr(z),
-                            _ptr(norm_w), _ptr(S0), _ptr(cu_seqlens), _ptr(out), _ptr(S_final),
-                            _stream(stream))
+    with torch.cuda.device(_device(q, k, v, conv_w, a_logit, b_logit, A, b_alpha, z, norm_w, S0, cu_seqlens,
+                                   out, S_final)):
+        rc = load().gdn_prefill(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w),
+                                _ptr(a_logit), _ptr(b_logit), _ptr(A), _ptr(b_alpha), _ptr(z),
+                                _ptr(norm_w), _ptr(S0), _ptr(cu_seqlens), _ptr(out), _ptr(S_final),
+                                _stream(stream))
     _check(rc, "gdn_prefill")
     return out, S_final
 
@@ -167,13 +225,18 @@ def prefill_backward(q, k, v, conv_w, a_logit, b_logit, A, b_alpha, z, norm_w, d
          "d_b_alpha": torch.empty_like(b_alpha), "d_z": torch.empty_like(z),
          "d_norm_w": torch.empty_like(norm_w),
          "d_S0": torch.empty((n_seq, H, dk, dv), dtype=f32, device=dev) if want_d_S0 else None}
+    _check_mixer(q, k, v, conv_w, a_logit, b_logit, A, b_alpha, z, norm_w, S0, cu_seqlens, d_out, d_S_final,
+                 n_seq, names=("d_out", "d_S_final"))
+    _expect("d_out", d_out, (n_tok, H, dv), q.dtype)
     dims = Dims(n_seq, n_tok, H, dk, dv, conv_w.shape[1], _dt(q), _dt(d_out))
-    rc = load().gdn_prefill_backward(
-        ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w), _ptr(a_logit), _ptr(b_logit),
-        _ptr(A), _ptr(b_alpha), _ptr(z), _ptr(norm_w), _ptr(S0), _ptr(cu_seqlens), _ptr(d_out),
-        _ptr(d_S_final), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["d_conv_w"]),
-        _ptr(g["d_a_logit"]), _ptr(g["d_b_logit"]), _ptr(g["d_A"]), _ptr(g["d_b_alpha"]), _ptr(g["d_z"]),
-        _ptr(g["d_norm_w"]), _ptr(g["d_S0"]), _stream(stream))
+    with torch.cuda.device(_device(q, k, v, conv_w, a_logit, b_logit, A, b_alpha, z, norm_w, S0, cu_seqlens,
+                                   d_out, d_S_final)):
+        rc = load().gdn_prefill_backward(
+            ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w), _ptr(a_logit), _ptr(b_logit),
+            _ptr(A), _ptr(b_alpha), _ptr(z), _ptr(norm_w), _ptr(S0), _ptr(cu_seqlens), _ptr(d_out),
+            _ptr(d_S_final), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["d_conv_w"]),
+            _ptr(g["d_a_logit"]), _ptr(g["d_b_logit"]), _ptr(g["d_A"]), _ptr(g["d_b_alpha"]), _ptr(g["d_z"]),
+            _ptr(g["d_norm_w"]), _ptr(g["d_S0"]), _stream(stream))
     _check(rc, "gdn_prefill_backward")
     return g
 
@@ -194,13 +257,22 @@ def qsa_indexer(q, k, w_q, w_k, budget=2048, *, sel=None, scores=None, want_scor
     squeeze = q.dim() == 3
     if squeeze:
         q, k = q.unsqueeze(0), k.unsqueeze(0)
+    if q.dim() != 4:
+        raise ValueError("q [B, n, heads, d] (or [n, heads, d]) expected")
     B, n, H, d = q.shape
     if sel is None:
         sel = torch.empty((B, n, budget // 4), dtype=torch.int32, device=q.device)
     if scores is None and want_scores:
         scores = torch.empty((B, n, n // 4), dtype=torch.float32, device=q.device)
-    rc = load().gdn_qsa_indexer(B, n, H, d, 4, budget, _ptr(q), _ptr(k), _ptr(w_q), _ptr(w_k), _ptr(sel),
-                                _ptr(scores), _stream(stream))
+    _expect("q", q, (B, n, H, d), BF16)
+    _expect("k", k, (B, n, d), BF16)
+    _expect("w_q", w_q, (d,), F32)
+    _expect("w_k", w_k, (d,), F32)
+    _expect("sel", sel, (B, n, budget // 4), I32)
+    _expect("scores", scores, (B, n, n // 4), F32)
+    with torch.cuda.device(_device(q, k, w_q, w_k, sel, scores)):
+        rc = load().gdn_qsa_indexer(B, n, H, d, 4, budget, _ptr(q), _ptr(k), _ptr(w_q), _ptr(w_k), _ptr(sel),
+                                    _ptr(scores), _stream(stream))
     _check(rc, "gdn_qsa_indexer")
     if squeeze:
         sel = sel[0]
@@ -223,10 +295,22 @@ def layer_forward(x, w_in, conv_w, A, b_alpha, norm_w, w_o, H, dk, dv, S0=None, 
         y = torch.empty((n_tok, d_model), dtype=torch.bfloat16, device=x.device)
     if S_final is None and want_state:
         S_final = torch.empty((n_seq, H, dk, dv), dtype=torch.float32, device=x.device)
+    _expect("x", x, (n_tok, d_model), BF16)
+    _expect("w_in", w_in, (d_model, H * (2 * dk + 2 * dv) + 2 * H), BF16)
+    _expect("w_o", w_o, (H * dv, d_model), BF16)
+    _expect("conv_w", conv_w, (H * (2 * dk + dv), None), F32)
+    _expect("A", A, (H,), F32)
+    _expect("b_alpha", b_alpha, (H,), F32)
+    _expect("norm_w", norm_w, (dv,), F32)
+    _expect("S0", S0, (n_seq, H, dk, dv), F32)
+    _expect("cu_seqlens", cu_seqlens, (n_seq + 1,), I32)
+    _expect("y", y, (n_tok, d_model), BF16)
+    _expect("S_final", S_final, (n_seq, H, dk, dv), F32)
     dims = Dims(n_seq, n_tok, H, dk, dv, conv_w.shape[1], GDN_BF16, GDN_BF16)
-    rc = load().gdn_layer_forward(ctypes.byref(dims), d_model, _ptr(x), _ptr(w_in), _ptr(conv_w), _ptr(A),
-                                  _ptr(b_alpha), _ptr(norm_w), _ptr(w_o), _ptr(S0), _ptr(cu_seqlens), _ptr(y),
-                                  _ptr(S_final), _stream(stream))
+    with torch.cuda.device(_device(x, w_in, conv_w, A, b_alpha, norm_w, w_o, S0, cu_seqlens, y, S_final)):
+        rc = load().gdn_layer_forward(ctypes.byref(dims), d_model, _ptr(x), _ptr(w_in), _ptr(conv_w), _ptr(A),
+                                      _ptr(b_alpha), _ptr(norm_w), _ptr(w_o), _ptr(S0), _ptr(cu_seqlens),
+                                      _ptr(y), _ptr(S_final), _stream(stream))
     _check(rc, "gdn_layer_forward")
     return y, S_final
 
@@ -248,11 +332,14 @@ def prefill_noalloc(q, k, v, conv_w, a_logit, b_logit, A, b_alpha, z, norm_w, S0
         out = torch.empty((n_tok, H, dv), dtype=out_dtype, device=q.device)
     if S_final is None and want_state:
         S_final = torch.empty((n_seq, H, dk, dv), dtype=torch.float32, device=q.device)
+    _check_mixer(q, k, v, conv_w, a_logit, b_logit, A, b_alpha, z, norm_w, S0, cu_seqlens, out, S_final, n_seq)
     dims = Dims(n_seq, n_tok, H, dk, dv, conv_w.shape[1], _dt(q), _dt(out))
-    rc = load().gdn_prefill_noalloc(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w),
-                                    _ptr(a_logit), _ptr(b_logit), _ptr(A), _ptr(b_alpha), _ptr(z),
-                                    _ptr(norm_w), _ptr(S0), _ptr(cu_seqlens), _ptr(out),
-                                    _ptr(S_final), _stream(stream))
+    with torch.cuda.device(_device(q, k, v, conv_w, a_logit, b_logit, A, b_alpha, z, norm_w, S0, cu_seqlens,
+                                   out, S_final)):
+        rc = load().gdn_prefill_noalloc(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w),
+                                        _ptr(a_logit), _ptr(b_logit), _ptr(A), _ptr(b_alpha), _ptr(z),
+                                        _ptr(norm_w), _ptr(S0), _ptr(cu_seqlens), _ptr(out),
+                                        _ptr(S_final), _stream(stream))
     _check(rc, "gdn_prefill_noalloc")
     return out, S_final
 
@@ -275,11 +362,25 @@ def decode_step(q, k, v, conv_w, conv_hist, a_logit, b_logit, A, b_alpha, z, nor
     dv = v.shape[2]
     if out is None:
         out = torch.empty((B, H, dv), dtype=out_dtype, device=q.device)
-    dims = Dims(B, B, H, dk, dv, conv_w.shape[1], _dt(q), _dt(out))
-    rc = load().gdn_decode_step(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w),
-                                _ptr(conv_hist), _ptr(a_logit), _ptr(b_logit), _ptr(A),
-                                _ptr(b_alpha), _ptr(z), _ptr(norm_w), _ptr(S), _ptr(out),
-                                _stream(stream))
+    K = conv_w.shape[1]
+    C = H * (2 * dk + dv)
+    _expect("q", q, (B, H, dk), (BF16, F32))
+    for name, t, shape in (("k", k, (B, H, dk)), ("v", v, (B, H, dv)), ("z", z, (B, H, dv)),
+                           ("conv_hist", conv_hist, (B, K - 1, C)), ("a_logit", a_logit, (B, H)),
+                           ("b_logit", b_logit, (B, H))):
+        _expect(name, t, shape, q.dtype)
+    _expect("conv_w", conv_w, (C, K), F32)
+    _expect("A", A, (H,), F32)
+    _expect("b_alpha", b_alpha, (H,), F32)
+    _expect("norm_w", norm_w, (dv,), F32)
+    _expect("S", S, (B, H, dk, dv), F32)
+    _expect("out", out, (B, H, dv), (F32, BF16))
+    dims = Dims(B, B, H, dk, dv, K, _dt(q), _dt(out))
+    with torch.cuda.device(_device(q, k, v, conv_w, conv_hist, a_logit, b_logit, A, b_alpha, z, norm_w, S, out)):
+        rc = load().gdn_decode_step(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w),
+                                    _ptr(conv_hist), _ptr(a_logit), _ptr(b_logit), _ptr(A),
+                                    _ptr(b_alpha), _ptr(z), _ptr(norm_w), _ptr(S), _ptr(out),
+                                    _stream(stream))
     _check(rc, "gdn_decode_step")
     return out
 
@@ -293,11 +394,27 @@ def decode_multi(q, k, v, conv_w, conv_hist, a_logit, b_logit, A, b_alpha, z, no
     dv = v.shape[3]
     if out is None:
         out = torch.empty((B, T, H, dv), dtype=out_dtype, device=q.device)
-    dims = Dims(B, B * T, H, dk, dv, conv_w.shape[1], _dt(q), _dt(out))
-    rc = load().gdn_decode_multi(ctypes.byref(dims), T, _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w),
-                                 _ptr(conv_hist), _ptr(a_logit), _ptr(b_logit), _ptr(A), _ptr(b_alpha),
-                                 _ptr(z), _ptr(norm_w), _ptr(S), _ptr(out), _ptr(n_keep),
-                                 _stream(stream))
+    K = conv_w.shape[1]
+    C = H * (2 * dk + dv)
+    _expect("q", q, (B, T, H, dk), (BF16, F32))
+    for name, t, shape in (("k", k, (B, T, H, dk)), ("v", v, (B, T, H, dv)), ("z", z, (B, T, H, dv)),
+                           ("conv_hist", conv_hist, (B, K - 1, C)), ("a_logit", a_logit, (B, T, H)),
+                           ("b_logit", b_logit, (B, T, H))):
+        _expect(name, t, shape, q.dtype)
+    _expect("conv_w", conv_w, (C, K), F32)
+    _expect("A", A, (H,), F32)
+    _expect("b_alpha", b_alpha, (H,), F32)
+    _expect("norm_w", norm_w, (dv,), F32)
+    _expect("S", S, (B, H, dk, dv), F32)
+    _expect("out", out, (B, T, H, dv), (F32, BF16))
+    _expect("n_keep", n_keep, (B,), I32)
+    dims = Dims(B, B * T, H, dk, dv, K, _dt(q), _dt(out))
+    with torch.cuda.device(_device(q, k, v, conv_w, conv_hist, a_logit, b_logit, A, b_alpha, z, norm_w, S, out,
+                                   n_keep)):
+        rc = load().gdn_decode_multi(ctypes.byref(dims), T, _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w),
+                                     _ptr(conv_hist), _ptr(a_logit), _ptr(b_logit), _ptr(A), _ptr(b_alpha),
+                                     _ptr(z), _ptr(norm_w), _ptr(S), _ptr(out), _ptr(n_keep),
+                                     _stream(stream))
     _check(rc, "gdn_decode_multi")
     return out
 
