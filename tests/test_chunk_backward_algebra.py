@@ -32,33 +32,37 @@ import torch
 import oracle
 
 
-def _chunk_forward(Q, K, V, g, b, S):
+def _chunk_forward(Q, K, V, g, b, S, mm=np.matmul):
     n = Q.shape[0]
     G = np.cumsum(g)
     incl = np.tril(np.ones((n, n)))
     SL = np.tril(np.ones((n, n)), -1)
     Gam = np.exp(np.where(incl > 0, G[:, None] - G[None, :], -np.inf))
-    KK = K @ K.T
+    KK = mm(K, K.T)
     L = b[:, None] * KK * Gam * SL
     T = np.linalg.inv(np.eye(n) + L)
     eG = np.exp(G)
     X1 = b[:, None] * V
     X2 = (b * eG)[:, None] * K
-    W = T @ X2
-    U = T @ X1 - W @ S
-    QK = Q @ K.T
+    W = mm(T, X2)
+    U = mm(T, X1) - mm(W, S)
+    QK = mm(Q, K.T)
     A = QK * Gam
     Qt = eG[:, None] * Q
     r = np.exp(G[-1] - G)
     Kt = r[:, None] * K
-    Y = Qt @ S + A @ U
-    S_next = np.exp(G[-1]) * S + Kt.T @ U
+    Y = mm(Qt, S) + mm(A, U)
+    S_next = np.exp(G[-1]) * S + mm(Kt.T, U)
     return dict(G=G, incl=incl, SL=SL, Gam=Gam, KK=KK, T=T, eG=eG, X1=X1, X2=X2, W=W, U=U, QK=QK, A=A, Qt=Qt,
                 Kt=Kt, r=r), Y, S_next
 
 
-def chunked_delta_rule_backward(q, k, v, log_alpha, beta, S0, C, dY, dS_final):
-    """Gradients (dq, dk, dv, dlog_alpha, dbeta, dS0) of <dY, Y> + <dS_final, S_T>."""
+def chunked_delta_rule_backward(q, k, v, log_alpha, beta, S0, C, dY, dS_final, mm=np.matmul,
+                                keep=lambda x: x):
+    """Gradients (dq, dk, dv, dlog_alpha, dbeta, dS0) of <dY, Y> + <dS_final, S_T>.
+    `mm` computes every matrix product (an emulation of reduced-precision operands
+    may stand in); `keep` rounds the state and its gradient where a kernel would
+    store them."""
     T_len = q.shape[0]
     starts = list(range(0, T_len, C))
     S_at = []                                   # the state at each chunk's start (checkpoints)
@@ -66,29 +70,30 @@ def chunked_delta_rule_backward(q, k, v, log_alpha, beta, S0, C, dY, dS_final):
     for c0 in starts:
         sl = slice(c0, min(c0 + C, T_len))
         S_at.append(S)
-        _, _, S = _chunk_forward(q[sl], k[sl], v[sl], log_alpha[sl], beta[sl], S)
+        _, _, S = _chunk_forward(q[sl], k[sl], v[sl], log_alpha[sl], beta[sl], S, mm)
+        S = keep(S)
     dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
     dg, db = np.zeros_like(log_alpha), np.zeros_like(beta)
     dS = dS_final.copy()
     for c0, S in zip(reversed(starts), reversed(S_at)):
         sl = slice(c0, min(c0 + C, T_len))
         Q, K, V, b, dYc = q[sl], k[sl], v[sl], beta[sl], dY[sl]
-        f, _, _ = _chunk_forward(Q, K, V, log_alpha[sl], b, S)
+        f, _, _ = _chunk_forward(Q, K, V, log_alpha[sl], b, S, mm)
         eGC = np.exp(f["G"][-1])
         # through Y = Qt S + A U and S' = e^{G_C} S + Kt^T U
-        dU = f["A"].T @ dYc + f["Kt"] @ dS
-        dA = (dYc @ f["U"].T) * f["incl"]
-        dQt = dYc @ S.T
-        dKt = f["U"] @ dS.T
-        dS_prev = f["Qt"].T @ dYc + eGC * dS
+        dU = mm(f["A"].T, dYc) + mm(f["Kt"], dS)
+        dA = mm(dYc, f["U"].T) * f["incl"]
+        dQt = mm(dYc, S.T)
+        dKt = mm(f["U"], dS.T)
+        dS_prev = mm(f["Qt"].T, dYc) + eGC * dS
         dGC = eGC * np.sum(dS * S)
         # through U = U' - W S, U' = T X1, W = T X2, T = (I + L)^-1
-        dW = -dU @ S.T
-        dS_prev -= f["W"].T @ dU
-        dT = dU @ f["X1"].T + dW @ f["X2"].T
-        dX1 = f["T"].T @ dU
-        dX2 = f["T"].T @ dW
-        dL = -(f["T"].T @ dT @ f["T"].T) * f["SL"]
+        dW = -mm(dU, S.T)
+        dS_prev -= mm(f["W"].T, dU)
+        dT = mm(dU, f["X1"].T) + mm(dW, f["X2"].T)
+        dX1 = mm(f["T"].T, dU)
+        dX2 = mm(f["T"].T, dW)
+        dL = -mm(mm(f["T"].T, dT), f["T"].T) * f["SL"]
         # leaves: V, beta, K, Q
         dv[sl] = b[:, None] * dX1
         db[sl] = (np.sum(dX1 * V, 1) + np.sum(dX2 * f["eG"][:, None] * K, 1)
@@ -96,15 +101,16 @@ def chunked_delta_rule_backward(q, k, v, log_alpha, beta, S0, C, dY, dS_final):
         P = b[:, None] * dL                              # gradient of K K^T * Gamma (strict lower)
         dKK = P * f["Gam"]
         dQK = dA * f["Gam"]
-        dk[sl] = ((b * f["eG"])[:, None] * dX2 + f["r"][:, None] * dKt + dKK @ K + dKK.T @ K + dQK.T @ Q)
-        dq[sl] = f["eG"][:, None] * dQt + dQK @ K
+        dk[sl] = ((b * f["eG"])[:, None] * dX2 + f["r"][:, None] * dKt + mm(dKK, K) + mm(dKK.T, K)
+                  + mm(dQK.T, Q))
+        dq[sl] = f["eG"][:, None] * dQt + mm(dQK, K)
         # log-decays: every factor e^{G_i - G_j}, e^{G_i}, e^{G_C - G_i}, e^{G_C}
         E = (P * f["KK"] + dA * f["QK"]) * f["Gam"]
         dG = E.sum(1) - E.sum(0)
         dG += np.sum(dQt * f["Qt"], 1) + np.sum(dX2 * f["X2"], 1) - np.sum(dKt * f["Kt"], 1)
         dG[-1] += np.sum(dKt * f["Kt"]) + dGC
         dg[sl] = np.cumsum(dG[::-1])[::-1]
-        dS = dS_prev
+        dS = keep(dS_prev)
     return dq, dk, dv, dg, db, dS
 
 
