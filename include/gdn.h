@@ -101,7 +101,9 @@ typedef struct {
  *              may be NULL when not wanted)
  *
  * Each sequence starts with an empty conv history.  `out` must not alias any
- * input.  On the tensor-core path (bf16 inputs, dk = 128) a call with
+ * input.  The log-decay -exp(A) softplus(a_logit + b_alpha) must be finite in
+ * fp32: on the tensor-core path a decay that overflows to -inf (a logit near
+ * 3e38 / exp(A)) makes that chunk's outputs NaN.  On the tensor-core path (bf16 inputs, dk = 128) a call with
  * dk = dv = 128 and at most SMs / 4 (sequence, head) pairs runs as one
  * cooperative persistent kernel on `stream` (one CTA per SM); other long inputs
  * run in chunk segments whose kernels overlap on `stream` and on two
