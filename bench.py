@@ -32,7 +32,7 @@ sys.path.insert(0, ROOT)
 
 from linear_attention_token_shortconv_b200 import dist as rankio  # noqa: E402
 from linear_attention_token_shortconv_b200 import gdn  # noqa: E402
-from linear_attention_token_shortconv_b200.workloads import (DECODE, LONG, PRETRAIN, QSA,  # noqa: E402
+from linear_attention_token_shortconv_b200.workloads import (DECODE, LONG, PRETRAIN, QSA, VARLEN,  # noqa: E402
                                                              make_decode_inputs, make_layer_inputs,
                                                              make_prefill_inputs, make_qsa_inputs, to_oracle_bits)
 
@@ -67,7 +67,7 @@ KERNEL_ROOFLINE = {"chunk_prep": ("hbm", 3 * 128 * 2 + 2 * 2),                  
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per unit from one
 # ncu capture of each kernel (profiles/), valid only while the kernel's sources
 # are the ones captured (sha1 over them); otherwise the JSON reports traffic null.
-#   prefill_fused: `profile_case prefill 8192` (T = 8192, H = 32): 276.6 MB read +
+#   prefill_fused: `bench.py --profile-case prefill 8192` (T = 8192, H = 32): 276.6 MB read +
 #     344.2 MB written for 262,144 token-heads; per token-head, scaled to the launch.
 NCU_TRAFFIC = {
     "prefill_fused": {"sources": ["prefill_tc.cu", "prep_body.cuh", "chain_body.cuh"],
@@ -91,6 +91,11 @@ def kernel_traffic(name, units):
     except OSError:
         return None
     return rec["bytes_per_unit"] * units if h.hexdigest() == rec["sha1"] else None
+
+
+# Peaks used only when MEASURED_PEAKS.json is absent: an earlier measurement on
+# the same B200 pool (STREAM-style copy; cuBLAS bf16 burst and sustained).
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
 def peaks():
@@ -266,6 +271,24 @@ def bench_prefill(cfg, steps, warmup, world, rank, dev):
                          "avg_launch_ms": max_over_ranks(statistics.fmean(xs), world),
                          "ms_per_step": max_over_ranks(sum(xs) / steps, world)}
     return ms, kern_ms, clk.summary(), kernels, launches, inp
+
+
+def prefill_summary(cfg, steps, ms, kern_ms, kernels, pk):
+    """Whole-call throughput and roofline fractions of one timed prefill workload,
+    with each kernel's share of the call (from its per-launch events)."""
+    th = cfg.total_tokens * cfg.H
+    gbs = PREFILL_BYTES_PER_TOKEN_HEAD * th / (kern_ms * 1e-3) / 1e9
+    tf = PREFILL_FLOP_PER_TOKEN_HEAD * th / (kern_ms * 1e-3) / 1e12
+    total = sum(k["ms_per_step"] for k in kernels.values()) or 1.0
+    return {"workload": cfg.name, "steps": steps, "ms_per_step": ms, "call_ms": kern_ms,
+            "tokens_per_s": cfg.total_tokens / (ms * 1e-3),
+            "hbm": {"bytes_per_token_head": PREFILL_BYTES_PER_TOKEN_HEAD, "achieved_gbs": gbs,
+                    "peak_gbs": pk["hbm_gbs"], "frac": gbs / pk["hbm_gbs"]},
+            "tc": {"flop_per_token_head": PREFILL_FLOP_PER_TOKEN_HEAD, "achieved_tflops": tf,
+                   "peak_tflops": pk["bf16_tflops"], "frac": tf / pk["bf16_tflops"]},
+            "kernels": {n: {"launches_per_step": k["launches_per_step"], "ms_per_step": k["ms_per_step"],
+                            "avg_launch_ms": k["avg_launch_ms"], "share": k["ms_per_step"] / total}
+                        for n, k in kernels.items()}}
 
 
 def bench_e2e(cfg, steps, warmup, world, rank, dev):
@@ -521,6 +544,58 @@ def run_reference(args, world, rank):
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
 
 
+def profile_case(kind, size):
+    """Small workloads for ncu captures (a few hundred MB on the device, inputs
+    larger than L2), run through the public binding on cuda:0:
+      prefill T   the long-prefill shape with T tokens (H = 32, d = 128, S0):
+                  two warm-up calls, then one call
+      pretrain T  the pretraining shape with 4 sequences of T tokens (H = 16):
+                  two warm-up calls, then one call
+      decode B    decode steps for B sequences x 32 heads, d = 128: three steps
+      backward T  prefill backward, 4 sequences x T tokens, H = 16, d = 128, fp32: three calls
+      qsa n       QSA indexer on one sequence of n tokens, K = 2048: three calls"""
+    dev = torch.device("cuda", 0)
+    if kind in ("prefill", "pretrain"):
+        cfg = replace(LONG, lengths=(size,)) if kind == "prefill" else replace(PRETRAIN, lengths=(size,) * 4)
+        inp = make_prefill_inputs(cfg, dev)
+        out = torch.empty((cfg.total_tokens, cfg.H, cfg.dv), dtype=torch.bfloat16, device=dev)
+        S = torch.empty((cfg.num_seqs, cfg.H, cfg.dk, cfg.dv), device=dev)
+        for _ in range(3):
+            prefill_call(inp, out, S)
+        torch.cuda.synchronize()
+        print("ok", float(out.float().abs().mean()))
+    elif kind == "decode":
+        cfg = replace(DECODE, B=size)
+        d = make_decode_inputs(cfg, dev)
+        out = torch.empty((cfg.B, cfg.H, cfg.dv), dtype=torch.bfloat16, device=dev)
+        for t in range(3):
+            gdn.decode_step(d["q"][t], d["k"][t], d["v"][t], d["conv_w"], d["ring"], d["a_logit"][t],
+                            d["b_logit"][t], d["A"], d["b_alpha"], d["z"][t], d["norm_w"], d["S"], out=out)
+        torch.cuda.synchronize()
+        print("ok", float(out.float().abs().mean()))
+    elif kind == "backward":
+        cfg = replace(PRETRAIN, lengths=(size,) * 4, in_dtype=torch.float32)
+        inp = make_prefill_inputs(cfg, dev)
+        g = torch.Generator(device=dev)
+        g.manual_seed(cfg.seed + 100)
+        d_out = torch.randn((cfg.total_tokens, cfg.H, cfg.dv), generator=g, device=dev)
+        for _ in range(3):
+            grads = gdn.prefill_backward(inp["q"], inp["k"], inp["v"], inp["conv_w"], inp["a_logit"],
+                                         inp["b_logit"], inp["A"], inp["b_alpha"], inp["z"], inp["norm_w"],
+                                         d_out, S0=inp.get("S0"), num_seqs=cfg.num_seqs)
+        torch.cuda.synchronize()
+        print("ok", float(grads["dq"].abs().mean()))
+    elif kind == "qsa":
+        cfg = replace(QSA, n=size)
+        inp = make_qsa_inputs(cfg, dev)
+        for _ in range(3):
+            sel, _ = gdn.qsa_indexer(inp["q"], inp["k"], inp["w_q"], inp["w_k"], budget=cfg.budget)
+        torch.cuda.synchronize()
+        print("ok", int(sel[-1, -1, 0]))
+    else:
+        raise SystemExit(f"unknown profile case {kind!r}")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -530,9 +605,24 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--profile-case", nargs=2, metavar=("KIND", "SIZE"),
+                    help="run one small workload for an ncu capture instead of the benchmark "
+                         "(prefill T | pretrain T | decode B | backward T | qsa n)")
     args = ap.parse_args()
+    if args.profile_case:
+        profile_case(args.profile_case[0], int(args.profile_case[1]))
+        return
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")
+    if args.gpus < 1:
+        ap.error("--gpus must be at least 1")
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        # not under a launcher: start one process per GPU (each re-enters here
+        # with its rank in the environment) and pass on their exit status
+        sys.exit(rankio.launch(args.gpus, os.path.abspath(__file__), sys.argv[1:]))
+    if "WORLD_SIZE" in os.environ and rankio.env_ranks()[0] != args.gpus:
+        print(f"bench.py: --gpus {args.gpus}, but the launcher started {rankio.env_ranks()[0]} ranks; "
+              "timing the launcher's ranks", file=sys.stderr)
 
     world, rank, local = rankio.setup("nccl") if args.impl == "ours" else rankio.env_ranks()
     if args.impl == "reference":
@@ -572,6 +662,7 @@ def main():
         "config": {"workload": "long prefill: 1 seq x T=32768, H=32, dk=dv=128, bf16 in/out, "
                                "fp32 state, S0~N(0,0.02), per GPU",
                    "global_batch": world, "seq_len": cfg.total_tokens, "parallelism": f"dp{world}",
+                   "process_group_size": rankio.group_size(),
                    "l2": "inputs larger than L2 (1.07 GB of bf16 q,k,v,z read per step)"},
         "roofline": {"bound": bound, "achieved": dom_ach, "peak": dom_peak, "unit": dom_unit,
                      "frac": dom_ach / dom_peak, "traffic": traffic, "kernel": dom,
@@ -590,6 +681,16 @@ def main():
     }
     del inp
     torch.cuda.empty_cache()
+
+    if rank == 0:
+        # the other prefill workloads (several sequences: the segmented pipeline of
+        # chunk_prep / chunk_chain launches), timed on this rank alone
+        for key, pcfg in (("pretrain", PRETRAIN), ("varlen", VARLEN)):
+            p_ms, p_kern, _, p_kernels, p_launch, p_inp = bench_prefill(pcfg, 5, 3, 1, 0, dev)
+            result[key] = prefill_summary(pcfg, 5, p_ms, p_kern, p_kernels, pk)
+            result[key]["gpu_launches"] = p_launch
+            del p_inp
+            torch.cuda.empty_cache()
 
     if rank == 0 and args.decode_steps > 0:
         dms, dk_ms, sbytes, dlaunch, dclk = bench_decode(DECODE, args.decode_steps, dev)

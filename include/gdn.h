@@ -101,9 +101,11 @@ typedef struct {
  *              may be NULL when not wanted)
  *
  * Each sequence starts with an empty conv history.  `out` must not alias any
- * input.  The log-decay -exp(A) softplus(a_logit + b_alpha) must be finite in
- * fp32: on the tensor-core path a decay that overflows to -inf (a logit near
- * 3e38 / exp(A)) makes that chunk's outputs NaN.  On the tensor-core path (bf16 inputs, dk = 128) a call with
+ * input.  Any finite decay logit is accepted: on the tensor-core path the
+ * log-decay -exp(A) softplus(a_logit + b_alpha) is clamped below at -128, where
+ * exp() of it is already exactly 0 in fp32, so a logit that makes it overflow to
+ * -inf (near 3e38 / exp(A)) gives alpha = 0 as in exact arithmetic instead of
+ * NaN.  On the tensor-core path (bf16 inputs, dk = 128) a call with
  * dk = dv = 128 and at most SMs / 4 (sequence, head) pairs runs as one
  * cooperative persistent kernel on `stream` (one CTA per SM); other long inputs
  * run in chunk segments whose kernels overlap on `stream` and on two
@@ -298,8 +300,12 @@ GDN_API gdn_status_t gdn_decode_multi(const gdn_dims_t *dims, int T, const void 
  *     GDN_NOALLOC_SCRATCH_BYTES, about 29,000 token-heads at dk = dv = 128;
  *     larger calls return GDN_ERR_INVALID_ARG and launch nothing.
  *   - The array exists once per GPU that loads the library, until exit.  The
- *     first call on a device looks up its device address; make that first call
- *     before any stream capture.
+ *     first call on a device looks up its device address and keeps it; make
+ *     that first call before any stream capture, and do not use the library
+ *     across a cudaDeviceReset() of that device (the kept address would be
+ *     stale).
+ *   - The profiling hooks gdn_set_timing_events and gdn_set_kernel_events
+ *     record nothing for this call.
  *   - All calls on a device share the array, which keeps the last call's
  *     contents (nothing in it must start at zero).  Calls whose GPU work
  *     overlaps, e.g. on two streams at once, race on it: serialise them.

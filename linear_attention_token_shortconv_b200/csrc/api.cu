@@ -101,22 +101,6 @@ cudaError_t get_pool(cudaMemPool_t *pool) {
     return cudaSuccess;
 }
 
-// SM count of the current device (cached per device).
-cudaError_t sm_count(int *out) {
-    static int cache[64] = {};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!cache[dev]) {
-        int n = 0;
-        if ((e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-        cache[dev] = n;
-    }
-    *out = cache[dev];
-    return cudaSuccess;
-}
-
 // Per-device side streams (chain: highest priority; prep2: default priority)
 // and event pool for the segments.
 struct SideStream {
@@ -210,7 +194,7 @@ cudaError_t prefill_dispatch(const gdn::PrefillArgs &a) {
         const Segments g = segments(dims);
         int slot = 0, sms = 0;
         e = record(g_ev_begin, a.stream);
-        if (e == cudaSuccess) e = sm_count(&sms);
+        if (e == cudaSuccess) e = gdn::sm_count(&sms);
         if (e == cudaSuccess && gdn::fused_chain_ctas(a, sms) > 0) {
             // few (sequence, head) chains: one persistent launch, prep and chain
             // ordered by per-chunk flags
@@ -275,6 +259,21 @@ cudaError_t prefill_dispatch(const gdn::PrefillArgs &a) {
 }  // namespace
 
 namespace gdn {
+cudaError_t sm_count(int *out) {
+    static int cache[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!cache[dev]) {
+        int n = 0;
+        if ((e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+        cache[dev] = n;
+    }
+    *out = cache[dev];
+    return cudaSuccess;
+}
+
 void note_launch() { ++tl_launches; }
 void reset_launch_count() { tl_launches = 0; }
 }  // namespace gdn

@@ -768,7 +768,11 @@ bwd_reduce_kernel(const float *__restrict__ dw_part, int n_tiles, int C4, const 
 
 // ---------------------------------------------------------------------- host
 namespace bwd {
-constexpr int EPI_BLOCKS = 4 * 148;   // grid of the output-stage kernel (fixed: its partial sums have a fixed order)
+// Grid of the output-stage kernel: 592 blocks (four per SM of a 148-SM B200).
+// Deliberately a constant rather than a multiple of the queried SM count: the
+// kernel's norm-weight partial sums are one per block and are added in block
+// order, so a fixed grid keeps the results bit-identical on every device.
+constexpr int EPI_BLOCKS = 592;
 }  // namespace bwd
 
 size_t backward_workspace_bytes(int n_seq, int n_tok, int H, int D) {

@@ -55,6 +55,15 @@ __device__ __forceinline__ float sigmoid_acc(float x) { return 1.0f / (1.0f + ex
 __device__ __forceinline__ float softplus_acc(float x) {
     return x > 0.0f ? x + log1pf(expf(-x)) : log1pf(expf(x));
 }
+// Lower bound of the log-decay on the chunked (tensor-core) path.  That path
+// forms e^{G_i - G_j} from in-chunk cumulative sums of log alpha, so a log-decay
+// that overflows to -inf (a decay logit near the top of the bf16 range) would
+// give -inf - (-inf) = NaN.  Every log-decay at or below -104 already makes
+// e^g, and every product that contains it, exactly 0 in fp32, so clamping at
+// -128 changes no result and keeps the sums finite.  A NaN logit stays NaN.
+constexpr float kLogDecayFloor = -128.f;
+__device__ __forceinline__ float clamp_log_decay(float g) { return g < kLogDecayFloor ? kLogDecayFloor : g; }
+
 // log alpha = -exp(A) * softplus(a + b_alpha)
 __device__ __forceinline__ float log_decay(float a_logit, float A, float b_alpha) {
     return -expf(A) * softplus_acc(a_logit + b_alpha);

@@ -123,6 +123,9 @@ cudaError_t launch_decode_stream(const DecodeArgs &a);
 // logits [B, T, H]; the state and history advance by n_keep[b] tokens (NULL: T).
 cudaError_t launch_decode_stream(const DecodeArgs &a, int T, const int32_t *n_keep);
 
+// SM count of the current device (queried once per device, then cached).
+cudaError_t sm_count(int *out);
+
 // Kernel-launch accounting for gdn_last_call_launches(): every launcher returns
 // launched() right after its <<<...>>>, which counts the launch on this thread.
 void note_launch();

@@ -63,10 +63,12 @@ PrepArgs prep_args(const PrefillArgs &a, const TcWorkspace &w) {
 cudaError_t launch_chunk_prep(const PrefillArgs &a, const TcWorkspace &w, int c_lo, int c_hi,
                               cudaStream_t stream) {
     if (a.n_tok == 0 || c_hi <= c_lo) return cudaSuccess;
-    // blocks per (head, sequence): ~8 x 148 / H in total, at most one per chunk
+    // blocks per (head, sequence): ~8 per SM / H in total, at most one per chunk
     // of the range (the longest sequence may fill it); blocks past the end exit
     const int max_chunks = (a.n_tok + 63) / 64;
-    int split = max(1, (8 * 148) / a.H);
+    int sms = 0;
+    if (cudaError_t es = sm_count(&sms)) return es;
+    int split = max(1, (8 * sms) / a.H);
     split = min(split, min(c_hi, max_chunks) - c_lo);
     if (split <= 0) return cudaSuccess;
     dim3 grid(a.H, a.n_seq, split);

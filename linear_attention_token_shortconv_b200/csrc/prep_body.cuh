@@ -353,7 +353,7 @@ __device__ __forceinline__ bool prep_one_chunk(const Sync &sy, const PrepArgs pa
     if (tid < C) {
         float g = 0.f, be = 0.f;
         if (tid < len) {
-            g = -eA * softplus_fast(to_f32(a_raw) + ba);
+            g = clamp_log_decay(-eA * softplus_fast(to_f32(a_raw) + ba));
             be = sigmoid_fast(to_f32(b_raw));
         }
         // inclusive scan of the log decays within each warp, then across the two

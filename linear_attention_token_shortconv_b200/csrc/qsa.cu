@@ -474,7 +474,10 @@ cudaError_t launch_qsa_indexer(const QsaArgs &a, void *ws) {
     const long long items = (long long)a.B * a.n + (long long)a.B * nb;
     if (items == 0) return cudaSuccess;
     const long long want_blocks = (items + 7) / 8;
-    const int grid = (int)(want_blocks < 148LL * 16 ? want_blocks : 148LL * 16);
+    int sms = 0;
+    if ((e = sm_count(&sms)) != cudaSuccess) return e;
+    const long long cap = 16LL * sms;   // 16 blocks of 256 threads per SM
+    const int grid = (int)(want_blocks < cap ? want_blocks : cap);
     qsa_prep_kernel<<<grid, 256, 0, a.stream>>>((const bf16 *)a.q, (const bf16 *)a.k, a.w_q, a.w_k, a.B, a.n, qr, kb);
     if ((e = launched()) != cudaSuccess) return e;
     if (nb > 0) {

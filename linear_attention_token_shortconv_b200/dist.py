@@ -9,6 +9,9 @@ reduction of its duration; every rank takes them in the same order.
 from __future__ import annotations
 
 import os
+import socket
+import subprocess
+import sys
 from datetime import timedelta
 
 import torch
@@ -21,6 +24,32 @@ def env_ranks() -> tuple[int, int, int]:
     """(world size, global rank, local rank) from the launcher's environment."""
     return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
             int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def free_port() -> int:
+    """A TCP port on 127.0.0.1 that is free right now (for a rendezvous)."""
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def launch(n: int, script: str, argv: list, env: dict | None = None) -> int:
+    """Runs `python script *argv` as n ranks on this node, one process per rank,
+    under torch.distributed.run with the rendezvous on 127.0.0.1 and a free port;
+    every rank finds RANK, LOCAL_RANK, WORLD_SIZE and MASTER_* in its
+    environment.  Returns the launcher's exit code (non-zero if any rank failed)."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", f"--master-port={free_port()}", script, *argv]
+    full_env = dict(os.environ)
+    for k in ("RANK", "LOCAL_RANK", "WORLD_SIZE", "MASTER_ADDR", "MASTER_PORT"):
+        full_env.pop(k, None)
+    full_env.update(env or {})
+    return subprocess.run(cmd, env=full_env).returncode
+
+
+def group_size() -> int:
+    """World size of the joined process group (1 when no group was joined)."""
+    return dist.get_world_size() if dist.is_available() and dist.is_initialized() else 1
 
 
 def setup(backend: str = "nccl", timeout_s: float = 300.0) -> tuple[int, int, int]:

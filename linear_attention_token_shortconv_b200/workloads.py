@@ -57,6 +57,7 @@ class DecodeConfig:
     steps: int = 1000
     pool: int = 8             # distinct per-step input sets, used cyclically
     random_ring_pos: bool = False
+    long_memory: bool = False  # alpha close to 1 (A = log U[0.01, 0.1], a ~ N(-2, 1))
 
 
 def varlen_lengths(total: int = 262144, n: int = 8, lo: int = 4096, hi: int = 131072,
@@ -176,14 +177,17 @@ def make_decode_inputs(cfg: DecodeConfig, device="cpu", seed=None) -> dict:
     else:
         d["ring_pos"] = torch.zeros(B, dtype=torch.int32, device=device)
     d["conv_w"] = _normal((C, K), gen, device, std=0.5)
-    d["A"] = torch.log(_uniform((H,), gen, device, 1.0, 16.0))
+    if cfg.long_memory:
+        d["A"] = torch.log(_uniform((H,), gen, device, 0.01, 0.1))
+    else:
+        d["A"] = torch.log(_uniform((H,), gen, device, 1.0, 16.0))
     d["b_alpha"] = torch.zeros(H, device=device)
     d["norm_w"] = torch.zeros(dv, device=device)
     d["q"] = _normal((P, B, H, dk), gen, device).to(dt)
     d["k"] = _normal((P, B, H, dk), gen, device).to(dt)
     d["v"] = _normal((P, B, H, dv), gen, device).to(dt)
     d["z"] = _normal((P, B, H, dv), gen, device).to(dt)
-    d["a_logit"] = _normal((P, B, H), gen, device).to(dt)
+    d["a_logit"] = _normal((P, B, H), gen, device, mean=-2.0 if cfg.long_memory else 0.0).to(dt)
     d["b_logit"] = _normal((P, B, H), gen, device).to(dt)
     return d
 

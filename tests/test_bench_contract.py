@@ -24,6 +24,16 @@ def _run(args, env_extra=None, timeout=600):
                           capture_output=True, text=True, timeout=timeout)
 
 
+def test_gpus_flag_starts_the_ranks_itself():
+    """`bench.py --gpus 2` outside a launcher starts two ranks itself; under the
+    reference arm only rank 0 works and prints, and it reports both ranks."""
+    r = _run(["--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3"])
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    assert json.loads(lines[0])["n_gpus"] == 2
+
+
 def test_reference_arm_json_line():
     r = _run(["--impl", "reference", "--steps", "1", "--warmup", "3"])
     assert r.returncode == 0, r.stderr[-2000:]

@@ -78,6 +78,26 @@ def test_decode_multi_matches_token_by_token(cuda_device, T, keep, out_dtype):
     assert np.array_equal(to_oracle_bits(hist), h_ref)
 
 
+@pytest.mark.parametrize("T", [2, 4])
+def test_decode_multi_long_memory(cuda_device, T):
+    """alpha close to 1 (A = log U[0.01, 0.1], a ~ N(-2, 1)): every token's output
+    depends on the carried state, not only on its own write."""
+    cfg = replace(DECODE, B=12, H=4, seed=13, long_memory=True)
+    inp, multi = _multi_inputs(cfg, T)
+    n_keep = [b % (T + 1) for b in range(cfg.B)]
+    g, m = to_device(inp, cuda_device), to_device(multi, cuda_device)
+    S, hist = g["S"].clone(), g["ring"].clone()
+    nk = torch.tensor(n_keep, dtype=torch.int32, device=cuda_device)
+    out = gdn.decode_multi(m["q"], m["k"], m["v"], g["conv_w"], hist, m["a_logit"], m["b_logit"], g["A"],
+                           g["b_alpha"], m["z"], g["norm_w"], S, n_keep=nk)
+    torch.cuda.synchronize()
+    o_ref, S_ref, h_ref = _oracle(inp, T, n_keep)
+    e_o, e_s = normwise(out.cpu().numpy(), o_ref), normwise(S.cpu().numpy(), S_ref)
+    print(f"long memory T={T}: out {e_o:.1e} S {e_s:.1e}")
+    assert e_o <= TOL_BF16 and e_s <= TOL_BF16
+    assert np.array_equal(to_oracle_bits(hist), h_ref)
+
+
 def test_decode_multi_zero_keep_leaves_state_untouched(cuda_device):
     cfg = replace(DECODE, B=8, H=2, seed=12)
     inp, multi = _multi_inputs(cfg, 4)

@@ -71,3 +71,15 @@ def test_single_rank_helpers_are_local():
     rankio.barrier(1)
     assert rankio.shard_seed(7, 0) == 7 and rankio.shard_seed(7, 3) == 7 + 3 * rankio.SEED_STRIDE
     assert rankio.job_throughput(1, 1000, 2.0) == pytest.approx(5e5)
+
+
+def test_launcher_starts_one_process_per_rank(tmp_path):
+    """dist.launch (what `bench.py --gpus N` runs when no launcher started it)
+    starts N processes that join one process group with distinct ranks."""
+    probe = os.path.join(os.path.dirname(os.path.abspath(__file__)), "rank_probe.py")
+    rc = rankio.launch(WORLD, probe, [str(tmp_path)])
+    assert rc == 0
+    res = [json.load(open(tmp_path / f"rank{r}.json")) for r in range(WORLD)]
+    for r in res:
+        assert r["world"] == WORLD and r["group"] == WORLD
+        assert sorted(tuple(x) for x in r["seen"]) == [(0, 0), (1, 1)]

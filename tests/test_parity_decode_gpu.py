@@ -48,6 +48,22 @@ def test_decode_small_many_steps(cuda_device):
     print("worst", _run_steps(cfg, 20, cuda_device, TOL_BF16))
 
 
+def test_decode_small_long_memory(cuda_device):
+    """alpha close to 1: the state carries over many steps, so an error in reading
+    or writing S shows in every later step's output."""
+    cfg = replace(DECODE, B=5, H=3, pool=4, long_memory=True)
+    print("worst", _run_steps(cfg, 40, cuda_device, TOL_BF16))
+
+
+@pytest.mark.parametrize("long_memory", [False, True], ids=["short-memory", "long-memory"])
+def test_decode_trajectory_1000_steps(cuda_device, long_memory):
+    """The decode workload's 1000 consecutive steps (its 8-entry input pool used
+    cyclically, state N(0, 0.02)) on a slice of 8 sequences x 4 heads, against the
+    oracle run step by step; compared every 100 steps and at the end."""
+    cfg = replace(DECODE, B=8, H=4, long_memory=long_memory)
+    print("worst", _run_steps(cfg, cfg.steps, cuda_device, TOL_BF16, check_every=100))
+
+
 def test_decode_fp32(cuda_device):
     cfg = replace(DECODE, B=3, H=2, dk=64, dv=64, in_dtype=torch.float32, pool=3)
     print("worst", _run_steps(cfg, 12, cuda_device, TOL_F32))

@@ -3,6 +3,7 @@
 Small cases span several 64-token chunks, ragged tails, empty and one-token
 sequences; full-size workloads are checked on sampled (sequence, head) chains
 that the oracle recomputes token by token."""
+import math
 from dataclasses import replace
 
 import numpy as np
@@ -53,6 +54,25 @@ def test_bf16_output(cuda_device):
     o_ref, _ = oracle_full(inp)
     assert out.dtype == torch.bfloat16
     assert normwise(out.float().cpu().numpy(), o_ref) <= TOL_BF16 + 2.0 ** -9
+
+
+def test_overflowing_log_decay_gives_alpha_zero(cuda_device):
+    """Decay logits near the top of the bf16 range make -e^A softplus(a) overflow
+    to -inf in fp32.  The oracle (fp64) sees alpha = 0 there; the tensor-core path
+    must stay finite and agree (its log-decay is clamped where e^g is already 0)."""
+    cfg = scaled(PRETRAIN, lengths=(200, 70), H=2, s0_var=0.02)
+    inp = make_prefill_inputs(cfg, "cpu")
+    a = inp["a_logit"].float()
+    a[[5, 63, 64, 100, 150, 199, 230], 0] = 3.0e38
+    a[[0, 64, 128, 269], 1] = 3.0e38
+    inp["a_logit"] = a.to(torch.bfloat16)
+    inp["A"] = torch.full_like(inp["A"], math.log(16.0))
+    out, SF = gpu_prefill(to_device(inp, cuda_device), cfg.num_seqs)
+    o_ref, s_ref = oracle_full(inp)
+    assert torch.isfinite(out).all() and torch.isfinite(SF).all()
+    e_out, e_s = normwise(out.cpu().numpy(), o_ref), normwise(SF.cpu().numpy(), s_ref)
+    print(f"out {e_out:.2e} S_final {e_s:.2e}")
+    assert e_out <= TOL_BF16 and e_s <= TOL_BF16
 
 
 def test_empty_batch_returns_initial_state(cuda_device):
@@ -118,6 +138,9 @@ def _oracle_heads(inp, n, heads, cu):
 
 FULL = [("pretrain", PRETRAIN, [(0, [0, 15]), (3, [7])]),
         ("long", LONG, [(0, [0, 17, 31])]),
+        # alpha close to 1 over all 512 chunks: the fp32 state carries across every
+        # chunk, and its fp16 copy (the tensor-core operand) feeds every chunk's U
+        ("long-memory", replace(LONG, long_memory=True), [(0, [0, 31])]),
         ("varlen", VARLEN, None)]
 
 
