@@ -220,7 +220,7 @@ def max_over_ranks(x, world):
 def prefill_call(inp, out, S_final):
     gdn.prefill(inp["q"], inp["k"], inp["v"], inp["conv_w"], inp["a_logit"], inp["b_logit"],
                 inp["A"], inp["b_alpha"], inp["z"], inp["norm_w"], S0=inp["S0"],
-                cu_seqlens=inp["cu_seqlens"], out=out, S_final=S_final)
+                cu_seqlens=inp["cu_seqlens"], num_seqs=S_final.shape[0], out=out, S_final=S_final)
 
 
 def bench_prefill(cfg, steps, warmup, world, rank, dev):

@@ -127,6 +127,44 @@ GDN_API gdn_status_t gdn_prefill(const gdn_dims_t *dims, const void *q, const vo
 GDN_API gdn_status_t gdn_prefill_workspace_size(const gdn_dims_t *dims, size_t *bytes);
 
 /*
+ * gdn_prefill_ws -- gdn_prefill with the workspace supplied by the caller, so
+ * that the call allocates no memory at all.  Same arguments and results as
+ * gdn_prefill (the same kernels run; the results are bit-identical), plus
+ *   workspace        device buffer of at least gdn_prefill_workspace_size()
+ *                    bytes, 256-byte aligned (may be NULL when that size is 0)
+ *   workspace_bytes  its size
+ * The call reads and writes the workspace on `stream`; the caller must not use
+ * it for anything else until that work is done.  Its contents need no
+ * initialisation and are meaningless afterwards.  A workspace that is NULL or
+ * too small returns GDN_ERR_INVALID_ARG, a misaligned one GDN_ERR_ALIGNMENT,
+ * both before any launch.
+ */
+GDN_API gdn_status_t gdn_prefill_ws(const gdn_dims_t *dims, const void *q, const void *k, const void *v,
+                                    const float *conv_w, const void *a_logit, const void *b_logit,
+                                    const float *A, const float *b_alpha, const void *z,
+                                    const float *norm_w, const float *S0, const int32_t *cu_seqlens,
+                                    void *out, float *S_final, void *workspace, size_t workspace_bytes,
+                                    gdn_stream_t stream);
+
+/*
+ * gdn_prefill_conv_tail -- the ShortConv history that continues each prefilled
+ * sequence in decode: the causal depthwise convolution (slinene.github.io
+ * write-up of "On the Design of Qwen3.8-Next Architecture", 模块 A, 参数化) looks
+ * back conv_k - 1 = 3 raw tokens, and gdn_decode_step reads them from its
+ * history buffer.
+ *   q, k, v, cu_seqlens  as for gdn_prefill (raw, pre-conv projections)
+ *   conv_hist  [N_seq, 3, H(2dk + dv)] in_dtype, written: row j of sequence n is
+ *              the raw token cu[n+1] - 3 + j as [q heads | k heads | v heads],
+ *              or zeros where that token lies before the sequence's start.
+ * With this history and S_final of gdn_prefill as the state, gdn_decode_step on
+ * the following tokens continues every sequence exactly as a longer prefill
+ * would.  One kernel on `stream`; no workspace.
+ */
+GDN_API gdn_status_t gdn_prefill_conv_tail(const gdn_dims_t *dims, const void *q, const void *k,
+                                           const void *v, const int32_t *cu_seqlens, void *conv_hist,
+                                           gdn_stream_t stream);
+
+/*
  * gdn_prefill_backward -- gradients of L = <d_out, out> + <d_S_final, S_final>
  * for the gdn_prefill call with the same arguments, with respect to every
  * input: the reverse-mode derivative of the forward the two web write-ups

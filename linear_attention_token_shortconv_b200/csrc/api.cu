@@ -156,8 +156,9 @@ cudaError_t slot_launch(int *slot, cudaStream_t s, F &&launch) {
     return e;
 }
 
-// The prefill after validation: workspace from the pool, then the kernels.
-cudaError_t prefill_dispatch(const gdn::PrefillArgs &a) {
+// The prefill after validation: workspace from the pool (ext_ws NULL) or the
+// caller's buffer of at least workspace_bytes(), then the kernels.
+cudaError_t prefill_run(const gdn::PrefillArgs &a, char *ext_ws) {
     gdn_dims_t dd;
     dd.num_seqs = a.n_seq;
     dd.total_tokens = a.n_tok;
@@ -170,8 +171,9 @@ cudaError_t prefill_dispatch(const gdn::PrefillArgs &a) {
     const gdn_dims_t *dims = &dd;
     const size_t nt = (size_t)a.n_tok * a.H;
     const size_t ws_bytes = workspace_bytes(dims);
-    char *ws = nullptr;
-    if (ws_bytes) {
+    char *ws = ext_ws;
+    const bool own_ws = ext_ws == nullptr && ws_bytes > 0;
+    if (own_ws) {
         cudaMemPool_t pool;
         cudaError_t ep = get_pool(&pool);
         if (ep != cudaSuccess) return ep;
@@ -249,12 +251,14 @@ cudaError_t prefill_dispatch(const gdn::PrefillArgs &a) {
             e = slot_launch(&slot, a.stream, [&] { return gdn::launch_recurrent(a, qn, kn, vn); });
         if (e == cudaSuccess) e = record(g_ev_end, a.stream);
     }
-    if (ws) {
+    if (own_ws) {
         cudaError_t ef = cudaFreeAsync(ws, a.stream);
         if (e == cudaSuccess) e = ef;
     }
     return e;
 }
+
+cudaError_t prefill_dispatch(const gdn::PrefillArgs &a) { return prefill_run(a, nullptr); }
 
 }  // namespace
 
@@ -334,12 +338,15 @@ gdn_status_t gdn_prefill_workspace_size(const gdn_dims_t *dims, size_t *bytes) {
     return GDN_OK;
 }
 
-gdn_status_t gdn_prefill(const gdn_dims_t *dims, const void *q, const void *k, const void *v,
-                         const float *conv_w, const void *a_logit, const void *b_logit,
-                         const float *A, const float *b_alpha, const void *z,
-                         const float *norm_w, const float *S0, const int32_t *cu_seqlens,
-                         void *out, float *S_final, gdn_stream_t stream) {
-    tl_launches = 0;
+}  // extern "C"
+
+namespace {
+// Argument checks of gdn_prefill and gdn_prefill_ws; fills *a on success.
+gdn_status_t prefill_args(const gdn_dims_t *dims, const void *q, const void *k, const void *v,
+                          const float *conv_w, const void *a_logit, const void *b_logit,
+                          const float *A, const float *b_alpha, const void *z,
+                          const float *norm_w, const float *S0, const int32_t *cu_seqlens,
+                          void *out, float *S_final, gdn_stream_t stream, gdn::PrefillArgs *ap) {
     gdn_status_t st = check_dims(dims, false);
     if (st != GDN_OK) return st;
     if (!cu_seqlens && dims->total_tokens % dims->num_seqs != 0) return GDN_ERR_INVALID_ARG;
@@ -368,7 +375,7 @@ gdn_status_t gdn_prefill(const gdn_dims_t *dims, const void *q, const void *k, c
         if (p && !aligned16(p)) return GDN_ERR_ALIGNMENT;
     if (cu_seqlens && !aligned_to(cu_seqlens, 4)) return GDN_ERR_ALIGNMENT;
 
-    gdn::PrefillArgs a;
+    gdn::PrefillArgs &a = *ap;
     a.n_seq = dims->num_seqs;
     a.n_tok = dims->total_tokens;
     a.H = dims->H;
@@ -382,8 +389,40 @@ gdn_status_t gdn_prefill(const gdn_dims_t *dims, const void *q, const void *k, c
     a.out = out;
     a.S_final = S_final;
     a.stream = reinterpret_cast<cudaStream_t>(stream);
+    return GDN_OK;
+}
+}  // namespace
 
+extern "C" {
+
+gdn_status_t gdn_prefill(const gdn_dims_t *dims, const void *q, const void *k, const void *v,
+                         const float *conv_w, const void *a_logit, const void *b_logit,
+                         const float *A, const float *b_alpha, const void *z,
+                         const float *norm_w, const float *S0, const int32_t *cu_seqlens,
+                         void *out, float *S_final, gdn_stream_t stream) {
+    tl_launches = 0;
+    gdn::PrefillArgs a;
+    const gdn_status_t st = prefill_args(dims, q, k, v, conv_w, a_logit, b_logit, A, b_alpha, z, norm_w, S0,
+                                         cu_seqlens, out, S_final, stream, &a);
+    if (st != GDN_OK) return st;
     return prefill_dispatch(a) == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status_t gdn_prefill_ws(const gdn_dims_t *dims, const void *q, const void *k, const void *v,
+                            const float *conv_w, const void *a_logit, const void *b_logit,
+                            const float *A, const float *b_alpha, const void *z,
+                            const float *norm_w, const float *S0, const int32_t *cu_seqlens,
+                            void *out, float *S_final, void *workspace, size_t workspace_bytes_given,
+                            gdn_stream_t stream) {
+    tl_launches = 0;
+    gdn::PrefillArgs a;
+    const gdn_status_t st = prefill_args(dims, q, k, v, conv_w, a_logit, b_logit, A, b_alpha, z, norm_w, S0,
+                                         cu_seqlens, out, S_final, stream, &a);
+    if (st != GDN_OK) return st;
+    const size_t need = workspace_bytes(dims);
+    if (need > 0 && (!workspace || workspace_bytes_given < need)) return GDN_ERR_INVALID_ARG;
+    if (workspace && !aligned_to(workspace, 256)) return GDN_ERR_ALIGNMENT;
+    return prefill_run(a, static_cast<char *>(workspace)) == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
 gdn_status_t gdn_prefill_backward_workspace_size(const gdn_dims_t *dims, size_t *bytes) {

@@ -94,7 +94,7 @@ decode_stream_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
     constexpr int NSTAGE = Lo::NSTAGE, STAGE = Lo::STAGE, OFF_TOK = Lo::OFF_TOK, OFF_HIST = Lo::OFF_HIST;
     const int T = TMAX == 1 ? 1 : T_rt;     // tokens per sequence in this call (<= TMAX)
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    uint8_t *sm = umma::align_smem<128>(smem_raw);
     uint8_t *misc = sm + Lo::OFF_MISC;
     uint64_t *full = reinterpret_cast<uint64_t *>(misc);                          // [NSTAGE]
     volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 32);

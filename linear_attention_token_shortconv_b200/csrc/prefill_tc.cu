@@ -27,7 +27,7 @@ chunk_prep_kernel(const PrepArgs pa, const int32_t *__restrict__ cu_seqlens, int
                   int n_tok, int c_lo, int c_hi) {
     using namespace prep;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sm = umma::align_smem<1024>(smem_raw);
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + OFF_MISC + 768);
     uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + OFF_MISC + 784);
     const int tid = threadIdx.x, warp = tid >> 5;
@@ -44,8 +44,12 @@ chunk_prep_kernel(const PrepArgs pa, const int32_t *__restrict__ cu_seqlens, int
     __syncthreads();
     const uint32_t tbase = *tslot;
     uint32_t phase = 0;
-    for (int c = c_lo + blockIdx.z; c < c_end; c += gridDim.z)
+    for (int c = c_lo + blockIdx.z; c < c_end; c += gridDim.z) {
+        // this block's next chunk: its raw rows into L2 while this one is processed
+        if (c + (int)gridDim.z < c_end)
+            prefetch_chunk_rows<DV>(pa.q, pa.k, pa.v, pa.H, h, s_begin + (c + gridDim.z) * C, s_end, tid);
         if (!prep_one_chunk<DV>(PrepBlockSync{}, pa, sm, tbase, bar, phase, tid, h, s_begin, s_end, c)) break;
+    }
     umma::tc_fence_before();
     __syncthreads();
     if (warp == 0) umma::tmem_dealloc(tbase, TMEM_COLS);
@@ -111,13 +115,13 @@ cudaError_t prep_error_word(unsigned *v, bool clear, cudaStream_t s) {
 
 
 template <int DV, typename Tout>
-__global__ void __launch_bounds__(4 * DV, 1)
+__global__ void __launch_bounds__(chain_threads<DV>(), 1)
 chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const float *__restrict__ decay,
                    const float *__restrict__ norm_w, const float *state_in,
                    const int32_t *__restrict__ cu_seqlens, int n_seq, int n_tok, int H, int c_lo,
-                   int c_hi, Tout *__restrict__ out, float *state_out) {
+                   int c_hi, const bf16 *__restrict__ z, Tout *__restrict__ out, float *state_out) {
     chain_body<DV, Tout>(maps, decay, norm_w, state_in, cu_seqlens, n_seq, n_tok, H, blockIdx.x, blockIdx.y,
-                         c_lo, c_hi, out, state_out, nullptr);
+                         c_lo, c_hi, z, out, state_out, nullptr);
 }
 
 cudaError_t launch_chunk_chain(const PrefillArgs &a, const TcWorkspace &w, int c_lo, int c_hi,
@@ -132,8 +136,6 @@ cudaError_t launch_chunk_chain(const PrefillArgs &a, const TcWorkspace &w, int c
         if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.aqk), w.Aqk, false, 64, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
         if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.up), w.Up, false, a.dv, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
         if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.z), a.z, true, a.dv, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
-        if (a.out_bf16 &&
-            (e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.out), a.out, true, a.dv, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
     }
     dim3 grid(a.H, a.n_seq);
     cudaError_t e;
@@ -141,9 +143,9 @@ cudaError_t launch_chunk_chain(const PrefillArgs &a, const TcWorkspace &w, int c
     e = cudaFuncSetAttribute(chunk_chain_kernel<DV_, TOUT>,                                       \
                              cudaFuncAttributeMaxDynamicSharedMemorySize, chain::SMEM);            \
     if (e != cudaSuccess) return e;                                                               \
-    chunk_chain_kernel<DV_, TOUT><<<grid, 4 * DV_, chain::SMEM, stream>>>(                        \
+    chunk_chain_kernel<DV_, TOUT><<<grid, chain_threads<DV_>(), chain::SMEM, stream>>>(           \
         m, w.decay, a.norm_w, state_in, a.cu_seqlens, a.n_seq, a.n_tok, a.H, c_lo, c_hi,        \
-        (TOUT *)a.out, state_out)
+        (const bf16 *)a.z, (TOUT *)a.out, state_out)
     if (a.dv == 128) {
         if (a.out_bf16) { GDN_CHAIN(128, bf16); } else { GDN_CHAIN(128, float); }
     } else {
@@ -191,17 +193,20 @@ cudaError_t chain_error_word(unsigned *v, bool clear, cudaStream_t s) {
 // chain CTA, so every flag gets set; every wait is bounded all the same.
 namespace fused {
 constexpr int NT = 512;
-constexpr int PREP_REGION = 102400;   // one prep worker's shared memory (1 KB aligned)
+static_assert(chain_threads<128>() == NT, "chain role uses the whole CTA");
+constexpr int PREP_REGION = 104448;   // one prep worker's shared memory (1 KB aligned)
 constexpr int SMEM = chain::SMEM > 2 * PREP_REGION + 1024 ? chain::SMEM : 2 * PREP_REGION + 1024;
-static_assert(prep::OFF_MISC + 1024 + 3 * 256 * 4 <= PREP_REGION, "prep worker region");
+static_assert(prep::OFF_MISC + prep::MISC_BYTES <= PREP_REGION, "prep worker region");
 }  // namespace fused
 
 struct FusedParams {
     ChainMaps maps;
+    CUtensorMap raw_q, raw_k, raw_v;   // L2 prefetch of a chunk's raw rows (box: 67 rows of one head)
     PrepArgs pa;
     const float *norm_w, *S0;
     float *S_final;
     const int32_t *cu_seqlens;
+    const bf16 *z;
     void *out;
     int *ready;        // [n_items][max_chunks], zero at launch
     int *next_task;    // zero at launch
@@ -214,14 +219,14 @@ __global__ void __launch_bounds__(fused::NT, 1) prefill_fused_kernel(const __gri
     if ((int)blockIdx.x < P.n_chain) {   // chain role: item blockIdx.x
         const int item = blockIdx.x, n = item / P.H, h = item % P.H;
         chain_body<128, Tout>(P.maps, P.pa.decay, P.norm_w, P.S0, P.cu_seqlens, P.n_seq, P.n_tok, P.H, h, n, 0,
-                              P.max_chunks + 1, reinterpret_cast<Tout *>(P.out), P.S_final,
+                              P.max_chunks + 1, P.z, reinterpret_cast<Tout *>(P.out), P.S_final,
                               P.ready + (size_t)item * P.max_chunks);
         return;
     }
     // prep role: two workers
     using namespace prep;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sm = umma::align_smem<1024>(smem_raw);
     const int tid = threadIdx.x, half = tid >> 8, wtid = tid & 255;
     uint8_t *wsm = sm + half * fused::PREP_REGION;
     uint64_t *bar = reinterpret_cast<uint64_t *>(wsm + OFF_MISC + 768);
@@ -241,12 +246,29 @@ __global__ void __launch_bounds__(fused::NT, 1) prefill_fused_kernel(const __gri
     uint32_t phase = 0;
     // the next task index is fetched one task ahead (slot 1) so the atomic's round
     // trip overlaps a chunk; a chunk's ready flag is published during the next one
-    if (wtid == 0) task_slot[0] = atomicAdd(P.next_task, 1);
+    // raw q, k, v rows of a task's chunk (and the three rows before it) into L2
+    auto prefetch_raw = [&](int t) {
+        if (t >= n_tasks) return;
+        const int it = t % n_items, ns = it / P.H, hs = it % P.H;
+        const int sb = P.cu_seqlens ? __ldg(P.cu_seqlens + ns) : ns * (P.n_tok / P.n_seq);
+        const int row = sb + (t / n_items) * C - 3;
+        umma::tma_prefetch_l2_3d(&P.raw_q, 0, hs, row);
+        umma::tma_prefetch_l2_3d(&P.raw_k, 0, hs, row);
+        umma::tma_prefetch_l2_3d(&P.raw_v, 0, hs, row);
+    };
+    if (wtid == 0) {
+        task_slot[0] = atomicAdd(P.next_task, 1);
+        prefetch_raw(task_slot[0]);
+    }
     sy.sync();
     int task = task_slot[0];
     int *pending = nullptr;   // ready flag of the last chunk this worker wrote
     while (task < n_tasks) {
-        if (wtid == 0) task_slot[1] = atomicAdd(P.next_task, 1);
+        if (wtid == 0) {
+            const int nt = atomicAdd(P.next_task, 1);
+            task_slot[1] = nt;
+            prefetch_raw(nt);
+        }
         const int c = task / n_items, item = task % n_items;
         const int n = item / P.H, h = item % P.H;
         int s_begin, s_end;
@@ -290,13 +312,15 @@ cudaError_t launch_prefill_fused(const PrefillArgs &a, const TcWorkspace &w, int
     if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&P.maps.aqk), w.Aqk, false, 64, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
     if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&P.maps.up), w.Up, false, 128, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
     if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&P.maps.z), a.z, true, 128, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
-    if (a.out_bf16 &&
-        (e = make_tma_3d(reinterpret_cast<TmaMap *>(&P.maps.out), a.out, true, 128, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
+    if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&P.raw_q), a.q, true, 128, a.H, a.n_tok, 128, 67, false)) != cudaSuccess) return e;
+    if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&P.raw_k), a.k, true, 128, a.H, a.n_tok, 128, 67, false)) != cudaSuccess) return e;
+    if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&P.raw_v), a.v, true, 128, a.H, a.n_tok, 128, 67, false)) != cudaSuccess) return e;
     P.pa = prep_args(a, w);
     P.norm_w = a.norm_w;
     P.S0 = a.S0;
     P.S_final = a.S_final;
     P.cu_seqlens = a.cu_seqlens;
+    P.z = (const bf16 *)a.z;
     P.out = a.out;
     P.n_seq = a.n_seq;
     P.n_tok = a.n_tok;

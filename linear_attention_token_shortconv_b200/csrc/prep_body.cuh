@@ -22,11 +22,12 @@
 // q.k and k.k products therefore use a two-term fp16 split of the fp32 q and k
 // (x = hi + lo): [Qh;Kh]Kh^T + [Qh;Kh]Kl^T + [Ql;Kl]Kh^T, fp32 accumulation.
 //
-// Per chunk: prelude in registers -> fp16 hi/lo tiles in smem; the split
-// [Q;K]K^T on tcgen05 (M=128, N=64) -> TMEM, with Qt and Kt written out while
-// it runs; Aqk and L from TMEM; T by blocked forward substitution in fp32 over
-// all 256 threads; [T diag(beta e^G); T diag(beta)] times K and V on tcgen05 ->
-// TMEM; results to global memory in fp16.
+// Per chunk: the gates and their in-chunk cumulative log decays first; then the
+// prelude in registers -> fp16 hi/lo tiles in smem, with Qt and Kt written to
+// global memory straight from it; the split [Q;K]K^T on tcgen05 (M=128, N=64) ->
+// TMEM; Aqk and L from TMEM; T = (I + L)^-1 by 16 x 16 blocks (warp-level tensor
+// cores, tf32 with a two-term split); [T diag(beta e^G); T diag(beta)] times K and
+// V on tcgen05 -> TMEM; results to global memory in fp16.
 //
 // Device code only: the kernels that run it and the device error word it raises
 // (g_prep_err, defined before this header is included) live in prefill_tc.cu.
@@ -78,27 +79,53 @@ constexpr int OFF_HI = 0;      // [Qh;Kh] K-major, 2 k-blocks x 16 KB
 constexpr int OFF_LO = 32768;  // [Ql;Kl] K-major, 2 k-blocks x 16 KB; later L and T fp32 [64][64]
 constexpr int OFF_V = 65536;   // V MN-major, DV/64 mn-blocks x 8 KB
 constexpr int OFF_T = 81920;   // [T'; T''] K-major, 1 k-block x 16 KB
-constexpr int OFF_MISC = 98304;  // G, beta, barriers [0, 1024); block products [1024, 4096)
-constexpr int SMEM = OFF_MISC + 4096 + 1024;
+constexpr int OFF_MISC = 98304;  // G, beta, barriers [0, 1024); block products [1024, 4096);
+                                 // per-token factors e^G, e^{G_C - G}, beta e^G [4096, 4864)
+constexpr int MISC_BYTES = 4864;
+constexpr int SMEM = OFF_MISC + MISC_BYTES + 1024;
 constexpr uint32_t TMEM_COLS = 256;
 }  // namespace prep
+
+// 2^x on the special-function unit (ex2.approx: about 2 ulp; inputs here are at
+// most 60, and underflow to 0 is what the callers want)
+__device__ __forceinline__ float ex2_fast(float x) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+// Ask L2 to fetch the raw q, k and v rows of chunk c of head h (and the three rows
+// before it): one 256-byte row per thread for the first 3 * (C + 3) threads.
+template <int DV>
+__device__ __forceinline__ void prefetch_chunk_rows(const bf16 *q, const bf16 *k, const bf16 *v, int H, int h,
+                                                    int t0, int t_end, int tid) {
+    constexpr int R = 64 + 3;
+    if (tid >= 3 * R) return;
+    const int which = tid / R, t = t0 - 3 + tid % R;
+    if (t < 0 || t >= t_end) return;
+    const bf16 *row = which == 0 ? q + ((size_t)t * H + h) * 128
+                    : which == 1 ? k + ((size_t)t * H + h) * 128 : v + ((size_t)t * H + h) * DV;
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(row), "r"(which == 2 ? DV * 2 : 256) : "memory");
+}
 
 // Conv + SiLU of 8 channels (4 pairs) for tokens [i0, i0 + N) of a chunk: all
 // N + 3 raw rows (zero before the sequence start and past its end) are loaded
 // first, then a sliding window of converted rows produces y[N][4] (pairs).
 template <int N>
-__device__ __forceinline__ void conv_silu(const bf16 *src, size_t row_stride, int col,
-                                          const float2 (&w)[4][4], int t0, int s_begin, int i0,
-                                          int len, float2 (&y)[N][4]) {
-    uint4 raw[N + 3];
+__device__ __forceinline__ void conv_load(const bf16 *src, size_t row_stride, int col, int t0, int s_begin, int i0,
+                                          int len, uint4 (&raw)[N + 3]) {
+    const bf16 *base = src + (size_t)(t0 + i0 - 3) * row_stride + col;
 #pragma unroll
     for (int r = 0; r < N + 3; ++r) {
         const int i = i0 + r - 3;            // chunk-relative row
-        const int t = t0 + i;
-        const bool ok = (i < len) && (t >= s_begin);
-        raw[r] = ok ? __ldg(reinterpret_cast<const uint4 *>(src + (size_t)t * row_stride + col))
-                    : make_uint4(0, 0, 0, 0);
+        const bool ok = (i < len) && (t0 + i >= s_begin);
+        raw[r] = ok ? __ldg(reinterpret_cast<const uint4 *>(base + (size_t)r * row_stride)) : make_uint4(0, 0, 0, 0);
     }
+}
+
+template <int N>
+__device__ __forceinline__ void conv_silu(const uint4 (&raw)[N + 3], const float2 (&w)[4][4], int i0, int len,
+                                          float2 (&y)[N][4]) {
     auto cvt = [](uint4 u, float2 (&x)[4]) {
         x[0] = make_float2(bf16lo(u.x), bf16hi(u.x));
         x[1] = make_float2(bf16lo(u.y), bf16hi(u.y));
@@ -121,10 +148,12 @@ __device__ __forceinline__ void conv_silu(const bf16 *src, size_t row_stride, in
             a = ffma2(w[p][1], h1[p], a);
             a = ffma2(w[p][2], h2[p], a);
             a = ffma2(w[p][3], x[p], a);
-            // silu(a) = a / (1 + 2^(-a log2 e))
+            // silu(a) = a / (1 + 2^(-a log2 e)); the pair shares one reciprocal,
+            // 1 / (d.x d.y), with the exponents clamped to 60 so the product stays finite
             const float2 e = fmul2(a, nl2e);
-            const float2 d = fadd2(one, make_float2(exp2f(e.x), exp2f(e.y)));
-            y[ii][p] = make_float2(__fdividef(a.x, d.x), __fdividef(a.y, d.y));
+            const float2 d = fadd2(one, make_float2(ex2_fast(fminf(e.x, 60.f)), ex2_fast(fminf(e.y, 60.f))));
+            const float r = __fdividef(1.0f, d.x * d.y);
+            y[ii][p] = fmul2(fmul2(a, make_float2(d.y, d.x)), make_float2(r, r));
             h0[p] = h1[p]; h1[p] = h2[p]; h2[p] = x[p];
         }
         if (i0 + ii >= len) {
@@ -144,86 +173,137 @@ __device__ __forceinline__ void load_conv_w(const float *conv_w, int chan, float
     }
 }
 
-// acc(r, c) += sum_k A[ar + r][ac + k] * B[br + k][bc + c] over a 16 x 16 block
-// product, A and B row-major fp32 [64][64] in shared memory.
-__device__ __forceinline__ float blk16(const float *A, int ar, int ac, const float *B, int br, int bc,
-                                       int r, int c, float acc) {
-    const float4 *a = reinterpret_cast<const float4 *>(A + (ar + r) * 64 + ac);
-#pragma unroll
-    for (int k4 = 0; k4 < 4; ++k4) {
-        const float4 av = a[k4];
-        acc = fmaf(av.x, B[(br + 4 * k4 + 0) * 64 + bc + c], acc);
-        acc = fmaf(av.y, B[(br + 4 * k4 + 1) * 64 + bc + c], acc);
-        acc = fmaf(av.z, B[(br + 4 * k4 + 2) * 64 + bc + c], acc);
-        acc = fmaf(av.w, B[(br + 4 * k4 + 3) * 64 + bc + c], acc);
-    }
-    return acc;
+// ---- T = (I + L)^-1 for the strictly lower triangular 64 x 64 L of a chunk.
+//
+// L and T are kept as their ten 16 x 16 blocks on or below the diagonal
+// ("block-compact": block (bi, bj), bj <= bi, at index bi (bi + 1) / 2 + bj, rows
+// of 20 floats so that the fragment loads below are free of bank conflicts).
+// Diagonal blocks D_b = (I + L_bb)^-1 by forward substitution; then the 2 x 2
+// block recursion on 32 x 32 halves,
+//   T_10 = -D_1 L_10 D_0,  T_32 = -D_3 L_32 D_2,
+//   X_a0 = L_{2+a,0} D_0 + L_{2+a,1} T_10,  X_a1 = L_{2+a,1} D_1   (a = 0, 1),
+//   T_2b = -D_2 X_0b,  T_3b = -(T_32 X_0b + D_3 X_1b)               (b = 0, 1),
+// whose 16 x 16 x 16 block products run on the warp-level tensor-core MMA
+// (m16n8k8, tf32) with each operand split into two tf32 terms, x = hi + lo, and
+// the three products hi*hi + hi*lo + lo*hi accumulated in fp32: about fp32
+// accuracy, as the solve needs (T multiplies every row of W and U').  The
+// products are far too small for tcgen05 (whose M is at least 64).
+namespace tsolve {
+constexpr int BS = 20;                 // row stride of a block (floats)
+constexpr int BLK = 16 * BS;           // floats per block
+__device__ __forceinline__ int bidx(int bi, int bj) { return bi * (bi + 1) / 2 + bj; }
+
+__device__ __forceinline__ uint32_t tf32_hi(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ void split(float x, uint32_t &hi, uint32_t &lo) {
+    hi = tf32_hi(x);
+    lo = tf32_hi(x - __uint_as_float(hi));
+}
+__device__ __forceinline__ void mma_tf32(float (&c)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%0,%1,%2,%3};"
+                 : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-// T = (I + L)^-1 for a strictly lower triangular 64 x 64 L, by 16 x 16 blocks:
-// diagonal blocks by forward substitution, then block row-diagonals
-//   T_{b+d,b} = -D_{b+d} sum_{j=b}^{b+d-1} L_{b+d,j} T_{j,b},  D_b = (I + L_bb)^-1.
-// NT threads synchronised by `sy` (the worker); X is a [3][16][16] scratch.  Only
-// the block-lower part of T is written.
-template <int NT, class Sync>
-__device__ __forceinline__ void solve_unit_lower(const Sync &sy, const float *L, float *T, float *X, int tid) {
-    if (tid < 64) {   // diagonal blocks: thread (b, c) owns column c of D_b
-        const int b = tid >> 4, cc = tid & 15, o = 16 * b;
+// c += A B[:, 8 nt .. 8 nt + 8): A a 16 x 16 block (row stride BS), B a 16 x 16
+// block (row stride bs) of which the n-tile nt is used.  Lane (g, t) = (lane / 4,
+// lane % 4) holds c[0..3] = C(g, 2t), C(g, 2t + 1), C(g + 8, 2t), C(g + 8, 2t + 1).
+__device__ __forceinline__ void prod(float (&c)[4], const float *A, const float *B, int bs, int nt, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+        uint32_t ah[4], al[4], bh[2], bl[2];
+        split(A[g * BS + 8 * ks + t], ah[0], al[0]);
+        split(A[(g + 8) * BS + 8 * ks + t], ah[1], al[1]);
+        split(A[g * BS + 8 * ks + t + 4], ah[2], al[2]);
+        split(A[(g + 8) * BS + 8 * ks + t + 4], ah[3], al[3]);
+        split(B[(8 * ks + t) * bs + 8 * nt + g], bh[0], bl[0]);
+        split(B[(8 * ks + t + 4) * bs + 8 * nt + g], bh[1], bl[1]);
+        mma_tf32(c, al, bh);
+        mma_tf32(c, ah, bl);
+        mma_tf32(c, ah, bh);
+    }
+}
+
+// Store -c (an n-tile of a 16 x 16 result) into a block of row stride bs.
+__device__ __forceinline__ void store_neg(float *B, int bs, int nt, const float (&c)[4], int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    *reinterpret_cast<float2 *>(B + g * bs + 8 * nt + 2 * t) = make_float2(-c[0], -c[1]);
+    *reinterpret_cast<float2 *>(B + (g + 8) * bs + 8 * nt + 2 * t) = make_float2(-c[2], -c[3]);
+}
+__device__ __forceinline__ void store_pos(float *B, int bs, int nt, const float (&c)[4], int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    *reinterpret_cast<float2 *>(B + g * bs + 8 * nt + 2 * t) = make_float2(c[0], c[1]);
+    *reinterpret_cast<float2 *>(B + (g + 8) * bs + 8 * nt + 2 * t) = make_float2(c[2], c[3]);
+}
+}  // namespace tsolve
+
+// T = (I + L)^-1 (block-compact L and T, see above) by 256 threads = 8 warps
+// synchronised by `sy`; `scratch` holds 4 blocks plus 4 warp tiles of 16 x 8.
+template <class Sync>
+__device__ __forceinline__ void solve_unit_lower(const Sync &sy, const float *L, float *T, float *scratch, int tid) {
+    using namespace tsolve;
+    const int warp = tid >> 5, lane = tid & 31;
+    if (tid < 64) {   // diagonal blocks: thread (b, cc) owns column cc of D_b
+        const int b = tid >> 4, cc = tid & 15;
+        const float *Lb = L + bidx(b, b) * BLK;
+        float *Tb = T + bidx(b, b) * BLK;
         float x[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
             float acc = (r == cc) ? 1.f : 0.f;
 #pragma unroll
-            for (int j = 0; j < r; ++j) acc = fmaf(-L[(o + r) * 64 + o + j], x[j], acc);
+            for (int j = 0; j < r; ++j) acc = fmaf(-Lb[r * BS + j], x[j], acc);
             x[r] = acc;
         }
 #pragma unroll
-        for (int r = 0; r < 16; ++r) T[(o + r) * 64 + o + cc] = x[r];
+        for (int r = 0; r < 16; ++r) Tb[r * BS + cc] = x[r];
     }
     sy.sync();
-    // d = 1: X_b = L_{b+1,b} D_b, then T_{b+1,b} = -D_{b+1} X_b   (b = 0, 1, 2)
-    for (int e = tid; e < 3 * 256; e += NT) {
-        const int b = e >> 8, r = (e >> 4) & 15, cc = e & 15;
-        X[e] = blk16(L, 16 * (b + 1), 16 * b, T, 16 * b, 16 * b, r, cc, 0.f);
+    float *X = scratch;                     // X_ab at X + (2a + b) * BLK
+    float *W8 = scratch + 4 * BLK;          // warp tiles 16 x 8 for the first level
+    if (warp < 4) {
+        // T_10 (warps 0, 1) and T_32 (warps 2, 3), n-tile warp & 1
+        const int bi = warp < 2 ? 1 : 3, bj = bi - 1, nt = warp & 1;
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        prod(c, L + bidx(bi, bj) * BLK, T + bidx(bj, bj) * BLK, BS, nt, lane);
+        float *w8 = W8 + warp * 128;
+        // the n-tile as a 16 x 8 B operand (columns 0..7 of a row stride 8)
+        const int g = lane >> 2, t = lane & 3;
+        *reinterpret_cast<float2 *>(w8 + g * 8 + 2 * t) = make_float2(c[0], c[1]);
+        *reinterpret_cast<float2 *>(w8 + (g + 8) * 8 + 2 * t) = make_float2(c[2], c[3]);
+        __syncwarp();
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+        prod(d, T + bidx(bi, bi) * BLK, w8, 8, 0, lane);
+        store_neg(T + bidx(bi, bj) * BLK, BS, nt, d, lane);
     }
     sy.sync();
-    for (int e = tid; e < 3 * 256; e += NT) {
-        const int b = e >> 8, r = (e >> 4) & 15, cc = e & 15;
-        float acc = 0.f;
-#pragma unroll
-        for (int k = 0; k < 16; ++k) acc = fmaf(T[(16 * (b + 1) + r) * 64 + 16 * (b + 1) + k], X[(b << 8) + k * 16 + cc], acc);
-        T[(16 * (b + 1) + r) * 64 + 16 * b + cc] = -acc;
+    {   // X_ab, n-tile: warp = (a, b, nt)
+        const int a = warp >> 2, b = (warp >> 1) & 1, nt = warp & 1;
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        if (b == 0) {
+            prod(c, L + bidx(2 + a, 0) * BLK, T + bidx(0, 0) * BLK, BS, nt, lane);
+            prod(c, L + bidx(2 + a, 1) * BLK, T + bidx(1, 0) * BLK, BS, nt, lane);
+        } else {
+            prod(c, L + bidx(2 + a, 1) * BLK, T + bidx(1, 1) * BLK, BS, nt, lane);
+        }
+        store_pos(X + (2 * a + b) * BLK, BS, nt, c, lane);
     }
     sy.sync();
-    // d = 2: X_b = L_{b+2,b} D_b + L_{b+2,b+1} T_{b+1,b}, then T_{b+2,b} = -D_{b+2} X_b   (b = 0, 1)
-    for (int e = tid; e < 2 * 256; e += NT) {
-        const int b = e >> 8, r = (e >> 4) & 15, cc = e & 15;
-        float acc = blk16(L, 16 * (b + 2), 16 * b, T, 16 * b, 16 * b, r, cc, 0.f);
-        X[e] = blk16(L, 16 * (b + 2), 16 * (b + 1), T, 16 * (b + 1), 16 * b, r, cc, acc);
-    }
-    sy.sync();
-    for (int e = tid; e < 2 * 256; e += NT) {
-        const int b = e >> 8, r = (e >> 4) & 15, cc = e & 15;
-        float acc = 0.f;
-#pragma unroll
-        for (int k = 0; k < 16; ++k) acc = fmaf(T[(16 * (b + 2) + r) * 64 + 16 * (b + 2) + k], X[(b << 8) + k * 16 + cc], acc);
-        T[(16 * (b + 2) + r) * 64 + 16 * b + cc] = -acc;
-    }
-    sy.sync();
-    // d = 3: X = L_30 D_0 + L_31 T_10 + L_32 T_20, then T_30 = -D_3 X
-    for (int e = tid; e < 256; e += NT) {
-        const int r = e >> 4, cc = e & 15;
-        float acc = blk16(L, 48, 0, T, 0, 0, r, cc, 0.f);
-        acc = blk16(L, 48, 16, T, 16, 0, r, cc, acc);
-        X[e] = blk16(L, 48, 32, T, 32, 0, r, cc, acc);
-    }
-    sy.sync();
-    for (int e = tid; e < 256; e += NT) {
-        const int r = e >> 4, cc = e & 15;
-        float acc = 0.f;
-#pragma unroll
-        for (int k = 0; k < 16; ++k) acc = fmaf(T[(48 + r) * 64 + 48 + k], X[k * 16 + cc], acc);
-        T[(48 + r) * 64 + cc] = -acc;
+    {   // T_{2+a, b}, n-tile: warp = (a, b, nt)
+        const int a = warp >> 2, b = (warp >> 1) & 1, nt = warp & 1;
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        if (a == 0) {
+            prod(c, T + bidx(2, 2) * BLK, X + b * BLK, BS, nt, lane);
+        } else {
+            prod(c, T + bidx(3, 2) * BLK, X + b * BLK, BS, nt, lane);
+            prod(c, T + bidx(3, 3) * BLK, X + (2 + b) * BLK, BS, nt, lane);
+        }
+        store_neg(T + bidx(2 + a, b) * BLK, BS, nt, c, lane);
     }
     sy.sync();
 }
@@ -258,12 +338,17 @@ __device__ __forceinline__ bool prep_one_chunk(const Sync &sy, const PrepArgs pa
     __half *Qt = pa.Qt, *Kt = pa.Kt, *Wn = pa.Wn, *Up = pa.Up, *Aqk = pa.Aqk;
     float *decay = pa.decay;
     uint8_t *sHI = sm + OFF_HI, *sLO = sm + OFF_LO, *sV = sm + OFF_V, *sT = sm + OFF_T;
-    float *sL = reinterpret_cast<float *>(sm + OFF_LO);          // aliases [Ql;Kl] after the q.k MMA
-    float *sTf = sL + 64 * 64;                                   // fp32 T, same region
-    float *sX = reinterpret_cast<float *>(sm + OFF_MISC + 1024); // [3][16][16]
+    // L and T block-compact fp32 (10 blocks of 16 x 20 each) alias [Ql;Kl] after the
+    // q.k MMA; the solve's scratch uses the [T'; T''] tile's region, written after it
+    float *sL = reinterpret_cast<float *>(sm + OFF_LO);
+    float *sTf = sL + 10 * tsolve::BLK;
+    float *sX = reinterpret_cast<float *>(sm + OFF_T);
     float *sG = reinterpret_cast<float *>(sm + OFF_MISC);        // 64
     float *sBeta = sG + 64;                                      // 64
-    float *sTot = sBeta + 64;                                    // 1
+    float *sTot = sBeta + 64;                                    // 2: partial sums of warps 0, 1
+    float *sEG = reinterpret_cast<float *>(sm + OFF_MISC + 4096);  // 64: e^{G_i}
+    float *sEK = sEG + 64;                                       // 64: e^{G_C - G_i}
+    float *sBE = sEK + 64;                                       // 64: beta_i e^{G_i}
     const int warp = tid >> 5, lane = tid & 31;
     const uint32_t trow = tbase + ((uint32_t)(32 * (warp & 3)) << 16);
     const float eA = expf(__ldg(pa.A + h)), ba = __ldg(pa.b_alpha + h);
@@ -283,27 +368,68 @@ __device__ __forceinline__ bool prep_one_chunk(const Sync &sy, const PrepArgs pa
     bool ok = true;
     const int t0 = s_begin + c * C;
     const int len = min(C, s_end - t0);
-    // the token's gate logits (thread tid < len), loaded first so that their latency
-    // passes while the convolutions run
+    // the token's gate logits (thread tid < len) and the first raw q/k rows are
+    // loaded first, so that their latency passes while the gates are computed
     bf16 a_raw = __float2bfloat16(0.f), b_raw = __float2bfloat16(0.f);
     if (tid < len) {
         const size_t gi = (size_t)(t0 + tid) * H + h;
         a_raw = a_logit[gi];
         b_raw = b_logit[gi];
     }
-    // ---- 1. prelude: q, k -> L2-normalised fp32 -> hi/lo fp16 tiles; v -> fp16 tile
+    const bf16 *qk_src = is_k ? k : q;
+    uint4 raw[7];
+    conv_load<4>(qk_src, (size_t)H * DK, qk_col, t0, s_begin, 8 * warp, len, raw);
+
+    // ---- 1. gates: beta, log alpha and their in-chunk cumulative sum G, then the
+    //         per-token factors e^{G_i}, e^{G_C - G_i}, beta_i e^{G_i}
+    if (tid < C) {
+        float g = 0.f, be = 0.f;
+        if (tid < len) {
+            g = clamp_log_decay(-eA * softplus_fast(to_f32(a_raw) + ba));
+            be = sigmoid_fast(to_f32(b_raw));
+        }
+        // inclusive scan of the log decays within each warp, then across the two
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, g, o);
+            if (lane >= o) g += y;
+        }
+        if (tid == 31) sTot[0] = g;
+        if (tid == 63) sTot[1] = g;
+        sBeta[tid] = be;
+        sG[tid] = g;
+    }
+    sy.sync();
+    if (tid < C) {   // each thread finishes its own token: G_i, and the per-token factors
+        const float w0 = sTot[0];
+        const float Gi = sG[tid] + (tid >= 32 ? w0 : 0.f);
+        const float GC = w0 + sTot[1];
+        const float eg = __expf(Gi);
+        sG[tid] = Gi;
+        sEG[tid] = eg;
+        sEK[tid] = __expf(GC - Gi);
+        sBE[tid] = sBeta[tid] * eg;
+        if (tid == 0) decay[(size_t)t0 * H + h] = __expf(GC);
+    }
+    sy.sync();
+
+    // ---- 2. prelude: q, k -> L2-normalised fp32 -> hi/lo fp16 tiles, and Qt = e^G q,
+    //         Kt = e^{G_C - G} k (fp16) straight to global memory; v -> fp16 tile
     // (conv weights re-read per chunk from L1/L2 to keep them out of the solve's registers)
     {
         float2 w[4][4];
         load_conv_w(conv_w, qk_chan, w);
         const int oc = qk_oct & 15;
         uint8_t *hb = sHI + (oc / 8) * 16384, *lb = sLO + (oc / 8) * 16384;
+        const float *fac = is_k ? sEK : sEG;
+        __half *dst_t = is_k ? Kt : Qt;
         // the warp's 8 tokens in two halves of 4 (a 7-row window each; the halo rows
         // are re-read from L1), which keeps the prelude's registers in bounds
 #pragma unroll 1
         for (int hf = 0; hf < 2; ++hf) {
+            if (hf == 1) conv_load<4>(qk_src, (size_t)H * DK, qk_col, t0, s_begin, 8 * warp + 4, len, raw);
             float2 y[4][4];
-            conv_silu<4>(is_k ? k : q, (size_t)H * DK, qk_col, w, t0, s_begin, 8 * warp + 4 * hf, len, y);
+            conv_silu<4>(raw, w, 8 * warp + 4 * hf, len, y);
             // L2 norm over the 16 lanes that hold this head's q (or k): 4 tokens at once
             float ss[4];
 #pragma unroll
@@ -320,9 +446,12 @@ __device__ __forceinline__ bool prep_one_chunk(const Sync &sy, const PrepArgs pa
             }
 #pragma unroll
             for (int ii = 0; ii < 4; ++ii) {
+                const int i = 8 * warp + 4 * hf + ii;   // token of the chunk
                 const float r = rsqrtf(ss[ii] + kNormEps);
                 const float2 rr = make_float2(r, r);
-                uint32_t hw[4], lw[4];
+                const float sc = fac[i];
+                const float2 scs = make_float2(sc, sc);
+                uint32_t hw[4], lw[4], tw[4];
 #pragma unroll
                 for (int p = 0; p < 4; ++p) {
                     const float2 x = fmul2(y[ii][p], rr);
@@ -331,10 +460,15 @@ __device__ __forceinline__ bool prep_one_chunk(const Sync &sy, const PrepArgs pa
                     const __half2 ll = __floats2half2_rn(x.x - hf2.x, x.y - hf2.y);
                     hw[p] = *reinterpret_cast<const uint32_t *>(&hh);
                     lw[p] = *reinterpret_cast<const uint32_t *>(&ll);
+                    const float2 xt = fmul2(x, scs);
+                    tw[p] = umma::pack_half2(xt.x, xt.y);
                 }
-                const int row = (is_k ? 64 : 0) + 8 * warp + 4 * hf + ii;
+                const int row = (is_k ? 64 : 0) + i;
                 umma::st_chunk(hb, row, oc % 8, make_uint4(hw[0], hw[1], hw[2], hw[3]));
                 umma::st_chunk(lb, row, oc % 8, make_uint4(lw[0], lw[1], lw[2], lw[3]));
+                if (i < len)
+                    *reinterpret_cast<uint4 *>(dst_t + ((size_t)(t0 + i) * H + h) * DK + oc * 8) =
+                        make_uint4(tw[0], tw[1], tw[2], tw[3]);
             }
         }
     }
@@ -342,32 +476,16 @@ __device__ __forceinline__ bool prep_one_chunk(const Sync &sy, const PrepArgs pa
         float2 w[4][4];
         load_conv_w(conv_w, v_chan, w);
         constexpr int NV = C / VPARTS;
+        uint4 vraw[NV + 3];
+        conv_load<NV>(v, (size_t)H * DV, v_col, t0, s_begin, NV * v_part, len, vraw);
         float2 y[NV][4];
-        conv_silu<NV>(v, (size_t)H * DV, v_col, w, t0, s_begin, NV * v_part, len, y);
+        conv_silu<NV>(vraw, w, NV * v_part, len, y);
 #pragma unroll
         for (int ii = 0; ii < NV; ++ii)
             umma::st_chunk(sV + (v_oct / 8) * 8192, NV * v_part + ii, v_oct % 8,
                            make_uint4(umma::pack_half2(y[ii][0].x, y[ii][0].y), umma::pack_half2(y[ii][1].x, y[ii][1].y),
                                       umma::pack_half2(y[ii][2].x, y[ii][2].y), umma::pack_half2(y[ii][3].x, y[ii][3].y)));
     }
-    if (tid < C) {
-        float g = 0.f, be = 0.f;
-        if (tid < len) {
-            g = clamp_log_decay(-eA * softplus_fast(to_f32(a_raw) + ba));
-            be = sigmoid_fast(to_f32(b_raw));
-        }
-        // inclusive scan of the log decays within each warp, then across the two
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const float y = __shfl_up_sync(0xffffffffu, g, o);
-            if (lane >= o) g += y;
-        }
-        if (tid == 31) *sTot = g;
-        sBeta[tid] = be;
-        sG[tid] = g;
-    }
-    sy.sync();
-    if (tid >= 32 && tid < C) sG[tid] += *sTot;
     umma::fence_proxy_async_smem();
     sy.sync();
     if (publish && tid == 0) {   // the previous chunk's writes precede this worker's barriers
@@ -375,7 +493,7 @@ __device__ __forceinline__ bool prep_one_chunk(const Sync &sy, const PrepArgs pa
         asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(publish), "r"(1) : "memory");
     }
 
-    // ---- 2. [Q;K] K^T = [Qh;Kh]Kh^T + [Qh;Kh]Kl^T + [Ql;Kl]Kh^T -> TMEM [0, 64)
+    // ---- 3. [Q;K] K^T = [Qh;Kh]Kh^T + [Qh;Kh]Kl^T + [Ql;Kl]Kh^T -> TMEM [0, 64)
     if (tid == 0) {
         umma::tc_fence_after();
         const uint32_t hi = umma::smem_u32(sHI), lo = umma::smem_u32(sLO);
@@ -391,36 +509,12 @@ __device__ __forceinline__ bool prep_one_chunk(const Sync &sy, const PrepArgs pa
         }
         umma::mma_commit(bar);
     }
-    // while the MMA runs: Qt = e^{G_i} q_i, Kt = e^{G_C - G_i} k_i (fp16) and e^{G_C}
-    {
-        const float GC = sG[C - 1];
-        for (int idx = tid; idx < len * (DK / 8); idx += NT) {
-            const int i = idx / (DK / 8), ch = idx % (DK / 8);
-            const float sq = __expf(sG[i]), sk = __expf(GC - sG[i]);
-            const uint4 qv = *reinterpret_cast<const uint4 *>(sHI + (ch / 8) * 16384 + umma::sw128_offset(i, ch % 8));
-            const uint4 kv = *reinterpret_cast<const uint4 *>(sHI + (ch / 8) * 16384 + umma::sw128_offset(64 + i, ch % 8));
-            const __half2 *q2 = reinterpret_cast<const __half2 *>(&qv);
-            const __half2 *k2 = reinterpret_cast<const __half2 *>(&kv);
-            uint4 qo, ko;
-            uint32_t *qo32 = reinterpret_cast<uint32_t *>(&qo), *ko32 = reinterpret_cast<uint32_t *>(&ko);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 qf = __half22float2(q2[e]), kf = __half22float2(k2[e]);
-                qo32[e] = umma::pack_half2(qf.x * sq, qf.y * sq);
-                ko32[e] = umma::pack_half2(kf.x * sk, kf.y * sk);
-            }
-            const size_t g = ((size_t)(t0 + i) * H + h) * DK + ch * 8;
-            *reinterpret_cast<uint4 *>(Qt + g) = qo;
-            *reinterpret_cast<uint4 *>(Kt + g) = ko;
-        }
-        if (tid == 0) decay[(size_t)t0 * H + h] = __expf(GC);
-    }
     ok = prep_wait(sy, bar, phase, kPrepMaxPolls, tid);
     phase ^= 1;
     umma::tc_fence_after();
     if (!ok) return false;
 
-    // ---- 3. rows 0..63: Aqk (masked, decayed q.k) -> global; rows 64..127: L -> smem
+    // ---- 4. rows 0..63: Aqk (masked, decayed q.k) -> global; rows 64..127: L -> smem
     //         warp w reads lane quadrant w % 4, columns [32 (w / 4), + 32)
     {
         float v[32];
@@ -444,40 +538,53 @@ __device__ __forceinline__ bool prep_one_chunk(const Sync &sy, const PrepArgs pa
                 }
             }
         } else {
+            // L_ij = beta_i (k_i . k_j) e^{G_i - G_j} (j < i) into the blocks (i / 16, jb)
+            // on or below the diagonal (the solve reads the diagonal block's lower part only)
             const float bi = sBeta[i];
-            float4 *dst = reinterpret_cast<float4 *>(sL + i * C + j0);
 #pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4) {
-                float x[4];
+            for (int hb = 0; hb < 2; ++hb) {
+                const int jb = (j0 >> 4) + hb;
+                if (jb > (i >> 4)) continue;
+                float4 *dst = reinterpret_cast<float4 *>(sL + tsolve::bidx(i >> 4, jb) * tsolve::BLK +
+                                                         (i & 15) * tsolve::BS);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int j = j0 + q4 * 4 + e;
-                    x[e] = (j < i) ? bi * v[q4 * 4 + e] * __expf(Gi - sG[j]) : 0.f;
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    float x[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int j = 16 * jb + q4 * 4 + e;
+                        x[e] = (j < i) ? bi * v[16 * hb + q4 * 4 + e] * __expf(Gi - sG[j]) : 0.f;
+                    }
+                    dst[q4] = make_float4(x[0], x[1], x[2], x[3]);
                 }
-                dst[q4] = make_float4(x[0], x[1], x[2], x[3]);
             }
         }
     }
     umma::tc_fence_before();
     sy.sync();
 
-    // ---- 4. T = (I + L)^-1 (fp32, blocked); then T' = T diag(beta e^G) in rows
+    // ---- 5. T = (I + L)^-1 (fp32, blocked); then T' = T diag(beta e^G) in rows
     //         0..63 and T'' = T diag(beta) in rows 64..127 of an fp16 K-major tile
-    solve_unit_lower<NT>(sy, sL, sTf, sX, tid);
+    solve_unit_lower(sy, sL, sTf, sX, tid);
     for (int idx = tid; idx < C * 8; idx += NT) {
         const int i = idx >> 3, ch = idx & 7;
-        const float4 *tr = reinterpret_cast<const float4 *>(sTf + i * C + ch * 8);
-        const float4 t0v = tr[0], t1v = tr[1];
+        // only the blocks on or below the diagonal of T exist: the rest is zero
+        const bool in = (ch >> 1) <= (i >> 4);
+        float4 t0v = make_float4(0.f, 0.f, 0.f, 0.f), t1v = t0v;
+        if (in) {
+            const float4 *tr = reinterpret_cast<const float4 *>(sTf + tsolve::bidx(i >> 4, ch >> 1) * tsolve::BLK +
+                                                                (i & 15) * tsolve::BS + (ch & 1) * 8);
+            t0v = tr[0];
+            t1v = tr[1];
+        }
         const float tv[8] = {t0v.x, t0v.y, t0v.z, t0v.w, t1v.x, t1v.y, t1v.z, t1v.w};
         float a1[8], a2[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
             const int j = ch * 8 + e;
-            // only the block-lower part of T was written: zero the rest
-            const float t = ((j >> 4) <= (i >> 4)) ? tv[e] : 0.f;
-            const float bj = sBeta[j];
-            a1[e] = t * bj * __expf(sG[j]);
-            a2[e] = t * bj;
+            const float t = tv[e];
+            a1[e] = t * sBE[j];
+            a2[e] = t * sBeta[j];
         }
         umma::st_chunk(sT, i, ch, make_uint4(umma::pack_half2(a1[0], a1[1]), umma::pack_half2(a1[2], a1[3]),
                                              umma::pack_half2(a1[4], a1[5]), umma::pack_half2(a1[6], a1[7])));
@@ -487,7 +594,7 @@ __device__ __forceinline__ bool prep_one_chunk(const Sync &sy, const PrepArgs pa
     umma::fence_proxy_async_smem();
     sy.sync();
 
-    // ---- 5. W-part = T' K -> TMEM [0, DK);  U'-part = T'' V -> TMEM [DK, DK + DV)
+    // ---- 6. W-part = T' K -> TMEM [0, DK);  U'-part = T'' V -> TMEM [DK, DK + DV)
     if (tid == 0) {
         umma::tc_fence_after();
         const uint32_t aT = umma::smem_u32(sT), aK = umma::smem_u32(sHI) + 8192, aV = umma::smem_u32(sV);
@@ -506,7 +613,7 @@ __device__ __forceinline__ bool prep_one_chunk(const Sync &sy, const PrepArgs pa
     umma::tc_fence_after();
     if (!ok) return false;
 
-    // ---- 6. rows 0..63 of the W-part -> -W; rows 64..127 of the U'-part -> U'
+    // ---- 7. rows 0..63 of the W-part -> -W; rows 64..127 of the U'-part -> U'
     //         (warp w: lane quadrant w % 4, column half w / 4; TMEM loads are
     //         warp-collective: every lane loads, valid rows store)
     {

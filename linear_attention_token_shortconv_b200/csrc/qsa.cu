@@ -129,7 +129,7 @@ __global__ void __launch_bounds__(256, 1)
 qsa_score_kernel(const __grid_constant__ QsaMaps maps, int n, float *__restrict__ scores) {
     using namespace qsa;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sm = umma::align_smem<1024>(smem_raw);
     uint64_t *bar_ld = reinterpret_cast<uint64_t *>(sm + OFF_BAR);        // operand loads
     uint64_t *bar_mma = reinterpret_cast<uint64_t *>(sm + OFF_BAR + 8);   // MMA completion
     uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 16);

@@ -26,7 +26,7 @@ umma_selftest_kernel(int a_mn, int b_mn, int neg_a, int N, int K, const __half *
                      const __half *__restrict__ B, const float *__restrict__ init,
                      float *__restrict__ D) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sm = umma::align_smem<1024>(smem_raw);
     uint8_t *As = sm + kStA, *Bs = sm + kStB;
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + kStMisc);
     uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + kStMisc + 16);

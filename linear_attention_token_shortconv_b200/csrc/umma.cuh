@@ -28,6 +28,16 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// Round a pointer into dynamic shared memory up to a multiple of A bytes.  The
+// offset is added to the shared pointer itself: a round trip through an integer
+// would hide from the compiler that the result points into shared memory, and
+// every access through it would then use generic addressing.
+template <int A>
+__device__ __forceinline__ uint8_t *align_smem(uint8_t *p) {
+    const uint32_t a = smem_u32(p);
+    return p + ((A - (a & (A - 1))) & (A - 1));
+}
+
 // byte offset of 16-byte chunk `chunk` (0..7) of row `r` inside a 128B-swizzled block
 __device__ __forceinline__ uint32_t sw128_offset(int r, int chunk) {
     return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((chunk ^ (r & 7)) << 4));
@@ -275,6 +285,14 @@ template <int N> __device__ __forceinline__ void bulk_wait_read() {
     asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
 }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Prefetch one tile of a tensor into L2 (no shared-memory destination, no completion).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap *map, int x, int y, int z) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

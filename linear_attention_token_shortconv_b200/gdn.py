@@ -26,7 +26,7 @@ EXPORTS = ("gdn_prefill", "gdn_prefill_workspace_size", "gdn_decode_step", "gdn_
            "gdn_set_kernel_events", "gdn_last_call_launches", "gdn_device_error_status",
            "gdn_selftest_wait_timeout", "gdn_decode_multi", "gdn_prefill_backward",
            "gdn_prefill_backward_workspace_size", "gdn_qsa_indexer", "gdn_qsa_indexer_workspace_size",
-           "gdn_layer_forward", "gdn_layer_workspace_size")
+           "gdn_layer_forward", "gdn_layer_workspace_size", "gdn_prefill_ws", "gdn_prefill_conv_tail")
 ERRF_PREP, ERRF_CHAIN, ERRF_DECODE, ERRF_QSA = 1, 2, 4, 8
 
 
@@ -91,6 +91,10 @@ def load() -> ctypes.CDLL:
         lib.gdn_selftest_wait_timeout.restype = ctypes.c_int
         lib.gdn_status_string.argtypes = [ctypes.c_int]
         lib.gdn_status_string.restype = ctypes.c_char_p
+        lib.gdn_prefill_ws.argtypes = [D] + [P] * 15 + [ctypes.c_size_t, P]
+        lib.gdn_prefill_ws.restype = ctypes.c_int
+        lib.gdn_prefill_conv_tail.argtypes = [D] + [P] * 6
+        lib.gdn_prefill_conv_tail.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -342,6 +346,55 @@ def prefill_noalloc(q, k, v, conv_w, a_logit, b_logit, A, b_alpha, z, norm_w, S0
                                         _ptr(S_final), _stream(stream))
     _check(rc, "gdn_prefill_noalloc")
     return out, S_final
+
+
+def prefill_ws(q, k, v, conv_w, a_logit, b_logit, A, b_alpha, z, norm_w, workspace, S0=None,
+               cu_seqlens=None, *, num_seqs=None, out=None, S_final=None, out_dtype=torch.float32,
+               want_state=True, stream=None):
+    """gdn_prefill_ws on torch tensors: `prefill` with the workspace supplied as a
+    uint8 CUDA tensor of at least prefill_workspace_size() bytes."""
+    n_tok, H, dk = q.shape
+    dv = v.shape[2]
+    if cu_seqlens is not None:
+        n_seq = cu_seqlens.shape[0] - 1
+    else:
+        n_seq = num_seqs if num_seqs is not None else (S0.shape[0] if S0 is not None else 1)
+    if out is None:
+        out = torch.empty((n_tok, H, dv), dtype=out_dtype, device=q.device)
+    if S_final is None and want_state:
+        S_final = torch.empty((n_seq, H, dk, dv), dtype=torch.float32, device=q.device)
+    _check_mixer(q, k, v, conv_w, a_logit, b_logit, A, b_alpha, z, norm_w, S0, cu_seqlens, out, S_final, n_seq)
+    if workspace.dtype != torch.uint8 or workspace.dim() != 1:
+        raise ValueError("workspace: a 1-D uint8 tensor expected")
+    dims = Dims(n_seq, n_tok, H, dk, dv, conv_w.shape[1], _dt(q), _dt(out))
+    with torch.cuda.device(_device(q, k, v, conv_w, a_logit, b_logit, A, b_alpha, z, norm_w, S0, cu_seqlens,
+                                   out, S_final, workspace)):
+        rc = load().gdn_prefill_ws(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w),
+                                   _ptr(a_logit), _ptr(b_logit), _ptr(A), _ptr(b_alpha), _ptr(z),
+                                   _ptr(norm_w), _ptr(S0), _ptr(cu_seqlens), _ptr(out), _ptr(S_final),
+                                   _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(rc, "gdn_prefill_ws")
+    return out, S_final
+
+
+def prefill_conv_tail(q, k, v, cu_seqlens=None, *, num_seqs=None, conv_hist=None, stream=None):
+    """gdn_prefill_conv_tail on torch tensors: the decode conv history
+    [N_seq, 3, H(2dk+dv)] (q.dtype) that continues each prefilled sequence."""
+    n_tok, H, dk = q.shape
+    dv = v.shape[2]
+    n_seq = cu_seqlens.shape[0] - 1 if cu_seqlens is not None else (num_seqs or 1)
+    _expect("k", k, (n_tok, H, dk), q.dtype)
+    _expect("v", v, (n_tok, H, dv), q.dtype)
+    _expect("cu_seqlens", cu_seqlens, (n_seq + 1,), I32)
+    if conv_hist is None:
+        conv_hist = torch.empty((n_seq, 3, H * (2 * dk + dv)), dtype=q.dtype, device=q.device)
+    _expect("conv_hist", conv_hist, (n_seq, 3, H * (2 * dk + dv)), q.dtype)
+    dims = Dims(n_seq, n_tok, H, dk, dv, 4, _dt(q), _dt(q))
+    with torch.cuda.device(_device(q, k, v, cu_seqlens, conv_hist)):
+        rc = load().gdn_prefill_conv_tail(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens),
+                                          _ptr(conv_hist), _stream(stream))
+    _check(rc, "gdn_prefill_conv_tail")
+    return conv_hist
 
 
 def prefill_workspace_size(n_seq, n_tok, H, dk, dv, conv_k=4, in_dtype=torch.bfloat16,

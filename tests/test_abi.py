@@ -205,3 +205,25 @@ def test_qsa_argument_validation(lib):
     assert call(1, 64, 4, 128, 4, 2048, q=P(4100)) == 3
     assert call(1, 64, 4, 128, 4, 2048, sel=None) == 1
     assert call(1, 0, 4, 128, 4, 2048, q=None, sel=None) == 0        # nothing to do
+
+
+def test_prefill_ws_checks_its_workspace(lib):
+    """Workspace NULL or short -> GDN_ERR_INVALID_ARG, misaligned -> GDN_ERR_ALIGNMENT,
+    both before any CUDA call."""
+    d = _dims()
+    need = ctypes.c_size_t(0)
+    assert lib.gdn_prefill_workspace_size(ctypes.byref(d), ctypes.byref(need)) == 0 and need.value > 0
+    a = _args()
+    ws_args = a[:-1]
+    assert lib.gdn_prefill_ws(ctypes.byref(d), *ws_args, None, need.value, None) == 1
+    assert lib.gdn_prefill_ws(ctypes.byref(d), *ws_args, ctypes.c_void_p(1 << 20), need.value - 1, None) == 1
+    assert lib.gdn_prefill_ws(ctypes.byref(d), *ws_args, ctypes.c_void_p((1 << 20) + 16), need.value, None) == 3
+
+
+def test_conv_tail_rejects_bad_arguments(lib):
+    d = _dims()
+    q, k, v = FAKE[0], FAKE[1], FAKE[2]
+    assert lib.gdn_prefill_conv_tail(ctypes.byref(d), q, k, v, None, None, None) == 1
+    assert lib.gdn_prefill_conv_tail(ctypes.byref(d), q, k, v, None, ctypes.c_void_p(4104), None) == 3
+    bad = _dims(dk=96)
+    assert lib.gdn_prefill_conv_tail(ctypes.byref(bad), q, k, v, None, FAKE[4], None) == 2

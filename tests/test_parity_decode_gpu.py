@@ -104,3 +104,41 @@ def test_prefill_then_decode_continues_the_sequence(cuda_device):
     got = torch.cat(outs).cpu().numpy()
     assert normwise(got, out_all[T:].cpu().numpy()) <= TOL_BF16
     assert normwise(S.cpu().numpy(), S_all.cpu().numpy()) <= TOL_BF16
+
+
+def test_prefill_conv_tail_hands_off_to_decode(cuda_device):
+    """Three sequences (150, 2 and 67 tokens, then 5 more each): a prefill of the
+    first part, gdn_prefill_conv_tail's history (checked bit-exact against the raw
+    rows, zero rows before a short sequence's start) and S_final continue every
+    sequence through decode steps as one prefill of the whole does."""
+    T_list, n = [150, 2, 67], 5
+    cfg = scaled(PRETRAIN, lengths=tuple(T + n for T in T_list), H=2, s0_var=0.02, varlen=True)
+    inp = to_device(make_prefill_inputs(cfg, "cpu"), cuda_device)
+    out_all, S_all = gpu_prefill(inp, 3)
+    cu_all = inp["cu_seqlens"].cpu().tolist()
+    idx = torch.cat([torch.arange(cu_all[s], cu_all[s] + T_list[s]) for s in range(3)]).to(cuda_device)
+    tok_keys = ("q", "k", "v", "z", "a_logit", "b_logit")
+    head = {key: (val.index_select(0, idx).contiguous() if key in tok_keys else val) for key, val in inp.items()}
+    cu_head = [0, T_list[0], T_list[0] + T_list[1], sum(T_list)]
+    head["cu_seqlens"] = torch.tensor(cu_head, dtype=torch.int32, device=cuda_device)
+    _, S = gpu_prefill(head, 3)
+    hist = gdn.prefill_conv_tail(head["q"], head["k"], head["v"], head["cu_seqlens"])
+    torch.cuda.synchronize()
+    N = sum(T_list)
+    raw = torch.cat([head["q"].reshape(N, -1), head["k"].reshape(N, -1), head["v"].reshape(N, -1)], dim=1)
+    for s in range(3):
+        for j in range(3):
+            t = cu_head[s + 1] - 3 + j
+            want = raw[t] if t >= cu_head[s] else torch.zeros_like(raw[0])
+            assert torch.equal(hist[s, j], want), (s, j)
+    outs = []
+    for step in range(n):
+        rows = torch.tensor([cu_all[s] + T_list[s] + step for s in range(3)], device=cuda_device)
+        sl = lambda key: inp[key].index_select(0, rows).contiguous()
+        outs.append(gdn.decode_step(sl("q"), sl("k"), sl("v"), inp["conv_w"], hist, sl("a_logit"),
+                                    sl("b_logit"), inp["A"], inp["b_alpha"], sl("z"), inp["norm_w"], S))
+    torch.cuda.synchronize()
+    got = torch.stack(outs, dim=1).cpu().numpy()
+    want = torch.stack([out_all[cu_all[s] + T_list[s]:cu_all[s] + T_list[s] + n] for s in range(3)]).cpu().numpy()
+    assert normwise(got, want) <= TOL_BF16
+    assert normwise(S.cpu().numpy(), S_all.cpu().numpy()) <= TOL_BF16

@@ -75,6 +75,28 @@ def test_overflowing_log_decay_gives_alpha_zero(cuda_device):
     assert e_out <= TOL_BF16 and e_s <= TOL_BF16
 
 
+@pytest.mark.parametrize("cfg", [scaled(LONG, lengths=(700,), H=2),
+                                 scaled(PRETRAIN, lengths=(700, 129), H=20, s0_var=0.02)],
+                         ids=["fused", "segmented"])
+def test_prefill_ws_matches_prefill(cuda_device, cfg):
+    """gdn_prefill_ws runs gdn_prefill's kernels on a workspace the caller owns:
+    the results are bit-identical, and a workspace one byte short is rejected
+    before anything runs."""
+    inp = to_device(make_prefill_inputs(cfg, "cpu"), cuda_device)
+    ref_out, ref_S = gpu_prefill(inp, cfg.num_seqs)
+    nbytes = gdn.prefill_workspace_size(cfg.num_seqs, cfg.total_tokens, cfg.H, cfg.dk, cfg.dv)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=cuda_device)
+    args = (inp["q"], inp["k"], inp["v"], inp["conv_w"], inp["a_logit"], inp["b_logit"], inp["A"],
+            inp["b_alpha"], inp["z"], inp["norm_w"])
+    kw = dict(S0=inp.get("S0"), cu_seqlens=inp.get("cu_seqlens"), num_seqs=cfg.num_seqs)
+    out, S = gdn.prefill_ws(*args, ws, **kw)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref_out) and torch.equal(S, ref_S)
+    with pytest.raises(gdn.GdnError) as ei:
+        gdn.prefill_ws(*args, ws[:nbytes - 1], **kw)
+    assert ei.value.status == 1   # GDN_ERR_INVALID_ARG
+
+
 def test_empty_batch_returns_initial_state(cuda_device):
     cfg = scaled(PRETRAIN, lengths=(0, 0), H=2, s0_var=0.02, varlen=True)
     inp = to_device(make_prefill_inputs(cfg, "cpu"), cuda_device)
