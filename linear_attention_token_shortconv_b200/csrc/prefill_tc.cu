@@ -115,13 +115,13 @@ cudaError_t prep_error_word(unsigned *v, bool clear, cudaStream_t s) {
 
 
 template <int DV, typename Tout>
-__global__ void __launch_bounds__(chain_threads<DV>(), 1)
+__global__ void __launch_bounds__(4 * DV, 1)
 chunk_chain_kernel(const __grid_constant__ ChainMaps maps, const float *__restrict__ decay,
                    const float *__restrict__ norm_w, const float *state_in,
                    const int32_t *__restrict__ cu_seqlens, int n_seq, int n_tok, int H, int c_lo,
-                   int c_hi, const bf16 *__restrict__ z, Tout *__restrict__ out, float *state_out) {
+                   int c_hi, Tout *__restrict__ out, float *state_out) {
     chain_body<DV, Tout>(maps, decay, norm_w, state_in, cu_seqlens, n_seq, n_tok, H, blockIdx.x, blockIdx.y,
-                         c_lo, c_hi, z, out, state_out, nullptr);
+                         c_lo, c_hi, out, state_out, nullptr);
 }
 
 cudaError_t launch_chunk_chain(const PrefillArgs &a, const TcWorkspace &w, int c_lo, int c_hi,
@@ -136,6 +136,8 @@ cudaError_t launch_chunk_chain(const PrefillArgs &a, const TcWorkspace &w, int c
         if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.aqk), w.Aqk, false, 64, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
         if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.up), w.Up, false, a.dv, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
         if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.z), a.z, true, a.dv, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
+        if (a.out_bf16 &&
+            (e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.out), a.out, true, a.dv, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
     }
     dim3 grid(a.H, a.n_seq);
     cudaError_t e;
@@ -143,9 +145,9 @@ cudaError_t launch_chunk_chain(const PrefillArgs &a, const TcWorkspace &w, int c
     e = cudaFuncSetAttribute(chunk_chain_kernel<DV_, TOUT>,                                       \
                              cudaFuncAttributeMaxDynamicSharedMemorySize, chain::SMEM);            \
     if (e != cudaSuccess) return e;                                                               \
-    chunk_chain_kernel<DV_, TOUT><<<grid, chain_threads<DV_>(), chain::SMEM, stream>>>(           \
+    chunk_chain_kernel<DV_, TOUT><<<grid, 4 * DV_, chain::SMEM, stream>>>(                        \
         m, w.decay, a.norm_w, state_in, a.cu_seqlens, a.n_seq, a.n_tok, a.H, c_lo, c_hi,        \
-        (const bf16 *)a.z, (TOUT *)a.out, state_out)
+        (TOUT *)a.out, state_out)
     if (a.dv == 128) {
         if (a.out_bf16) { GDN_CHAIN(128, bf16); } else { GDN_CHAIN(128, float); }
     } else {
@@ -193,7 +195,6 @@ cudaError_t chain_error_word(unsigned *v, bool clear, cudaStream_t s) {
 // chain CTA, so every flag gets set; every wait is bounded all the same.
 namespace fused {
 constexpr int NT = 512;
-static_assert(chain_threads<128>() == NT, "chain role uses the whole CTA");
 constexpr int PREP_REGION = 104448;   // one prep worker's shared memory (1 KB aligned)
 constexpr int SMEM = chain::SMEM > 2 * PREP_REGION + 1024 ? chain::SMEM : 2 * PREP_REGION + 1024;
 static_assert(prep::OFF_MISC + prep::MISC_BYTES <= PREP_REGION, "prep worker region");
@@ -206,7 +207,6 @@ struct FusedParams {
     const float *norm_w, *S0;
     float *S_final;
     const int32_t *cu_seqlens;
-    const bf16 *z;
     void *out;
     int *ready;        // [n_items][max_chunks], zero at launch
     int *next_task;    // zero at launch
@@ -219,7 +219,7 @@ __global__ void __launch_bounds__(fused::NT, 1) prefill_fused_kernel(const __gri
     if ((int)blockIdx.x < P.n_chain) {   // chain role: item blockIdx.x
         const int item = blockIdx.x, n = item / P.H, h = item % P.H;
         chain_body<128, Tout>(P.maps, P.pa.decay, P.norm_w, P.S0, P.cu_seqlens, P.n_seq, P.n_tok, P.H, h, n, 0,
-                              P.max_chunks + 1, P.z, reinterpret_cast<Tout *>(P.out), P.S_final,
+                              P.max_chunks + 1, reinterpret_cast<Tout *>(P.out), P.S_final,
                               P.ready + (size_t)item * P.max_chunks);
         return;
     }
@@ -312,6 +312,8 @@ cudaError_t launch_prefill_fused(const PrefillArgs &a, const TcWorkspace &w, int
     if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&P.maps.aqk), w.Aqk, false, 64, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
     if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&P.maps.up), w.Up, false, 128, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
     if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&P.maps.z), a.z, true, 128, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
+    if (a.out_bf16 &&
+        (e = make_tma_3d(reinterpret_cast<TmaMap *>(&P.maps.out), a.out, true, 128, a.H, a.n_tok, 64, 64, true)) != cudaSuccess) return e;
     if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&P.raw_q), a.q, true, 128, a.H, a.n_tok, 128, 67, false)) != cudaSuccess) return e;
     if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&P.raw_k), a.k, true, 128, a.H, a.n_tok, 128, 67, false)) != cudaSuccess) return e;
     if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&P.raw_v), a.v, true, 128, a.H, a.n_tok, 128, 67, false)) != cudaSuccess) return e;
@@ -320,7 +322,6 @@ cudaError_t launch_prefill_fused(const PrefillArgs &a, const TcWorkspace &w, int
     P.S0 = a.S0;
     P.S_final = a.S_final;
     P.cu_seqlens = a.cu_seqlens;
-    P.z = (const bf16 *)a.z;
     P.out = a.out;
     P.n_seq = a.n_seq;
     P.n_tok = a.n_tok;

@@ -108,6 +108,27 @@ __device__ __forceinline__ void prefetch_chunk_rows(const bf16 *q, const bf16 *k
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(row), "r"(which == 2 ? DV * 2 : 256) : "memory");
 }
 
+// Row staging for coalesced global stores.  A tile of 16-bit rows is staged in
+// shared memory with its 16-byte chunks rotated by the row (chunk c of row r at
+// position c ^ (r % 8)), so that both the row-per-lane writes out of tensor
+// memory and the row-contiguous reads that follow are free of bank conflicts.
+// RB: bytes per row.
+template <int RB>
+__device__ __forceinline__ uint32_t stage_off(int r, int c) {
+    return (uint32_t)(r * RB + ((c ^ (r & 7)) << 4));
+}
+// Copy rows [0, len) of a staged tile of 64 rows to global memory, a warp storing
+// whole rows (RB / 16 lanes per row), NT threads.  Row r goes to dst + r * stride.
+template <int RB, int NT>
+__device__ __forceinline__ void store_rows(const uint8_t *stage, __half *dst, size_t stride, int len, int tid) {
+    constexpr int CPR = RB / 16;   // 16-byte chunks per row
+    for (int e = tid; e < len * CPR; e += NT) {
+        const int r = e / CPR, c = e % CPR;
+        *reinterpret_cast<uint4 *>(dst + (size_t)r * stride + c * 8) =
+            *reinterpret_cast<const uint4 *>(stage + stage_off<RB>(r, c));
+    }
+}
+
 // Conv + SiLU of 8 channels (4 pairs) for tokens [i0, i0 + N) of a chunk: all
 // N + 3 raw rows (zero before the sequence start and past its end) are loaded
 // first, then a sliding window of converted rows produces y[N][4] (pairs).
@@ -342,7 +363,8 @@ __device__ __forceinline__ bool prep_one_chunk(const Sync &sy, const PrepArgs pa
     // q.k MMA; the solve's scratch uses the [T'; T''] tile's region, written after it
     float *sL = reinterpret_cast<float *>(sm + OFF_LO);
     float *sTf = sL + 10 * tsolve::BLK;
-    float *sX = reinterpret_cast<float *>(sm + OFF_T);
+    float *sX = reinterpret_cast<float *>(sm + OFF_T);             // solve scratch: [0, 7 KB)
+    uint8_t *sAqk = sm + OFF_T + 8192;                            // Aqk row stage: 64 x 128 B
     float *sG = reinterpret_cast<float *>(sm + OFF_MISC);        // 64
     float *sBeta = sG + 64;                                      // 64
     float *sTot = sBeta + 64;                                    // 2: partial sums of warps 0, 1
@@ -488,7 +510,10 @@ __device__ __forceinline__ bool prep_one_chunk(const Sync &sy, const PrepArgs pa
     }
     umma::fence_proxy_async_smem();
     sy.sync();
-    if (publish && tid == 0) {   // the previous chunk's writes precede this worker's barriers
+    if (publish && tid == 32) {
+        // the previous chunk's writes (every thread's) precede this worker's barriers;
+        // a thread other than the MMA issuer makes them visible and sets the flag, so
+        // that the fence's wait for the stores does not delay the MMA below
         __threadfence();
         asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(publish), "r"(1) : "memory");
     }
@@ -523,19 +548,18 @@ __device__ __forceinline__ bool prep_one_chunk(const Sync &sy, const PrepArgs pa
         const int i = (32 * (warp & 3) + lane) & 63;
         const float Gi = sG[i];
         if ((warp & 3) < 2) {
-            if (i < len) {
-                uint4 *dst = reinterpret_cast<uint4 *>(Aqk + ((size_t)(t0 + i) * H + h) * C + j0);
+            // Aqk row i (its 32 columns j0..) into the row stage; stored after the barrier
 #pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) {
-                    float x[8];
+            for (int q8 = 0; q8 < 4; ++q8) {
+                float x[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int j = j0 + q8 * 8 + e;
-                        x[e] = (j <= i) ? v[q8 * 8 + e] * __expf(Gi - sG[j]) : 0.f;
-                    }
-                    dst[q8] = make_uint4(umma::pack_half2(x[0], x[1]), umma::pack_half2(x[2], x[3]),
-                                         umma::pack_half2(x[4], x[5]), umma::pack_half2(x[6], x[7]));
+                for (int e = 0; e < 8; ++e) {
+                    const int j = j0 + q8 * 8 + e;
+                    x[e] = (j <= i) ? v[q8 * 8 + e] * __expf(Gi - sG[j]) : 0.f;
                 }
+                *reinterpret_cast<uint4 *>(sAqk + stage_off<C * 2>(i, j0 / 8 + q8)) =
+                    make_uint4(umma::pack_half2(x[0], x[1]), umma::pack_half2(x[2], x[3]),
+                               umma::pack_half2(x[4], x[5]), umma::pack_half2(x[6], x[7]));
             }
         } else {
             // L_ij = beta_i (k_i . k_j) e^{G_i - G_j} (j < i) into the blocks (i / 16, jb)
@@ -562,6 +586,9 @@ __device__ __forceinline__ bool prep_one_chunk(const Sync &sy, const PrepArgs pa
     }
     umma::tc_fence_before();
     sy.sync();
+    // Aqk rows to global memory, whole rows per warp (its stage is not reused before
+    // the barriers of the solve)
+    store_rows<C * 2, NT>(sAqk, Aqk + ((size_t)t0 * H + h) * C, (size_t)H * C, len, tid);
 
     // ---- 5. T = (I + L)^-1 (fp32, blocked); then T' = T diag(beta e^G) in rows
     //         0..63 and T'' = T diag(beta) in rows 64..127 of an fp16 K-major tile
@@ -615,39 +642,39 @@ __device__ __forceinline__ bool prep_one_chunk(const Sync &sy, const PrepArgs pa
 
     // ---- 7. rows 0..63 of the W-part -> -W; rows 64..127 of the U'-part -> U'
     //         (warp w: lane quadrant w % 4, column half w / 4; TMEM loads are
-    //         warp-collective: every lane loads, valid rows store)
+    //         warp-collective), through row stages in the [Ql;Kl] region (free since
+    //         the T' build) so that the global stores are whole rows per warp
     {
+        uint8_t *sW = sLO, *sU = sLO + 64 * DK * 2;
         const int i = (32 * (warp & 3) + lane) & 63;
         const int half = warp >> 2;
         if ((warp & 3) < 2) {
-            __half *dst = Wn + ((size_t)(t0 + i) * H + h) * DK;
 #pragma unroll
             for (int c0 = half * (DK / 2); c0 < (half + 1) * (DK / 2); c0 += 32) {
                 float vv[32];
                 umma::tmem_ld32(trow + c0, vv);
-                if (i < len) {
 #pragma unroll
-                    for (int q8 = 0; q8 < 4; ++q8)
-                        reinterpret_cast<uint4 *>(dst + c0)[q8] = make_uint4(
-                            umma::pack_half2(-vv[q8 * 8 + 0], -vv[q8 * 8 + 1]), umma::pack_half2(-vv[q8 * 8 + 2], -vv[q8 * 8 + 3]),
-                            umma::pack_half2(-vv[q8 * 8 + 4], -vv[q8 * 8 + 5]), umma::pack_half2(-vv[q8 * 8 + 6], -vv[q8 * 8 + 7]));
-                }
+                for (int q8 = 0; q8 < 4; ++q8)
+                    *reinterpret_cast<uint4 *>(sW + stage_off<DK * 2>(i, c0 / 8 + q8)) = make_uint4(
+                        umma::pack_half2(-vv[q8 * 8 + 0], -vv[q8 * 8 + 1]), umma::pack_half2(-vv[q8 * 8 + 2], -vv[q8 * 8 + 3]),
+                        umma::pack_half2(-vv[q8 * 8 + 4], -vv[q8 * 8 + 5]), umma::pack_half2(-vv[q8 * 8 + 6], -vv[q8 * 8 + 7]));
             }
         } else {
-            __half *dst = Up + ((size_t)(t0 + i) * H + h) * DV;
 #pragma unroll
             for (int c0 = half * (DV / 2); c0 < (half + 1) * (DV / 2); c0 += 32) {
                 float vv[32];
                 umma::tmem_ld32(trow + DK + c0, vv);
-                if (i < len) {
 #pragma unroll
-                    for (int q8 = 0; q8 < 4; ++q8)
-                        reinterpret_cast<uint4 *>(dst + c0)[q8] = make_uint4(
-                            umma::pack_half2(vv[q8 * 8 + 0], vv[q8 * 8 + 1]), umma::pack_half2(vv[q8 * 8 + 2], vv[q8 * 8 + 3]),
-                            umma::pack_half2(vv[q8 * 8 + 4], vv[q8 * 8 + 5]), umma::pack_half2(vv[q8 * 8 + 6], vv[q8 * 8 + 7]));
-                }
+                for (int q8 = 0; q8 < 4; ++q8)
+                    *reinterpret_cast<uint4 *>(sU + stage_off<DV * 2>(i, c0 / 8 + q8)) = make_uint4(
+                        umma::pack_half2(vv[q8 * 8 + 0], vv[q8 * 8 + 1]), umma::pack_half2(vv[q8 * 8 + 2], vv[q8 * 8 + 3]),
+                        umma::pack_half2(vv[q8 * 8 + 4], vv[q8 * 8 + 5]), umma::pack_half2(vv[q8 * 8 + 6], vv[q8 * 8 + 7]));
             }
         }
+        umma::tc_fence_before();
+        sy.sync();
+        store_rows<DK * 2, NT>(sW, Wn + ((size_t)t0 * H + h) * DK, (size_t)H * DK, len, tid);
+        store_rows<DV * 2, NT>(sU, Up + ((size_t)t0 * H + h) * DV, (size_t)H * DV, len, tid);
     }
     umma::tc_fence_before();
     sy.sync();
