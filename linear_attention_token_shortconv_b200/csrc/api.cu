@@ -47,11 +47,16 @@ bool use_tensor_cores(const gdn_dims_t *d) { return d->in_dtype == GDN_BF16 && d
 // SMs that segment s's last CTAs leave idle.  The chain kernel of segment s runs
 // on a third, highest-priority stream after prep s and chain s - 1 (events);
 // the state passes from one chain launch to the next through a state buffer.
+// Segments cut the chunks of the longest sequence: N_tok / N_seq of them for
+// equal lengths; with cu_seqlens the host does not know the longest, and the
+// bound N_tok / 64 is used (launches past a sequence's end exit at once).  The
+// workspace size takes the bound, so it covers both.
 struct Segments {
     int seg, n;
 };
-Segments segments(const gdn_dims_t *d) {
-    const int max_chunks = (d->total_tokens + 63) / 64;
+Segments segments(const gdn_dims_t *d, bool equal_lengths = false) {
+    const int longest = equal_lengths && d->num_seqs > 0 ? d->total_tokens / d->num_seqs : d->total_tokens;
+    const int max_chunks = (longest + 63) / 64;
     Segments g;
     g.seg = max(8, (max_chunks + 15) / 16);
     g.n = max(1, (max_chunks + g.seg - 1) / g.seg);
@@ -193,7 +198,7 @@ cudaError_t prefill_run(const gdn::PrefillArgs &a, char *ext_ws) {
         w.Aqk = reinterpret_cast<__half *>(take(nt * 64 * 2));
         w.decay = reinterpret_cast<float *>(take(nt * 4));
         int *ready = reinterpret_cast<int *>(take(((size_t)a.n_seq * a.H * ((a.n_tok + 63) / 64) + 1) * 4));
-        const Segments g = segments(dims);
+        const Segments g = segments(dims, a.cu_seqlens == nullptr);
         int slot = 0, sms = 0;
         e = record(g_ev_begin, a.stream);
         if (e == cudaSuccess) e = gdn::sm_count(&sms);

@@ -14,13 +14,16 @@
 // a verifier can compute the outputs of a draft without committing it
 // (n_keep = 0: the state is not written at all) and commit the accepted prefix.
 //
-// One persistent CTA per SM walks the (sequence, head) items.  Each item's
-// inputs -- the 64 KB fp32 state, the tokens' q, k, v, z rows and the three
-// history rows -- arrive by bulk copies (TMA, cp.async.bulk) into one of the
-// shared-memory stages, completing on the stage's mbarrier.  The CTA moves the
-// stage into registers at once and refills it with a later item, so
-// NSTAGE - 1 state loads are in flight while it computes; S' leaves from
-// registers with coalesced streaming stores.  Every wait is bounded.
+// Persistent CTAs walk the (sequence, head) items.  Each item's inputs -- the
+// 64 KB fp32 state, the tokens' q, k, v, z rows and the three history rows --
+// arrive by bulk copies (TMA, cp.async.bulk) into one of the CTA's shared-memory
+// stages, completing on the stage's mbarrier.  The CTA moves the stage into
+// registers at once and refills it with a later item, so loads stay in flight
+// while it computes; S' leaves from registers with coalesced streaming stores.
+// One token: one CTA per SM with three stages.  Several tokens: the step is
+// latency-bound in its barrier phases (a prelude, the state products, a small
+// solve, the update), so two CTAs share each SM with one stage each and one
+// CTA's phases fill the other's waits.  Every wait is bounded.
 #include <cuda_bf16.h>
 
 #include "gdn_device.cuh"
@@ -36,22 +39,27 @@ constexpr int D = 128;                      // dk = dv
 constexpr int NT = 256;
 constexpr int STATE = D * D * 4;            // 64 KB
 constexpr uint32_t kMaxPolls = 1u << 24;
-// Layout for up to TMAX tokens per item: one token (three stages in flight) or
-// four (two stages: the state is read once for four tokens).
+// Layout for up to TMAX tokens per item: one token (one CTA per SM, three
+// stages in flight) or four (two CTAs per SM, one stage each: the state is read
+// once for four tokens).
 template <int TMAX> struct Layout {
-    static constexpr int NSTAGE = TMAX == 1 ? 3 : 2;
+    static constexpr int CTAS_PER_SM = TMAX == 1 ? 1 : 2;
+    static constexpr int NSTAGE = TMAX == 1 ? 3 : 1;
     static constexpr int OFF_TOK = STATE;                      // q, k, v, z rows: [4][TMAX] x 256 B
     static constexpr int OFF_HIST = OFF_TOK + 4 * TMAX * 256;  // 3 slots x (q, k, v) x 256 B
     static constexpr int STAGE = OFF_HIST + 2304;
     static constexpr int OFF_MISC = NSTAGE * STAGE;            // barriers, reductions, prelude values
     // misc: barriers / flag [0, 64), gates [TMAX][2], Gram products [4][TMAX][TMAX],
-    // then xs [2][TMAX][384], red [2][TMAX][8][128], e [TMAX][128], y [TMAX][128]
+    // then xs [TMAX][384] (conv + SiLU values), red [2][TMAX][8][128] (per-warp
+    // partial state products; e and y later take slot w = 0 of each token's k and
+    // q partials), kb [TMAX][128] (the update's scaled keys), zb [TMAX][128] bf16
     static constexpr int OFF_GATE = 64;
     static constexpr int OFF_GRAM = OFF_GATE + 8 * TMAX;
     static constexpr int OFF_XS = (OFF_GRAM + 16 * TMAX * TMAX + 15) / 16 * 16;
-    static constexpr int SMEM = OFF_MISC + OFF_XS + (2 * TMAX * 384 + 2 * TMAX * 8 * 128 + 2 * TMAX * 128) * 4 + 128;
+    static constexpr int SMEM = OFF_MISC + OFF_XS + (TMAX * 384 + 2 * TMAX * 8 * 128 + TMAX * 128) * 4 +
+                                TMAX * 128 * 2 + 128;
     static_assert(STAGE % 128 == 0, "stage alignment");
-    static_assert(SMEM <= 232448, "227 KB per block");
+    static_assert(SMEM * CTAS_PER_SM + 1024 * CTAS_PER_SM <= 233472, "shared memory per SM");
 };
 }  // namespace dstream
 
@@ -81,7 +89,7 @@ __device__ __forceinline__ bool dwait(uint64_t *bar, uint32_t parity, volatile i
 }
 
 template <typename Tout, int TMAX>
-__global__ void __launch_bounds__(dstream::NT, 1)
+__global__ void __launch_bounds__(dstream::NT, dstream::Layout<TMAX>::CTAS_PER_SM)
 decode_stream_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
                      const bf16 *__restrict__ v, const float *__restrict__ conv_w,
                      bf16 *__restrict__ hist, const bf16 *__restrict__ a_logit,
@@ -100,13 +108,18 @@ decode_stream_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
     volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 32);
     float *gate = reinterpret_cast<float *>(misc + Lo::OFF_GATE);                 // [TMAX][2]: alpha, beta
     float *gram = reinterpret_cast<float *>(misc + Lo::OFF_GRAM);                 // [4][TMAX][TMAX]
-    float *xs2 = reinterpret_cast<float *>(misc + Lo::OFF_XS);                    // [2][TMAX][384] conv+SiLU values
-    float *red = xs2 + 2 * TMAX * 384;                                             // [2][TMAX][8][128]
-    float *e_s = red + 2 * TMAX * 8 * 128;                                         // e [TMAX][128]
-    float *y_s = e_s + TMAX * 128;                                                 // y [TMAX][128]
+    float *xs = reinterpret_cast<float *>(misc + Lo::OFF_XS);                     // [TMAX][384] conv+SiLU values
+    float *red = xs + TMAX * 384;                                                  // [2][TMAX][8][128]
+    constexpr int ES = 8 * D;                                                      // e_t, y_t: stride between tokens
+    float *e_s = red;                                                              // e_t at e_s + t ES
+    float *y_s = red + TMAX * 8 * D;                                               // y_t at y_s + t ES
+    float *kb = red + 2 * TMAX * 8 * D;                                            // [TMAX][128]
+    bf16 *zb = reinterpret_cast<bf16 *>(kb + TMAX * D);                            // [TMAX][128], warp 7 only
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n_items = B * H;
+    // row of the state held in this thread's register r
+    auto row_of = [&](int r) { return TMAX == 1 ? 16 * warp + r : warp + 8 * r; };
     const size_t C = (size_t)H * 3 * D;   // conv channels per token
 
     if (tid == 0) {
@@ -116,31 +129,49 @@ decode_stream_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
     }
     __syncthreads();
 
-    auto issue = [&](int item, int s) {   // tid 0 only
+    // Stage s's loads for `item`, issued by warp 0: lane 0 arms the barrier, then
+    // lanes 0-3 take the state's quarters, lanes 4 .. 4 + 4T - 1 the token rows
+    // (q, k, v, z of each token) and the next nine lanes the history rows.  With
+    // one token, lane 0 issues all 17 copies (measured 1% faster there).
+    auto issue = [&](int item, int s) {   // warp 0
         const int b = item / H, h = item % H;
         uint8_t *st = sm + s * STAGE;
         uint64_t *bar = full + s;
-        umma::mbar_expect_tx(bar, STATE + T * 1024 + 2304);
-        const float *Sh = S + ((size_t)b * H + h) * D * D;
+        if (lane == 0) umma::mbar_expect_tx(bar, STATE + T * 1024 + 2304);
+        if constexpr (TMAX == 1) {
+            if (lane == 0) {
 #pragma unroll
-        for (int p = 0; p < 4; ++p) bulk_load(st + p * (STATE / 4), Sh + p * (D * D / 4), STATE / 4, bar);
-        for (int t = 0; t < T; ++t) {
-            const size_t tok = (((size_t)b * T + t) * H + h) * D;
-            bulk_load(st + OFF_TOK + (0 * TMAX + t) * 256, q + tok, 256, bar);
-            bulk_load(st + OFF_TOK + (1 * TMAX + t) * 256, k + tok, 256, bar);
-            bulk_load(st + OFF_TOK + (2 * TMAX + t) * 256, v + tok, 256, bar);
-            bulk_load(st + OFF_TOK + (3 * TMAX + t) * 256, z + tok, 256, bar);
+                for (int p = 0; p < 4; ++p)
+                    bulk_load(st + p * (STATE / 4), S + ((size_t)b * H + h) * D * D + p * (D * D / 4), STATE / 4, bar);
+                const size_t tok = ((size_t)b * H + h) * D;
+                bulk_load(st + OFF_TOK + 0 * 256, q + tok, 256, bar);
+                bulk_load(st + OFF_TOK + 1 * 256, k + tok, 256, bar);
+                bulk_load(st + OFF_TOK + 2 * 256, v + tok, 256, bar);
+                bulk_load(st + OFF_TOK + 3 * 256, z + tok, 256, bar);
+#pragma unroll
+                for (int j = 0; j < 3; ++j)
+#pragma unroll
+                    for (int part = 0; part < 3; ++part)
+                        bulk_load(st + OFF_HIST + j * 768 + part * 256,
+                                  hist + ((size_t)b * 3 + j) * C + (size_t)part * H * D + (size_t)h * D, 256, bar);
+            }
+            return;
         }
-#pragma unroll
-        for (int j = 0; j < 3; ++j) {
+        __syncwarp();
+        if (lane < 4) {
+            bulk_load(st + lane * (STATE / 4), S + ((size_t)b * H + h) * D * D + lane * (D * D / 4), STATE / 4, bar);
+        } else if (lane < 4 + 4 * T) {
+            const int u = lane - 4, part = u / T, t = u % T;
+            const bf16 *src = part == 0 ? q : part == 1 ? k : part == 2 ? v : z;
+            bulk_load(st + OFF_TOK + (part * TMAX + t) * 256, src + (((size_t)b * T + t) * H + h) * D, 256, bar);
+        } else if (lane < 13 + 4 * T) {
+            const int u = lane - 4 - 4 * T, j = u / 3, part = u % 3;
             const bf16 *hr = hist + ((size_t)b * 3 + j) * C;
-            bulk_load(st + OFF_HIST + j * 768, hr + (size_t)h * D, 256, bar);
-            bulk_load(st + OFF_HIST + j * 768 + 256, hr + (size_t)H * D + (size_t)h * D, 256, bar);
-            bulk_load(st + OFF_HIST + j * 768 + 512, hr + (size_t)2 * H * D + (size_t)h * D, 256, bar);
+            bulk_load(st + OFF_HIST + j * 768 + part * 256, hr + (size_t)part * H * D + (size_t)h * D, 256, bar);
         }
     };
     const int first = blockIdx.x, stride = gridDim.x;
-    if (tid == 0) {
+    if (warp == 0) {
 #pragma unroll
         for (int i = 0; i < NSTAGE; ++i)
             if (first + i * stride < n_items) issue(first + i * stride, i);
@@ -151,7 +182,6 @@ decode_stream_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
         const int s = j % NSTAGE;
         const uint32_t parity = (uint32_t)(j / NSTAGE) & 1u;
         const uint8_t *st = sm + s * STAGE;
-        float *xs = xs2 + (j & 1) * TMAX * 384;
         const int b = item / H, h = item % H;
         const size_t gi = (size_t)b * H + h;
         // tokens of sequence b committed to the state and history
@@ -163,28 +193,33 @@ decode_stream_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
             a_l = __bfloat162float(a_logit[gt]);
             b_l = __bfloat162float(b_logit[gt]);
         }
-        // this thread's conv weights: channel tid (q or k) and, for tid < 128, v channel tid
+        // this thread's conv weights: channel tid (q or k) and v channel tid % 128
+        // (one token: threads < 128 only)
         const float4 w0 = __ldg(reinterpret_cast<const float4 *>(conv_w) +
                                 (tid < D ? (size_t)h * D + tid : (size_t)H * D + (size_t)h * D + (tid - D)));
-        const float4 w1 = tid < D ? __ldg(reinterpret_cast<const float4 *>(conv_w) + (size_t)2 * H * D + (size_t)h * D + tid)
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 w1 = (TMAX > 1 || tid < D)
+                              ? __ldg(reinterpret_cast<const float4 *>(conv_w) + (size_t)2 * H * D + (size_t)h * D + tid % D)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
         dwait(full + s, parity, abort_flag);
 
-        // ---- take everything out of the stage: the state into registers (thread t
-        // holds float4 t + 256 r, i.e. row t/32 + 8 r, columns 4 (t%32) ..), the
+        // ---- take everything out of the stage: the state into registers (lane l
+        // holds columns 4 l .. 4 l + 3 of 16 rows: rows 16 w .. 16 w + 15 of warp w
+        // for one token, rows w, w + 8, .. for several -- each measured faster
+        // in its kernel), the
         // conv inputs through the prelude into xs, z into warp 7's registers; the
         // advanced history goes straight back to global memory.
         const float4 *Sv = reinterpret_cast<const float4 *>(st);
         float4 sreg[16];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) sreg[r] = Sv[tid + r * NT];
+        for (int r = 0; r < 16; ++r) sreg[r] = Sv[row_of(r) * 32 + lane];
         const bf16 *tok = reinterpret_cast<const bf16 *>(st + OFF_TOK);
         const bf16 *hs = reinterpret_cast<const bf16 *>(st + OFF_HIST);
         bf16 *hb = hist + (size_t)b * 3 * C;
-        for (int ch = tid; ch < 3 * D; ch += NT) {
-            const int part = ch / D, i = ch % D;   // part 0 q, 1 k, 2 v
-            const float4 w = ch < NT ? w0 : w1;
-            // the window [history slots 0..2, tokens 0..T-1] of this channel
+        // One channel over the window [history slots 0..2, tokens 0..T-1]: the conv +
+        // SiLU values of tokens [t_lo, t_hi) into xs and, if `adv`, the history
+        // advanced by the committed tokens.
+        auto channel = [&](int part, int i, const float4 w, int t_lo, int t_hi, bool adv) {
+            const int ch = part * D + i;   // part 0 q, 1 k, 2 v
             bf16 win[3 + TMAX];
 #pragma unroll
             for (int r = 0; r < 3; ++r) win[r] = hs[r * 384 + part * 128 + i];
@@ -193,7 +228,7 @@ decode_stream_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
                 if (t < T) win[3 + t] = tok[(part * TMAX + t) * 128 + i];
 #pragma unroll
             for (int t = 0; t < TMAX; ++t) {
-                if (t < T) {
+                if (t < T && t >= t_lo && t < t_hi) {
                     float acc = w.x * __bfloat162float(win[t]);
                     acc = fmaf(w.y, __bfloat162float(win[t + 1]), acc);
                     acc = fmaf(w.z, __bfloat162float(win[t + 2]), acc);
@@ -201,7 +236,7 @@ decode_stream_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
                     xs[t * 384 + ch] = __fdividef(acc, 1.0f + __expf(-acc));
                 }
             }
-            if (nk > 0) {   // the history advances by the committed tokens
+            if (adv && nk > 0) {
                 const size_t c = (size_t)part * H * D + (size_t)h * D + i;
 #pragma unroll
                 for (int r = 0; r < 3; ++r) {
@@ -212,17 +247,25 @@ decode_stream_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
                     hb[r * C + c] = val;
                 }
             }
+        };
+        if constexpr (TMAX == 1) {
+            for (int ch = tid; ch < 3 * D; ch += NT) channel(ch / D, ch % D, ch < NT ? w0 : w1, 0, 1, true);
+        } else {
+            // q or k channel tid over all tokens, and half of v channel tid % 128:
+            // the first half of the tokens (threads < 128, which also advance its
+            // history) or the second
+            channel(tid / D, tid % D, w0, 0, TMAX, true);
+            const int half = tid / D;
+            channel(2, tid % D, w1, half * (TMAX / 2), half ? TMAX : TMAX / 2, half == 0);
         }
-        float zr[TMAX][4];
-        if (warp == NT / 32 - 1) {
+        if (warp == NT / 32 - 1) {   // z rows out of the stage; warp 7 alone reads them back
+            const uint2 *zsrc = reinterpret_cast<const uint2 *>(tok + 3 * TMAX * 128);
 #pragma unroll
             for (int t = 0; t < TMAX; ++t)
-#pragma unroll
-                for (int m = 0; m < 4; ++m)
-                    zr[t][m] = t < T ? __bfloat162float(tok[(3 * TMAX + t) * 128 + lane + 32 * m]) : 0.f;
+                if (t < T) reinterpret_cast<uint2 *>(zb)[t * 32 + lane] = zsrc[t * 32 + lane];
         }
         __syncthreads();   // stage s is consumed and xs is complete
-        if (tid == 0 && item + NSTAGE * stride < n_items) issue(item + NSTAGE * stride, s);
+        if (warp == 0 && item + NSTAGE * stride < n_items) issue(item + NSTAGE * stride, s);
 
         // ---- the Gram products of the raw conv outputs, alongside pass 1.  Token t
         // owns entries t (t + 2) .. (t + 1)(t + 3) - 1: q_t.q_t (type 0), k_t.k_t
@@ -248,30 +291,54 @@ decode_stream_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
             gate[lane * 2 + 0] = expf(log_decay(a_l, __ldg(A + h), __ldg(b_alpha + h)));
             gate[lane * 2 + 1] = sigmoid_acc(b_l);
         }
-        // ---- pass 1: partial S0^T k_t and S0^T q_t over this thread's 16 rows
-        {
-            float4 pk[TMAX], pq[TMAX];
+        // ---- pass 1: partial S0^T k_t and S0^T q_t over this thread's 16 rows, two
+        // tokens per sweep over the register state (fewer live accumulators)
+        constexpr int TG = TMAX < 2 ? TMAX : 2;
 #pragma unroll
-            for (int t = 0; t < TMAX; ++t) { pk[t] = make_float4(0.f, 0.f, 0.f, 0.f); pq[t] = pk[t]; }
+        for (int t0 = 0; t0 < TMAX; t0 += TG) {
+            if (t0 < T) {
+                float4 pk[TG], pq[TG];
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                const int i = warp + 8 * r;
+                for (int u = 0; u < TG; ++u) { pk[u] = make_float4(0.f, 0.f, 0.f, 0.f); pq[u] = pk[u]; }
+                // row r of the state against token t0 + u's key and query entries kk, qq
+                auto acc_row = [&](int r, int u, float kk, float qq) {
+                    const float2 s01 = make_float2(sreg[r].x, sreg[r].y), s23 = make_float2(sreg[r].z, sreg[r].w);
+                    const float2 k2 = make_float2(kk, kk), q2 = make_float2(qq, qq);
+                    float2 lo = ffma2(s01, k2, make_float2(pk[u].x, pk[u].y));
+                    float2 hi = ffma2(s23, k2, make_float2(pk[u].z, pk[u].w));
+                    pk[u] = make_float4(lo.x, lo.y, hi.x, hi.y);
+                    lo = ffma2(s01, q2, make_float2(pq[u].x, pq[u].y));
+                    hi = ffma2(s23, q2, make_float2(pq[u].z, pq[u].w));
+                    pq[u] = make_float4(lo.x, lo.y, hi.x, hi.y);
+                };
+                if constexpr (TMAX == 1) {   // consecutive rows: one 16-byte load per four
 #pragma unroll
-                for (int t = 0; t < TMAX; ++t) {
-                    if (t < T) {
-                        const float kk = xs[t * 384 + D + i], qq = xs[t * 384 + i];
-                        pk[t].x = fmaf(sreg[r].x, kk, pk[t].x); pk[t].y = fmaf(sreg[r].y, kk, pk[t].y);
-                        pk[t].z = fmaf(sreg[r].z, kk, pk[t].z); pk[t].w = fmaf(sreg[r].w, kk, pk[t].w);
-                        pq[t].x = fmaf(sreg[r].x, qq, pq[t].x); pq[t].y = fmaf(sreg[r].y, qq, pq[t].y);
-                        pq[t].z = fmaf(sreg[r].z, qq, pq[t].z); pq[t].w = fmaf(sreg[r].w, qq, pq[t].w);
+                    for (int g = 0; g < 4; ++g) {
+                        const float4 kv = *reinterpret_cast<const float4 *>(xs + D + 16 * warp + 4 * g);
+                        const float4 qv = *reinterpret_cast<const float4 *>(xs + 16 * warp + 4 * g);
+                        acc_row(4 * g + 0, 0, kv.x, qv.x);
+                        acc_row(4 * g + 1, 0, kv.y, qv.y);
+                        acc_row(4 * g + 2, 0, kv.z, qv.z);
+                        acc_row(4 * g + 3, 0, kv.w, qv.w);
+                    }
+                } else {
+#pragma unroll
+                    for (int r = 0; r < 16; ++r) {
+                        const int i = row_of(r);
+#pragma unroll
+                        for (int u = 0; u < TG; ++u) {
+                            const int t = t0 + u;
+                            if (t < T) acc_row(r, u, xs[t * 384 + D + i], xs[t * 384 + i]);
+                        }
                     }
                 }
-            }
 #pragma unroll
-            for (int t = 0; t < TMAX; ++t) {
-                if (t < T) {
-                    reinterpret_cast<float4 *>(red + (t * 8 + warp) * D)[lane] = pk[t];
-                    reinterpret_cast<float4 *>(red + ((TMAX + t) * 8 + warp) * D)[lane] = pq[t];
+                for (int u = 0; u < TG; ++u) {
+                    const int t = t0 + u;
+                    if (t < T) {
+                        reinterpret_cast<float4 *>(red + (t * 8 + warp) * D)[lane] = pk[u];
+                        reinterpret_cast<float4 *>(red + ((TMAX + t) * 8 + warp) * D)[lane] = pq[u];
+                    }
                 }
             }
         }
@@ -330,47 +397,70 @@ decode_stream_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
                             yv = fmaf(ratio * be[s2] * rk[s2] * rq[t] * gram[(3 * TMAX + t) * TMAX + s2], e[s2], yv);
                         }
                     }
-                    e_s[t * D + tid] = ev;
-                    y_s[t * D + tid] = yv;
+                    e_s[t * ES + tid] = ev;   // over slot w = 0, which this thread alone read
+                    y_s[t * ES + tid] = yv;
+                }
+            }
+            // the update's keys, (cum_nk / cum_{s+1}) beta_s k_s with unit-norm k_s
+            float ratio = 1.f;
+#pragma unroll
+            for (int s2 = TMAX - 1; s2 >= 0; --s2) {
+                if (s2 < nk) {
+                    kb[s2 * D + tid] = ratio * be[s2] * rk[s2] * xs[s2 * 384 + D + tid];
+                    ratio *= al[s2];
                 }
             }
         }
-        __syncthreads();   // e and y are complete
+        __syncthreads();   // e, y and kb are complete
         // ---- pass 2: the committed state
         //   S_nk = cum_nk S0 + sum_{s<nk} (cum_nk/cum_{s+1}) beta_s k_s e_s^T
         // from registers straight to HBM (nothing is written when nk = 0)
         if (nk > 0) {
-            float cs[TMAX];
-            float4 e4[TMAX];
-            float ratio = 1.f;
-#pragma unroll
-            for (int s2 = TMAX - 1; s2 >= 0; --s2) {
-                cs[s2] = 0.f;
-                if (s2 < nk) {
-                    cs[s2] = ratio * be[s2] * rk[s2];
-                    ratio *= al[s2];
-                }
-            }
-            const float decay = cum[0] * ratio;   // = cum_nk
+            float decay = 1.f;   // cum_nk
 #pragma unroll
             for (int s2 = 0; s2 < TMAX; ++s2)
-                e4[s2] = s2 < nk ? reinterpret_cast<const float4 *>(e_s + s2 * D)[lane] : make_float4(0.f, 0.f, 0.f, 0.f);
-            float4 *Sg = reinterpret_cast<float4 *>(S + gi * D * D);
+                if (s2 < nk) decay *= al[s2];
+            float2 e01[TMAX], e23[TMAX];
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                const int i = warp + 8 * r;
-                float4 o = make_float4(decay * sreg[r].x, decay * sreg[r].y, decay * sreg[r].z, decay * sreg[r].w);
+            for (int s2 = 0; s2 < TMAX; ++s2) {
+                const float4 e4 = s2 < nk ? reinterpret_cast<const float4 *>(e_s + s2 * ES)[lane]
+                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+                e01[s2] = make_float2(e4.x, e4.y);
+                e23[s2] = make_float2(e4.z, e4.w);
+            }
+            const float2 dec2 = make_float2(decay, decay);
+            float4 *Sg = reinterpret_cast<float4 *>(S + gi * D * D);
+            // row r of S' from the register state and the keys' entries bk[s2] at row r
+            auto store_row = [&](int r, const float (&bk)[TMAX]) {
+                float2 lo = fmul2(dec2, make_float2(sreg[r].x, sreg[r].y));
+                float2 hi = fmul2(dec2, make_float2(sreg[r].z, sreg[r].w));
 #pragma unroll
                 for (int s2 = 0; s2 < TMAX; ++s2) {
                     if (s2 < nk) {
-                        const float bk = cs[s2] * xs[s2 * 384 + D + i];
-                        o.x = fmaf(bk, e4[s2].x, o.x);
-                        o.y = fmaf(bk, e4[s2].y, o.y);
-                        o.z = fmaf(bk, e4[s2].z, o.z);
-                        o.w = fmaf(bk, e4[s2].w, o.w);
+                        const float2 b2 = make_float2(bk[s2], bk[s2]);
+                        lo = ffma2(b2, e01[s2], lo);
+                        hi = ffma2(b2, e23[s2], hi);
                     }
                 }
-                __stcs(Sg + tid + r * NT, o);
+                __stcs(Sg + row_of(r) * 32 + lane, make_float4(lo.x, lo.y, hi.x, hi.y));
+            };
+            if constexpr (TMAX == 1) {
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    const float4 kv = *reinterpret_cast<const float4 *>(kb + 16 * warp + 4 * g);
+                    store_row(4 * g + 0, {kv.x});
+                    store_row(4 * g + 1, {kv.y});
+                    store_row(4 * g + 2, {kv.z});
+                    store_row(4 * g + 3, {kv.w});
+                }
+            } else {
+#pragma unroll
+                for (int r = 0; r < 16; ++r) {
+                    float bk[TMAX];
+#pragma unroll
+                    for (int s2 = 0; s2 < TMAX; ++s2) bk[s2] = s2 < nk ? kb[s2 * D + row_of(r)] : 0.f;
+                    store_row(r, bk);
+                }
             }
         }
         // ---- outputs (warp 7)
@@ -380,20 +470,23 @@ decode_stream_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
                 if (t < T) {
                     float yv[4], ss = 0.f;
 #pragma unroll
-                    for (int m = 0; m < 4; ++m) { yv[m] = y_s[t * D + lane + 32 * m]; ss = fmaf(yv[m], yv[m], ss); }
+                    for (int m = 0; m < 4; ++m) { yv[m] = y_s[t * ES + lane + 32 * m]; ss = fmaf(yv[m], yv[m], ss); }
                     ss = group_sum<32>(ss);
                     const float rr = rsqrtf(ss / D + kNormEps);
                     const size_t go = (((size_t)b * T + t) * H + h) * D;
 #pragma unroll
                     for (int m = 0; m < 4; ++m) {
                         const int col = lane + 32 * m;
-                        out[go + col] = from_f32<Tout>(sigmoid_fast(zr[t][m]) * yv[m] * rr * (1.0f + __ldg(norm_w + col)));
+                        const float zv = __bfloat162float(zb[t * D + col]);
+                        out[go + col] = from_f32<Tout>(sigmoid_fast(zv) * yv[m] * rr * (1.0f + __ldg(norm_w + col)));
                     }
                 }
             }
         }
-        // No barrier here: the next item writes the other xs buffer before its
-        // first barrier, and red / gram / gate / e / y only after it.
+        // No barrier here: after the third barrier nothing reads xs, so the next
+        // item's prelude may overwrite it; red (with e and y), kb, gram and gate
+        // are written only after the next item's first barrier, which every
+        // thread reaches after its own reads here; zb is warp 7's alone.
     }
 }
 
@@ -409,7 +502,8 @@ cudaError_t launch_decode_stream(const DecodeArgs &a, int T, const int32_t *n_ke
     if (T < 1 || T > 4) return cudaErrorInvalidValue;
     const int items = a.B * a.H;
     if (items == 0) return cudaSuccess;
-    const int grid = items < sms ? items : sms;
+    const int per_sm = T == 1 && !n_keep ? dstream::Layout<1>::CTAS_PER_SM : dstream::Layout<4>::CTAS_PER_SM;
+    const int grid = items < sms * per_sm ? items : sms * per_sm;
 #define GDN_DSTREAM(TOUT, TM)                                                                      \
     e = cudaFuncSetAttribute(decode_stream_kernel<TOUT, TM>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                              dstream::Layout<TM>::SMEM);                                          \

@@ -64,12 +64,18 @@ PrepArgs prep_args(const PrefillArgs &a, const TcWorkspace &w) {
     return p;
 }
 
+// Tokens of the longest sequence, or their bound N_tok when cu_seqlens is given
+// (device memory, not read on the host).
+int longest_seq(const PrefillArgs &a) {
+    return a.cu_seqlens || a.n_seq <= 0 ? a.n_tok : a.n_tok / a.n_seq;
+}
+
 cudaError_t launch_chunk_prep(const PrefillArgs &a, const TcWorkspace &w, int c_lo, int c_hi,
                               cudaStream_t stream) {
     if (a.n_tok == 0 || c_hi <= c_lo) return cudaSuccess;
     // blocks per (head, sequence): ~8 per SM / H in total, at most one per chunk
     // of the range (the longest sequence may fill it); blocks past the end exit
-    const int max_chunks = (a.n_tok + 63) / 64;
+    const int max_chunks = (longest_seq(a) + 63) / 64;
     int sms = 0;
     if (cudaError_t es = sm_count(&sms)) return es;
     int split = max(1, (8 * sms) / a.H);
@@ -326,7 +332,7 @@ cudaError_t launch_prefill_fused(const PrefillArgs &a, const TcWorkspace &w, int
     P.n_seq = a.n_seq;
     P.n_tok = a.n_tok;
     P.H = a.H;
-    P.max_chunks = (a.n_tok + 63) / 64;
+    P.max_chunks = (longest_seq(a) + 63) / 64;
     P.n_chain = n_chain;
     P.ready = ready;
     P.next_task = ready + (size_t)a.n_seq * a.H * P.max_chunks;

@@ -15,12 +15,13 @@
 //  K5a qsa_prep_kernel: one warp per query row (all 4 heads) or key block:
 //      RMSNorm, rotation (the angle reduced in double precision: positions reach
 //      1e5 and more), fp16 rows [(i, h)][128] and [b][128].
-//  K5b qsa_score_kernel: tcgen05, one CTA of 8 warps per (32 queries = 128 rows
-//      of (i, h), 256 blocks): both operands by TMA in the 128-byte swizzled
-//      K-major layout, eight K = 16 MMAs into 256 TMEM columns; the epilogue
-//      (two warps per TMEM lane quadrant, half the columns each) applies ReLU,
-//      sums the 4 heads (lanes 4q .. 4q + 3) with two shuffles and stores the
-//      scores of complete blocks.  Tiles entirely past the causal limit do nothing.
+//  K5b qsa_score_kernel: tcgen05, persistent (one CTA per SM): a tile of 128
+//      queries x 4 heads stays in shared memory while 64-block tiles stream
+//      through three stages by TMA (128-byte swizzled, K-major); per block tile
+//      one M = 128, N = 64 product per head into its own TMEM columns, two TMEM
+//      stages; warp-specialised producer, MMA issuer and four epilogue warps
+//      (ReLU, head sum, 128-byte row segments of the complete blocks' scores).
+//      Only block tiles that hold a complete block of the query tile are visited.
 //  K5c qsa_topk_kernel: one CTA per query row: a radix select on the score bits
 //      (scores are >= 0, so their bit patterns order like the values; digits of
 //      11, 11 and 9 bits, the first counted while the row is read into shared
@@ -42,12 +43,6 @@ __device__ unsigned int g_qsa_err;
 
 namespace qsa {
 constexpr int D = 128, HI = 4, R = 4;
-constexpr int QT = 32;          // queries per score tile (128 MMA rows)
-constexpr int BT = 256;         // blocks per score tile (MMA N)
-constexpr int OFF_A = 0;        // 2 k-blocks x 128 rows x 128 B
-constexpr int OFF_B = 32768;    // 2 k-blocks x 256 rows x 128 B
-constexpr int OFF_BAR = 98304;
-constexpr int SMEM = OFF_BAR + 64 + 1024;
 constexpr double ROPE_BASE = 10000.0;
 }  // namespace qsa
 
@@ -113,7 +108,7 @@ qsa_prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const fl
 }
 
 // ------------------------------------------------------------------ K5b: scores
-// Bounded wait of the score kernel: false (and the device error word raised)
+// Bounded wait of the indexer kernels: false (and the device error word raised)
 // when the phase does not complete within max_polls polls.
 __device__ __forceinline__ bool qsa_wait(uint64_t *bar, uint32_t parity, uint32_t max_polls) {
     const bool ok = umma::mbar_wait_bounded(bar, parity, max_polls);
@@ -121,108 +116,259 @@ __device__ __forceinline__ bool qsa_wait(uint64_t *bar, uint32_t parity, uint32_
     return ok;
 }
 
-struct QsaMaps {
-    CUtensorMap q, k;   // [rows][128] fp16, box {64, 128} and {64, 256}, 128-byte swizzle
+namespace qsa {
+// Persistent score kernel.  A work item is (sequence s, query tile qt of QT
+// queries, a run of at most CH block tiles of BN blocks); items enumerate the
+// (s, qt) pairs in order and cut each query tile's block tiles into runs of CH.
+constexpr int QT = 128;                  // queries per tile (TMEM lanes)
+constexpr int BN = 64;                   // blocks per block tile (MMA N, per head)
+constexpr int CH = 8;                    // block tiles per work item at most
+constexpr int NSB = 3;                   // block-tile stages in shared memory
+constexpr int A_HEAD = 2 * 16384;        // one head's query tile: 2 k-blocks x [128 rows x 128 B]
+constexpr int B_STAGE = 2 * 8192;        // one block tile: 2 k-blocks x [64 rows x 128 B]
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + HI * A_HEAD;             // 131072
+constexpr int OFF_BAR = OFF_B + NSB * B_STAGE;         // 180224
+constexpr int SMEM = OFF_BAR + 256 + 1024;             // barriers, TMEM slot, abort flag; alignment slack
+constexpr uint32_t TMEM_COLS = 512;                    // 2 stages x 4 heads x 64 columns
+constexpr uint32_t MAX_POLLS = 1u << 24;
+}  // namespace qsa
+
+namespace {
+
+__device__ __forceinline__ void mbar_arrive_local(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(umma::smem_u32(bar)) : "memory");
+}
+
+struct QsaItem {
+    int s, qt, bt0, nbt;
 };
 
-__global__ void __launch_bounds__(256, 1)
-qsa_score_kernel(const __grid_constant__ QsaMaps maps, int n, float *__restrict__ scores) {
+// block tiles of query tile qt: those holding a block complete for its last query
+__host__ __device__ __forceinline__ int qsa_tiles_of(int n, int qt) {
+    const int last = min(qsa::QT * qt + qsa::QT - 1, n - 1);
+    return ((last + 1) / qsa::R + qsa::BN - 1) / qsa::BN;
+}
+
+// Item `it` of the enumeration; every role walks the same increasing item
+// indices, so the cursor (first item of the current (s, qt)) only moves forward.
+struct QsaCursor {
+    int s = 0, qt = 0, first = 0;
+};
+
+__device__ __forceinline__ bool qsa_find_item(int it, int B, int n, QsaCursor &c, QsaItem &out) {
+    const int n_qt = (n + qsa::QT - 1) / qsa::QT;
+    while (c.s < B) {
+        const int nbt = qsa_tiles_of(n, c.qt);
+        const int k = (nbt + qsa::CH - 1) / qsa::CH;
+        if (it < c.first + k) {
+            const int j = it - c.first;
+            out.s = c.s;
+            out.qt = c.qt;
+            out.bt0 = j * qsa::CH;
+            out.nbt = min(qsa::CH, nbt - out.bt0);
+            return true;
+        }
+        c.first += k;
+        if (++c.qt == n_qt) {
+            c.qt = 0;
+            ++c.s;
+        }
+    }
+    return false;
+}
+
+}  // namespace
+
+struct QsaMaps {
+    CUtensorMap q;   // [B n][4][128] fp16, box {64, 1, 128}, 128-byte swizzle
+    CUtensorMap k;   // [B nb][1][128] fp16, box {64, 1, 64}
+};
+
+// One CTA per SM walks the work items.  The four heads' query rows of the tile
+// (4 x 128 rows x 128 dims fp16 = 128 KB) stay in shared memory for the item;
+// block tiles (64 x 128 fp16 = 16 KB) stream through NSB stages.  Each head's
+// product (M = 128 queries, N = 64 blocks, K = 128) goes to its own 64 TMEM
+// columns, so the epilogue sums ReLU over the heads per (query lane, block
+// column) with no shuffles; two TMEM stages let the MMAs of block tile j + 1 run
+// while tile j's epilogue drains.
+// Roles: warp 0 lane 0 issues the TMA loads, warp 1 lane 0 the MMAs (warp 1 owns
+// the TMEM allocation), warps 2-5 are the epilogue (TMEM lane quadrant w % 4,
+// one query per lane, 128-byte row segments of scores).  Barriers: full_a /
+// empty_a (query tile), full_b / empty_b (block stages), tfull / tempty (TMEM
+// stages; tempty takes one arrival per epilogue warp).  Every wait is bounded;
+// a timeout raises the error word and an abort flag the other roles check.
+__global__ void __launch_bounds__(192, 1)
+qsa_score_kernel(const __grid_constant__ QsaMaps maps, int B, int n, int n_items, float *__restrict__ scores) {
     using namespace qsa;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = umma::align_smem<1024>(smem_raw);
-    uint64_t *bar_ld = reinterpret_cast<uint64_t *>(sm + OFF_BAR);        // operand loads
-    uint64_t *bar_mma = reinterpret_cast<uint64_t *>(sm + OFF_BAR + 8);   // MMA completion
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 16);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
+    uint64_t *full_a = bars, *empty_a = bars + 1;
+    uint64_t *full_b = bars + 2, *empty_b = bars + 2 + NSB;
+    uint64_t *tfull = bars + 2 + 2 * NSB, *tempty = bars + 4 + 2 * NSB;
+    uint64_t *mma_done = bars + 6 + 2 * NSB;   // teardown after an abort: issued MMAs completed
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + 7 + 2 * NSB);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nb = n / R;
-    const int bt = blockIdx.x, qt = blockIdx.y, s = blockIdx.z;
-    const int i_last = min(QT * qt + QT - 1, n - 1);
-    // complete blocks of the tile's last query; nothing to do past them
-    if (BT * bt >= (i_last + 1) / R) return;   // uniform per CTA
 
-    if (warp == 0) umma::tmem_alloc(tslot, BT);
     if (tid == 0) {
-        umma::mbar_init(bar_ld, 1);
-        umma::mbar_init(bar_mma, 1);
+        umma::mbar_init(full_a, 1);
+        umma::mbar_init(empty_a, 1);
+        for (int i = 0; i < NSB; ++i) {
+            umma::mbar_init(full_b + i, 1);
+            umma::mbar_init(empty_b + i, 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            umma::mbar_init(tfull + i, 1);
+            umma::mbar_init(tempty + i, 4);
+        }
+        umma::mbar_init(mma_done, 1);
+        *abort_flag = 0;
         umma::fence_mbar_init();
     }
+    if (warp == 1) umma::tmem_alloc(tslot, TMEM_COLS);
     umma::tc_fence_before();
     __syncthreads();
     umma::tc_fence_after();
     const uint32_t tbase = *tslot;
-    bool ok = true;
-    if (tid == 0) {
-        umma::mbar_expect_tx(bar_ld, 2 * 128 * 128 + 2 * 256 * 128);
-        const int qrow = (s * n + QT * qt) * HI, krow = s * nb + BT * bt;
-#pragma unroll
-        for (int kb = 0; kb < 2; ++kb) {
-            umma::tma_load_3d(sm + OFF_A + kb * 16384, &maps.q, 64 * kb, 0, qrow, bar_ld);
-            umma::tma_load_3d(sm + OFF_B + kb * 32768, &maps.k, 64 * kb, 0, krow, bar_ld);
+
+    auto wait = [&](uint64_t *bar, uint32_t parity) -> bool {
+        if (*abort_flag) return false;
+        if (qsa_wait(bar, parity, MAX_POLLS)) return true;
+        *abort_flag = 1;
+        return false;
+    };
+
+    if (warp == 0 && lane == 0) {
+        // ---------------------------------------------------------------- producer
+        QsaCursor cur;
+        QsaItem item;
+        int a_it = 0, b_it = 0;
+        bool ok = true;
+        for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+            if (!qsa_find_item(it, B, n, cur, item)) break;
+            if (!(ok = wait(empty_a, (a_it + 1) & 1))) break;
+            umma::mbar_expect_tx(full_a, HI * A_HEAD);
+            for (int h = 0; h < HI; ++h)
+                for (int kb = 0; kb < 2; ++kb)
+                    umma::tma_load_3d(sm + OFF_A + h * A_HEAD + kb * 16384, &maps.q, 64 * kb, h,
+                                      item.s * n + QT * item.qt, full_a);
+            ++a_it;
+            for (int j = 0; j < item.nbt; ++j, ++b_it) {
+                const int st = b_it % NSB, u = b_it / NSB;
+                if (!(ok = wait(empty_b + st, (u + 1) & 1))) break;
+                umma::mbar_expect_tx(full_b + st, B_STAGE);
+                for (int kb = 0; kb < 2; ++kb)
+                    umma::tma_load_3d(sm + OFF_B + st * B_STAGE + kb * 8192, &maps.k, 64 * kb, 0,
+                                      item.s * nb + BN * (item.bt0 + j), full_b + st);
+            }
         }
-        ok = qsa_wait(bar_ld, 0, 1u << 24);
-        if (ok) {
-            umma::tc_fence_after();
-            const uint32_t a = umma::smem_u32(sm + OFF_A), b = umma::smem_u32(sm + OFF_B);
-            const uint32_t idesc = umma::idesc_f16(128, BT, false, false);
-#pragma unroll
-            for (int st = 0; st < D / 16; ++st) {
-                const uint64_t ad = umma::sw128_desc(a + (st / 4) * 16384 + (st % 4) * 32, 16, 1024);
-                const uint64_t bd = umma::sw128_desc(b + (st / 4) * 32768 + (st % 4) * 32, 16, 1024);
-                umma::mma_f16(tbase, ad, bd, idesc, st > 0);
-            }
-            umma::mma_commit(bar_mma);
+        // after an abort, loads still in flight land before the CTA leaves
+        if (*abort_flag) {
+            if (a_it > 0) umma::mbar_wait_bounded(full_a, (a_it - 1) & 1, MAX_POLLS);
+            for (int k = max(0, b_it - NSB); k < b_it; ++k)
+                umma::mbar_wait_bounded(full_b + k % NSB, (k / NSB) & 1, MAX_POLLS);
         }
-    }
-    ok = __syncthreads_and(ok);   // the MMA was issued
-    if (ok) ok = __syncthreads_and(qsa_wait(bar_mma, 0, 1u << 24));
-    if (ok) {
-        umma::tc_fence_after();
-        // warps w and w + 4: TMEM lanes 32 (w % 4) .. + 31 = rows (query 8 (w % 4) + l / 4,
-        // head l % 4); warp w takes block columns 128 (w / 4) .. + 127
-        const int quad = warp & 3, half = warp >> 2;
-        const int i = QT * qt + 8 * quad + (lane >> 2);
-        const int n_valid = (i + 1) / R;   // complete blocks of query i
-        const uint32_t trow = tbase + ((uint32_t)(32 * quad) << 16);
-        float *dst = scores + ((size_t)s * n + i) * nb;
-        const bool vec = (nb & 3) == 0;   // rows start on 16-byte boundaries
-#pragma unroll 1
-        for (int c0 = (BT / 2) * half; c0 < (BT / 2) * (half + 1); c0 += 32) {
-            if (BT * bt + c0 >= (i_last + 1) / R) break;   // uniform: nothing valid past here
-            float v[32];
-            umma::tmem_ld32(trow + c0, v);
+    } else if (warp == 1 && lane == 0) {
+        // --------------------------------------------------------------- MMA issuer
+        QsaCursor cur;
+        QsaItem item;
+        int a_it = 0, t_it = 0;
+        bool ok = true;
+        const uint32_t idesc = umma::idesc_f16(128, BN, false, false);
+        const uint32_t a0 = umma::smem_u32(sm + OFF_A), b0 = umma::smem_u32(sm + OFF_B);
+        for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+            if (!qsa_find_item(it, B, n, cur, item)) break;
+            if (!(ok = wait(full_a, a_it & 1))) break;
+            for (int j = 0; j < item.nbt; ++j, ++t_it) {
+                const int st = t_it % NSB, u = t_it / NSB;
+                const int ts = t_it & 1, v = t_it >> 1;
+                if (!(ok = wait(full_b + st, u & 1))) break;
+                if (!(ok = wait(tempty + ts, (v + 1) & 1))) break;
+                umma::tc_fence_after();
+                for (int h = 0; h < HI; ++h) {
+                    const uint32_t d = tbase + ts * (HI * BN) + h * BN;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                float x = fmaxf(v[j], 0.f);
-                x += __shfl_xor_sync(0xffffffffu, x, 1);
-                x += __shfl_xor_sync(0xffffffffu, x, 2);
-                v[j] = x;
-            }
-            // the 4 lanes of a query hold the same sums: lane 4q + j stores scores
-            // 8j .. 8j + 7 of the chunk (two 16-byte stores when rows are aligned)
-            const int j8 = 8 * (lane & 3);
-            float o[8];
-#pragma unroll
-            for (int x = 0; x < 8; ++x) {
-                const float a0 = v[x], a1 = v[8 + x], a2 = v[16 + x], a3 = v[24 + x];
-                o[x] = j8 == 0 ? a0 : (j8 == 8 ? a1 : (j8 == 16 ? a2 : a3));
-            }
-            const int b0 = BT * bt + c0 + j8;
-            if (i < n) {
-                if (vec && b0 + 8 <= n_valid) {
-                    float4 *d4 = reinterpret_cast<float4 *>(dst + b0);
-                    d4[0] = make_float4(o[0], o[1], o[2], o[3]);
-                    d4[1] = make_float4(o[4], o[5], o[6], o[7]);
-                } else {
-#pragma unroll
-                    for (int x = 0; x < 8; ++x)
-                        if (b0 + x < n_valid) dst[b0 + x] = o[x];
+                    for (int k = 0; k < D / 16; ++k) {
+                        const uint64_t ad = umma::sw128_desc(a0 + h * A_HEAD + (k / 4) * 16384 + (k % 4) * 32, 16, 1024);
+                        const uint64_t bd = umma::sw128_desc(b0 + st * B_STAGE + (k / 4) * 8192 + (k % 4) * 32, 16, 1024);
+                        umma::mma_f16(d, ad, bd, idesc, k > 0);
+                    }
                 }
+                umma::mma_commit(empty_b + st);
+                umma::mma_commit(tfull + ts);
+            }
+            if (!ok) break;
+            umma::mma_commit(empty_a);
+            ++a_it;
+        }
+        // after an abort the epilogue may not have waited for the last MMAs: they
+        // complete before the tensor memory is released
+        if (t_it > 0 && *abort_flag) {
+            umma::mma_commit(mma_done);
+            umma::mbar_wait_bounded(mma_done, 0, MAX_POLLS);
+        }
+    } else if (warp >= 2) {
+        // ----------------------------------------------------------------- epilogue
+        const int qd = warp & 3;
+        const uint32_t trow = tbase + ((uint32_t)(32 * qd) << 16);
+        const bool vec = (nb & 3) == 0;   // rows start on 16-byte boundaries
+        QsaCursor cur;
+        QsaItem item;
+        int t_it = 0;
+        bool ok = true;
+        for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+            if (!qsa_find_item(it, B, n, cur, item)) break;
+            const int i = QT * item.qt + 32 * qd + lane;   // this lane's query
+            const int n_valid = i < n ? (i + 1) / R : 0;  // its complete blocks
+            float *dst = scores + ((size_t)item.s * n + (i < n ? i : 0)) * nb;
+            for (int j = 0; j < item.nbt; ++j, ++t_it) {
+                const int ts = t_it & 1, v = t_it >> 1;
+                ok = __all_sync(0xffffffffu, wait(tfull + ts, v & 1));
+                if (!ok) break;
+                umma::tc_fence_after();
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 32) {
+                    float acc[32], x[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) acc[e] = 0.f;
+#pragma unroll
+                    for (int h = 0; h < HI; ++h) {
+                        umma::tmem_ld32(trow + ts * (HI * BN) + h * BN + c, x);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) acc[e] += fmaxf(x[e], 0.f);
+                    }
+                    const int bs = BN * (item.bt0 + j) + c;
+                    if (vec && bs + 32 <= n_valid) {
+                        float4 *d4 = reinterpret_cast<float4 *>(dst + bs);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            d4[e] = make_float4(acc[4 * e], acc[4 * e + 1], acc[4 * e + 2], acc[4 * e + 3]);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (bs + e < n_valid) dst[bs + e] = acc[e];
+                    }
+                }
+                umma::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_local(tempty + ts);
             }
         }
     }
     umma::tc_fence_before();
     __syncthreads();
-    if (warp == 0) umma::tmem_dealloc(tbase, BT);
+    if (warp == 1) umma::tmem_dealloc(tbase, TMEM_COLS);
+}
+
+// Work items of the score kernel for B sequences of n tokens.
+long long qsa_score_items(int B, int n) {
+    const int n_qt = (n + qsa::QT - 1) / qsa::QT;
+    long long total = 0;
+    for (int qt = 0; qt < n_qt; ++qt) total += (qsa_tiles_of(n, qt) + qsa::CH - 1) / qsa::CH;
+    return total * B;
 }
 
 // ------------------------------------------------------------------ K5c: top-k
@@ -483,15 +629,18 @@ cudaError_t launch_qsa_indexer(const QsaArgs &a, void *ws) {
     if (nb > 0) {
         QsaMaps m;
         std::memset(&m, 0, sizeof m);
-        if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.q), qr, false, D, 1, a.B * a.n * HI, 64, 128, true)) != cudaSuccess)
+        if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.q), qr, false, D, HI, a.B * a.n, 64, QT, true)) != cudaSuccess)
             return e;
-        if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.k), kb, false, D, 1, a.B * nb, 64, BT, true)) != cudaSuccess)
+        if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.k), kb, false, D, 1, a.B * nb, 64, BN, true)) != cudaSuccess)
             return e;
         if ((e = cudaFuncSetAttribute(qsa_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM)) != cudaSuccess)
             return e;
-        const dim3 g((nb + BT - 1) / BT, (a.n + QT - 1) / QT, a.B);
-        qsa_score_kernel<<<g, 256, SMEM, a.stream>>>(m, a.n, scores);
-        if ((e = launched()) != cudaSuccess) return e;
+        const long long n_items = qsa_score_items(a.B, a.n);
+        const int g = (int)(n_items < sms ? n_items : sms);
+        if (g > 0) {
+            qsa_score_kernel<<<g, 192, SMEM, a.stream>>>(m, a.B, a.n, (int)n_items, scores);
+            if ((e = launched()) != cudaSuccess) return e;
+        }
     }
     if (a.n > 0) {
         // the row's keys, rounded up to whole 16-byte quads
