@@ -65,6 +65,7 @@ cudaError_t launch_chunk_chain(const PrefillArgs &a, const TcWorkspace &w, int c
 struct TmaMap { alignas(64) unsigned char bytes[128]; };
 cudaError_t make_tma_3d(TmaMap *out, const void *base, bool bf16, int inner, int H, int n_tok,
                         int box_inner, int box_rows, bool swizzle128);
+cudaError_t make_tma_rows_f32(TmaMap *out, const void *base, int cols, int rows, int box_cols, int box_rows);
 
 // K4: prefill backward (fp32 inputs, dk = dv in {64, 128}); `f` holds the forward's
 // inputs (f.out and f.S_final are unused), the rest the incoming and outgoing

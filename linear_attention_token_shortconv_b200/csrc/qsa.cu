@@ -19,15 +19,16 @@
 //      queries x 4 heads stays in shared memory while 64-block tiles stream
 //      through three stages by TMA (128-byte swizzled, K-major); per block tile
 //      one M = 128, N = 64 product per head into its own TMEM columns, two TMEM
-//      stages; warp-specialised producer, MMA issuer and four epilogue warps
+//      stages; warp-specialised producer, MMA issuer and eight epilogue warps
 //      (ReLU, head sum, 128-byte row segments of the complete blocks' scores).
 //      Only block tiles that hold a complete block of the query tile are visited.
-//  K5c qsa_topk_kernel: one CTA per query row: a radix select on the score bits
-//      (scores are >= 0, so their bit patterns order like the values; digits of
-//      11, 11 and 9 bits, the first counted while the row is read into shared
-//      memory, stopping at the first digit whose bucket is taken whole) finds the
-//      threshold, then warp segments write the selected blocks in ascending
-//      order, equal scores at the threshold taken from the smallest index.
+//  K5c qsa_topk_kernel: one warp per query row, no block barriers: a radix
+//      select on the score bits (scores are >= 0, so their bit patterns order
+//      like the values; digits of 11, 11 and 9 bits counted in the warp's own
+//      shared histogram, stopping at the first digit whose bucket is taken
+//      whole) finds the threshold, then one walk over the row in index order
+//      writes the selected blocks ascending, equal scores at the threshold taken
+//      from the smallest index.
 #include <cuda.h>
 #include <cuda_fp16.h>
 
@@ -128,7 +129,10 @@ constexpr int A_HEAD = 2 * 16384;        // one head's query tile: 2 k-blocks x 
 constexpr int B_STAGE = 2 * 8192;        // one block tile: 2 k-blocks x [64 rows x 128 B]
 constexpr int OFF_A = 0;
 constexpr int OFF_B = OFF_A + HI * A_HEAD;             // 131072
-constexpr int OFF_BAR = OFF_B + NSB * B_STAGE;         // 180224
+constexpr int EPI_WARPS = 8;             // two per TMEM lane quadrant, one 32-column half each
+constexpr int OFF_STG = OFF_B + NSB * B_STAGE;         // 180224: per epilogue warp, a 32 x 32 fp32 store tile
+constexpr int STG_TILE = 32 * 32 * 4;
+constexpr int OFF_BAR = OFF_STG + EPI_WARPS * STG_TILE;   // 212992
 constexpr int SMEM = OFF_BAR + 256 + 1024;             // barriers, TMEM slot, abort flag; alignment slack
 constexpr uint32_t TMEM_COLS = 512;                    // 2 stages x 4 heads x 64 columns
 constexpr uint32_t MAX_POLLS = 1u << 24;
@@ -183,6 +187,7 @@ __device__ __forceinline__ bool qsa_find_item(int it, int B, int n, QsaCursor &c
 struct QsaMaps {
     CUtensorMap q;   // [B n][4][128] fp16, box {64, 1, 128}, 128-byte swizzle
     CUtensorMap k;   // [B nb][1][128] fp16, box {64, 1, 64}
+    CUtensorMap sc;  // scores [B n][1][nb] fp32, box {32, 1, 32}, 128-byte swizzle (when nb % 4 == 0)
 };
 
 // One CTA per SM walks the work items.  The four heads' query rows of the tile
@@ -193,13 +198,18 @@ struct QsaMaps {
 // column) with no shuffles; two TMEM stages let the MMAs of block tile j + 1 run
 // while tile j's epilogue drains.
 // Roles: warp 0 lane 0 issues the TMA loads, warp 1 lane 0 the MMAs (warp 1 owns
-// the TMEM allocation), warps 2-5 are the epilogue (TMEM lane quadrant w % 4,
-// one query per lane, 128-byte row segments of scores).  Barriers: full_a /
+// the TMEM allocation), warps 2-9 are the epilogue (TMEM lane quadrant w % 4, one
+// query per lane; warps 2-5 take block columns 0-31 of each tile, warps 6-9
+// columns 32-63).  A 32-query x 32-block piece whose blocks are all complete for
+// its 32 queries leaves by one TMA store from the warp's swizzled tile; pieces on
+// the causal edge or past the sequence's end are stored lane by lane, complete
+// blocks only.  Barriers: full_a /
 // empty_a (query tile), full_b / empty_b (block stages), tfull / tempty (TMEM
 // stages; tempty takes one arrival per epilogue warp).  Every wait is bounded;
 // a timeout raises the error word and an abort flag the other roles check.
-__global__ void __launch_bounds__(192, 1)
-qsa_score_kernel(const __grid_constant__ QsaMaps maps, int B, int n, int n_items, float *__restrict__ scores) {
+__global__ void __launch_bounds__(64 + 32 * qsa::EPI_WARPS, 1)
+qsa_score_kernel(const __grid_constant__ QsaMaps maps, int B, int n, int n_items, bool tma_out,
+                 float *__restrict__ scores) {
     using namespace qsa;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = umma::align_smem<1024>(smem_raw);
@@ -222,7 +232,7 @@ qsa_score_kernel(const __grid_constant__ QsaMaps maps, int B, int n, int n_items
         }
         for (int i = 0; i < 2; ++i) {
             umma::mbar_init(tfull + i, 1);
-            umma::mbar_init(tempty + i, 4);
+            umma::mbar_init(tempty + i, EPI_WARPS);
         }
         umma::mbar_init(mma_done, 1);
         *abort_flag = 0;
@@ -312,36 +322,56 @@ qsa_score_kernel(const __grid_constant__ QsaMaps maps, int B, int n, int n_items
         }
     } else if (warp >= 2) {
         // ----------------------------------------------------------------- epilogue
-        const int qd = warp & 3;
+        const int qd = warp & 3, c = 32 * ((warp - 2) >> 2);   // lane quadrant, column half
         const uint32_t trow = tbase + ((uint32_t)(32 * qd) << 16);
         const bool vec = (nb & 3) == 0;   // rows start on 16-byte boundaries
+        float *tile = reinterpret_cast<float *>(sm + OFF_STG + (warp - 2) * STG_TILE);
         QsaCursor cur;
         QsaItem item;
         int t_it = 0;
         bool ok = true;
         for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
             if (!qsa_find_item(it, B, n, cur, item)) break;
-            const int i = QT * item.qt + 32 * qd + lane;   // this lane's query
-            const int n_valid = i < n ? (i + 1) / R : 0;  // its complete blocks
+            const int i0 = QT * item.qt + 32 * qd;            // this warp's first query
+            const int i = i0 + lane;                          // this lane's query
+            const int n_valid = i < n ? (i + 1) / R : 0;      // its complete blocks
+            const int n_full = i0 + 31 < n ? (i0 + 1) / R : 0;   // blocks complete for all 32 queries
             float *dst = scores + ((size_t)item.s * n + (i < n ? i : 0)) * nb;
             for (int j = 0; j < item.nbt; ++j, ++t_it) {
                 const int ts = t_it & 1, v = t_it >> 1;
                 ok = __all_sync(0xffffffffu, wait(tfull + ts, v & 1));
                 if (!ok) break;
                 umma::tc_fence_after();
-#pragma unroll 1
-                for (int c = 0; c < BN; c += 32) {
-                    float acc[32], x[32];
+                {
+                    // the four heads' columns in flight together, one wait
+                    uint32_t x[HI][32];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) acc[e] = 0.f;
+                    for (int h = 0; h < HI; ++h) umma::tmem_ld32_nowait(trow + ts * (HI * BN) + h * BN + c, x[h]);
+                    umma::tmem_wait_ld();
+                    float acc[32];
 #pragma unroll
-                    for (int h = 0; h < HI; ++h) {
-                        umma::tmem_ld32(trow + ts * (HI * BN) + h * BN + c, x);
+                    for (int e = 0; e < 32; ++e) {
+                        float a = fmaxf(__uint_as_float(x[0][e]), 0.f);
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) acc[e] += fmaxf(x[e], 0.f);
+                        for (int h = 1; h < HI; ++h) a += fmaxf(__uint_as_float(x[h][e]), 0.f);
+                        acc[e] = a;
                     }
                     const int bs = BN * (item.bt0 + j) + c;
-                    if (vec && bs + 32 <= n_valid) {
+                    if (tma_out && bs + 32 <= n_full) {   // uniform across the warp
+                        if (lane == 0) umma::bulk_wait_read<0>();   // the last store has read the tile
+                        __syncwarp();
+                        // row `lane`, 16-byte chunk e at chunk e ^ (lane % 8): the 128-byte swizzle
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            reinterpret_cast<float4 *>(tile + lane * 32)[e ^ (lane & 7)] =
+                                make_float4(acc[4 * e], acc[4 * e + 1], acc[4 * e + 2], acc[4 * e + 3]);
+                        umma::fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            umma::tma_store_3d(&maps.sc, bs, 0, item.s * n + i0, tile);
+                            umma::bulk_commit();
+                        }
+                    } else if (vec && bs + 32 <= n_valid) {
                         float4 *d4 = reinterpret_cast<float4 *>(dst + bs);
 #pragma unroll
                         for (int e = 0; e < 8; ++e)
@@ -357,6 +387,7 @@ qsa_score_kernel(const __grid_constant__ QsaMaps maps, int B, int n, int n_items
                 if (lane == 0) mbar_arrive_local(tempty + ts);
             }
         }
+        if (lane == 0) umma::bulk_wait_all();   // the last stores have left shared memory
     }
     umma::tc_fence_before();
     __syncthreads();
@@ -373,229 +404,214 @@ long long qsa_score_items(int B, int n) {
 
 // ------------------------------------------------------------------ K5c: top-k
 namespace qsa {
-constexpr int TOPK_CAP = 12288;      // row keys kept in shared memory up to this many blocks (48 KB)
-constexpr int HB = 2048;             // buckets of the 11-bit digits
-constexpr int HB_SLOTS = HB + HB / 32;   // with one pad counter per 32
+constexpr int HB = 2048;                  // buckets of the 11-bit digits
+constexpr int WH_SLOTS = HB + HB / 64;    // one warp's counters, one pad word per 64
+constexpr int TOPK_WARPS = 8;             // rows (warps) per CTA
 }  // namespace qsa
-
-// Counter of the bucket at descending rank u (u = NB - 1 - digit): one pad word
-// per 32 counters, so the PER consecutive ranks that each thread of a warp scans
-// fall in distinct banks (thread t reads ranks PER t .. PER t + PER - 1).
-__device__ __forceinline__ int topk_slot(int u) { return u + (u >> 5); }
-
-// One digit of the radix select: among the keys matching `prefix`, the bucket of
-// the digit at `shift` (NB buckets) that holds the remaining-th largest key.
-// Thread t sums the buckets of ranks PER t .. PER t + PER - 1 (descending
-// digits); a block scan of those sums crosses `remaining` at exactly one thread,
-// which walks its buckets and publishes the extended prefix, the rank left
-// inside the bucket and the bucket's count.  Ends with a block barrier.
-template <int NB>
-__device__ __forceinline__ void topk_pick(const int *hist, int *wsum, int remaining, unsigned prefix, int shift,
-                                          int tid, unsigned *sh_prefix, int *sh_rem, int *sh_cnt) {
-    constexpr int PER = NB / 256;
-    const int warp = tid >> 5, lane = tid & 31;
-    int c = 0;
-#pragma unroll
-    for (int j = 0; j < PER; ++j) c += hist[topk_slot(PER * tid + j)];
-    int incl = c;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-    }
-    if (lane == 31) wsum[warp] = incl;
-    __syncthreads();
-    for (int w = 0; w < warp; ++w) incl += wsum[w];
-    int run = incl - c;
-    if (incl >= remaining && run < remaining) {
-#pragma unroll
-        for (int j = 0; j < PER; ++j) {
-            const int h = hist[topk_slot(PER * tid + j)];
-            if (run + h >= remaining) {
-                *sh_prefix = prefix | ((unsigned)(NB - 1 - (PER * tid + j)) << shift);
-                *sh_rem = remaining - run;
-                *sh_cnt = h;
-                break;
-            }
-            run += h;
-        }
-    }
-    __syncthreads();
-}
 
 __device__ __forceinline__ unsigned topk_key(float v) {
     return v > 0.f ? __float_as_uint(v) : 0u;   // scores >= 0: bits order like values (-0 -> 0)
 }
 
-// Shared state of one row's select.
-struct TopkSmem {
-    int hist[qsa::HB_SLOTS];
-    int wsum[8];
-    int wcnt[8][2];
-    unsigned prefix;
-    int rem, cnt;
-};
+// Counter of the bucket at descending rank u (u = NB - 1 - digit).  With one pad
+// word per 64 counters, the 64 consecutive ranks each lane sums in a pick of the
+// 11-bit digit fall in distinct banks across the warp.
+__device__ __forceinline__ int topk_slot(int u) { return u + (u >> 6); }
 
-// Histogram of the digit (key >> shift) & (NB - 1) over the keys with
-// (key & mask) == prefix; SMEM: the keys are in shared memory (read 16 bytes at
-// a time), else they are read from the score row.
-template <bool SMEM, int NB>
-__device__ __forceinline__ void topk_count(TopkSmem &S, const uint4 *keys4, const float *sc, int n_valid,
-                                           unsigned mask, unsigned prefix, int shift, int tid) {
-    if (SMEM) {
-        const int n4 = (n_valid + 3) >> 2;
-        for (int q = tid; q < n4; q += 256) {
-            const uint4 kk = keys4[q];
-            const unsigned k[4] = {kk.x, kk.y, kk.z, kk.w};
+__device__ __forceinline__ int warp_incl_scan(int x, int lane) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                if (4 * q + j < n_valid && (k[j] & mask) == prefix)
-                    atomicAdd(&S.hist[topk_slot(NB - 1 - (int)((k[j] >> shift) & (NB - 1)))], 1);
-        }
-    } else {
-        for (int b = tid; b < n_valid; b += 256) {
-            const unsigned key = topk_key(sc[b]);
-            if ((key & mask) == prefix) atomicAdd(&S.hist[topk_slot(NB - 1 - (int)((key >> shift) & (NB - 1)))], 1);
-        }
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
     }
+    return x;
 }
 
-template <bool SMEM>
-__device__ __forceinline__ void topk_row(TopkSmem &S, uint4 *keys4, const float *__restrict__ sc, int nb,
-                                         int n_valid, int KB, int32_t *__restrict__ out, int tid) {
-    unsigned *keys_s = reinterpret_cast<unsigned *>(keys4);
-    const int warp = tid >> 5, lane = tid & 31;
-    for (int j = tid; j < qsa::HB_SLOTS; j += 256) S.hist[j] = 0;
-    __syncthreads();
-    // The keys (into shared memory when they fit) and the histogram of their first
-    // digit, bits 30..20 (bit 31 of a key is 0).  Rows start on 16-byte boundaries
-    // when nb % 4 == 0; the last quad may reach past n_valid, never past the row.
-    if (SMEM && (nb & 3) == 0) {
-        const float4 *sc4 = reinterpret_cast<const float4 *>(sc);
-        const int n4 = (n_valid + 3) >> 2;
-        for (int q = tid; q < n4; q += 256) {
-            const float4 v = sc4[q];
-            const unsigned k[4] = {topk_key(v.x), topk_key(v.y), topk_key(v.z), topk_key(v.w)};
-            keys4[q] = make_uint4(k[0], k[1], k[2], k[3]);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                if (4 * q + j < n_valid) atomicAdd(&S.hist[topk_slot(qsa::HB - 1 - (int)(k[j] >> 20))], 1);
-        }
-    } else {
-        for (int b = tid; b < n_valid; b += 256) {
-            const unsigned key = topk_key(sc[b]);
-            if (SMEM) keys_s[b] = key;
-            atomicAdd(&S.hist[topk_slot(qsa::HB - 1 - (int)(key >> 20))], 1);
-        }
-    }
-    __syncthreads();
-    // Radix select of the KB-th largest key with digits of 11, 11 and 9 bits.  A
-    // digit whose bucket holds exactly the keys still wanted ends it early: every
-    // key of that bucket is taken, so the lower bits need not be resolved.
-    topk_pick<qsa::HB>(S.hist, S.wsum, KB, 0u, 20, tid, &S.prefix, &S.rem, &S.cnt);
-    unsigned prefix = S.prefix, mask = 0xFFF00000u;
-    int remaining = S.rem;
-    if (S.cnt != remaining) {   // uniform
-        for (int j = tid; j < qsa::HB_SLOTS; j += 256) S.hist[j] = 0;
-        __syncthreads();
-        topk_count<SMEM, qsa::HB>(S, keys4, sc, n_valid, mask, prefix, 9, tid);
-        __syncthreads();
-        topk_pick<qsa::HB>(S.hist, S.wsum, remaining, prefix, 9, tid, &S.prefix, &S.rem, &S.cnt);
-        prefix = S.prefix;
-        remaining = S.rem;
-        mask = 0xFFFFFE00u;
-        if (S.cnt != remaining) {
-            for (int j = tid; j < topk_slot(512); j += 256) S.hist[j] = 0;
-            __syncthreads();
-            topk_count<SMEM, 512>(S, keys4, sc, n_valid, mask, prefix, 0, tid);
-            __syncthreads();
-            topk_pick<512>(S.hist, S.wsum, remaining, prefix, 0, tid, &S.prefix, &S.rem, &S.cnt);
-            prefix = S.prefix;
-            remaining = S.rem;
-            mask = 0xFFFFFFFFu;
-        }
-    }
-    // Selection: the keys whose masked bits are above the prefix, and the first
-    // `remaining` equal to it in index order.  Warp w owns a contiguous segment of
-    // the row (starting on a multiple of 32 when not empty); it counts its keys
-    // above and equal, the warps exchange counts once, and each warp then writes
-    // its selected blocks at their ascending positions.
-    auto key_at = [&](int b) -> unsigned { return SMEM ? keys_s[b] : topk_key(sc[b]); };
-    const int seg = (((n_valid + 7) / 8) + 31) / 32 * 32;
-    const int b_lo = min(warp * seg, n_valid), b_hi = min(b_lo + seg, n_valid);
-    int n_gt = 0, n_eq = 0;
-    if (SMEM) {
-        for (int q = (b_lo >> 2) + lane; 4 * q < b_hi; q += 32) {
-            const uint4 kk = keys4[q];
-            const unsigned k[4] = {kk.x, kk.y, kk.z, kk.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const unsigned km = k[j] & mask;
-                const bool in = 4 * q + j >= b_lo && 4 * q + j < b_hi;   // an empty segment starts mid-quad
-                n_gt += in && km > prefix;
-                n_eq += in && km == prefix;
+// One digit of the radix select, by one warp: among the keys matching `prefix`,
+// the bucket of the digit at `shift` (NB buckets) that holds the remaining-th
+// largest key.  Lane l sums the buckets of ranks PER l .. PER l + PER - 1
+// (descending digits); a warp scan of those sums crosses `remaining` at exactly
+// one lane, which walks its buckets; the extended prefix, the rank left inside
+// the bucket and the bucket's count come back to every lane.
+template <int NB>
+__device__ __forceinline__ void topk_pick(const int *hist, int remaining, unsigned prefix, int shift, int lane,
+                                          unsigned &out_prefix, int &out_rem, int &out_cnt) {
+    constexpr int PER = NB / 32;
+    int c = 0;
+#pragma unroll 8
+    for (int j = 0; j < PER; ++j) c += hist[topk_slot(PER * lane + j)];
+    const int incl = warp_incl_scan(c, lane);
+    const bool mine = incl >= remaining && incl - c < remaining;
+    const int src = max(__ffs(__ballot_sync(0xffffffffu, mine)) - 1, 0);   // one lane when the counts cover `remaining`
+    unsigned p = 0u;
+    int r = 0, cnt = 0;
+    if (mine) {
+        int run = incl - c;
+        for (int j = 0; j < PER; ++j) {
+            const int h = hist[topk_slot(PER * lane + j)];
+            if (run + h >= remaining) {
+                p = prefix | ((unsigned)(NB - 1 - (PER * lane + j)) << shift);
+                r = remaining - run;
+                cnt = h;
+                break;
             }
-        }
-    } else {
-        for (int b = b_lo + lane; b < b_hi; b += 32) {
-            const unsigned km = key_at(b) & mask;
-            n_gt += km > prefix;
-            n_eq += km == prefix;
+            run += h;
         }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        n_gt += __shfl_xor_sync(0xffffffffu, n_gt, o);
-        n_eq += __shfl_xor_sync(0xffffffffu, n_eq, o);
-    }
-    if (lane == 0) {
-        S.wcnt[warp][0] = n_gt;
-        S.wcnt[warp][1] = n_eq;
-    }
-    __syncthreads();
-    int gt_before = 0, eq_before = 0;
-    for (int w = 0; w < warp; ++w) {
-        gt_before += S.wcnt[w][0];
-        eq_before += S.wcnt[w][1];
-    }
-    const unsigned lt = (1u << lane) - 1u;
-    int eq_run = eq_before, out_run = gt_before + min(eq_before, remaining);
-    for (int b0 = b_lo; b0 < b_hi; b0 += 32) {
-        const int b = b0 + lane;
-        const bool in = b < b_hi;
-        const unsigned km = in ? (key_at(b) & mask) : 0u;
-        const bool eq = in && km == prefix;
-        bool take = in && km > prefix;
-        const unsigned eq_mask = __ballot_sync(0xffffffffu, eq);
-        if (eq_mask) {   // uniform
-            take = take || (eq && eq_run + __popc(eq_mask & lt) < remaining);
-            eq_run += __popc(eq_mask);
-        }
-        const unsigned take_mask = __ballot_sync(0xffffffffu, take);
-        if (take) out[out_run + __popc(take_mask & lt)] = b;
-        out_run += __popc(take_mask);
-    }
+    out_prefix = __shfl_sync(0xffffffffu, p, src);
+    out_rem = __shfl_sync(0xffffffffu, r, src);
+    out_cnt = __shfl_sync(0xffffffffu, cnt, src);
 }
 
-__global__ void __launch_bounds__(256)
-qsa_topk_kernel(const float *__restrict__ scores, int n, int KB, int32_t *__restrict__ sel) {
-    extern __shared__ uint4 keys4[];   // the row's keys when n_valid <= TOPK_CAP
-    __shared__ TopkSmem S;
-    const int tid = threadIdx.x;
-    const unsigned row = blockIdx.x;   // s * n + i (batch * n < 2^29)
-    const int i = (int)(row % (unsigned)n);
-    const int nb = n / qsa::R;
-    const int n_valid = (i + 1) / qsa::R;
+// One warp per query row, no block barriers: the row's keys (score bits) are read
+// from the score matrix for each pass -- the first from HBM, the rest from L2 --
+// and counted into the warp's own histogram with shared atomics.  A radix select
+// on digits of 11, 11 and 9 bits finds the threshold (stopping at the first
+// digit whose bucket is taken whole); the selection then walks the row in index
+// order, 128 keys per step (a 16-byte load per lane when rows are aligned): the
+// keys above the threshold, and the first `remaining` equal to it, are written at
+// ascending positions found by warp scans of per-lane counts.
+__global__ void __launch_bounds__(32 * qsa::TOPK_WARPS)
+qsa_topk_kernel(const float *__restrict__ scores, int n, long long n_rows, int KB, int32_t *__restrict__ sel) {
+    using namespace qsa;
+    extern __shared__ int hist_all[];   // [TOPK_WARPS][WH_SLOTS]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long row = (long long)blockIdx.x * TOPK_WARPS + warp;
+    if (row >= n_rows) return;   // no block barriers below
+    int *hist = hist_all + warp * WH_SLOTS;
+    const int i = (int)(row % n);
+    const int nb = n / R;
+    const int n_valid = (i + 1) / R;
     const float *sc = scores + (size_t)row * nb;
     int32_t *out = sel + (size_t)row * KB;
     if (n_valid <= KB) {   // every complete block
-        for (int j = tid; j < KB; j += 256) out[j] = j < n_valid ? j : -1;
+        for (int j = lane; j < KB; j += 32) out[j] = j < n_valid ? j : -1;
         return;
     }
-    if (n_valid <= qsa::TOPK_CAP)   // uniform
-        topk_row<true>(S, keys4, sc, nb, n_valid, KB, out, tid);
-    else
-        topk_row<false>(S, keys4, sc, nb, n_valid, KB, out, tid);
+    // Rows start on 16-byte boundaries when nb % 4 == 0; the last quad may reach
+    // past n_valid, never past the row.
+    const bool vec = (nb & 3) == 0;
+    const int n4 = (n_valid + 3) >> 2;
+    // f(key) for every complete block's key, any order; U 16-byte loads per lane
+    // are issued before their keys are counted, so several loads are in flight
+    constexpr int U = 4;
+    const float4 *sc4 = reinterpret_cast<const float4 *>(sc);
+    auto for_keys = [&](auto &&f) {
+        if (vec) {
+            for (int q0 = lane; q0 < n4; q0 += 32 * U) {
+                float4 v[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    v[u] = q0 + 32 * u < n4 ? __ldg(sc4 + q0 + 32 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int q = q0 + 32 * u;
+                    const unsigned k[4] = {topk_key(v[u].x), topk_key(v[u].y), topk_key(v[u].z), topk_key(v[u].w)};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        if (4 * q + j < n_valid) f(k[j]);
+                }
+            }
+        } else {
+            for (int b0 = lane; b0 < n_valid; b0 += 32 * U) {
+                float v[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u) v[u] = b0 + 32 * u < n_valid ? __ldg(sc + b0 + 32 * u) : 0.f;
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    if (b0 + 32 * u < n_valid) f(topk_key(v[u]));
+            }
+        }
+    };
+    for (int j = lane; j < WH_SLOTS; j += 32) hist[j] = 0;
+    __syncwarp();
+    for_keys([&](unsigned key) { atomicAdd(&hist[topk_slot(HB - 1 - (int)(key >> 20))], 1); });
+    __syncwarp();
+    unsigned prefix;
+    int remaining, cnt;
+    topk_pick<HB>(hist, KB, 0u, 20, lane, prefix, remaining, cnt);
+    unsigned mask = 0xFFF00000u;
+    if (cnt != remaining) {   // uniform
+        __syncwarp();
+        for (int j = lane; j < WH_SLOTS; j += 32) hist[j] = 0;
+        __syncwarp();
+        for_keys([&](unsigned key) {
+            if ((key & mask) == prefix) atomicAdd(&hist[topk_slot(HB - 1 - (int)((key >> 9) & (HB - 1)))], 1);
+        });
+        __syncwarp();
+        topk_pick<HB>(hist, remaining, prefix, 9, lane, prefix, remaining, cnt);
+        mask = 0xFFFFFE00u;
+        if (cnt != remaining) {
+            __syncwarp();
+            for (int j = lane; j < topk_slot(512); j += 32) hist[j] = 0;
+            __syncwarp();
+            for_keys([&](unsigned key) {
+                if ((key & mask) == prefix) atomicAdd(&hist[topk_slot(511 - (int)(key & 511u))], 1);
+            });
+            __syncwarp();
+            topk_pick<512>(hist, remaining, prefix, 0, lane, prefix, remaining, cnt);
+            mask = 0xFFFFFFFFu;
+        }
+    }
+    // Selection in index order: every key above the threshold, and the first
+    // `remaining` equal to it.  Per step of 128 keys one warp scan of the lanes'
+    // (above, equal) counts, packed in one word, gives each lane the keys taken
+    // before its own: the above ones, plus the equal ones while fewer than
+    // `remaining` equal keys lie before them.
+    int eq_run = 0, out_run = 0;
+    if (vec) {
+        for (int q0 = 0; q0 < n4 && out_run < KB; q0 += 32 * U) {   // out_run is uniform
+            float4 v[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                v[u] = q0 + 32 * u + lane < n4 ? __ldg(sc4 + q0 + 32 * u + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int q = q0 + 32 * u + lane;
+                const unsigned k[4] = {topk_key(v[u].x), topk_key(v[u].y), topk_key(v[u].z), topk_key(v[u].w)};
+                unsigned gt = 0u, eq = 0u;   // bit j: key 4 q + j
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const bool in = 4 * q + j < n_valid;
+                    const unsigned km = k[j] & mask;
+                    gt |= (unsigned)(in && km > prefix) << j;
+                    eq |= (unsigned)(in && km == prefix) << j;
+                }
+                const int packed = (__popc(gt) << 16) | __popc(eq);
+                const int incl = warp_incl_scan(packed, lane);
+                const int excl = incl - packed;
+                const int eq_left = max(remaining - eq_run, 0);   // equal keys still to take
+                int eq_before = excl & 0xFFFF;                     // equal keys of earlier lanes in this step
+                int pos = out_run + (excl >> 16) + min(eq_before, eq_left);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const bool e = (eq >> j) & 1u;
+                    const bool take = ((gt >> j) & 1u) || (e && eq_before < eq_left);
+                    eq_before += e;
+                    if (take) out[pos++] = 4 * q + j;
+                }
+                const int tot = __shfl_sync(0xffffffffu, incl, 31);
+                out_run += (tot >> 16) + min(tot & 0xFFFF, eq_left);
+                eq_run += tot & 0xFFFF;
+            }
+        }
+    } else {
+        const unsigned lt = (1u << lane) - 1u;
+        for (int b0 = 0; b0 < n_valid; b0 += 32) {
+            const int b = b0 + lane;
+            const bool in = b < n_valid;
+            const unsigned km = in ? (topk_key(sc[b]) & mask) : 0u;
+            const bool eq = in && km == prefix;
+            bool take = in && km > prefix;
+            const unsigned eq_mask = __ballot_sync(0xffffffffu, eq);
+            take = take || (eq && eq_run + __popc(eq_mask & lt) < remaining);
+            eq_run += __popc(eq_mask);
+            const unsigned take_mask = __ballot_sync(0xffffffffu, take);
+            if (take) out[out_run + __popc(take_mask & lt)] = b;
+            out_run += __popc(take_mask);
+            if (out_run >= KB) break;   // uniform
+        }
+    }
 }
 
 // ------------------------------------------------------------------ host
@@ -633,23 +649,28 @@ cudaError_t launch_qsa_indexer(const QsaArgs &a, void *ws) {
             return e;
         if ((e = make_tma_3d(reinterpret_cast<TmaMap *>(&m.k), kb, false, D, 1, a.B * nb, 64, BN, true)) != cudaSuccess)
             return e;
+        // score rows on 16-byte boundaries
+        const bool tma_out = (nb & 3) == 0 && (reinterpret_cast<uintptr_t>(scores) & 15) == 0;
+        if (tma_out && (e = make_tma_rows_f32(reinterpret_cast<TmaMap *>(&m.sc), scores, nb, a.B * a.n, 32, 32)) !=
+                           cudaSuccess)
+            return e;
         if ((e = cudaFuncSetAttribute(qsa_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM)) != cudaSuccess)
             return e;
         const long long n_items = qsa_score_items(a.B, a.n);
         const int g = (int)(n_items < sms ? n_items : sms);
         if (g > 0) {
-            qsa_score_kernel<<<g, 192, SMEM, a.stream>>>(m, a.B, a.n, (int)n_items, scores);
+            qsa_score_kernel<<<g, 64 + 32 * EPI_WARPS, SMEM, a.stream>>>(m, a.B, a.n, (int)n_items, tma_out, scores);
             if ((e = launched()) != cudaSuccess) return e;
         }
     }
     if (a.n > 0) {
-        // the row's keys, rounded up to whole 16-byte quads
-        const int cap = ((nb < qsa::TOPK_CAP ? nb : qsa::TOPK_CAP) + 3) & ~3;
-        if ((e = cudaFuncSetAttribute(qsa_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, cap * 4)) !=
+        const long long rows = (long long)a.B * a.n;
+        const size_t smem = (size_t)TOPK_WARPS * WH_SLOTS * 4;
+        if ((e = cudaFuncSetAttribute(qsa_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
             cudaSuccess)
             return e;
-        qsa_topk_kernel<<<(unsigned)((long long)a.B * a.n), 256, (size_t)cap * 4, a.stream>>>(scores, a.n, a.KB,
-                                                                                             a.sel);
+        qsa_topk_kernel<<<(unsigned)((rows + TOPK_WARPS - 1) / TOPK_WARPS), 32 * TOPK_WARPS, smem, a.stream>>>(
+            scores, a.n, rows, a.KB, a.sel);
         if ((e = launched()) != cudaSuccess) return e;
     }
     return cudaSuccess;
