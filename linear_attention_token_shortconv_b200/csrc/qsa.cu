@@ -554,12 +554,13 @@ qsa_topk_kernel(const float *__restrict__ scores, int n, long long n_rows, int K
         }
     }
     // Selection in index order: every key above the threshold, and the first
-    // `remaining` equal to it.  Per step of 128 keys one warp scan of the lanes'
-    // (above, equal) counts, packed in one word, gives each lane the keys taken
-    // before its own: the above ones, plus the equal ones while fewer than
-    // `remaining` equal keys lie before them.
+    // `remaining` equal to it.  Key 4 q + j of a step sits in lane q % 32, so the
+    // keys taken before it are those of the lower lanes (one ballot per j) and of
+    // its own lane's lower j.  Equal keys need their rank among the equal ones
+    // seen so far; a step without any (the common case) skips that count.
     int eq_run = 0, out_run = 0;
     if (vec) {
+        const unsigned lt = (1u << lane) - 1u;
         for (int q0 = 0; q0 < n4 && out_run < KB; q0 += 32 * U) {   // out_run is uniform
             float4 v[U];
 #pragma unroll
@@ -569,30 +570,37 @@ qsa_topk_kernel(const float *__restrict__ scores, int n, long long n_rows, int K
             for (int u = 0; u < U; ++u) {
                 const int q = q0 + 32 * u + lane;
                 const unsigned k[4] = {topk_key(v[u].x), topk_key(v[u].y), topk_key(v[u].z), topk_key(v[u].w)};
-                unsigned gt = 0u, eq = 0u;   // bit j: key 4 q + j
+                bool take[4], eq[4];
+                bool any_eq = false;
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const bool in = 4 * q + j < n_valid;
                     const unsigned km = k[j] & mask;
-                    gt |= (unsigned)(in && km > prefix) << j;
-                    eq |= (unsigned)(in && km == prefix) << j;
+                    take[j] = in && km > prefix;
+                    eq[j] = in && km == prefix;
+                    any_eq |= eq[j];
                 }
-                const int packed = (__popc(gt) << 16) | __popc(eq);
-                const int incl = warp_incl_scan(packed, lane);
-                const int excl = incl - packed;
-                const int eq_left = max(remaining - eq_run, 0);   // equal keys still to take
-                int eq_before = excl & 0xFFFF;                     // equal keys of earlier lanes in this step
-                int pos = out_run + (excl >> 16) + min(eq_before, eq_left);
+                if (__any_sync(0xffffffffu, any_eq)) {   // uniform: rank the equal keys in index order
+                    const int n_eq = eq[0] + eq[1] + eq[2] + eq[3];
+                    const int incl = warp_incl_scan(n_eq, lane);
+                    int eq_before = eq_run + incl - n_eq;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        take[j] = take[j] || (eq[j] && eq_before < remaining);
+                        eq_before += eq[j];
+                    }
+                    eq_run += __shfl_sync(0xffffffffu, incl, 31);
+                }
+                int pos = out_run, mine = 0;
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    const bool e = (eq >> j) & 1u;
-                    const bool take = ((gt >> j) & 1u) || (e && eq_before < eq_left);
-                    eq_before += e;
-                    if (take) out[pos++] = 4 * q + j;
+                    const unsigned m = __ballot_sync(0xffffffffu, take[j]);
+                    pos += __popc(m & lt);
+                    out_run += __popc(m);
                 }
-                const int tot = __shfl_sync(0xffffffffu, incl, 31);
-                out_run += (tot >> 16) + min(tot & 0xFFFF, eq_left);
-                eq_run += tot & 0xFFFF;
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (take[j]) out[pos + mine++] = 4 * q + j;
             }
         }
     } else {
