@@ -553,7 +553,8 @@ def profile_case(kind, size):
                   two warm-up calls, then one call
       decode B    decode steps for B sequences x 32 heads, d = 128: three steps
       backward T  prefill backward, 4 sequences x T tokens, H = 16, d = 128, fp32: three calls
-      qsa n       QSA indexer on one sequence of n tokens, K = 2048: three calls"""
+      qsa n       QSA indexer on one sequence of n tokens, K = 2048: three calls
+      layer T     layer forward, 4 sequences x T tokens, H = 16, d_model = 2048: three calls"""
     dev = torch.device("cuda", 0)
     if kind in ("prefill", "pretrain"):
         cfg = replace(LONG, lengths=(size,)) if kind == "prefill" else replace(PRETRAIN, lengths=(size,) * 4)
@@ -585,6 +586,15 @@ def profile_case(kind, size):
                                          d_out, S0=inp.get("S0"), num_seqs=cfg.num_seqs)
         torch.cuda.synchronize()
         print("ok", float(grads["dq"].abs().mean()))
+    elif kind == "layer":
+        cfg = replace(PRETRAIN, lengths=(size,) * 4)
+        inp = make_layer_inputs(cfg, 2048, dev)
+        y = torch.empty((cfg.total_tokens, 2048), dtype=torch.bfloat16, device=dev)
+        for _ in range(3):
+            gdn.layer_forward(inp["x"], inp["w_in"], inp["conv_w"], inp["A"], inp["b_alpha"], inp["norm_w"],
+                              inp["w_o"], cfg.H, cfg.dk, cfg.dv, S0=inp["S0"], num_seqs=cfg.num_seqs, y=y)
+        torch.cuda.synchronize()
+        print("ok", float(y.float().abs().mean()))
     elif kind == "qsa":
         cfg = replace(QSA, n=size)
         inp = make_qsa_inputs(cfg, dev)
@@ -607,7 +617,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--profile-case", nargs=2, metavar=("KIND", "SIZE"),
                     help="run one small workload for an ncu capture instead of the benchmark "
-                         "(prefill T | pretrain T | decode B | backward T | qsa n)")
+                         "(prefill T | pretrain T | decode B | backward T | qsa n | layer T)")
     args = ap.parse_args()
     if args.profile_case:
         profile_case(args.profile_case[0], int(args.profile_case[1]))
@@ -714,7 +724,7 @@ def main():
         l_tf = (l_gemm + l_mix) / (l_ms * 1e-3) / 1e12
         result["layer"] = {
             "workload": f"layer forward, B=4 x T=4096, H=16, d=128, d_model={l_dm}, bf16 "
-                        "(in-projection GEMMs on cuBLAS, the mixer, W_o)",
+                        "(in-projection GEMMs and W_o on the library's tcgen05 GEMM, the mixer)",
             "steps": 5, "ms_per_step": l_ms, "tokens_per_s": lcfg.total_tokens / (l_ms * 1e-3),
             "bound": "tensor", "flop_per_call": l_gemm + l_mix, "achieved_tflops": l_tf,
             "peak_tflops": pk["bf16_tflops"], "frac": l_tf / pk["bf16_tflops"],

@@ -250,13 +250,13 @@ GDN_API gdn_status_t gdn_qsa_indexer_workspace_size(int batch, int n, size_t *by
  *   w_o    [H dv, d_model] bf16, row-major
  *   y      [N_tok, d_model] bf16, written
  * and the mixer's parameters as gdn_prefill (dims->in_dtype and out_dtype must be
- * GDN_BF16; d_model a multiple of 8).  The projections are stored in bf16 between
- * the steps.  The three GEMM steps are plain bf16 GEMMs with fp32 accumulation on
- * cuBLAS, loaded at the first call (GDN_ERR_UNSUPPORTED when it cannot be
- * loaded); they are not fused with the mixer's prelude.  Each host thread gets its
- * own cuBLAS handle per device (created at its first call), so threads may run
- * layers at the same time.  Stream-ordered workspace from the library's pool:
- * gdn_layer_workspace_size() bytes.
+ * GDN_BF16; d_model a multiple of 8, else GDN_ERR_UNSUPPORTED).  The projections
+ * are stored in bf16 between the steps.
+ * The GEMM steps are bf16 products with fp32 accumulation on the library's own
+ * tcgen05 GEMM kernel; they are not fused with the mixer's prelude.  Stateless
+ * apart from the workspace, so threads may run layers at the same time.
+ * Stream-ordered workspace from the library's pool: gdn_layer_workspace_size()
+ * bytes.  An expired wait inside a GEMM raises GDN_ERRF_GEMM.
  */
 GDN_API gdn_status_t gdn_layer_forward(const gdn_dims_t *dims, int d_model, const void *x, const void *w_in,
                                        const float *conv_w, const float *A, const float *b_alpha,
@@ -404,6 +404,7 @@ GDN_API int gdn_last_call_launches(void);
 #define GDN_ERRF_CHAIN 2u   /* chunk_chain (gdn_prefill, tensor-core path) */
 #define GDN_ERRF_DECODE 4u  /* streaming decode kernel (gdn_decode_step) */
 #define GDN_ERRF_QSA 8u     /* QSA indexer score kernel (gdn_qsa_indexer) */
+#define GDN_ERRF_GEMM 16u   /* projection GEMMs (gdn_layer_forward) */
 
 /*
  * gdn_device_error_status -- reads the current device's error words into

@@ -40,7 +40,8 @@ GDN_API gdn_status_t gdn_selftest_umma(int a_mn, int b_mn, int negate_a, int N, 
  * gdn_device_error_status then reports.  Nothing faults and the context stays
  * usable.
  *
- *   family     GDN_ERRF_PREP, GDN_ERRF_CHAIN, GDN_ERRF_DECODE or GDN_ERRF_QSA (one bit)
+ *   family     GDN_ERRF_PREP, GDN_ERRF_CHAIN, GDN_ERRF_DECODE, GDN_ERRF_QSA or
+ *              GDN_ERRF_GEMM (one bit)
  *   max_polls  1 .. 65536
  *
  * Asynchronous on `stream`.  GDN_ERR_INVALID_ARG for another family value or

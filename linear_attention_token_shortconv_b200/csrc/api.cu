@@ -304,14 +304,16 @@ int gdn_last_call_launches(void) { return tl_launches; }
 
 gdn_status_t gdn_device_error_status(unsigned *flags, int clear, gdn_stream_t stream) {
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    unsigned w[4] = {0, 0, 0, 0};
+    unsigned w[5] = {0, 0, 0, 0, 0};
     cudaError_t e = gdn::prep_error_word(&w[0], clear != 0, s);
     if (e == cudaSuccess) e = gdn::chain_error_word(&w[1], clear != 0, s);
     if (e == cudaSuccess) e = gdn::decode_error_word(&w[2], clear != 0, s);
     if (e == cudaSuccess) e = gdn::qsa_error_word(&w[3], clear != 0, s);
+    if (e == cudaSuccess) e = gdn::gemm_error_word(&w[4], clear != 0, s);
     if (e != cudaSuccess) return GDN_ERR_CUDA;
     const unsigned f = (w[0] ? GDN_ERRF_PREP : 0u) | (w[1] ? GDN_ERRF_CHAIN : 0u) |
-                       (w[2] ? GDN_ERRF_DECODE : 0u) | (w[3] ? GDN_ERRF_QSA : 0u);
+                       (w[2] ? GDN_ERRF_DECODE : 0u) | (w[3] ? GDN_ERRF_QSA : 0u) |
+                       (w[4] ? GDN_ERRF_GEMM : 0u);
     if (flags) *flags = f;
     return f ? GDN_ERR_TIMEOUT : GDN_OK;
 }
@@ -571,7 +573,7 @@ gdn_status_t gdn_layer_workspace_size(const gdn_dims_t *dims, int d_model, size_
     gdn_status_t st = check_dims(dims, false);
     if (st != GDN_OK) return st;
     if (!bytes || d_model <= 0) return GDN_ERR_INVALID_ARG;
-    *bytes = gdn::layer_workspace_bytes(dims->total_tokens, dims->H, dims->dk, dims->dv) + workspace_bytes(dims);
+    *bytes = gdn::layer_workspace_bytes(dims->total_tokens, dims->H, dims->dk, dims->dv, d_model) + workspace_bytes(dims);
     return GDN_OK;
 }
 
@@ -606,7 +608,6 @@ gdn_status_t gdn_layer_forward(const gdn_dims_t *dims, int d_model, const void *
     for (const void *p : opt)
         if (p && !aligned16(p)) return GDN_ERR_ALIGNMENT;
     if (cu_seqlens && !aligned_to(cu_seqlens, 4)) return GDN_ERR_ALIGNMENT;
-    if (!no_tokens && !gdn::layer_blas_available()) return GDN_ERR_UNSUPPORTED;
 
     gdn::LayerArgs L;
     gdn::PrefillArgs &a = L.f;
@@ -629,7 +630,7 @@ gdn_status_t gdn_layer_forward(const gdn_dims_t *dims, int d_model, const void *
     L.w_o = w_o;
     L.y = y;
     if (no_tokens) return prefill_dispatch(a) == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
-    const size_t ws_bytes = gdn::layer_workspace_bytes(a.n_tok, a.H, a.dk, a.dv);
+    const size_t ws_bytes = gdn::layer_workspace_bytes(a.n_tok, a.H, a.dk, a.dv, d_model);
     char *ws = nullptr;
     cudaMemPool_t pool;
     if (get_pool(&pool) != cudaSuccess) return GDN_ERR_CUDA;

@@ -66,6 +66,18 @@ struct TmaMap { alignas(64) unsigned char bytes[128]; };
 cudaError_t make_tma_3d(TmaMap *out, const void *base, bool bf16, int inner, int H, int n_tok,
                         int box_inner, int box_rows, bool swizzle128);
 cudaError_t make_tma_rows_f32(TmaMap *out, const void *base, int cols, int rows, int box_cols, int box_rows);
+cudaError_t make_tma_mat_bf16(TmaMap *out, const void *base, int inner, int rows, int ld, int box_inner,
+                              int box_rows);
+// K7: C [M, N] = A [M, K] B [K, N], bf16 row-major with leading dimensions lda,
+// ldb, ldc (elements; lda and K multiples of 8, A 16-byte aligned; for N >= 64
+// also ldb a multiple of 8 and B 16-byte aligned), fp32 accumulation.  N < 64
+// takes gemm_workspace_bytes(N, K) of 16-byte-aligned workspace (B transposed);
+// N >= 64 none.
+size_t gemm_workspace_bytes(int N, int K);
+cudaError_t launch_gemm_bf16(int M, int N, int K, const void *A, int lda, const void *B, int ldb, void *C, int ldc,
+                             void *ws, cudaStream_t stream);
+cudaError_t gemm_error_word(unsigned *v, bool clear, cudaStream_t s);
+cudaError_t gemm_wait_selftest(uint32_t max_polls, cudaStream_t s);
 
 // K4: prefill backward (fp32 inputs, dk = dv in {64, 128}); `f` holds the forward's
 // inputs (f.out and f.S_final are unused), the rest the incoming and outgoing
@@ -107,8 +119,7 @@ struct LayerArgs {
     const void *x, *w_in, *w_o;
     void *y;
 };
-size_t layer_workspace_bytes(int n_tok, int H, int dk, int dv);
-bool layer_blas_available();
+size_t layer_workspace_bytes(int n_tok, int H, int dk, int dv, int d_model);
 cudaError_t launch_layer(const LayerArgs &L, void *ws, cudaError_t (*run_prefill)(const PrefillArgs &));
 
 // K2f: token-by-token recurrence with the fused gates and output stage (SIMT fp32).

@@ -7,85 +7,47 @@
 //   o = gdn_prefill(q, k, v, ..., z, ...) (the mixer, bf16 out)
 //   y = o W_o                              (bf16 GEMM)
 //
-// The projections are plain GEMMs and run on cuBLAS (loaded with dlopen at first
-// use, so the library itself loads without it); each column block of the packed
-// W_in is its own GEMM, writing the contiguous [N, H, d] tensor the mixer reads.
-// Not fused: the GEMM epilogues do not run the conv / SiLU / norm prelude.
-#include <cublas_v2.h>
-#include <dlfcn.h>
-
-#include <mutex>
+// The projections run on the library's own tcgen05 GEMM (K7, gemm.cu); each
+// column block of the packed W_in is its own GEMM, writing the contiguous
+// [N, H, d] tensor the mixer reads.  Not fused: the GEMM epilogues do not run
+// the conv / SiLU / norm prelude.
+#include <cuda_bf16.h>
 
 #include "gdn_internal.h"
 
 namespace gdn {
 
 namespace {
-
-typedef cublasStatus_t (*CreateFn)(cublasHandle_t *);
-typedef cublasStatus_t (*SetStreamFn)(cublasHandle_t, cudaStream_t);
-typedef cublasStatus_t (*GemmExFn)(cublasHandle_t, cublasOperation_t, cublasOperation_t, int, int, int,
-                                   const void *, const void *, cudaDataType, int, const void *, cudaDataType, int,
-                                   const void *, void *, cudaDataType, int, cublasComputeType_t, cublasGemmAlgo_t);
-
-struct Blas {
-    bool tried = false, ok = false;
-    CreateFn create = nullptr;
-    SetStreamFn set_stream = nullptr;
-    GemmExFn gemm = nullptr;
-};
-std::mutex g_blas_mu;
-Blas g_blas;
-
-// The cuBLAS entry points (resolved once) and the calling thread's handle for this
-// device.  A handle carries the stream of the call in progress, so threads that
-// run layers at the same time must not share one: each (host thread, device)
-// gets its own, created at its first use and kept for the thread's lifetime.
-bool blas_handle(int dev, cublasHandle_t *h) {
-    {
-        std::lock_guard<std::mutex> lock(g_blas_mu);
-        if (!g_blas.tried) {
-            g_blas.tried = true;
-            void *lib = dlopen("libcublas.so.12", RTLD_NOW | RTLD_GLOBAL);
-            if (lib) {
-                g_blas.create = reinterpret_cast<CreateFn>(dlsym(lib, "cublasCreate_v2"));
-                g_blas.set_stream = reinterpret_cast<SetStreamFn>(dlsym(lib, "cublasSetStream_v2"));
-                g_blas.gemm = reinterpret_cast<GemmExFn>(dlsym(lib, "cublasGemmEx"));
-                g_blas.ok = g_blas.create && g_blas.set_stream && g_blas.gemm;
-            }
-        }
-    }
-    if (!g_blas.ok || dev < 0 || dev >= 64) return false;
-    thread_local cublasHandle_t tl_handle[64] = {};
-    if (!tl_handle[dev] && g_blas.create(&tl_handle[dev]) != CUBLAS_STATUS_SUCCESS) return false;
-    *h = tl_handle[dev];
-    return true;
+// dst [rows][cols] (contiguous) = the column block [rows][c0, c0 + cols) of src
+// (leading dimension ld): a W_in block whose rows do not start on 16-byte
+// boundaries, made readable by TMA.
+__global__ void copy_cols_kernel(const __nv_bfloat16 *__restrict__ src, int ld, int c0, int rows, int cols,
+                                 __nv_bfloat16 *__restrict__ dst) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (long long)rows * cols) return;
+    const int r = (int)(i / cols), c = (int)(i % cols);
+    dst[i] = src[(size_t)r * ld + c0 + c];
 }
 
-// Row-major C [M, Nc] = A [M, K] (lda) x B [K, Nc] (ldb), bf16 in and out, fp32
-// accumulation: cuBLAS's column-major C^T = B^T A^T.
-cudaError_t gemm_bf16(cublasHandle_t h, int M, int Nc, int K, const void *A, int lda, const void *B, int ldb,
-                      void *C, int ldc) {
-    if (M == 0 || Nc == 0) return cudaSuccess;
-    const float one = 1.0f, zero = 0.0f;
-    const cublasStatus_t st = g_blas.gemm(h, CUBLAS_OP_N, CUBLAS_OP_N, Nc, M, K, &one, B, CUDA_R_16BF, ldb, A,
-                                          CUDA_R_16BF, lda, &zero, C, CUDA_R_16BF, ldc, CUBLAS_COMPUTE_32F,
-                                          CUBLAS_GEMM_DEFAULT);
-    return st == CUBLAS_STATUS_SUCCESS ? cudaSuccess : cudaErrorUnknown;
+// The gate logits [rows][a_0 .. a_{H-1} b_0 .. b_{H-1}] of one GEMM into the
+// mixer's a [rows][H] and b [rows][H].
+__global__ void split_gates_kernel(const __nv_bfloat16 *__restrict__ ab, int rows, int H,
+                                   __nv_bfloat16 *__restrict__ a, __nv_bfloat16 *__restrict__ b) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (long long)rows * 2 * H) return;
+    const long long r = i / (2 * H);
+    const int j = (int)(i % (2 * H));
+    if (j < H) a[r * H + j] = ab[i];
+    else b[r * H + j - H] = ab[i];
 }
-
 }  // namespace
 
-size_t layer_workspace_bytes(int n_tok, int H, int dk, int dv) {
+size_t layer_workspace_bytes(int n_tok, int H, int dk, int dv, int d_model) {
     auto ru = [](size_t x) { return (x + 255) & ~(size_t)255; };
     const size_t n = (size_t)n_tok;
-    return 2 * ru(n * H * dk * 2) + 3 * ru(n * H * dv * 2) + 2 * ru(n * H * 2);
-}
-
-bool layer_blas_available() {
-    int dev = 0;
-    cublasHandle_t h;
-    return cudaGetDevice(&dev) == cudaSuccess && blas_handle(dev, &h);
+    const int wide = dk > dv ? dk : dv;
+    return 2 * ru(n * H * dk * 2) + 3 * ru(n * H * dv * 2) + 2 * ru(n * H * 2) + ru(n * 2 * H * 2) +
+           ru(gemm_workspace_bytes(2 * H, d_model)) + ru((size_t)d_model * H * wide * 2);
 }
 
 cudaError_t launch_layer(const LayerArgs &L, void *ws, cudaError_t (*run_prefill)(const PrefillArgs &)) {
@@ -99,20 +61,39 @@ cudaError_t launch_layer(const LayerArgs &L, void *ws, cudaError_t (*run_prefill
     char *v = take((size_t)N * H * dv * 2), *z = take((size_t)N * H * dv * 2);
     char *al = take((size_t)N * H * 2), *bl = take((size_t)N * H * 2);
     char *o = take((size_t)N * H * dv * 2);
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    cublasHandle_t h;
-    if (!blas_handle(dev, &h)) return cudaErrorNotSupported;
-    if (g_blas.set_stream(h, a.stream) != CUBLAS_STATUS_SUCCESS) return cudaErrorUnknown;
+    char *ab = take((size_t)N * 2 * H * 2);                   // both gate logits, one GEMM
+    char *gw = take(gemm_workspace_bytes(2 * H, D));
+    char *wcopy = take((size_t)D * H * (dk > dv ? dk : dv) * 2);
+    // W_in rows start on 16-byte boundaries only when its width is a multiple of 8
+    const bool w_aligned = c_in % 8 == 0;
     const char *w_in = static_cast<const char *>(L.w_in);
-    // column blocks of W_in: q, k [H dk], v, z [H dv], a, b [H]
-    struct Part { char *dst; int cols; } parts[6] = {{q, H * dk}, {k, H * dk}, {v, H * dv}, {z, H * dv}, {al, H}, {bl, H}};
+    // column blocks of W_in: q, k [H dk], v, z [H dv], then a and b [H] side by
+    // side, one GEMM of 2H columns (x is read once for both)
+    struct Part { char *dst; int cols; } parts[5] = {
+        {q, H * dk}, {k, H * dk}, {v, H * dv}, {z, H * dv}, {ab, 2 * H}};
+    cudaError_t e;
     int c0 = 0;
     for (const Part &pt : parts) {
-        if ((e = gemm_bf16(h, N, pt.cols, D, L.x, D, w_in + (size_t)c0 * 2, c_in, pt.dst, pt.cols)) != cudaSuccess)
+        const void *B = w_in + (size_t)c0 * 2;
+        int ldb = c_in;
+        if (!w_aligned && pt.cols >= 64) {   // a block read by TMA: copy it out, contiguous
+            const long long n_el = (long long)D * pt.cols;
+            copy_cols_kernel<<<(unsigned)((n_el + 255) / 256), 256, 0, a.stream>>>(
+                static_cast<const __nv_bfloat16 *>(L.w_in), c_in, c0, D, pt.cols, reinterpret_cast<__nv_bfloat16 *>(wcopy));
+            if ((e = launched()) != cudaSuccess) return e;
+            B = wcopy;
+            ldb = pt.cols;
+        }
+        if ((e = launch_gemm_bf16(N, pt.cols, D, L.x, D, B, ldb, pt.dst, pt.cols, gw, a.stream)) != cudaSuccess)
             return e;
         c0 += pt.cols;
+    }
+    {
+        const long long n_el = (long long)N * 2 * H;
+        split_gates_kernel<<<(unsigned)((n_el + 255) / 256), 256, 0, a.stream>>>(
+            reinterpret_cast<const __nv_bfloat16 *>(ab), N, H, reinterpret_cast<__nv_bfloat16 *>(al),
+            reinterpret_cast<__nv_bfloat16 *>(bl));
+        if ((e = launched()) != cudaSuccess) return e;
     }
     PrefillArgs m = a;
     m.q = q; m.k = k; m.v = v; m.z = z; m.a_logit = al; m.b_logit = bl;
@@ -120,8 +101,7 @@ cudaError_t launch_layer(const LayerArgs &L, void *ws, cudaError_t (*run_prefill
     m.in_bf16 = true;
     m.out_bf16 = true;
     if ((e = run_prefill(m)) != cudaSuccess) return e;
-    if (g_blas.set_stream(h, a.stream) != CUBLAS_STATUS_SUCCESS) return cudaErrorUnknown;
-    return gemm_bf16(h, N, D, H * dv, o, H * dv, L.w_o, D, L.y, D);
+    return launch_gemm_bf16(N, D, H * dv, o, H * dv, L.w_o, D, L.y, D, nullptr, a.stream);
 }
 
 }  // namespace gdn

@@ -347,7 +347,7 @@ qsa_score_kernel(const __grid_constant__ QsaMaps maps, int B, int n, int n_items
                     uint32_t x[HI][32];
 #pragma unroll
                     for (int h = 0; h < HI; ++h) umma::tmem_ld32_nowait(trow + ts * (HI * BN) + h * BN + c, x[h]);
-                    umma::tmem_wait_ld();
+                    umma::tmem_ld_wait();
                     float acc[32];
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {

@@ -158,6 +158,7 @@ extern "C" gdn_status_t gdn_selftest_wait_timeout(unsigned family, unsigned max_
     case GDN_ERRF_CHAIN: e = gdn::chain_wait_selftest(max_polls, s); break;
     case GDN_ERRF_DECODE: e = gdn::decode_wait_selftest(max_polls, s); break;
     case GDN_ERRF_QSA: e = gdn::qsa_wait_selftest(max_polls, s); break;
+    case GDN_ERRF_GEMM: e = gdn::gemm_wait_selftest(max_polls, s); break;
     default: return GDN_ERR_INVALID_ARG;
     }
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;

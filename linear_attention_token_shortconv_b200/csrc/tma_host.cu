@@ -69,4 +69,22 @@ cudaError_t make_tma_rows_f32(TmaMap *out, const void *base, int cols, int rows,
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// A row-major bf16 matrix [rows][inner] with leading dimension ld (elements; ld * 2
+// a multiple of 16) as a 3-D map {inner, 1, rows}, boxes {box_inner, 1, box_rows},
+// 128-byte swizzle (box_inner * 2 = 128).
+cudaError_t make_tma_mat_bf16(TmaMap *out, const void *base, int inner, int rows, int ld, int box_inner,
+                              int box_rows) {
+    EncodeTiledFn fn;
+    cudaError_t e = encoder(&fn);
+    if (e != cudaSuccess) return e;
+    const cuuint64_t dims[3] = {(cuuint64_t)inner, 1, (cuuint64_t)rows};
+    const cuuint64_t strides[2] = {(cuuint64_t)ld * 2, (cuuint64_t)ld * 2};
+    const cuuint32_t box[3] = {(cuuint32_t)box_inner, 1, (cuuint32_t)box_rows};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(reinterpret_cast<CUtensorMap *>(out->bytes), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                    const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 }  // namespace gdn

@@ -27,7 +27,7 @@ EXPORTS = ("gdn_prefill", "gdn_prefill_workspace_size", "gdn_decode_step", "gdn_
            "gdn_selftest_wait_timeout", "gdn_decode_multi", "gdn_prefill_backward",
            "gdn_prefill_backward_workspace_size", "gdn_qsa_indexer", "gdn_qsa_indexer_workspace_size",
            "gdn_layer_forward", "gdn_layer_workspace_size", "gdn_prefill_ws", "gdn_prefill_conv_tail")
-ERRF_PREP, ERRF_CHAIN, ERRF_DECODE, ERRF_QSA = 1, 2, 4, 8
+ERRF_PREP, ERRF_CHAIN, ERRF_DECODE, ERRF_QSA, ERRF_GEMM = 1, 2, 4, 8, 16
 
 
 class GdnError(RuntimeError):

@@ -119,7 +119,7 @@ def test_rejected_calls_launch_nothing(lib):
 
 
 def test_wait_selftest_validation(lib):
-    assert lib.gdn_selftest_wait_timeout(16, 16, None) == 1      # not a family bit
+    assert lib.gdn_selftest_wait_timeout(32, 16, None) == 1      # not a family bit
     assert lib.gdn_selftest_wait_timeout(3, 16, None) == 1       # two bits
     assert lib.gdn_selftest_wait_timeout(1, 0, None) == 1
     assert lib.gdn_selftest_wait_timeout(1, 65537, None) == 1

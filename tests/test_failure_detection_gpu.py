@@ -12,7 +12,7 @@ from linear_attention_token_shortconv_b200.workloads import PRETRAIN, make_prefi
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("family", [gdn.ERRF_PREP, gdn.ERRF_CHAIN, gdn.ERRF_DECODE, gdn.ERRF_QSA])
+@pytest.mark.parametrize("family", [gdn.ERRF_PREP, gdn.ERRF_CHAIN, gdn.ERRF_DECODE, gdn.ERRF_QSA, gdn.ERRF_GEMM])
 def test_expired_wait_is_reported(cuda_device, family):
     gdn.device_error_status(clear=True)    # start clean
     assert gdn.device_error_status() == (0, 0)
@@ -23,9 +23,9 @@ def test_expired_wait_is_reported(cuda_device, family):
 
 
 def test_context_usable_after_expired_waits(cuda_device):
-    for f in (gdn.ERRF_PREP, gdn.ERRF_CHAIN, gdn.ERRF_DECODE, gdn.ERRF_QSA):
+    for f in (gdn.ERRF_PREP, gdn.ERRF_CHAIN, gdn.ERRF_DECODE, gdn.ERRF_QSA, gdn.ERRF_GEMM):
         gdn.selftest_wait_timeout(f, max_polls=256)
-    assert gdn.device_error_status(clear=True) == (5, 15)
+    assert gdn.device_error_status(clear=True) == (5, 31)
     cfg = scaled(PRETRAIN, lengths=(200, 72), H=2)
     cpu = make_prefill_inputs(cfg, "cpu")
     out, SF = gpu_prefill(to_device(cpu, cuda_device), 2)
