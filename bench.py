@@ -67,12 +67,12 @@ KERNEL_ROOFLINE = {"chunk_prep": ("hbm", 3 * 128 * 2 + 2 * 2),                  
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per unit from one
 # ncu capture of each kernel (profiles/), valid only while the kernel's sources
 # are the ones captured (sha1 over them); otherwise the JSON reports traffic null.
-#   prefill_fused: `bench.py --profile-case prefill 8192` (T = 8192, H = 32): 276.6 MB read +
-#     344.2 MB written for 262,144 token-heads; per token-head, scaled to the launch.
+#   prefill_fused: `bench.py --profile-case prefill 8192` (T = 8192, H = 32): 355.7 MB read +
+#     332.1 MB written for 262,144 token-heads; per token-head, scaled to the launch.
 NCU_TRAFFIC = {
     "prefill_fused": {"sources": ["prefill_tc.cu", "prep_body.cuh", "chain_body.cuh"],
-                      "sha1": "7f9f4aba8627ebcc0087792eddc6533e5c331e11",
-                      "bytes_per_unit": (277.407232e6 + 324.293888e6) / (8192 * 32)},
+                      "sha1": "fb609260faf92392139e0fe20f0ed3cb53bc807f",
+                      "bytes_per_unit": (355.690752e6 + 332.133632e6) / (8192 * 32)},
 }
 
 

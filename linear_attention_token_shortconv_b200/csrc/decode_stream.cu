@@ -26,6 +26,8 @@
 // CTA's phases fill the other's waits.  Every wait is bounded.
 #include <cuda_bf16.h>
 
+#include <cstring>
+
 #include "gdn_device.cuh"
 #include "gdn_internal.h"
 #include "umma.cuh"
@@ -88,6 +90,13 @@ __device__ __forceinline__ bool dwait(uint64_t *bar, uint32_t parity, volatile i
     return false;
 }
 
+// The token rows and history rows arrive by tensor copies (one per tensor instead
+// of one per row).
+struct DecodeMaps {
+    CUtensorMap tok[4];   // q, k, v, z [B T][H][128] bf16, box {128, 1, TMAX}
+    CUtensorMap hist;     // conv_hist as [3B][3][H][128] bf16, box {128, 1, 3, 3}
+};
+
 template <typename Tout, int TMAX>
 __global__ void __launch_bounds__(dstream::NT, dstream::Layout<TMAX>::CTAS_PER_SM)
 decode_stream_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
@@ -96,7 +105,8 @@ decode_stream_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
                      const bf16 *__restrict__ b_logit, const float *__restrict__ A,
                      const float *__restrict__ b_alpha, const bf16 *__restrict__ z,
                      const float *__restrict__ norm_w, float *__restrict__ S,
-                     Tout *__restrict__ out, const int32_t *__restrict__ n_keep, int B, int H, int T_rt) {
+                     Tout *__restrict__ out, const int32_t *__restrict__ n_keep, int B, int H, int T_rt,
+                     const __grid_constant__ DecodeMaps maps) {
     using namespace dstream;
     using Lo = Layout<TMAX>;
     constexpr int NSTAGE = Lo::NSTAGE, STAGE = Lo::STAGE, OFF_TOK = Lo::OFF_TOK, OFF_HIST = Lo::OFF_HIST;
@@ -129,45 +139,21 @@ decode_stream_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
     }
     __syncthreads();
 
-    // Stage s's loads for `item`, issued by warp 0: lane 0 arms the barrier, then
-    // lanes 0-3 take the state's quarters, lanes 4 .. 4 + 4T - 1 the token rows
-    // (q, k, v, z of each token) and the next nine lanes the history rows.  With
-    // one token, lane 0 issues all 17 copies (measured 1% faster there).
+    // Stage s's loads for `item`, issued by lane 0 of warp 0: the state in one bulk
+    // copy, each token tensor's rows by one tensor copy and the history rows by one
+    // (per-row copies cost about 150 cycles of issue each, on the critical path).
     auto issue = [&](int item, int s) {   // warp 0
         const int b = item / H, h = item % H;
         uint8_t *st = sm + s * STAGE;
         uint64_t *bar = full + s;
-        if (lane == 0) umma::mbar_expect_tx(bar, STATE + T * 1024 + 2304);
-        if constexpr (TMAX == 1) {
-            if (lane == 0) {
+        // the token box is TMAX rows (for several tokens, rows past T are not read)
+        if (lane == 0) umma::mbar_expect_tx(bar, STATE + (TMAX == 1 ? T : TMAX) * 1024 + 2304);
+        if (lane == 0) {   // the state in one copy, then one tensor copy per token tensor and the history
+            bulk_load(st, S + ((size_t)b * H + h) * D * D, STATE, bar);
 #pragma unroll
-                for (int p = 0; p < 4; ++p)
-                    bulk_load(st + p * (STATE / 4), S + ((size_t)b * H + h) * D * D + p * (D * D / 4), STATE / 4, bar);
-                const size_t tok = ((size_t)b * H + h) * D;
-                bulk_load(st + OFF_TOK + 0 * 256, q + tok, 256, bar);
-                bulk_load(st + OFF_TOK + 1 * 256, k + tok, 256, bar);
-                bulk_load(st + OFF_TOK + 2 * 256, v + tok, 256, bar);
-                bulk_load(st + OFF_TOK + 3 * 256, z + tok, 256, bar);
-#pragma unroll
-                for (int j = 0; j < 3; ++j)
-#pragma unroll
-                    for (int part = 0; part < 3; ++part)
-                        bulk_load(st + OFF_HIST + j * 768 + part * 256,
-                                  hist + ((size_t)b * 3 + j) * C + (size_t)part * H * D + (size_t)h * D, 256, bar);
-            }
-            return;
-        }
-        __syncwarp();
-        if (lane < 4) {
-            bulk_load(st + lane * (STATE / 4), S + ((size_t)b * H + h) * D * D + lane * (D * D / 4), STATE / 4, bar);
-        } else if (lane < 4 + 4 * T) {
-            const int u = lane - 4, part = u / T, t = u % T;
-            const bf16 *src = part == 0 ? q : part == 1 ? k : part == 2 ? v : z;
-            bulk_load(st + OFF_TOK + (part * TMAX + t) * 256, src + (((size_t)b * T + t) * H + h) * D, 256, bar);
-        } else if (lane < 13 + 4 * T) {
-            const int u = lane - 4 - 4 * T, j = u / 3, part = u % 3;
-            const bf16 *hr = hist + ((size_t)b * 3 + j) * C;
-            bulk_load(st + OFF_HIST + j * 768 + part * 256, hr + (size_t)part * H * D + (size_t)h * D, 256, bar);
+            for (int part = 0; part < 4; ++part)
+                umma::tma_load_3d(st + OFF_TOK + part * TMAX * 256, &maps.tok[part], 0, h, b * T, bar);
+            umma::tma_load_4d(st + OFF_HIST, &maps.hist, 0, h, 0, 3 * b, bar);
         }
     };
     const int first = blockIdx.x, stride = gridDim.x;
@@ -504,6 +490,21 @@ cudaError_t launch_decode_stream(const DecodeArgs &a, int T, const int32_t *n_ke
     if (items == 0) return cudaSuccess;
     const int per_sm = T == 1 && !n_keep ? dstream::Layout<1>::CTAS_PER_SM : dstream::Layout<4>::CTAS_PER_SM;
     const int grid = items < sms * per_sm ? items : sms * per_sm;
+    DecodeMaps maps;
+    std::memset(&maps, 0, sizeof maps);
+    {   // tensor maps of the token rows and the history
+        const long long C = 3LL * a.H * 128;
+        const void *tok[4] = {a.q, a.k, a.v, a.z};
+        const long long td[3] = {128, a.H, (long long)a.B * T}, ts[2] = {256, (long long)a.H * 256};
+        const int tb[3] = {128, 1, T == 1 && !n_keep ? 1 : 4};
+        for (int p = 0; p < 4; ++p)
+            if ((e = make_tma_plain_bf16(reinterpret_cast<TmaMap *>(&maps.tok[p]), tok[p], 3, td, ts, tb)) != cudaSuccess)
+                return e;
+        const long long hd[4] = {128, a.H, 3, 3LL * a.B}, hs[3] = {256, (long long)a.H * 256, C * 2};
+        const int hbx[4] = {128, 1, 3, 3};
+        if ((e = make_tma_plain_bf16(reinterpret_cast<TmaMap *>(&maps.hist), a.conv_hist, 4, hd, hs, hbx)) != cudaSuccess)
+            return e;
+    }
 #define GDN_DSTREAM(TOUT, TM)                                                                      \
     e = cudaFuncSetAttribute(decode_stream_kernel<TOUT, TM>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                              dstream::Layout<TM>::SMEM);                                          \
@@ -511,7 +512,7 @@ cudaError_t launch_decode_stream(const DecodeArgs &a, int T, const int32_t *n_ke
     decode_stream_kernel<TOUT, TM><<<grid, dstream::NT, dstream::Layout<TM>::SMEM, a.stream>>>(    \
         (const bf16 *)a.q, (const bf16 *)a.k, (const bf16 *)a.v, a.conv_w, (bf16 *)a.conv_hist,   \
         (const bf16 *)a.a_logit, (const bf16 *)a.b_logit, a.A, a.b_alpha, (const bf16 *)a.z,      \
-        a.norm_w, a.S, (TOUT *)a.out, n_keep, a.B, a.H, T)
+        a.norm_w, a.S, (TOUT *)a.out, n_keep, a.B, a.H, T, maps)
     if (T == 1 && !n_keep) {
         if (a.out_bf16) { GDN_DSTREAM(bf16, 1); } else { GDN_DSTREAM(float, 1); }
     } else {

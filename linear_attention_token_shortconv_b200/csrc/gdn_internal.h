@@ -68,6 +68,8 @@ cudaError_t make_tma_3d(TmaMap *out, const void *base, bool bf16, int inner, int
 cudaError_t make_tma_rows_f32(TmaMap *out, const void *base, int cols, int rows, int box_cols, int box_rows);
 cudaError_t make_tma_mat_bf16(TmaMap *out, const void *base, int inner, int rows, int ld, int box_inner,
                               int box_rows);
+cudaError_t make_tma_plain_bf16(TmaMap *out, const void *base, int rank, const long long *dims,
+                                const long long *strides, const int *box);
 // K7: C [M, N] = A [M, K] B [K, N], bf16 row-major with leading dimensions lda,
 // ldb, ldc (elements; lda and K multiples of 8, A 16-byte aligned; for N >= 64
 // also ldb a multiple of 8 and B 16-byte aligned), fp32 accumulation.  N < 64

@@ -69,6 +69,27 @@ cudaError_t make_tma_rows_f32(TmaMap *out, const void *base, int cols, int rows,
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// A bf16 tensor of rank 3 or 4 without swizzle: dims[0] contiguous, strides[i]
+// the byte stride of dimension i + 1 (multiples of 16), box[] the copied tile.
+cudaError_t make_tma_plain_bf16(TmaMap *out, const void *base, int rank, const long long *dims,
+                                const long long *strides, const int *box) {
+    EncodeTiledFn fn;
+    cudaError_t e = encoder(&fn);
+    if (e != cudaSuccess) return e;
+    if (rank < 3 || rank > 4) return cudaErrorInvalidValue;
+    cuuint64_t d[4], st[3];
+    cuuint32_t bx[4], estr[4] = {1, 1, 1, 1};
+    for (int i = 0; i < rank; ++i) {
+        d[i] = (cuuint64_t)dims[i];
+        bx[i] = (cuuint32_t)box[i];
+        if (i + 1 < rank) st[i] = (cuuint64_t)strides[i];
+    }
+    CUresult r = fn(reinterpret_cast<CUtensorMap *>(out->bytes), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank,
+                    const_cast<void *>(base), d, st, bx, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 // A row-major bf16 matrix [rows][inner] with leading dimension ld (elements; ld * 2
 // a multiple of 16) as a 3-D map {inner, 1, rows}, boxes {box_inner, 1, box_rows},
 // 128-byte swizzle (box_inner * 2 = 128).
