@@ -209,7 +209,7 @@ struct QsaMaps {
 // a timeout raises the error word and an abort flag the other roles check.
 __global__ void __launch_bounds__(64 + 32 * qsa::EPI_WARPS, 1)
 qsa_score_kernel(const __grid_constant__ QsaMaps maps, int B, int n, int n_items, bool tma_out,
-                 float *__restrict__ scores) {
+                 float *__restrict__ scores, float *__restrict__ rowmax) {
     using namespace qsa;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = umma::align_smem<1024>(smem_raw);
@@ -337,6 +337,7 @@ qsa_score_kernel(const __grid_constant__ QsaMaps maps, int B, int n, int n_items
             const int n_valid = i < n ? (i + 1) / R : 0;      // its complete blocks
             const int n_full = i0 + 31 < n ? (i0 + 1) / R : 0;   // blocks complete for all 32 queries
             float *dst = scores + ((size_t)item.s * n + (i < n ? i : 0)) * nb;
+            float lmax = 0.f;   // this lane's largest score in the item (for the top-k's buckets)
             for (int j = 0; j < item.nbt; ++j, ++t_it) {
                 const int ts = t_it & 1, v = t_it >> 1;
                 ok = __all_sync(0xffffffffu, wait(tfull + ts, v & 1));
@@ -357,6 +358,9 @@ qsa_score_kernel(const __grid_constant__ QsaMaps maps, int B, int n, int n_items
                         acc[e] = a;
                     }
                     const int bs = BN * (item.bt0 + j) + c;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (bs + e < n_valid) lmax = fmaxf(lmax, acc[e]);
                     if (tma_out && bs + 32 <= n_full) {   // uniform across the warp
                         if (lane == 0) umma::bulk_wait_read<0>();   // the last store has read the tile
                         __syncwarp();
@@ -386,6 +390,8 @@ qsa_score_kernel(const __grid_constant__ QsaMaps maps, int B, int n, int n_items
                 __syncwarp();
                 if (lane == 0) mbar_arrive_local(tempty + ts);
             }
+            // scores are >= 0, so their bit patterns order like the values
+            if (ok && lmax > 0.f) atomicMax(reinterpret_cast<int *>(rowmax) + (size_t)item.s * n + i, __float_as_int(lmax));
         }
         if (lane == 0) umma::bulk_wait_all();   // the last stores have left shared memory
     }
@@ -472,7 +478,8 @@ __device__ __forceinline__ void topk_pick(const int *hist, int remaining, unsign
 // keys above the threshold, and the first `remaining` equal to it, are written at
 // ascending positions found by warp scans of per-lane counts.
 __global__ void __launch_bounds__(32 * qsa::TOPK_WARPS)
-qsa_topk_kernel(const float *__restrict__ scores, int n, long long n_rows, int KB, int32_t *__restrict__ sel) {
+qsa_topk_kernel(const float *__restrict__ scores, const float *__restrict__ rowmax, int n, long long n_rows, int KB,
+                int32_t *__restrict__ sel) {
     using namespace qsa;
     extern __shared__ int hist_all[];   // [TOPK_WARPS][WH_SLOTS]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -523,6 +530,143 @@ qsa_topk_kernel(const float *__restrict__ scores, int n, long long n_rows, int K
             }
         }
     };
+    // ---- Fast path: buckets of the value scaled by the row's largest score (from
+    // the score kernel), 2048 across [0, max].  Near the threshold a bucket then
+    // holds a few keys, so one more walk over the row, in index order, settles the
+    // selection: keys above the threshold bucket are taken, the bucket's keys
+    // (candidates, at most CAND) are ranked among themselves.  The list of both,
+    // in index order, and the candidates' keys reuse the histogram's space.
+    constexpr int CAND = 64;
+    const float rmax = rowmax[row];
+    if (!(rmax > 0.f)) {   // every complete block scores 0: ties go to the smallest blocks
+        for (int j = lane; j < KB; j += 32) out[j] = j;
+        return;
+    }
+    const float scale = (float)HB / rmax;
+    auto vbucket = [&](unsigned key) { return min(HB - 1, (int)(__uint_as_float(key) * scale)); };
+    for (int j = lane; j < WH_SLOTS; j += 32) hist[j] = 0;
+    __syncwarp();
+    for_keys([&](unsigned key) { atomicAdd(&hist[topk_slot(HB - 1 - vbucket(key))], 1); });
+    __syncwarp();
+    {
+        unsigned bstar;
+        int rem, cnt;
+        topk_pick<HB>(hist, KB, 0u, 0, lane, bstar, rem, cnt);
+        __syncwarp();
+        if (cnt <= CAND && KB + 3 * CAND <= WH_SLOTS) {   // uniform
+            int *list = hist;                                               // [KB + CAND]
+            unsigned *ckey = reinterpret_cast<unsigned *>(hist + KB + CAND);   // [CAND]
+            int *cidx = hist + KB + 2 * CAND;                               // [CAND]
+            const unsigned lt = (1u << lane) - 1u;
+            // bucket(v) >= b* exactly when v * scale >= b* (truncation of a value >= 0;
+            // the top bucket also holds v * scale = 2048)
+            const float lo = (float)bstar, hi = bstar == (unsigned)(HB - 1) ? 3.0e38f : (float)(bstar + 1);
+            int list_run = 0, cand_run = 0;
+            // keys at or above the threshold bucket, in index order: index, or
+            // 0x80000000 | candidate ordinal
+            auto place = [&](const bool (&keep)[4], const bool (&cnd)[4], const unsigned (&k)[4], int base, int per) {
+                int pos = list_run, cpos = cand_run, mine = 0, cmine = 0;
+                bool any_cnd = false;
+                for (int j = 0; j < per; ++j) {
+                    const unsigned m = __ballot_sync(0xffffffffu, keep[j]);
+                    pos += __popc(m & lt);
+                    list_run += __popc(m);
+                    any_cnd |= cnd[j];
+                }
+                if (__any_sync(0xffffffffu, any_cnd)) {   // uniform; rare: the threshold bucket's keys
+                    for (int j = 0; j < per; ++j) {
+                        const unsigned cm = __ballot_sync(0xffffffffu, cnd[j]);
+                        cpos += __popc(cm & lt);
+                        cand_run += __popc(cm);
+                    }
+                }
+                for (int j = 0; j < per; ++j) {
+                    if (cnd[j]) {
+                        const int o = cpos + cmine++;
+                        ckey[o] = k[j];
+                        cidx[o] = base + j;
+                        list[pos + mine++] = (int)(0x80000000u | (unsigned)o);
+                    } else if (keep[j]) {
+                        list[pos + mine++] = base + j;
+                    }
+                }
+            };
+            if (vec) {
+                for (int q0 = 0; q0 < n4; q0 += 32 * U) {
+                    float4 v[U];
+#pragma unroll
+                    for (int u = 0; u < U; ++u)
+                        v[u] = q0 + 32 * u + lane < n4 ? __ldg(sc4 + q0 + 32 * u + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        const int q = q0 + 32 * u + lane;
+                        const unsigned k[4] = {topk_key(v[u].x), topk_key(v[u].y), topk_key(v[u].z), topk_key(v[u].w)};
+                        bool keep[4], cnd[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const bool in = 4 * q + j < n_valid;
+                            const float x = __uint_as_float(k[j]) * scale;
+                            keep[j] = in && x >= lo;
+                            cnd[j] = keep[j] && x < hi;
+                        }
+                        place(keep, cnd, k, 4 * q, 4);
+                    }
+                }
+            } else {
+                for (int b0 = 0; b0 < n_valid; b0 += 32) {
+                    const int b = b0 + lane;
+                    const bool in = b < n_valid;
+                    const unsigned k[4] = {in ? topk_key(sc[b]) : 0u, 0u, 0u, 0u};
+                    const float x = __uint_as_float(k[0]) * scale;
+                    const bool keep[4] = {in && x >= lo, false, false, false};
+                    const bool cnd[4] = {keep[0] && x < hi, false, false, false};
+                    place(keep, cnd, k, b, 1);
+                }
+            }
+            __syncwarp();
+            // the candidates taken: the `rem` largest keys, equal keys by index order
+            unsigned taken[CAND / 32];
+#pragma unroll
+            for (int h = 0; h < CAND / 32; ++h) {
+                const int o = 32 * h + lane;
+                bool t = false;
+                if (o < cnt) {
+                    const unsigned ko = ckey[o];
+                    int rank = 0;
+                    for (int o2 = 0; o2 < cnt; ++o2) {
+                        const unsigned k2 = ckey[o2];
+                        rank += k2 > ko || (k2 == ko && o2 < o);
+                    }
+                    t = rank < rem;
+                }
+                taken[h] = __ballot_sync(0xffffffffu, t);
+            }
+            // the list without the candidates not taken, in order: exactly KB entries
+            int out_run = 0;
+            for (int e0 = 0; e0 < list_run; e0 += 32) {
+                const int e = e0 + lane;
+                int val = 0;
+                bool keep = false;
+                if (e < list_run) {
+                    const int x = list[e];
+                    if (x < 0) {
+                        const int o = x & 0x7FFFFFFF;
+                        keep = (taken[o >> 5] >> (o & 31)) & 1u;
+                        val = cidx[o];
+                    } else {
+                        keep = true;
+                        val = x;
+                    }
+                }
+                const unsigned m = __ballot_sync(0xffffffffu, keep);
+                if (keep) out[out_run + __popc(m & lt)] = val;
+                out_run += __popc(m);
+            }
+            return;
+        }
+    }
+    // ---- Fallback (a threshold bucket of more than CAND keys, e.g. many equal
+    // scores): the radix select on the key bits, then the selection walk.
     for (int j = lane; j < WH_SLOTS; j += 32) hist[j] = 0;
     __syncwarp();
     for_keys([&](unsigned key) { atomicAdd(&hist[topk_slot(HB - 1 - (int)(key >> 20))], 1); });
@@ -627,7 +771,8 @@ size_t qsa_scores_bytes(int B, int n) { return (size_t)B * n * (n / qsa::R) * 4;
 
 size_t qsa_workspace_bytes(int B, int n) {
     auto ru = [](size_t x) { return (x + 255) & ~(size_t)255; };
-    return ru((size_t)B * n * qsa::HI * qsa::D * 2) + ru((size_t)B * (n / qsa::R) * qsa::D * 2) + ru(qsa_scores_bytes(B, n));
+    return ru((size_t)B * n * qsa::HI * qsa::D * 2) + ru((size_t)B * (n / qsa::R) * qsa::D * 2) + ru((size_t)B * n * 4) +
+           ru(qsa_scores_bytes(B, n));
 }
 
 cudaError_t launch_qsa_indexer(const QsaArgs &a, void *ws) {
@@ -639,6 +784,8 @@ cudaError_t launch_qsa_indexer(const QsaArgs &a, void *ws) {
     p += ru((size_t)a.B * a.n * HI * D * 2);
     __half *kb = reinterpret_cast<__half *>(p);
     p += ru((size_t)a.B * nb * D * 2);
+    float *rowmax = reinterpret_cast<float *>(p);   // per query row: its largest score
+    p += ru((size_t)a.B * a.n * 4);
     float *scores = a.scores ? a.scores : reinterpret_cast<float *>(p);
     cudaError_t e;
     const long long items = (long long)a.B * a.n + (long long)a.B * nb;
@@ -664,10 +811,12 @@ cudaError_t launch_qsa_indexer(const QsaArgs &a, void *ws) {
             return e;
         if ((e = cudaFuncSetAttribute(qsa_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM)) != cudaSuccess)
             return e;
+        if ((e = cudaMemsetAsync(rowmax, 0, (size_t)a.B * a.n * 4, a.stream)) != cudaSuccess) return e;
         const long long n_items = qsa_score_items(a.B, a.n);
         const int g = (int)(n_items < sms ? n_items : sms);
         if (g > 0) {
-            qsa_score_kernel<<<g, 64 + 32 * EPI_WARPS, SMEM, a.stream>>>(m, a.B, a.n, (int)n_items, tma_out, scores);
+            qsa_score_kernel<<<g, 64 + 32 * EPI_WARPS, SMEM, a.stream>>>(m, a.B, a.n, (int)n_items, tma_out, scores,
+                                                                          rowmax);
             if ((e = launched()) != cudaSuccess) return e;
         }
     }
@@ -678,7 +827,7 @@ cudaError_t launch_qsa_indexer(const QsaArgs &a, void *ws) {
             cudaSuccess)
             return e;
         qsa_topk_kernel<<<(unsigned)((rows + TOPK_WARPS - 1) / TOPK_WARPS), 32 * TOPK_WARPS, smem, a.stream>>>(
-            scores, a.n, rows, a.KB, a.sel);
+            scores, rowmax, a.n, rows, a.KB, a.sel);
         if ((e = launched()) != cudaSuccess) return e;
     }
     return cudaSuccess;
