@@ -87,6 +87,29 @@ def test_qsa_ties_are_bit_exact(cuda_device):
     np.testing.assert_array_equal(sel[0].cpu().numpy(), want)
 
 
+def test_qsa_equal_positive_scores(cuda_device):
+    """Keys that live in the unrotated dims 64..127 only and are the same for every
+    token: every block's pooled, rotated key is the same vector, so all complete
+    blocks of a row score the same positive value (bit-identical products).  More
+    equal keys than the threshold bucket's candidate list holds: the kernel's
+    fallback path; the smallest blocks win, as in the oracle."""
+    cfg = replace(QSA, B=1, n=900, budget=64)
+    inp = make_qsa_inputs(cfg, "cpu")
+    k = torch.zeros_like(inp["k"])
+    k[..., 64:] = inp["k"][0, 0, 64:].abs() + 0.5      # one positive key for every token
+    q = inp["q"].clone()
+    q[..., 64:] = q[..., 64:].abs()                       # positive products in every head
+    sel, sc = gdn.qsa_indexer(q.to(cuda_device), k.to(cuda_device), inp["w_q"].to(cuda_device),
+                              inp["w_k"].to(cuda_device), budget=cfg.budget, want_scores=True)
+    torch.cuda.synchronize()
+    sc = sc[0].cpu().numpy()
+    last = cfg.n - 1
+    assert (sc[last, :(last + 1) // 4] > 0).all() and np.unique(sc[last, :(last + 1) // 4]).size == 1
+    want, _ = oq.indexer(q[0].float().numpy(), k[0].float().numpy(), inp["w_q"].numpy(), inp["w_k"].numpy(),
+                         K=cfg.budget)
+    np.testing.assert_array_equal(sel[0].cpu().numpy(), want)
+
+
 def test_qsa_full_size_sampled_rows(cuda_device):
     """The bench workload (n = 32768, K = 2048): sampled rows against the oracle."""
     cfg = QSA
