@@ -267,6 +267,21 @@ GDN_API gdn_status_t gdn_layer_forward(const gdn_dims_t *dims, int d_model, cons
 GDN_API gdn_status_t gdn_layer_workspace_size(const gdn_dims_t *dims, int d_model, size_t *bytes);
 
 /*
+ * gdn_gemm_bf16 -- C [M, N] = A [M, K] B [K, N], the product the layer's
+ * projections use (slinene.github.io write-up of "On the Design of Qwen3.8-Next
+ * Architecture", 模块 A, 参数化: q, k, v, z and the gate logits are linear maps of
+ * the hidden state), on the library's tcgen05 GEMM: bf16 row-major operands with
+ * leading dimensions lda, ldb, ldc (elements), fp32 accumulation, C rounded to
+ * bf16 (round to nearest even).  K, lda and ldc multiples of 8; for N >= 64 also
+ * ldb; A, B and C 16-byte aligned (else GDN_ERR_ALIGNMENT; other violations
+ * GDN_ERR_INVALID_ARG).  N < 64 takes a stream-ordered workspace from the
+ * library's pool (B transposed).  M = 0 or N = 0 writes nothing.  An expired
+ * wait raises GDN_ERRF_GEMM.  Asynchronous on `stream`.
+ */
+GDN_API gdn_status_t gdn_gemm_bf16(int M, int N, int K, const void *A, int lda, const void *B, int ldb, void *C,
+                                   int ldc, gdn_stream_t stream);
+
+/*
  * gdn_decode_step -- one token for each of B = dims->num_seqs sequences,
  * reading and updating the per-head state in place.
  *

@@ -569,6 +569,31 @@ gdn_status_t gdn_qsa_indexer(int batch, int n, int heads, int d, int block, int 
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
+gdn_status_t gdn_gemm_bf16(int M, int N, int K, const void *A, int lda, const void *B, int ldb, void *C, int ldc,
+                           gdn_stream_t stream) {
+    tl_launches = 0;
+    if (M < 0 || N < 0 || K <= 0 || lda < K || ldb < N || ldc < N) return GDN_ERR_INVALID_ARG;
+    if (K % 8 || lda % 8 || ldc % 8 || (N >= 64 && ldb % 8)) return GDN_ERR_INVALID_ARG;
+    if (M == 0 || N == 0) return GDN_OK;
+    if (!A || !B || !C) return GDN_ERR_INVALID_ARG;
+    if (!aligned16(A) || !aligned16(B) || !aligned16(C)) return GDN_ERR_ALIGNMENT;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const size_t ws_bytes = gdn::gemm_workspace_bytes(N, K);
+    char *ws = nullptr;
+    if (ws_bytes) {
+        cudaMemPool_t pool;
+        if (get_pool(&pool) != cudaSuccess) return GDN_ERR_CUDA;
+        if (cudaMallocFromPoolAsync(reinterpret_cast<void **>(&ws), ws_bytes, pool, s) != cudaSuccess)
+            return GDN_ERR_CUDA;
+    }
+    cudaError_t e = gdn::launch_gemm_bf16(M, N, K, A, lda, B, ldb, C, ldc, ws, s);
+    if (ws) {
+        cudaError_t ef = cudaFreeAsync(ws, s);
+        if (e == cudaSuccess) e = ef;
+    }
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
 gdn_status_t gdn_layer_workspace_size(const gdn_dims_t *dims, int d_model, size_t *bytes) {
     gdn_status_t st = check_dims(dims, false);
     if (st != GDN_OK) return st;

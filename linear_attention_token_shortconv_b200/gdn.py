@@ -26,7 +26,8 @@ EXPORTS = ("gdn_prefill", "gdn_prefill_workspace_size", "gdn_decode_step", "gdn_
            "gdn_set_kernel_events", "gdn_last_call_launches", "gdn_device_error_status",
            "gdn_selftest_wait_timeout", "gdn_decode_multi", "gdn_prefill_backward",
            "gdn_prefill_backward_workspace_size", "gdn_qsa_indexer", "gdn_qsa_indexer_workspace_size",
-           "gdn_layer_forward", "gdn_layer_workspace_size", "gdn_prefill_ws", "gdn_prefill_conv_tail")
+           "gdn_layer_forward", "gdn_layer_workspace_size", "gdn_prefill_ws", "gdn_prefill_conv_tail",
+           "gdn_gemm_bf16")
 ERRF_PREP, ERRF_CHAIN, ERRF_DECODE, ERRF_QSA, ERRF_GEMM = 1, 2, 4, 8, 16
 
 
@@ -75,6 +76,9 @@ def load() -> ctypes.CDLL:
         lib.gdn_layer_forward.restype = ctypes.c_int
         lib.gdn_layer_workspace_size.argtypes = [D, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)]
         lib.gdn_layer_workspace_size.restype = ctypes.c_int
+        lib.gdn_gemm_bf16.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, P, ctypes.c_int, P, ctypes.c_int, P,
+                                      ctypes.c_int, P]
+        lib.gdn_gemm_bf16.restype = ctypes.c_int
         lib.gdn_prefill_noalloc.argtypes = [D] + [P] * 15
         lib.gdn_prefill_noalloc.restype = ctypes.c_int
         lib.gdn_selftest_umma.argtypes = [ctypes.c_int] * 5 + [P] * 5
@@ -282,6 +286,30 @@ def qsa_indexer(q, k, w_q, w_k, budget=2048, *, sel=None, scores=None, want_scor
         sel = sel[0]
         scores = None if scores is None else scores[0]
     return sel, scores
+
+
+def gemm_bf16(a, b, *, out=None, stream=None):
+    """gdn_gemm_bf16 on torch tensors: a [M, K], b [K, N] bf16 (row-major views
+    whose last dimension is contiguous) -> out [M, N] bf16."""
+    M, K = a.shape
+    K2, N = b.shape
+    if K2 != K:
+        raise ValueError(f"gemm_bf16: inner dimensions {K} and {K2}")
+    for name, t in (("a", a), ("b", b)):
+        if t.dtype != BF16 or t.device.type != "cuda" or t.stride(1) != 1:
+            raise ValueError(f"gemm_bf16: {name} must be a bf16 CUDA matrix with contiguous rows")
+    if out is None:
+        out = torch.empty((M, N), dtype=BF16, device=a.device)
+    if out.shape != (M, N) or out.dtype != BF16 or out.stride(1) != 1:
+        raise ValueError("gemm_bf16: out must be a bf16 [M, N] matrix with contiguous rows")
+    def mat_ptr(t):   # a row-strided matrix: rows need not be adjacent
+        return ctypes.c_void_p(t.data_ptr()) if t.numel() else None
+
+    with torch.cuda.device(_device(a, b, out)):
+        rc = load().gdn_gemm_bf16(M, N, K, mat_ptr(a), a.stride(0), mat_ptr(b), b.stride(0), mat_ptr(out),
+                                  out.stride(0), _stream(stream))
+    _check(rc, "gdn_gemm_bf16")
+    return out
 
 
 def layer_forward(x, w_in, conv_w, A, b_alpha, norm_w, w_o, H, dk, dv, S0=None, cu_seqlens=None, *,

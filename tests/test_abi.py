@@ -227,3 +227,16 @@ def test_conv_tail_rejects_bad_arguments(lib):
     assert lib.gdn_prefill_conv_tail(ctypes.byref(d), q, k, v, None, ctypes.c_void_p(4104), None) == 3
     bad = _dims(dk=96)
     assert lib.gdn_prefill_conv_tail(ctypes.byref(bad), q, k, v, None, FAKE[4], None) == 2
+
+
+def test_gemm_argument_validation(lib):
+    P = ctypes.c_void_p
+    a, b, c = P(4096), P(8192), P(12288)
+    assert lib.gdn_gemm_bf16(128, 256, 0, a, 64, b, 256, c, 256, None) == 1      # K = 0
+    assert lib.gdn_gemm_bf16(128, 256, 60, a, 64, b, 256, c, 256, None) == 1     # K not a multiple of 8
+    assert lib.gdn_gemm_bf16(128, 256, 64, a, 32, b, 256, c, 256, None) == 1     # lda < K
+    assert lib.gdn_gemm_bf16(128, 256, 64, a, 64, b, 260, c, 256, None) == 1     # wide: ldb not a multiple of 8
+    assert lib.gdn_gemm_bf16(128, 256, 64, P(4100), 64, b, 256, c, 256, None) == 3   # A misaligned
+    assert lib.gdn_gemm_bf16(128, 256, 64, a, 64, b, 256, None, 256, None) == 1   # no C
+    assert lib.gdn_gemm_bf16(0, 256, 64, None, 64, None, 256, None, 256, None) == 0   # nothing to do
+    assert lib.gdn_last_call_launches() == 0
