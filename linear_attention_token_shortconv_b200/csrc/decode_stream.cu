@@ -73,12 +73,6 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t b
         : "memory");
 }
 
-__device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
-                 "r"(umma::smem_u32(src)), "r"(bytes)
-                 : "memory");
-}
-
 __device__ __forceinline__ bool dwait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                       uint32_t max_polls = dstream::kMaxPolls) {
     for (uint32_t i = 0; i < max_polls; ++i) {
