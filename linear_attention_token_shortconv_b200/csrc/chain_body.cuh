@@ -135,7 +135,7 @@ __device__ __forceinline__ void chain_body(const ChainMaps &maps, const float *_
                                            const int32_t *__restrict__ cu_seqlens, int n_seq, int n_tok,
                                            int H, int h, int n, int c_lo, int c_hi,
                                            Tout *__restrict__ out, float *state_out,
-                                           const int *ready) {
+                                           const int *ready, bool own_tmem = true, uint32_t tmem_given = 0) {
     using namespace chain;
     // 4 * DV threads: warp w reads TMEM lane quadrant q = w % 4 and owns the
     // 32-column group cg = w / 4 of every row it touches.
@@ -166,7 +166,9 @@ __device__ __forceinline__ void chain_body(const ChainMaps &maps, const float *_
     const int c_end = min((s_end - s_begin + C - 1) / C, c_hi);
     const int n_chunks = max(0, c_end - c_lo);   // chunks handled by this launch
 
-    if (warp == 0) umma::tmem_alloc(tslot, TMEM_COLS);
+    // the tensor memory: allocated here, or (a CTA that runs several chains in turn:
+    // an allocation gives up the CTA's permit to allocate again) passed in
+    if (own_tmem && warp == 0) umma::tmem_alloc(tslot, TMEM_COLS);
     if (tid == 0) {
         for (int i = 0; i < 7; ++i) umma::mbar_init(full_a + i, 1);
         *abort_flag = 0;
@@ -194,7 +196,7 @@ __device__ __forceinline__ void chain_body(const ChainMaps &maps, const float *_
     umma::tc_fence_before();
     __syncthreads();
     umma::tc_fence_after();
-    const uint32_t tbase = *tslot;
+    const uint32_t tbase = own_tmem ? *tslot : tmem_given;
     const uint32_t tD = tbase + 2 * DV;
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
     // output gain of this thread's 32 columns, halved: sigmoid(z) (1 + w) y =
@@ -420,7 +422,7 @@ __device__ __forceinline__ void chain_body(const ChainMaps &maps, const float *_
             umma::mbar_wait_bounded(full_z + b, (uint32_t)(last >> 1) & 1u, 1u << 16);
         }
     }
-    if (warp == 0) umma::tmem_dealloc(tbase, TMEM_COLS);
+    if (own_tmem && warp == 0) umma::tmem_dealloc(tbase, TMEM_COLS);
 }
 
 }  // namespace gdn

@@ -222,11 +222,22 @@ struct FusedParams {
 template <typename Tout>
 __global__ void __launch_bounds__(fused::NT, 1) prefill_fused_kernel(const __grid_constant__ FusedParams P) {
     const int n_items = P.H * P.n_seq;
-    if ((int)blockIdx.x < P.n_chain) {   // chain role: item blockIdx.x
-        const int item = blockIdx.x, n = item / P.H, h = item % P.H;
-        chain_body<128, Tout>(P.maps, P.pa.decay, P.norm_w, P.S0, P.cu_seqlens, P.n_seq, P.n_tok, P.H, h, n, 0,
-                              P.max_chunks + 1, reinterpret_cast<Tout *>(P.out), P.S_final,
-                              P.ready + (size_t)item * P.max_chunks);
+    if ((int)blockIdx.x < P.n_chain) {   // chain role: items blockIdx.x, + n_chain, .. in turn
+        __shared__ uint32_t chain_tmem;
+        if (threadIdx.x < 32) umma::tmem_alloc(&chain_tmem, 512);   // once: one permit per CTA
+        umma::tc_fence_before();
+        __syncthreads();
+        umma::tc_fence_after();
+        const uint32_t tbase = chain_tmem;
+        for (int item = blockIdx.x; item < n_items; item += P.n_chain) {
+            const int n = item / P.H, h = item % P.H;
+            chain_body<128, Tout>(P.maps, P.pa.decay, P.norm_w, P.S0, P.cu_seqlens, P.n_seq, P.n_tok, P.H, h, n, 0,
+                                  P.max_chunks + 1, reinterpret_cast<Tout *>(P.out), P.S_final,
+                                  P.ready + (size_t)item * P.max_chunks, false, tbase);
+        }
+        umma::tc_fence_before();
+        __syncthreads();
+        if (threadIdx.x < 32) umma::tmem_dealloc(tbase, 512);
         return;
     }
     // prep role: two workers
@@ -253,11 +264,23 @@ __global__ void __launch_bounds__(fused::NT, 1) prefill_fused_kernel(const __gri
     // the next task index is fetched one task ahead (slot 1) so the atomic's round
     // trip overlaps a chunk; a chunk's ready flag is published during the next one
     // raw q, k, v rows of a task's chunk (and the three rows before it) into L2
+    // Task t -> (chunk c, item): the items come in rounds of n_chain (the chain CTAs
+    // take one item of each round in turn), and within a round chunk-major, so a
+    // round's chunks are prepped in the order its chains consume them.
+    auto task_at = [&](int t, int &c, int &item) {
+        const int per_round = P.n_chain * P.max_chunks;
+        const int r = t / per_round, local = t - r * per_round;
+        const int in_round = min(P.n_chain, n_items - r * P.n_chain);
+        c = local / in_round;
+        item = r * P.n_chain + local % in_round;
+    };
     auto prefetch_raw = [&](int t) {
         if (t >= n_tasks) return;
-        const int it = t % n_items, ns = it / P.H, hs = it % P.H;
+        int tc, it;
+        task_at(t, tc, it);
+        const int ns = it / P.H, hs = it % P.H;
         const int sb = P.cu_seqlens ? __ldg(P.cu_seqlens + ns) : ns * (P.n_tok / P.n_seq);
-        const int row = sb + (t / n_items) * C - 3;
+        const int row = sb + tc * C - 3;
         umma::tma_prefetch_l2_3d(&P.raw_q, 0, hs, row);
         umma::tma_prefetch_l2_3d(&P.raw_k, 0, hs, row);
         umma::tma_prefetch_l2_3d(&P.raw_v, 0, hs, row);
@@ -275,7 +298,8 @@ __global__ void __launch_bounds__(fused::NT, 1) prefill_fused_kernel(const __gri
             task_slot[1] = nt;
             prefetch_raw(nt);
         }
-        const int c = task / n_items, item = task % n_items;
+        int c, item;
+        task_at(task, c, item);
         const int n = item / P.H, h = item % P.H;
         int s_begin, s_end;
         if (P.cu_seqlens) { s_begin = __ldg(P.cu_seqlens + n); s_end = __ldg(P.cu_seqlens + n + 1); }
@@ -299,10 +323,17 @@ __global__ void __launch_bounds__(fused::NT, 1) prefill_fused_kernel(const __gri
 }
 
 int fused_chain_ctas(const PrefillArgs &a, int sms) {
-    // the fused kernel needs one chain CTA per (sequence, head) and leaves at least
-    // three quarters of the SMs to the prep workers
+    // The fused kernel leaves at least three quarters of the SMs to the prep
+    // workers: one chain CTA per (sequence, head) up to sms / 4 of them.  With equal
+    // lengths and up to one item per SM, sms / 4 chain CTAs take the items in turn
+    // (an item's chunks are prepped in chunk order across all items, so the chains
+    // a CTA takes later find theirs ready).  Packed varlen batches with more items
+    // use the segmented pipeline: their task space would be the longest sequence's
+    // chunks times the items, mostly empty.
     const int items = a.H * a.n_seq;
-    return (a.in_bf16 && a.dk == 128 && a.dv == 128 && a.n_tok > 0 && items <= sms / 4) ? items : 0;
+    if (!(a.in_bf16 && a.dk == 128 && a.dv == 128 && a.n_tok > 0)) return 0;
+    if (items <= sms / 4) return items;
+    return !a.cu_seqlens && items <= sms ? sms / 4 : 0;
 }
 
 cudaError_t launch_prefill_fused(const PrefillArgs &a, const TcWorkspace &w, int *ready, int sms,

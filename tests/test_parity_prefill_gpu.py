@@ -29,6 +29,12 @@ SMALL = [
     ("long-memory", scaled(PRETRAIN, lengths=(700, 64), H=2, long_memory=True, s0_var=0.02), TOL_BF16),
     # 40 (sequence, head) chains: the segmented pipeline (two segments) instead of the fused kernel
     ("many-chains-segmented", scaled(PRETRAIN, lengths=(700, 129), H=20, s0_var=0.02), TOL_BF16),
+    # equal lengths, more (sequence, head) items than a quarter of the SMs: the fused
+    # kernel's chain CTAs take several items in turn
+    ("many-chains-fused", scaled(PRETRAIN, lengths=(150,) * 6, H=10, s0_var=0.02), TOL_BF16),
+    # equal lengths, more items than SMs: the segmented pipeline with segments cut
+    # over one sequence's chunks
+    ("many-chains-equal-segmented", scaled(PRETRAIN, lengths=(70,) * 4, H=40, s0_var=0.02), TOL_BF16),
     ("dk64-dv128", replace(scaled(PRETRAIN, lengths=(190,), H=2), dk=64, dv=128, s0_var=0.02), TOL_BF16),
     ("dk128-dv64", replace(scaled(PRETRAIN, lengths=(190, 3), H=2), dk=128, dv=64, s0_var=0.02), TOL_BF16),
 ]
