@@ -70,7 +70,11 @@ Segments segments(const gdn_dims_t *d, bool equal_lengths = false) {
 size_t workspace_bytes(const gdn_dims_t *d) {
     const size_t nt = (size_t)d->total_tokens * d->H;
     if (use_tensor_cores(d)) {
-        const size_t flags = ((size_t)d->num_seqs * d->H * ((d->total_tokens + 63) / 64) + 1) * 4;
+        // ready flags and the task counter, then the varlen task list, its count and
+        // the item order
+        const size_t flags = ((size_t)d->num_seqs * d->H * ((d->total_tokens + 63) / 64) + 1) * 4 +
+                             (gdn::fused_task_capacity(d->total_tokens, d->num_seqs, d->H) + 1 +
+                              (size_t)d->num_seqs * d->H) * 4;
         return 3 * round_up(nt * d->dk * 2) + round_up(nt * d->dv * 2) + round_up(nt * 64 * 2) +
                round_up(nt * 4) + round_up(flags) +
                (segments(d).n > 1 ? round_up((size_t)d->num_seqs * d->H * d->dk * d->dv * 4) : 0);
@@ -197,7 +201,9 @@ cudaError_t prefill_run(const gdn::PrefillArgs &a, char *ext_ws) {
         w.Up = reinterpret_cast<__half *>(take(nt * a.dv * 2));
         w.Aqk = reinterpret_cast<__half *>(take(nt * 64 * 2));
         w.decay = reinterpret_cast<float *>(take(nt * 4));
-        int *ready = reinterpret_cast<int *>(take(((size_t)a.n_seq * a.H * ((a.n_tok + 63) / 64) + 1) * 4));
+        int *ready = reinterpret_cast<int *>(take(((size_t)a.n_seq * a.H * ((a.n_tok + 63) / 64) + 1) * 4 +
+                                                  (gdn::fused_task_capacity(a.n_tok, a.n_seq, a.H) + 1 +
+                                                   (size_t)a.n_seq * a.H) * 4));
         const Segments g = segments(dims, a.cu_seqlens == nullptr);
         int slot = 0, sms = 0;
         e = record(g_ev_begin, a.stream);

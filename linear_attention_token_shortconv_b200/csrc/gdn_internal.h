@@ -52,6 +52,7 @@ cudaError_t launch_chunk_prep(const PrefillArgs &a, const TcWorkspace &w);
 // the shape does not suit it.  `ready` holds n_seq * H * ceil(n_tok / 64) + 1
 // ints (flags and the task counter), zeroed by the launcher on `stream`.
 int fused_chain_ctas(const PrefillArgs &a, int sms);
+size_t fused_task_capacity(int n_tok, int n_seq, int H);
 cudaError_t launch_prefill_fused(const PrefillArgs &a, const TcWorkspace &w, int *ready, int sms,
                                  cudaStream_t stream);
 cudaError_t launch_chunk_chain(const PrefillArgs &a, const TcWorkspace &w);

@@ -64,6 +64,10 @@ PrepArgs prep_args(const PrefillArgs &a, const TcWorkspace &w) {
     return p;
 }
 
+// Entries of the fused kernel's varlen task list: at most one per chunk of every
+// (sequence, head), ceil(len / 64) <= len / 64 + 1 per sequence.
+size_t fused_task_capacity(int n_tok, int n_seq, int H) { return ((size_t)n_tok / prep::C + n_seq) * H; }
+
 // Tokens of the longest sequence, or their bound N_tok when cu_seqlens is given
 // (device memory, not read on the host).
 int longest_seq(const PrefillArgs &a) {
@@ -216,6 +220,9 @@ struct FusedParams {
     void *out;
     int *ready;        // [n_items][max_chunks], zero at launch
     int *next_task;    // zero at launch
+    // packed varlen batches: the tasks (chunk << 8 | item) in order, their count, and
+    // the items sorted by length (longest first); NULL for equal lengths
+    const int *task_table, *n_tasks_dev, *order;
     int n_seq, n_tok, H, max_chunks, n_chain;
 };
 
@@ -229,7 +236,8 @@ __global__ void __launch_bounds__(fused::NT, 1) prefill_fused_kernel(const __gri
         __syncthreads();
         umma::tc_fence_after();
         const uint32_t tbase = chain_tmem;
-        for (int item = blockIdx.x; item < n_items; item += P.n_chain) {
+        for (int slot = blockIdx.x; slot < n_items; slot += P.n_chain) {
+            const int item = P.order ? __ldg(P.order + slot) : slot;
             const int n = item / P.H, h = item % P.H;
             chain_body<128, Tout>(P.maps, P.pa.decay, P.norm_w, P.S0, P.cu_seqlens, P.n_seq, P.n_tok, P.H, h, n, 0,
                                   P.max_chunks + 1, reinterpret_cast<Tout *>(P.out), P.S_final,
@@ -259,7 +267,7 @@ __global__ void __launch_bounds__(fused::NT, 1) prefill_fused_kernel(const __gri
     umma::tc_fence_after();
     const uint32_t tbase = *tslot + 256 * half;
     const PrepGroupSync sy{1 + half};
-    const int n_tasks = P.max_chunks * n_items;
+    const int n_tasks = P.task_table ? __ldg(P.n_tasks_dev) : P.max_chunks * n_items;
     uint32_t phase = 0;
     // the next task index is fetched one task ahead (slot 1) so the atomic's round
     // trip overlaps a chunk; a chunk's ready flag is published during the next one
@@ -268,6 +276,12 @@ __global__ void __launch_bounds__(fused::NT, 1) prefill_fused_kernel(const __gri
     // take one item of each round in turn), and within a round chunk-major, so a
     // round's chunks are prepped in the order its chains consume them.
     auto task_at = [&](int t, int &c, int &item) {
+        if (P.task_table) {
+            const int e = __ldg(P.task_table + t);
+            c = e >> 8;
+            item = e & 255;
+            return;
+        }
         const int per_round = P.n_chain * P.max_chunks;
         const int r = t / per_round, local = t - r * per_round;
         const int in_round = min(P.n_chain, n_items - r * P.n_chain);
@@ -322,18 +336,65 @@ __global__ void __launch_bounds__(fused::NT, 1) prefill_fused_kernel(const __gri
     if (tid < 32) umma::tmem_dealloc(*tslot, 512);
 }
 
+// The fused kernel's task list for a packed varlen batch (one CTA): the items
+// sorted by chunk count, longest first (equal counts by item index), taken in
+// rounds of n_chain (the chain CTAs take one item of each round in turn), each
+// round's tasks chunk-major: chunk c of every item of the round that has one.
+// The task at (round r, chunk c, k-th item of the round) sits at
+// base_r + sum_k' min(c, chunks_k') + k.
+__global__ void fused_tasks_kernel(const int32_t *__restrict__ cu_seqlens, int n_seq, int H, int n_chain,
+                                   int *__restrict__ table, int *__restrict__ n_tasks, int *__restrict__ order) {
+    __shared__ int ch[256], ord[256], base[256];
+    const int n_items = n_seq * H, tid = threadIdx.x;
+    for (int i = tid; i < n_items; i += blockDim.x) {
+        const int n = i / H;
+        ch[i] = (__ldg(cu_seqlens + n + 1) - __ldg(cu_seqlens + n) + prep::C - 1) / prep::C;
+    }
+    __syncthreads();
+    for (int i = tid; i < n_items; i += blockDim.x) {
+        int rank = 0;
+        for (int j = 0; j < n_items; ++j) rank += ch[j] > ch[i] || (ch[j] == ch[i] && j < i);
+        ord[rank] = i;
+    }
+    __syncthreads();
+    const int rounds = (n_items + n_chain - 1) / n_chain;
+    if (tid == 0) {
+        int run = 0;
+        for (int r = 0; r < rounds; ++r) {
+            base[r] = run;
+            for (int k = r * n_chain; k < min(n_items, (r + 1) * n_chain); ++k) run += ch[ord[k]];
+        }
+        *n_tasks = run;
+    }
+    for (int i = tid; i < n_items; i += blockDim.x) order[i] = ord[i];
+    __syncthreads();
+    for (int r = 0; r < rounds; ++r) {
+        const int k0 = r * n_chain, in_r = min(n_chain, n_items - k0);
+        const int maxc = ch[ord[k0]];   // the round's longest item
+        for (int c = tid; c < maxc; c += blockDim.x) {
+            int off = base[r], alive = 0;
+            for (int k = 0; k < in_r; ++k) {
+                const int chk = ch[ord[k0 + k]];
+                off += min(c, chk);
+                alive += chk > c;   // the items still alive at c lead the round (sorted)
+            }
+            for (int k = 0; k < alive; ++k) table[off + k] = (c << 8) | ord[k0 + k];
+        }
+    }
+}
+
 int fused_chain_ctas(const PrefillArgs &a, int sms) {
     // The fused kernel leaves at least three quarters of the SMs to the prep
     // workers: one chain CTA per (sequence, head) up to sms / 4 of them.  With equal
     // lengths and up to one item per SM, sms / 4 chain CTAs take the items in turn
     // (an item's chunks are prepped in chunk order across all items, so the chains
-    // a CTA takes later find theirs ready).  Packed varlen batches with more items
-    // use the segmented pipeline: their task space would be the longest sequence's
-    // chunks times the items, mostly empty.
+    // a CTA takes later find theirs ready).  Packed varlen batches take a task list
+    // built on the device (fused_tasks_kernel; items up to 256, chunk rows up to 2^23).
     const int items = a.H * a.n_seq;
     if (!(a.in_bf16 && a.dk == 128 && a.dv == 128 && a.n_tok > 0)) return 0;
-    if (items <= sms / 4) return items;
-    return !a.cu_seqlens && items <= sms ? sms / 4 : 0;
+    if (items <= sms / 4 && !a.cu_seqlens) return items;
+    if (items > sms || items > 256 || (a.cu_seqlens && a.n_tok / prep::C > (1 << 22))) return 0;
+    return items <= sms / 4 ? items : sms / 4;
 }
 
 cudaError_t launch_prefill_fused(const PrefillArgs &a, const TcWorkspace &w, int *ready, int sms,
@@ -369,6 +430,16 @@ cudaError_t launch_prefill_fused(const PrefillArgs &a, const TcWorkspace &w, int
     P.next_task = ready + (size_t)a.n_seq * a.H * P.max_chunks;
     if ((e = cudaMemsetAsync(ready, 0, ((size_t)a.n_seq * a.H * P.max_chunks + 1) * sizeof(int), stream)) != cudaSuccess)
         return e;
+    if (a.cu_seqlens) {   // the task list, after the flags and the counter
+        int *tasks = P.next_task + 1;
+        int *n_tasks = tasks + fused_task_capacity(a.n_tok, a.n_seq, a.H);
+        int *order = n_tasks + 1;
+        fused_tasks_kernel<<<1, 1024, 0, stream>>>(a.cu_seqlens, a.n_seq, a.H, n_chain, tasks, n_tasks, order);
+        if ((e = launched()) != cudaSuccess) return e;
+        P.task_table = tasks;
+        P.n_tasks_dev = n_tasks;
+        P.order = order;
+    }
     void *args[] = {&P};
     const void *fn = a.out_bf16 ? reinterpret_cast<const void *>(prefill_fused_kernel<bf16>)
                                 : reinterpret_cast<const void *>(prefill_fused_kernel<float>);
