@@ -71,8 +71,8 @@ KERNEL_ROOFLINE = {"chunk_prep": ("hbm", 3 * 128 * 2 + 2 * 2),                  
 #     332.1 MB written for 262,144 token-heads; per token-head, scaled to the launch.
 NCU_TRAFFIC = {
     "prefill_fused": {"sources": ["prefill_tc.cu", "prep_body.cuh", "chain_body.cuh"],
-                      "sha1": "fb609260faf92392139e0fe20f0ed3cb53bc807f",
-                      "bytes_per_unit": (355.690752e6 + 332.133632e6) / (8192 * 32)},
+                      "sha1": "cd4ffa49425fd1dbb4527f4f543020e441674f18",
+                      "bytes_per_unit": (355.041280e6 + 332.478464e6) / (8192 * 32)},
 }
 
 
@@ -233,11 +233,11 @@ def bench_prefill(cfg, steps, warmup, world, rank, dev):
     S_final = torch.empty((cfg.num_seqs, H, cfg.dk, cfg.dv), dtype=torch.float32, device=dev)
     for _ in range(warmup):
         prefill_call(inp, out, S_final)
-    n_launch = gdn.last_call_launches()
+    n_slot = gdn.last_call_slots()
     torch.cuda.synchronize()
     mk = lambda n: [torch.cuda.Event(enable_timing=True) for _ in range(n)]
     evb, eve = mk(steps), mk(steps)
-    kb, ke = [mk(n_launch) for _ in range(steps)], [mk(n_launch) for _ in range(steps)]
+    kb, ke = [mk(n_slot) for _ in range(steps)], [mk(n_slot) for _ in range(steps)]
     for e in evb + eve + sum(kb, []) + sum(ke, []):   # materialise the CUDA handles
         e.record()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -259,11 +259,12 @@ def bench_prefill(cfg, steps, warmup, world, rank, dev):
     barrier(world)
     ms = max_over_ranks(start.elapsed_time(end) / steps, world)
     kern_ms = max_over_ranks(sum(b.elapsed_time(e) for b, e in zip(evb, eve)) / steps, world)
-    # launch slots: one fused persistent kernel, or chunk_prep / chunk_chain per segment
-    names = ("prefill_fused",) if n_launch == 1 else ("chunk_prep", "chunk_chain")
+    # launch slots: the fused persistent kernel (with its task-list builder for
+    # unequal lengths), or chunk_prep / chunk_chain per segment
+    names = ("prefill_fused",) if n_slot == 1 else ("chunk_prep", "chunk_chain")
     per = {n: [] for n in names}
     for i in range(steps):
-        for j in range(n_launch):
+        for j in range(n_slot):
             per[names[j % len(names)]].append(kb[i][j].elapsed_time(ke[i][j]))
     kernels = {}
     for name, xs in per.items():
@@ -680,7 +681,7 @@ def main():
                      "token_heads_per_launch": units_per_launch,
                      "avg_launch_ms": kd["avg_launch_ms"], "peak_kind": pk_kind,
                      "kernels": kernels,
-                     "path": {"what": "whole gdn_prefill call (both kernels, two streams)",
+                     "path": {"what": "whole gdn_prefill call (every kernel it launches)",
                               "call_ms": kern_ms, "bytes_per_token_head": PREFILL_BYTES_PER_TOKEN_HEAD,
                               "achieved_gbs": path_gbs, "frac": path_gbs / pk["hbm_gbs"]}},
         "tc": {"achieved_tflops": tc_achieved, "peak_tflops": pk["bf16_tflops"],

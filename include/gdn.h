@@ -410,6 +410,15 @@ GDN_API gdn_status_t gdn_set_kernel_events(void *const *begin, void *const *end,
 GDN_API int gdn_last_call_launches(void);
 
 /*
+ * Number of launch slots of the same call: the kernels, or groups of kernels,
+ * that gdn_set_kernel_events brackets with one (begin, end) pair each.  Equal
+ * to gdn_last_call_launches() except where a slot holds more than one kernel
+ * (the fused prefill of a packed batch of unequal lengths: its task-list
+ * builder and the fused kernel share one slot).  Host-side count.
+ */
+GDN_API int gdn_last_call_slots(void);
+
+/*
  * Device error flags.  Every wait inside the kernels (on an mbarrier fed by TMA
  * or by the tensor cores) is bounded; when one expires the kernel raises its
  * family's device error word, gives up its remaining waits promptly and

@@ -154,10 +154,12 @@ cudaError_t record(cudaEvent_t ev, cudaStream_t s) {
 // around that call's i-th kernel launch, on the stream the kernel runs on.
 std::vector<cudaEvent_t> g_kev_begin, g_kev_end;
 thread_local int tl_launches = 0;
+thread_local int tl_slots = 0;   // launch slots of the calling thread's last call
 
 template <class F>
 cudaError_t slot_launch(int *slot, cudaStream_t s, F &&launch) {
     const int i = (*slot)++;
+    ++tl_slots;
     const bool rec = i < (int)g_kev_begin.size();
     cudaError_t e = rec ? cudaEventRecord(g_kev_begin[i], s) : cudaSuccess;
     if (e == cudaSuccess) e = launch();
@@ -290,7 +292,10 @@ cudaError_t sm_count(int *out) {
 }
 
 void note_launch() { ++tl_launches; }
-void reset_launch_count() { tl_launches = 0; }
+void reset_launch_count() {
+    tl_launches = 0;
+    tl_slots = 0;
+}
 }  // namespace gdn
 
 extern "C" {
@@ -307,6 +312,8 @@ gdn_status_t gdn_set_kernel_events(void *const *begin, void *const *end, int n) 
 }
 
 int gdn_last_call_launches(void) { return tl_launches; }
+
+int gdn_last_call_slots(void) { return tl_slots; }
 
 gdn_status_t gdn_device_error_status(unsigned *flags, int clear, gdn_stream_t stream) {
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -414,6 +421,7 @@ gdn_status_t gdn_prefill(const gdn_dims_t *dims, const void *q, const void *k, c
                          const float *norm_w, const float *S0, const int32_t *cu_seqlens,
                          void *out, float *S_final, gdn_stream_t stream) {
     tl_launches = 0;
+    tl_slots = 0;
     gdn::PrefillArgs a;
     const gdn_status_t st = prefill_args(dims, q, k, v, conv_w, a_logit, b_logit, A, b_alpha, z, norm_w, S0,
                                          cu_seqlens, out, S_final, stream, &a);
@@ -428,6 +436,7 @@ gdn_status_t gdn_prefill_ws(const gdn_dims_t *dims, const void *q, const void *k
                             void *out, float *S_final, void *workspace, size_t workspace_bytes_given,
                             gdn_stream_t stream) {
     tl_launches = 0;
+    tl_slots = 0;
     gdn::PrefillArgs a;
     const gdn_status_t st = prefill_args(dims, q, k, v, conv_w, a_logit, b_logit, A, b_alpha, z, norm_w, S0,
                                          cu_seqlens, out, S_final, stream, &a);
@@ -456,6 +465,7 @@ gdn_status_t gdn_prefill_backward(const gdn_dims_t *dims, const void *q, const v
                                   void *d_a_logit, void *d_b_logit, float *d_A, float *d_b_alpha, void *d_z,
                                   float *d_norm_w, float *d_S0, gdn_stream_t stream) {
     tl_launches = 0;
+    tl_slots = 0;
     gdn_status_t st = check_dims(dims, false);
     if (st != GDN_OK) return st;
     if (dims->in_dtype != GDN_F32 || dims->out_dtype != GDN_F32 || dims->dk != dims->dv)
@@ -531,6 +541,7 @@ gdn_status_t gdn_qsa_indexer(int batch, int n, int heads, int d, int block, int 
                              const void *k, const float *w_q, const float *w_k, int32_t *sel, float *scores,
                              gdn_stream_t stream) {
     tl_launches = 0;
+    tl_slots = 0;
     if (batch <= 0 || n < 0 || heads <= 0 || d <= 0 || block <= 0 || budget <= 0) return GDN_ERR_INVALID_ARG;
     if (heads != 4 || d != 128 || block != 4 || budget % block != 0) return GDN_ERR_UNSUPPORTED;
     // row coordinates of the score kernel's tensor maps stay within int32
@@ -578,6 +589,7 @@ gdn_status_t gdn_qsa_indexer(int batch, int n, int heads, int d, int block, int 
 gdn_status_t gdn_gemm_bf16(int M, int N, int K, const void *A, int lda, const void *B, int ldb, void *C, int ldc,
                            gdn_stream_t stream) {
     tl_launches = 0;
+    tl_slots = 0;
     if (M < 0 || N < 0 || K <= 0 || lda < K || ldb < N || ldc < N) return GDN_ERR_INVALID_ARG;
     if (K % 8 || lda % 8 || ldc % 8 || (N >= 64 && ldb % 8)) return GDN_ERR_INVALID_ARG;
     if (M == 0 || N == 0) return GDN_OK;
@@ -613,6 +625,7 @@ gdn_status_t gdn_layer_forward(const gdn_dims_t *dims, int d_model, const void *
                                const void *w_o, const float *S0, const int32_t *cu_seqlens, void *y, float *S_final,
                                gdn_stream_t stream) {
     tl_launches = 0;
+    tl_slots = 0;
     gdn_status_t st = check_dims(dims, false);
     if (st != GDN_OK) return st;
     if (dims->in_dtype != GDN_BF16 || dims->out_dtype != GDN_BF16) return GDN_ERR_UNSUPPORTED;
@@ -679,6 +692,7 @@ gdn_status_t gdn_decode_step(const gdn_dims_t *dims, const void *q, const void *
                              const float *b_alpha, const void *z, const float *norm_w, float *S,
                              void *out, gdn_stream_t stream) {
     tl_launches = 0;
+    tl_slots = 0;
     gdn_status_t st = check_dims(dims, true);
     if (st != GDN_OK) return st;
     const void *vec[] = {q, k, v, conv_w, conv_hist, z, S, out};
@@ -726,6 +740,7 @@ gdn_status_t gdn_decode_multi(const gdn_dims_t *dims, int T, const void *q, cons
                               const float *norm_w, float *S, void *out, const int32_t *n_keep,
                               gdn_stream_t stream) {
     tl_launches = 0;
+    tl_slots = 0;
     if (!dims) return GDN_ERR_INVALID_ARG;
     if (T < 1 || T > 4) return GDN_ERR_INVALID_ARG;
     gdn_dims_t one = *dims;   // validate as a single-token step of the same shape

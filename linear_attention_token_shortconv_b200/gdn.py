@@ -23,7 +23,8 @@ STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "G
 # Every function the header declares (checked by the tests).
 EXPORTS = ("gdn_prefill", "gdn_prefill_workspace_size", "gdn_decode_step", "gdn_status_string",
            "gdn_set_timing_events", "gdn_selftest_umma", "gdn_prefill_noalloc",
-           "gdn_set_kernel_events", "gdn_last_call_launches", "gdn_device_error_status",
+           "gdn_set_kernel_events", "gdn_last_call_launches", "gdn_last_call_slots",
+           "gdn_device_error_status",
            "gdn_selftest_wait_timeout", "gdn_decode_multi", "gdn_prefill_backward",
            "gdn_prefill_backward_workspace_size", "gdn_qsa_indexer", "gdn_qsa_indexer_workspace_size",
            "gdn_layer_forward", "gdn_layer_workspace_size", "gdn_prefill_ws", "gdn_prefill_conv_tail",
@@ -89,6 +90,8 @@ def load() -> ctypes.CDLL:
         lib.gdn_set_kernel_events.restype = ctypes.c_int
         lib.gdn_last_call_launches.argtypes = []
         lib.gdn_last_call_launches.restype = ctypes.c_int
+        lib.gdn_last_call_slots.argtypes = []
+        lib.gdn_last_call_slots.restype = ctypes.c_int
         lib.gdn_device_error_status.argtypes = [ctypes.POINTER(ctypes.c_uint), ctypes.c_int, P]
         lib.gdn_device_error_status.restype = ctypes.c_int
         lib.gdn_selftest_wait_timeout.argtypes = [ctypes.c_uint, ctypes.c_uint, P]
@@ -525,6 +528,11 @@ def set_kernel_events(begins=(), ends=()):
 def last_call_launches() -> int:
     """Kernels launched by this thread's most recent prefill / decode call."""
     return int(load().gdn_last_call_launches())
+
+
+def last_call_slots() -> int:
+    """Launch slots (event-bracketed kernels or kernel groups) of the same call."""
+    return int(load().gdn_last_call_slots())
 
 
 def device_error_status(clear=False, stream=None):
