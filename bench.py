@@ -67,8 +67,8 @@ KERNEL_ROOFLINE = {"chunk_prep": ("hbm", 3 * 128 * 2 + 2 * 2),                  
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per unit from one
 # ncu capture of each kernel (profiles/), valid only while the kernel's sources
 # are the ones captured (sha1 over them); otherwise the JSON reports traffic null.
-#   prefill_fused: `bench.py --profile-case prefill 8192` (T = 8192, H = 32): 355.7 MB read +
-#     332.1 MB written for 262,144 token-heads; per token-head, scaled to the launch.
+#   prefill_fused: `bench.py --profile-case prefill 8192` (T = 8192, H = 32): 355.0 MB read +
+#     332.5 MB written for 262,144 token-heads; per token-head, scaled to the launch.
 NCU_TRAFFIC = {
     "prefill_fused": {"sources": ["prefill_tc.cu", "prep_body.cuh", "chain_body.cuh"],
                       "sha1": "cd4ffa49425fd1dbb4527f4f543020e441674f18",

@@ -419,6 +419,17 @@ __device__ __forceinline__ unsigned topk_key(float v) {
     return v > 0.f ? __float_as_uint(v) : 0u;   // scores >= 0: bits order like values (-0 -> 0)
 }
 
+// Descending rank HB - 1 - b of the value bucket b = min(HB - 1, floor(v * scale))
+// of a key v >= 0.  One fma rounded toward -inf adds the exact product to 2^23:
+// in [2^23, 2^24) the floats are the integers, so the sum's bits are 0x4B000000 +
+// floor(v * scale), with no float-to-integer conversion; larger products (and
+// +inf) clamp to the top bucket, rank 0.
+__device__ __forceinline__ int topk_vrank(unsigned key, float scale) {
+    float f;
+    asm("fma.rm.f32 %0, %1, %2, 0f4B000000;" : "=f"(f) : "f"(__uint_as_float(key)), "f"(scale));
+    return max(0, (qsa::HB - 1 + 0x4B000000) - __float_as_int(f));
+}
+
 // Counter of the bucket at descending rank u (u = NB - 1 - digit).  With one pad
 // word per 64 counters, the 64 consecutive ranks each lane sums in a pick of the
 // 11-bit digit fall in distinct banks across the warp.
@@ -543,10 +554,9 @@ qsa_topk_kernel(const float *__restrict__ scores, const float *__restrict__ rowm
         return;
     }
     const float scale = (float)HB / rmax;
-    auto vbucket = [&](unsigned key) { return min(HB - 1, (int)(__uint_as_float(key) * scale)); };
-    for (int j = lane; j < WH_SLOTS; j += 32) hist[j] = 0;
+    for (int j = lane; j < WH_SLOTS / 4; j += 32) reinterpret_cast<int4 *>(hist)[j] = make_int4(0, 0, 0, 0);
     __syncwarp();
-    for_keys([&](unsigned key) { atomicAdd(&hist[topk_slot(HB - 1 - vbucket(key))], 1); });
+    for_keys([&](unsigned key) { atomicAdd(&hist[topk_slot(topk_vrank(key, scale))], 1); });
     __syncwarp();
     {
         unsigned bstar;
@@ -558,9 +568,9 @@ qsa_topk_kernel(const float *__restrict__ scores, const float *__restrict__ rowm
             unsigned *ckey = reinterpret_cast<unsigned *>(hist + KB + CAND);   // [CAND]
             int *cidx = hist + KB + 2 * CAND;                               // [CAND]
             const unsigned lt = (1u << lane) - 1u;
-            // bucket(v) >= b* exactly when v * scale >= b* (truncation of a value >= 0;
-            // the top bucket also holds v * scale = 2048)
-            const float lo = (float)bstar, hi = bstar == (unsigned)(HB - 1) ? 3.0e38f : (float)(bstar + 1);
+            // the threshold bucket's rank: keys of a rank below it are taken, keys of
+            // its rank are the candidates (the same rank function as the histogram's)
+            const int rstar = HB - 1 - (int)bstar;
             int list_run = 0, cand_run = 0;
             // keys at or above the threshold bucket, in index order: index, or
             // 0x80000000 | candidate ordinal
@@ -605,9 +615,9 @@ qsa_topk_kernel(const float *__restrict__ scores, const float *__restrict__ rowm
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
                             const bool in = 4 * q + j < n_valid;
-                            const float x = __uint_as_float(k[j]) * scale;
-                            keep[j] = in && x >= lo;
-                            cnd[j] = keep[j] && x < hi;
+                            const int r = topk_vrank(k[j], scale);
+                            keep[j] = in && r <= rstar;
+                            cnd[j] = in && r == rstar;
                         }
                         place(keep, cnd, k, 4 * q, 4);
                     }
@@ -617,9 +627,9 @@ qsa_topk_kernel(const float *__restrict__ scores, const float *__restrict__ rowm
                     const int b = b0 + lane;
                     const bool in = b < n_valid;
                     const unsigned k[4] = {in ? topk_key(sc[b]) : 0u, 0u, 0u, 0u};
-                    const float x = __uint_as_float(k[0]) * scale;
-                    const bool keep[4] = {in && x >= lo, false, false, false};
-                    const bool cnd[4] = {keep[0] && x < hi, false, false, false};
+                    const int r = topk_vrank(k[0], scale);
+                    const bool keep[4] = {in && r <= rstar, false, false, false};
+                    const bool cnd[4] = {in && r == rstar, false, false, false};
                     place(keep, cnd, k, b, 1);
                 }
             }
