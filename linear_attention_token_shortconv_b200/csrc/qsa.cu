@@ -129,9 +129,10 @@ constexpr int A_HEAD = 2 * 16384;        // one head's query tile: 2 k-blocks x 
 constexpr int B_STAGE = 2 * 8192;        // one block tile: 2 k-blocks x [64 rows x 128 B]
 constexpr int OFF_A = 0;
 constexpr int OFF_B = OFF_A + HI * A_HEAD;             // 131072
-constexpr int EPI_WARPS = 8;             // two per TMEM lane quadrant, one 32-column half each
-constexpr int OFF_STG = OFF_B + NSB * B_STAGE;         // 180224: per epilogue warp, a 32 x 32 fp32 store tile
-constexpr int STG_TILE = 32 * 32 * 4;
+constexpr int EPI_WARPS = 8;             // two per TMEM lane quadrant (16, four per quadrant, measured slower)
+constexpr int EC = 4 * BN / EPI_WARPS;   // block columns per epilogue warp: 32 (or 16)
+constexpr int OFF_STG = OFF_B + NSB * B_STAGE;         // 180224: per epilogue warp, a 32 x EC fp32 store tile
+constexpr int STG_TILE = 32 * EC * 4;
 constexpr int OFF_BAR = OFF_STG + EPI_WARPS * STG_TILE;   // 212992
 constexpr int SMEM = OFF_BAR + 256 + 1024;             // barriers, TMEM slot, abort flag; alignment slack
 constexpr uint32_t TMEM_COLS = 512;                    // 2 stages x 4 heads x 64 columns
@@ -139,6 +140,14 @@ constexpr uint32_t MAX_POLLS = 1u << 24;
 }  // namespace qsa
 
 namespace {
+
+// N (32 or 16) consecutive TMEM columns of the warp's lane quadrant, no wait
+template <int N>
+__device__ __forceinline__ void qsa_tmem_ld(uint32_t taddr, uint32_t (&r)[N]) {
+    static_assert(N == 32 || N == 16, "32 or 16 columns");
+    if constexpr (N == 32) umma::tmem_ld32_nowait(taddr, r);
+    else umma::tmem_ld16_nowait(taddr, r);
+}
 
 __device__ __forceinline__ void mbar_arrive_local(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(umma::smem_u32(bar)) : "memory");
@@ -322,7 +331,7 @@ qsa_score_kernel(const __grid_constant__ QsaMaps maps, int B, int n, int n_items
         }
     } else if (warp >= 2) {
         // ----------------------------------------------------------------- epilogue
-        const int qd = warp & 3, c = 32 * ((warp - 2) >> 2);   // lane quadrant, column half
+        const int qd = warp & 3, c = EC * ((warp - 2) >> 2);   // lane quadrant, first column
         const uint32_t trow = tbase + ((uint32_t)(32 * qd) << 16);
         const bool vec = (nb & 3) == 0;   // rows start on 16-byte boundaries
         float *tile = reinterpret_cast<float *>(sm + OFF_STG + (warp - 2) * STG_TILE);
@@ -344,14 +353,20 @@ qsa_score_kernel(const __grid_constant__ QsaMaps maps, int B, int n, int n_items
                 if (!ok) break;
                 umma::tc_fence_after();
                 {
-                    // the four heads' columns in flight together, one wait
-                    uint32_t x[HI][32];
+                    // the four heads' columns in flight together, one wait; the TMEM
+                    // stage is free for the MMAs as soon as they are in registers
+                    uint32_t x[HI][EC];
 #pragma unroll
-                    for (int h = 0; h < HI; ++h) umma::tmem_ld32_nowait(trow + ts * (HI * BN) + h * BN + c, x[h]);
+                    for (int h = 0; h < HI; ++h) {
+                        qsa_tmem_ld(trow + ts * (HI * BN) + h * BN + c, x[h]);
+                    }
                     umma::tmem_ld_wait();
-                    float acc[32];
+                    umma::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_local(tempty + ts);
+                    float acc[EC];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
+                    for (int e = 0; e < EC; ++e) {
                         float a = fmaxf(__uint_as_float(x[0][e]), 0.f);
 #pragma unroll
                         for (int h = 1; h < HI; ++h) a += fmaxf(__uint_as_float(x[h][e]), 0.f);
@@ -359,15 +374,18 @@ qsa_score_kernel(const __grid_constant__ QsaMaps maps, int B, int n, int n_items
                     }
                     const int bs = BN * (item.bt0 + j) + c;
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
+                    for (int e = 0; e < EC; ++e)
                         if (bs + e < n_valid) lmax = fmaxf(lmax, acc[e]);
-                    if (tma_out && bs + 32 <= n_full) {   // uniform across the warp
+                    if (tma_out && bs + EC <= n_full) {   // uniform across the warp
                         if (lane == 0) umma::bulk_wait_read<0>();   // the last store has read the tile
                         __syncwarp();
-                        // row `lane`, 16-byte chunk e at chunk e ^ (lane % 8): the 128-byte swizzle
+                        // row `lane`, 16-byte chunk e at chunk e ^ (lane % 8) (128-byte
+                        // swizzle of 128-byte rows) or e ^ (lane / 2 % 4) (64-byte swizzle
+                        // of 64-byte rows)
+                        const int sw = EC == 32 ? (lane & 7) : ((lane >> 1) & 3);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            reinterpret_cast<float4 *>(tile + lane * 32)[e ^ (lane & 7)] =
+                        for (int e = 0; e < EC / 4; ++e)
+                            reinterpret_cast<float4 *>(tile + lane * EC)[e ^ sw] =
                                 make_float4(acc[4 * e], acc[4 * e + 1], acc[4 * e + 2], acc[4 * e + 3]);
                         umma::fence_proxy_async_smem();
                         __syncwarp();
@@ -375,20 +393,17 @@ qsa_score_kernel(const __grid_constant__ QsaMaps maps, int B, int n, int n_items
                             umma::tma_store_3d(&maps.sc, bs, 0, item.s * n + i0, tile);
                             umma::bulk_commit();
                         }
-                    } else if (vec && bs + 32 <= n_valid) {
+                    } else if (vec && bs + EC <= n_valid) {
                         float4 *d4 = reinterpret_cast<float4 *>(dst + bs);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e)
+                        for (int e = 0; e < EC / 4; ++e)
                             d4[e] = make_float4(acc[4 * e], acc[4 * e + 1], acc[4 * e + 2], acc[4 * e + 3]);
                     } else {
 #pragma unroll
-                        for (int e = 0; e < 32; ++e)
+                        for (int e = 0; e < EC; ++e)
                             if (bs + e < n_valid) dst[bs + e] = acc[e];
                     }
                 }
-                umma::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_local(tempty + ts);
             }
             // scores are >= 0, so their bit patterns order like the values
             if (ok && lmax > 0.f) atomicMax(reinterpret_cast<int *>(rowmax) + (size_t)item.s * n + i, __float_as_int(lmax));
@@ -411,7 +426,7 @@ long long qsa_score_items(int B, int n) {
 // ------------------------------------------------------------------ K5c: top-k
 namespace qsa {
 constexpr int HB = 2048;                  // buckets of the 11-bit digits
-constexpr int WH_SLOTS = HB + HB / 64;    // one warp's counters, one pad word per 64
+constexpr int WH_SLOTS = HB;              // one warp's counters
 constexpr int TOPK_WARPS = 8;             // rows (warps) per CTA
 }  // namespace qsa
 
@@ -420,20 +435,16 @@ __device__ __forceinline__ unsigned topk_key(float v) {
 }
 
 // Descending rank HB - 1 - b of the value bucket b = min(HB - 1, floor(v * scale))
-// of a key v >= 0.  One fma rounded toward -inf adds the exact product to 2^23:
-// in [2^23, 2^24) the floats are the integers, so the sum's bits are 0x4B000000 +
-// floor(v * scale), with no float-to-integer conversion; larger products (and
-// +inf) clamp to the top bucket, rank 0.
-__device__ __forceinline__ int topk_vrank(unsigned key, float scale) {
+// of a score v, taken as max(v, 0) (the same bucket as its topk_key).  One fma
+// rounded toward -inf adds the exact product to 2^23: in [2^23, 2^24) the floats
+// are the integers, so the sum's bits are 0x4B000000 + floor(v * scale), with no
+// float-to-integer conversion; larger products (and +inf) clamp to the top
+// bucket, rank 0.
+__device__ __forceinline__ int topk_vrank(float v, float scale) {
     float f;
-    asm("fma.rm.f32 %0, %1, %2, 0f4B000000;" : "=f"(f) : "f"(__uint_as_float(key)), "f"(scale));
+    asm("fma.rm.f32 %0, %1, %2, 0f4B000000;" : "=f"(f) : "f"(fmaxf(v, 0.f)), "f"(scale));
     return max(0, (qsa::HB - 1 + 0x4B000000) - __float_as_int(f));
 }
-
-// Counter of the bucket at descending rank u (u = NB - 1 - digit).  With one pad
-// word per 64 counters, the 64 consecutive ranks each lane sums in a pick of the
-// 11-bit digit fall in distinct banks across the warp.
-__device__ __forceinline__ int topk_slot(int u) { return u + (u >> 6); }
 
 __device__ __forceinline__ int warp_incl_scan(int x, int lane) {
 #pragma unroll
@@ -445,18 +456,20 @@ __device__ __forceinline__ int warp_incl_scan(int x, int lane) {
 }
 
 // One digit of the radix select, by one warp: among the keys matching `prefix`,
-// the bucket of the digit at `shift` (NB buckets) that holds the remaining-th
-// largest key.  Lane l sums the buckets of ranks PER l .. PER l + PER - 1
-// (descending digits); a warp scan of those sums crosses `remaining` at exactly
-// one lane, which walks its buckets; the extended prefix, the rank left inside
-// the bucket and the bucket's count come back to every lane.
+// the bucket of the digit at `shift` (NB buckets, counter u for descending rank
+// u = NB - 1 - digit) that holds the remaining-th largest key.  Lane l sums the
+// counters PER l .. PER l + PER - 1, starting at a lane-rotated one so that the
+// warp's reads fall in distinct banks; a warp scan of those sums crosses
+// `remaining` at exactly one lane, which walks its counters in order; the
+// extended prefix, the rank left inside the bucket and the bucket's count come
+// back to every lane.
 template <int NB>
 __device__ __forceinline__ void topk_pick(const int *hist, int remaining, unsigned prefix, int shift, int lane,
                                           unsigned &out_prefix, int &out_rem, int &out_cnt) {
     constexpr int PER = NB / 32;
     int c = 0;
 #pragma unroll 8
-    for (int j = 0; j < PER; ++j) c += hist[topk_slot(PER * lane + j)];
+    for (int j = 0; j < PER; ++j) c += hist[PER * lane + ((j + lane) & (PER - 1))];
     const int incl = warp_incl_scan(c, lane);
     const bool mine = incl >= remaining && incl - c < remaining;
     const int src = max(__ffs(__ballot_sync(0xffffffffu, mine)) - 1, 0);   // one lane when the counts cover `remaining`
@@ -465,7 +478,7 @@ __device__ __forceinline__ void topk_pick(const int *hist, int remaining, unsign
     if (mine) {
         int run = incl - c;
         for (int j = 0; j < PER; ++j) {
-            const int h = hist[topk_slot(PER * lane + j)];
+            const int h = hist[PER * lane + j];
             if (run + h >= remaining) {
                 p = prefix | ((unsigned)(NB - 1 - (PER * lane + j)) << shift);
                 r = remaining - run;
@@ -516,19 +529,28 @@ qsa_topk_kernel(const float *__restrict__ scores, const float *__restrict__ rowm
     const float4 *sc4 = reinterpret_cast<const float4 *>(sc);
     auto for_keys = [&](auto &&f) {
         if (vec) {
-            for (int q0 = lane; q0 < n4; q0 += 32 * U) {
+            const int nq = n_valid >> 2;   // quads of four complete blocks
+            for (int q0 = lane; q0 < nq; q0 += 32 * U) {
                 float4 v[U];
 #pragma unroll
                 for (int u = 0; u < U; ++u)
-                    v[u] = q0 + 32 * u < n4 ? __ldg(sc4 + q0 + 32 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    v[u] = q0 + 32 * u < nq ? __ldg(sc4 + q0 + 32 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
-                    const int q = q0 + 32 * u;
-                    const unsigned k[4] = {topk_key(v[u].x), topk_key(v[u].y), topk_key(v[u].z), topk_key(v[u].w)};
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        if (4 * q + j < n_valid) f(k[j]);
+                    if (q0 + 32 * u < nq) {
+                        f(v[u].x);
+                        f(v[u].y);
+                        f(v[u].z);
+                        f(v[u].w);
+                    }
                 }
+            }
+            if (lane == 0 && (n_valid & 3)) {   // the last quad, partly complete blocks
+                const float4 t = __ldg(sc4 + nq);
+                const float x[3] = {t.x, t.y, t.z};
+#pragma unroll
+                for (int j = 0; j < 3; ++j)
+                    if (j < (n_valid & 3)) f(x[j]);
             }
         } else {
             for (int b0 = lane; b0 < n_valid; b0 += 32 * U) {
@@ -537,7 +559,7 @@ qsa_topk_kernel(const float *__restrict__ scores, const float *__restrict__ rowm
                 for (int u = 0; u < U; ++u) v[u] = b0 + 32 * u < n_valid ? __ldg(sc + b0 + 32 * u) : 0.f;
 #pragma unroll
                 for (int u = 0; u < U; ++u)
-                    if (b0 + 32 * u < n_valid) f(topk_key(v[u]));
+                    if (b0 + 32 * u < n_valid) f(v[u]);
             }
         }
     };
@@ -556,7 +578,7 @@ qsa_topk_kernel(const float *__restrict__ scores, const float *__restrict__ rowm
     const float scale = (float)HB / rmax;
     for (int j = lane; j < WH_SLOTS / 4; j += 32) reinterpret_cast<int4 *>(hist)[j] = make_int4(0, 0, 0, 0);
     __syncwarp();
-    for_keys([&](unsigned key) { atomicAdd(&hist[topk_slot(topk_vrank(key, scale))], 1); });
+    for_keys([&](float v) { atomicAdd(&hist[topk_vrank(v, scale)], 1); });
     __syncwarp();
     {
         unsigned bstar;
@@ -602,32 +624,67 @@ qsa_topk_kernel(const float *__restrict__ scores, const float *__restrict__ rowm
                 }
             };
             if (vec) {
+                // lane l walks quads q0 + U l .. + U - 1: 4 U consecutive blocks, as bit
+                // masks of the kept keys and the candidates; one warp scan of the
+                // per-lane counts places the step's keys
                 for (int q0 = 0; q0 < n4; q0 += 32 * U) {
+                    const int qa = q0 + U * lane, base = 4 * qa;
                     float4 v[U];
 #pragma unroll
                     for (int u = 0; u < U; ++u)
-                        v[u] = q0 + 32 * u + lane < n4 ? __ldg(sc4 + q0 + 32 * u + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
+                        v[u] = qa + u < n4 ? __ldg(sc4 + qa + u) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    const int lim = n_valid - base;   // this lane's complete blocks
+                    const unsigned vmask = lim >= 4 * U ? (1u << (4 * U)) - 1u : lim > 0 ? (1u << lim) - 1u : 0u;
+                    unsigned kb = 0u, cb = 0u;
 #pragma unroll
                     for (int u = 0; u < U; ++u) {
-                        const int q = q0 + 32 * u + lane;
-                        const unsigned k[4] = {topk_key(v[u].x), topk_key(v[u].y), topk_key(v[u].z), topk_key(v[u].w)};
-                        bool keep[4], cnd[4];
+                        const float x[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
-                            const bool in = 4 * q + j < n_valid;
-                            const int r = topk_vrank(k[j], scale);
-                            keep[j] = in && r <= rstar;
-                            cnd[j] = in && r == rstar;
+                            const int r = topk_vrank(x[j], scale);
+                            kb |= (unsigned)(r <= rstar) << (4 * u + j);
+                            cb |= (unsigned)(r == rstar) << (4 * u + j);
                         }
-                        place(keep, cnd, k, 4 * q, 4);
+                    }
+                    kb &= vmask;
+                    cb &= vmask;
+                    const int c = __popc(kb);
+                    const int incl = warp_incl_scan(c, lane);
+                    const int pos = list_run + incl - c;
+                    list_run += __shfl_sync(0xffffffffu, incl, 31);
+                    if (__any_sync(0xffffffffu, cb != 0u)) {   // uniform; rare: the threshold bucket's keys
+                        const int cc = __popc(cb);
+                        const int cincl = warp_incl_scan(cc, lane);
+                        const int cpos = cand_run + cincl - cc;
+                        cand_run += __shfl_sync(0xffffffffu, cincl, 31);
+#pragma unroll
+                        for (int u = 0; u < U; ++u) {
+                            const float x[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const int e = 4 * u + j;
+                                if ((cb >> e) & 1u) {
+                                    const unsigned below = (1u << e) - 1u;
+                                    const int o = cpos + __popc(cb & below);
+                                    ckey[o] = topk_key(x[j]);
+                                    cidx[o] = base + e;
+                                    list[pos + __popc(kb & below)] = (int)(0x80000000u | (unsigned)o);
+                                }
+                            }
+                        }
+                    }
+                    for (unsigned m = kb & ~cb; m != 0u; m &= m - 1u) {
+                        const int e = __ffs(m) - 1;
+                        list[pos + __popc(kb & ((1u << e) - 1u))] = base + e;
                     }
                 }
             } else {
                 for (int b0 = 0; b0 < n_valid; b0 += 32) {
                     const int b = b0 + lane;
                     const bool in = b < n_valid;
-                    const unsigned k[4] = {in ? topk_key(sc[b]) : 0u, 0u, 0u, 0u};
-                    const int r = topk_vrank(k[0], scale);
+                    const float x = in ? sc[b] : 0.f;
+                    const unsigned k[4] = {topk_key(x), 0u, 0u, 0u};
+                    const int r = topk_vrank(x, scale);
                     const bool keep[4] = {in && r <= rstar, false, false, false};
                     const bool cnd[4] = {in && r == rstar, false, false, false};
                     place(keep, cnd, k, b, 1);
@@ -679,7 +736,7 @@ qsa_topk_kernel(const float *__restrict__ scores, const float *__restrict__ rowm
     // scores): the radix select on the key bits, then the selection walk.
     for (int j = lane; j < WH_SLOTS; j += 32) hist[j] = 0;
     __syncwarp();
-    for_keys([&](unsigned key) { atomicAdd(&hist[topk_slot(HB - 1 - (int)(key >> 20))], 1); });
+    for_keys([&](float v) { atomicAdd(&hist[HB - 1 - (int)(topk_key(v) >> 20)], 1); });
     __syncwarp();
     unsigned prefix;
     int remaining, cnt;
@@ -689,18 +746,20 @@ qsa_topk_kernel(const float *__restrict__ scores, const float *__restrict__ rowm
         __syncwarp();
         for (int j = lane; j < WH_SLOTS; j += 32) hist[j] = 0;
         __syncwarp();
-        for_keys([&](unsigned key) {
-            if ((key & mask) == prefix) atomicAdd(&hist[topk_slot(HB - 1 - (int)((key >> 9) & (HB - 1)))], 1);
+        for_keys([&](float v) {
+            const unsigned key = topk_key(v);
+            if ((key & mask) == prefix) atomicAdd(&hist[HB - 1 - (int)((key >> 9) & (HB - 1))], 1);
         });
         __syncwarp();
         topk_pick<HB>(hist, remaining, prefix, 9, lane, prefix, remaining, cnt);
         mask = 0xFFFFFE00u;
         if (cnt != remaining) {
             __syncwarp();
-            for (int j = lane; j < topk_slot(512); j += 32) hist[j] = 0;
+            for (int j = lane; j < 512; j += 32) hist[j] = 0;
             __syncwarp();
-            for_keys([&](unsigned key) {
-                if ((key & mask) == prefix) atomicAdd(&hist[topk_slot(511 - (int)(key & 511u))], 1);
+            for_keys([&](float v) {
+                const unsigned key = topk_key(v);
+                if ((key & mask) == prefix) atomicAdd(&hist[511 - (int)(key & 511u)], 1);
             });
             __syncwarp();
             topk_pick<512>(hist, remaining, prefix, 0, lane, prefix, remaining, cnt);
@@ -816,7 +875,7 @@ cudaError_t launch_qsa_indexer(const QsaArgs &a, void *ws) {
             return e;
         // score rows on 16-byte boundaries
         const bool tma_out = (nb & 3) == 0 && (reinterpret_cast<uintptr_t>(scores) & 15) == 0;
-        if (tma_out && (e = make_tma_rows_f32(reinterpret_cast<TmaMap *>(&m.sc), scores, nb, a.B * a.n, 32, 32)) !=
+        if (tma_out && (e = make_tma_rows_f32(reinterpret_cast<TmaMap *>(&m.sc), scores, nb, a.B * a.n, EC, 32)) !=
                            cudaSuccess)
             return e;
         if ((e = cudaFuncSetAttribute(qsa_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM)) != cudaSuccess)

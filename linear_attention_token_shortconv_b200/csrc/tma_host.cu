@@ -53,8 +53,8 @@ cudaError_t make_tma_3d(TmaMap *out, const void *base, bool bf16, int inner, int
 }
 
 // Rows of fp32 values [rows][cols] (row stride cols * 4 bytes, a multiple of 16)
-// as a 3-D map {cols, 1, rows} with boxes {box_cols, 1, box_rows}, 128-byte
-// swizzle: box_cols * 4 must be at most 128.
+// as a 3-D map {cols, 1, rows} with boxes {box_cols, 1, box_rows}: box_cols = 32
+// (128-byte rows, 128-byte swizzle) or 16 (64-byte rows, 64-byte swizzle).
 cudaError_t make_tma_rows_f32(TmaMap *out, const void *base, int cols, int rows, int box_cols, int box_rows) {
     EncodeTiledFn fn;
     cudaError_t e = encoder(&fn);
@@ -65,7 +65,8 @@ cudaError_t make_tma_rows_f32(TmaMap *out, const void *base, int cols, int rows,
     const cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(reinterpret_cast<CUtensorMap *>(out->bytes), CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
                     const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                    box_cols == 32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
