@@ -48,7 +48,17 @@ constexpr double ROPE_BASE = 10000.0;
 }  // namespace qsa
 
 // ------------------------------------------------------------------ K5a: prep
-__device__ __forceinline__ void qsa_norm_rope(float (&x)[4], const float *__restrict__ w, long long pos,
+// cos and sin of the rotation of the pair (lane, lane + 32) at position pos:
+// the angle pos * base^(-lane / 32) (inv_freq) formed and reduced in double
+// precision, since positions reach 1e5 and more
+__device__ __forceinline__ void qsa_rope_cs(long long pos, double inv_freq, float &c, float &s) {
+    double sd, cd;
+    sincos((double)pos * inv_freq, &sd, &cd);
+    c = (float)cd;
+    s = (float)sd;
+}
+
+__device__ __forceinline__ void qsa_norm_rope(float (&x)[4], const float *__restrict__ w, float c, float s,
                                               int lane) {
     // lane holds dims lane, lane + 32, lane + 64, lane + 96
     float ss = 0.f;
@@ -58,11 +68,7 @@ __device__ __forceinline__ void qsa_norm_rope(float (&x)[4], const float *__rest
     const float rn = 1.0f / sqrtf(ss / qsa::D + kNormEps);
 #pragma unroll
     for (int u = 0; u < 4; ++u) x[u] *= rn * __ldg(w + lane + 32 * u);
-    // rotate the pair (lane, lane + 32) by pos * base^(-lane / 32)
-    const double ang = (double)pos * pow(qsa::ROPE_BASE, -(double)lane / 32.0);
-    double sd, cd;
-    sincos(ang, &sd, &cd);
-    const float c = (float)cd, s = (float)sd;
+    // rotate the pair (lane, lane + 32)
     const float a = x[0], b = x[1];
     x[0] = a * c - b * s;
     x[1] = a * s + b * c;
@@ -75,16 +81,18 @@ qsa_prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const fl
     const int nb = n / R;
     const long long n_q = (long long)B * n, n_items = n_q + (long long)B * nb;
     const int lane = threadIdx.x & 31;
+    const double inv_freq = pow(ROPE_BASE, -(double)lane / 32.0);   // base^(-lane / 32), once per thread
     for (long long it = (long long)blockIdx.x * 8 + (threadIdx.x >> 5); it < n_items; it += (long long)gridDim.x * 8) {
-        if (it < n_q) {   // query row (sequence it / n, token it % n), all heads
-            const long long i = it % n;
+        if (it < n_q) {   // query row (sequence it / n, token it % n), all heads: one rotation
+            float c, s;
+            qsa_rope_cs(it % n, inv_freq, c, s);
 #pragma unroll
             for (int h = 0; h < HI; ++h) {
                 const bf16 *src = q + (it * HI + h) * D;
                 float x[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) x[u] = __bfloat162float(src[lane + 32 * u]);
-                qsa_norm_rope(x, w_q, i, lane);
+                qsa_norm_rope(x, w_q, c, s, lane);
                 __half *dst = qr + (it * HI + h) * D;
 #pragma unroll
                 for (int u = 0; u < 4; ++u) dst[lane + 32 * u] = __float2half_rn(x[u]);
@@ -100,7 +108,9 @@ qsa_prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const fl
                 for (int t = 0; t < R; ++t) acc += __bfloat162float(src[t * D + lane + 32 * u]);
                 x[u] = acc * (1.0f / R);
             }
-            qsa_norm_rope(x, w_k, b * R, lane);
+            float c, sn;
+            qsa_rope_cs(b * R, inv_freq, c, sn);
+            qsa_norm_rope(x, w_k, c, sn, lane);
             __half *dst = kb + jb * D;
 #pragma unroll
             for (int u = 0; u < 4; ++u) dst[lane + 32 * u] = __float2half_rn(x[u]);
