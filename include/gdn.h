@@ -106,8 +106,10 @@ typedef struct {
  * exp() of it is already exactly 0 in fp32, so a logit that makes it overflow to
  * -inf (near 3e38 / exp(A)) gives alpha = 0 as in exact arithmetic instead of
  * NaN.  On the tensor-core path (bf16 inputs, dk = 128) a call with
- * dk = dv = 128 and at most SMs / 4 (sequence, head) pairs runs as one
- * cooperative persistent kernel on `stream` (one CTA per SM); other long inputs
+ * dk = dv = 128 and at most as many (sequence, head) pairs as the device has
+ * SMs (and at most 256) runs as one cooperative persistent kernel on `stream`
+ * (one CTA per SM; with cu_seqlens after a one-CTA kernel that builds its task
+ * list on the device); other long inputs
  * run in chunk segments whose kernels overlap on `stream` and on two
  * library-owned streams of the same device, forked from and joined back into
  * `stream` with events, so work queued on `stream` afterwards sees the results.  When
@@ -388,9 +390,11 @@ GDN_API gdn_status_t gdn_set_timing_events(void *begin, void *end);
  * the caller; the library copies the n handles) are recorded around launch
  * slot i of every following gdn_prefill / gdn_decode_step call, on the stream
  * that slot's kernel runs on.  Slots in launch order:
- *   gdn_prefill, tensor-core path with dk = dv = 128 and at most a quarter as
- *     many (sequence, head) pairs as the device has SMs: one slot, the fused
- *     persistent kernel, on the caller's stream;
+ *   gdn_prefill, tensor-core path with dk = dv = 128 and at most as many
+ *     (sequence, head) pairs as the device has SMs (and at most 256): one slot,
+ *     the fused persistent kernel, on the caller's stream; with cu_seqlens the
+ *     slot also holds the one-CTA kernel that builds its task list, launched
+ *     just before it (two launches, one slot);
  *   gdn_prefill, other tensor-core shapes, n segments: chunk_prep(0),
  *     chunk_chain(0), chunk_prep(1), chunk_chain(1), ... -- chunk_prep of even
  *     segments on the caller's stream, of odd segments on a second library
