@@ -270,7 +270,9 @@ __global__ void __launch_bounds__(fused::NT, 1) prefill_fused_kernel(const __gri
     const int n_tasks = P.task_table ? __ldg(P.n_tasks_dev) : P.max_chunks * n_items;
     uint32_t phase = 0;
     // the next task index is fetched one task ahead (slot 1) so the atomic's round
-    // trip overlaps a chunk; a chunk's ready flag is published during the next one
+    // trip overlaps a chunk, by a thread of warp 7: warps 0 and 1 compute the
+    // gates first thing in a chunk, warp 7 has time to wait for the atomic; a
+    // chunk's ready flag is published during the next one
     // raw q, k, v rows of a task's chunk (and the three rows before it) into L2
     // Task t -> (chunk c, item): the items come in rounds of n_chain (the chain CTAs
     // take one item of each round in turn), and within a round chunk-major, so a
@@ -299,17 +301,23 @@ __global__ void __launch_bounds__(fused::NT, 1) prefill_fused_kernel(const __gri
         umma::tma_prefetch_l2_3d(&P.raw_k, 0, hs, row);
         umma::tma_prefetch_l2_3d(&P.raw_v, 0, hs, row);
     };
-    if (wtid == 0) {
+    constexpr int kFetcher = 224;   // lane 0 of the worker's warp 7
+    if (wtid == kFetcher) {
         task_slot[0] = atomicAdd(P.next_task, 1);
         prefetch_raw(task_slot[0]);
     }
     sy.sync();
     int task = task_slot[0];
     int *pending = nullptr;   // ready flag of the last chunk this worker wrote
-    while (task < n_tasks) {
-        if (wtid == 0) {
+    // Two task slots in turn: in iteration k the fetcher writes the next task to
+    // slot (k + 1) % 2 before the chunk, and every thread reads it after the chunk.
+    // The chunk's own barriers order that write before those reads, and the reads
+    // of iteration k - 1 (the same slot) before the write.
+    for (int k = 0; task < n_tasks; ++k) {
+        const int ns = (k + 1) & 1;
+        if (wtid == kFetcher) {
             const int nt = atomicAdd(P.next_task, 1);
-            task_slot[1] = nt;
+            task_slot[ns] = nt;
             prefetch_raw(nt);
         }
         int c, item;
@@ -318,14 +326,14 @@ __global__ void __launch_bounds__(fused::NT, 1) prefill_fused_kernel(const __gri
         int s_begin, s_end;
         if (P.cu_seqlens) { s_begin = __ldg(P.cu_seqlens + n); s_end = __ldg(P.cu_seqlens + n + 1); }
         else { const int L = P.n_tok / P.n_seq; s_begin = n * L; s_end = s_begin + L; }
-        if (s_begin + c * C < s_end) {   // else: past this sequence's end, no such chunk
+        if (s_begin + c * C < s_end) {
             if (!prep_one_chunk<128>(sy, P.pa, wsm, tbase, bar, phase, wtid, h, s_begin, s_end, c, pending))
                 break;
             pending = P.ready + (size_t)item * P.max_chunks + c;
+        } else {
+            sy.sync();   // past this sequence's end, no such chunk: the barrier the slots need
         }
-        sy.sync();   // slot 1 is written (thread 0, before the chunk) and read by all after it
-        task = task_slot[1];
-        sy.sync();   // every thread has read slot 1 before thread 0 rewrites it
+        task = task_slot[ns];
     }
     if (pending && wtid == 0) {
         __threadfence();
