@@ -22,13 +22,15 @@
 //      stages; warp-specialised producer, MMA issuer and eight epilogue warps
 //      (ReLU, head sum, 128-byte row segments of the complete blocks' scores).
 //      Only block tiles that hold a complete block of the query tile are visited.
-//  K5c qsa_topk_kernel: one warp per query row, no block barriers: a radix
-//      select on the score bits (scores are >= 0, so their bit patterns order
-//      like the values; digits of 11, 11 and 9 bits counted in the warp's own
-//      shared histogram, stopping at the first digit whose bucket is taken
-//      whole) finds the threshold, then one walk over the row in index order
-//      writes the selected blocks ascending, equal scores at the threshold taken
-//      from the smallest index.
+//  K5c qsa_topk_kernel: one warp per query row, no block barriers: the row's
+//      scores counted into 2048 value buckets over [0, row max] (the score kernel
+//      leaves each row's largest score) in the warp's own shared histogram; the
+//      bucket holding the K_B-th largest score is the threshold, and one walk over
+//      the row in index order takes the keys above it and ranks the few inside
+//      it, equal scores taken from the smallest index.  A threshold bucket of
+//      more than 64 keys (many equal scores) falls back to a radix select on the
+//      score bits (scores are >= 0, so their bit patterns order like the values;
+//      digits of 11, 11 and 9 bits).  The selected blocks come out ascending.
 #include <cuda.h>
 #include <cuda_fp16.h>
 
@@ -503,13 +505,16 @@ __device__ __forceinline__ void topk_pick(const int *hist, int remaining, unsign
     out_cnt = __shfl_sync(0xffffffffu, cnt, src);
 }
 
-// One warp per query row, no block barriers: the row's keys (score bits) are read
-// from the score matrix for each pass -- the first from HBM, the rest from L2 --
-// and counted into the warp's own histogram with shared atomics.  A radix select
-// on digits of 11, 11 and 9 bits finds the threshold (stopping at the first
-// digit whose bucket is taken whole); the selection then walks the row in index
-// order, 128 keys per step (a 16-byte load per lane when rows are aligned): the
-// keys above the threshold, and the first `remaining` equal to it, are written at
+// One warp per query row, no block barriers: the row's keys are read from the
+// score matrix for each pass -- the first from HBM, the rest from L2 -- and
+// counted into the warp's own histogram with shared atomics.  Fast path: value
+// buckets over [0, row max] find the threshold bucket, and one walk places the
+// keys above it and the bucket's candidates in index order (see below).
+// Fallback (a crowded threshold bucket): a radix select on digits of 11, 11 and
+// 9 bits of the score bits finds the threshold (stopping at the first digit
+// whose bucket is taken whole); the selection then walks the row in index order,
+// 128 keys per step (a 16-byte load per lane when rows are aligned): the keys
+// above the threshold, and the first `remaining` equal to it, are written at
 // ascending positions found by warp scans of per-lane counts.
 __global__ void __launch_bounds__(32 * qsa::TOPK_WARPS)
 qsa_topk_kernel(const float *__restrict__ scores, const float *__restrict__ rowmax, int n, long long n_rows, int KB,
