@@ -582,13 +582,17 @@ def profile_case(kind, size):
                   two warm-up calls, then one call
       pretrain T  the pretraining shape with 4 sequences of T tokens (H = 16):
                   two warm-up calls, then one call
+      segmented T 4 sequences of T tokens with H = 40 (160 (sequence, head)
+                  items, more than the SMs: the segmented prep + chain
+                  pipeline): two warm-up calls, then one call
       decode B    decode steps for B sequences x 32 heads, d = 128: three steps
       backward T  prefill backward, 4 sequences x T tokens, H = 16, d = 128, fp32: three calls
       qsa n       QSA indexer on one sequence of n tokens, K = 2048: three calls
       layer T     layer forward, 4 sequences x T tokens, H = 16, d_model = 2048: three calls"""
     dev = torch.device("cuda", 0)
-    if kind in ("prefill", "pretrain"):
-        cfg = replace(LONG, lengths=(size,)) if kind == "prefill" else replace(PRETRAIN, lengths=(size,) * 4)
+    if kind in ("prefill", "pretrain", "segmented"):
+        cfg = (replace(LONG, lengths=(size,)) if kind == "prefill" else
+               replace(PRETRAIN, lengths=(size,) * 4, H=40 if kind == "segmented" else PRETRAIN.H))
         inp = make_prefill_inputs(cfg, dev)
         out = torch.empty((cfg.total_tokens, cfg.H, cfg.dv), dtype=torch.bfloat16, device=dev)
         S = torch.empty((cfg.num_seqs, cfg.H, cfg.dk, cfg.dv), device=dev)
@@ -648,7 +652,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--profile-case", nargs=2, metavar=("KIND", "SIZE"),
                     help="run one small workload for an ncu capture instead of the benchmark "
-                         "(prefill T | pretrain T | decode B | backward T | qsa n | layer T)")
+                         "(prefill T | pretrain T | segmented T | decode B | backward T | qsa n | layer T)")
     args = ap.parse_args()
     if args.profile_case:
         profile_case(args.profile_case[0], int(args.profile_case[1]))
