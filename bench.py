@@ -586,6 +586,8 @@ def profile_case(kind, size):
                   items, more than the SMs: the segmented prep + chain
                   pipeline): two warm-up calls, then one call
       decode B    decode steps for B sequences x 32 heads, d = 128: three steps
+      decode4 B   multi-token decode steps (4 tokens per sequence, all committed)
+                  for B sequences x 32 heads, d = 128: three steps
       backward T  prefill backward, 4 sequences x T tokens, H = 16, d = 128, fp32: three calls
       qsa n       QSA indexer on one sequence of n tokens, K = 2048: three calls
       layer T     layer forward, 4 sequences x T tokens, H = 16, d_model = 2048: three calls"""
@@ -607,6 +609,16 @@ def profile_case(kind, size):
         for t in range(3):
             gdn.decode_step(d["q"][t], d["k"][t], d["v"][t], d["conv_w"], d["ring"], d["a_logit"][t],
                             d["b_logit"][t], d["A"], d["b_alpha"], d["z"][t], d["norm_w"], d["S"], out=out)
+        torch.cuda.synchronize()
+        print("ok", float(out.float().abs().mean()))
+    elif kind == "decode4":
+        cfg = replace(DECODE, B=size)
+        d = make_decode_inputs(cfg, dev)
+        m = {key: d[key][:4].transpose(0, 1).contiguous() for key in ("q", "k", "v", "z", "a_logit", "b_logit")}
+        out = torch.empty((cfg.B, 4, cfg.H, cfg.dv), dtype=torch.bfloat16, device=dev)
+        for _ in range(3):
+            gdn.decode_multi(m["q"], m["k"], m["v"], d["conv_w"], d["ring"], m["a_logit"], m["b_logit"], d["A"],
+                             d["b_alpha"], m["z"], d["norm_w"], d["S"], out=out)
         torch.cuda.synchronize()
         print("ok", float(out.float().abs().mean()))
     elif kind == "backward":
@@ -652,7 +664,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--profile-case", nargs=2, metavar=("KIND", "SIZE"),
                     help="run one small workload for an ncu capture instead of the benchmark "
-                         "(prefill T | pretrain T | segmented T | decode B | backward T | qsa n | layer T)")
+                         "(prefill T | pretrain T | segmented T | decode B | decode4 B | backward T | qsa n | layer T)")
     args = ap.parse_args()
     if args.profile_case:
         profile_case(args.profile_case[0], int(args.profile_case[1]))
