@@ -113,6 +113,7 @@ def test_kernel_events_hook_validation(lib):
 def test_rejected_calls_launch_nothing(lib):
     assert _prefill(lib, _dims(dk=96), _args()) == 2
     assert lib.gdn_last_call_launches() == 0
+    assert lib.gdn_last_call_slots() == 0
     args = [FAKE[i] for i in range(11)] + [ctypes.c_void_p(8192), ctypes.c_void_p(12288), None]
     assert lib.gdn_decode_step(ctypes.byref(_dims(num_seqs=4, total_tokens=5)), *args) == 1
     assert lib.gdn_last_call_launches() == 0
