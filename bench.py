@@ -109,8 +109,9 @@ def peaks():
 
 class ClockSampler:
     """SM clock, power and clock-event (throttle) reasons sampled during a
-    region: NVML polled every 5 ms from a thread (the counters nvidia-smi
-    prints), else nvidia-smi every 200 ms.  Read-only: no setting is changed."""
+    region: NVML polled every millisecond from a thread (the counters
+    nvidia-smi prints; a 16 ms timed region still gets several samples), else
+    nvidia-smi every 200 ms.  Read-only: no setting is changed."""
     REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
                0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
     SMI_FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -149,7 +150,7 @@ class ClockSampler:
                                   {n for bit, n in self.REASONS.items() if r & bit}))
             except Exception:
                 break
-            self._stop.wait(0.005)
+            self._stop.wait(0.001)
 
     def __enter__(self):
         import threading
@@ -158,7 +159,7 @@ class ClockSampler:
             self._stop = threading.Event()
             self._thread = threading.Thread(target=self._poll, args=(nv, h), daemon=True)
             self._thread.start()
-            self.source = "nvml 5 ms"
+            self.source = "nvml 1 ms"
             return self
         except Exception:
             pass
