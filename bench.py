@@ -107,6 +107,13 @@ def peaks():
         return FALLBACK_PEAKS, "fallback"
 
 
+def wait_event(ev):
+    """Wait for a recorded event by polling it with short sleeps: the clock
+    sampler's thread runs meanwhile (a device synchronisation can keep it out)."""
+    while not ev.query():
+        time.sleep(0.0002)
+
+
 class ClockSampler:
     """SM clock, power and clock-event (throttle) reasons sampled during a
     region: NVML polled every millisecond from a thread (the counters
@@ -150,15 +157,20 @@ class ClockSampler:
                                   {n for bit, n in self.REASONS.items() if r & bit}))
             except Exception:
                 break
+            self._polling.set()
             self._stop.wait(0.001)
+        self._polling.set()
 
     def __enter__(self):
         import threading
         try:
             nv, h = self._nvml_handle()
             self._stop = threading.Event()
+            self._polling = threading.Event()
             self._thread = threading.Thread(target=self._poll, args=(nv, h), daemon=True)
             self._thread.start()
+            self._polling.wait(timeout=2.0)   # the poll loop is running before the region starts
+            self.rows.clear()                 # samples from before the region
             self.source = "nvml 1 ms"
             return self
         except Exception:
@@ -256,6 +268,7 @@ def bench_prefill(cfg, steps, warmup, world, rank, dev):
         end.record()
         gdn.set_timing_events(None, None)
         gdn.set_kernel_events()
+        wait_event(end)
         torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(start.elapsed_time(end) / steps, world)
@@ -390,6 +403,7 @@ def bench_decode(cfg, steps, dev):
             launches += gdn.last_call_launches()
         end.record()
         gdn.set_timing_events(None, None)
+        wait_event(end)
         torch.cuda.synchronize()
     ms = start.elapsed_time(end) / steps
     kern_ms = sum(b.elapsed_time(e) for b, e in zip(evb, eve)) / steps
