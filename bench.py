@@ -67,12 +67,12 @@ KERNEL_ROOFLINE = {"chunk_prep": ("hbm", 3 * 128 * 2 + 2 * 2),                  
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per unit from one
 # ncu capture of each kernel (profiles/), valid only while the kernel's sources
 # are the ones captured (sha1 over them); otherwise the JSON reports traffic null.
-#   prefill_fused: `bench.py --profile-case prefill 8192` (T = 8192, H = 32): 359.6 MB read +
-#     333.8 MB written for 262,144 token-heads; per token-head, scaled to the launch.
+#   prefill_fused: `bench.py --profile-case prefill 8192` (T = 8192, H = 32): 347.4 MB read +
+#     332.6 MB written for 262,144 token-heads; per token-head, scaled to the launch.
 NCU_TRAFFIC = {
     "prefill_fused": {"sources": ["prefill_tc.cu", "prep_body.cuh", "chain_body.cuh"],
-                      "sha1": "7195f07619fa5a914cd5e937cdbf53b5740b6a36",
-                      "bytes_per_unit": (359.594752e6 + 333.776384e6) / (8192 * 32)},
+                      "sha1": "736a70aa4f6290e66b2141af8ad45a411a4f9a00",
+                      "bytes_per_unit": (347.356160e6 + 332.615680e6) / (8192 * 32)},
 }
 
 

@@ -269,10 +269,10 @@ __global__ void __launch_bounds__(fused::NT, 1) prefill_fused_kernel(const __gri
     const PrepGroupSync sy{1 + half};
     const int n_tasks = P.task_table ? __ldg(P.n_tasks_dev) : P.max_chunks * n_items;
     uint32_t phase = 0;
-    // the next task index is fetched one task ahead (slot 1) so the atomic's round
-    // trip overlaps a chunk, by a thread of warp 7: warps 0 and 1 compute the
-    // gates first thing in a chunk, warp 7 has time to wait for the atomic; a
-    // chunk's ready flag is published during the next one
+    // the next task index is fetched one task ahead so the atomic's round trip
+    // overlaps a chunk, by a thread of warp 7: warps 0 and 1 compute the gates
+    // first thing in a chunk, warp 7 has time to wait for the atomic; a chunk's
+    // ready flag is published during the next one
     // raw q, k, v rows of a task's chunk (and the three rows before it) into L2
     // Task t -> (chunk c, item): the items come in rounds of n_chain (the chain CTAs
     // take one item of each round in turn), and within a round chunk-major, so a
